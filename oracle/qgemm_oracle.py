@@ -1,0 +1,331 @@
+"""Oracle for the weight-quantised GEMM: plain, slow, obviously correct CPU code.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call or
+execute this module: only the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it. It shares
+no code with the CUDA library (no kernels, headers, tables or helpers); the
+two meet only through the seeded inputs of ``workloads.py``.
+
+What the method computes
+------------------------
+stable-diffusion.rs README (andreinknv), introduction: weights are held
+quantised at rest as packed bits and are dequantised inside the matmul, one
+tile at a time. The result it reaches is, up to rounding order, the plain
+product of the activations with the dequantised weights, so this oracle is
+that definition written out in fp64:
+
+    out[M, N] = X[M, K] . Wq[N, K]^T (+ bias[N])
+
+Formats (this library's definition; the pages give no bit layout, no scale
+formula and no rounding rule):
+
+* 4-bit and 8-bit group-wise affine, groups of 64 consecutive k in a row:
+  ``w ~ s16 * q + b16`` with fp16 scale s16 and fp16 bias b16 per group,
+  q in [0, 2^b - 1]. The pages' "4-bit everywhere ... held at 8 bits and the
+  rest at 4" (stable-diffusion.rs README, introduction) names the two widths.
+* ternary {-1, 0, +1} with one fp16 scale per group of 128
+  (pictor README, "Extreme quantization is first-class": TQ2_0_g128).
+
+Packing is round-to-nearest (RTN) in fp64, ties to even:
+
+* affine: lo = min, hi = max of the group; s16 = fp16(fl64((hi - lo) /
+  (2^b - 1))), b16 = fp16(lo); q = clamp(rint((w - b16) / s16), 0, 2^b - 1),
+  q = 0 where s16 == 0.
+* ternary: s16 = fp16(max |w|); t = clamp(rint(w / s16), -1, 1), t = 0 where
+  s16 == 0.
+
+Bit layout, row-major over N with K contiguous, little-endian 32-bit words:
+
+* 8-bit: byte k holds q[k].
+* 4-bit: a word holds 8 consecutive k; offset j = 2i (even) sits in bits
+  4i..4i+3 and offset j = 2i + 1 (odd) in bits 16+4i..19+4i.
+* ternary: a word holds 16 consecutive k; offset j = 2i in bits 2i..2i+1 and
+  j = 2i + 1 in bits 16+2i..17+2i. The 2-bit code is t in two's complement
+  (0 -> 00, +1 -> 01, -1 -> 11); code 10 is invalid.
+* scales and biases: fp16 [N, K / group], row-major.
+
+Dequantised weight (the bit-exact contract of the dequant-tile entry point):
+
+* affine: wdeq = bf16_rn( fl32(s16 * q + b16) ). s16 * q is exact in fp32
+  (11 + 8 significant bits), so this equals one fp32 FMA followed by one
+  round-to-nearest-even to bf16.
+* ternary: wdeq = t * bf16_rn(fl32(s16)), with +0 for t = 0.
+
+Numerics of the matmul: fp32 accumulation is what the kernels keep (pictor
+README, numerics: "FP32 accumulate is kept", no TF32 or FP16-MAC shortcuts);
+the oracle accumulates in fp64.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+AFFINE_BITS = (4, 8)
+TERNARY_BITS = 2
+
+
+# ----------------------------------------------------------------------------
+# rounding helpers
+# ----------------------------------------------------------------------------
+
+def fp16_rn(x) -> np.ndarray:
+    """fp64 -> fp16, round to nearest even, in one rounding (numpy's double->half).
+
+    Pinned in the tests against CPython's own IEEE half packing
+    (``struct.pack('e')``) on every fp16 value, every midpoint and random doubles.
+    """
+    return np.asarray(x, dtype=np.float64).astype(np.float16)
+
+
+def bf16_rn_bits(x32) -> np.ndarray:
+    """fp32 -> bf16 storage bits, round to nearest even on the fp32 bit pattern.
+
+    bf16 keeps the top 16 bits of an fp32. Rounding adds 0x7FFF plus the
+    lowest kept bit (the tie-to-even correction) before truncating. NaN keeps
+    its sign and top payload bits and is made quiet.
+    """
+    u = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    lsb = (u >> np.uint64(16)) & np.uint64(1)
+    r = ((u + np.uint64(0x7FFF) + lsb) >> np.uint64(16)).astype(np.uint32)
+    nan = (u & np.uint64(0x7FFFFFFF)) > np.uint64(0x7F800000)
+    r = np.where(nan, ((u >> np.uint64(16)) | np.uint64(0x40)).astype(np.uint32), r)
+    return r.astype(np.uint16)
+
+
+def bf16_bits_to_f64(b) -> np.ndarray:
+    """bf16 storage bits -> fp64 values (exact)."""
+    u = np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return u.view(np.float32).astype(np.float64)
+
+
+# ----------------------------------------------------------------------------
+# bit layout
+# ----------------------------------------------------------------------------
+
+def codes_per_word(bits: int) -> int:
+    return 32 // bits
+
+
+def code_bit_position(bits: int, j: int) -> int:
+    """Bit position, inside its 32-bit word, of the code for in-word offset j."""
+    if bits == 8:
+        return 8 * j
+    i, odd = divmod(j, 2)
+    return 16 * odd + bits * i
+
+
+def pack_codes(codes, bits: int) -> np.ndarray:
+    """Integer codes [N, K] -> packed bytes [N, K * bits / 8].
+
+    Affine codes are q in [0, 2^b - 1]; ternary codes are t in {-1, 0, +1}
+    and are stored as 2-bit two's complement.
+    """
+    codes = np.asarray(codes)
+    N, K = codes.shape
+    per = codes_per_word(bits)
+    if K % per:
+        raise ValueError("K must fill whole 32-bit words")
+    mask = (1 << bits) - 1
+    field = codes.astype(np.int64) & mask           # two's complement for t = -1
+    field = field.astype(np.uint32).reshape(N, K // per, per)
+    words = np.zeros((N, K // per), dtype=np.uint32)
+    for j in range(per):
+        words |= field[:, :, j] << np.uint32(code_bit_position(bits, j))
+    return words.astype("<u4").view(np.uint8).reshape(N, K * bits // 8)
+
+
+def unpack_codes(packed, bits: int, K: int) -> np.ndarray:
+    """Packed bytes [N, K * bits / 8] -> integer codes [N, K] (int32).
+
+    Raises ValueError on the invalid ternary code 10.
+    """
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    N = packed.shape[0]
+    per = codes_per_word(bits)
+    words = packed.reshape(N, -1).view("<u4").astype(np.uint32)
+    if words.shape[1] * per != K:
+        raise ValueError("packed width does not match K")
+    mask = np.uint32((1 << bits) - 1)
+    out = np.empty((N, words.shape[1], per), dtype=np.int32)
+    for j in range(per):
+        out[:, :, j] = (words >> np.uint32(code_bit_position(bits, j))) & mask
+    out = out.reshape(N, K)
+    if bits == TERNARY_BITS:
+        if np.any(out == 2):
+            raise ValueError("invalid ternary code 0b10")
+        out = np.where(out == 3, -1, out)
+    return out
+
+
+# ----------------------------------------------------------------------------
+# packing (RTN)
+# ----------------------------------------------------------------------------
+
+def check_format(bits: int, group: int, K: int) -> None:
+    if bits in AFFINE_BITS:
+        if group != 64:
+            raise ValueError("affine formats use groups of 64")
+    elif bits == TERNARY_BITS:
+        if group != 128:
+            raise ValueError("ternary uses groups of 128")
+    else:
+        raise ValueError("bits must be 2 (ternary), 4 or 8")
+    if K % group:
+        raise ValueError("K must be a multiple of the group size")
+
+
+def pack_ref(W, bits: int, group: int):
+    """RTN group quantisation of fp32 W [N, K].
+
+    Returns (packed uint8 [N, K*b/8], scales fp16 [N, K/g], biases fp16
+    [N, K/g] or None for ternary).
+    """
+    W = np.asarray(W, dtype=np.float32)
+    N, K = W.shape
+    check_format(bits, group, K)
+    if not np.all(np.isfinite(W)):
+        raise ValueError("non-finite weight")
+    Wg = W.astype(np.float64).reshape(N, K // group, group)
+    if bits in AFFINE_BITS:
+        qmax = (1 << bits) - 1
+        lo = Wg.min(axis=2)
+        hi = Wg.max(axis=2)
+        s16 = fp16_rn((hi - lo) / qmax)
+        b16 = fp16_rn(lo)
+        if not (np.all(np.isfinite(s16)) and np.all(np.isfinite(b16))):
+            raise OverflowError("scale or bias overflows fp16")
+        s = s16.astype(np.float64)[:, :, None]
+        b = b16.astype(np.float64)[:, :, None]
+        with np.errstate(divide="ignore", invalid="ignore"):
+            q = np.clip(np.rint((Wg - b) / s), 0, qmax)
+        q = np.where(s == 0, 0, q)
+        codes = q.reshape(N, K).astype(np.int64)
+        return pack_codes(codes, bits), s16, b16
+    s16 = fp16_rn(np.abs(Wg).max(axis=2))
+    if not np.all(np.isfinite(s16)):
+        raise OverflowError("scale overflows fp16")
+    s = s16.astype(np.float64)[:, :, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = np.clip(np.rint(Wg / s), -1, 1)
+    t = np.where(s == 0, 0, t)
+    return pack_codes(t.reshape(N, K).astype(np.int64), bits), s16, None
+
+
+# ----------------------------------------------------------------------------
+# dequantisation
+# ----------------------------------------------------------------------------
+
+def _expand(groupwise, group: int) -> np.ndarray:
+    return np.repeat(np.asarray(groupwise, dtype=np.float16).astype(np.float64), group, axis=1)
+
+
+def wq_exact(packed, scales, biases, bits: int, group: int, K: int) -> np.ndarray:
+    """The quantised weight before any bf16 rounding, fp64 [N, K]: s16*q + b16 or s16*t."""
+    codes = unpack_codes(packed, bits, K).astype(np.float64)
+    s = _expand(scales, group)
+    if bits == TERNARY_BITS:
+        return s * codes
+    return s * codes + _expand(biases, group)
+
+
+def dequant_ref_bits(packed, scales, biases, bits: int, group: int, K: int) -> np.ndarray:
+    """The dequantised weight as bf16 bits [N, K] (the bit-exact contract).
+
+    affine: s16*q + b16 is exact in fp64 (at most 11+8 significant bits in the
+    product and an fp16 addend; the sum spans under 53 bits), so casting it to
+    fp32 rounds exactly once, like an fp32 FMA; bf16_rn then rounds again.
+    ternary: t * bf16_rn(fp32(s16)), i.e. the sign bit flipped for t = -1 and
+    +0 for t = 0.
+    """
+    codes = unpack_codes(packed, bits, K)
+    s = _expand(scales, group)
+    if bits == TERNARY_BITS:
+        sb = bf16_rn_bits(s.astype(np.float32))
+        out = np.where(codes < 0, sb | np.uint16(0x8000), sb)
+        return np.where(codes == 0, np.uint16(0), out).astype(np.uint16)
+    v = s * codes.astype(np.float64) + _expand(biases, group)
+    return bf16_rn_bits(v.astype(np.float32))
+
+
+def dequant_ref(packed, scales, biases, bits: int, group: int, K: int) -> np.ndarray:
+    """The dequantised weight as fp64 values [N, K]."""
+    return bf16_bits_to_f64(dequant_ref_bits(packed, scales, biases, bits, group, K))
+
+
+# ----------------------------------------------------------------------------
+# the matmul
+# ----------------------------------------------------------------------------
+
+def qgemm_ref(X_bits, packed, scales, biases, bits: int, group: int, K: int,
+              bias_bits=None) -> np.ndarray:
+    """fp64 out[M, N] = X . Wq_exact^T (+ bias): the reference the kernels are judged by."""
+    X = bf16_bits_to_f64(X_bits)
+    out = X @ wq_exact(packed, scales, biases, bits, group, K).T
+    if bias_bits is not None:
+        out = out + bf16_bits_to_f64(bias_bits)[None, :]
+    return out
+
+
+def qgemm_ref_bf16w(X_bits, packed, scales, biases, bits: int, group: int, K: int,
+                    bias_bits=None) -> np.ndarray:
+    """fp64 out = X . wdeq^T (+ bias), with the bf16 dequantised weights: a tighter diagnostic."""
+    X = bf16_bits_to_f64(X_bits)
+    out = X @ dequant_ref(packed, scales, biases, bits, group, K).T
+    if bias_bits is not None:
+        out = out + bf16_bits_to_f64(bias_bits)[None, :]
+    return out
+
+
+def qgemm_ref_rows(rows, X_bits, packed, scales, biases, bits: int, group: int, K: int,
+                   bias_bits=None) -> np.ndarray:
+    """Reference for a subset of output rows (large shapes, sampled checking)."""
+    rows = np.asarray(rows)
+    return qgemm_ref(np.asarray(X_bits)[rows], packed, scales, biases, bits, group, K, bias_bits)
+
+
+def dense_ref(X_bits, W, bias_bits=None) -> np.ndarray:
+    """fp64 X . bf16_rn(W)^T (+ bias): the dense bf16 layer the quantised one replaces."""
+    X = bf16_bits_to_f64(X_bits)
+    Wb = bf16_bits_to_f64(bf16_rn_bits(np.asarray(W, dtype=np.float32)))
+    out = X @ Wb.T
+    if bias_bits is not None:
+        out = out + bf16_bits_to_f64(bias_bits)[None, :]
+    return out
+
+
+# ----------------------------------------------------------------------------
+# error metrics
+# ----------------------------------------------------------------------------
+
+REL_FROB_TOL = 5e-3      # ||Y - ref||_F / ||ref||_F
+MAX_ABS_TOL = 3e-2       # max |Y - ref| / max |ref|
+
+
+def rel_frobenius(y, ref) -> float:
+    y = np.asarray(y, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = np.linalg.norm(ref)
+    return float(np.linalg.norm(y - ref) / den) if den > 0 else float(np.linalg.norm(y))
+
+
+def max_abs_rel(y, ref) -> float:
+    y = np.asarray(y, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = np.max(np.abs(ref)) if ref.size else 0.0
+    err = np.max(np.abs(y - ref)) if ref.size else 0.0
+    return float(err / den) if den > 0 else float(err)
+
+
+def cosine(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64).ravel()
+    b = np.asarray(b, dtype=np.float64).ravel()
+    return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b)))
+
+
+def within_tolerance(y, ref) -> bool:
+    return rel_frobenius(y, ref) <= REL_FROB_TOL and max_abs_rel(y, ref) <= MAX_ABS_TOL
+
+
+def format_bytes(N: int, K: int, bits: int, group: int) -> int:
+    """Bytes of one packed weight at rest: codes + fp16 scales (+ fp16 biases)."""
+    per_group = 2 if bits == TERNARY_BITS else 4
+    return N * K * bits // 8 + N * (K // group) * per_group

@@ -1,0 +1,386 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test checks the oracle against an independent fact: CPython's IEEE half
+packing, torch's bf16 conversion, hand-derived bit layouts, closed forms of
+the RTN quantiser, exact round trips of constructed weights, and a
+pure-Python triple loop. A plausible slip anywhere in the oracle (a dropped
+bias term, a wrong sign, a swapped nibble, a transposed operand, a wrong
+rounding mode) fails at least one of them.
+"""
+import math
+import struct
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as WL
+
+
+# ----------------------------------------------------------------------------
+# rounding helpers
+# ----------------------------------------------------------------------------
+
+def _struct_half_bits(x: float) -> int:
+    return struct.unpack("<H", struct.pack("<e", x))[0]
+
+
+def test_fp16_rn_every_half_and_midpoint():
+    """Every finite fp16 value maps to itself; every midpoint ties to even.
+
+    Reference: CPython's ``struct.pack('e')`` (IEEE 754 binary16, round half to even).
+    """
+    bits = np.arange(0, 0x7C00, dtype=np.uint16)          # +0 .. max finite
+    vals = bits.view(np.float16).astype(np.float64)
+    assert np.array_equal(O.fp16_rn(vals).view(np.uint16), bits)
+    assert np.array_equal(O.fp16_rn(-vals).view(np.uint16), bits | 0x8000)
+    mids = (vals[:-1] + vals[1:]) / 2.0                    # exact in fp64
+    got = O.fp16_rn(mids).view(np.uint16)
+    ref = np.array([_struct_half_bits(float(m)) for m in mids], dtype=np.uint16)
+    assert np.array_equal(got, ref)
+    # ties go to the even neighbour
+    assert np.all(got % 2 == 0)
+
+
+def test_fp16_rn_random_doubles_match_struct():
+    g = np.random.default_rng(11)
+    x = np.concatenate([g.standard_normal(20000) * 10.0 ** g.integers(-9, 5, 20000),
+                        g.uniform(-65504, 65504, 2000)])
+    got = O.fp16_rn(x).view(np.uint16)
+    ref = np.array([_struct_half_bits(float(v)) for v in x], dtype=np.uint16)
+    assert np.array_equal(got, ref)
+
+
+def test_bf16_rn_matches_torch_on_stratified_fp32_patterns():
+    """All 65536 upper halves x low halves {0, 1, 0x7FFF, 0x8000, 0x8001, 0xFFFF, random}."""
+    hi = np.arange(65536, dtype=np.uint32) << 16
+    lows = [0x0000, 0x0001, 0x7FFF, 0x8000, 0x8001, 0xFFFF]
+    g = np.random.default_rng(3)
+    pats = np.concatenate([hi | np.uint32(lo) for lo in lows]
+                          + [hi | g.integers(0, 65536, 65536).astype(np.uint32)])
+    f = pats.view(np.float32)
+    finite = np.isfinite(f)
+    got = O.bf16_rn_bits(f[finite])
+    ref = torch.from_numpy(f[finite].copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, ref)
+    # NaN stays NaN
+    nan_out = O.bf16_rn_bits(f[np.isnan(f)])
+    assert np.all((nan_out & 0x7F80) == 0x7F80) and np.all((nan_out & 0x7F) != 0)
+
+
+def test_bf16_rn_ties_to_even_examples():
+    # 1 + 2^-8 is halfway between bf16 1.0 (0x3F80) and 1 + 2^-7 (0x3F81): ties to 0x3F80
+    assert O.bf16_rn_bits(np.float32(1.0 + 2.0 ** -8))[()] == 0x3F80
+    # 1 + 3*2^-8 is halfway between 0x3F81 and 0x3F82: ties to the even 0x3F82
+    assert O.bf16_rn_bits(np.float32(1.0 + 3 * 2.0 ** -8))[()] == 0x3F82
+    # just above the tie rounds up
+    assert O.bf16_rn_bits(np.float32(1.0 + 2.0 ** -8 + 2.0 ** -20))[()] == 0x3F81
+
+
+# ----------------------------------------------------------------------------
+# bit layout
+# ----------------------------------------------------------------------------
+
+def test_layout_hand_derived_4bit():
+    # codes 1..8 for k = 0..7. Even k in the low half-word, odd k in the high one:
+    # bits 0-3 k0=1, 4-7 k2=3, 8-11 k4=5, 12-15 k6=7, 16-19 k1=2, 20-23 k3=4,
+    # 24-27 k5=6, 28-31 k7=8  ->  word 0x86427531, little-endian bytes 31 75 42 86
+    packed = O.pack_codes(np.array([[1, 2, 3, 4, 5, 6, 7, 8]]), 4)
+    assert packed.tolist() == [[0x31, 0x75, 0x42, 0x86]]
+
+
+def test_layout_hand_derived_8bit():
+    packed = O.pack_codes(np.array([[0, 1, 127, 128, 255, 7, 9, 200]]), 8)
+    assert packed.tolist() == [[0, 1, 127, 128, 255, 7, 9, 200]]
+
+
+def test_layout_hand_derived_ternary():
+    # t = +1 at k=0 (code 01 at bits 0-1), -1 at k=1 (code 11 at bits 16-17),
+    # -1 at k=2 (11 at bits 2-3), +1 at k=15 (01 at bits 30-31), rest 0:
+    # word = 0x1 | 0xC | 0x30000 | 0x40000000 = 0x4003000D -> bytes 0D 00 03 40
+    t = np.zeros((1, 16), dtype=np.int64)
+    t[0, 0], t[0, 1], t[0, 2], t[0, 15] = 1, -1, -1, 1
+    assert O.pack_codes(t, 2).tolist() == [[0x0D, 0x00, 0x03, 0x40]]
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_pack_unpack_bijection_every_code_every_position(bits):
+    values = [-1, 0, 1] if bits == 2 else list(range(1 << bits))
+    per = O.codes_per_word(bits)
+    K = per * len(values)
+    rows = []
+    for r in range(len(values)):
+        rows.append([values[(r + k) % len(values)] for k in range(K)])
+    codes = np.array(rows)
+    # each value appears at each in-word position in some row
+    for j in range(per):
+        assert set(codes[:, j].tolist()) == set(values)
+    packed = O.pack_codes(codes, bits)
+    assert packed.shape == (len(values), K * bits // 8)
+    assert np.array_equal(O.unpack_codes(packed, bits, K), codes)
+    # and the map on bytes is onto the valid patterns: repacking an unpacked
+    # random byte stream (affine formats) reproduces it exactly
+    if bits != 2:
+        g = np.random.default_rng(bits)
+        raw = g.integers(0, 256, size=(5, 64), dtype=np.uint8)
+        Kr = 64 * 8 // bits
+        assert np.array_equal(O.pack_codes(O.unpack_codes(raw, bits, Kr), bits), raw)
+
+
+def test_ternary_invalid_code_rejected():
+    bad = np.array([[0x02, 0, 0, 0]], dtype=np.uint8)   # code 10 at k = 0
+    with pytest.raises(ValueError):
+        O.unpack_codes(bad, 2, 16)
+
+
+def test_single_code_positions_match_layout_definition():
+    """A lone code at each k lands at the bit the layout definition names."""
+    for bits in (2, 4, 8):
+        per = O.codes_per_word(bits)
+        K = 2 * per
+        for k in range(K):
+            c = np.zeros((1, K), dtype=np.int64)
+            c[0, k] = 1
+            words = O.pack_codes(c, bits).view("<u4")[0]
+            w, j = divmod(k, per)
+            if bits == 8:
+                expect_bit = 8 * j
+            else:
+                expect_bit = (16 if j % 2 else 0) + bits * (j // 2)
+            assert int(words[w]) == 1 << expect_bit
+            assert all(int(words[x]) == 0 for x in range(len(words)) if x != w)
+
+
+# ----------------------------------------------------------------------------
+# RTN quantiser: closed forms and exact round trips
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_affine_error_bound(bits):
+    g = np.random.default_rng(5 + bits)
+    W = (g.standard_normal((64, 512)) * 0.02).astype(np.float32)
+    packed, s16, b16 = O.pack_ref(W, bits, 64)
+    q = O.unpack_codes(packed, bits, 512)
+    qmax = (1 << bits) - 1
+    assert q.min() >= 0 and q.max() <= qmax
+    s = np.repeat(s16.astype(np.float64), 64, axis=1)
+    b = np.repeat(b16.astype(np.float64), 64, axis=1)
+    Wg = W.astype(np.float64).reshape(64, 8, 64)
+    lo = np.repeat(Wg.min(axis=2), 64, axis=1)
+    hi = np.repeat(Wg.max(axis=2), 64, axis=1)
+    err = np.abs(W.astype(np.float64) - (s * q + b))
+    bound = s / 2 + np.abs(lo - b) + np.abs(hi - (b + qmax * s)) + 1e-12
+    assert np.all(err <= bound)
+    # unclamped entries are within half a step
+    inner = (q > 0) & (q < qmax)
+    assert np.all(err[inner] <= s[inner] / 2 * (1 + 1e-9))
+    # the scale is the fp16 rounding of the range over 2^b - 1
+    rng = Wg.max(axis=2) - Wg.min(axis=2)
+    assert np.all(np.abs(s16.astype(np.float64) - rng / qmax) <= np.abs(rng / qmax) * 2.0 ** -11)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_affine_exact_grid_is_recovered(bits):
+    """A group laid exactly on lo + s*{0..2^b-1} (fp16 s and lo) packs back exactly."""
+    qmax = (1 << bits) - 1
+    g = np.random.default_rng(bits)
+    N = 16
+    s = np.array([2.0 ** -e for e in g.integers(4, 12, N)])
+    lo = -np.array([float(np.float16(v)) for v in g.uniform(0.0, 0.5, N)])
+    q_true = np.stack([g.permutation(np.concatenate([[0, qmax], g.integers(0, qmax + 1, 62)]))
+                       for _ in range(N)])
+    W = (lo[:, None] + s[:, None] * q_true).astype(np.float32)
+    assert np.array_equal(W.astype(np.float64), lo[:, None] + s[:, None] * q_true)  # exact in fp32
+    packed, s16, b16 = O.pack_ref(W, bits, 64)
+    assert np.array_equal(s16[:, 0].astype(np.float64), s)
+    assert np.array_equal(b16[:, 0].astype(np.float64), lo)
+    assert np.array_equal(O.unpack_codes(packed, bits, 64), q_true)
+
+
+def test_affine_degenerate_groups():
+    W = np.zeros((3, 64), dtype=np.float32)
+    W[1, :] = 0.25                 # constant group
+    W[2, :] = -0.0                 # negative zeros
+    packed, s16, b16 = O.pack_ref(W, 4, 64)
+    assert np.all(s16 == 0)
+    assert b16[1, 0] == np.float16(0.25)
+    assert np.all(O.unpack_codes(packed, 4, 64) == 0)
+    wd = O.dequant_ref(packed, s16, b16, 4, 64, 64)
+    assert np.all(wd[1] == 0.25) and np.all(wd[0] == 0) and np.all(wd[2] == 0)
+
+
+def test_ternary_constructed_weights_round_trip_exactly():
+    """W = s16 * t (the ternary workload's construction) packs back to t and s16."""
+    lin = WL.workload(3).linears[0]
+    W = WL.make_w(3, 0, 256, lin.K, "ternary", 128)
+    g = np.random.default_rng(np.random.SeedSequence([0, 3, 0, 5, 0]))
+    t = g.integers(-1, 2, size=(lin.N, lin.K))[:256].astype(np.int64)
+    packed, s16, b = O.pack_ref(W, 2, 128)
+    assert b is None
+    codes = O.unpack_codes(packed, 2, lin.K)
+    assert set(np.unique(codes).tolist()) <= {-1, 0, 1}
+    assert np.array_equal(codes, t)
+    recon = np.repeat(s16.astype(np.float32), 128, axis=1) * codes
+    assert np.array_equal(recon.astype(np.float32), W)
+
+
+def test_ternary_rtn_threshold_and_clamp():
+    w = np.zeros((1, 128), dtype=np.float32)
+    w[0, 0] = 1.0                  # the absmax: scale 1.0
+    w[0, 1] = 0.5                  # exactly half: rint(0.5) = 0 (ties to even)
+    w[0, 2] = 0.5000001            # just above half -> +1
+    w[0, 3] = -0.75                # -> -1
+    w[0, 4] = -0.25                # -> 0
+    packed, s16, _ = O.pack_ref(w, 2, 128)
+    t = O.unpack_codes(packed, 2, 128)
+    assert s16[0, 0] == 1.0
+    assert t[0, :5].tolist() == [1, 0, 1, -1, 0]
+
+
+def test_pack_rejects_bad_inputs():
+    W = np.zeros((2, 128), dtype=np.float32)
+    with pytest.raises(ValueError):
+        O.pack_ref(W, 3, 64)
+    with pytest.raises(ValueError):
+        O.pack_ref(W, 4, 128)
+    with pytest.raises(ValueError):
+        O.pack_ref(np.zeros((2, 96), np.float32), 4, 64)
+    W[0, 0] = np.nan
+    with pytest.raises(ValueError):
+        O.pack_ref(W, 4, 64)
+    big = np.zeros((1, 64), dtype=np.float32)
+    big[0, 0] = -1e6
+    big[0, 1] = 1e6
+    with pytest.raises(OverflowError):
+        O.pack_ref(big, 4, 64)
+
+
+# ----------------------------------------------------------------------------
+# dequantisation
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_dequant_exact_when_representable(bits):
+    """s16 = 1/2, b16 = -4: every s*q + b is a bf16 value, so dequant is exact."""
+    qmax = (1 << bits) - 1
+    q = np.resize(np.arange(qmax + 1), (4, 256))
+    packed = O.pack_codes(q, bits)
+    s16 = np.full((4, 4), 0.5, dtype=np.float16)
+    b16 = np.full((4, 4), -4.0, dtype=np.float16)
+    wd = O.dequant_ref(packed, s16, b16, bits, 64, 256)
+    assert np.array_equal(wd, 0.5 * q - 4.0)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_dequant_monotone_and_within_bf16_rounding(bits):
+    g = np.random.default_rng(20 + bits)
+    W = (g.standard_normal((32, 256)) * 0.02).astype(np.float32)
+    packed, s16, b16 = O.pack_ref(W, bits, 64)
+    q = O.unpack_codes(packed, bits, 256)
+    wd = O.dequant_ref(packed, s16, b16, bits, 64, 256)
+    exact = O.wq_exact(packed, s16, b16, bits, 64, 256)
+    # bf16 keeps 8 significant bits: RNE error <= half an ulp <= 2^-8 relative (+ the fp32 step)
+    assert np.all(np.abs(wd - exact) <= np.abs(exact) * (2.0 ** -8 + 2.0 ** -23) + 1e-45)
+    # within a group, larger codes never give smaller weights (s16 >= 0)
+    for n in range(32):
+        for gi in range(4):
+            sl = slice(64 * gi, 64 * gi + 64)
+            order = np.argsort(q[n, sl], kind="stable")
+            assert np.all(np.diff(wd[n, sl][order]) >= 0)
+    # q = 0 gives the bias rounded to bf16
+    zero = q == 0
+    b = np.repeat(b16, 64, axis=1)
+    tb = torch.from_numpy(b.astype(np.float32)).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(wd[zero], tb[zero].astype(np.float64))
+
+
+def test_dequant_final_rounding_matches_torch_bf16():
+    """The bf16 step of the dequant agrees with torch's own fp32->bf16 conversion."""
+    g = np.random.default_rng(31)
+    W = (g.standard_normal((16, 256)) * 0.05).astype(np.float32)
+    packed, s16, b16 = O.pack_ref(W, 4, 64)
+    exact32 = O.wq_exact(packed, s16, b16, 4, 64, 256).astype(np.float32)
+    tb = torch.from_numpy(exact32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(O.dequant_ref_bits(packed, s16, b16, 4, 64, 256), tb)
+
+
+def test_ternary_dequant_is_signed_scale():
+    g = np.random.default_rng(8)
+    t = g.integers(-1, 2, size=(8, 256))
+    s16 = g.uniform(0.01, 0.05, size=(8, 2)).astype(np.float16)
+    packed = O.pack_codes(t, 2)
+    bits = O.dequant_ref_bits(packed, s16, None, 2, 128, 256)
+    sb = torch.from_numpy(np.repeat(s16.astype(np.float32), 128, axis=1)).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(O.bf16_bits_to_f64(bits), t * sb.astype(np.float64))
+    assert np.all(bits[t == 0] == 0)                      # +0, not -0
+    assert np.all((bits[t < 0] & 0x8000) == 0x8000)
+
+
+# ----------------------------------------------------------------------------
+# the matmul
+# ----------------------------------------------------------------------------
+
+def _naive(X, Wq, bias):
+    M, K = X.shape
+    N = Wq.shape[0]
+    out = [[0.0] * N for _ in range(M)]
+    for m in range(M):
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                acc = math.fsum([acc, float(X[m, k]) * float(Wq[n, k])])
+            out[m][n] = acc + (float(bias[n]) if bias is not None else 0.0)
+    return np.array(out)
+
+
+@pytest.mark.parametrize("bits,K", [(4, 128), (8, 64), (2, 128)])
+def test_qgemm_ref_equals_naive_triple_loop(bits, K):
+    X, W, bias = WL.random_case(1, 5, 7, K, bits, with_bias=True)
+    group = 128 if bits == 2 else 64
+    packed, s, b = O.pack_ref(W, bits, group)
+    ref = O.qgemm_ref(X, packed, s, b, bits, group, K, bias)
+    Wq = O.wq_exact(packed, s, b, bits, group, K)
+    brute = _naive(O.bf16_bits_to_f64(X), Wq, O.bf16_bits_to_f64(bias))
+    assert np.allclose(ref, brute, rtol=1e-12, atol=1e-14)
+
+
+def test_qgemm_ref_orientation():
+    """out[m, n] pairs activation row m with weight row n (not its transpose)."""
+    K = 64
+    W = np.zeros((3, K), dtype=np.float32)
+    for n in range(3):
+        W[n, :] = np.linspace(-1, 1, K) * (n + 1)
+    X = np.zeros((2, K), dtype=np.uint16)
+    X[0, 5] = 0x3F80                 # 1.0 at k = 5
+    X[1, 40] = 0x4000                # 2.0 at k = 40
+    packed, s, b = O.pack_ref(W, 8, 64)
+    ref = O.qgemm_ref(X, packed, s, b, 8, 64, K)
+    Wq = O.wq_exact(packed, s, b, 8, 64, K)
+    assert np.array_equal(ref[0], Wq[:, 5])
+    assert np.array_equal(ref[1], 2 * Wq[:, 40])
+
+
+def test_metrics():
+    ref = np.array([[1.0, -2.0], [3.0, 4.0]])
+    assert O.rel_frobenius(ref, ref) == 0.0
+    assert abs(O.rel_frobenius(ref * 1.01, ref) - 0.01) < 1e-12
+    assert abs(O.max_abs_rel(ref + 0.04, ref) - 0.01) < 1e-12
+    assert abs(O.cosine(ref, 3 * ref) - 1.0) < 1e-15
+    assert abs(O.cosine([1, 0], [0, 1])) < 1e-15
+
+
+@pytest.mark.parametrize("bits,expect", [(4, 0.996), (8, 0.99998)])
+def test_cosine_against_dense_matches_rtn_noise_model(bits, expect):
+    """E cos(X Wq^T, X W^T) ~ cos(vec Wq, vec W); for Gaussian groups of 64 the
+    RTN step is about range/(2^b - 1) with error variance step^2 / 12."""
+    g = np.random.default_rng(42)
+    W = (g.standard_normal((256, 1024)) * 0.02).astype(np.float32)
+    packed, s, b = O.pack_ref(W, bits, 64)
+    Wq = O.wq_exact(packed, s, b, bits, 64, 1024)
+    c = O.cosine(Wq, W)
+    tol = 2e-3 if bits == 4 else 2e-5
+    assert abs(c - expect) < tol
+    X = WL.f32_to_bf16_bits(g.standard_normal((64, 1024)).astype(np.float32))
+    cy = O.cosine(O.qgemm_ref(X, packed, s, b, bits, 64, 1024), O.bf16_bits_to_f64(X) @ W.astype(np.float64).T)
+    assert abs(cy - c) < 5 * (1 - c) + 1e-6
