@@ -29,8 +29,9 @@ formula and no rounding rule):
 Packing is round-to-nearest (RTN) in fp64, ties to even:
 
 * affine: lo = min, hi = max of the group; s16 = fp16(fl64((hi - lo) /
-  (2^b - 1))), b16 = fp16(lo); q = clamp(rint((w - b16) / s16), 0, 2^b - 1),
-  q = 0 where s16 == 0.
+  (2^b - 1))), b16 = fp16(lo) (a zero minimum as +0, so the sign of a zero
+  weight never decides a stored bit); q = clamp(rint((w - b16) / s16), 0,
+  2^b - 1), q = 0 where s16 == 0.
 * ternary: s16 = fp16(max |w|); t = clamp(rint(w / s16), -1, 1), t = 0 where
   s16 == 0.
 
@@ -187,7 +188,7 @@ def pack_ref(W, bits: int, group: int):
     Wg = W.astype(np.float64).reshape(N, K // group, group)
     if bits in AFFINE_BITS:
         qmax = (1 << bits) - 1
-        lo = Wg.min(axis=2)
+        lo = Wg.min(axis=2) + 0.0      # a zero minimum is stored as +0, never -0
         hi = Wg.max(axis=2)
         s16 = fp16_rn((hi - lo) / qmax)
         b16 = fp16_rn(lo)

@@ -208,6 +208,9 @@ def test_affine_degenerate_groups():
     assert np.all(O.unpack_codes(packed, 4, 64) == 0)
     wd = O.dequant_ref(packed, s16, b16, 4, 64, 64)
     assert np.all(wd[1] == 0.25) and np.all(wd[0] == 0) and np.all(wd[2] == 0)
+    # a group of negative zeros stores a +0 bias, so it dequantises to +0 bits
+    assert b16.view(np.uint16)[2, 0] == 0
+    assert np.all(O.dequant_ref_bits(packed, s16, b16, 4, 64, 64)[2] == 0)
 
 
 def test_ternary_constructed_weights_round_trip_exactly():
