@@ -1,0 +1,181 @@
+/*
+ * qgemm — weight-only quantised GEMM for NVIDIA B200 (sm_100a).
+ *
+ * The operation (stable-diffusion.rs README, introduction): weights are held
+ * quantised at rest as packed bits and are dequantised inside the matmul one
+ * tile at a time, so a layer whose dense weights would not fit still runs.
+ *
+ *     out[M, N] = X[M, K] . dequant(W)[N, K]^T (+ bias[N])
+ *
+ * with X and out in bf16, W packed in one of three formats, and fp32
+ * accumulation throughout (pictor README, numerics: fp32 accumulate is kept,
+ * no TF32 or FP16-MAC shortcuts).
+ *
+ * Formats (the pages give no bit layout, scale formula or rounding rule; this
+ * library fixes the following):
+ *   bits = 4 or 8, group = 64   group-wise affine, w ~ s * q + b, with an fp16
+ *                               scale s and an fp16 bias b per 64 consecutive
+ *                               k of a row, q in [0, 2^bits - 1]
+ *                               (stable-diffusion.rs README, introduction: the
+ *                               layers that multiply the residual stream at 8
+ *                               bits, the rest at 4);
+ *   bits = 2, group = 128       ternary t in {-1, 0, +1} with one fp16 scale per
+ *                               128 consecutive k (pictor README, "Extreme
+ *                               quantization is first-class": TQ2_0_g128).
+ *
+ * Bit layout (row-major over N, K contiguous, little-endian 32-bit words):
+ *   8-bit   byte k holds q[k];
+ *   4-bit   a word holds 8 consecutive k: in-word offset j = 2i in bits
+ *           4i..4i+3, j = 2i+1 in bits 16+4i..19+4i;
+ *   ternary a word holds 16 consecutive k: j = 2i in bits 2i..2i+1, j = 2i+1
+ *           in bits 16+2i..17+2i; the code is t in 2-bit two's complement
+ *           (00 = 0, 01 = +1, 11 = -1; 10 is invalid);
+ *   scales, biases: fp16 [N, K / group], row-major.
+ * Even and odd k sit in the two half-words so that one shift and one mask
+ * move a neighbouring pair of codes into the two lanes of a bf16x2 register.
+ *
+ * Dequantised weight (what the kernels multiply; bit-exact contract):
+ *   affine   wdeq = bf16_rn( fp32(s) * q + fp32(b) )  — one fp32 FMA, whose
+ *            product is exact, then one round-to-nearest-even to bf16;
+ *   ternary  wdeq = t * bf16_rn(fp32(s)), +0 for t = 0.
+ *
+ * Ownership: the caller allocates every buffer passed in; the library never
+ * allocates, frees or keeps user memory. Device-side state is one static
+ * status word per device (no allocation).
+ * Errors: every call returns a qgemm_status; nothing throws across the ABI.
+ * Asynchrony: device calls only enqueue work on the given stream (a
+ * cudaStream_t passed as void*, NULL = the legacy default stream) and return
+ * without synchronising, except qgemm_get_device_status.
+ * Threads: calls are thread-safe; concurrent calls need distinct output
+ * buffers.
+ */
+#ifndef QGEMM_H
+#define QGEMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum qgemm_status {
+  QGEMM_OK = 0,
+  QGEMM_ERR_INVALID_ARG = 1,     /* null pointer, negative or inconsistent size */
+  QGEMM_ERR_UNSUPPORTED = 2,     /* format, shape or device this build does not handle */
+  QGEMM_ERR_ALIGNMENT = 3,       /* a pointer is not 16-byte aligned */
+  QGEMM_ERR_NONFINITE = 4,       /* a weight to pack is NaN or infinite */
+  QGEMM_ERR_CUDA = 5,            /* a CUDA runtime or driver call failed */
+  QGEMM_ERR_DEVICE_TIMEOUT = 6   /* a kernel's bounded wait ran out (see qgemm_get_device_status) */
+} qgemm_status;
+
+/* Kernel path selection for qgemm_ex. */
+enum {
+  QGEMM_PATH_AUTO = 0,     /* pick per shape from the measured table */
+  QGEMM_PATH_SMALL_M = 1,  /* memory-bound path: registers + mma.sync, M <= 16 */
+  QGEMM_PATH_LARGE_M = 2   /* tensor-core path: TMA + smem dequant + tcgen05 MMA into TMEM */
+};
+
+/* A packed weight matrix resident in device memory. */
+typedef struct qgemm_weights {
+  int32_t N;             /* output features (rows of W) */
+  int32_t K;             /* input features (columns of W) */
+  int32_t bits;          /* 2 (ternary), 4 or 8 */
+  int32_t group;         /* 128 for ternary, 64 for 4- and 8-bit */
+  const void* packed;    /* uint8 [N, K * bits / 8], 16-byte aligned */
+  const void* scales;    /* fp16 [N, K / group], 16-byte aligned */
+  const void* biases;    /* fp16 [N, K / group], 16-byte aligned; NULL for ternary */
+} qgemm_weights;
+
+/*
+ * Byte sizes of the three packed arrays for an [N, K] weight.
+ * Defined by the layout above. biases_bytes is 0 for ternary.
+ * Returns INVALID_ARG for non-positive sizes or null outputs, UNSUPPORTED
+ * for a (bits, group) pair other than (4,64), (8,64), (2,128) or for K not a
+ * multiple of 128.
+ */
+int qgemm_pack_sizes(int32_t N, int32_t K, int32_t bits, int32_t group,
+                     size_t* packed_bytes, size_t* scales_bytes, size_t* biases_bytes);
+
+/*
+ * Round-to-nearest group quantisation of a host fp32 matrix W [N, K]
+ * (row-major) into caller-allocated host buffers sized by qgemm_pack_sizes.
+ * Arithmetic is fp64, ties to even:
+ *   affine:  s = fp16(fl64((max - min) / (2^bits - 1))), b = fp16(min),
+ *            q = clamp(rint((w - b) / s), 0, 2^bits - 1), q = 0 where s == 0;
+ *   ternary: s = fp16(max |w|), t = clamp(rint(w / s), -1, 1), t = 0 where s == 0.
+ * The weights stay packed at rest (stable-diffusion.rs README, introduction).
+ * Returns NONFINITE if W holds NaN/Inf, UNSUPPORTED if a scale or bias
+ * overflows fp16, plus the errors of qgemm_pack_sizes. biases may be NULL for
+ * ternary. Host-only; no device is touched.
+ */
+int qgemm_pack(const float* W, int32_t N, int32_t K, int32_t bits, int32_t group,
+               void* packed, void* scales, void* biases);
+
+/*
+ * out = X . dequant(W)^T (+ bias), enqueued on `stream`.
+ *   X     device bf16 [M, K] row-major, 16-byte aligned
+ *   M     tokens (rows of X); M = 0 is a no-op returning OK
+ *   W     device-resident packed weights (struct itself is host memory)
+ *   out   device bf16 [M, N] row-major, 16-byte aligned
+ *   bias  device bf16 [N] or NULL
+ * Requires K % 128 == 0 and N % 16 == 0. The path (small-M register path or
+ * large-M tensor-core path) is chosen per (bits, M, N, K) from a measured
+ * table; the environment variable QGEMM_PATH=small|large overrides it.
+ * Returns after enqueueing; a device-side failure (a bounded wait that ran
+ * out) is reported later by qgemm_get_device_status.
+ */
+int qgemm(const void* X, int32_t M, const qgemm_weights* W, void* out,
+          const void* bias, void* stream);
+
+/* As qgemm, with an explicit QGEMM_PATH_* choice (AUTO defers to the table and
+ * the QGEMM_PATH variable). */
+int qgemm_ex(const void* X, int32_t M, const qgemm_weights* W, void* out,
+             const void* bias, int32_t path, void* stream);
+
+/* The path qgemm would take for this shape: QGEMM_PATH_SMALL_M or
+ * QGEMM_PATH_LARGE_M, or a negative qgemm_status for an invalid shape. */
+int qgemm_select_path(int32_t M, int32_t N, int32_t K, int32_t bits);
+
+/*
+ * Debug entry point for the bit-exact gate: writes the dequantised weights
+ * W[n0 : n0+rows, k0 : k0+cols] as bf16 [rows, cols] (row-major, `out` a
+ * 16-byte aligned device buffer), using the same device dequantisation
+ * routine the large-M kernel applies to each shared-memory tile.
+ * Requires n0, k0 >= 0, n0 + rows <= N, k0 + cols <= K, k0 % 8 == 0 and
+ * cols % 8 == 0. Enqueued on `stream`.
+ */
+int qgemm_dequant_tile(const qgemm_weights* W, int32_t n0, int32_t k0, int32_t rows,
+                       int32_t cols, void* out, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's status
+ * word. Returns QGEMM_OK, QGEMM_ERR_DEVICE_TIMEOUT if a kernel gave up a
+ * bounded wait since the last read, or QGEMM_ERR_CUDA if the stream reports
+ * an error.
+ */
+int qgemm_get_device_status(void* stream);
+
+/* Upper bound, in nanoseconds, on any single wait inside a kernel (default
+ * 2e9, also settable with QGEMM_WAIT_LIMIT_NS). 0 restores the default. */
+int qgemm_set_wait_limit_ns(uint64_t limit_ns);
+
+/* Test hook for the timeout path: launches one block that waits on a
+ * barrier nothing will complete, giving up after `limit_ns`; the device
+ * status word then reads QGEMM_ERR_DEVICE_TIMEOUT. Faults and traps nothing. */
+int qgemm_debug_wait_timeout(uint64_t limit_ns, void* stream);
+
+/* Static description of a status code. */
+const char* qgemm_status_str(int status);
+
+/* Detail of the calling thread's last failed call ("" if none). */
+const char* qgemm_last_error(void);
+
+/* Library version string. */
+const char* qgemm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QGEMM_H */

