@@ -1,0 +1,610 @@
+#!/usr/bin/env python
+"""Benchmark of the weight-quantised GEMM at FLUX DiT linear shapes on B200.
+
+One step = one qgemm over the headline workload (FLUX double-stream image
+QKV projection: X bf16 [4096, 3072] times a 4-bit group-64 W [9216, 3072]
+plus a bf16 bias), inputs resident in HBM. Prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one process per GPU): the GEMM runs as independent
+replicas, one per rank, with no collective on the data path ("scaling":
+"weak"); the time is the max over ranks.
+
+Timing: CUDA events on the launching stream, after warm-up, with a barrier
+and synchronize on both sides. Inputs rotate over enough copies that the
+working set of consecutive steps exceeds the 126 MB L2. The per-shape sweep
+(every workload, both paths) times a CUDA graph of back-to-back launches.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HEADLINE_CID, HEADLINE_LIN = 1, 0
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "qgemm TFLOP/s (GB/s at small M) and % of roofline at FLUX DiT linear shapes"
+
+
+# ----------------------------------------------------------------------------
+# peaks
+# ----------------------------------------------------------------------------
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured (MEASURED_PEAKS.json)"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback (earlier measurement on this pool)"}
+
+
+def alg_bytes(lin, M=None):
+    """Bytes the method must move: packed W + scales (+ biases) + X + out (+ bias)."""
+    from weight_quantised_gemm_b200 import qgemm_pack_sizes
+    M = lin.M if M is None else M
+    p, s, b = qgemm_pack_sizes(lin.N, lin.K, lin.bits, lin.group)
+    return p + s + b + M * lin.K * 2 + M * lin.N * 2 + (lin.N * 2 if lin.bias else 0)
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "weight_quantised_gemm_b200", "csrc")
+    for f in ("large_m.cu", "dequant.cuh", "ptx.cuh"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the headline kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "large_m_qkv_4096x9216x3072_counters.json")
+    if not os.path.exists(p):
+        return None, "no ncu summary committed"
+    d = json.load(open(p))
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None, "kernel changed since the ncu capture"
+    return int(d["dram_bytes_read"]) + int(d["dram_bytes_write"]), "ncu capture " + d.get("when", "")
+
+
+# ----------------------------------------------------------------------------
+# clocks
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        rows = []
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) != 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [r for r in rows if r[3] >= 50.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[4]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing
+# ----------------------------------------------------------------------------
+
+def smi_device_id(local_rank: int) -> str:
+    """nvidia-smi's id for this process's GPU (CUDA_VISIBLE_DEVICES may list indices or UUIDs)."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def make_device_inputs(lin, cid, li, copies, M=None):
+    """Packed weights, X, bias and out buffers, `copies` independent sets."""
+    import numpy as np
+    import torch
+
+    import weight_quantised_gemm_b200 as wq
+    import workloads as WL
+    X, W, bias = WL.make_inputs(lin, cid, li, M=M)
+    pw = wq.qgemm_pack(W, lin.bits)
+    M = X.shape[0]
+    sets = []
+    for _ in range(copies):
+        dw = pw.to_device("cuda")
+        Xd = torch.from_numpy(X.view(np.int16)).cuda().view(torch.bfloat16)
+        bd = None if bias is None else torch.from_numpy(bias.view(np.int16)).cuda().view(torch.bfloat16)
+        out = torch.empty((M, lin.N), dtype=torch.bfloat16, device="cuda")
+        sets.append((Xd, dw, bd, out))
+    return sets, (X, W, bias, pw)
+
+
+def copies_for(nbytes: int, minimum: int) -> int:
+    return max(minimum, -(-3 * L2_BYTES // max(nbytes, 1)))
+
+
+def time_graph(fn_list, reps: int = 5):
+    """Per-launch device time of a CUDA graph replaying fn_list (back-to-back launches)."""
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for fn in fn_list[:3]:
+            fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for fn in fn_list:
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e-3 / len(fn_list))
+    del g
+    return statistics.median(times)
+
+
+def sweep(peaks):
+    """Every workload linear: time, TFLOP/s, GB/s and roofline fraction, plus
+    the small-M sweep on both paths and config 4's cosine against dense bf16."""
+    import torch
+
+    import weight_quantised_gemm_b200 as wq
+    import workloads as WL
+    res = []
+    P = peaks["bf16_tflops"] * 1e12
+    BW = peaks["hbm_gbs"] * 1e9
+
+    def one(cid, li, lin, M, path, launches):
+        ab = alg_bytes(lin, M)
+        ncopy = copies_for(ab, 3 if M > 16 else 32)
+        sets, host = make_device_inputs(lin, cid, li, ncopy, M=M)
+        fns = [(lambda s=s: wq.qgemm(s[0], s[1], bias=s[2], out=s[3], path=path)) for s in sets]
+        reps_list = (fns * (-(-launches // len(fns))))[:max(launches, len(fns))]
+        t = time_graph(reps_list)
+        wq.check_device_status()
+        flops = 2 * M * lin.N * lin.K
+        t_roof = max(flops / P, ab / BW)
+        entry = {"workload": cid, "linear": lin.name, "M": M, "N": lin.N, "K": lin.K, "bits": lin.bits,
+                 "path": "small" if path == wq.QGEMM_PATH_SMALL_M else "large" if path == wq.QGEMM_PATH_LARGE_M
+                 else ("small" if wq.qgemm_select_path(M, lin.N, lin.K, lin.bits) == 1 else "large"),
+                 "us": round(t * 1e6, 2), "tflops": round(flops / t / 1e12, 1), "gbs": round(ab / t / 1e9, 1),
+                 "bound": "tensor" if flops / P >= ab / BW else "hbm",
+                 "roofline_us": round(t_roof * 1e6, 2), "frac_of_roofline": round(t_roof / t, 3),
+                 "copies": ncopy}
+        return entry, sets, host
+
+    for cid in range(5):
+        wl = WL.workload(cid)
+        for li, lin in enumerate(wl.linears):
+            entry, sets, host = one(cid, li, lin, lin.M, wq.QGEMM_PATH_AUTO, 100 if lin.M <= 16 else 20)
+            if cid == 4:
+                Xd, dw, bd, out = sets[0]
+                X, W, bias, pw = host
+                Wb = torch.from_numpy(W).cuda().to(torch.bfloat16)
+                yq = wq.qgemm(Xd, dw, bias=bd).double()
+                yd = (Xd @ Wb.T).double()
+                entry["cosine_vs_dense_bf16"] = float(torch.nn.functional.cosine_similarity(
+                    yq.flatten(), yd.flatten(), dim=0))
+                entry["packed_bytes_over_dense_bf16"] = round(pw.nbytes / (lin.N * lin.K * 2), 4)
+                entry["packed_bytes_over_dense_fp32"] = round(pw.nbytes / (lin.N * lin.K * 4), 4)
+                entry["_yq"], entry["_yd"] = yq.flatten().cpu(), yd.flatten().cpu()
+                del Wb
+            res.append(entry)
+            del sets
+            torch.cuda.empty_cache()
+    # config 4 as a whole block
+    blk = [e for e in res if e["workload"] == 4]
+    yq = torch.cat([e.pop("_yq") for e in blk])
+    yd = torch.cat([e.pop("_yd") for e in blk])
+    block = {"cosine_vs_dense_bf16_all_five": float(torch.nn.functional.cosine_similarity(yq, yd, dim=0)),
+             "us_total": round(sum(e["us"] for e in blk), 1)}
+    wl4 = WL.workload(4)
+    packed = sum(wq.qgemm_pack_sizes(l.N, l.K, l.bits, l.group)[0] + 2 * wq.qgemm_pack_sizes(l.N, l.K, l.bits,
+                                                                                             l.group)[1]
+                 for l in wl4.linears)
+    dense = sum(l.N * l.K for l in wl4.linears)
+    block["packed_over_dense_bf16"] = round(packed / (2 * dense), 4)
+    block["packed_over_dense_fp32"] = round(packed / (4 * dense), 4)
+    block["tflops"] = round(sum(2 * l.M * l.N * l.K for l in wl4.linears) / (block["us_total"] * 1e-6) / 1e12, 1)
+    # small-M crossover sweep: both paths on the ternary and 4-bit decode shapes
+    cross = []
+    lin3 = WL.workload(3).linears[0]
+    import dataclasses
+    for bits in (2, 4, 8):
+        lin = dataclasses.replace(lin3, bits=bits, group=wq.GROUP_OF_BITS[bits],
+                                  w_dist="ternary" if bits == 2 else "normal")
+        for M in (1, 4, 8, 16, 32, 64):
+            for path in (wq.QGEMM_PATH_SMALL_M, wq.QGEMM_PATH_LARGE_M):
+                if path == wq.QGEMM_PATH_SMALL_M and M > 16:
+                    continue
+                e, sets, _ = one(3, 0, lin, M, path, 100)
+                cross.append({k: e[k] for k in ("bits", "M", "path", "us", "gbs", "frac_of_roofline")})
+                del sets
+    torch.cuda.empty_cache()
+    return res, block, cross
+
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import weight_quantised_gemm_b200 as wq
+    import workloads as WL
+    peaks = load_peaks()
+    lin = WL.workload(HEADLINE_CID).linears[HEADLINE_LIN]
+    ab = alg_bytes(lin)
+    ncopy = copies_for(ab, 3)
+    sets, host = make_device_inputs(lin, HEADLINE_CID, HEADLINE_LIN, ncopy)
+    flops = 2 * lin.M * lin.N * lin.K
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        Xd, dw, bd, out = sets[i % ncopy]
+        wq.qgemm(Xd, dw, bias=bd, out=out, stream=stream)
+
+    clocks = ClockSampler(smi_device_id(local_rank))
+    clocks.start()
+    for i in range(args.warmup):
+        step(i)
+    barrier(world)
+    st = wq.qgemm_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    t0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step(i)
+        ev[i][1].record(stream)
+    t1.record(stream)
+    barrier(world)
+    clk = clocks.stop()
+    st = wq.qgemm_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after timing")
+    elapsed = t0.elapsed_time(t1) * 1e-3
+    kernel_t = statistics.fmean(a.elapsed_time(b) for a, b in ev) * 1e-3
+    elapsed_max = max_over_ranks(elapsed, world)
+    kernel_max = max_over_ranks(kernel_t, world)
+
+    # end to end through the public API with host buffers: pinned X in, out back
+    X, W, bias, pw = host
+    e2e = run_e2e(sets, X, lin, args, world)
+
+    result = None
+    if rank == 0:
+        value = world * flops * args.steps / elapsed_max / 1e12
+        achieved = flops / kernel_max / 1e12
+        traffic, traffic_src = profiled_traffic()
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": traffic,
+                "peak_source": peaks["source"] + ", burst bf16 (kernel timed on its own)",
+                "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": ab,
+                "traffic_source": traffic_src, "kernel": "large_m_kernel<4>"}
+        result = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(elapsed_max / args.steps * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; W ~ N(0,0.02) RTN 4-bit g64, X ~ N(0,1), bias ~ N(0,0.01))",
+            "config": {"workload": "FLUX double-stream image QKV projection: X bf16 [4096,3072] x W 4-bit "
+                                   "group-64 [9216,3072] + bias bf16 [9216] -> bf16 [4096,9216]",
+                       "M": lin.M, "N": lin.N, "K": lin.K, "bits": lin.bits, "group": lin.group,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": f"inputs rotate over {ncopy} copies ({ncopy * ab / 1e6:.0f} MB > 126 MB L2)"},
+            "gbs": round(ab * args.steps * world / elapsed_max / 1e9, 1),
+            "roofline": roof,
+            "e2e": e2e,
+            "gpu_launches": args.steps,
+            "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+            "clocks_detail": clk,
+            "impl": "ours",
+        }
+    return result, peaks
+
+
+def run_e2e(sets, X_host_bits, lin, args, world):
+    """Pipelined host->device->host: per step, copy X in from pinned memory,
+    qgemm, copy out back to pinned memory, on three streams (PCIe in, compute,
+    PCIe out) with double buffers."""
+    import numpy as np
+    import torch
+
+    import weight_quantised_gemm_b200 as wq
+    M = lin.M
+    xh = [torch.from_numpy(X_host_bits.view(np.int16).copy()).view(torch.bfloat16).pin_memory() for _ in range(2)]
+    oh = [torch.empty((M, lin.N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    xd = [sets[i % len(sets)][0] for i in range(2)]
+    od = [sets[i % len(sets)][3] for i in range(2)]
+    dw, bd = sets[0][1], sets[0][2]
+    s_in, s_c, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_c = [torch.cuda.Event() for _ in range(2)]
+    ev_o = [torch.cuda.Event() for _ in range(2)]
+    steps = max(10, min(args.steps, 100))
+
+    def run(n):
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_c[b])
+                xd[b].copy_(xh[b], non_blocking=True)
+                ev_in[b].record(s_in)
+            with torch.cuda.stream(s_c):
+                s_c.wait_event(ev_in[b])
+                if i >= 2:
+                    s_c.wait_event(ev_o[b])
+                wq.qgemm(xd[b], dw, bias=bd, out=od[b], stream=s_c)
+                ev_c[b].record(s_c)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_c[b])
+                oh[b].copy_(od[b], non_blocking=True)
+                ev_o[b].record(s_out)
+
+    run(4)
+    barrier(world)
+    t0 = time.perf_counter()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    run(steps)
+    s_in.wait_stream(s_out)
+    e1.record(s_in)
+    barrier(world)
+    dt = e0.elapsed_time(e1) * 1e-3
+    wall = time.perf_counter() - t0
+    dt = max_over_ranks(dt, world)
+    flops = 2 * M * lin.N * lin.K
+    return {"value": round(world * flops * steps / dt / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": M * lin.K * 2, "d2h_bytes_per_step": M * lin.N * 2,
+            "steps": steps, "ms_per_step": round(dt / steps * 1e3, 4), "wall_s": round(wall, 3),
+            "how": "pinned host X -> device, qgemm, device out -> pinned host; copies and compute on three "
+                   "streams with double buffers; weights resident on the device"}
+
+
+# ----------------------------------------------------------------------------
+# CPU baseline: the oracle as it stands
+# ----------------------------------------------------------------------------
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_oracle_sample(target_s: float, lin=None, cid=HEADLINE_CID, li=HEADLINE_LIN):
+    """Times the oracle (dequant of the whole W + fp64 matmul) on a bounded
+    sample of the workload's rows and extrapolates to the full M: returns
+    (TFLOP/s, seconds spent, description)."""
+    import numpy as np
+
+    import oracle as O
+    import workloads as WL
+    lin = WL.workload(cid).linears[li] if lin is None else lin
+    X, W, bias = WL.make_inputs(lin, cid, li)
+    p, s, b = O.pack_ref(W, lin.bits, lin.group)
+    t0 = time.perf_counter()
+    Wq = O.wq_exact(p, s, b, lin.bits, lin.group, lin.K)
+    t_deq = time.perf_counter() - t0
+    rows = 16
+    spent = t_deq
+    t_mm = 0.0
+    while True:
+        t1 = time.perf_counter()
+        Xs = O.bf16_bits_to_f64(X[:rows])
+        out = Xs @ Wq.T
+        if bias is not None:
+            out += O.bf16_bits_to_f64(bias)[None, :]
+        t_mm = time.perf_counter() - t1
+        spent += t_mm
+        if spent >= target_s * 0.5 or rows >= lin.M:
+            break
+        rows = min(lin.M, rows * 4)
+    t_full = t_deq + t_mm * lin.M / rows
+    flops = 2 * lin.M * lin.N * lin.K
+    desc = (f"oracle (numpy fp64): dequant of the full W [{lin.N},{lin.K}] ({t_deq:.2f} s) + matmul of "
+            f"X rows 0..{rows - 1} of {lin.M} ({t_mm:.2f} s), extrapolated to all {lin.M} rows")
+    return flops / t_full / 1e12, spent, desc, rows
+
+
+def run_reference(args, rank, world):
+    """The base contract's reference arm, here the oracle on the host cores:
+    each step is a bounded sample of the headline workload."""
+    if rank != 0:
+        return None
+    import numpy as np
+
+    import oracle as O
+    import workloads as WL
+    lin = WL.workload(HEADLINE_CID).linears[HEADLINE_LIN]
+    X, W, bias = WL.make_inputs(lin, HEADLINE_CID, HEADLINE_LIN)
+    p, s, b = O.pack_ref(W, lin.bits, lin.group)
+    total_steps = args.steps + args.warmup
+    budget = 150.0 / max(total_steps, 1)       # seconds per step so the run ends within minutes
+    # a step: dequantise a block of W rows and multiply a block of X rows with it
+    n_rows = lin.N
+    t0 = time.perf_counter()
+    Wq = O.wq_exact(p[:256], s[:256], None if b is None else b[:256], lin.bits, lin.group, lin.K)
+    t_deq_256 = time.perf_counter() - t0
+    n_rows = int(max(64, min(lin.N, 256 * budget * 0.5 / max(t_deq_256, 1e-6))))
+    n_rows -= n_rows % 16
+    m_rows = 64
+
+    def one_step():
+        Wq = O.wq_exact(p[:n_rows], s[:n_rows], None if b is None else b[:n_rows], lin.bits, lin.group, lin.K)
+        out = O.bf16_bits_to_f64(X[:m_rows]) @ Wq.T
+        if bias is not None:
+            out += O.bf16_bits_to_f64(bias[:n_rows])[None, :]
+        return out
+
+    for _ in range(args.warmup):
+        one_step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one_step()
+    dt = time.perf_counter() - t0
+    flops = 2 * m_rows * n_rows * lin.K
+    value = flops * args.steps / dt / 1e12
+    cores = blas_threads()
+    sample = (f"per step: dequantise W rows 0..{n_rows - 1} of {lin.N} and multiply X rows 0..{m_rows - 1} of "
+              f"{lin.M} with them in fp64 (oracle as it stands)")
+    return {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "FLUX double-stream image QKV projection: X bf16 [4096,3072] x W 4-bit "
+                                   "group-64 [9216,3072] + bias bf16 [9216] -> bf16 [4096,9216]",
+                       "M": lin.M, "N": lin.N, "K": lin.K, "bits": lin.bits, "group": lin.group},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the per-workload sweep")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local_rank = dist_env()
+    if world != args.gpus and "RANK" in os.environ:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+
+    import torch
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res, peaks = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if not args.no_sweep and world == 1:
+                per, block, cross = sweep(peaks)
+                res["sweep"] = per
+                res["workload4_block"] = block
+                res["path_crossover"] = cross
+            if not args.no_cpu and world == 1:
+                v, spent, desc, _ = cpu_oracle_sample(args.cpu_seconds)
+                res["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOP/s", "cores": blas_threads(),
+                                       "kind": "oracle", "sample": desc, "seconds": round(spent, 2)}
+            res["peaks"] = peaks
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -135,12 +135,17 @@ def test_zero_weights_give_the_bias(path, M):
     assert np.array_equal(y, np.broadcast_to(bias, (M, 256)))
 
 
-def test_both_paths_agree_closely_at_m16():
+def test_both_paths_agree_at_m16():
+    """The paths differ by the large path's bf16 rounding of the dequantised
+    weight (~1.1e-3 rms relative) plus each one's bf16 output rounding."""
     X, W, bias = WL.random_case(77, 16, 512, 1024, 4, with_bias=True)
     ys, dw = gpu_qgemm(X, W, bias, 4, path=SMALL)
     yl = gpu_qgemm_packed(X, dw, bias, path=LARGE)
     a, b = O.bf16_bits_to_f64(ys), O.bf16_bits_to_f64(yl)
-    assert O.rel_frobenius(a, b) < 2e-3
+    assert O.rel_frobenius(a, b) < O.REL_FROB_TOL
+    ref = _ref(X, W, bias, 4)
+    # the small path keeps s*q + b exact, so it sits closer to the oracle
+    assert O.rel_frobenius(a, ref) < O.rel_frobenius(b, ref)
 
 
 def test_runs_on_a_side_stream_and_repeats_identically():
