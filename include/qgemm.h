@@ -30,7 +30,9 @@
  *   ternary a word holds 16 consecutive k: j = 2i in bits 2i..2i+1, j = 2i+1
  *           in bits 16+2i..17+2i; the code is t in 2-bit two's complement
  *           (00 = 0, 01 = +1, 11 = -1; 10 is invalid);
- *   scales, biases: fp16 [N, K / group], row-major.
+ *   scales, biases: fp16 [K / group, N], group-major: the values of one
+ *           group of k for all N rows are contiguous, so a tile's scales
+ *           arrive in one TMA box with its codes.
  * Even and odd k sit in the two half-words so that one shift and one mask
  * move a neighbouring pair of codes into the two lanes of a bf16x2 register.
  *
@@ -83,8 +85,8 @@ typedef struct qgemm_weights {
   int32_t bits;          /* 2 (ternary), 4 or 8 */
   int32_t group;         /* 128 for ternary, 64 for 4- and 8-bit */
   const void* packed;    /* uint8 [N, K * bits / 8], 16-byte aligned */
-  const void* scales;    /* fp16 [N, K / group], 16-byte aligned */
-  const void* biases;    /* fp16 [N, K / group], 16-byte aligned; NULL for ternary */
+  const void* scales;    /* fp16 [K / group, N], 16-byte aligned */
+  const void* biases;    /* fp16 [K / group, N], 16-byte aligned; NULL for ternary */
 } qgemm_weights;
 
 /*

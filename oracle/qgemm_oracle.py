@@ -43,7 +43,8 @@ Bit layout, row-major over N with K contiguous, little-endian 32-bit words:
 * ternary: a word holds 16 consecutive k; offset j = 2i in bits 2i..2i+1 and
   j = 2i + 1 in bits 16+2i..17+2i. The 2-bit code is t in two's complement
   (0 -> 00, +1 -> 01, -1 -> 11); code 10 is invalid.
-* scales and biases: fp16 [N, K / group], row-major.
+* scales and biases: fp16 [K / group, N], group-major (the scales of one
+  group of k for all rows are contiguous).
 
 Dequantised weight (the bit-exact contract of the dequant-tile entry point):
 
@@ -177,8 +178,8 @@ def check_format(bits: int, group: int, K: int) -> None:
 def pack_ref(W, bits: int, group: int):
     """RTN group quantisation of fp32 W [N, K].
 
-    Returns (packed uint8 [N, K*b/8], scales fp16 [N, K/g], biases fp16
-    [N, K/g] or None for ternary).
+    Returns (packed uint8 [N, K*b/8], scales fp16 [K/g, N], biases fp16
+    [K/g, N] or None for ternary), in the at-rest layout.
     """
     W = np.asarray(W, dtype=np.float32)
     N, K = W.shape
@@ -200,7 +201,7 @@ def pack_ref(W, bits: int, group: int):
             q = np.clip(np.rint((Wg - b) / s), 0, qmax)
         q = np.where(s == 0, 0, q)
         codes = q.reshape(N, K).astype(np.int64)
-        return pack_codes(codes, bits), s16, b16
+        return pack_codes(codes, bits), np.ascontiguousarray(s16.T), np.ascontiguousarray(b16.T)
     s16 = fp16_rn(np.abs(Wg).max(axis=2))
     if not np.all(np.isfinite(s16)):
         raise OverflowError("scale overflows fp16")
@@ -208,7 +209,7 @@ def pack_ref(W, bits: int, group: int):
     with np.errstate(divide="ignore", invalid="ignore"):
         t = np.clip(np.rint(Wg / s), -1, 1)
     t = np.where(s == 0, 0, t)
-    return pack_codes(t.reshape(N, K).astype(np.int64), bits), s16, None
+    return pack_codes(t.reshape(N, K).astype(np.int64), bits), np.ascontiguousarray(s16.T), None
 
 
 # ----------------------------------------------------------------------------
@@ -216,7 +217,8 @@ def pack_ref(W, bits: int, group: int):
 # ----------------------------------------------------------------------------
 
 def _expand(groupwise, group: int) -> np.ndarray:
-    return np.repeat(np.asarray(groupwise, dtype=np.float16).astype(np.float64), group, axis=1)
+    """At-rest [K/g, N] per-group values -> fp64 [N, K], one per weight."""
+    return np.repeat(np.asarray(groupwise, dtype=np.float16).T.astype(np.float64), group, axis=1)
 
 
 def wq_exact(packed, scales, biases, bits: int, group: int, K: int) -> np.ndarray:

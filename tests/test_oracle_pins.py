@@ -161,6 +161,8 @@ def test_affine_error_bound(bits):
     g = np.random.default_rng(5 + bits)
     W = (g.standard_normal((64, 512)) * 0.02).astype(np.float32)
     packed, s16, b16 = O.pack_ref(W, bits, 64)
+    assert s16.shape == (8, 64) and b16.shape == (8, 64)     # at rest: [K/group, N]
+    s16, b16 = s16.T, b16.T
     q = O.unpack_codes(packed, bits, 512)
     qmax = (1 << bits) - 1
     assert q.min() >= 0 and q.max() <= qmax
@@ -193,8 +195,8 @@ def test_affine_exact_grid_is_recovered(bits):
     W = (lo[:, None] + s[:, None] * q_true).astype(np.float32)
     assert np.array_equal(W.astype(np.float64), lo[:, None] + s[:, None] * q_true)  # exact in fp32
     packed, s16, b16 = O.pack_ref(W, bits, 64)
-    assert np.array_equal(s16[:, 0].astype(np.float64), s)
-    assert np.array_equal(b16[:, 0].astype(np.float64), lo)
+    assert np.array_equal(s16[0, :].astype(np.float64), s)
+    assert np.array_equal(b16[0, :].astype(np.float64), lo)
     assert np.array_equal(O.unpack_codes(packed, bits, 64), q_true)
 
 
@@ -204,12 +206,12 @@ def test_affine_degenerate_groups():
     W[2, :] = -0.0                 # negative zeros
     packed, s16, b16 = O.pack_ref(W, 4, 64)
     assert np.all(s16 == 0)
-    assert b16[1, 0] == np.float16(0.25)
+    assert b16[0, 1] == np.float16(0.25)
     assert np.all(O.unpack_codes(packed, 4, 64) == 0)
     wd = O.dequant_ref(packed, s16, b16, 4, 64, 64)
     assert np.all(wd[1] == 0.25) and np.all(wd[0] == 0) and np.all(wd[2] == 0)
     # a group of negative zeros stores a +0 bias, so it dequantises to +0 bits
-    assert b16.view(np.uint16)[2, 0] == 0
+    assert b16.view(np.uint16)[0, 2] == 0
     assert np.all(O.dequant_ref_bits(packed, s16, b16, 4, 64, 64)[2] == 0)
 
 
@@ -224,7 +226,7 @@ def test_ternary_constructed_weights_round_trip_exactly():
     codes = O.unpack_codes(packed, 2, lin.K)
     assert set(np.unique(codes).tolist()) <= {-1, 0, 1}
     assert np.array_equal(codes, t)
-    recon = np.repeat(s16.astype(np.float32), 128, axis=1) * codes
+    recon = np.repeat(s16.T.astype(np.float32), 128, axis=1) * codes
     assert np.array_equal(recon.astype(np.float32), W)
 
 
@@ -293,7 +295,7 @@ def test_dequant_monotone_and_within_bf16_rounding(bits):
             assert np.all(np.diff(wd[n, sl][order]) >= 0)
     # q = 0 gives the bias rounded to bf16
     zero = q == 0
-    b = np.repeat(b16, 64, axis=1)
+    b = np.repeat(b16.T, 64, axis=1)
     tb = torch.from_numpy(b.astype(np.float32)).to(torch.bfloat16).float().numpy()
     assert np.array_equal(wd[zero], tb[zero].astype(np.float64))
 
@@ -311,9 +313,9 @@ def test_dequant_final_rounding_matches_torch_bf16():
 def test_ternary_dequant_is_signed_scale():
     g = np.random.default_rng(8)
     t = g.integers(-1, 2, size=(8, 256))
-    s16 = g.uniform(0.01, 0.05, size=(8, 2)).astype(np.float16)
+    s16 = g.uniform(0.01, 0.05, size=(8, 2)).astype(np.float16)      # [N, K/128]
     packed = O.pack_codes(t, 2)
-    bits = O.dequant_ref_bits(packed, s16, None, 2, 128, 256)
+    bits = O.dequant_ref_bits(packed, np.ascontiguousarray(s16.T), None, 2, 128, 256)
     sb = torch.from_numpy(np.repeat(s16.astype(np.float32), 128, axis=1)).to(torch.bfloat16).float().numpy()
     assert np.array_equal(O.bf16_bits_to_f64(bits), t * sb.astype(np.float64))
     assert np.all(bits[t == 0] == 0)                      # +0, not -0

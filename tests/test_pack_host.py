@@ -76,4 +76,5 @@ def test_multithreaded_pack_matches_single_rows():
     whole = wq.qgemm_pack(W, 4)
     part = wq.qgemm_pack(W[1000:1016], 4)
     assert np.array_equal(whole.packed[1000:1016], part.packed)
-    assert np.array_equal(whole.scales[1000:1016].view(np.uint16), part.scales.view(np.uint16))
+    assert np.array_equal(whole.scales[:, 1000:1016].view(np.uint16), part.scales.view(np.uint16))
+    assert whole.scales.shape == (lin.K // 64, 2048)

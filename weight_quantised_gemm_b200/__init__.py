@@ -118,8 +118,8 @@ class PackedWeights:
     bits: int
     group: int
     packed: np.ndarray   # uint8 [N, K*bits/8]
-    scales: np.ndarray   # float16 [N, K/group]
-    biases: Optional[np.ndarray]
+    scales: np.ndarray   # float16 [K/group, N] (group-major)
+    biases: Optional[np.ndarray]  # float16 [K/group, N]
 
     @property
     def nbytes(self) -> int:
@@ -168,8 +168,8 @@ def qgemm_pack(W, bits: int, group: Optional[int] = None) -> PackedWeights:
     biases = np.empty(bb // 2, dtype=np.float16) if bb else None
     _check(_lib.qgemm_pack(W.ctypes.data, N, K, bits, group, packed.ctypes.data, scales.ctypes.data,
                            None if biases is None else biases.ctypes.data), "qgemm_pack")
-    return PackedWeights(N, K, bits, group, packed.reshape(N, -1), scales.reshape(N, -1),
-                         None if biases is None else biases.reshape(N, -1))
+    return PackedWeights(N, K, bits, group, packed.reshape(N, -1), scales.reshape(K // group, N),
+                         None if biases is None else biases.reshape(K // group, N))
 
 
 def _stream_handle(stream) -> Optional[int]:

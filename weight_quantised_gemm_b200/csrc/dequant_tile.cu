@@ -10,7 +10,7 @@ namespace {
 
 template <int BITS>
 __global__ void dequant_tile_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ scales,
-                                    const uint16_t* __restrict__ biases, int K, int n0, int k0, int rows,
+                                    const uint16_t* __restrict__ biases, int N, int K, int n0, int k0, int rows,
                                     int cols, uint4* __restrict__ out) {
   constexpr int G = BITS == 2 ? 128 : 64;
   const int chunks_per_row = cols / 8;
@@ -23,7 +23,7 @@ __global__ void dequant_tile_kernel(const uint8_t* __restrict__ packed, const ui
     const int n = n0 + r;
     const int k = k0 + 8 * cc;  // first k of the chunk (a multiple of 8)
     const int grp = k / G;
-    const size_t sidx = static_cast<size_t>(n) * (K / G) + grp;
+    const size_t sidx = static_cast<size_t>(grp) * N + n;  // scales are [K/G, N]
     const uint8_t* row = packed + static_cast<size_t>(n) * row_bytes;
     uint4 o;
     if constexpr (BITS == 4) {
@@ -53,15 +53,15 @@ int launch_dequant_tile(const Problem& p, int n0, int k0, int rows, int cols) {
   uint4* out = static_cast<uint4*>(p.out);
   switch (p.bits) {
     case 4:
-      dequant_tile_kernel<4><<<blocks, threads, 0, p.stream>>>(p.packed, p.scales, p.biases, p.K, n0, k0, rows,
+      dequant_tile_kernel<4><<<blocks, threads, 0, p.stream>>>(p.packed, p.scales, p.biases, p.N, p.K, n0, k0, rows,
                                                                cols, out);
       break;
     case 8:
-      dequant_tile_kernel<8><<<blocks, threads, 0, p.stream>>>(p.packed, p.scales, p.biases, p.K, n0, k0, rows,
+      dequant_tile_kernel<8><<<blocks, threads, 0, p.stream>>>(p.packed, p.scales, p.biases, p.N, p.K, n0, k0, rows,
                                                                cols, out);
       break;
     default:
-      dequant_tile_kernel<2><<<blocks, threads, 0, p.stream>>>(p.packed, p.scales, p.biases, p.K, n0, k0, rows,
+      dequant_tile_kernel<2><<<blocks, threads, 0, p.stream>>>(p.packed, p.scales, p.biases, p.N, p.K, n0, k0, rows,
                                                                cols, out);
   }
   return cuda_check(cudaGetLastError(), "dequant_tile_kernel launch");

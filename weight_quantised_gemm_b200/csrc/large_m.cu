@@ -10,17 +10,27 @@
 // tokens (the widest N an instruction takes) instead of 128, halving the
 // dequantisation work per FLOP against the usual orientation.
 //
-// Warp roles (448 threads):
-//   warp 0        TMA producer: per 64-wide K block, the activation tile
-//                 X[256 x 64] (128-byte swizzle) and the packed weight tile
-//                 [128 rows x 64 k] land in one pipeline stage.
+// Three shared-memory rings, each with its own full/empty mbarriers, keep the
+// three producers of an MMA operand independent:
+//   X ring   activation tiles X[256 x 64] (128-byte swizzle), filled by TMA,
+//            emptied by the MMA;
+//   W ring   packed weight tiles [128 rows x 64 k] plus the tile's 128 fp16
+//            scales and biases (group-major at rest, so one 256-byte TMA box
+//            each), filled by TMA, emptied by the dequantisers;
+//   A ring   dequantised bf16 weight tiles in the 128-byte-swizzled K-major
+//            layout of the UMMA descriptor, filled by the dequantisers,
+//            emptied by the MMA.
+// The W ring is deep and cheap, so dequantisation runs ahead of the MMA
+// without waiting for activation tiles.
+//
+// Warp roles (480 threads):
+//   warp 0        TMA producer of the X ring
 //   warp 1        MMA issuer (one thread) and TMEM owner (512 columns: two
 //                 256-column fp32 accumulators, so one tile's epilogue
-//                 overlaps the next tile's main loop).
-//   warps 2..9    dequantisers: unpack the packed tile, apply scale and bias
-//                 (the exact contract of include/qgemm.h) and write bf16 in
-//                 the 128-byte-swizzled K-major layout the MMA reads.
-//   warps 10..13  epilogue: tcgen05.ld the accumulator (each warp owns one
+//                 overlaps the next tile's main loop)
+//   warp 2        TMA producer of the W ring
+//   warps 3..10   dequantisers (one thread per tile row and 32-k half)
+//   warps 11..14  epilogue: tcgen05.ld the accumulator (each warp owns one
 //                 32-lane quarter = 32 weight rows), add the bias, round to
 //                 bf16, transpose through shared memory and TMA-store
 //                 [32 tokens x 128 features] boxes (coalesced 16-byte rows).
@@ -43,13 +53,15 @@ constexpr int BK = 64;       // K per pipeline stage: one 128-byte swizzle row o
 constexpr int UMMA_K = 16;
 constexpr int NUM_DEQ_WARPS = 8;
 constexpr int NUM_EPI_WARPS = 4;
-constexpr int WARP_PRODUCER = 0;
+constexpr int WARP_XLOAD = 0;
 constexpr int WARP_MMA = 1;
-constexpr int WARP_DEQ0 = 2;
-constexpr int WARP_EPI0 = WARP_DEQ0 + NUM_DEQ_WARPS;  // 10
-constexpr int NUM_THREADS = 32 * (WARP_EPI0 + NUM_EPI_WARPS);  // 448
+constexpr int WARP_WLOAD = 2;
+constexpr int WARP_DEQ0 = 3;
+constexpr int WARP_EPI0 = WARP_DEQ0 + NUM_DEQ_WARPS;            // 11
+constexpr int NUM_THREADS = 32 * (WARP_EPI0 + NUM_EPI_WARPS);   // 480
 constexpr int X_STAGE_BYTES = TILE_M * BK * 2;  // 32 KB
 constexpr int A_STAGE_BYTES = TILE_N * BK * 2;  // 16 KB
+constexpr int SB_BYTES = TILE_N * 2;            // one group's scales (or biases) for the tile's rows
 constexpr int OUT_ROWS = 32;                    // tokens per TMA store box
 constexpr int OUT_BUF_BYTES = OUT_ROWS * TILE_N * 2;
 constexpr int NUM_OUT_BUFS = 2;
@@ -62,36 +74,47 @@ template <int BITS>
 struct Cfg {
   static constexpr int kGroup = BITS == 2 ? 128 : 64;
   static constexpr int kWRowBytes = BK * BITS / 8;  // packed bytes per row per stage
-  static constexpr int kWStageBytes = TILE_N * kWRowBytes;
-  static constexpr int kStages = BITS == 8 ? 3 : 4;
+  static constexpr int kWTileBytes = TILE_N * kWRowBytes;
+  static constexpr int kSBBytes = BITS == 2 ? SB_BYTES : 2 * SB_BYTES;  // scales (+ biases)
+  static constexpr int kWStride = kWTileBytes + kSBBytes;             // one W-ring stage
+  static constexpr int kSX = 4;                          // X ring depth
+  static constexpr int kSA = 2;                          // A ring depth
+  static constexpr int kSW = BITS == 8 ? 5 : 8;          // W ring depth
   static constexpr int kOffX = 0;
-  static constexpr int kOffA = kOffX + kStages * X_STAGE_BYTES;
-  static constexpr int kOffW = kOffA + kStages * A_STAGE_BYTES;
-  static constexpr int kOffOut = kOffW + kStages * kWStageBytes;
+  static constexpr int kOffA = kOffX + kSX * X_STAGE_BYTES;
+  static constexpr int kOffW = kOffA + kSA * A_STAGE_BYTES;
+  static constexpr int kOffOut = kOffW + kSW * kWStride;
   static constexpr int kOffBar = kOffOut + NUM_OUT_BUFS * OUT_BUF_BYTES;
-  static constexpr int kNumBars = 3 * kStages + 5;
+  static constexpr int kNumBars = 2 * kSX + 2 * kSW + 2 * kSA + 5;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024 B
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(kOffA % 1024 == 0 && kOffW % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+  static_assert(kWStride % 128 == 0 && kOffOut % 128 == 0, "TMA boxes land on 128-byte boundaries");
 };
 
 struct Params {
   int M, N, K;
   int num_m_tiles, num_tiles, num_kb;
-  const uint16_t* scales;
-  const uint16_t* biases;
   const uint16_t* bias;
   uint64_t wait_limit_ns;
   unsigned int* status;
 };
 
+// Bounded wait of a whole warp: every lane waits, and the warp gives up as
+// one if any lane ran out of time (so no lane is left at a warp barrier).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_t lim, const volatile int* abort) {
+  const bool ok = ptx::mbar_wait(bar, parity, lim, abort);
+  return __all_sync(0xffffffffu, ok);
+}
+
 template <int BITS>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     large_m_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                   const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_out, const Params p) {
   using C = Cfg<BITS>;
-  constexpr int S = C::kStages;
+  constexpr int SX = C::kSX, SA = C::kSA, SW = C::kSW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = ptx::smem_u32(smem);
@@ -100,23 +123,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   auto x_stage = [&](int s) { return sbase + C::kOffX + s * X_STAGE_BYTES; };
   auto a_stage = [&](int s) { return sbase + C::kOffA + s * A_STAGE_BYTES; };
-  auto w_stage = [&](int s) { return C::kOffW + s * C::kWStageBytes; };  // offset into smem
+  auto w_stage = [&](int s) { return C::kOffW + s * C::kWStride; };  // byte offset into smem
   const uint32_t bar0 = sbase + C::kOffBar;
-  auto full_tma = [&](int s) { return bar0 + 8u * s; };
-  auto full_a = [&](int s) { return bar0 + 8u * (S + s); };
-  auto empty = [&](int s) { return bar0 + 8u * (2 * S + s); };
-  auto acc_full = [&](int b) { return bar0 + 8u * (3 * S + b); };
-  auto acc_empty = [&](int b) { return bar0 + 8u * (3 * S + 2 + b); };
-  const uint32_t drain_bar = bar0 + 8u * (3 * S + 4);
+  auto full_x = [&](int s) { return bar0 + 8u * s; };
+  auto empty_x = [&](int s) { return bar0 + 8u * (SX + s); };
+  auto full_w = [&](int s) { return bar0 + 8u * (2 * SX + s); };
+  auto empty_w = [&](int s) { return bar0 + 8u * (2 * SX + SW + s); };
+  auto full_a = [&](int s) { return bar0 + 8u * (2 * SX + 2 * SW + s); };
+  auto empty_a = [&](int s) { return bar0 + 8u * (2 * SX + 2 * SW + SA + s); };
+  const uint32_t bar1 = bar0 + 8u * (2 * SX + 2 * SW + 2 * SA);
+  auto acc_full = [&](int b) { return bar1 + 8u * b; };
+  auto acc_empty = [&](int b) { return bar1 + 8u * (2 + b); };
+  const uint32_t drain_bar = bar1 + 32u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   volatile int* epi_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      ptx::mbar_init(full_tma(s), 1);
+    for (int s = 0; s < SX; ++s) {
+      ptx::mbar_init(full_x(s), 1);
+      ptx::mbar_init(empty_x(s), 1);
+    }
+    for (int s = 0; s < SW; ++s) {
+      ptx::mbar_init(full_w(s), 1);
+      ptx::mbar_init(empty_w(s), NUM_DEQ_WARPS);
+    }
+    for (int s = 0; s < SA; ++s) {
       ptx::mbar_init(full_a(s), NUM_DEQ_WARPS);
-      ptx::mbar_init(empty(s), 1);
+      ptx::mbar_init(empty_a(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(acc_full(b), 1);
@@ -131,10 +165,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tmem_alloc(ptx::smem_u32(tmem_slot), TMEM_COLS);
     ptx::tmem_relinquish();
   }
-  if (warp == WARP_PRODUCER && lane == 0) {
+  if (warp == WARP_XLOAD && lane == 0) {
     ptx::tma_prefetch_desc(&tm_x);
-    ptx::tma_prefetch_desc(&tm_w);
     ptx::tma_prefetch_desc(&tm_out);
+  }
+  if (warp == WARP_WLOAD && lane == 0) {
+    ptx::tma_prefetch_desc(&tm_w);
+    ptx::tma_prefetch_desc(&tm_s);
+    if (BITS != 2) ptx::tma_prefetch_desc(&tm_b);
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -147,31 +185,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::set_status(p.status, kStatusTimeout);
   };
 
-  if (warp == WARP_PRODUCER) {
+  if (warp == WARP_XLOAD || warp == WARP_WLOAD) {
+    // ---------------- TMA producers ----------------
     if (lane == 0) {
+      const bool is_x = warp == WARP_XLOAD;
+      const int S = is_x ? SX : SW;
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
         const int n_tile = tile / p.num_m_tiles, m_tile = tile % p.num_m_tiles;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
           const int s = it % S;
-          const uint32_t round = it / S;
-          if (!ptx::mbar_wait(empty(s), (round & 1) ^ 1, lim, abort_flag)) {
+          const uint32_t par = ((it / S) & 1) ^ 1;
+          if (!ptx::mbar_wait(is_x ? empty_x(s) : empty_w(s), par, lim, abort_flag)) {
             give_up();
             ok = false;
             break;
           }
-          ptx::mbar_arrive_expect_tx(full_tma(s), X_STAGE_BYTES + C::kWStageBytes);
-          ptx::tma_load_2d(x_stage(s), &tm_x, kb * BK, m_tile * TILE_M, full_tma(s));
-          ptx::tma_load_2d(sbase + w_stage(s), &tm_w, kb * C::kWRowBytes, n_tile * TILE_N, full_tma(s));
+          if (is_x) {
+            ptx::mbar_arrive_expect_tx(full_x(s), X_STAGE_BYTES);
+            ptx::tma_load_2d(x_stage(s), &tm_x, kb * BK, m_tile * TILE_M, full_x(s));
+          } else {
+            const uint32_t dst = sbase + w_stage(s);
+            const int grp = (kb * BK) / C::kGroup;
+            ptx::mbar_arrive_expect_tx(full_w(s), C::kWStride);
+            ptx::tma_load_2d(dst, &tm_w, kb * C::kWRowBytes, n_tile * TILE_N, full_w(s));
+            ptx::tma_load_2d(dst + C::kWTileBytes, &tm_s, n_tile * TILE_N, grp, full_w(s));
+            if (BITS != 2) ptx::tma_load_2d(dst + C::kWTileBytes + SB_BYTES, &tm_b, n_tile * TILE_N, grp, full_w(s));
+          }
         }
       }
       // Let every load this thread issued land before the block can exit.
-      const uint32_t issued = it;
-      const uint32_t first = issued > static_cast<uint32_t>(S) ? issued - S : 0;
-      for (uint32_t i = first; i < issued; ++i) ptx::mbar_wait(full_tma(i % S), (i / S) & 1, lim, nullptr);
+      const uint32_t first = it > static_cast<uint32_t>(S) ? it - S : 0;
+      for (uint32_t i = first; i < it; ++i)
+        ptx::mbar_wait(is_x ? full_x(i % S) : full_w(i % S), (i / S) & 1, lim, nullptr);
     }
   } else if (warp == WARP_MMA) {
+    // ---------------- MMA issuer ----------------
     if (lane == 0) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
@@ -185,9 +235,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * ACC_COLS;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-          const int s = it % S;
-          const uint32_t par = (it / S) & 1;
-          if (!ptx::mbar_wait(full_tma(s), par, lim, abort_flag) || !ptx::mbar_wait(full_a(s), par, lim, abort_flag)) {
+          const int sx = it % SX, sa = it % SA;
+          if (!ptx::mbar_wait(full_x(sx), (it / SX) & 1, lim, abort_flag) ||
+              !ptx::mbar_wait(full_a(sa), (it / SA) & 1, lim, abort_flag)) {
             give_up();
             ok = false;
             break;
@@ -195,11 +245,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ptx::tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-            const uint64_t adesc = ptx::smem_desc_sw128_kmajor(a_stage(s) + kk * UMMA_K * 2);
-            const uint64_t bdesc = ptx::smem_desc_sw128_kmajor(x_stage(s) + kk * UMMA_K * 2);
+            const uint64_t adesc = ptx::smem_desc_sw128_kmajor(a_stage(sa) + kk * UMMA_K * 2);
+            const uint64_t bdesc = ptx::smem_desc_sw128_kmajor(x_stage(sx) + kk * UMMA_K * 2);
             ptx::tc_mma_f16_ss(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0);
           }
-          ptx::tc_commit(empty(s));
+          ptx::tc_commit(empty_x(sx));
+          ptx::tc_commit(empty_a(sa));
         }
         if (!ok) break;
         ptx::tc_commit(acc_full(buf));
@@ -213,32 +264,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int dq = threadIdx.x - 32 * WARP_DEQ0;  // 0..255
     const int r = dq & (TILE_N - 1);              // tile row this thread writes
     const int h = dq >> 7;                        // which 32-k half of the 64-k block
-    const int groups = p.K / C::kGroup;
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-      const int n = (tile / p.num_m_tiles) * TILE_N + r;
-      const bool row_ok = n < p.N;
-      const size_t srow = static_cast<size_t>(row_ok ? n : 0) * groups;
-      auto load_sb = [&](int kb, float& s, float& b) {
-        const size_t gi = srow + (kb * BK) / C::kGroup;
-        s = row_ok ? deq::h2f(__ldg(p.scales + gi)) : 0.f;
-        b = (BITS != 2 && row_ok) ? deq::h2f(__ldg(p.biases + gi)) : 0.f;
-      };
-      float s_nxt, b_nxt;
-      load_sb(0, s_nxt, b_nxt);
       for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-        const float s_cur = s_nxt, b_cur = b_nxt;
-        if (kb + 1 < p.num_kb) load_sb(kb + 1, s_nxt, b_nxt);
-        const int s = it % S;
-        bool got = ptx::mbar_wait(full_tma(s), (it / S) & 1, lim, abort_flag);
-        got = __all_sync(0xffffffffu, got);
-        if (!got) {
+        const int sw = it % SW, sa = it % SA;
+        if (!warp_wait(full_w(sw), (it / SW) & 1, lim, abort_flag) ||
+            !warp_wait(empty_a(sa), ((it / SA) & 1) ^ 1, lim, abort_flag)) {
           if (lane == 0) give_up();
           ok = false;
           break;
         }
-        const uint8_t* wsrc = smem + w_stage(s) + r * C::kWRowBytes + h * (C::kWRowBytes / 2);
+        const uint8_t* wst = smem + w_stage(sw);
+        const float s_cur = deq::h2f(reinterpret_cast<const uint16_t*>(wst + C::kWTileBytes)[r]);
+        const float b_cur =
+            BITS == 2 ? 0.f : deq::h2f(reinterpret_cast<const uint16_t*>(wst + C::kWTileBytes + SB_BYTES)[r]);
+        const uint8_t* wsrc = wst + r * C::kWRowBytes + h * (C::kWRowBytes / 2);
         uint4 o[4];
         if constexpr (BITS == 4) {
           const uint4 v = *reinterpret_cast<const uint4*>(wsrc);  // 4 words = 32 k
@@ -261,9 +302,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           o[2] = deq::chunk_ternary<0>(v.y, hs);
           o[3] = deq::chunk_ternary<1>(v.y, hs);
         }
+        // The packed stage has been read: give it back to the W producer.
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(empty_w(sw));
         // 128-byte swizzle, K-major: row r holds 8 chunks of 16 B; logical
         // chunk c sits at physical chunk c ^ (r % 8).
-        uint8_t* arow = smem + C::kOffA + s * A_STAGE_BYTES + r * (BK * 2);
+        uint8_t* arow = smem + C::kOffA + sa * A_STAGE_BYTES + r * (BK * 2);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int cidx = 4 * h + i;
@@ -271,7 +315,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         ptx::fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(full_a(s));
+        if (lane == 0) ptx::mbar_arrive(full_a(sa));
       }
     }
   } else {
@@ -288,8 +332,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int n = n0 + n_local;
       const float bias_f =
           (p.bias && n < p.N) ? __bfloat162float(__ushort_as_bfloat16(p.bias[n])) : 0.f;
-      bool got = ptx::mbar_wait(acc_full(buf), use & 1, lim, abort_flag);
-      got = __all_sync(0xffffffffu, got);
+      const bool got = warp_wait(acc_full(buf), use & 1, lim, abort_flag);
       if (!got && lane == 0) {
         *epi_abort = 1;
         give_up();
@@ -360,14 +403,16 @@ int get_encoder(EncodeTiledFn* fn) {
   return QGEMM_OK;
 }
 
-int make_map_2d(EncodeTiledFn enc, CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base,
-                uint64_t inner, uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+// 2-D tensor map: `inner` x `outer` elements, rows `row_stride_bytes` apart,
+// box `box_inner` x `box_outer`. Reads outside the tensor return zeros and
+// stores outside it are dropped.
+int make_map_2d(EncodeTiledFn enc, CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
                 CUtensorMapSwizzle swz, const char* what) {
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_stride_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  (void)elem_bytes;
   const CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -387,16 +432,28 @@ int launch_fmt(const Problem& pr, int nsm) {
   if (st != QGEMM_OK) return st;
   EncodeTiledFn enc;
   if ((st = get_encoder(&enc)) != QGEMM_OK) return st;
-  CUtensorMap tm_x, tm_w, tm_out;
+  CUtensorMap tm_x, tm_w, tm_s, tm_b, tm_out;
   const uint64_t wbytes = static_cast<uint64_t>(pr.K) * BITS / 8;
-  if ((st = make_map_2d(enc, &tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pr.X, pr.K, pr.M, uint64_t(pr.K) * 2, BK,
+  const uint64_t groups = static_cast<uint64_t>(pr.K) / C::kGroup;
+  const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;
+  if ((st = make_map_2d(enc, &tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pr.X, pr.K, pr.M, uint64_t(pr.K) * 2, BK,
                         TILE_M, CU_TENSOR_MAP_SWIZZLE_128B, "X")) != QGEMM_OK)
     return st;
-  if ((st = make_map_2d(enc, &tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pr.packed, wbytes, pr.N, wbytes,
-                        C::kWRowBytes, TILE_N, CU_TENSOR_MAP_SWIZZLE_NONE, "W")) != QGEMM_OK)
+  if ((st = make_map_2d(enc, &tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.packed, wbytes, pr.N, wbytes,
+                        C::kWRowBytes, TILE_N, none, "W")) != QGEMM_OK)
     return st;
-  if ((st = make_map_2d(enc, &tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pr.out, pr.N, pr.M, uint64_t(pr.N) * 2,
-                        TILE_N, OUT_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE, "out")) != QGEMM_OK)
+  if ((st = make_map_2d(enc, &tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.scales, pr.N, groups, uint64_t(pr.N) * 2,
+                        TILE_N, 1, none, "scales")) != QGEMM_OK)
+    return st;
+  if (BITS != 2) {
+    if ((st = make_map_2d(enc, &tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.biases, pr.N, groups, uint64_t(pr.N) * 2,
+                          TILE_N, 1, none, "biases")) != QGEMM_OK)
+      return st;
+  } else {
+    tm_b = tm_s;  // unused for ternary
+  }
+  if ((st = make_map_2d(enc, &tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pr.out, pr.N, pr.M, uint64_t(pr.N) * 2,
+                        TILE_N, OUT_ROWS, none, "out")) != QGEMM_OK)
     return st;
   unsigned int* status;
   if ((st = status_word(&status)) != QGEMM_OK) return st;
@@ -408,13 +465,11 @@ int launch_fmt(const Problem& pr, int nsm) {
   const int num_n_tiles = (pr.N + TILE_N - 1) / TILE_N;
   kp.num_tiles = kp.num_m_tiles * num_n_tiles;
   kp.num_kb = pr.K / BK;
-  kp.scales = pr.scales;
-  kp.biases = pr.biases;
   kp.bias = pr.bias;
   kp.wait_limit_ns = wait_limit_ns();
   kp.status = status;
   const int grid = kp.num_tiles < nsm ? kp.num_tiles : nsm;
-  large_m_kernel<BITS><<<grid, NUM_THREADS, C::kSmemBytes, pr.stream>>>(tm_x, tm_w, tm_out, kp);
+  large_m_kernel<BITS><<<grid, NUM_THREADS, C::kSmemBytes, pr.stream>>>(tm_x, tm_w, tm_s, tm_b, tm_out, kp);
   return cuda_check(cudaGetLastError(), "large_m_kernel launch");
 }
 

@@ -101,7 +101,7 @@ int pack_rows(const PackJob& jb, int r0, int r1) {
       for (int i = 0; i < G; ++i) {
         if (!std::isfinite(wg[i])) return QGEMM_ERR_NONFINITE;
       }
-      const size_t sidx = static_cast<size_t>(n) * groups + g;
+      const size_t sidx = static_cast<size_t>(g) * jb.N + n;  // group-major [K/group, N]
       if (bits == 2) {
         double amax = 0.0;
         for (int i = 0; i < G; ++i) amax = std::max(amax, std::fabs(static_cast<double>(wg[i])));

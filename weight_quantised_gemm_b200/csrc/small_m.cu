@@ -36,8 +36,8 @@ constexpr int kThreads = 32 * kKSplit;
 struct SmallParams {
   const uint16_t* X;       // bf16 [M, K]
   const uint8_t* packed;   // [N, K*bits/8]
-  const uint16_t* scales;  // fp16 [N, K/G]
-  const uint16_t* biases;  // fp16 [N, K/G] (affine)
+  const uint16_t* scales;  // fp16 [K/G, N]
+  const uint16_t* biases;  // fp16 [K/G, N] (affine)
   const uint16_t* bias;    // bf16 [N] or null
   uint16_t* out;           // bf16 [M, N]
   int M, N, K;
@@ -135,7 +135,6 @@ __global__ void __launch_bounds__(kThreads) small_m_kernel(const SmallParams p) 
   const int g_begin = warp * per_warp;
   const int g_end = min(groups, g_begin + per_warp);
   const size_t row_bytes = static_cast<size_t>(p.K) * BITS / 8;
-  const int sgroups = groups;
 
   // rows this thread decodes (B operand column g of each n8 block)
   const uint8_t* wrow[2];
@@ -196,16 +195,23 @@ __global__ void __launch_bounds__(kThreads) small_m_kernel(const SmallParams p) 
     }
     if (gi + 1 < g_end) load_group(gi + 1, w_nxt, xg_nxt, xg8_nxt);
 
-    // scale / bias of the two weight rows this thread's accumulators cover
+    // scale / bias of the two adjacent weight rows this thread's accumulators
+    // cover: one 32-bit load each from the group-major [K/G, N] arrays
     float s[2][2], bb[2][2];
 #pragma unroll
-    for (int b = 0; b < 2; ++b)
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const size_t si = static_cast<size_t>(n_base + 8 * b + 2 * c + j) * sgroups + gi;
-        s[b][j] = deq::h2f(__ldg(p.scales + si));
-        bb[b][j] = BITS == 2 ? 0.f : deq::h2f(__ldg(p.biases + si));
+    for (int b = 0; b < 2; ++b) {
+      const size_t si = static_cast<size_t>(gi) * p.N + n_base + 8 * b + 2 * c;
+      const uint32_t sv = __ldg(reinterpret_cast<const uint32_t*>(p.scales + si));
+      s[b][0] = deq::h2f(static_cast<uint16_t>(sv & 0xFFFFu));
+      s[b][1] = deq::h2f(static_cast<uint16_t>(sv >> 16));
+      if constexpr (BITS != 2) {
+        const uint32_t bv = __ldg(reinterpret_cast<const uint32_t*>(p.biases + si));
+        bb[b][0] = deq::h2f(static_cast<uint16_t>(bv & 0xFFFFu));
+        bb[b][1] = deq::h2f(static_cast<uint16_t>(bv >> 16));
+      } else {
+        bb[b][0] = bb[b][1] = 0.f;
       }
+    }
 
     float tmp[2][4], xs[4];
 #pragma unroll
