@@ -384,42 +384,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-int get_encoder(EncodeTiledFn* fn) {
-  static EncodeTiledFn cached = nullptr;
-  static std::once_flag once;
-  static cudaError_t err = cudaSuccess;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
-    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) cached = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  if (!cached) return fail(QGEMM_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorName(err));
-  *fn = cached;
-  return QGEMM_OK;
-}
-
-// 2-D tensor map: `inner` x `outer` elements, rows `row_stride_bytes` apart,
-// box `box_inner` x `box_outer`. Reads outside the tensor return zeros and
-// stores outside it are dropped.
-int make_map_2d(EncodeTiledFn enc, CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
-                uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
-                CUtensorMapSwizzle swz, const char* what) {
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {row_stride_bytes};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(QGEMM_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with %d", what, int(r));
-  return QGEMM_OK;
-}
-
 template <int BITS>
 int launch_fmt(const Problem& pr, int nsm) {
   using C = Cfg<BITS>;
@@ -430,29 +394,27 @@ int launch_fmt(const Problem& pr, int nsm) {
   });
   int st = cuda_check(attr_err, "cudaFuncSetAttribute(large_m_kernel)");
   if (st != QGEMM_OK) return st;
-  EncodeTiledFn enc;
-  if ((st = get_encoder(&enc)) != QGEMM_OK) return st;
   CUtensorMap tm_x, tm_w, tm_s, tm_b, tm_out;
   const uint64_t wbytes = static_cast<uint64_t>(pr.K) * BITS / 8;
   const uint64_t groups = static_cast<uint64_t>(pr.K) / C::kGroup;
   const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;
-  if ((st = make_map_2d(enc, &tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pr.X, pr.K, pr.M, uint64_t(pr.K) * 2, BK,
+  if ((st = make_tensor_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pr.X, pr.K, pr.M, uint64_t(pr.K) * 2, BK,
                         TILE_M, CU_TENSOR_MAP_SWIZZLE_128B, "X")) != QGEMM_OK)
     return st;
-  if ((st = make_map_2d(enc, &tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.packed, wbytes, pr.N, wbytes,
+  if ((st = make_tensor_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.packed, wbytes, pr.N, wbytes,
                         C::kWRowBytes, TILE_N, none, "W")) != QGEMM_OK)
     return st;
-  if ((st = make_map_2d(enc, &tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.scales, pr.N, groups, uint64_t(pr.N) * 2,
+  if ((st = make_tensor_map_2d(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.scales, pr.N, groups, uint64_t(pr.N) * 2,
                         TILE_N, 1, none, "scales")) != QGEMM_OK)
     return st;
   if (BITS != 2) {
-    if ((st = make_map_2d(enc, &tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.biases, pr.N, groups, uint64_t(pr.N) * 2,
+    if ((st = make_tensor_map_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.biases, pr.N, groups, uint64_t(pr.N) * 2,
                           TILE_N, 1, none, "biases")) != QGEMM_OK)
       return st;
   } else {
     tm_b = tm_s;  // unused for ternary
   }
-  if ((st = make_map_2d(enc, &tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pr.out, pr.N, pr.M, uint64_t(pr.N) * 2,
+  if ((st = make_tensor_map_2d(&tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pr.out, pr.N, pr.M, uint64_t(pr.N) * 2,
                         TILE_N, OUT_ROWS, none, "out")) != QGEMM_OK)
     return st;
   unsigned int* status;

@@ -1,6 +1,7 @@
 // Internal interface between the host ABI layer and the kernel launchers.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstddef>
@@ -32,6 +33,13 @@ uint64_t wait_limit_ns();
 // Device address of the current device's status word (cached per device).
 int status_word(unsigned int** ptr);
 int sm_count(int* n);
+
+// 2-D TMA descriptor: `inner` x `outer` elements, rows `row_stride_bytes`
+// apart, box `box_inner` x `box_outer`. Reads outside the tensor return zeros
+// and stores outside it are dropped.
+int make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz,
+                       const char* what);
 
 // Kernel launchers (one per kernel family). Each enqueues on p.stream.
 int launch_small_m(const Problem& p);

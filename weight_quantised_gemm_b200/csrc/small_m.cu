@@ -1,46 +1,77 @@
-// Small-M path (M <= 16): a memory-bound GEMV-like kernel.
+// Small-M path (M <= 16): a memory-bound kernel that streams the packed
+// weights once.
 //
-// The packed weights stream from HBM with 8- or 16-byte loads straight into
-// registers; each thread turns its codes into bf16 in registers and feeds
-// them to the tensor cores through warp-level mma.sync (m16n8k16, bf16 in,
-// fp32 accumulate). The activations are the 16-row A operand (rows past M
-// are zero), the weights the 8-column B operand.
+// pictor's README ("Extreme quantization is first-class") names GEMV paths
+// built for sub-byte weights; at decode-sized M the packed bytes set the time,
+// so this kernel is built around keeping HBM busy:
+//
+// * One CTA per SM owns a contiguous range of weight rows (whole n8 blocks).
+//   A producer warp streams that range through a shared-memory ring with TMA:
+//   per stage, the packed codes of 128 bytes of K for every row (128-byte
+//   swizzle), the stage's fp16 scales (and biases) as one box, and the
+//   matching slice of the activations, copied row by row with bulk copies
+//   into a padded layout. The ring holds up to eight stages, so at the
+//   workloads' K every load of the CTA is in flight from the start.
+// * Eight consumer warps turn codes into bf16 in registers and feed warp-level
+//   mma.sync (m16n8k16, bf16 in, fp32 accumulate): the activations are the
+//   16-row A operand (rows past M are zero), the weights the 8-column B.
+//   The warps split each stage by whole groups and meet once, at the end, in
+//   shared memory.
 //
 // Scale and bias are applied per group on the fp32 partial sums instead of
-// per weight, which is algebraically the same product:
+// per weight, which is the same product:
 //     sum_k x_k (s q_k + b) = s * sum_k x_k q_k + b * sum_k x_k
-// so the per-weight register work is only "code -> bf16": q as an exact bf16
-// integer (4-bit: 128 + q, the offset removed per group; 8-bit: q), ternary
-// t as the bf16 {-2, 0, +2} (the factor 2 folded into s / 2). sum_k x_k per
-// group comes from one extra mma against a B operand of ones.
+// so the per-weight work is only "code -> bf16": 4-bit q as bf16 128 + q (the
+// offset removed per group as -128 * sum x), ternary t as bf16 {-2, 0, +2}
+// (the factor 2 folded into s / 2), 8-bit q exactly through an fp32 magic
+// number. sum_k x_k per group comes from one extra mma against ones.
 //
-// The k order inside one mma step is free (the tensor core sums over all 16
-// slots), so each thread of a quad takes 4 consecutive k of its quarter of
-// the group: its activation loads are plain contiguous vectors and its code
-// pairs sit where the packed layout puts them (even/odd k in the two
-// half-words of a 32-bit word).
-//
-// Work split: a CTA owns 16 weight rows (two mma n8 blocks); its 4 warps split
-// the K range by whole groups, and their partial sums meet in shared memory.
+// Inside one mma step (16 consecutive k of one group) thread c of each quad
+// takes k = 4c .. 4c+3: the tensor core sums all 16 slots, so any assignment
+// works, and this one makes each activation fetch one 8-byte vector and puts
+// the thread's code pairs where the packed layout keeps them (even and odd k
+// in the two half-words of a 32-bit word).
+
+#include <cuda.h>
+
+#include <mutex>
 
 #include "dequant.cuh"
 #include "qgemm_internal.h"
 
 namespace qg {
-namespace {
+namespace sm {
 
-constexpr int kRowsPerCta = 16;
-constexpr int kKSplit = 4;
-constexpr int kThreads = 32 * kKSplit;
+constexpr int NBMAX = 12;             // n8 blocks (of 8 weight rows) per CTA, at most
+constexpr int NUM_CONSUMER_WARPS = 8;
+constexpr int WARP_PRODUCER = NUM_CONSUMER_WARPS;
+constexpr int NUM_THREADS = 32 * (NUM_CONSUMER_WARPS + 1);  // 288
+constexpr int MAX_STAGES = 8;
+constexpr int ROW_BYTES_PER_STAGE = 128;  // one 128-byte swizzle row of packed codes
+constexpr int RING_BUDGET = 196608;       // bytes of shared memory for the ring
 
-struct SmallParams {
-  const uint16_t* X;       // bf16 [M, K]
-  const uint8_t* packed;   // [N, K*bits/8]
-  const uint16_t* scales;  // fp16 [K/G, N]
-  const uint16_t* biases;  // fp16 [K/G, N] (affine)
-  const uint16_t* bias;    // bf16 [N] or null
-  uint16_t* out;           // bf16 [M, N]
+template <int BITS>
+struct Fmt {
+  static constexpr int G = BITS == 2 ? 128 : 64;          // group size
+  static constexpr int KS = ROW_BYTES_PER_STAGE * 8 / BITS;  // k per stage: 512, 256 or 128
+  static constexpr int GS = KS / G;                        // groups per stage: 4, 4, 2
+  static constexpr int STEPS = G / 16;                     // mma k-steps per group
+  static constexpr int NSETS = NUM_CONSUMER_WARPS / GS;    // warps sharing out the stages
+  static constexpr int GBYTES = G * BITS / 8;              // packed bytes per row and group
+};
+
+struct Params {
+  const uint16_t* X;     // bf16 [M, K]
+  const uint16_t* bias;  // bf16 [N] or null
+  uint16_t* out;         // bf16 [M, N]
   int M, N, K;
+  int bpc;               // n8 blocks per CTA
+  int num_stages;        // K / KS, rounded up
+  int ring;              // ring depth
+  int stage_bytes;       // bytes per ring stage (multiple of 1024)
+  int off_s, off_b, off_x, x_stride;  // offsets inside a stage; X row stride in bytes
+  uint64_t wait_limit_ns;
+  unsigned int* status;
 };
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -51,238 +82,344 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-template <int BITS>
-struct SmallFmt {
-  static constexpr int G = BITS == 2 ? 128 : 64;  // group size
-  static constexpr int STEPS = G / 16;            // mma k-steps per group
-  static constexpr int QCODES = G / 4;            // codes per thread per group (its quarter)
-  static constexpr int QWORDS = QCODES * BITS / 32;  // 32-bit words per thread per group and row
-  static constexpr int XWORDS = QCODES / 2;       // bf16x2 words of X per thread per group and token row
-};
-
-// B operand (two bf16x2 registers) for step `st` from the thread's words.
-template <int BITS, int ST>
-__device__ __forceinline__ void decode_step(const uint32_t* w, uint32_t& b0, uint32_t& b1) {
-  if constexpr (BITS == 4) {
-    // 8 codes per word; step ST uses in-word offsets 4(ST%2) .. +3 of word ST/2
-    const uint32_t x = w[ST / 2];
-    constexpr int I0 = 2 * (ST % 2);
-    b0 = ((x >> (4 * I0)) & 0x000F000Fu) | 0x43004300u;        // bf16 128 + q
-    b1 = ((x >> (4 * (I0 + 1))) & 0x000F000Fu) | 0x43004300u;
-  } else if constexpr (BITS == 2) {
-    // 16 codes per word; step ST uses offsets 4(ST%4) .. +3 of word ST/4
-    const uint32_t x = w[ST / 4];
-    constexpr int I0 = 2 * (ST % 4);
-    b0 = deq::ternary_pair_pm2<I0>(x);                          // bf16 {-2, 0, 2}
-    b1 = deq::ternary_pair_pm2<I0 + 1>(x);
-  } else {
-    // 4 codes per word, one word per step: exact integer q in bf16
-    const uint32_t x = w[ST];
-    const float2 q01 = ptx::add2(make_float2(__uint_as_float(ptx::prmt(x, deq::kMagic, 0x7650u)),
-                                             __uint_as_float(ptx::prmt(x, deq::kMagic, 0x7651u))),
-                                 make_float2(-deq::kMagicF, -deq::kMagicF));
-    const float2 q23 = ptx::add2(make_float2(__uint_as_float(ptx::prmt(x, deq::kMagic, 0x7652u)),
-                                             __uint_as_float(ptx::prmt(x, deq::kMagic, 0x7653u))),
-                                 make_float2(-deq::kMagicF, -deq::kMagicF));
-    b0 = ptx::cvt_bf16x2(q01.x, q01.y);
-    b1 = ptx::cvt_bf16x2(q23.x, q23.y);
-  }
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
 }
 
-template <int BITS, int ST, int STEPS>
-struct StepLoop {
-  template <int MT>
-  __device__ __forceinline__ static void run(const uint32_t (&xg)[SmallFmt<BITS>::XWORDS],
-                                             const uint32_t (&xg8)[SmallFmt<BITS>::XWORDS],
-                                             const uint32_t (&w)[2][SmallFmt<BITS>::QWORDS], float (&tmp)[2][4],
-                                             float (&xs)[4]) {
-    uint32_t a[4];
-    a[0] = xg[2 * ST];
-    a[2] = xg[2 * ST + 1];
-    a[1] = MT > 8 ? xg8[2 * ST] : 0u;
-    a[3] = MT > 8 ? xg8[2 * ST + 1] : 0u;
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_t lim, const volatile int* abort) {
+  const bool ok = ptx::mbar_wait(bar, parity, lim, abort);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// The packed codes a thread needs for one group of one weight row, fetched
+// from the stage's 128-byte-swizzled row (logical 16-byte chunk j of row r
+// sits at physical chunk j ^ (r % 8)).
+//   ternary, 4-bit: the group's 32 bytes (8 words); quad threads share them.
+//   8-bit: the group's 64 bytes are 4 words per step; thread c keeps word c.
+template <int BITS>
+struct Codes {
+  static constexpr int WPT = BITS == 8 ? 4 : 8;
+  uint32_t w[WPT];
+
+  __device__ __forceinline__ void load(const uint8_t* row, int gs, int r, int c) {
+    if constexpr (BITS == 8) {
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      uint32_t b0, b1;
-      decode_step<BITS, ST>(w[b], b0, b1);
-      mma_bf16_16816(tmp[b], a, b0, b1);
+      for (int st = 0; st < 4; ++st)
+        w[st] = *reinterpret_cast<const uint32_t*>(row + (((4 * gs + st) ^ (r & 7)) << 4) + 4 * c);
+    } else {
+      const uint4 lo = *reinterpret_cast<const uint4*>(row + (((2 * gs) ^ (r & 7)) << 4));
+      const uint4 hi = *reinterpret_cast<const uint4*>(row + (((2 * gs + 1) ^ (r & 7)) << 4));
+      w[0] = lo.x; w[1] = lo.y; w[2] = lo.z; w[3] = lo.w;
+      w[4] = hi.x; w[5] = hi.y; w[6] = hi.z; w[7] = hi.w;
     }
-    if constexpr (BITS != 2) mma_bf16_16816(xs, a, 0x3F803F80u, 0x3F803F80u);  // sum of x over the step
-    StepLoop<BITS, ST + 1, STEPS>::template run<MT>(xg, xg8, w, tmp, xs);
+  }
+
+  // B operand of step ST for quad thread c: codes 4c .. 4c+3 of the step's
+  // 16 k as two bf16x2 registers (k pairs (4c, 4c+1) and (4c+2, 4c+3)).
+  template <int ST>
+  __device__ __forceinline__ void decode(int c, uint32_t& b0, uint32_t& b1) const {
+    if constexpr (BITS == 2) {
+      // one word = one step (16 codes); pairs 2c and 2c+1 of the word
+      const uint32_t x = w[ST];
+      b0 = (x << (14 - 4 * c)) & 0xC000C000u;  // bf16 {-2, 0, +2}
+      b1 = (x << (12 - 4 * c)) & 0xC000C000u;
+    } else if constexpr (BITS == 4) {
+      // two words per step; thread c reads word c/2, pairs 2(c%2) and 2(c%2)+1
+      const uint32_t x = (c >> 1) ? w[2 * ST + 1] : w[2 * ST];
+      const int sh = 8 * (c & 1);
+      b0 = ((x >> sh) & 0x000F000Fu) | 0x43004300u;  // bf16 128 + q
+      b1 = ((x >> (sh + 4)) & 0x000F000Fu) | 0x43004300u;
+    } else {
+      // byte j of the thread's word is code 4c + j; exact q through an fp32 magic number
+      const uint32_t x = w[ST];
+      const float2 q01 = ptx::add2(make_float2(__uint_as_float(ptx::prmt(x, deq::kMagic, 0x7650u)),
+                                               __uint_as_float(ptx::prmt(x, deq::kMagic, 0x7651u))),
+                                   make_float2(-deq::kMagicF, -deq::kMagicF));
+      const float2 q23 = ptx::add2(make_float2(__uint_as_float(ptx::prmt(x, deq::kMagic, 0x7652u)),
+                                               __uint_as_float(ptx::prmt(x, deq::kMagic, 0x7653u))),
+                                   make_float2(-deq::kMagicF, -deq::kMagicF));
+      b0 = ptx::cvt_bf16x2(q01.x, q01.y);
+      b1 = ptx::cvt_bf16x2(q23.x, q23.y);
+    }
+  }
+};
+
+// One group of one weight block: 16-k steps against the activation
+// fragments, accumulated into tmp (one mma per step).
+template <int BITS, int ST, int STEPS>
+struct GroupSteps {
+  __device__ __forceinline__ static void run(const Codes<BITS>& cd, int c, const uint2 (&xa)[STEPS],
+                                             const uint2 (&xb)[STEPS], float (&tmp)[4]) {
+    uint32_t a[4] = {xa[ST].x, xb[ST].x, xa[ST].y, xb[ST].y};
+    uint32_t b0, b1;
+    cd.template decode<ST>(c, b0, b1);
+    mma_bf16_16816(tmp, a, b0, b1);
+    GroupSteps<BITS, ST + 1, STEPS>::run(cd, c, xa, xb, tmp);
   }
 };
 
 template <int BITS, int STEPS>
-struct StepLoop<BITS, STEPS, STEPS> {
-  template <int MT>
-  __device__ __forceinline__ static void run(const uint32_t (&)[SmallFmt<BITS>::XWORDS],
-                                             const uint32_t (&)[SmallFmt<BITS>::XWORDS],
-                                             const uint32_t (&)[2][SmallFmt<BITS>::QWORDS], float (&)[2][4],
+struct GroupSteps<BITS, STEPS, STEPS> {
+  __device__ __forceinline__ static void run(const Codes<BITS>&, int, const uint2 (&)[STEPS], const uint2 (&)[STEPS],
                                              float (&)[4]) {}
 };
 
 template <int BITS, int MT>
-__global__ void __launch_bounds__(kThreads) small_m_kernel(const SmallParams p) {
-  using F = SmallFmt<BITS>;
-  constexpr int G = F::G;
-  __shared__ float red[kKSplit][MT][kRowsPerCta];
-
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    small_m_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
+                   const __grid_constant__ CUtensorMap tm_b, const Params p) {
+  using F = Fmt<BITS>;
+  constexpr int STEPS = F::STEPS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = ptx::smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
-  const int n_base = blockIdx.x * kRowsPerCta;
-  const int groups = p.K / G;
-  const int per_warp = (groups + kKSplit - 1) / kKSplit;
-  const int g_begin = warp * per_warp;
-  const int g_end = min(groups, g_begin + per_warp);
-  const size_t row_bytes = static_cast<size_t>(p.K) * BITS / 8;
 
-  // rows this thread decodes (B operand column g of each n8 block)
-  const uint8_t* wrow[2];
-#pragma unroll
-  for (int b = 0; b < 2; ++b) wrow[b] = p.packed + static_cast<size_t>(n_base + 8 * b + g) * row_bytes;
-  // activation rows of the A operand (zero past M)
-  const bool xg_ok = g < p.M;
-  const bool xg8_ok = MT > 8 && (g + 8) < p.M;
-  const uint16_t* xrow_g = p.X + static_cast<size_t>(xg_ok ? g : 0) * p.K;
-  const uint16_t* xrow_g8 = p.X + static_cast<size_t>(xg8_ok ? g + 8 : 0) * p.K;
+  const int nblocks_total = p.N / 8;
+  const int blk0 = blockIdx.x * p.bpc;
+  const int nb = min(p.bpc, nblocks_total - blk0);
+  const int n0 = 8 * blk0;
+  const int R = 8 * p.bpc;  // rows per TMA box (rows past N read as zeros)
+  const int data_bytes = max(p.ring * p.stage_bytes, NUM_CONSUMER_WARPS * NBMAX * 32 * 16);
+  const uint32_t bar0 = sbase + data_bytes;
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (MAX_STAGES + s); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + data_bytes + 16 * MAX_STAGES);
+  const uint64_t lim = p.wait_limit_ns;
 
-  float acc[2][4];
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.ring; ++s) {
+      ptx::mbar_init(full(s), 1);
+      ptx::mbar_init(empty(s), F::GS);
+    }
+    *abort_flag = 0;
+    ptx::fence_mbarrier_init();
+  }
+  __syncthreads();
+  auto give_up = [&]() {
+    *abort_flag = 1;
+    ptx::set_status(p.status, kStatusTimeout);
+  };
+
+  float acc[NBMAX][4];
 #pragma unroll
-  for (int b = 0; b < 2; ++b)
+  for (int b = 0; b < NBMAX; ++b)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[b][j] = 0.f;
 
-  uint32_t w_cur[2][F::QWORDS], w_nxt[2][F::QWORDS];
-  uint32_t xg_cur[F::XWORDS], xg_nxt[F::XWORDS], xg8_cur[F::XWORDS], xg8_nxt[F::XWORDS];
-
-  auto load_group = [&](int gi, uint32_t (&w)[2][F::QWORDS], uint32_t (&xa)[F::XWORDS],
-                        uint32_t (&xb)[F::XWORDS]) {
-    const size_t wofs = static_cast<size_t>(gi) * (G * BITS / 8) + c * (F::QWORDS * 4);
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      if constexpr (F::QWORDS == 4) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(wrow[b] + wofs));
-        w[b][0] = v.x; w[b][1] = v.y; w[b][2] = v.z; w[b][3] = v.w;
-      } else {
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(wrow[b] + wofs));
-        w[b][0] = v.x; w[b][1] = v.y;
+  if (warp == WARP_PRODUCER) {
+    // ---------------- producer: TMA boxes and bulk copies into the ring ----------------
+    if (lane == 0) {
+      ptx::tma_prefetch_desc(&tm_w);
+      ptx::tma_prefetch_desc(&tm_s);
+      const int sb_bytes = F::GS * R * 2;
+      int t = 0;
+      for (; t < p.num_stages; ++t) {
+        const int s = t % p.ring;
+        if (!ptx::mbar_wait(empty(s), ((t / p.ring) & 1) ^ 1, lim, abort_flag)) {
+          give_up();
+          break;
+        }
+        const int valid = min(F::KS, p.K - t * F::KS);
+        const uint32_t st = sbase + s * p.stage_bytes;
+        ptx::mbar_arrive_expect_tx(full(s), R * ROW_BYTES_PER_STAGE + sb_bytes * (BITS == 2 ? 1 : 2) +
+                                                p.M * valid * 2);
+        ptx::tma_load_2d(st, &tm_w, t * ROW_BYTES_PER_STAGE, n0, full(s));
+        ptx::tma_load_2d(st + p.off_s, &tm_s, n0, t * F::GS, full(s));
+        if (BITS != 2) ptx::tma_load_2d(st + p.off_b, &tm_b, n0, t * F::GS, full(s));
+        for (int m = 0; m < p.M; ++m)
+          bulk_copy_g2s(st + p.off_x + m * p.x_stride, p.X + static_cast<size_t>(m) * p.K + t * F::KS, valid * 2,
+                        full(s));
       }
+      // Let every copy this thread issued land before the ring is reused.
+      const int first = t > p.ring ? t - p.ring : 0;
+      for (int i = first; i < t; ++i) ptx::mbar_wait(full(i % p.ring), (i / p.ring) & 1, lim, nullptr);
     }
-    const int k0 = gi * G + c * F::QCODES;
-#pragma unroll
-    for (int i = 0; i < F::XWORDS / 4; ++i) {
-      uint4 v = xg_ok ? __ldg(reinterpret_cast<const uint4*>(xrow_g + k0) + i) : make_uint4(0, 0, 0, 0);
-      xa[4 * i] = v.x; xa[4 * i + 1] = v.y; xa[4 * i + 2] = v.z; xa[4 * i + 3] = v.w;
-      if constexpr (MT > 8) {
-        v = xg8_ok ? __ldg(reinterpret_cast<const uint4*>(xrow_g8 + k0) + i) : make_uint4(0, 0, 0, 0);
-        xb[4 * i] = v.x; xb[4 * i + 1] = v.y; xb[4 * i + 2] = v.z; xb[4 * i + 3] = v.w;
-      } else {
-        xb[4 * i] = xb[4 * i + 1] = xb[4 * i + 2] = xb[4 * i + 3] = 0u;
+  } else {
+    // ---------------- consumers ----------------
+    const int gs = warp % F::GS;  // group of the stage this warp takes
+    for (int t = warp / F::GS; t < p.num_stages; t += F::NSETS) {
+      const int s = t % p.ring;
+      if (!warp_wait(full(s), (t / p.ring) & 1, lim, abort_flag)) {
+        if (lane == 0) give_up();
+        break;
       }
-    }
-  };
-
-  if (g_begin < g_end) load_group(g_begin, w_nxt, xg_nxt, xg8_nxt);
-  for (int gi = g_begin; gi < g_end; ++gi) {
+      const uint8_t* st = smem + s * p.stage_bytes;
+      if (t * F::KS + gs * F::G < p.K) {
+        // activation fragments of this group's steps: k = gs*G + 16*step + 4c .. +3
+        uint2 xa[STEPS], xb[STEPS];
+        const uint8_t* xg = st + p.off_x + g * p.x_stride + (gs * F::G + 4 * c) * 2;
 #pragma unroll
-    for (int b = 0; b < 2; ++b)
+        for (int k = 0; k < STEPS; ++k) {
+          xa[k] = g < p.M ? *reinterpret_cast<const uint2*>(xg + 32 * k) : make_uint2(0u, 0u);
+          xb[k] = (MT > 8 && g + 8 < p.M) ? *reinterpret_cast<const uint2*>(xg + 8 * p.x_stride + 32 * k)
+                                           : make_uint2(0u, 0u);
+        }
+        float xs[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (BITS != 2) {
 #pragma unroll
-      for (int i = 0; i < F::QWORDS; ++i) w_cur[b][i] = w_nxt[b][i];
+          for (int k = 0; k < STEPS; ++k) {
+            uint32_t a[4] = {xa[k].x, xb[k].x, xa[k].y, xb[k].y};
+            mma_bf16_16816(xs, a, 0x3F803F80u, 0x3F803F80u);  // sum of x over the group
+          }
+        }
+        const uint16_t* sc = reinterpret_cast<const uint16_t*>(st + p.off_s) + gs * R;
+        const uint16_t* bi = reinterpret_cast<const uint16_t*>(st + p.off_b) + gs * R;
 #pragma unroll
-    for (int i = 0; i < F::XWORDS; ++i) {
-      xg_cur[i] = xg_nxt[i];
-      xg8_cur[i] = xg8_nxt[i];
-    }
-    if (gi + 1 < g_end) load_group(gi + 1, w_nxt, xg_nxt, xg8_nxt);
-
-    // scale / bias of the two adjacent weight rows this thread's accumulators
-    // cover: one 32-bit load each from the group-major [K/G, N] arrays
-    float s[2][2], bb[2][2];
+        for (int b = 0; b < NBMAX; ++b) {
+          if (b < nb) {
+            const int r = 8 * b + g;
+            Codes<BITS> cd;
+            cd.load(st + r * ROW_BYTES_PER_STAGE, gs, r, c);
+            float tmp[4] = {0.f, 0.f, 0.f, 0.f};
+            GroupSteps<BITS, 0, STEPS>::run(cd, c, xa, xb, tmp);
+            // rows 8b + 2c and 8b + 2c + 1 of the accumulator fragment
+            const uint32_t sv = *reinterpret_cast<const uint32_t*>(sc + 8 * b + 2 * c);
+            const float s2[2] = {deq::h2f(static_cast<uint16_t>(sv & 0xFFFFu)), deq::h2f(static_cast<uint16_t>(sv >> 16))};
+            if constexpr (BITS == 2) {
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      const size_t si = static_cast<size_t>(gi) * p.N + n_base + 8 * b + 2 * c;
-      const uint32_t sv = __ldg(reinterpret_cast<const uint32_t*>(p.scales + si));
-      s[b][0] = deq::h2f(static_cast<uint16_t>(sv & 0xFFFFu));
-      s[b][1] = deq::h2f(static_cast<uint16_t>(sv >> 16));
-      if constexpr (BITS != 2) {
-        const uint32_t bv = __ldg(reinterpret_cast<const uint32_t*>(p.biases + si));
-        bb[b][0] = deq::h2f(static_cast<uint16_t>(bv & 0xFFFFu));
-        bb[b][1] = deq::h2f(static_cast<uint16_t>(bv >> 16));
-      } else {
-        bb[b][0] = bb[b][1] = 0.f;
-      }
-    }
-
-    float tmp[2][4], xs[4];
+              for (int j = 0; j < 4; ++j) acc[b][j] = fmaf(0.5f * s2[j & 1], tmp[j], acc[b][j]);
+            } else {
+              const uint32_t bv = *reinterpret_cast<const uint32_t*>(bi + 8 * b + 2 * c);
+              const float b2[2] = {deq::h2f(static_cast<uint16_t>(bv & 0xFFFFu)),
+                                   deq::h2f(static_cast<uint16_t>(bv >> 16))};
 #pragma unroll
-    for (int b = 0; b < 2; ++b)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) tmp[b][j] = 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) xs[j] = 0.f;
-
-    StepLoop<BITS, 0, F::STEPS>::template run<MT>(xg_cur, xg8_cur, w_cur, tmp, xs);
-
-#pragma unroll
-    for (int b = 0; b < 2; ++b)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float ss = s[b][j & 1];
-        if constexpr (BITS == 2) {
-          acc[b][j] = fmaf(0.5f * ss, tmp[b][j], acc[b][j]);
-        } else {
-          const float d = BITS == 4 ? fmaf(-128.f, xs[j], tmp[b][j]) : tmp[b][j];
-          const float e = fmaf(bb[b][j & 1], xs[j], acc[b][j]);
-          acc[b][j] = fmaf(ss, d, e);
+              for (int j = 0; j < 4; ++j) {
+                const float d = BITS == 4 ? fmaf(-128.f, xs[j], tmp[j]) : tmp[j];
+                const float e = fmaf(b2[j & 1], xs[j], acc[b][j]);
+                acc[b][j] = fmaf(s2[j & 1], d, e);
+              }
+            }
+          }
         }
       }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(empty(s));
+    }
   }
 
-  // partial sums of this warp's K range -> shared memory
+  // ---------------- the warps' partial sums meet in shared memory ----------------
+  __syncthreads();  // the ring is drained: reuse it
+  float4* red = reinterpret_cast<float4*>(smem);
+  if (warp < NUM_CONSUMER_WARPS) {
 #pragma unroll
-  for (int b = 0; b < 2; ++b)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int m = g + (j >= 2 ? 8 : 0);
-      if (m < MT) red[warp][m][8 * b + 2 * c + (j & 1)] = acc[b][j];
-    }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < MT * kRowsPerCta; idx += kThreads) {
-    const int m = idx / kRowsPerCta, col = idx % kRowsPerCta;
-    if (m >= p.M) continue;
-    float v = red[0][m][col];
-#pragma unroll
-    for (int w = 1; w < kKSplit; ++w) v += red[w][m][col];
-    const int n = n_base + col;
-    if (p.bias) v += __bfloat162float(__ushort_as_bfloat16(p.bias[n]));
-    p.out[static_cast<size_t>(m) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    for (int b = 0; b < NBMAX; ++b)
+      if (b < nb) red[(warp * NBMAX + b) * 32 + lane] = make_float4(acc[b][0], acc[b][1], acc[b][2], acc[b][3]);
   }
+  __syncthreads();
+  const int per_m = nb * 4;
+  for (int i = threadIdx.x; i < p.M * per_m; i += NUM_THREADS) {
+    const int m = i / per_m, rem = i % per_m;
+    const int b = rem >> 2, cc = rem & 3;
+    const int ln = 4 * (m & 7) + cc;
+    float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+    for (int w = 0; w < NUM_CONSUMER_WARPS; ++w) {
+      const float4 f = red[(w * NBMAX + b) * 32 + ln];
+      v0 += m >= 8 ? f.z : f.x;
+      v1 += m >= 8 ? f.w : f.y;
+    }
+    const int n = n0 + 8 * b + 2 * cc;
+    if (p.bias) {
+      v0 += __bfloat162float(__ushort_as_bfloat16(p.bias[n]));
+      v1 += __bfloat162float(__ushort_as_bfloat16(p.bias[n + 1]));
+    }
+    const uint32_t packed = ptx::cvt_bf16x2(v0, v1);
+    *reinterpret_cast<uint32_t*>(p.out + static_cast<size_t>(m) * p.N + n) = packed;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+constexpr int kMaxSmem = 232448;
+
+template <int BITS, int MT>
+int launch_fmt(const Problem& pr, int nsm) {
+  using F = Fmt<BITS>;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(small_m_kernel<BITS, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  });
+  int st = cuda_check(attr_err, "cudaFuncSetAttribute(small_m_kernel)");
+  if (st != QGEMM_OK) return st;
+
+  Params kp;
+  kp.X = static_cast<const uint16_t*>(pr.X);
+  kp.bias = pr.bias;
+  kp.out = static_cast<uint16_t*>(pr.out);
+  kp.M = pr.M;
+  kp.N = pr.N;
+  kp.K = pr.K;
+  const int nblocks = pr.N / 8;
+  int bpc = (nblocks + nsm - 1) / nsm;
+  bpc = bpc < NBMAX ? bpc : NBMAX;
+  const int grid = (nblocks + bpc - 1) / bpc;
+  const int R = 8 * bpc;
+  kp.bpc = bpc;
+  kp.num_stages = (pr.K + F::KS - 1) / F::KS;
+  const int sb = F::GS * R * 2;
+  // TMA tile destinations start on 128-byte boundaries (the packed box on a
+  // 1024-byte one, for its 128-byte swizzle); bulk copies need 16 bytes.
+  kp.off_s = R * ROW_BYTES_PER_STAGE;
+  kp.off_b = (kp.off_s + sb + 127) & ~127;
+  kp.off_x = (kp.off_b + (BITS == 2 ? 0 : sb) + 127) & ~127;
+  kp.x_stride = F::KS * 2 + 16;  // +16 B staggers rows across banks
+  kp.stage_bytes = (kp.off_x + pr.M * kp.x_stride + 1023) & ~1023;
+  int ring = RING_BUDGET / kp.stage_bytes;
+  ring = ring < MAX_STAGES ? ring : MAX_STAGES;
+  ring = ring < kp.num_stages ? ring : kp.num_stages;
+  kp.ring = ring < 1 ? 1 : ring;
+  const int red_bytes = NUM_CONSUMER_WARPS * NBMAX * 32 * 16;
+  const int data_bytes = kp.ring * kp.stage_bytes > red_bytes ? kp.ring * kp.stage_bytes : red_bytes;
+  const int smem = data_bytes + 16 * MAX_STAGES + 16 + 1024;
+  if (smem > kMaxSmem) return fail(QGEMM_ERR_UNSUPPORTED, "small-M stage of %d bytes does not fit", kp.stage_bytes);
+  if (kp.off_s % 128 || kp.off_b % 128 || kp.off_x % 16 || kp.x_stride % 16 || kp.stage_bytes % 1024)
+    return fail(QGEMM_ERR_UNSUPPORTED, "internal: small-M stage layout misaligned");
+  kp.wait_limit_ns = wait_limit_ns();
+  if ((st = status_word(&kp.status)) != QGEMM_OK) return st;
+
+  CUtensorMap tm_w, tm_s, tm_b;
+  const uint64_t wbytes = static_cast<uint64_t>(pr.K) * BITS / 8;
+  const uint64_t groups = static_cast<uint64_t>(pr.K) / F::G;
+  if ((st = make_tensor_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.packed, wbytes, pr.N, wbytes,
+                               ROW_BYTES_PER_STAGE, R, CU_TENSOR_MAP_SWIZZLE_128B, "W")) != QGEMM_OK)
+    return st;
+  if ((st = make_tensor_map_2d(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.scales, pr.N, groups,
+                               uint64_t(pr.N) * 2, R, F::GS, CU_TENSOR_MAP_SWIZZLE_NONE, "scales")) != QGEMM_OK)
+    return st;
+  if (BITS != 2) {
+    if ((st = make_tensor_map_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.biases, pr.N, groups,
+                                 uint64_t(pr.N) * 2, R, F::GS, CU_TENSOR_MAP_SWIZZLE_NONE, "biases")) != QGEMM_OK)
+      return st;
+  } else {
+    tm_b = tm_s;  // unused for ternary
+  }
+  small_m_kernel<BITS, MT><<<grid, NUM_THREADS, smem, pr.stream>>>(tm_w, tm_s, tm_b, kp);
+  return cuda_check(cudaGetLastError(), "small_m_kernel launch");
 }
 
 template <int BITS>
-void launch_fmt(const SmallParams& sp, int grid, cudaStream_t stream) {
-  if (sp.M <= 8)
-    small_m_kernel<BITS, 8><<<grid, kThreads, 0, stream>>>(sp);
-  else
-    small_m_kernel<BITS, 16><<<grid, kThreads, 0, stream>>>(sp);
+int launch_bits(const Problem& pr, int nsm) {
+  return pr.M <= 8 ? launch_fmt<BITS, 8>(pr, nsm) : launch_fmt<BITS, 16>(pr, nsm);
 }
 
-}  // namespace
+}  // namespace sm
 
 int launch_small_m(const Problem& p) {
   int nsm;
   int st = sm_count(&nsm);
   if (st != QGEMM_OK) return st;
   if (p.M > 16) return fail(QGEMM_ERR_UNSUPPORTED, "small-M path takes M <= 16");
-  SmallParams sp{static_cast<const uint16_t*>(p.X), p.packed, p.scales, p.biases, p.bias,
-                 static_cast<uint16_t*>(p.out), p.M, p.N, p.K};
-  const int grid = p.N / kRowsPerCta;
   switch (p.bits) {
-    case 4: launch_fmt<4>(sp, grid, p.stream); break;
-    case 8: launch_fmt<8>(sp, grid, p.stream); break;
-    default: launch_fmt<2>(sp, grid, p.stream);
+    case 4: return sm::launch_bits<4>(p, nsm);
+    case 8: return sm::launch_bits<8>(p, nsm);
+    default: return sm::launch_bits<2>(p, nsm);
   }
-  return cuda_check(cudaGetLastError(), "small_m_kernel launch");
 }
 
 }  // namespace qg
