@@ -392,6 +392,41 @@ def run_ours(args, rank, world, local_rank):
     return result, peaks
 
 
+def run_case(args):
+    """One workload linear, launched back to back with a CUDA event pair per
+    launch (the form a profiler captures). --case 3:tern_m1:M=16"""
+    import torch
+
+    import weight_quantised_gemm_b200 as wq
+    import workloads as WL
+    parts = args.case.split(":")
+    cid = int(parts[0])
+    names = [l.name for l in WL.workload(cid).linears]
+    li = names.index(parts[1]) if len(parts) > 1 else 0
+    lin = WL.workload(cid).linears[li]
+    M = int(parts[2].split("=")[1]) if len(parts) > 2 else lin.M
+    ab = alg_bytes(lin, M)
+    ncopy = copies_for(ab, 3 if M > 16 else 32)
+    sets, _ = make_device_inputs(lin, cid, li, ncopy, M=M)
+    for i in range(args.warmup):
+        Xd, dw, bd, out = sets[i % ncopy]
+        wq.qgemm(Xd, dw, bias=bd, out=out)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        Xd, dw, bd, out = sets[i % ncopy]
+        ev[i][0].record()
+        wq.qgemm(Xd, dw, bias=bd, out=out)
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    wq.check_device_status()
+    t = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e-3
+    return {"case": args.case, "M": M, "N": lin.N, "K": lin.K, "bits": lin.bits,
+            "path": "small" if wq.qgemm_select_path(M, lin.N, lin.K, lin.bits) == 1 else "large",
+            "us_per_launch_events": round(t * 1e6, 2), "copies": ncopy,
+            "note": "per-launch events include host launch gaps for short kernels; the sweep's graph timing does not"}
+
+
 def run_e2e(sets, X_host_bits, lin, args, world):
     """Pipelined host->device->host: per step, copy X in from pinned memory,
     qgemm, copy out back to pinned memory, on three streams (PCIe in, compute,
@@ -563,6 +598,8 @@ def main(argv=None):
     ap.add_argument("--no-sweep", action="store_true", help="skip the per-workload sweep")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--case", default=None,
+                    help="time one workload linear alone, e.g. 3:tern_m1:M=16 (workload:linear[:M=..])")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -578,6 +615,9 @@ def main(argv=None):
 
     import torch
     torch.cuda.set_device(local_rank)
+    if args.case:
+        print(json.dumps(run_case(args)), flush=True)
+        return 0
     if world > 1:
         import datetime
 

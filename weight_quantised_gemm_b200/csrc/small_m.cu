@@ -43,6 +43,8 @@ namespace qg {
 namespace sm {
 
 constexpr int NBMAX = 12;             // n8 blocks (of 8 weight rows) per CTA, at most
+constexpr int NPMAX = NBMAX / 2;      // n16 pairs of blocks: the weight rows of one mma
+constexpr int PPW = NPMAX;            // pairs per consumer warp
 constexpr int NUM_CONSUMER_WARPS = 8;
 constexpr int WARP_PRODUCER = NUM_CONSUMER_WARPS;
 constexpr int NUM_THREADS = 32 * (NUM_CONSUMER_WARPS + 1);  // 288
@@ -56,7 +58,7 @@ struct Fmt {
   static constexpr int KS = ROW_BYTES_PER_STAGE * 8 / BITS;  // k per stage: 512, 256 or 128
   static constexpr int GS = KS / G;                        // groups per stage: 4, 4, 2
   static constexpr int STEPS = G / 16;                     // mma k-steps per group
-  static constexpr int NSETS = NUM_CONSUMER_WARPS / GS;    // warps sharing out the stages
+  static constexpr int NSETS = NUM_CONSUMER_WARPS / GS;  // warp sets sharing out the stages
   static constexpr int GBYTES = G * BITS / 8;              // packed bytes per row and group
 };
 
@@ -93,78 +95,53 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_
   return __all_sync(0xffffffffu, ok);
 }
 
-// The packed codes a thread needs for one group of one weight row, fetched
-// from the stage's 128-byte-swizzled row (logical 16-byte chunk j of row r
-// sits at physical chunk j ^ (r % 8)).
-//   ternary, 4-bit: the group's 32 bytes (8 words); quad threads share them.
-//   8-bit: the group's 64 bytes are 4 words per step; thread c keeps word c.
+// Byte offset, inside a stage row, of the 32-bit word that holds quad thread
+// c's 4 codes (k = 4c .. 4c+3) of step k of group gs. Rows carry the 128-byte
+// swizzle: logical 16-byte chunk j of row r sits at physical chunk j ^ (r % 8).
+//   ternary: one word per 16-k step (quad threads share it);
+//   4-bit:   two words per step, thread c reads word c / 2;
+//   8-bit:   four words per step, thread c reads word c.
 template <int BITS>
-struct Codes {
-  static constexpr int WPT = BITS == 8 ? 4 : 8;
-  uint32_t w[WPT];
-
-  __device__ __forceinline__ void load(const uint8_t* row, int gs, int r, int c) {
-    if constexpr (BITS == 8) {
-#pragma unroll
-      for (int st = 0; st < 4; ++st)
-        w[st] = *reinterpret_cast<const uint32_t*>(row + (((4 * gs + st) ^ (r & 7)) << 4) + 4 * c);
-    } else {
-      const uint4 lo = *reinterpret_cast<const uint4*>(row + (((2 * gs) ^ (r & 7)) << 4));
-      const uint4 hi = *reinterpret_cast<const uint4*>(row + (((2 * gs + 1) ^ (r & 7)) << 4));
-      w[0] = lo.x; w[1] = lo.y; w[2] = lo.z; w[3] = lo.w;
-      w[4] = hi.x; w[5] = hi.y; w[6] = hi.z; w[7] = hi.w;
-    }
+__device__ __forceinline__ int word_offset(int gs, int k, int c, int r7) {
+  int chunk, wic;
+  if constexpr (BITS == 2) {
+    chunk = 2 * gs + (k >> 2);
+    wic = k & 3;
+  } else if constexpr (BITS == 4) {
+    chunk = 2 * gs + (k >> 1);
+    wic = 2 * (k & 1) + (c >> 1);
+  } else {
+    chunk = 4 * gs + k;
+    wic = c;
   }
+  return ((chunk ^ r7) << 4) + 4 * wic;
+}
 
-  // B operand of step ST for quad thread c: codes 4c .. 4c+3 of the step's
-  // 16 k as two bf16x2 registers (k pairs (4c, 4c+1) and (4c+2, 4c+3)).
-  template <int ST>
-  __device__ __forceinline__ void decode(int c, uint32_t& b0, uint32_t& b1) const {
-    if constexpr (BITS == 2) {
-      // one word = one step (16 codes); pairs 2c and 2c+1 of the word
-      const uint32_t x = w[ST];
-      b0 = (x << (14 - 4 * c)) & 0xC000C000u;  // bf16 {-2, 0, +2}
-      b1 = (x << (12 - 4 * c)) & 0xC000C000u;
-    } else if constexpr (BITS == 4) {
-      // two words per step; thread c reads word c/2, pairs 2(c%2) and 2(c%2)+1
-      const uint32_t x = (c >> 1) ? w[2 * ST + 1] : w[2 * ST];
-      const int sh = 8 * (c & 1);
-      b0 = ((x >> sh) & 0x000F000Fu) | 0x43004300u;  // bf16 128 + q
-      b1 = ((x >> (sh + 4)) & 0x000F000Fu) | 0x43004300u;
-    } else {
-      // byte j of the thread's word is code 4c + j; exact q through an fp32 magic number
-      const uint32_t x = w[ST];
-      const float2 q01 = ptx::add2(make_float2(__uint_as_float(ptx::prmt(x, deq::kMagic, 0x7650u)),
-                                               __uint_as_float(ptx::prmt(x, deq::kMagic, 0x7651u))),
-                                   make_float2(-deq::kMagicF, -deq::kMagicF));
-      const float2 q23 = ptx::add2(make_float2(__uint_as_float(ptx::prmt(x, deq::kMagic, 0x7652u)),
-                                               __uint_as_float(ptx::prmt(x, deq::kMagic, 0x7653u))),
-                                   make_float2(-deq::kMagicF, -deq::kMagicF));
-      b0 = ptx::cvt_bf16x2(q01.x, q01.y);
-      b1 = ptx::cvt_bf16x2(q23.x, q23.y);
-    }
+// B operand of one step for quad thread c from its word: codes 4c .. 4c+3 as
+// two bf16x2 registers (k pairs (4c, 4c+1) and (4c+2, 4c+3)).
+template <int BITS>
+__device__ __forceinline__ void decode_word(uint32_t x, int c, uint32_t& b0, uint32_t& b1) {
+  if constexpr (BITS == 2) {
+    // pairs 2c and 2c+1 of the 16-code word: bf16 {-2, 0, +2}
+    b0 = (x << (14 - 4 * c)) & 0xC000C000u;
+    b1 = (x << (12 - 4 * c)) & 0xC000C000u;
+  } else if constexpr (BITS == 4) {
+    // pairs 2(c%2) and 2(c%2)+1 of the 8-code word: bf16 128 + q
+    const int sh = 8 * (c & 1);
+    b0 = ((x >> sh) & 0x000F000Fu) | 0x43004300u;
+    b1 = ((x >> (sh + 4)) & 0x000F000Fu) | 0x43004300u;
+  } else {
+    // byte j is code 4c + j; exact q through an fp32 magic number
+    const float2 q01 = ptx::add2(make_float2(__uint_as_float(ptx::prmt(x, deq::kMagic, 0x7650u)),
+                                             __uint_as_float(ptx::prmt(x, deq::kMagic, 0x7651u))),
+                                 make_float2(-deq::kMagicF, -deq::kMagicF));
+    const float2 q23 = ptx::add2(make_float2(__uint_as_float(ptx::prmt(x, deq::kMagic, 0x7652u)),
+                                             __uint_as_float(ptx::prmt(x, deq::kMagic, 0x7653u))),
+                                 make_float2(-deq::kMagicF, -deq::kMagicF));
+    b0 = ptx::cvt_bf16x2(q01.x, q01.y);
+    b1 = ptx::cvt_bf16x2(q23.x, q23.y);
   }
-};
-
-// One group of one weight block: 16-k steps against the activation
-// fragments, accumulated into tmp (one mma per step).
-template <int BITS, int ST, int STEPS>
-struct GroupSteps {
-  __device__ __forceinline__ static void run(const Codes<BITS>& cd, int c, const uint2 (&xa)[STEPS],
-                                             const uint2 (&xb)[STEPS], float (&tmp)[4]) {
-    uint32_t a[4] = {xa[ST].x, xb[ST].x, xa[ST].y, xb[ST].y};
-    uint32_t b0, b1;
-    cd.template decode<ST>(c, b0, b1);
-    mma_bf16_16816(tmp, a, b0, b1);
-    GroupSteps<BITS, ST + 1, STEPS>::run(cd, c, xa, xb, tmp);
-  }
-};
-
-template <int BITS, int STEPS>
-struct GroupSteps<BITS, STEPS, STEPS> {
-  __device__ __forceinline__ static void run(const Codes<BITS>&, int, const uint2 (&)[STEPS], const uint2 (&)[STEPS],
-                                             float (&)[4]) {}
-};
+}
 
 template <int BITS, int MT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -183,7 +160,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int nb = min(p.bpc, nblocks_total - blk0);
   const int n0 = 8 * blk0;
   const int R = 8 * p.bpc;  // rows per TMA box (rows past N read as zeros)
-  const int data_bytes = max(p.ring * p.stage_bytes, NUM_CONSUMER_WARPS * NBMAX * 32 * 16);
+  const int data_bytes = max(p.ring * p.stage_bytes, NUM_CONSUMER_WARPS * PPW * 2 * 32 * 16);
   const uint32_t bar0 = sbase + data_bytes;
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (MAX_STAGES + s); };
@@ -204,11 +181,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::set_status(p.status, kStatusTimeout);
   };
 
-  float acc[NBMAX][4];
+  // acc[p][h][j]: weight rows 16p + g (j < 2) and 16p + g + 8 (j >= 2), tokens
+  // 8h + 2c + (j & 1)
+  constexpr int TH = MT > 8 ? 2 : 1;
+  float acc[PPW][TH][4];
 #pragma unroll
-  for (int b = 0; b < NBMAX; ++b)
+  for (int q = 0; q < PPW; ++q)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[b][j] = 0.f;
+    for (int h = 0; h < TH; ++h)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[q][h][j] = 0.f;
+  // Every CTA runs NPMAX n16 pairs with no per-pair branch, so the compiler can
+  // interleave the pairs' loads, decodes and mma. Rows past the CTA's own
+  // (past 8 * nb) are computed from whatever the stage holds there and are
+  // never written out; the stage reserves room for all 16 * NPMAX rows.
 
   if (warp == WARP_PRODUCER) {
     // ---------------- producer: TMA boxes and bulk copies into the ring ----------------
@@ -240,8 +226,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ---------------- consumers ----------------
-    const int gs = warp % F::GS;  // group of the stage this warp takes
-    for (int t = warp / F::GS; t < p.num_stages; t += F::NSETS) {
+    const int gs = warp % F::GS;                   // group of the stage this warp takes
+    const int half = 0;                            // every warp takes all of the CTA's pairs
+    for (int t = (warp / F::GS) % F::NSETS; t < p.num_stages; t += F::NSETS) {
       const int s = t % p.ring;
       if (!warp_wait(full(s), (t / p.ring) & 1, lim, abort_flag)) {
         if (lane == 0) give_up();
@@ -249,50 +236,72 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       const uint8_t* st = smem + s * p.stage_bytes;
       if (t * F::KS + gs * F::G < p.K) {
-        // activation fragments of this group's steps: k = gs*G + 16*step + 4c .. +3
-        uint2 xa[STEPS], xb[STEPS];
+        // activations of this group (the B operand): tokens g and g + 8,
+        // k = gs*G + 16*step + 4c .. +3
         const uint8_t* xg = st + p.off_x + g * p.x_stride + (gs * F::G + 4 * c) * 2;
+        const bool ga = g < p.M, gb = MT > 8 && g + 8 < p.M;
+        float xs[TH][4];  // sum of x over the group per token (affine)
+        float tmp[PPW][TH][4];
+#pragma unroll
+        for (int h = 0; h < TH; ++h)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) xs[h][j] = 0.f;
+#pragma unroll
+        for (int q = 0; q < PPW; ++q)
+#pragma unroll
+          for (int h = 0; h < TH; ++h)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tmp[q][h][j] = 0.f;
+        // weight row 16 * (half * PPW + q) + g of this warp's pair q
+        const uint8_t* rowg = st + (16 * half * PPW + g) * ROW_BYTES_PER_STAGE;
 #pragma unroll
         for (int k = 0; k < STEPS; ++k) {
-          xa[k] = g < p.M ? *reinterpret_cast<const uint2*>(xg + 32 * k) : make_uint2(0u, 0u);
-          xb[k] = (MT > 8 && g + 8 < p.M) ? *reinterpret_cast<const uint2*>(xg + 8 * p.x_stride + 32 * k)
-                                           : make_uint2(0u, 0u);
-        }
-        float xs[4] = {0.f, 0.f, 0.f, 0.f};
-        if constexpr (BITS != 2) {
+          const uint2 x0 = ga ? *reinterpret_cast<const uint2*>(xg + 32 * k) : make_uint2(0u, 0u);
+          const uint2 x1 = gb ? *reinterpret_cast<const uint2*>(xg + 8 * p.x_stride + 32 * k) : make_uint2(0u, 0u);
+          if constexpr (BITS != 2) {
+            const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};
+            mma_bf16_16816(xs[0], ones, x0.x, x0.y);
+            if constexpr (TH > 1) mma_bf16_16816(xs[TH - 1], ones, x1.x, x1.y);
+          }
+          const int wo = word_offset<BITS>(gs, k, c, g);  // rows g and g + 8 share the swizzle
 #pragma unroll
-          for (int k = 0; k < STEPS; ++k) {
-            uint32_t a[4] = {xa[k].x, xb[k].x, xa[k].y, xb[k].y};
-            mma_bf16_16816(xs, a, 0x3F803F80u, 0x3F803F80u);  // sum of x over the group
+          for (int q = 0; q < PPW; ++q) {
+            const uint8_t* r0 = rowg + q * 16 * ROW_BYTES_PER_STAGE;
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(r0 + wo);
+            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(r0 + 8 * ROW_BYTES_PER_STAGE + wo);
+            uint32_t a[4];
+            decode_word<BITS>(w0, c, a[0], a[2]);  // row g: k pairs (4c, 4c+1), (4c+2, 4c+3)
+            decode_word<BITS>(w1, c, a[1], a[3]);  // row g + 8
+            mma_bf16_16816(tmp[q][0], a, x0.x, x0.y);
+            if constexpr (TH > 1) mma_bf16_16816(tmp[q][TH - 1], a, x1.x, x1.y);
           }
         }
+        // apply the group's scale (and bias) of rows 16q + g and 16q + g + 8
         const uint16_t* sc = reinterpret_cast<const uint16_t*>(st + p.off_s) + gs * R;
         const uint16_t* bi = reinterpret_cast<const uint16_t*>(st + p.off_b) + gs * R;
 #pragma unroll
-        for (int b = 0; b < NBMAX; ++b) {
-          if (b < nb) {
-            const int r = 8 * b + g;
-            Codes<BITS> cd;
-            cd.load(st + r * ROW_BYTES_PER_STAGE, gs, r, c);
-            float tmp[4] = {0.f, 0.f, 0.f, 0.f};
-            GroupSteps<BITS, 0, STEPS>::run(cd, c, xa, xb, tmp);
-            // rows 8b + 2c and 8b + 2c + 1 of the accumulator fragment
-            const uint32_t sv = *reinterpret_cast<const uint32_t*>(sc + 8 * b + 2 * c);
-            const float s2[2] = {deq::h2f(static_cast<uint16_t>(sv & 0xFFFFu)), deq::h2f(static_cast<uint16_t>(sv >> 16))};
-            if constexpr (BITS == 2) {
+        for (int q = 0; q < PPW; ++q) {
+          {
+            const int r0 = 16 * (half * PPW + q) + g;
+            const float s2[2] = {deq::h2f(sc[r0]), deq::h2f(sc[r0 + 8])};
+            float b2[2] = {0.f, 0.f};
+            if constexpr (BITS != 2) {
+              b2[0] = deq::h2f(bi[r0]);
+              b2[1] = deq::h2f(bi[r0 + 8]);
+            }
 #pragma unroll
-              for (int j = 0; j < 4; ++j) acc[b][j] = fmaf(0.5f * s2[j & 1], tmp[j], acc[b][j]);
-            } else {
-              const uint32_t bv = *reinterpret_cast<const uint32_t*>(bi + 8 * b + 2 * c);
-              const float b2[2] = {deq::h2f(static_cast<uint16_t>(bv & 0xFFFFu)),
-                                   deq::h2f(static_cast<uint16_t>(bv >> 16))};
+            for (int h = 0; h < TH; ++h)
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const float d = BITS == 4 ? fmaf(-128.f, xs[j], tmp[j]) : tmp[j];
-                const float e = fmaf(b2[j & 1], xs[j], acc[b][j]);
-                acc[b][j] = fmaf(s2[j & 1], d, e);
+                const float sj = s2[j >> 1];
+                if constexpr (BITS == 2) {
+                  acc[q][h][j] = fmaf(0.5f * sj, tmp[q][h][j], acc[q][h][j]);
+                } else {
+                  const float d = BITS == 4 ? fmaf(-128.f, xs[h][j], tmp[q][h][j]) : tmp[q][h][j];
+                  const float e = fmaf(b2[j >> 1], xs[h][j], acc[q][h][j]);
+                  acc[q][h][j] = fmaf(sj, d, e);
+                }
               }
-            }
           }
         }
       }
@@ -303,32 +312,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   // ---------------- the warps' partial sums meet in shared memory ----------------
   __syncthreads();  // the ring is drained: reuse it
-  float4* red = reinterpret_cast<float4*>(smem);
+  float4* red = reinterpret_cast<float4*>(smem);  // [warp][pair of the warp][token half][lane]
   if (warp < NUM_CONSUMER_WARPS) {
 #pragma unroll
-    for (int b = 0; b < NBMAX; ++b)
-      if (b < nb) red[(warp * NBMAX + b) * 32 + lane] = make_float4(acc[b][0], acc[b][1], acc[b][2], acc[b][3]);
+    for (int q = 0; q < PPW; ++q)
+#pragma unroll
+        for (int h = 0; h < TH; ++h)
+          red[((warp * PPW + q) * TH + h) * 32 + lane] =
+              make_float4(acc[q][h][0], acc[q][h][1], acc[q][h][2], acc[q][h][3]);
   }
   __syncthreads();
-  const int per_m = nb * 4;
-  for (int i = threadIdx.x; i < p.M * per_m; i += NUM_THREADS) {
-    const int m = i / per_m, rem = i % per_m;
-    const int b = rem >> 2, cc = rem & 3;
-    const int ln = 4 * (m & 7) + cc;
-    float v0 = 0.f, v1 = 0.f;
+  const int rows = 8 * nb;
+  for (int i = threadIdx.x; i < p.M * rows; i += NUM_THREADS) {
+    const int m = i / rows, nl = i % rows;
+    const int q = nl >> 4, hrow = (nl >> 3) & 1, gg = nl & 7;
+    const int h = m >> 3, cc = (m & 7) >> 1;
+    const int j = 2 * hrow + (m & 1);
+    const int ln = 4 * gg + cc;
+    float v = 0.f;
+    const int wh = q / PPW, ql = q % PPW;  // the warps holding pair q: those of half wh
+    constexpr int WPH = NUM_CONSUMER_WARPS;
 #pragma unroll
-    for (int w = 0; w < NUM_CONSUMER_WARPS; ++w) {
-      const float4 f = red[(w * NBMAX + b) * 32 + ln];
-      v0 += m >= 8 ? f.z : f.x;
-      v1 += m >= 8 ? f.w : f.y;
+    for (int w = wh * WPH; w < (wh + 1) * WPH; ++w) {
+      const float4 f = red[((w * PPW + ql) * TH + h) * 32 + ln];
+      v += j == 0 ? f.x : j == 1 ? f.y : j == 2 ? f.z : f.w;
     }
-    const int n = n0 + 8 * b + 2 * cc;
-    if (p.bias) {
-      v0 += __bfloat162float(__ushort_as_bfloat16(p.bias[n]));
-      v1 += __bfloat162float(__ushort_as_bfloat16(p.bias[n + 1]));
-    }
-    const uint32_t packed = ptx::cvt_bf16x2(v0, v1);
-    *reinterpret_cast<uint32_t*>(p.out + static_cast<size_t>(m) * p.N + n) = packed;
+    const int n = n0 + nl;
+    if (p.bias) v += __bfloat162float(__ushort_as_bfloat16(p.bias[n]));
+    p.out[static_cast<size_t>(m) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
   }
 }
 
@@ -365,7 +376,8 @@ int launch_fmt(const Problem& pr, int nsm) {
   const int sb = F::GS * R * 2;
   // TMA tile destinations start on 128-byte boundaries (the packed box on a
   // 1024-byte one, for its 128-byte swizzle); bulk copies need 16 bytes.
-  kp.off_s = R * ROW_BYTES_PER_STAGE;
+  const int rows_read = R > 16 * NPMAX ? R : 16 * NPMAX;  // rows the consumers touch
+  kp.off_s = rows_read * ROW_BYTES_PER_STAGE;
   kp.off_b = (kp.off_s + sb + 127) & ~127;
   kp.off_x = (kp.off_b + (BITS == 2 ? 0 : sb) + 127) & ~127;
   kp.x_stride = F::KS * 2 + 16;  // +16 B staggers rows across banks
@@ -374,7 +386,7 @@ int launch_fmt(const Problem& pr, int nsm) {
   ring = ring < MAX_STAGES ? ring : MAX_STAGES;
   ring = ring < kp.num_stages ? ring : kp.num_stages;
   kp.ring = ring < 1 ? 1 : ring;
-  const int red_bytes = NUM_CONSUMER_WARPS * NBMAX * 32 * 16;
+  const int red_bytes = NUM_CONSUMER_WARPS * PPW * 2 * 32 * 16;
   const int data_bytes = kp.ring * kp.stage_bytes > red_bytes ? kp.ring * kp.stage_bytes : red_bytes;
   const int smem = data_bytes + 16 * MAX_STAGES + 16 + 1024;
   if (smem > kMaxSmem) return fail(QGEMM_ERR_UNSUPPORTED, "small-M stage of %d bytes does not fit", kp.stage_bytes);
