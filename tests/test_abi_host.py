@@ -136,3 +136,19 @@ def test_select_path_table():
         assert wq.qgemm_select_path(4096, 9216, 3072, bits) == wq.QGEMM_PATH_LARGE_M
     with pytest.raises(wq.QGemmError):
         wq.qgemm_select_path(1, 16, 128, 3)
+
+
+def test_missing_library_fails_loudly_on_first_call(tmp_path):
+    """Without libqgemm.so the package still imports (so its build module can
+    run on a fresh checkout) but every entry point raises: no CPU fallback."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = tmp_path / "weight_quantised_gemm_b200"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "weight_quantised_gemm_b200", "__init__.py"), pkg / "__init__.py")
+    code = ("import weight_quantised_gemm_b200 as wq\n"
+            "try:\n    wq.qgemm_version()\nexcept ImportError as e:\n    print('raised', 'not built' in str(e))\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == "raised True"

@@ -2,7 +2,9 @@
 
 Argument marshalling only: every step of the GEMM runs in the library's CUDA
 kernels; torch provides device memory and streams. There is no CPU fallback:
-if the shared library is missing, importing this package raises.
+the shared library is loaded on first use, and every entry point raises if
+it is missing (the package itself imports without it, so that its build
+module can run on a fresh checkout).
 
     import weight_quantised_gemm_b200 as wq
     pw = wq.qgemm_pack(W_fp32_numpy, bits=4)          # host, RTN, packed at rest
@@ -75,7 +77,17 @@ def _load():
     return lib
 
 
-_lib = _load()
+class _LazyLib:
+    """The loaded libqgemm.so, opened on first attribute access."""
+    _handle = None
+
+    def __getattr__(self, name):
+        if _LazyLib._handle is None:
+            _LazyLib._handle = _load()
+        return getattr(_LazyLib._handle, name)
+
+
+_lib = _LazyLib()
 EXPORTED = ("qgemm_pack_sizes", "qgemm_pack", "qgemm", "qgemm_ex", "qgemm_select_path", "qgemm_dequant_tile",
             "qgemm_get_device_status", "qgemm_set_wait_limit_ns", "qgemm_debug_wait_timeout",
             "qgemm_status_str", "qgemm_last_error", "qgemm_version")
