@@ -116,7 +116,6 @@ def test_qgemm_rejects_bad_operands_without_device():
     assert _call(d, M=0) == wq.QGEMM_OK
     # ternary needs no biases
     assert _call(_desc(bits=2, group=128, biases=0), M=0) == wq.QGEMM_OK
-    assert "16-byte" in wq.qgemm_last_error() or wq.qgemm_last_error() == "" or True
 
 
 def test_dequant_tile_rejects_bad_windows_without_device():
