@@ -29,7 +29,7 @@
 //                 256-column fp32 accumulators, so one tile's epilogue
 //                 overlaps the next tile's main loop)
 //   warp 2        TMA producer of the W ring
-//   warps 3..10   dequantisers (one thread per tile row and 32-k half)
+//   warps 3..10   dequantisers (lanes share out each tile row's 8-k chunks)
 //   warps 11..14  epilogue: tcgen05.ld the accumulator (each warp owns one
 //                 32-lane quarter = 32 weight rows), add the bias, round to
 //                 bf16, transpose through shared memory and TMA-store
@@ -261,9 +261,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp < WARP_EPI0) {
     // ---------------- dequantisers ----------------
-    const int dq = threadIdx.x - 32 * WARP_DEQ0;  // 0..255
-    const int r = dq & (TILE_N - 1);              // tile row this thread writes
-    const int h = dq >> 7;                        // which 32-k half of the 64-k block
+    // Lane layout: LPR lanes share a tile row, each taking CPT consecutive
+    // 8-k chunks, so a warp's packed read is one contiguous span of shared
+    // memory and its 16-byte stores hit distinct banks under the swizzle.
+    constexpr int LPR = NUM_DEQ_WARPS / 4;           // lanes per tile row
+    constexpr int CPT = (BK / 8) / LPR;              // 8-k chunks per thread
+    constexpr int RPW = 32 / LPR;                    // tile rows per warp
+    constexpr int CHUNK_BYTES = 8 * BITS / 8;        // packed bytes per 8-k chunk
+    const int wd = warp - WARP_DEQ0;
+    const int r = RPW * wd + lane / LPR;             // tile row this thread writes
+    const int c0 = (lane % LPR) * CPT;               // its first chunk
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
@@ -279,28 +286,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float s_cur = deq::h2f(reinterpret_cast<const uint16_t*>(wst + C::kWTileBytes)[r]);
         const float b_cur =
             BITS == 2 ? 0.f : deq::h2f(reinterpret_cast<const uint16_t*>(wst + C::kWTileBytes + SB_BYTES)[r]);
-        const uint8_t* wsrc = wst + r * C::kWRowBytes + h * (C::kWRowBytes / 2);
-        uint4 o[4];
-        if constexpr (BITS == 4) {
-          const uint4 v = *reinterpret_cast<const uint4*>(wsrc);  // 4 words = 32 k
-          o[0] = deq::chunk_4bit(v.x, s_cur, b_cur);
-          o[1] = deq::chunk_4bit(v.y, s_cur, b_cur);
-          o[2] = deq::chunk_4bit(v.z, s_cur, b_cur);
-          o[3] = deq::chunk_4bit(v.w, s_cur, b_cur);
-        } else if constexpr (BITS == 8) {
+        const uint8_t* wsrc = wst + r * C::kWRowBytes + c0 * CHUNK_BYTES;
+        // packed words of this thread's CPT chunks
+        constexpr int NWORDS = CPT * CHUNK_BYTES / 4;
+        uint32_t wv[NWORDS > 0 ? NWORDS : 1];
+        if constexpr (NWORDS == 8) {
           const uint4 v0 = *reinterpret_cast<const uint4*>(wsrc);
           const uint4 v1 = *reinterpret_cast<const uint4*>(wsrc + 16);
-          o[0] = deq::chunk_8bit(v0.x, v0.y, s_cur, b_cur);
-          o[1] = deq::chunk_8bit(v0.z, v0.w, s_cur, b_cur);
-          o[2] = deq::chunk_8bit(v1.x, v1.y, s_cur, b_cur);
-          o[3] = deq::chunk_8bit(v1.z, v1.w, s_cur, b_cur);
+          wv[0] = v0.x; wv[1] = v0.y; wv[2] = v0.z; wv[3] = v0.w;
+          wv[4] = v1.x; wv[5] = v1.y; wv[6] = v1.z; wv[7] = v1.w;
+        } else if constexpr (NWORDS == 4) {
+          const uint4 v = *reinterpret_cast<const uint4*>(wsrc);
+          wv[0] = v.x; wv[1] = v.y; wv[2] = v.z; wv[3] = v.w;
+        } else if constexpr (NWORDS == 2) {
+          const uint2 v = *reinterpret_cast<const uint2*>(wsrc);
+          wv[0] = v.x; wv[1] = v.y;
         } else {
-          const uint2 v = *reinterpret_cast<const uint2*>(wsrc);  // 2 words = 32 k
+          wv[0] = *reinterpret_cast<const uint32_t*>(wsrc);
+        }
+        uint4 o[CPT];
+        if constexpr (BITS == 2) {
           const uint32_t hs = deq::ternary_half_scale2(s_cur);
-          o[0] = deq::chunk_ternary<0>(v.x, hs);
-          o[1] = deq::chunk_ternary<1>(v.x, hs);
-          o[2] = deq::chunk_ternary<0>(v.y, hs);
-          o[3] = deq::chunk_ternary<1>(v.y, hs);
+#pragma unroll
+          for (int i = 0; i < CPT; ++i)
+            o[i] = (i & 1) ? deq::chunk_ternary<1>(wv[i / 2], hs) : deq::chunk_ternary<0>(wv[i / 2], hs);
+        } else if constexpr (BITS == 4) {
+#pragma unroll
+          for (int i = 0; i < CPT; ++i) o[i] = deq::chunk_4bit(wv[i], s_cur, b_cur);
+        } else {
+#pragma unroll
+          for (int i = 0; i < CPT; ++i) o[i] = deq::chunk_8bit(wv[2 * i], wv[2 * i + 1], s_cur, b_cur);
         }
         // The packed stage has been read: give it back to the W producer.
         __syncwarp();
@@ -309,8 +324,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // chunk c sits at physical chunk c ^ (r % 8).
         uint8_t* arow = smem + C::kOffA + sa * A_STAGE_BYTES + r * (BK * 2);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int cidx = 4 * h + i;
+        for (int i = 0; i < CPT; ++i) {
+          const int cidx = c0 + i;
           *reinterpret_cast<uint4*>(arow + ((cidx ^ (r & 7)) << 4)) = o[i];
         }
         ptx::fence_proxy_async_smem();

@@ -166,6 +166,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto empty = [&](int s) { return bar0 + 8u * (MAX_STAGES + s); };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + data_bytes + 16 * MAX_STAGES);
   const uint64_t lim = p.wait_limit_ns;
+  // Each CTA walks the K slices starting at its own offset: every CTA reads
+  // the same activations, and rotating the order spreads those reads over
+  // the L2 instead of sending all CTAs to the same lines at once.
+  const int rot = blockIdx.x % p.num_stages;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.ring; ++s) {
@@ -209,15 +213,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           give_up();
           break;
         }
-        const int valid = min(F::KS, p.K - t * F::KS);
+        const int kt = (t + rot) % p.num_stages;  // which K slice this ring slot carries
+        const int valid = min(F::KS, p.K - kt * F::KS);
         const uint32_t st = sbase + s * p.stage_bytes;
         ptx::mbar_arrive_expect_tx(full(s), R * ROW_BYTES_PER_STAGE + sb_bytes * (BITS == 2 ? 1 : 2) +
                                                 p.M * valid * 2);
-        ptx::tma_load_2d(st, &tm_w, t * ROW_BYTES_PER_STAGE, n0, full(s));
-        ptx::tma_load_2d(st + p.off_s, &tm_s, n0, t * F::GS, full(s));
-        if (BITS != 2) ptx::tma_load_2d(st + p.off_b, &tm_b, n0, t * F::GS, full(s));
+        ptx::tma_load_2d(st, &tm_w, kt * ROW_BYTES_PER_STAGE, n0, full(s));
+        ptx::tma_load_2d(st + p.off_s, &tm_s, n0, kt * F::GS, full(s));
+        if (BITS != 2) ptx::tma_load_2d(st + p.off_b, &tm_b, n0, kt * F::GS, full(s));
         for (int m = 0; m < p.M; ++m)
-          bulk_copy_g2s(st + p.off_x + m * p.x_stride, p.X + static_cast<size_t>(m) * p.K + t * F::KS, valid * 2,
+          bulk_copy_g2s(st + p.off_x + m * p.x_stride, p.X + static_cast<size_t>(m) * p.K + kt * F::KS, valid * 2,
                         full(s));
       }
       // Let every copy this thread issued land before the ring is reused.
@@ -235,7 +240,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       const uint8_t* st = smem + s * p.stage_bytes;
-      if (t * F::KS + gs * F::G < p.K) {
+      const int kt = (t + rot) % p.num_stages;
+      if (kt * F::KS + gs * F::G < p.K) {
         // activations of this group (the B operand): tokens g and g + 8,
         // k = gs*G + 16*step + 4c .. +3
         const uint8_t* xg = st + p.off_x + g * p.x_stride + (gs * F::G + 4 * c) * 2;
