@@ -1,5 +1,6 @@
-// Large-M path: TMA -> shared-memory dequant -> tcgen05 MMA into TMEM ->
-// TMA-store epilogue. One persistent CTA per SM.
+// Large-M path: TMA -> dequantisation into tensor memory -> tcgen05 MMA
+// (A from TMEM, B from shared memory) -> TMA-store epilogue. One persistent
+// CTA per SM.
 //
 // "Dequantised inside the matmul kernel a tile at a time" (stable-diffusion.rs
 // README, introduction) maps onto Blackwell as follows. Each output tile is
@@ -10,30 +11,33 @@
 // tokens (the widest N an instruction takes) instead of 128, halving the
 // dequantisation work per FLOP against the usual orientation.
 //
-// Three shared-memory rings, each with its own full/empty mbarriers, keep the
-// three producers of an MMA operand independent:
-//   X ring   activation tiles X[256 x 64] (128-byte swizzle), filled by TMA,
-//            emptied by the MMA;
-//   W ring   packed weight tiles [128 rows x 64 k] plus the tile's 128 fp16
-//            scales and biases (group-major at rest, so one 256-byte TMA box
-//            each), filled by TMA, emptied by the dequantisers;
-//   A ring   dequantised bf16 weight tiles in the 128-byte-swizzled K-major
-//            layout of the UMMA descriptor, filled by the dequantisers,
-//            emptied by the MMA.
-// The W ring is deep and cheap, so dequantisation runs ahead of the MMA
-// without waiting for activation tiles.
+// The dequantised weight tile never touches shared memory: the dequantising
+// warps write it straight into tensor memory (one lane per weight row, two
+// bf16 per 32-bit column along K) and the MMA reads its A operand from there.
+// Shared memory then carries only the TMA-loaded activation and packed-weight
+// tiles and the MMA's activation reads, which keeps the tensor pipe ahead of
+// the shared-memory port.
+//
+// Rings, each with its own full/empty mbarriers:
+//   X ring (smem)  activation tiles X[256 x 64], 128-byte swizzle; TMA in,
+//                  emptied by the MMA;
+//   W ring (smem)  packed weight tiles [128 rows x 64 k] plus the tile's 128
+//                  fp16 scales and biases (group-major at rest, so one 256-byte
+//                  TMA box each); TMA in, emptied by the dequantisers;
+//   A ring (TMEM)  dequantised bf16 weight tiles [128 lanes x 32 columns];
+//                  written by the dequantisers, emptied by the MMA.
+// TMEM columns: the fp32 accumulator in 0..255, the A ring in 256..383.
 //
 // Warp roles (480 threads):
 //   warp 0        TMA producer of the X ring
-//   warp 1        MMA issuer (one thread) and TMEM owner (512 columns: two
-//                 256-column fp32 accumulators, so one tile's epilogue
-//                 overlaps the next tile's main loop)
+//   warp 1        MMA issuer (one thread) and TMEM owner
 //   warp 2        TMA producer of the W ring
-//   warps 3..10   dequantisers (lanes share out each tile row's 8-k chunks)
-//   warps 11..14  epilogue: tcgen05.ld the accumulator (each warp owns one
-//                 32-lane quarter = 32 weight rows), add the bias, round to
-//                 bf16, transpose through shared memory and TMA-store
-//                 [32 tokens x 128 features] boxes (coalesced 16-byte rows).
+//   warps 3..10   dequantisers: warp w writes TMEM lanes 32 (w % 4) ..+31
+//                 (its lane quarter), one 32-k half of each 64-k block
+//   warps 11..14  epilogue: tcgen05.ld the accumulator (each warp one lane
+//                 quarter = 32 weight rows), add the bias, round to bf16 into a
+//                 shared-memory copy of the whole tile, hand the accumulator
+//                 back, then one TMA store of [256 tokens x 128 features].
 // Every wait is bounded: on expiry the kernel records a status code, drains
 // what it has in flight, frees TMEM and returns.
 
@@ -60,15 +64,17 @@ constexpr int WARP_DEQ0 = 3;
 constexpr int WARP_EPI0 = WARP_DEQ0 + NUM_DEQ_WARPS;            // 11
 constexpr int NUM_THREADS = 32 * (WARP_EPI0 + NUM_EPI_WARPS);   // 480
 constexpr int X_STAGE_BYTES = TILE_M * BK * 2;  // 32 KB
-constexpr int A_STAGE_BYTES = TILE_N * BK * 2;  // 16 KB
 constexpr int SB_BYTES = TILE_N * 2;            // one group's scales (or biases) for the tile's rows
-constexpr int OUT_ROWS = 32;                    // tokens per TMA store box
-constexpr int OUT_BUF_BYTES = OUT_ROWS * TILE_N * 2;
-constexpr int NUM_OUT_BUFS = 2;
+constexpr int OUT_BYTES = TILE_M * TILE_N * 2;  // the whole bf16 output tile
+constexpr int OUT_ROWS = 32;                    // tokens per accumulator chunk read back
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_COLS = TILE_M;  // fp32 columns per accumulator
+constexpr uint32_t ACC_COL = 0;                 // fp32 accumulator: columns 0..255
+constexpr uint32_t A_COL = TILE_M;              // A ring: columns 256..
+constexpr uint32_t A_STAGE_COLS = BK / 2;       // 64 bf16 per row = 32 columns
+constexpr int SA = 4;                           // A ring depth
 constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TILE_N, TILE_M);
 constexpr int EPI_BAR_ID = 1;
+static_assert(A_COL + SA * A_STAGE_COLS <= TMEM_COLS, "TMEM budget");
 
 template <int BITS>
 struct Cfg {
@@ -77,19 +83,17 @@ struct Cfg {
   static constexpr int kWTileBytes = TILE_N * kWRowBytes;
   static constexpr int kSBBytes = BITS == 2 ? SB_BYTES : 2 * SB_BYTES;  // scales (+ biases)
   static constexpr int kWStride = kWTileBytes + kSBBytes;             // one W-ring stage
-  static constexpr int kSX = 4;                          // X ring depth
-  static constexpr int kSA = 2;                          // A ring depth
-  static constexpr int kSW = BITS == 8 ? 5 : 8;          // W ring depth
+  static constexpr int kSX = 4;                                       // X ring depth
+  static constexpr int kSW = BITS == 8 ? 3 : BITS == 4 ? 6 : 8;       // W ring depth
   static constexpr int kOffX = 0;
-  static constexpr int kOffA = kOffX + kSX * X_STAGE_BYTES;
-  static constexpr int kOffW = kOffA + kSA * A_STAGE_BYTES;
-  static constexpr int kOffOut = kOffW + kSW * kWStride;
-  static constexpr int kOffBar = kOffOut + NUM_OUT_BUFS * OUT_BUF_BYTES;
-  static constexpr int kNumBars = 2 * kSX + 2 * kSW + 2 * kSA + 5;
+  static constexpr int kOffW = kOffX + kSX * X_STAGE_BYTES;
+  static constexpr int kOffOut = (kOffW + kSW * kWStride + 1023) & ~1023;
+  static constexpr int kOffBar = kOffOut + OUT_BYTES;
+  static constexpr int kNumBars = 2 * kSX + 2 * kSW + 2 * SA + 3;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024 B
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(kOffA % 1024 == 0 && kOffW % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+  static_assert(kOffW % 1024 == 0, "swizzle atoms need 1024-byte alignment");
   static_assert(kWStride % 128 == 0 && kOffOut % 128 == 0, "TMA boxes land on 128-byte boundaries");
 };
 
@@ -114,7 +118,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                    const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_out, const Params p) {
   using C = Cfg<BITS>;
-  constexpr int SX = C::kSX, SA = C::kSA, SW = C::kSW;
+  constexpr int SX = C::kSX, SW = C::kSW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = ptx::smem_u32(smem);
@@ -122,7 +126,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int lane = threadIdx.x & 31;
 
   auto x_stage = [&](int s) { return sbase + C::kOffX + s * X_STAGE_BYTES; };
-  auto a_stage = [&](int s) { return sbase + C::kOffA + s * A_STAGE_BYTES; };
   auto w_stage = [&](int s) { return C::kOffW + s * C::kWStride; };  // byte offset into smem
   const uint32_t bar0 = sbase + C::kOffBar;
   auto full_x = [&](int s) { return bar0 + 8u * s; };
@@ -131,10 +134,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto empty_w = [&](int s) { return bar0 + 8u * (2 * SX + SW + s); };
   auto full_a = [&](int s) { return bar0 + 8u * (2 * SX + 2 * SW + s); };
   auto empty_a = [&](int s) { return bar0 + 8u * (2 * SX + 2 * SW + SA + s); };
-  const uint32_t bar1 = bar0 + 8u * (2 * SX + 2 * SW + 2 * SA);
-  auto acc_full = [&](int b) { return bar1 + 8u * b; };
-  auto acc_empty = [&](int b) { return bar1 + 8u * (2 + b); };
-  const uint32_t drain_bar = bar1 + 32u;
+  const uint32_t acc_full = bar0 + 8u * (2 * SX + 2 * SW + 2 * SA);
+  const uint32_t acc_empty = acc_full + 8u;
+  const uint32_t drain_bar = acc_full + 16u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   volatile int* epi_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
@@ -152,10 +154,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(full_a(s), NUM_DEQ_WARPS);
       ptx::mbar_init(empty_a(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(acc_full(b), 1);
-      ptx::mbar_init(acc_empty(b), NUM_EPI_WARPS);
-    }
+    ptx::mbar_init(acc_full, 1);
+    ptx::mbar_init(acc_empty, NUM_EPI_WARPS);
     ptx::mbar_init(drain_bar, 1);
     *abort_flag = 0;
     *epi_abort = 0;
@@ -226,14 +226,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tcount) {
-        const int buf = tcount & 1;
-        const uint32_t use = tcount >> 1;
-        if (!ptx::mbar_wait(acc_empty(buf), (use & 1) ^ 1, lim, abort_flag)) {
+        // the epilogue has read the previous tile's accumulator out
+        if (!ptx::mbar_wait(acc_empty, (tcount & 1) ^ 1, lim, abort_flag)) {
           give_up();
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t d_tmem = tmem_base + buf * ACC_COLS;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
           const int sx = it % SX, sa = it % SA;
           if (!ptx::mbar_wait(full_x(sx), (it / SX) & 1, lim, abort_flag) ||
@@ -245,32 +243,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ptx::tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-            const uint64_t adesc = ptx::smem_desc_sw128_kmajor(a_stage(sa) + kk * UMMA_K * 2);
+            const uint32_t a_tmem = tmem_base + A_COL + sa * A_STAGE_COLS + kk * (UMMA_K / 2);
             const uint64_t bdesc = ptx::smem_desc_sw128_kmajor(x_stage(sx) + kk * UMMA_K * 2);
-            ptx::tc_mma_f16_ss(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0);
+            ptx::tc_mma_f16_ts(tmem_base + ACC_COL, a_tmem, bdesc, IDESC, (kb | kk) != 0);
           }
           ptx::tc_commit(empty_x(sx));
           ptx::tc_commit(empty_a(sa));
         }
         if (!ok) break;
-        ptx::tc_commit(acc_full(buf));
+        ptx::tc_commit(acc_full);
       }
       // All MMAs issued above complete before TMEM is released.
       ptx::tc_commit(drain_bar);
       ptx::mbar_wait(drain_bar, 0, lim, nullptr);
     }
   } else if (warp < WARP_EPI0) {
-    // ---------------- dequantisers ----------------
-    // Lane layout: LPR lanes share a tile row, each taking CPT consecutive
-    // 8-k chunks, so a warp's packed read is one contiguous span of shared
-    // memory and its 16-byte stores hit distinct banks under the swizzle.
-    constexpr int LPR = NUM_DEQ_WARPS / 4;           // lanes per tile row
-    constexpr int CPT = (BK / 8) / LPR;              // 8-k chunks per thread
-    constexpr int RPW = 32 / LPR;                    // tile rows per warp
-    constexpr int CHUNK_BYTES = 8 * BITS / 8;        // packed bytes per 8-k chunk
-    const int wd = warp - WARP_DEQ0;
-    const int r = RPW * wd + lane / LPR;             // tile row this thread writes
-    const int c0 = (lane % LPR) * CPT;               // its first chunk
+    // ---------------- dequantisers: packed smem tile -> bf16 in TMEM ----------------
+    const int q = warp & 3;                      // TMEM lane quarter this warp may write
+    const int h = (warp - WARP_DEQ0) >> 2;       // which 32-k half of each 64-k block
+    const int r = 32 * q + lane;                 // tile row = TMEM lane
+    const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
@@ -282,53 +274,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ok = false;
           break;
         }
+        ptx::tc_fence_after();  // the MMA that last read this A stage has completed
         const uint8_t* wst = smem + w_stage(sw);
         const float s_cur = deq::h2f(reinterpret_cast<const uint16_t*>(wst + C::kWTileBytes)[r]);
         const float b_cur =
             BITS == 2 ? 0.f : deq::h2f(reinterpret_cast<const uint16_t*>(wst + C::kWTileBytes + SB_BYTES)[r]);
-        const uint8_t* wsrc = wst + r * C::kWRowBytes + c0 * CHUNK_BYTES;
-        // packed words of this thread's CPT chunks
-        constexpr int NWORDS = CPT * CHUNK_BYTES / 4;
-        uint32_t wv[NWORDS > 0 ? NWORDS : 1];
-        if constexpr (NWORDS == 8) {
+        const uint8_t* wsrc = wst + r * C::kWRowBytes + h * (C::kWRowBytes / 2);
+        uint4 o[4];  // 4 chunks of 8 consecutive k = this thread's 32 k
+        if constexpr (BITS == 4) {
+          const uint4 v = *reinterpret_cast<const uint4*>(wsrc);
+          o[0] = deq::chunk_4bit(v.x, s_cur, b_cur);
+          o[1] = deq::chunk_4bit(v.y, s_cur, b_cur);
+          o[2] = deq::chunk_4bit(v.z, s_cur, b_cur);
+          o[3] = deq::chunk_4bit(v.w, s_cur, b_cur);
+        } else if constexpr (BITS == 8) {
           const uint4 v0 = *reinterpret_cast<const uint4*>(wsrc);
           const uint4 v1 = *reinterpret_cast<const uint4*>(wsrc + 16);
-          wv[0] = v0.x; wv[1] = v0.y; wv[2] = v0.z; wv[3] = v0.w;
-          wv[4] = v1.x; wv[5] = v1.y; wv[6] = v1.z; wv[7] = v1.w;
-        } else if constexpr (NWORDS == 4) {
-          const uint4 v = *reinterpret_cast<const uint4*>(wsrc);
-          wv[0] = v.x; wv[1] = v.y; wv[2] = v.z; wv[3] = v.w;
-        } else if constexpr (NWORDS == 2) {
+          o[0] = deq::chunk_8bit(v0.x, v0.y, s_cur, b_cur);
+          o[1] = deq::chunk_8bit(v0.z, v0.w, s_cur, b_cur);
+          o[2] = deq::chunk_8bit(v1.x, v1.y, s_cur, b_cur);
+          o[3] = deq::chunk_8bit(v1.z, v1.w, s_cur, b_cur);
+        } else {
           const uint2 v = *reinterpret_cast<const uint2*>(wsrc);
-          wv[0] = v.x; wv[1] = v.y;
-        } else {
-          wv[0] = *reinterpret_cast<const uint32_t*>(wsrc);
-        }
-        uint4 o[CPT];
-        if constexpr (BITS == 2) {
           const uint32_t hs = deq::ternary_half_scale2(s_cur);
-#pragma unroll
-          for (int i = 0; i < CPT; ++i)
-            o[i] = (i & 1) ? deq::chunk_ternary<1>(wv[i / 2], hs) : deq::chunk_ternary<0>(wv[i / 2], hs);
-        } else if constexpr (BITS == 4) {
-#pragma unroll
-          for (int i = 0; i < CPT; ++i) o[i] = deq::chunk_4bit(wv[i], s_cur, b_cur);
-        } else {
-#pragma unroll
-          for (int i = 0; i < CPT; ++i) o[i] = deq::chunk_8bit(wv[2 * i], wv[2 * i + 1], s_cur, b_cur);
+          o[0] = deq::chunk_ternary<0>(v.x, hs);
+          o[1] = deq::chunk_ternary<1>(v.x, hs);
+          o[2] = deq::chunk_ternary<0>(v.y, hs);
+          o[3] = deq::chunk_ternary<1>(v.y, hs);
         }
         // The packed stage has been read: give it back to the W producer.
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(empty_w(sw));
-        // 128-byte swizzle, K-major: row r holds 8 chunks of 16 B; logical
-        // chunk c sits at physical chunk c ^ (r % 8).
-        uint8_t* arow = smem + C::kOffA + sa * A_STAGE_BYTES + r * (BK * 2);
-#pragma unroll
-        for (int i = 0; i < CPT; ++i) {
-          const int cidx = c0 + i;
-          *reinterpret_cast<uint4*>(arow + ((cidx ^ (r & 7)) << 4)) = o[i];
-        }
-        ptx::fence_proxy_async_smem();
+        const uint32_t regs[16] = {o[0].x, o[0].y, o[0].z, o[0].w, o[1].x, o[1].y, o[1].z, o[1].w,
+                                   o[2].x, o[2].y, o[2].z, o[2].w, o[3].x, o[3].y, o[3].z, o[3].w};
+        ptx::tmem_st_32x32b_x16(tmem_base + lane_addr + A_COL + sa * A_STAGE_COLS + h * 16, regs);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(full_a(sa));
       }
@@ -338,51 +319,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int q = warp & 3;                        // TMEM lane quarter this warp may access
     const int ep = threadIdx.x - 32 * WARP_EPI0;   // 0..127
     const int n_local = 32 * q + lane;
-    uint32_t tcount = 0, chunk_count = 0;
+    uint16_t* stg = reinterpret_cast<uint16_t*>(smem + C::kOffOut);
+    uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
-      const int buf = tcount & 1;
-      const uint32_t use = tcount >> 1;
       const int n0 = (tile / p.num_m_tiles) * TILE_N;
       const int m0 = (tile % p.num_m_tiles) * TILE_M;
       const int n = n0 + n_local;
       const float bias_f =
           (p.bias && n < p.N) ? __bfloat162float(__ushort_as_bfloat16(p.bias[n])) : 0.f;
-      const bool got = warp_wait(acc_full(buf), use & 1, lim, abort_flag);
+      const bool got = warp_wait(acc_full, tcount & 1, lim, abort_flag);
       if (!got && lane == 0) {
         *epi_abort = 1;
         give_up();
       }
+      // the staging copy of the previous tile has been read by its TMA store
+      if (ep == 0) ptx::bulk_wait_group_read<0>();
       ptx::named_bar_sync(EPI_BAR_ID, 32 * NUM_EPI_WARPS);  // all four warps agree before going on
       if (*epi_abort) break;
       ptx::tc_fence_after();
       const int rows_left = p.M - m0;
       const int chunks = rows_left >= TILE_M ? TILE_M / OUT_ROWS : (rows_left + OUT_ROWS - 1) / OUT_ROWS;
-      for (int cch = 0; cch < chunks; ++cch, ++chunk_count) {
+      for (int cch = 0; cch < chunks; ++cch) {
         uint32_t v[32];
-        ptx::tmem_ld_32x32b_x32(tmem_base + buf * ACC_COLS + cch * OUT_ROWS + (static_cast<uint32_t>(32 * q) << 16),
-                                v);
+        ptx::tmem_ld_32x32b_x32(tmem_base + ACC_COL + cch * OUT_ROWS + (static_cast<uint32_t>(32 * q) << 16), v);
         ptx::tmem_wait_ld();
-        if (cch == chunks - 1) {
-          // this warp has read its whole accumulator quarter: hand it back
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(acc_empty(buf));
-        }
-        const int ob = chunk_count & 1;
-        if (ep == 0) ptx::bulk_wait_group_read<NUM_OUT_BUFS - 1>();  // the store that last used `ob` has read it
-        ptx::named_bar_sync(EPI_BAR_ID, 32 * NUM_EPI_WARPS);
-        uint16_t* stg = reinterpret_cast<uint16_t*>(smem + C::kOffOut + ob * OUT_BUF_BYTES);
 #pragma unroll
         for (int j = 0; j < OUT_ROWS; ++j) {
           const float f = __uint_as_float(v[j]) + bias_f;
-          stg[j * TILE_N + n_local] = __bfloat16_as_ushort(__float2bfloat16_rn(f));
+          stg[(cch * OUT_ROWS + j) * TILE_N + n_local] = __bfloat16_as_ushort(__float2bfloat16_rn(f));
         }
-        ptx::fence_proxy_async_smem();
-        ptx::named_bar_sync(EPI_BAR_ID, 32 * NUM_EPI_WARPS);
-        if (ep == 0) {
-          ptx::tma_store_2d(&tm_out, sbase + C::kOffOut + ob * OUT_BUF_BYTES, n0, m0 + cch * OUT_ROWS);
-          ptx::bulk_commit_group();
-        }
+      }
+      // this warp has read its whole accumulator quarter: hand it back
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(acc_empty);
+      ptx::fence_proxy_async_smem();
+      ptx::named_bar_sync(EPI_BAR_ID, 32 * NUM_EPI_WARPS);
+      if (ep == 0) {
+        ptx::tma_store_2d(&tm_out, sbase + C::kOffOut, n0, m0);
+        ptx::bulk_commit_group();
       }
     }
     if (ep == 0) ptx::bulk_wait_group<0>();
@@ -430,7 +405,7 @@ int launch_fmt(const Problem& pr, int nsm) {
     tm_b = tm_s;  // unused for ternary
   }
   if ((st = make_tensor_map_2d(&tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pr.out, pr.N, pr.M, uint64_t(pr.N) * 2,
-                        TILE_N, OUT_ROWS, none, "out")) != QGEMM_OK)
+                        TILE_N, TILE_M, none, "out")) != QGEMM_OK)
     return st;
   unsigned int* status;
   if ((st = status_word(&status)) != QGEMM_OK) return st;
