@@ -55,14 +55,16 @@ constexpr int TILE_N = 128;  // weight rows per tile (MMA M)
 constexpr int TILE_M = 256;  // tokens per tile (MMA N)
 constexpr int BK = 64;       // K per pipeline stage: one 128-byte swizzle row of bf16
 constexpr int UMMA_K = 16;
-constexpr int NUM_DEQ_WARPS = 8;
+constexpr int DEQ_SETS = 2;                    // dequantiser sets, taking K blocks in turn
+constexpr int DEQ_WARPS_PER_SET = 8;           // one set covers a 128 x 64 block
+constexpr int NUM_DEQ_WARPS = DEQ_SETS * DEQ_WARPS_PER_SET;
 constexpr int NUM_EPI_WARPS = 4;
 constexpr int WARP_XLOAD = 0;
 constexpr int WARP_MMA = 1;
 constexpr int WARP_WLOAD = 2;
 constexpr int WARP_DEQ0 = 3;
-constexpr int WARP_EPI0 = WARP_DEQ0 + NUM_DEQ_WARPS;            // 11
-constexpr int NUM_THREADS = 32 * (WARP_EPI0 + NUM_EPI_WARPS);   // 480
+constexpr int WARP_EPI0 = WARP_DEQ0 + NUM_DEQ_WARPS;
+constexpr int NUM_THREADS = 32 * (WARP_EPI0 + NUM_EPI_WARPS);
 constexpr int X_STAGE_BYTES = TILE_M * BK * 2;  // 32 KB
 constexpr int SB_BYTES = TILE_N * 2;            // one group's scales (or biases) for the tile's rows
 constexpr int OUT_BYTES = TILE_M * TILE_N * 2;  // the whole bf16 output tile
@@ -75,6 +77,7 @@ constexpr int SA = 4;                           // A ring depth
 constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TILE_N, TILE_M);
 constexpr int EPI_BAR_ID = 1;
 static_assert(A_COL + SA * A_STAGE_COLS <= TMEM_COLS, "TMEM budget");
+static_assert(NUM_THREADS <= 1024, "one CTA holds at most 1024 threads");
 
 template <int BITS>
 struct Cfg {
@@ -99,11 +102,23 @@ struct Cfg {
 
 struct Params {
   int M, N, K;
-  int num_m_tiles, num_tiles, num_kb;
+  int num_m_tiles, num_n_tiles, num_tiles, num_kb;
+  int m_fastest;  // tile order: 1 = consecutive tiles walk the token dimension, 0 = the feature dimension
   const uint16_t* bias;
   uint64_t wait_limit_ns;
   unsigned int* status;
 };
+
+// Output tile `tile` -> (feature tile, token tile) in the order the host chose.
+__device__ __forceinline__ void tile_coords(const Params& p, int tile, int& n_tile, int& m_tile) {
+  if (p.m_fastest) {
+    n_tile = tile / p.num_m_tiles;
+    m_tile = tile - n_tile * p.num_m_tiles;
+  } else {
+    m_tile = tile / p.num_n_tiles;
+    n_tile = tile - m_tile * p.num_n_tiles;
+  }
+}
 
 // Bounded wait of a whole warp: every lane waits, and the warp gives up as
 // one if any lane ran out of time (so no lane is left at a warp barrier).
@@ -148,10 +163,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int s = 0; s < SW; ++s) {
       ptx::mbar_init(full_w(s), 1);
-      ptx::mbar_init(empty_w(s), NUM_DEQ_WARPS);
+      ptx::mbar_init(empty_w(s), DEQ_WARPS_PER_SET);
     }
     for (int s = 0; s < SA; ++s) {
-      ptx::mbar_init(full_a(s), NUM_DEQ_WARPS);
+      ptx::mbar_init(full_a(s), DEQ_WARPS_PER_SET);
       ptx::mbar_init(empty_a(s), 1);
     }
     ptx::mbar_init(acc_full, 1);
@@ -193,7 +208,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-        const int n_tile = tile / p.num_m_tiles, m_tile = tile % p.num_m_tiles;
+        int n_tile, m_tile;
+        tile_coords(p, tile, n_tile, m_tile);
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
           const int s = it % S;
           const uint32_t par = ((it / S) & 1) ^ 1;
@@ -259,19 +275,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp < WARP_EPI0) {
     // ---------------- dequantisers: packed smem tile -> bf16 in TMEM ----------------
+    // Set `set` takes the CTA's K blocks it = set, set + DEQ_SETS, ... (counted
+    // over all its tiles), so DEQ_SETS blocks are in flight per weight row.
+    const int d = warp - WARP_DEQ0;
+    const int set = d / DEQ_WARPS_PER_SET;
     const int q = warp & 3;                      // TMEM lane quarter this warp may write
-    const int h = (warp - WARP_DEQ0) >> 2;       // which 32-k half of each 64-k block
+    const int h = (d >> 2) & 1;                  // which 32-k half of each 64-k block
     const int r = 32 * q + lane;                 // tile row = TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-    uint32_t it = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-      for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+    const int my_tiles = (p.num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                         static_cast<int>(gridDim.x);
+    const uint32_t total = static_cast<uint32_t>(my_tiles) * static_cast<uint32_t>(p.num_kb);
+    for (uint32_t it = set; it < total; it += DEQ_SETS) {
+      {
         const int sw = it % SW, sa = it % SA;
         if (!warp_wait(full_w(sw), (it / SW) & 1, lim, abort_flag) ||
             !warp_wait(empty_a(sa), ((it / SA) & 1) ^ 1, lim, abort_flag)) {
           if (lane == 0) give_up();
-          ok = false;
           break;
         }
         ptx::tc_fence_after();  // the MMA that last read this A stage has completed
@@ -322,8 +342,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint16_t* stg = reinterpret_cast<uint16_t*>(smem + C::kOffOut);
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
-      const int n0 = (tile / p.num_m_tiles) * TILE_N;
-      const int m0 = (tile % p.num_m_tiles) * TILE_M;
+      int n_tile, m_tile;
+      tile_coords(p, tile, n_tile, m_tile);
+      const int n0 = n_tile * TILE_N;
+      const int m0 = m_tile * TILE_M;
       const int n = n0 + n_local;
       const float bias_f =
           (p.bias && n < p.N) ? __bfloat162float(__ushort_as_bfloat16(p.bias[n])) : 0.f;
@@ -414,13 +436,26 @@ int launch_fmt(const Problem& pr, int nsm) {
   kp.N = pr.N;
   kp.K = pr.K;
   kp.num_m_tiles = (pr.M + TILE_M - 1) / TILE_M;
-  const int num_n_tiles = (pr.N + TILE_N - 1) / TILE_N;
-  kp.num_tiles = kp.num_m_tiles * num_n_tiles;
+  kp.num_n_tiles = (pr.N + TILE_N - 1) / TILE_N;
+  kp.num_tiles = kp.num_m_tiles * kp.num_n_tiles;
+  const int grid = kp.num_tiles < nsm ? kp.num_tiles : nsm;
+  // The grid works on `grid` consecutive tiles at a time. Walk the dimension
+  // that keeps fewer bytes of activation panels (256 tokens x K) and weight
+  // panels (128 rows x K, packed) live in L2 at once.
+  {
+    const double x_panel = double(TILE_M) * pr.K * 2;
+    const double w_panel = double(TILE_N) * pr.K * BITS / 8;
+    auto live = [&](int fast, int slow, double fast_panel, double slow_panel) {
+      const int f = fast < grid ? fast : grid;
+      return f * fast_panel + double((grid + fast - 1) / fast) * slow_panel;
+    };
+    kp.m_fastest = live(kp.num_m_tiles, kp.num_n_tiles, x_panel, w_panel) <=
+                   live(kp.num_n_tiles, kp.num_m_tiles, w_panel, x_panel);
+  }
   kp.num_kb = pr.K / BK;
   kp.bias = pr.bias;
   kp.wait_limit_ns = wait_limit_ns();
   kp.status = status;
-  const int grid = kp.num_tiles < nsm ? kp.num_tiles : nsm;
   large_m_kernel<BITS><<<grid, NUM_THREADS, C::kSmemBytes, pr.stream>>>(tm_x, tm_w, tm_s, tm_b, tm_out, kp);
   return cuda_check(cudaGetLastError(), "large_m_kernel launch");
 }
