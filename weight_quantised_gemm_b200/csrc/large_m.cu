@@ -40,9 +40,13 @@
 //   warps 3..18   dequantisers: warp w writes TMEM lanes 32 (w % 4) ..+31 (its
 //                 lane quarter), one 32-k slice of every stage
 //   warps 19..26  epilogue: tcgen05.ld one lane quarter x 128 tokens of the
-//                 accumulator, add the bias, round to bf16 and store straight
-//                 to global memory (a warp writes 64 contiguous bytes per
-//                 token), handing the accumulator back after its last load.
+//                 accumulator 32 tokens at a time, add the bias, round to bf16
+//                 into the warp's own 2 KB shared-memory slot (transposed to
+//                 token-major) and TMA-store the 32 x 32 block; the
+//                 accumulator goes back to the MMA after the warp's last load.
+// Shared memory is laid out without slack: the kernel checks that its dynamic
+// shared memory starts on a 1024-byte boundary and otherwise records a status
+// code and returns.
 // Every wait is bounded: on expiry the kernel records a status code, drains
 // what it has in flight, frees TMEM and returns.
 
@@ -73,6 +77,7 @@ constexpr int NUM_THREADS = 32 * (WARP_EPI0 + NUM_EPI_WARPS);
 constexpr int X_BOX_BYTES = TILE_M * BOX_K * 2;  // 32 KB
 constexpr int X_STAGE_BYTES = 2 * X_BOX_BYTES;    // 64 KB
 constexpr int EPI_ROWS = 32;                      // tokens per tcgen05.ld
+constexpr int EPI_SLOT_BYTES = EPI_ROWS * 32 * 2; // one 32 tokens x 32 features bf16 block
 constexpr int EPI_TOKENS = TILE_M / (NUM_EPI_WARPS / 4);  // tokens per epilogue warp
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;                   // fp32 accumulator: columns 0..255
@@ -98,14 +103,16 @@ struct Cfg {
   static constexpr int kSBytes = kGroupsPerStage * TILE_N * 2;  // one stage's scales (or biases)
   static constexpr int kSBStride = BITS == 2 ? kSBytes : 2 * kSBytes;
   static constexpr int kS = BITS == 8 ? 2 : 3;                   // stage ring depth
-  static constexpr int kSW = BITS == 8 ? 4 : BITS == 4 ? 3 : 6;  // W ring depth
+  static constexpr int kSW = BITS == 8 ? 3 : BITS == 4 ? 2 : 4;  // W ring depth
+  static constexpr int kSlots = BITS == 8 ? 2 : 1;               // epilogue store slots per warp
   static constexpr int kOffX = 0;
   static constexpr int kOffW = kOffX + kS * X_STAGE_BYTES;
-  static constexpr int kOffSB = kOffW + kSW * kWTileBytes;
+  static constexpr int kOffOut = kOffW + kSW * kWTileBytes;
+  static constexpr int kOffSB = kOffOut + NUM_EPI_WARPS * kSlots * EPI_SLOT_BYTES;
   static constexpr int kOffBar = kOffSB + kSW * kSBStride;
   static constexpr int kNumBars = 2 * kS + 2 * kSW + 3;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024 B
+  static constexpr int kSmemBytes = kOffMisc + 16;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(A_COL + kS * A_STAGE_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(kOffW % 1024 == 0 && kWTileBytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
@@ -118,7 +125,6 @@ struct Params {
   int num_m_tiles, num_n_tiles, num_tiles, num_kb;
   int m_fastest;  // tile order: 1 = consecutive tiles walk the token dimension, 0 = the feature dimension
   const uint16_t* bias;
-  uint16_t* out;
   uint64_t wait_limit_ns;
   unsigned int* status;
 };
@@ -152,12 +158,15 @@ template <int BITS>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     large_m_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                    const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_b,
-                   const Params p) {
+                   const __grid_constant__ CUtensorMap tm_out, const Params p) {
   using C = Cfg<BITS>;
   constexpr int S = C::kS, SW = C::kSW;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = ptx::smem_u32(smem);
+  if (sbase & 1023u) {  // the swizzled tiles need it; uniform across the block
+    if (threadIdx.x == 0) ptx::set_status(p.status, kStatusLayout);
+    return;
+  }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -194,7 +203,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tmem_alloc(ptx::smem_u32(tmem_slot), TMEM_COLS);
     ptx::tmem_relinquish();
   }
-  if (warp == WARP_XLOAD && lane == 0) ptx::tma_prefetch_desc(&tm_x);
+  if (warp == WARP_XLOAD && lane == 0) {
+    ptx::tma_prefetch_desc(&tm_x);
+    ptx::tma_prefetch_desc(&tm_out);
+  }
   if (warp == WARP_WLOAD && lane == 0) {
     ptx::tma_prefetch_desc(&tm_w);
     ptx::tma_prefetch_desc(&tm_s);
@@ -352,17 +364,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ---------------- epilogue ----------------
     const int e = warp - WARP_EPI0;
-    const int q = warp & 3;               // TMEM lane quarter this warp may read
+    const int q = warp & 3;                // TMEM lane quarter this warp may read
     const int t0 = (e >> 2) * EPI_TOKENS;  // first token (accumulator column) of this warp
     const int n_local = 32 * q + lane;
-    uint32_t tcount = 0;
+    uint16_t* slots = reinterpret_cast<uint16_t*>(smem + C::kOffOut + e * C::kSlots * EPI_SLOT_BYTES);
+    const uint32_t slots_u32 = sbase + C::kOffOut + e * C::kSlots * EPI_SLOT_BYTES;
+    uint32_t tcount = 0, nstore = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
       int n_tile, m_tile;
       tile_coords(p, tile, n_tile, m_tile);
       const int n = n_tile * TILE_N + n_local;
       const int m0 = m_tile * TILE_M + t0;
-      const bool n_ok = n < p.N;
-      const float bias_f = (p.bias && n_ok) ? __bfloat162float(__ushort_as_bfloat16(p.bias[n])) : 0.f;
+      const float bias_f = (p.bias && n < p.N) ? __bfloat162float(__ushort_as_bfloat16(p.bias[n])) : 0.f;
       const bool got = warp_wait(acc_full, tcount & 1, lim, abort_flag);
       if (!got && lane == 0) {
         *epi_abort = 1;
@@ -374,7 +387,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int rows_left = p.M - m0;  // tokens of this warp's half still inside X
       const int chunks = rows_left >= EPI_TOKENS ? EPI_TOKENS / EPI_ROWS
                                                  : (rows_left > 0 ? (rows_left + EPI_ROWS - 1) / EPI_ROWS : 0);
-      uint16_t* orow = p.out + static_cast<size_t>(m0) * p.N + n;
       for (int c = 0; c < EPI_TOKENS / EPI_ROWS; ++c) {
         uint32_t v[32];
         if (c < chunks) {
@@ -387,18 +399,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(acc_empty);
         }
-        if (c < chunks && n_ok) {
-          const int rows = min(EPI_ROWS, rows_left - c * EPI_ROWS);
+        if (c < chunks && n_tile * TILE_N + 32 * q < p.N) {
+          const uint32_t slot = nstore % C::kSlots;
+          // the TMA store that last used this slot has finished reading it
+          if (lane == 0) ptx::bulk_wait_group_read<C::kSlots - 1>();
+          __syncwarp();
+          uint16_t* sl = slots + slot * (EPI_SLOT_BYTES / 2);
 #pragma unroll
-          for (int t = 0; t < EPI_ROWS; ++t) {
-            if (t < rows) {
-              const float f = __uint_as_float(v[t]) + bias_f;
-              orow[static_cast<size_t>(c * EPI_ROWS + t) * p.N] = __bfloat16_as_ushort(__float2bfloat16_rn(f));
-            }
+          for (int t = 0; t < EPI_ROWS; ++t)
+            sl[t * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[t]) + bias_f));
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            // rows past M and columns past N fall outside the tensor map and are dropped
+            ptx::tma_store_2d(&tm_out, slots_u32 + slot * EPI_SLOT_BYTES, n_tile * TILE_N + 32 * q, m0 + c * EPI_ROWS);
+            ptx::bulk_commit_group();
           }
+          ++nstore;
         }
       }
     }
+    if (lane == 0) ptx::bulk_wait_group<0>();
   }
 
   ptx::tc_fence_before();
@@ -442,6 +463,10 @@ int launch_fmt(const Problem& pr, int nsm) {
   } else {
     tm_b = tm_s;  // unused for ternary
   }
+  CUtensorMap tm_out;
+  if ((st = make_tensor_map_2d(&tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pr.out, pr.N, pr.M, uint64_t(pr.N) * 2, 32,
+                               EPI_ROWS, none, "out")) != QGEMM_OK)
+    return st;
   unsigned int* status;
   if ((st = status_word(&status)) != QGEMM_OK) return st;
   Params kp;
@@ -466,10 +491,9 @@ int launch_fmt(const Problem& pr, int nsm) {
     kp.m_fastest = live(kp.num_m_tiles, x_panel, w_panel) <= live(kp.num_n_tiles, w_panel, x_panel);
   }
   kp.bias = pr.bias;
-  kp.out = static_cast<uint16_t*>(pr.out);
   kp.wait_limit_ns = wait_limit_ns();
   kp.status = status;
-  large_m_kernel<BITS><<<grid, NUM_THREADS, C::kSmemBytes, pr.stream>>>(tm_x, tm_w, tm_s, tm_b, kp);
+  large_m_kernel<BITS><<<grid, NUM_THREADS, C::kSmemBytes, pr.stream>>>(tm_x, tm_w, tm_s, tm_b, tm_out, kp);
   return cuda_check(cudaGetLastError(), "large_m_kernel launch");
 }
 

@@ -17,8 +17,8 @@ struct Problem {
   int M, N, K;
   int bits, group;
   const uint8_t* packed;
-  const uint16_t* scales;  // fp16 bits [N, K/group]
-  const uint16_t* biases;  // fp16 bits [N, K/group] or nullptr (ternary)
+  const uint16_t* scales;  // fp16 bits [K/group, N] (group-major)
+  const uint16_t* biases;  // fp16 bits [K/group, N] or nullptr (ternary)
   void* out;             // bf16 [M, N]
   const uint16_t* bias;  // bf16 bits [N] or nullptr
   cudaStream_t stream;
@@ -49,5 +49,6 @@ int launch_debug_wait(uint64_t limit_ns, cudaStream_t stream);
 
 // Device status word values (0 = fine).
 constexpr unsigned kStatusTimeout = 1u;
+constexpr unsigned kStatusLayout = 2u;  // dynamic shared memory not aligned as the kernel requires
 
 }  // namespace qg

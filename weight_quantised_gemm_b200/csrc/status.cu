@@ -99,6 +99,8 @@ extern "C" int qgemm_get_device_status(void* stream) {
     const unsigned int zero = 0;
     st = cuda_check(cudaMemcpyToSymbol(g_status_word, &zero, sizeof zero), "clear status word");
     if (st != QGEMM_OK) return st;
+    if (v & kStatusLayout)
+      return fail(QGEMM_ERR_CUDA, "a kernel found its shared-memory base off its alignment (status word 0x%x)", v);
     return fail(QGEMM_ERR_DEVICE_TIMEOUT, "a kernel gave up a bounded wait (status word 0x%x)", v);
   }
   return QGEMM_OK;
