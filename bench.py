@@ -84,59 +84,109 @@ def profiled_traffic():
 # ----------------------------------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event reasons sampled every few milliseconds
+    while the bench runs (NVML, read-only; nvidia-smi as a fallback). The
+    report covers the samples taken between mark_begin() and mark_end(), the
+    timed region."""
+    REASONS = (("sw_power_cap", 0x4), ("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+               ("hw_thermal_slowdown", 0x40), ("hw_power_brake_slowdown", 0x80))
+    SMI_FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.sw_power_cap,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.hw_power_brake_slowdown")
 
-    def __init__(self, device_index: int):
-        self.dev = device_index
+    def __init__(self, device_id: str, period_s: float = 0.005):
+        self.dev = device_id
+        self.period = period_s
+        self.samples = []  # (t, sm_mhz, power_w, [reason names])
+        self.sm_max = None
+        self.source = None
+        self.t_begin = self.t_end = None
+        self._stop = threading.Event()
+        self.thread = None
         self.proc = None
-        self.lines = []
-        self.t = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        if self.dev.startswith("GPU-") or self.dev.startswith("MIG-"):
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(self.dev)
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(int(self.dev))
 
     def start(self):
         try:
+            nv, h = self._nvml_handle()
+            self.sm_max = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.source = "nvml"
+
+            def loop():
+                while not self._stop.is_set():
+                    try:
+                        t = time.monotonic()
+                        clk = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        bits = get_reasons(h)
+                        self.samples.append((t, float(clk), pw, [n for n, b in self.REASONS if bits & b]))
+                    except Exception:  # a failed read only loses that sample
+                        pass
+                    self._stop.wait(self.period)
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            pass
+        try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.SMI_FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, FileNotFoundError):
             self.proc = None
             return
-        self.t = threading.Thread(target=self._read, daemon=True)
-        self.t.start()
+        self.source = "nvidia-smi"
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+        def read():
+            for line in self.proc.stdout:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) != 8:
+                    continue
+                try:
+                    clk, mx, pw = float(parts[0]), float(parts[1]), float(parts[2])
+                except ValueError:
+                    continue
+                self.sm_max = mx
+                names = [n for (n, _), v in zip(self.REASONS, parts[3:]) if v.lower().startswith("active")]
+                self.samples.append((time.monotonic(), clk, pw, names))
+        self.thread = threading.Thread(target=read, daemon=True)
+        self.thread.start()
+
+    def mark_begin(self):
+        self.t_begin = time.monotonic()
+
+    def mark_end(self):
+        self.t_end = time.monotonic()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        if self.t:
-            self.t.join(timeout=2)
-        rows = []
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) != 8:
-                continue
+        self._stop.set()
+        if self.proc is not None:
+            self.proc.terminate()
             try:
-                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
-            except ValueError:
-                continue
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        rows = list(self.samples)
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        loaded = [r for r in rows if r[3] >= 50.0] or rows
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[4]) if v.lower().startswith("active")})
-        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded),
-                "power_w_max": max(r[2] for r in rows)}
+            return {"sm_mhz": None, "sm_max_mhz": self.sm_max, "reasons": [], "samples": 0, "source": self.source}
+        lo = self.t_begin if self.t_begin is not None else rows[0][0]
+        hi = self.t_end if self.t_end is not None else rows[-1][0]
+        timed = [r for r in rows if lo <= r[0] <= hi]
+        reasons = sorted({n for r in timed for n in r[3]})
+        return {"sm_mhz": statistics.median(r[1] for r in timed) if timed else None, "sm_max_mhz": self.sm_max,
+                "reasons": reasons, "samples": len(rows), "samples_in_timed_region": len(timed),
+                "sm_mhz_min_in_timed_region": min((r[1] for r in timed), default=None),
+                "power_w_max": max(r[2] for r in rows), "period_ms": self.period * 1e3, "source": self.source}
 
 
 # ----------------------------------------------------------------------------
@@ -352,6 +402,7 @@ def run_ours(args, rank, world, local_rank):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
+    clocks.mark_begin()
     t0.record(stream)
     for i in range(args.steps):
         ev[i][0].record(stream)
@@ -359,6 +410,7 @@ def run_ours(args, rank, world, local_rank):
         ev[i][1].record(stream)
     t1.record(stream)
     barrier(world)
+    clocks.mark_end()
     clk = clocks.stop()
     st = wq.qgemm_get_device_status()
     if st != 0:

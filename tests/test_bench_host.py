@@ -1,0 +1,41 @@
+"""bench.py host logic that needs no GPU: the clock report covers only the
+timed region, and every reason NVML can flag is named."""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def _sampler_with(samples, begin, end):
+    c = bench.ClockSampler("0")
+    c.samples = samples
+    c.sm_max = 1965.0
+    c.source = "test"
+    c.t_begin, c.t_end = begin, end
+    return c
+
+
+def test_clock_report_keeps_only_the_timed_region():
+    rows = [(0.0, 300.0, 90.0, []), (1.0, 1965.0, 700.0, []), (1.5, 1800.0, 990.0, ["sw_power_cap"]),
+            (2.0, 1900.0, 800.0, []), (3.0, 500.0, 100.0, ["hw_slowdown"])]
+    r = _sampler_with(rows, 0.9, 2.1).stop()
+    assert r["samples"] == 5 and r["samples_in_timed_region"] == 3
+    assert r["sm_mhz"] == 1900.0
+    assert r["sm_mhz_min_in_timed_region"] == 1800.0
+    assert r["reasons"] == ["sw_power_cap"]   # the slowdown after the region is not reported
+    assert r["sm_max_mhz"] == 1965.0
+
+
+def test_clock_report_without_samples():
+    r = _sampler_with([], 0.0, 1.0).stop()
+    assert r["sm_mhz"] is None and r["samples"] == 0
+
+
+def test_reason_bits_are_distinct():
+    bits = [b for _, b in bench.ClockSampler.REASONS]
+    assert len(set(bits)) == len(bits)
+    names = {n for n, _ in bench.ClockSampler.REASONS}
+    assert {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"} <= names

@@ -33,13 +33,13 @@
 //                  (group-major at rest, so one 256-byte TMA row per group).
 // TMEM columns: the fp32 accumulator in 0..255, the A stages from 256 on.
 //
-// Warp roles (864 threads):
+// Warp roles (608 threads):
 //   warp 0        TMA producer of X
 //   warp 1        MMA issuer (one thread) and TMEM owner
 //   warp 2        TMA producer of the W ring
-//   warps 3..18   dequantisers: warp w writes TMEM lanes 32 (w % 4) ..+31 (its
-//                 lane quarter), one 32-k slice of every stage
-//   warps 19..26  epilogue: tcgen05.ld one lane quarter x 128 tokens of the
+//   warps 3..10   dequantisers: warp w writes TMEM lanes 32 (w % 4) ..+31 (its
+//                 lane quarter), SLICES_PER_WARP 32-k slices of every stage
+//   warps 11..18  epilogue: tcgen05.ld one lane quarter x 128 tokens of the
 //                 accumulator 32 tokens at a time, add the bias, round to bf16
 //                 into the warp's own 2 KB shared-memory slot (transposed to
 //                 token-major) and TMA-store the 32 x 32 block; the
@@ -66,7 +66,8 @@ constexpr int BK = 128;      // K per pipeline stage
 constexpr int BOX_K = 64;    // K per X box: one 128-byte swizzle row of bf16
 constexpr int UMMA_K = 16;
 constexpr int SLICE_K = 32;  // K per dequantiser slice: four 8-element chunks
-constexpr int NUM_DEQ_WARPS = 4 * (BK / SLICE_K);  // a lane quarter x a slice each
+constexpr int SLICES_PER_WARP = 2;
+constexpr int NUM_DEQ_WARPS = 4 * (BK / SLICE_K) / SLICES_PER_WARP;  // a lane quarter x slices each
 constexpr int NUM_EPI_WARPS = 8;                   // a lane quarter x half the tokens each
 constexpr int WARP_XLOAD = 0;
 constexpr int WARP_MMA = 1;
@@ -272,50 +273,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == WARP_MMA) {
     // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      uint32_t it = 0, tcount = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tcount) {
-        // the epilogue has read the previous tile's accumulator out
-        if (!ptx::mbar_wait(acc_empty, (tcount & 1) ^ 1, lim, abort_flag)) {
-          give_up();
+    // The whole warp runs the loop and waits; one elected lane issues. Keeping
+    // the warp converged lets the loop state stay in uniform registers, which
+    // shortens the issuing thread's dependency chain per MMA.
+    uint32_t it = 0, tcount = 0;
+    bool ok = true;
+    const bool leader = ptx::elect_one();
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+      if (!warp_wait(acc_empty, (tcount & 1) ^ 1, lim, abort_flag)) {
+        if (leader) give_up();
+        break;
+      }
+      ptx::tc_fence_after();
+      for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+        const int s = it % S;
+        if (!warp_wait(full(s), (it / S) & 1, lim, abort_flag)) {
+          if (leader) give_up();
+          ok = false;
           break;
         }
         ptx::tc_fence_after();
-        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-          const int s = it % S;
-          if (!ptx::mbar_wait(full(s), (it / S) & 1, lim, abort_flag)) {
-            give_up();
-            ok = false;
-            break;
-          }
-          ptx::tc_fence_after();
+        if (leader) {
           const uint32_t a0 = tmem_base + A_COL + s * A_STAGE_COLS;
-          const uint32_t xs = x_stage(s);
+          const uint64_t d0 = ptx::smem_desc_sw128_kmajor(x_stage(s));
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk) {
             const uint32_t xo = (kk / (BOX_K / UMMA_K)) * X_BOX_BYTES + (kk % (BOX_K / UMMA_K)) * UMMA_K * 2;
-            ptx::tc_mma_f16_ts(tmem_base + ACC_COL, a0 + kk * (UMMA_K / 2), ptx::smem_desc_sw128_kmajor(xs + xo),
-                               IDESC, (kb | kk) != 0);
+            ptx::tc_mma_f16_ts(tmem_base + ACC_COL, a0 + kk * (UMMA_K / 2), d0 + (xo >> 4), IDESC, (kb | kk) != 0);
           }
           ptx::tc_commit(empty(s));
         }
-        if (!ok) break;
-        ptx::tc_commit(acc_full);
+        __syncwarp();
       }
-      // All MMAs issued above complete before TMEM is released.
+      if (!ok) break;
+      if (leader) ptx::tc_commit(acc_full);
+      __syncwarp();
+    }
+    if (leader) {
       ptx::tc_commit(drain_bar);
       ptx::mbar_wait(drain_bar, 0, lim, nullptr);
     }
+    __syncwarp();
   } else if (warp < WARP_EPI0) {
     // ---------------- dequantisers: packed smem tile -> bf16 in TMEM ----------------
     const int d = warp - WARP_DEQ0;
-    const int q = warp & 3;    // TMEM lane quarter this warp may write
-    const int j = d >> 2;      // 32-k slice of each stage
-    const int r = 32 * q + lane;  // tile row = TMEM lane
-    const int g = (j * SLICE_K) / C::kGroup;  // scale group of the slice within the stage
+    const int q = warp & 3;                     // TMEM lane quarter this warp may write
+    const int j0 = (d >> 2) * SLICES_PER_WARP;  // first 32-k slice of each stage
+    const int r = 32 * q + lane;                // tile row = TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-    const uint32_t w_off = static_cast<uint32_t>(r * C::kWRowBytes + j * C::kSliceBytes);
     for (uint32_t it = 0; it < total; ++it) {
       const int s = it % S, sw = it % SW;
       if (!warp_wait(full_w(sw), (it / SW) & 1, lim, abort_flag) ||
@@ -326,36 +331,50 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::tc_fence_after();  // the MMA that last read this A stage has completed
       const uint8_t* wt = smem + C::kOffW + sw * C::kWTileBytes;
       const uint16_t* sb = reinterpret_cast<const uint16_t*>(smem + C::kOffSB + sw * C::kSBStride);
-      const float s_cur = deq::h2f(sb[g * TILE_N + r]);
-      const float b_cur = BITS == 2 ? 0.f : deq::h2f(sb[C::kSBytes / 2 + g * TILE_N + r]);
-      uint4 o[4];  // 4 chunks of 8 consecutive k = this thread's 32 k
-      if constexpr (BITS == 4) {
-        const uint4 v = *reinterpret_cast<const uint4*>(wt + swz<C::kSwzMask>(w_off));
-        o[0] = deq::chunk_4bit(v.x, s_cur, b_cur);
-        o[1] = deq::chunk_4bit(v.y, s_cur, b_cur);
-        o[2] = deq::chunk_4bit(v.z, s_cur, b_cur);
-        o[3] = deq::chunk_4bit(v.w, s_cur, b_cur);
-      } else if constexpr (BITS == 8) {
-        const uint4 v0 = *reinterpret_cast<const uint4*>(wt + swz<C::kSwzMask>(w_off));
-        const uint4 v1 = *reinterpret_cast<const uint4*>(wt + swz<C::kSwzMask>(w_off + 16));
-        o[0] = deq::chunk_8bit(v0.x, v0.y, s_cur, b_cur);
-        o[1] = deq::chunk_8bit(v0.z, v0.w, s_cur, b_cur);
-        o[2] = deq::chunk_8bit(v1.x, v1.y, s_cur, b_cur);
-        o[3] = deq::chunk_8bit(v1.z, v1.w, s_cur, b_cur);
-      } else {
-        const uint2 v = *reinterpret_cast<const uint2*>(wt + swz<C::kSwzMask>(w_off));
-        const uint32_t hs = deq::ternary_half_scale2(s_cur);
-        o[0] = deq::chunk_ternary<0>(v.x, hs);
-        o[1] = deq::chunk_ternary<1>(v.x, hs);
-        o[2] = deq::chunk_ternary<0>(v.y, hs);
-        o[3] = deq::chunk_ternary<1>(v.y, hs);
+      uint32_t regs[SLICES_PER_WARP][16];
+#pragma unroll
+      for (int u = 0; u < SLICES_PER_WARP; ++u) {
+        const int j = j0 + u;
+        const int g = (j * SLICE_K) / C::kGroup;  // scale group of the slice within the stage
+        const uint32_t w_off = static_cast<uint32_t>(r * C::kWRowBytes + j * C::kSliceBytes);
+        const float s_cur = deq::h2f(sb[g * TILE_N + r]);
+        const float b_cur = BITS == 2 ? 0.f : deq::h2f(sb[C::kSBytes / 2 + g * TILE_N + r]);
+        uint4 o[4];  // 4 chunks of 8 consecutive k = the slice's 32 k
+        if constexpr (BITS == 4) {
+          const uint4 v = *reinterpret_cast<const uint4*>(wt + swz<C::kSwzMask>(w_off));
+          o[0] = deq::chunk_4bit(v.x, s_cur, b_cur);
+          o[1] = deq::chunk_4bit(v.y, s_cur, b_cur);
+          o[2] = deq::chunk_4bit(v.z, s_cur, b_cur);
+          o[3] = deq::chunk_4bit(v.w, s_cur, b_cur);
+        } else if constexpr (BITS == 8) {
+          const uint4 v0 = *reinterpret_cast<const uint4*>(wt + swz<C::kSwzMask>(w_off));
+          const uint4 v1 = *reinterpret_cast<const uint4*>(wt + swz<C::kSwzMask>(w_off + 16));
+          o[0] = deq::chunk_8bit(v0.x, v0.y, s_cur, b_cur);
+          o[1] = deq::chunk_8bit(v0.z, v0.w, s_cur, b_cur);
+          o[2] = deq::chunk_8bit(v1.x, v1.y, s_cur, b_cur);
+          o[3] = deq::chunk_8bit(v1.z, v1.w, s_cur, b_cur);
+        } else {
+          const uint2 v = *reinterpret_cast<const uint2*>(wt + swz<C::kSwzMask>(w_off));
+          const uint32_t hs = deq::ternary_half_scale2(s_cur);
+          o[0] = deq::chunk_ternary<0>(v.x, hs);
+          o[1] = deq::chunk_ternary<1>(v.x, hs);
+          o[2] = deq::chunk_ternary<0>(v.y, hs);
+          o[3] = deq::chunk_ternary<1>(v.y, hs);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          regs[u][4 * c + 0] = o[c].x;
+          regs[u][4 * c + 1] = o[c].y;
+          regs[u][4 * c + 2] = o[c].z;
+          regs[u][4 * c + 3] = o[c].w;
+        }
       }
       // The packed stage has been read: give it back to the W producer.
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(empty_w(sw));
-      const uint32_t regs[16] = {o[0].x, o[0].y, o[0].z, o[0].w, o[1].x, o[1].y, o[1].z, o[1].w,
-                                 o[2].x, o[2].y, o[2].z, o[2].w, o[3].x, o[3].y, o[3].z, o[3].w};
-      ptx::tmem_st_32x32b_x16(tmem_base + lane_addr + A_COL + s * A_STAGE_COLS + j * (SLICE_K / 2), regs);
+#pragma unroll
+      for (int u = 0; u < SLICES_PER_WARP; ++u)
+        ptx::tmem_st_32x32b_x16(tmem_base + lane_addr + A_COL + s * A_STAGE_COLS + (j0 + u) * (SLICE_K / 2), regs[u]);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();

@@ -216,9 +216,17 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
 // Waits until this thread's earlier tcgen05.st have completed.
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// One lane of the (converged) warp, chosen by the hardware.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(pred));
+  return pred != 0;
+}
+
 // Shared-memory matrix descriptor for tcgen05.mma: K-major operand laid out
 // with the 128-byte swizzle (rows of 128 B, 8-row atoms of 1024 B). The start
-// address may be advanced by 32 B steps inside an atom to select K slices.
+// address may be advanced by 32 B steps inside an atom to select K slices, by
+// adding (offset >> 4) to the descriptor (the address field does not carry).
 __device__ __forceinline__ uint64_t smem_desc_sw128_kmajor(uint32_t saddr) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);  // start address, bits 0-13
