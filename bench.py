@@ -320,6 +320,15 @@ def sweep(peaks):
                  "bound": "tensor" if flops / P >= ab / BW else "hbm",
                  "roofline_us": round(t_roof * 1e6, 2), "frac_of_roofline": round(t_roof / t, 3),
                  "copies": ncopy}
+        if entry["path"] == "small":
+            # the same launches with QGEMM_FLAG_OVERLAP_PREVIOUS: each GEMV's weight
+            # stream may start while the previous one in the stream finishes
+            fo = [(lambda s=s: wq.qgemm(s[0], s[1], bias=s[2], out=s[3], path=path, overlap_previous=True))
+                  for s in sets]
+            to = time_graph((fo * (-(-launches // len(fo))))[:max(launches, len(fo))])
+            wq.check_device_status()
+            entry["us_overlap_previous"] = round(to * 1e6, 2)
+            entry["frac_of_roofline_overlap_previous"] = round(t_roof / to, 3)
         return entry, sets, host
 
     for cid in range(5):
@@ -367,7 +376,8 @@ def sweep(peaks):
                 if path == wq.QGEMM_PATH_SMALL_M and M > 16:
                     continue
                 e, sets, _ = one(3, 0, lin, M, path, 100)
-                cross.append({k: e[k] for k in ("bits", "M", "path", "us", "gbs", "frac_of_roofline")})
+                cross.append({k: e[k] for k in ("bits", "M", "path", "us", "gbs", "frac_of_roofline",
+                                                "us_overlap_previous") if k in e})
                 del sets
     torch.cuda.empty_cache()
     return res, block, cross

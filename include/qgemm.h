@@ -71,11 +71,26 @@ typedef enum qgemm_status {
   QGEMM_ERR_DEVICE_TIMEOUT = 6   /* a kernel's bounded wait ran out (see qgemm_get_device_status) */
 } qgemm_status;
 
-/* Kernel path selection for qgemm_ex. */
+/* Kernel path selection for qgemm_ex (low byte of its `path` argument). */
 enum {
   QGEMM_PATH_AUTO = 0,     /* pick per shape from the measured table */
   QGEMM_PATH_SMALL_M = 1,  /* memory-bound path: registers + mma.sync, M <= 16 */
-  QGEMM_PATH_LARGE_M = 2   /* tensor-core path: TMA + smem dequant + tcgen05 MMA into TMEM */
+  QGEMM_PATH_LARGE_M = 2   /* tensor-core path: TMA + dequant into TMEM + tcgen05 MMA */
+};
+
+/* Flags OR-ed into qgemm_ex's `path` argument.
+ *
+ * QGEMM_FLAG_OVERLAP_PREVIOUS: launch the small-M kernel with programmatic
+ * dependent launch. Its CTAs may start while the previous kernel in the stream
+ * is still running and put the packed weights, scales and biases in flight at
+ * once; they wait for that kernel to complete (and its writes to be visible)
+ * before reading X or bias and before writing out. Ask for it only when the
+ * weight buffers are not written by the work that precedes the call in the
+ * stream (static weights, as in inference). It has no effect on the large-M
+ * path. No counterpart in the method's description: a launch-overlap option
+ * of this implementation. */
+enum {
+  QGEMM_FLAG_OVERLAP_PREVIOUS = 0x100
 };
 
 /* A packed weight matrix resident in device memory. */
@@ -131,7 +146,8 @@ int qgemm(const void* X, int32_t M, const qgemm_weights* W, void* out,
           const void* bias, void* stream);
 
 /* As qgemm, with an explicit QGEMM_PATH_* choice (AUTO defers to the table and
- * the QGEMM_PATH variable). */
+ * the QGEMM_PATH variable), optionally OR-ed with QGEMM_FLAG_* bits. Unknown
+ * path values or flag bits return QGEMM_ERR_INVALID_ARG. */
 int qgemm_ex(const void* X, int32_t M, const qgemm_weights* W, void* out,
              const void* bias, int32_t path, void* stream);
 

@@ -111,6 +111,8 @@ def test_qgemm_rejects_bad_operands_without_device():
     assert _call(d, out=0x20002) == wq.QGEMM_ERR_ALIGNMENT
     assert _call(d, bias=0x30001) == wq.QGEMM_ERR_ALIGNMENT
     assert _call(d, path=7) == wq.QGEMM_ERR_INVALID_ARG
+    assert _call(d, path=wq.QGEMM_PATH_LARGE_M | 0x200) == wq.QGEMM_ERR_INVALID_ARG   # unknown flag bit
+    assert _call(d, M=0, path=wq.QGEMM_PATH_SMALL_M | wq.QGEMM_FLAG_OVERLAP_PREVIOUS) == wq.QGEMM_OK
     assert _call(d, M=17, path=wq.QGEMM_PATH_SMALL_M) == wq.QGEMM_ERR_UNSUPPORTED
     # M = 0 is a no-op that never touches the device
     assert _call(d, M=0) == wq.QGEMM_OK

@@ -210,3 +210,56 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     X, W, bias = WL.random_case(1, 4, 128, 128, 4, with_bias=False)
     y, _ = gpu_qgemm(X, W, bias, 4)
     _assert_close(y, _ref(X, W, bias, 4), "after timeout")
+
+
+# ----------------------------------------------------------------------------
+# launch overlap (QGEMM_FLAG_OVERLAP_PREVIOUS): the activations are read only
+# after the previous kernel in the stream has finished
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_overlap_reads_the_previous_kernels_output(bits):
+    """A chain y1 = X W1^T, y2 = y1 W2^T with the second call overlapping the
+    first: y2 must be the GEMM of the y1 that the first call produced."""
+    M, K1, N1, N2 = 4, 1024, 1024, 2048
+    X, W1, _ = WL.random_case(91 + bits, M, N1, K1, bits, with_bias=False)
+    _, W2, bias2 = WL.random_case(92 + bits, M, N2, N1, bits, with_bias=True)
+    d1, d2 = wq.qgemm_pack(W1, bits).to_device(), wq.qgemm_pack(W2, bits).to_device()
+    Xd, b2 = to_dev_bf16(X), to_dev_bf16(bias2)
+    for _ in range(3):  # repeat: each round re-writes y1 and y2 in place
+        y1 = torch.full((M, N1), float("nan"), dtype=torch.bfloat16, device="cuda")
+        y1 = wq.qgemm(Xd, d1, out=y1, path=SMALL)
+        y2 = wq.qgemm(y1, d2, bias=b2, path=SMALL, overlap_previous=True)
+        wq.check_device_status()
+        y1_bits = from_dev_bf16(y1)
+        _assert_close(y1_bits, _ref(X, W1, None, bits), "first")
+        _assert_close(from_dev_bf16(y2), _ref(y1_bits, W2, bias2, bits), "second, overlapped")
+
+
+def test_overlap_after_a_torch_kernel_and_in_a_graph():
+    """The previous kernel is a plain torch one (no trigger of its own), and the
+    same overlapped call captured in a CUDA graph gives the same result."""
+    M, N, K, bits = 3, 1536, 2048, 4
+    X, W, bias = WL.random_case(95, M, N, K, bits, with_bias=True)
+    dw = wq.qgemm_pack(W, bits).to_device()
+    src, bd = to_dev_bf16(X), to_dev_bf16(bias)
+    Xd = torch.zeros_like(src)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    Xd.copy_(src)  # a device kernel writes X right before the call
+    wq.qgemm(Xd, dw, bias=bd, out=out, path=SMALL, overlap_previous=True)
+    wq.check_device_status()
+    y_eager = from_dev_bf16(out)
+    _assert_close(y_eager, _ref(X, W, bias, bits), "eager")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        Xd.copy_(src)
+        wq.qgemm(Xd, dw, bias=bd, out=out, path=SMALL, overlap_previous=True)
+    out.zero_()
+    Xd.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    wq.check_device_status()
+    assert np.array_equal(from_dev_bf16(out), y_eager)
+    del g

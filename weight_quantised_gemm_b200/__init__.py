@@ -33,6 +33,7 @@ QGEMM_ERR_DEVICE_TIMEOUT = 6
 QGEMM_PATH_AUTO = 0
 QGEMM_PATH_SMALL_M = 1
 QGEMM_PATH_LARGE_M = 2
+QGEMM_FLAG_OVERLAP_PREVIOUS = 0x100
 
 GROUP_OF_BITS = {2: 128, 4: 64, 8: 64}
 
@@ -191,9 +192,11 @@ def _stream_handle(stream) -> Optional[int]:
     return stream.cuda_stream
 
 
-def qgemm(X, W: DeviceWeights, bias=None, out=None, path: int = QGEMM_PATH_AUTO, stream=None):
+def qgemm(X, W: DeviceWeights, bias=None, out=None, path: int = QGEMM_PATH_AUTO, stream=None,
+          overlap_previous: bool = False):
     """out[M, N] = X[M, K] . dequant(W)^T (+ bias), bf16 in and out, on `stream`
-    (default: torch's current stream). Enqueues only; see qgemm_get_device_status."""
+    (default: torch's current stream). Enqueues only; see qgemm_get_device_status.
+    overlap_previous sets QGEMM_FLAG_OVERLAP_PREVIOUS (weights must be static)."""
     import torch
     if X.dtype != torch.bfloat16 or not X.is_cuda or X.dim() != 2 or not X.is_contiguous():
         raise ValueError("X must be a contiguous 2-D bf16 CUDA tensor")
@@ -207,8 +210,10 @@ def qgemm(X, W: DeviceWeights, bias=None, out=None, path: int = QGEMM_PATH_AUTO,
     if bias is not None and (bias.dtype != torch.bfloat16 or bias.numel() != W.N or not bias.is_cuda):
         raise ValueError("bias must be a bf16 CUDA tensor of N elements")
     desc = W.descriptor()
+    flags = QGEMM_FLAG_OVERLAP_PREVIOUS if overlap_previous else 0
     _check(_lib.qgemm_ex(X.data_ptr(), M, ctypes.byref(desc), out.data_ptr(),
-                         None if bias is None else bias.data_ptr(), int(path), _stream_handle(stream)), "qgemm")
+                         None if bias is None else bias.data_ptr(), int(path) | flags, _stream_handle(stream)),
+           "qgemm")
     return out
 
 

@@ -91,7 +91,10 @@ extern "C" int qgemm_ex(const void* X, int32_t M, const qgemm_weights* W, void* 
   int st = validate_weights(W);
   if (st != QGEMM_OK) return st;
   if (M < 0) return fail(QGEMM_ERR_INVALID_ARG, "M=%d is negative", M);
+  const int32_t flags = path & ~0xFF;
+  path &= 0xFF;
   if (path < QGEMM_PATH_AUTO || path > QGEMM_PATH_LARGE_M) return fail(QGEMM_ERR_INVALID_ARG, "bad path %d", path);
+  if (flags & ~QGEMM_FLAG_OVERLAP_PREVIOUS) return fail(QGEMM_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
   if (M == 0) return QGEMM_OK;
   if (!X || !out) return fail(QGEMM_ERR_INVALID_ARG, "null X or out");
   if (!aligned16(X) || !aligned16(out)) return fail(QGEMM_ERR_ALIGNMENT, "X and out must be 16-byte aligned");
@@ -103,7 +106,8 @@ extern "C" int qgemm_ex(const void* X, int32_t M, const qgemm_weights* W, void* 
     return fail(QGEMM_ERR_UNSUPPORTED, "the small-M path takes M <= 16 (M=%d)", M);
   Problem p{X, M, W->N, W->K, W->bits, W->group, static_cast<const uint8_t*>(W->packed),
             static_cast<const uint16_t*>(W->scales), static_cast<const uint16_t*>(W->biases), out,
-            static_cast<const uint16_t*>(bias), static_cast<cudaStream_t>(stream)};
+            static_cast<const uint16_t*>(bias), static_cast<cudaStream_t>(stream),
+            (flags & QGEMM_FLAG_OVERLAP_PREVIOUS) != 0};
   return path == QGEMM_PATH_SMALL_M ? launch_small_m(p) : launch_large_m(p);
 }
 

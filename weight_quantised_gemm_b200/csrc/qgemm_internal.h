@@ -22,6 +22,7 @@ struct Problem {
   void* out;             // bf16 [M, N]
   const uint16_t* bias;  // bf16 bits [N] or nullptr
   cudaStream_t stream;
+  bool overlap;          // launch with programmatic dependent launch (QGEMM_FLAG_OVERLAP_PREVIOUS)
 };
 
 // Records a detail message for qgemm_last_error and returns `code`.
@@ -39,6 +40,13 @@ int sm_count(int* n);
 // and stores outside it are dropped.
 int make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz,
+                       const char* what);
+
+// 3-D TMA descriptor: dims[0] x dims[1] x dims[2] elements with byte strides
+// strides_bytes[0] (dimension 1) and strides_bytes[1] (dimension 2), in any
+// order of size; box box[0] x box[1] x box[2].
+int make_tensor_map_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, const uint64_t dims[3],
+                       const uint64_t strides_bytes[2], const uint32_t box[3], CUtensorMapSwizzle swz,
                        const char* what);
 
 // Kernel launchers (one per kernel family). Each enqueues on p.stream.

@@ -3,20 +3,37 @@
 //
 // pictor's README ("Extreme quantization is first-class") names GEMV paths
 // built for sub-byte weights; at decode-sized M the packed bytes set the time,
-// so this kernel is built around keeping HBM busy:
+// so this kernel is built around keeping HBM busy from its first microsecond:
 //
-// * One CTA per SM owns a contiguous range of weight rows (whole n8 blocks).
-//   A producer warp streams that range through a shared-memory ring with TMA:
-//   per stage, the packed codes of 128 bytes of K for every row (128-byte
-//   swizzle), the stage's fp16 scales (and biases) as one box, and the
-//   matching slice of the activations, copied row by row with bulk copies
-//   into a padded layout. The ring holds up to eight stages, so at the
-//   workloads' K every load of the CTA is in flight from the start.
-// * Eight consumer warps turn codes into bf16 in registers and feed warp-level
-//   mma.sync (m16n8k16, bf16 in, fp32 accumulate): the activations are the
-//   16-row A operand (rows past M are zero), the weights the 8-column B.
-//   The warps split each stage by whole groups and meet once, at the end, in
-//   shared memory.
+// * One CTA per SM owns 16 * NP consecutive weight rows (it takes most of the
+//   SM's shared memory, so two CTAs of one grid never share an SM and split
+//   its load bandwidth). A producer warp streams the rows through a
+//   shared-memory ring, one stage per 8 scale groups of K. A stage takes one 3-D TMA box for the packed codes of all the CTA's
+//   rows (viewed as [row][unit][U bytes], U = 128, 64 or 32, the box lands as
+//   [unit][row][U bytes] with the U-byte swizzle, so the per-lane row reads
+//   are free of bank conflicts), one 2-D box each for the stage's fp16 scales
+//   and biases, and one bulk copy per token row of the activations, issued by
+//   the producer warp's lanes in parallel. (Per-lane 16-byte cp.async pieces
+//   for the activations were measured slower at M = 16.)
+// * Eight consumer warps. Normally warp w takes scale group w of every stage
+//   for all the CTA's rows; where that would not fit in registers (16 tokens
+//   and 12 or more row pairs) the rows split into two halves and warps w and
+//   w + 4 take groups w % 4 and w % 4 + 4 of every stage, each for its half.
+//   A warp turns codes into bf16 in registers and feeds warp-level mma.sync
+//   (m16n8k16, bf16 in, fp32 accumulate): the weights are the 16-row A
+//   operand, the activations the 8-column B (tokens past M are zero). At the
+//   end the warps' fp32 partial sums meet in shared memory (token-major,
+//   bank-conflict free) and a coalesced pass adds them, adds the bias and
+//   writes bf16.
+// * Overlap (programmatic dependent launch, when the caller asks for it): the
+//   producer puts the first stages' weight, scale and bias loads in flight,
+//   lets the next grid in the stream launch, and only then waits for the
+//   previous grid to finish before it copies activations. Every thread waits
+//   for the previous grid before it reads the bias or writes the output. A
+//   CTA of the next launch then takes an SM the moment this grid's CTA there
+//   exits, and its weight stream overlaps the other SMs' last stages instead
+//   of waiting for the whole grid and a fresh launch. Without the launch
+//   attribute both steps are no-ops.
 //
 // Scale and bias are applied per group on the fp32 partial sums instead of
 // per weight, which is the same product:
@@ -42,36 +59,45 @@
 namespace qg {
 namespace sm {
 
-constexpr int NBMAX = 12;             // n8 blocks (of 8 weight rows) per CTA, at most
-constexpr int NPMAX = NBMAX / 2;      // n16 pairs of blocks: the weight rows of one mma
-constexpr int PPW = NPMAX;            // pairs per consumer warp
 constexpr int NUM_CONSUMER_WARPS = 8;
 constexpr int WARP_PRODUCER = NUM_CONSUMER_WARPS;
 constexpr int NUM_THREADS = 32 * (NUM_CONSUMER_WARPS + 1);  // 288
 constexpr int MAX_STAGES = 8;
-constexpr int ROW_BYTES_PER_STAGE = 128;  // one 128-byte swizzle row of packed codes
-constexpr int RING_BUDGET = 196608;       // bytes of shared memory for the ring
+constexpr int SMEM_LIMIT = 232448;      // the most a CTA may have
+constexpr int RING_BUDGET = 196608;     // bytes of shared memory for the ring
+constexpr int SMEM_FLOOR = 118784;      // at least this much, so that one grid's CTAs never share an SM
+constexpr int GS = 8;                   // scale groups per stage
 
 template <int BITS>
 struct Fmt {
-  static constexpr int G = BITS == 2 ? 128 : 64;          // group size
-  static constexpr int KS = ROW_BYTES_PER_STAGE * 8 / BITS;  // k per stage: 512, 256 or 128
-  static constexpr int GS = KS / G;                        // groups per stage: 4, 4, 2
-  static constexpr int STEPS = G / 16;                     // mma k-steps per group
-  static constexpr int NSETS = NUM_CONSUMER_WARPS / GS;  // warp sets sharing out the stages
-  static constexpr int GBYTES = G * BITS / 8;              // packed bytes per row and group
+  static constexpr int G = BITS == 2 ? 128 : 64;  // group size
+  static constexpr int GBYTES = G * BITS / 8;     // packed bytes per row and group
+  static constexpr int KS = GS * G;               // k per stage
+  static constexpr int ROWB = GS * GBYTES;        // packed bytes per row and stage
+  static constexpr int STEPS = G / 16;            // mma k-steps per group
 };
+
+// Row halves for a CTA of NP pairs and MT tokens: 2 where one warp's
+// accumulators for all NP pairs would not fit in registers.
+__host__ __device__ constexpr int split_rows(int MT, int NP) { return MT > 8 && NP >= 6 ? 2 : 1; }
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 struct Params {
   const uint16_t* X;     // bf16 [M, K]
   const uint16_t* bias;  // bf16 [N] or null
   uint16_t* out;         // bf16 [M, N]
   int M, N, K;
-  int bpc;               // n8 blocks per CTA
-  int num_stages;        // K / KS, rounded up
+  int num_stages;        // ceil(K / KS)
   int ring;              // ring depth
+  int unit;              // U: bytes per swizzled row piece (128, 64 or 32)
   int stage_bytes;       // bytes per ring stage (multiple of 1024)
-  int off_s, off_b, off_x, x_stride;  // offsets inside a stage; X row stride in bytes
+  int data_bytes;        // ring (or the partial sums, if larger); the mbarriers follow
+  int off_s, off_b, off_x, x_stride;  // offsets inside a stage; activation row stride in bytes
+  int overlap;           // launched with programmatic dependent launch
   uint64_t wait_limit_ns;
   unsigned int* status;
 };
@@ -95,26 +121,27 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_
   return __all_sync(0xffffffffu, ok);
 }
 
-// Byte offset, inside a stage row, of the 32-bit word that holds quad thread
-// c's 4 codes (k = 4c .. 4c+3) of step k of group gs. Rows carry the 128-byte
-// swizzle: logical 16-byte chunk j of row r sits at physical chunk j ^ (r % 8).
+// Logical byte offset, inside a stage row of packed codes, of the 32-bit word
+// that holds quad thread c's 4 codes (k = 4c .. 4c+3) of step k of group gs:
 //   ternary: one word per 16-k step (quad threads share it);
 //   4-bit:   two words per step, thread c reads word c / 2;
 //   8-bit:   four words per step, thread c reads word c.
 template <int BITS>
-__device__ __forceinline__ int word_offset(int gs, int k, int c, int r7) {
-  int chunk, wic;
-  if constexpr (BITS == 2) {
-    chunk = 2 * gs + (k >> 2);
-    wic = k & 3;
-  } else if constexpr (BITS == 4) {
-    chunk = 2 * gs + (k >> 1);
-    wic = 2 * (k & 1) + (c >> 1);
-  } else {
-    chunk = 4 * gs + k;
-    wic = c;
-  }
-  return ((chunk ^ r7) << 4) + 4 * wic;
+__device__ __forceinline__ int word_offset(int gs, int k, int c) {
+  constexpr int GB = Fmt<BITS>::GBYTES;
+  if constexpr (BITS == 2) return gs * GB + 4 * k;
+  else if constexpr (BITS == 4) return gs * GB + 8 * k + 4 * (c >> 1);
+  else return gs * GB + 16 * k + 4 * c;
+}
+
+// Physical byte offset in the stage of logical byte `off` of row r: the box
+// lands as [off / U][row][U bytes], each U-byte row piece swizzled by the TMA
+// (16-byte unit index XORed with address bits 7.. of the piece).
+__device__ __forceinline__ int phys_offset(int off, int r, int R, int U) {
+  const int plane = off / U, o = off - plane * U;
+  const int x = r * U + o;  // offset inside the plane; planes start on the swizzle period
+  const int mask = U == 128 ? 7 : U == 64 ? 3 : 1;
+  return plane * R * U + (x ^ (((x >> 7) & mask) << 4));
 }
 
 // B operand of one step for quad thread c from its word: codes 4c .. 4c+3 as
@@ -143,30 +170,37 @@ __device__ __forceinline__ void decode_word(uint32_t x, int c, uint32_t& b0, uin
   }
 }
 
-template <int BITS, int MT>
+template <int BITS, int MT, int NP>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     small_m_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
                    const __grid_constant__ CUtensorMap tm_b, const Params p) {
   using F = Fmt<BITS>;
   constexpr int STEPS = F::STEPS;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int R = 16 * NP;                 // weight rows of the CTA
+  constexpr int PH = split_rows(MT, NP);     // row halves (1 or 2)
+  constexpr int GROUP_LANES = NUM_CONSUMER_WARPS / PH;  // warps w and w + GROUP_LANES share a group lane
+  constexpr int NPH = NP / PH;               // 16-row pairs per warp
+  constexpr int GPL = GS / GROUP_LANES;      // groups per warp and stage
+  constexpr int TH = MT > 8 ? 2 : 1;         // 8-token halves
+  constexpr int NLP = R + 4;                 // row pitch of the partial sums: 2 * NLP = 8 (mod 32) banks
+  static_assert(NP % PH == 0, "the halves take whole 16-row pairs");
+  extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = ptx::smem_u32(smem);
+  if (sbase & 1023u) {  // the swizzled boxes need it; uniform across the block
+    if (threadIdx.x == 0) ptx::set_status(p.status, kStatusLayout);
+    return;
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
+  const int n0 = blockIdx.x * R;
+  const int U = p.unit;
 
-  const int nblocks_total = p.N / 8;
-  const int blk0 = blockIdx.x * p.bpc;
-  const int nb = min(p.bpc, nblocks_total - blk0);
-  const int n0 = 8 * blk0;
-  const int R = 8 * p.bpc;  // rows per TMA box (rows past N read as zeros)
-  const int data_bytes = max(p.ring * p.stage_bytes, NUM_CONSUMER_WARPS * PPW * 2 * 32 * 16);
-  const uint32_t bar0 = sbase + data_bytes;
+  const uint32_t bar0 = sbase + p.data_bytes;
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (MAX_STAGES + s); };
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + data_bytes + 16 * MAX_STAGES);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + p.data_bytes + 16 * MAX_STAGES);
   const uint64_t lim = p.wait_limit_ns;
-  // Each CTA walks the K slices starting at its own offset: every CTA reads
+  // Each CTA walks the K stages starting at its own offset: every CTA reads
   // the same activations, and rotating the order spreads those reads over
   // the L2 instead of sending all CTAs to the same lines at once.
   const int rot = blockIdx.x % p.num_stages;
@@ -174,7 +208,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.ring; ++s) {
       ptx::mbar_init(full(s), 1);
-      ptx::mbar_init(empty(s), F::GS);
+      ptx::mbar_init(empty(s), NUM_CONSUMER_WARPS);
     }
     *abort_flag = 0;
     ptx::fence_mbarrier_init();
@@ -185,55 +219,88 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::set_status(p.status, kStatusTimeout);
   };
 
-  // acc[p][h][j]: weight rows 16p + g (j < 2) and 16p + g + 8 (j >= 2), tokens
-  // 8h + 2c + (j & 1)
-  constexpr int TH = MT > 8 ? 2 : 1;
-  float acc[PPW][TH][4];
+  // acc[q][h][j]: weight rows 16q + g (j < 2) and 16q + g + 8 (j >= 2) of this
+  // warp's half, tokens 8h + 2c + (j & 1)
+  float acc[NPH][TH][4];
 #pragma unroll
-  for (int q = 0; q < PPW; ++q)
+  for (int q = 0; q < NPH; ++q)
 #pragma unroll
     for (int h = 0; h < TH; ++h)
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[q][h][j] = 0.f;
-  // Every CTA runs NPMAX n16 pairs with no per-pair branch, so the compiler can
-  // interleave the pairs' loads, decodes and mma. Rows past the CTA's own
-  // (past 8 * nb) are computed from whatever the stage holds there and are
-  // never written out; the stage reserves room for all 16 * NPMAX rows.
 
   if (warp == WARP_PRODUCER) {
     // ---------------- producer: TMA boxes and bulk copies into the ring ----------------
+    constexpr int sb_bytes = GS * R * 2;
+    const int units = F::ROWB / U;  // row pieces per stage
+    const int pre = p.ring < p.num_stages ? p.ring : p.num_stages;
+    auto stage_k = [&](int t, int& kt, int& valid) {
+      kt = (t + rot) % p.num_stages;  // which K stage ring round t carries
+      valid = min(F::KS, p.K - kt * F::KS);
+    };
+    auto load_weights = [&](int t, int s) {  // lane 0: the stage's packed codes, scales and biases
+      int kt, valid;
+      stage_k(t, kt, valid);
+      const uint32_t st = sbase + s * p.stage_bytes;
+      ptx::mbar_arrive_expect_tx(full(s), R * F::ROWB + sb_bytes * (BITS == 2 ? 1 : 2) + p.M * valid * 2);
+      ptx::tma_load_3d(st, &tm_w, 0, n0, kt * units, full(s));
+      ptx::tma_load_2d(st + p.off_s, &tm_s, n0, kt * GS, full(s));
+      if (BITS != 2) ptx::tma_load_2d(st + p.off_b, &tm_b, n0, kt * GS, full(s));
+    };
+    auto load_x = [&](int t, int s) {  // all lanes: one bulk copy per token row
+      int kt, valid;
+      stage_k(t, kt, valid);
+      const uint32_t st = sbase + s * p.stage_bytes;
+      for (int m = lane; m < p.M; m += 32)
+        bulk_copy_g2s(st + p.off_x + m * p.x_stride, p.X + static_cast<size_t>(m) * p.K + kt * F::KS, valid * 2,
+                      full(s));
+    };
     if (lane == 0) {
       ptx::tma_prefetch_desc(&tm_w);
       ptx::tma_prefetch_desc(&tm_s);
-      const int sb_bytes = F::GS * R * 2;
-      int t = 0;
-      for (; t < p.num_stages; ++t) {
-        const int s = t % p.ring;
-        if (!ptx::mbar_wait(empty(s), ((t / p.ring) & 1) ^ 1, lim, abort_flag)) {
-          give_up();
-          break;
-        }
-        const int kt = (t + rot) % p.num_stages;  // which K slice this ring slot carries
-        const int valid = min(F::KS, p.K - kt * F::KS);
-        const uint32_t st = sbase + s * p.stage_bytes;
-        ptx::mbar_arrive_expect_tx(full(s), R * ROW_BYTES_PER_STAGE + sb_bytes * (BITS == 2 ? 1 : 2) +
-                                                p.M * valid * 2);
-        ptx::tma_load_2d(st, &tm_w, kt * ROW_BYTES_PER_STAGE, n0, full(s));
-        ptx::tma_load_2d(st + p.off_s, &tm_s, n0, kt * F::GS, full(s));
-        if (BITS != 2) ptx::tma_load_2d(st + p.off_b, &tm_b, n0, kt * F::GS, full(s));
-        for (int m = 0; m < p.M; ++m)
-          bulk_copy_g2s(st + p.off_x + m * p.x_stride, p.X + static_cast<size_t>(m) * p.K + kt * F::KS, valid * 2,
-                        full(s));
+      if (BITS != 2) ptx::tma_prefetch_desc(&tm_b);
+    }
+    if (p.overlap) {
+      // The weights do not depend on the previous grid: put the first stages
+      // in flight before waiting for it. (The TMA unit takes copies in issue
+      // order, so the activation copies then queue behind all of them.)
+      if (lane == 0)
+        for (int t = 0; t < pre; ++t) load_weights(t, t);
+      griddep_launch_dependents();
+      griddep_wait();  // the activations may be the previous grid's output
+      __syncwarp();  // the transaction counts are raised before any activation copy can land
+      for (int t = 0; t < pre; ++t) load_x(t, t);
+    } else {
+      // Nothing to wait for: each stage's activations right behind its weights,
+      // so that the first stage is complete as early as possible.
+      for (int t = 0; t < pre; ++t) {
+        if (lane == 0) load_weights(t, t);
+        __syncwarp();
+        load_x(t, t);
       }
-      // Let every copy this thread issued land before the ring is reused.
+    }
+    int t = pre;
+    for (; t < p.num_stages; ++t) {
+      const int s = t % p.ring;
+      if (!warp_wait(empty(s), ((t / p.ring) & 1) ^ 1, lim, abort_flag)) {
+        if (lane == 0) give_up();
+        break;
+      }
+      if (lane == 0) load_weights(t, s);
+      __syncwarp();
+      load_x(t, s);
+    }
+    // Let every copy issued above land before the block can exit.
+    if (lane == 0) {
       const int first = t > p.ring ? t - p.ring : 0;
       for (int i = first; i < t; ++i) ptx::mbar_wait(full(i % p.ring), (i / p.ring) & 1, lim, nullptr);
     }
   } else {
     // ---------------- consumers ----------------
-    const int gs = warp % F::GS;                   // group of the stage this warp takes
-    const int half = 0;                            // every warp takes all of the CTA's pairs
-    for (int t = (warp / F::GS) % F::NSETS; t < p.num_stages; t += F::NSETS) {
+    griddep_launch_dependents();
+    const int gl = warp % GROUP_LANES;  // group lane: groups gl, gl + GROUP_LANES, ... of every stage
+    const int q0 = (warp / GROUP_LANES) * NPH;  // first 16-row pair of this warp's half
+    for (int t = 0; t < p.num_stages; ++t) {
       const int s = t % p.ring;
       if (!warp_wait(full(s), (t / p.ring) & 1, lim, abort_flag)) {
         if (lane == 0) give_up();
@@ -241,25 +308,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       const uint8_t* st = smem + s * p.stage_bytes;
       const int kt = (t + rot) % p.num_stages;
-      if (kt * F::KS + gs * F::G < p.K) {
+#pragma unroll
+      for (int gi = 0; gi < GPL; ++gi) {
+        const int gs = gl + GROUP_LANES * gi;
+        if (kt * F::KS + gs * F::G >= p.K) break;
         // activations of this group (the B operand): tokens g and g + 8,
         // k = gs*G + 16*step + 4c .. +3
         const uint8_t* xg = st + p.off_x + g * p.x_stride + (gs * F::G + 4 * c) * 2;
         const bool ga = g < p.M, gb = MT > 8 && g + 8 < p.M;
         float xs[TH][4];  // sum of x over the group per token (affine)
-        float tmp[PPW][TH][4];
+        float tmp[NPH][TH][4];
 #pragma unroll
         for (int h = 0; h < TH; ++h)
 #pragma unroll
           for (int j = 0; j < 4; ++j) xs[h][j] = 0.f;
 #pragma unroll
-        for (int q = 0; q < PPW; ++q)
+        for (int q = 0; q < NPH; ++q)
 #pragma unroll
           for (int h = 0; h < TH; ++h)
 #pragma unroll
             for (int j = 0; j < 4; ++j) tmp[q][h][j] = 0.f;
-        // weight row 16 * (half * PPW + q) + g of this warp's pair q
-        const uint8_t* rowg = st + (16 * half * PPW + g) * ROW_BYTES_PER_STAGE;
 #pragma unroll
         for (int k = 0; k < STEPS; ++k) {
           const uint2 x0 = ga ? *reinterpret_cast<const uint2*>(xg + 32 * k) : make_uint2(0u, 0u);
@@ -269,12 +337,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mma_bf16_16816(xs[0], ones, x0.x, x0.y);
             if constexpr (TH > 1) mma_bf16_16816(xs[TH - 1], ones, x1.x, x1.y);
           }
-          const int wo = word_offset<BITS>(gs, k, c, g);  // rows g and g + 8 share the swizzle
+          const int wo = word_offset<BITS>(gs, k, c);
 #pragma unroll
-          for (int q = 0; q < PPW; ++q) {
-            const uint8_t* r0 = rowg + q * 16 * ROW_BYTES_PER_STAGE;
-            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(r0 + wo);
-            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(r0 + 8 * ROW_BYTES_PER_STAGE + wo);
+          for (int q = 0; q < NPH; ++q) {
+            // rows 16q + g and 16q + g + 8 share the swizzle phase (row % 8 = g)
+            const int r0 = 16 * (q0 + q) + g;
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(st + phys_offset(wo, r0, R, U));
+            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(st + phys_offset(wo, r0 + 8, R, U));
             uint32_t a[4];
             decode_word<BITS>(w0, c, a[0], a[2]);  // row g: k pairs (4c, 4c+1), (4c+2, 4c+3)
             decode_word<BITS>(w1, c, a[1], a[3]);  // row g + 8
@@ -286,29 +355,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint16_t* sc = reinterpret_cast<const uint16_t*>(st + p.off_s) + gs * R;
         const uint16_t* bi = reinterpret_cast<const uint16_t*>(st + p.off_b) + gs * R;
 #pragma unroll
-        for (int q = 0; q < PPW; ++q) {
-          {
-            const int r0 = 16 * (half * PPW + q) + g;
-            const float s2[2] = {deq::h2f(sc[r0]), deq::h2f(sc[r0 + 8])};
-            float b2[2] = {0.f, 0.f};
-            if constexpr (BITS != 2) {
-              b2[0] = deq::h2f(bi[r0]);
-              b2[1] = deq::h2f(bi[r0 + 8]);
-            }
-#pragma unroll
-            for (int h = 0; h < TH; ++h)
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const float sj = s2[j >> 1];
-                if constexpr (BITS == 2) {
-                  acc[q][h][j] = fmaf(0.5f * sj, tmp[q][h][j], acc[q][h][j]);
-                } else {
-                  const float d = BITS == 4 ? fmaf(-128.f, xs[h][j], tmp[q][h][j]) : tmp[q][h][j];
-                  const float e = fmaf(b2[j >> 1], xs[h][j], acc[q][h][j]);
-                  acc[q][h][j] = fmaf(sj, d, e);
-                }
-              }
+        for (int q = 0; q < NPH; ++q) {
+          const int r0 = 16 * (q0 + q) + g;
+          const float s2[2] = {deq::h2f(sc[r0]), deq::h2f(sc[r0 + 8])};
+          float b2[2] = {0.f, 0.f};
+          if constexpr (BITS != 2) {
+            b2[0] = deq::h2f(bi[r0]);
+            b2[1] = deq::h2f(bi[r0 + 8]);
           }
+#pragma unroll
+          for (int h = 0; h < TH; ++h)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float sj = s2[j >> 1];
+              if constexpr (BITS == 2) {
+                acc[q][h][j] = fmaf(0.5f * sj, tmp[q][h][j], acc[q][h][j]);
+              } else {
+                const float d = BITS == 4 ? fmaf(-128.f, xs[h][j], tmp[q][h][j]) : tmp[q][h][j];
+                const float e = fmaf(b2[j >> 1], xs[h][j], acc[q][h][j]);
+                acc[q][h][j] = fmaf(sj, d, e);
+              }
+            }
         }
       }
       __syncwarp();
@@ -317,33 +384,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 
   // ---------------- the warps' partial sums meet in shared memory ----------------
+  griddep_wait();   // the previous grid is done before this one writes the output or reads the bias
   __syncthreads();  // the ring is drained: reuse it
-  float4* red = reinterpret_cast<float4*>(smem);  // [warp][pair of the warp][token half][lane]
+  float* red = reinterpret_cast<float*>(smem);  // [group lane][token][NLP]
   if (warp < NUM_CONSUMER_WARPS) {
+    const int gl = warp % GROUP_LANES, q0 = (warp / GROUP_LANES) * NPH;
 #pragma unroll
-    for (int q = 0; q < PPW; ++q)
+    for (int q = 0; q < NPH; ++q)
 #pragma unroll
-        for (int h = 0; h < TH; ++h)
-          red[((warp * PPW + q) * TH + h) * 32 + lane] =
-              make_float4(acc[q][h][0], acc[q][h][1], acc[q][h][2], acc[q][h][3]);
+      for (int h = 0; h < TH; ++h)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int m = 8 * h + 2 * c + (j & 1), nl = 16 * (q0 + q) + g + 8 * (j >> 1);
+          red[(gl * MT + m) * NLP + nl] = acc[q][h][j];
+        }
   }
   __syncthreads();
-  const int rows = 8 * nb;
-  for (int i = threadIdx.x; i < p.M * rows; i += NUM_THREADS) {
-    const int m = i / rows, nl = i % rows;
-    const int q = nl >> 4, hrow = (nl >> 3) & 1, gg = nl & 7;
-    const int h = m >> 3, cc = (m & 7) >> 1;
-    const int j = 2 * hrow + (m & 1);
-    const int ln = 4 * gg + cc;
-    float v = 0.f;
-    const int wh = q / PPW, ql = q % PPW;  // the warps holding pair q: those of half wh
-    constexpr int WPH = NUM_CONSUMER_WARPS;
-#pragma unroll
-    for (int w = wh * WPH; w < (wh + 1) * WPH; ++w) {
-      const float4 f = red[((w * PPW + ql) * TH + h) * 32 + ln];
-      v += j == 0 ? f.x : j == 1 ? f.y : j == 2 ? f.z : f.w;
-    }
+  for (int i = threadIdx.x; i < p.M * R; i += NUM_THREADS) {
+    const int m = i / R, nl = i - m * R;
     const int n = n0 + nl;
+    if (n >= p.N) continue;
+    float v = 0.f;
+#pragma unroll
+    for (int l = 0; l < GROUP_LANES; ++l) v += red[(l * MT + m) * NLP + nl];
     if (p.bias) v += __bfloat162float(__ushort_as_bfloat16(p.bias[n]));
     p.out[static_cast<size_t>(m) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
   }
@@ -352,15 +415,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-constexpr int kMaxSmem = 232448;
-
-template <int BITS, int MT>
-int launch_fmt(const Problem& pr, int nsm) {
+template <int BITS, int MT, int NP>
+int launch_fmt(const Problem& pr, int grid) {
   using F = Fmt<BITS>;
+  constexpr int R = 16 * NP;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(small_m_kernel<BITS, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    attr_err =
+        cudaFuncSetAttribute(small_m_kernel<BITS, MT, NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_LIMIT);
   });
   int st = cuda_check(attr_err, "cudaFuncSetAttribute(small_m_kernel)");
   if (st != QGEMM_OK) return st;
@@ -372,58 +435,90 @@ int launch_fmt(const Problem& pr, int nsm) {
   kp.M = pr.M;
   kp.N = pr.N;
   kp.K = pr.K;
-  const int nblocks = pr.N / 8;
-  int bpc = (nblocks + nsm - 1) / nsm;
-  bpc = bpc < NBMAX ? bpc : NBMAX;
-  const int grid = (nblocks + bpc - 1) / bpc;
-  const int R = 8 * bpc;
-  kp.bpc = bpc;
   kp.num_stages = (pr.K + F::KS - 1) / F::KS;
-  const int sb = F::GS * R * 2;
+  const uint64_t wbytes = static_cast<uint64_t>(pr.K) * BITS / 8;  // packed bytes per weight row
+  kp.unit = wbytes % 128 == 0 ? 128 : wbytes % 64 == 0 ? 64 : 32;  // K % 128 == 0 makes it at least 32
+  if (F::ROWB % kp.unit) return fail(QGEMM_ERR_UNSUPPORTED, "internal: small-M stage is not whole row pieces");
+  const int sb = GS * R * 2;
   // TMA tile destinations start on 128-byte boundaries (the packed box on a
-  // 1024-byte one, for its 128-byte swizzle); bulk copies need 16 bytes.
-  const int rows_read = R > 16 * NPMAX ? R : 16 * NPMAX;  // rows the consumers touch
-  kp.off_s = rows_read * ROW_BYTES_PER_STAGE;
+  // 1024-byte one, for its swizzle); bulk copies need 16 bytes.
+  kp.off_s = R * F::ROWB;
   kp.off_b = (kp.off_s + sb + 127) & ~127;
   kp.off_x = (kp.off_b + (BITS == 2 ? 0 : sb) + 127) & ~127;
-  kp.x_stride = F::KS * 2 + 16;  // +16 B staggers rows across banks
+  kp.x_stride = F::KS * 2 + 32;  // +32 B: token rows 8 banks apart, so the 8-byte B fetches do not collide
   kp.stage_bytes = (kp.off_x + pr.M * kp.x_stride + 1023) & ~1023;
   int ring = RING_BUDGET / kp.stage_bytes;
   ring = ring < MAX_STAGES ? ring : MAX_STAGES;
   ring = ring < kp.num_stages ? ring : kp.num_stages;
   kp.ring = ring < 1 ? 1 : ring;
-  const int red_bytes = NUM_CONSUMER_WARPS * PPW * 2 * 32 * 16;
-  const int data_bytes = kp.ring * kp.stage_bytes > red_bytes ? kp.ring * kp.stage_bytes : red_bytes;
-  const int smem = data_bytes + 16 * MAX_STAGES + 16 + 1024;
-  if (smem > kMaxSmem) return fail(QGEMM_ERR_UNSUPPORTED, "small-M stage of %d bytes does not fit", kp.stage_bytes);
-  if (kp.off_s % 128 || kp.off_b % 128 || kp.off_x % 16 || kp.x_stride % 16 || kp.stage_bytes % 1024)
+  const int red_bytes = NUM_CONSUMER_WARPS / split_rows(MT, NP) * MT * (R + 4) * 4;
+  kp.data_bytes = kp.ring * kp.stage_bytes > red_bytes ? kp.ring * kp.stage_bytes : red_bytes;
+  if (kp.data_bytes < SMEM_FLOOR) kp.data_bytes = SMEM_FLOOR;
+  const int smem = kp.data_bytes + 16 * MAX_STAGES + 16;
+  if (smem > SMEM_LIMIT) return fail(QGEMM_ERR_UNSUPPORTED, "small-M stage of %d bytes does not fit", kp.stage_bytes);
+  if (kp.off_s % 1024 || kp.off_b % 128 || kp.off_x % 128 || kp.x_stride % 16 || kp.stage_bytes % 1024 ||
+      kp.data_bytes % 8)
     return fail(QGEMM_ERR_UNSUPPORTED, "internal: small-M stage layout misaligned");
   kp.wait_limit_ns = wait_limit_ns();
   if ((st = status_word(&kp.status)) != QGEMM_OK) return st;
 
   CUtensorMap tm_w, tm_s, tm_b;
-  const uint64_t wbytes = static_cast<uint64_t>(pr.K) * BITS / 8;
   const uint64_t groups = static_cast<uint64_t>(pr.K) / F::G;
-  if ((st = make_tensor_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.packed, wbytes, pr.N, wbytes,
-                               ROW_BYTES_PER_STAGE, R, CU_TENSOR_MAP_SWIZZLE_128B, "W")) != QGEMM_OK)
+  // packed codes as [row][piece][U bytes]; the box is U bytes x R rows x the stage's pieces
+  const uint64_t wdims[3] = {static_cast<uint64_t>(kp.unit), static_cast<uint64_t>(pr.N), wbytes / kp.unit};
+  const uint64_t wstrides[2] = {wbytes, static_cast<uint64_t>(kp.unit)};
+  const uint32_t wbox[3] = {static_cast<uint32_t>(kp.unit), static_cast<uint32_t>(R),
+                            static_cast<uint32_t>(F::ROWB / kp.unit)};
+  const CUtensorMapSwizzle wswz = kp.unit == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : kp.unit == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
+  if ((st = make_tensor_map_3d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.packed, wdims, wstrides, wbox, wswz, "W")) !=
+      QGEMM_OK)
     return st;
   if ((st = make_tensor_map_2d(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.scales, pr.N, groups,
-                               uint64_t(pr.N) * 2, R, F::GS, CU_TENSOR_MAP_SWIZZLE_NONE, "scales")) != QGEMM_OK)
+                               uint64_t(pr.N) * 2, R, GS, CU_TENSOR_MAP_SWIZZLE_NONE, "scales")) != QGEMM_OK)
     return st;
   if (BITS != 2) {
     if ((st = make_tensor_map_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.biases, pr.N, groups,
-                                 uint64_t(pr.N) * 2, R, F::GS, CU_TENSOR_MAP_SWIZZLE_NONE, "biases")) != QGEMM_OK)
+                                 uint64_t(pr.N) * 2, R, GS, CU_TENSOR_MAP_SWIZZLE_NONE, "biases")) != QGEMM_OK)
       return st;
   } else {
     tm_b = tm_s;  // unused for ternary
   }
-  small_m_kernel<BITS, MT><<<grid, NUM_THREADS, smem, pr.stream>>>(tm_w, tm_s, tm_b, kp);
-  return cuda_check(cudaGetLastError(), "small_m_kernel launch");
+  kp.overlap = pr.overlap ? 1 : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = pr.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pr.overlap ? 1 : 0;
+  return cuda_check(cudaLaunchKernelEx(&cfg, small_m_kernel<BITS, MT, NP>, tm_w, tm_s, tm_b, kp),
+                    "small_m_kernel launch");
+}
+
+// Rows per CTA: the fewest 16-row pairs (from the compiled set) that cover N
+// with at most one CTA per SM.
+template <int BITS, int MT>
+int launch_rows(const Problem& pr, int nsm) {
+  const int pairs = pr.N / 16;
+  const int need = (pairs + nsm - 1) / nsm;
+  const int np = need <= 2 ? 2 : need <= 4 ? 4 : need <= 6 ? 6 : 8;
+  const int grid = (pairs + np - 1) / np;
+  switch (np) {
+    case 2: return launch_fmt<BITS, MT, 2>(pr, grid);
+    case 4: return launch_fmt<BITS, MT, 4>(pr, grid);
+    case 6: return launch_fmt<BITS, MT, 6>(pr, grid);
+    default: return launch_fmt<BITS, MT, 8>(pr, grid);
+  }
 }
 
 template <int BITS>
 int launch_bits(const Problem& pr, int nsm) {
-  return pr.M <= 8 ? launch_fmt<BITS, 8>(pr, nsm) : launch_fmt<BITS, 16>(pr, nsm);
+  return pr.M <= 8 ? launch_rows<BITS, 8>(pr, nsm) : launch_rows<BITS, 16>(pr, nsm);
 }
 
 }  // namespace sm
