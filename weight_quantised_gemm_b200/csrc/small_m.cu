@@ -93,7 +93,7 @@ struct Params {
   int M, N, K;
   int num_stages;        // ceil(K / KS)
   int ring;              // ring depth
-  int unit;              // U: bytes per swizzled row piece (128, 64 or 32)
+  int unit_shift;        // log2 of U, the bytes per swizzled row piece (128, 64 or 32)
   int stage_bytes;       // bytes per ring stage (multiple of 1024)
   int data_bytes;        // ring (or the partial sums, if larger); the mbarriers follow
   int off_s, off_b, off_x, x_stride;  // offsets inside a stage; activation row stride in bytes
@@ -134,14 +134,19 @@ __device__ __forceinline__ int word_offset(int gs, int k, int c) {
   else return gs * GB + 16 * k + 4 * c;
 }
 
-// Physical byte offset in the stage of logical byte `off` of row r: the box
-// lands as [off / U][row][U bytes], each U-byte row piece swizzled by the TMA
-// (16-byte unit index XORed with address bits 7.. of the piece).
-__device__ __forceinline__ int phys_offset(int off, int r, int R, int U) {
-  const int plane = off / U, o = off - plane * U;
-  const int x = r * U + o;  // offset inside the plane; planes start on the swizzle period
-  const int mask = U == 128 ? 7 : U == 64 ? 3 : 1;
-  return plane * R * U + (x ^ (((x >> 7) & mask) << 4));
+// The box lands as [off / U][row][U bytes] (U = 2^ush), each U-byte row piece
+// swizzled by the TMA: the 16-byte unit index of byte x of a plane is XORed
+// with x's bits from 7 up (3, 2 or 1 of them). For row r that key is
+// (r >> (7 - ush)) & (U / 16 - 1), which for rows 16q + g and 16q + g + 8 is
+// the same function of g alone; so the physical offset of logical byte `off`
+// of row r splits into a per-step part and a per-row part:
+//   piece_offset(off) + (r << ush).
+__device__ __forceinline__ int swizzle_key16(int g, int ush) {
+  return ((g >> (7 - ush)) & ((1 << (ush - 4)) - 1)) << 4;
+}
+template <int R>
+__device__ __forceinline__ int piece_offset(int off, int ush, int key16) {
+  return ((off >> ush) * R << ush) + ((off & ((1 << ush) - 1)) ^ key16);
 }
 
 // B operand of one step for quad thread c from its word: codes 4c .. 4c+3 as
@@ -193,7 +198,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   const int n0 = blockIdx.x * R;
-  const int U = p.unit;
+  const int U = 1 << p.unit_shift;
 
   const uint32_t bar0 = sbase + p.data_bytes;
   auto full = [&](int s) { return bar0 + 8u * s; };
@@ -298,6 +303,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ---------------- consumers ----------------
     griddep_launch_dependents();
+    const int ush = p.unit_shift;
+    const int key16 = swizzle_key16(g, ush);
     const int gl = warp % GROUP_LANES;  // group lane: groups gl, gl + GROUP_LANES, ... of every stage
     const int q0 = (warp / GROUP_LANES) * NPH;  // first 16-row pair of this warp's half
     for (int t = 0; t < p.num_stages; ++t) {
@@ -337,13 +344,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mma_bf16_16816(xs[0], ones, x0.x, x0.y);
             if constexpr (TH > 1) mma_bf16_16816(xs[TH - 1], ones, x1.x, x1.y);
           }
-          const int wo = word_offset<BITS>(gs, k, c);
+          const uint8_t* wk = st + piece_offset<R>(word_offset<BITS>(gs, k, c), ush, key16);
 #pragma unroll
           for (int q = 0; q < NPH; ++q) {
-            // rows 16q + g and 16q + g + 8 share the swizzle phase (row % 8 = g)
+            // rows 16q + g and 16q + g + 8 share the swizzle key
             const int r0 = 16 * (q0 + q) + g;
-            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(st + phys_offset(wo, r0, R, U));
-            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(st + phys_offset(wo, r0 + 8, R, U));
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(wk + (r0 << ush));
+            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(wk + ((r0 + 8) << ush));
             uint32_t a[4];
             decode_word<BITS>(w0, c, a[0], a[2]);  // row g: k pairs (4c, 4c+1), (4c+2, 4c+3)
             decode_word<BITS>(w1, c, a[1], a[3]);  // row g + 8
@@ -437,8 +444,9 @@ int launch_fmt(const Problem& pr, int grid) {
   kp.K = pr.K;
   kp.num_stages = (pr.K + F::KS - 1) / F::KS;
   const uint64_t wbytes = static_cast<uint64_t>(pr.K) * BITS / 8;  // packed bytes per weight row
-  kp.unit = wbytes % 128 == 0 ? 128 : wbytes % 64 == 0 ? 64 : 32;  // K % 128 == 0 makes it at least 32
-  if (F::ROWB % kp.unit) return fail(QGEMM_ERR_UNSUPPORTED, "internal: small-M stage is not whole row pieces");
+  const int unit = wbytes % 128 == 0 ? 128 : wbytes % 64 == 0 ? 64 : 32;  // K % 128 == 0 makes it at least 32
+  kp.unit_shift = unit == 128 ? 7 : unit == 64 ? 6 : 5;
+  if (F::ROWB % unit) return fail(QGEMM_ERR_UNSUPPORTED, "internal: small-M stage is not whole row pieces");
   const int sb = GS * R * 2;
   // TMA tile destinations start on 128-byte boundaries (the packed box on a
   // 1024-byte one, for its swizzle); bulk copies need 16 bytes.
@@ -465,12 +473,12 @@ int launch_fmt(const Problem& pr, int grid) {
   CUtensorMap tm_w, tm_s, tm_b;
   const uint64_t groups = static_cast<uint64_t>(pr.K) / F::G;
   // packed codes as [row][piece][U bytes]; the box is U bytes x R rows x the stage's pieces
-  const uint64_t wdims[3] = {static_cast<uint64_t>(kp.unit), static_cast<uint64_t>(pr.N), wbytes / kp.unit};
-  const uint64_t wstrides[2] = {wbytes, static_cast<uint64_t>(kp.unit)};
-  const uint32_t wbox[3] = {static_cast<uint32_t>(kp.unit), static_cast<uint32_t>(R),
-                            static_cast<uint32_t>(F::ROWB / kp.unit)};
-  const CUtensorMapSwizzle wswz = kp.unit == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
-                                  : kp.unit == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+  const uint64_t wdims[3] = {static_cast<uint64_t>(unit), static_cast<uint64_t>(pr.N), wbytes / unit};
+  const uint64_t wstrides[2] = {wbytes, static_cast<uint64_t>(unit)};
+  const uint32_t wbox[3] = {static_cast<uint32_t>(unit), static_cast<uint32_t>(R),
+                            static_cast<uint32_t>(F::ROWB / unit)};
+  const CUtensorMapSwizzle wswz = unit == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : unit == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                   : CU_TENSOR_MAP_SWIZZLE_32B;
   if ((st = make_tensor_map_3d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.packed, wdims, wstrides, wbox, wswz, "W")) !=
       QGEMM_OK)
