@@ -335,6 +335,15 @@ def sweep(peaks):
         wl = WL.workload(cid)
         for li, lin in enumerate(wl.linears):
             entry, sets, host = one(cid, li, lin, lin.M, wq.QGEMM_PATH_AUTO, 100 if lin.M <= 16 else 20)
+            if lin.M > 16 and cid in (1, 2, 4):
+                # context: dense bf16 torch.matmul (cuBLAS) at the same shape, same graph timing
+                Xd0 = sets[0][0]
+                Wb = torch.from_numpy(host[1]).cuda().to(torch.bfloat16)
+                ob = torch.empty((lin.M, lin.N), dtype=torch.bfloat16, device="cuda")
+                td = time_graph([lambda: torch.matmul(Xd0, Wb.T, out=ob)] * 10)
+                entry["dense_bf16_torch_us"] = round(td * 1e6, 2)
+                entry["dense_bf16_torch_tflops"] = round(2 * lin.M * lin.N * lin.K / td / 1e12, 1)
+                del Wb, ob
             if cid == 4:
                 Xd, dw, bd, out = sets[0]
                 X, W, bias, pw = host
@@ -610,6 +619,26 @@ def cpu_oracle_sample(target_s: float, lin=None, cid=HEADLINE_CID, li=HEADLINE_L
     return flops / t_full / 1e12, spent, desc, rows
 
 
+def cpu_oracle_single_core():
+    """The oracle on one host core for config 0 (tiny) and config 3 at M=1
+    (ternary decode): seconds per GEMM, dequantisation included."""
+    from threadpoolctl import threadpool_limits
+
+    import oracle as O
+    import workloads as WL
+    out = {}
+    with threadpool_limits(limits=1):
+        for cid, li in ((0, 0), (3, 0)):
+            lin = WL.workload(cid).linears[li]
+            X, W, bias = WL.make_inputs(lin, cid, li)
+            p, s, b = O.pack_ref(W, lin.bits, lin.group)
+            t0 = time.perf_counter()
+            O.qgemm_ref(X, p, s, b, lin.bits, lin.group, lin.K, bias)
+            t = time.perf_counter() - t0
+            out[f"{cid}:{lin.name}"] = {"seconds": round(t, 4), "gflops": round(2 * lin.M * lin.N * lin.K / t / 1e9, 3)}
+    return out
+
+
 def run_reference(args, rank, world):
     """The base contract's reference arm, here the oracle on the host cores:
     each step is a bounded sample of the headline workload."""
@@ -711,6 +740,7 @@ def main(argv=None):
                 v, spent, desc, _ = cpu_oracle_sample(args.cpu_seconds)
                 res["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOP/s", "cores": blas_threads(),
                                        "kind": "oracle", "sample": desc, "seconds": round(spent, 2)}
+                res["cpu_oracle_single_core"] = cpu_oracle_single_core()
             res["peaks"] = peaks
             print(json.dumps(res), flush=True)
     finally:
