@@ -296,6 +296,45 @@ def dense_ref(X_bits, W, bias_bits=None) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------
+# fused epilogues: the elementwise steps on either side of a FLUX block's
+# linears (stable-diffusion.rs README, introduction: the layers "that multiply
+# the residual stream"). The pages give no formula; the readings are FLUX's
+# own: the MLP's up projection is followed by the tanh-approximate GELU, and a
+# residual-writing linear's output y updates the stream as r + gate * y with
+# one gate value per output feature.
+# ----------------------------------------------------------------------------
+
+EPI_NONE, EPI_GELU_TANH, EPI_RESIDUAL_GATE = 0, 1, 2
+
+
+def gelu_tanh_ref(y) -> np.ndarray:
+    """0.5 y (1 + tanh(sqrt(2 / pi) (y + 0.044715 y^3))), in fp64."""
+    y = np.asarray(y, dtype=np.float64)
+    return 0.5 * y * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (y + 0.044715 * y ** 3)))
+
+
+def epilogue_ref(y, op: int, residual_bits=None, gate_bits=None) -> np.ndarray:
+    """Applies the fused epilogue to y = X . Wq^T (+ bias), all in fp64."""
+    y = np.asarray(y, dtype=np.float64)
+    if op == EPI_NONE:
+        return y
+    if op == EPI_GELU_TANH:
+        return gelu_tanh_ref(y)
+    if op == EPI_RESIDUAL_GATE:
+        r = bf16_bits_to_f64(residual_bits)
+        g = bf16_bits_to_f64(gate_bits)
+        return r + g[None, :] * y
+    raise ValueError(f"unknown epilogue {op}")
+
+
+def qgemm_ref_epilogue(X_bits, packed, scales, biases, bits: int, group: int, K: int, bias_bits, op: int,
+                       residual_bits=None, gate_bits=None) -> np.ndarray:
+    """fp64 epilogue(X . Wq_exact^T (+ bias)): the reference of the fused calls."""
+    y = qgemm_ref(X_bits, packed, scales, biases, bits, group, K, bias_bits)
+    return epilogue_ref(y, op, residual_bits, gate_bits)
+
+
+# ----------------------------------------------------------------------------
 # error metrics
 # ----------------------------------------------------------------------------
 

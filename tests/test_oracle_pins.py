@@ -389,3 +389,67 @@ def test_cosine_against_dense_matches_rtn_noise_model(bits, expect):
     X = WL.f32_to_bf16_bits(g.standard_normal((64, 1024)).astype(np.float32))
     cy = O.cosine(O.qgemm_ref(X, packed, s, b, bits, 64, 1024), O.bf16_bits_to_f64(X) @ W.astype(np.float64).T)
     assert abs(cy - c) < 5 * (1 - c) + 1e-6
+
+
+# ----------------------------------------------------------------------------
+# fused epilogues
+# ----------------------------------------------------------------------------
+
+def test_gelu_tanh_matches_torch_and_its_identities():
+    """Against torch's tanh-approximate GELU in fp64 (a library routine), at 0,
+    far in both tails, and through the identity gelu(y) - gelu(-y) = y that
+    the tanh form satisfies exactly."""
+    y = np.concatenate([np.linspace(-12, 12, 4001), np.array([-1e3, -40.0, 0.0, 40.0, 1e3])])
+    ref = torch.nn.functional.gelu(torch.from_numpy(y), approximate="tanh").numpy()
+    got = O.gelu_tanh_ref(y)
+    # fp64 rounding order differs only where 1 + tanh cancels (|difference| < 1e-15)
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-14)
+    assert O.gelu_tanh_ref(0.0) == 0.0
+    assert abs(O.gelu_tanh_ref(20.0) - 20.0) < 1e-12 and abs(O.gelu_tanh_ref(-20.0)) < 1e-12
+    assert np.allclose(O.gelu_tanh_ref(y) - O.gelu_tanh_ref(-y), y, rtol=1e-12, atol=1e-12)
+    # the constant inside the tanh: the slope at 0 is 1/2, the curvature sqrt(2/pi)
+    h = 1e-5
+    assert abs((O.gelu_tanh_ref(h) - O.gelu_tanh_ref(-h)) / (2 * h) - 0.5) < 1e-9
+    second = (O.gelu_tanh_ref(h) - 2 * O.gelu_tanh_ref(0.0) + O.gelu_tanh_ref(-h)) / h ** 2
+    assert abs(second - math.sqrt(2 / math.pi)) < 1e-4
+
+
+def test_residual_gate_epilogue_special_cases():
+    """gate = 0 gives the residual exactly; residual 0 and gate 1 give y; the
+    update is linear in the gate; and one hand-computed element."""
+    rng = np.random.default_rng(3)
+    y = rng.standard_normal((5, 8))
+    r_bits = WL.f32_to_bf16_bits(rng.standard_normal((5, 8)).astype(np.float32))
+    zeros, ones = (WL.f32_to_bf16_bits(np.full(8, v, np.float32)) for v in (0.0, 1.0))
+    r = O.bf16_bits_to_f64(r_bits)
+    assert np.array_equal(O.epilogue_ref(y, O.EPI_RESIDUAL_GATE, r_bits, zeros), r)
+    assert np.array_equal(O.epilogue_ref(y, O.EPI_RESIDUAL_GATE, WL.f32_to_bf16_bits(np.zeros((5, 8), np.float32)),
+                                         ones), y)
+    g1 = WL.f32_to_bf16_bits(rng.standard_normal(8).astype(np.float32))
+    g2 = WL.f32_to_bf16_bits(rng.standard_normal(8).astype(np.float32))
+    g12 = WL.f32_to_bf16_bits((O.bf16_bits_to_f64(g1) + O.bf16_bits_to_f64(g2)).astype(np.float32))
+    if np.array_equal(O.bf16_bits_to_f64(g12), O.bf16_bits_to_f64(g1) + O.bf16_bits_to_f64(g2)):
+        lhs = O.epilogue_ref(y, O.EPI_RESIDUAL_GATE, r_bits, g12) - r
+        rhs = (O.epilogue_ref(y, O.EPI_RESIDUAL_GATE, r_bits, g1) - r) + \
+              (O.epilogue_ref(y, O.EPI_RESIDUAL_GATE, r_bits, g2) - r)
+        assert np.allclose(lhs, rhs, rtol=1e-12, atol=1e-12)
+    # out[0, 0] = r + g * y with r = 1.5, g = -0.25, y = 2: 1.0
+    rr = WL.f32_to_bf16_bits(np.array([[1.5]], np.float32))
+    gg = WL.f32_to_bf16_bits(np.array([-0.25], np.float32))
+    assert O.epilogue_ref(np.array([[2.0]]), O.EPI_RESIDUAL_GATE, rr, gg)[0, 0] == 1.0
+    # the gate indexes features (columns), not tokens
+    gcol = WL.f32_to_bf16_bits(np.arange(8, dtype=np.float32))
+    out = O.epilogue_ref(np.ones((5, 8)), O.EPI_RESIDUAL_GATE, WL.f32_to_bf16_bits(np.zeros((5, 8), np.float32)),
+                         gcol)
+    assert np.array_equal(out, np.broadcast_to(np.arange(8.0), (5, 8)))
+
+
+def test_fused_reference_composes_the_plain_gemm():
+    """qgemm_ref_epilogue is the plain reference followed by the epilogue."""
+    X, W, bias = WL.random_case(41, 6, 64, 128, 4, with_bias=True)
+    p, s, b = O.pack_ref(W, 4, 64)
+    y = O.qgemm_ref(X, p, s, b, 4, 64, 128, bias)
+    assert np.array_equal(O.qgemm_ref_epilogue(X, p, s, b, 4, 64, 128, bias, O.EPI_NONE), y)
+    assert np.array_equal(O.qgemm_ref_epilogue(X, p, s, b, 4, 64, 128, bias, O.EPI_GELU_TANH), O.gelu_tanh_ref(y))
+    with pytest.raises(ValueError):
+        O.epilogue_ref(y, 7)
