@@ -619,6 +619,46 @@ def cpu_oracle_sample(target_s: float, lin=None, cid=HEADLINE_CID, li=HEADLINE_L
     return flops / t_full / 1e12, spent, desc, rows
 
 
+def fused_sweep():
+    """The fused epilogues on the FLUX shapes they serve, against the unfused
+    sequence (qgemm, then a torch elementwise kernel), both in CUDA graphs."""
+    import torch
+
+    import weight_quantised_gemm_b200 as wq
+    import workloads as WL
+    rows = []
+    cases = [(2, 0, wq.QGEMM_EPI_GELU_TANH), (4, 2, wq.QGEMM_EPI_RESIDUAL_GATE), (4, 4, wq.QGEMM_EPI_RESIDUAL_GATE)]
+    for cid, li, op in cases:
+        lin = WL.workload(cid).linears[li]
+        ab = alg_bytes(lin)
+        ncopy = copies_for(ab, 3)
+        sets, _ = make_device_inputs(lin, cid, li, ncopy)
+        g = torch.Generator(device="cuda").manual_seed(0)
+        res = [torch.randn((lin.M, lin.N), device="cuda", generator=g).to(torch.bfloat16) for _ in range(ncopy)]
+        gate = torch.randn((lin.N,), device="cuda", generator=g).to(torch.bfloat16)
+
+        def fused(i):
+            Xd, dw, bd, out = sets[i]
+            return lambda: wq.qgemm_fused(Xd, dw, op, bias=bd, residual=res[i], gate=gate, out=out)
+
+        def unfused(i):
+            Xd, dw, bd, out = sets[i]
+            if op == wq.QGEMM_EPI_GELU_TANH:
+                return lambda: torch.nn.functional.gelu(wq.qgemm(Xd, dw, bias=bd, out=out), approximate="tanh")
+            return lambda: torch.addcmul(res[i], gate, wq.qgemm(Xd, dw, bias=bd, out=out))
+
+        n = max(ncopy, 12)
+        tf = time_graph([fused(i % ncopy) for i in range(n)])
+        tu = time_graph([unfused(i % ncopy) for i in range(n)])
+        wq.check_device_status()
+        rows.append({"workload": cid, "linear": lin.name, "epilogue": {1: "gelu_tanh", 2: "residual_gate"}[op],
+                     "M": lin.M, "N": lin.N, "K": lin.K, "bits": lin.bits, "fused_us": round(tf * 1e6, 2),
+                     "unfused_us": round(tu * 1e6, 2), "saved_us": round((tu - tf) * 1e6, 2)})
+        del sets, res
+        torch.cuda.empty_cache()
+    return rows
+
+
 def cpu_oracle_single_core():
     """The oracle on one host core for config 0 (tiny) and config 3 at M=1
     (ternary decode): seconds per GEMM, dequantisation included."""
@@ -736,6 +776,7 @@ def main(argv=None):
                 res["sweep"] = per
                 res["workload4_block"] = block
                 res["path_crossover"] = cross
+                res["fused_epilogues"] = fused_sweep()
             if not args.no_cpu and world == 1:
                 v, spent, desc, _ = cpu_oracle_sample(args.cpu_seconds)
                 res["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOP/s", "cores": blas_threads(),

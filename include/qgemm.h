@@ -151,6 +151,32 @@ int qgemm(const void* X, int32_t M, const qgemm_weights* W, void* out,
 int qgemm_ex(const void* X, int32_t M, const qgemm_weights* W, void* out,
              const void* bias, int32_t path, void* stream);
 
+/* Fused epilogues for qgemm_fused: the elementwise steps on either side of a
+ * FLUX block's linears. The pages (stable-diffusion.rs README, introduction)
+ * name "the layers that multiply the residual stream" without formulas; these
+ * are FLUX's: the MLP up projection's tanh GELU, and a residual-writing
+ * layer's gated update of the residual stream. v = acc + bias in fp32; the
+ * result is rounded to bf16 once. */
+enum {
+  QGEMM_EPI_NONE = 0,          /* out = bf16(v) */
+  QGEMM_EPI_GELU_TANH = 1,     /* out = bf16(0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3)))) */
+  QGEMM_EPI_RESIDUAL_GATE = 2  /* out = bf16(residual + gate[n] * v) */
+};
+
+typedef struct qgemm_epilogue {
+  int32_t op;            /* QGEMM_EPI_* */
+  const void* residual;  /* QGEMM_EPI_RESIDUAL_GATE: device bf16 [M, N], 16-byte aligned; may equal out
+                            (in-place update of the residual stream) */
+  const void* gate;      /* QGEMM_EPI_RESIDUAL_GATE: device bf16 [N], one gate per output feature */
+} qgemm_epilogue;
+
+/* As qgemm_ex, with a fused epilogue (NULL or QGEMM_EPI_NONE: plain qgemm_ex).
+ * Errors: unknown op, or a missing or misaligned residual or gate, return
+ * QGEMM_ERR_INVALID_ARG / QGEMM_ERR_ALIGNMENT before anything is enqueued.
+ * No counterpart as an interface in the pages. */
+int qgemm_fused(const void* X, int32_t M, const qgemm_weights* W, void* out,
+                const void* bias, const qgemm_epilogue* epi, int32_t path, void* stream);
+
 /* The path qgemm would take for this shape: QGEMM_PATH_SMALL_M or
  * QGEMM_PATH_LARGE_M, or a negative qgemm_status for an invalid shape. */
 int qgemm_select_path(int32_t M, int32_t N, int32_t K, int32_t bits);

@@ -153,3 +153,23 @@ def test_missing_library_fails_loudly_on_first_call(tmp_path):
     r = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == "raised True"
+
+
+def _fused(desc, op, residual=0x40000, gate=0x50000, M=64, path=0):
+    epi = wq._Epilogue(op, residual, gate)
+    return wq._lib.qgemm_fused(0x10000, M, ctypes.byref(desc), 0x20000, None, ctypes.byref(epi), path, None)
+
+
+def test_fused_rejects_bad_epilogues_without_device():
+    d = _desc()
+    assert _fused(d, 3) == wq.QGEMM_ERR_INVALID_ARG
+    assert _fused(d, -1) == wq.QGEMM_ERR_INVALID_ARG
+    assert _fused(d, wq.QGEMM_EPI_RESIDUAL_GATE, residual=None) == wq.QGEMM_ERR_INVALID_ARG
+    assert _fused(d, wq.QGEMM_EPI_RESIDUAL_GATE, gate=None) == wq.QGEMM_ERR_INVALID_ARG
+    assert _fused(d, wq.QGEMM_EPI_RESIDUAL_GATE, residual=0x40008) == wq.QGEMM_ERR_ALIGNMENT
+    assert _fused(d, wq.QGEMM_EPI_RESIDUAL_GATE, gate=0x50001) == wq.QGEMM_ERR_ALIGNMENT
+    # valid descriptors with M = 0: a no-op that never touches the device
+    for op in (wq.QGEMM_EPI_NONE, wq.QGEMM_EPI_GELU_TANH, wq.QGEMM_EPI_RESIDUAL_GATE):
+        assert _fused(d, op, M=0) == wq.QGEMM_OK
+    # a NULL epilogue is plain qgemm_ex
+    assert wq._lib.qgemm_fused(0x10000, 0, ctypes.byref(d), 0x20000, None, None, 0, None) == wq.QGEMM_OK

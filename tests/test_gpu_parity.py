@@ -263,3 +263,70 @@ def test_overlap_after_a_torch_kernel_and_in_a_graph():
     wq.check_device_status()
     assert np.array_equal(from_dev_bf16(out), y_eager)
     del g
+
+
+# ----------------------------------------------------------------------------
+# fused epilogues (qgemm_fused): tanh GELU and the gated residual update
+# ----------------------------------------------------------------------------
+
+def _bf16_normal(seed, shape, scale=1.0):
+    g = np.random.default_rng(np.random.SeedSequence([7, seed] + list(shape)))
+    return WL.f32_to_bf16_bits((scale * g.standard_normal(shape)).astype(np.float32))
+
+
+def _fused_case(bits, M, N, K, op, seed, path, in_place=False):
+    X, W, bias = WL.random_case(seed, M, N, K, bits, with_bias=True)
+    r_bits, g_bits = _bf16_normal(seed, (M, N)), _bf16_normal(seed + 1, (N,))
+    dw = wq.qgemm_pack(W, bits).to_device()
+    Xd, bd = to_dev_bf16(X), to_dev_bf16(bias)
+    rd, gd = to_dev_bf16(r_bits), to_dev_bf16(g_bits)
+    out = rd if in_place else None
+    y = wq.qgemm_fused(Xd, dw, op, bias=bd, residual=rd, gate=gd, out=out, path=path)
+    wq.check_device_status()
+    group = wq.GROUP_OF_BITS[bits]
+    p, s, b = O.pack_ref(W, bits, group)
+    ref = O.qgemm_ref_epilogue(X, p, s, b, bits, group, K, bias, op, r_bits, g_bits)
+    return from_dev_bf16(y), ref
+
+
+@pytest.mark.parametrize("op", [wq.QGEMM_EPI_GELU_TANH, wq.QGEMM_EPI_RESIDUAL_GATE])
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("path,M", [(SMALL, 1), (SMALL, 13), (LARGE, 300)])
+def test_fused_epilogue_parity(op, bits, path, M):
+    y, ref = _fused_case(bits, M, 400, 640, op, 100 + 10 * op + bits + M, path)
+    _assert_close(y, ref, f"op={op} bits={bits} path={path} M={M}")
+
+
+@pytest.mark.parametrize("path,M", [(SMALL, 5), (LARGE, 257)])
+def test_fused_residual_update_in_place(path, M):
+    """out may be the residual itself: the same bits as the out-of-place call."""
+    y_out, ref = _fused_case(4, M, 528, 512, wq.QGEMM_EPI_RESIDUAL_GATE, 77, path)
+    y_in, _ = _fused_case(4, M, 528, 512, wq.QGEMM_EPI_RESIDUAL_GATE, 77, path, in_place=True)
+    assert np.array_equal(y_in, y_out)
+    _assert_close(y_in, ref, "in place")
+
+
+def test_fused_none_equals_plain_qgemm():
+    X, W, bias = WL.random_case(5, 300, 256, 512, 8, with_bias=True)
+    dw = wq.qgemm_pack(W, 8).to_device()
+    Xd, bd = to_dev_bf16(X), to_dev_bf16(bias)
+    for path in (SMALL, LARGE):
+        Xp = Xd[:16] if path == SMALL else Xd
+        a = wq.qgemm(Xp, dw, bias=bd, path=path)
+        b = wq.qgemm_fused(Xp, dw, wq.QGEMM_EPI_NONE, bias=bd, path=path)
+        wq.check_device_status()
+        assert torch.equal(a, b)
+
+
+def test_fused_gelu_mlp_up_full_size_sampled_rows():
+    """The MLP up projection of the FLUX workload with its GELU fused, checked
+    on sampled rows against the oracle."""
+    lin = WL.workload(2).linears[0]
+    X, W, bias = WL.make_inputs(lin, 2, 0)
+    dw = wq.qgemm_pack(W, lin.bits).to_device()
+    y = from_dev_bf16(wq.qgemm_fused(to_dev_bf16(X), dw, wq.QGEMM_EPI_GELU_TANH))
+    wq.check_device_status()
+    p, s, b = O.pack_ref(W, lin.bits, lin.group)
+    rows = np.arange(0, lin.M, 257)
+    ref = O.gelu_tanh_ref(O.qgemm_ref_rows(rows, X, p, s, b, lin.bits, lin.group, lin.K, None))
+    _assert_close(y[rows], ref, "mlp_up + gelu sampled rows")

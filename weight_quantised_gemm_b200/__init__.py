@@ -35,6 +35,10 @@ QGEMM_PATH_SMALL_M = 1
 QGEMM_PATH_LARGE_M = 2
 QGEMM_FLAG_OVERLAP_PREVIOUS = 0x100
 
+QGEMM_EPI_NONE = 0
+QGEMM_EPI_GELU_TANH = 1
+QGEMM_EPI_RESIDUAL_GATE = 2
+
 GROUP_OF_BITS = {2: 128, 4: 64, 8: 64}
 
 
@@ -42,6 +46,10 @@ class QGemmError(RuntimeError):
     def __init__(self, status: int, where: str, detail: str):
         self.status = status
         super().__init__(f"{where}: {qgemm_status_str(status)} ({status}): {detail}")
+
+
+class _Epilogue(ctypes.Structure):
+    _fields_ = [("op", ctypes.c_int32), ("residual", ctypes.c_void_p), ("gate", ctypes.c_void_p)]
 
 
 class _Weights(ctypes.Structure):
@@ -62,6 +70,7 @@ def _load():
         "qgemm_pack": (ctypes.c_int, [vp, i32, i32, i32, i32, vp, vp, vp]),
         "qgemm": (ctypes.c_int, [vp, i32, W, vp, vp, vp]),
         "qgemm_ex": (ctypes.c_int, [vp, i32, W, vp, vp, i32, vp]),
+        "qgemm_fused": (ctypes.c_int, [vp, i32, W, vp, vp, ctypes.POINTER(_Epilogue), i32, vp]),
         "qgemm_select_path": (ctypes.c_int, [i32, i32, i32, i32]),
         "qgemm_dequant_tile": (ctypes.c_int, [W, i32, i32, i32, i32, vp, vp]),
         "qgemm_get_device_status": (ctypes.c_int, [vp]),
@@ -89,7 +98,8 @@ class _LazyLib:
 
 
 _lib = _LazyLib()
-EXPORTED = ("qgemm_pack_sizes", "qgemm_pack", "qgemm", "qgemm_ex", "qgemm_select_path", "qgemm_dequant_tile",
+EXPORTED = ("qgemm_pack_sizes", "qgemm_pack", "qgemm", "qgemm_ex", "qgemm_fused", "qgemm_select_path",
+            "qgemm_dequant_tile",
             "qgemm_get_device_status", "qgemm_set_wait_limit_ns", "qgemm_debug_wait_timeout",
             "qgemm_status_str", "qgemm_last_error", "qgemm_version")
 
@@ -214,6 +224,39 @@ def qgemm(X, W: DeviceWeights, bias=None, out=None, path: int = QGEMM_PATH_AUTO,
     _check(_lib.qgemm_ex(X.data_ptr(), M, ctypes.byref(desc), out.data_ptr(),
                          None if bias is None else bias.data_ptr(), int(path) | flags, _stream_handle(stream)),
            "qgemm")
+    return out
+
+
+def qgemm_fused(X, W: DeviceWeights, op: int, bias=None, residual=None, gate=None, out=None,
+                path: int = QGEMM_PATH_AUTO, stream=None, overlap_previous: bool = False):
+    """qgemm with a fused epilogue (QGEMM_EPI_*): GELU, or out = residual + gate * y.
+    `out` may be `residual` itself (in-place update of the residual stream)."""
+    import torch
+    if X.dtype != torch.bfloat16 or not X.is_cuda or X.dim() != 2 or not X.is_contiguous():
+        raise ValueError("X must be a contiguous 2-D bf16 CUDA tensor")
+    M, K = X.shape
+    if K != W.K:
+        raise ValueError(f"X has K={K}, weights have K={W.K}")
+    if out is None:
+        out = torch.empty((M, W.N), dtype=torch.bfloat16, device=X.device)
+    elif out.dtype != torch.bfloat16 or tuple(out.shape) != (M, W.N) or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 [M, N] tensor")
+    if bias is not None and (bias.dtype != torch.bfloat16 or bias.numel() != W.N or not bias.is_cuda):
+        raise ValueError("bias must be a bf16 CUDA tensor of N elements")
+    if op == QGEMM_EPI_RESIDUAL_GATE:
+        if residual is None or gate is None:
+            raise ValueError("the residual update needs residual and gate")
+        if residual.dtype != torch.bfloat16 or tuple(residual.shape) != (M, W.N) or not residual.is_contiguous():
+            raise ValueError("residual must be a contiguous bf16 [M, N] tensor")
+        if gate.dtype != torch.bfloat16 or gate.numel() != W.N or not gate.is_cuda:
+            raise ValueError("gate must be a bf16 CUDA tensor of N elements")
+    epi = _Epilogue(int(op), None if residual is None else residual.data_ptr(),
+                    None if gate is None else gate.data_ptr())
+    desc = W.descriptor()
+    flags = QGEMM_FLAG_OVERLAP_PREVIOUS if overlap_previous else 0
+    _check(_lib.qgemm_fused(X.data_ptr(), M, ctypes.byref(desc), out.data_ptr(),
+                            None if bias is None else bias.data_ptr(), ctypes.byref(epi), int(path) | flags,
+                            _stream_handle(stream)), "qgemm_fused")
     return out
 
 

@@ -53,8 +53,10 @@
 #include <cuda.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "dequant.cuh"
+#include "epilogue.cuh"
 #include "qgemm_internal.h"
 
 namespace qg {
@@ -126,6 +128,8 @@ struct Params {
   int num_m_tiles, num_n_tiles, num_tiles, num_kb;
   int m_fastest;  // tile order: 1 = consecutive tiles walk the token dimension, 0 = the feature dimension
   const uint16_t* bias;
+  const uint16_t* residual;  // bf16 [M, N] (residual update only)
+  const uint16_t* gate;      // bf16 [N] (residual update only)
   uint64_t wait_limit_ns;
   unsigned int* status;
 };
@@ -155,11 +159,12 @@ __device__ __forceinline__ uint32_t swz(uint32_t off) {
   return off ^ (((off >> 7) & MASK) << 4);
 }
 
-template <int BITS>
+template <int BITS, int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     large_m_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                    const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_b,
-                   const __grid_constant__ CUtensorMap tm_out, const Params p) {
+                   const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_res,
+                   const Params p) {
   using C = Cfg<BITS>;
   constexpr int S = C::kS, SW = C::kSW;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -394,7 +399,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tile_coords(p, tile, n_tile, m_tile);
       const int n = n_tile * TILE_N + n_local;
       const int m0 = m_tile * TILE_M + t0;
-      const float bias_f = (p.bias && n < p.N) ? __bfloat162float(__ushort_as_bfloat16(p.bias[n])) : 0.f;
+      const bool n_ok = n < p.N;
+      const float bias_f = (p.bias && n_ok) ? __bfloat162float(__ushort_as_bfloat16(p.bias[n])) : 0.f;
+      float gate_f = 0.f;
+      if constexpr (EPI == QGEMM_EPI_RESIDUAL_GATE) {
+        if (n_ok) gate_f = epi::bf16_to_f32(p.gate[n]);
+        // while the tile's MMAs run, bring its residual block into L2
+        if (e == 0 && lane == 0) ptx::tma_prefetch_l2_2d(&tm_res, n_tile * TILE_N, m_tile * TILE_M);
+      }
       const bool got = warp_wait(acc_full, tcount & 1, lim, abort_flag);
       if (!got && lane == 0) {
         *epi_abort = 1;
@@ -408,6 +420,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                                  : (rows_left > 0 ? (rows_left + EPI_ROWS - 1) / EPI_ROWS : 0);
       for (int c = 0; c < EPI_TOKENS / EPI_ROWS; ++c) {
         uint32_t v[32];
+        // the residual update's 32 residual values of this chunk, two tokens per
+        // register (a warp reads 64 contiguous bytes per token)
+        uint32_t res2[EPI == QGEMM_EPI_RESIDUAL_GATE ? EPI_ROWS / 2 : 1];
+        if constexpr (EPI == QGEMM_EPI_RESIDUAL_GATE) {
+#pragma unroll
+          for (int t = 0; t < EPI_ROWS; t += 2) {
+            const int m = m0 + c * EPI_ROWS + t;
+            const bool ok = c < chunks && n_ok;
+            const uint32_t lo = (ok && m < p.M) ? p.residual[static_cast<size_t>(m) * p.N + n] : 0u;
+            const uint32_t hi = (ok && m + 1 < p.M) ? p.residual[static_cast<size_t>(m + 1) * p.N + n] : 0u;
+            res2[t / 2] = lo | (hi << 16);
+          }
+        }
         if (c < chunks) {
           ptx::tmem_ld_32x32b_x32(tmem_base + ACC_COL + t0 + c * EPI_ROWS + (static_cast<uint32_t>(32 * q) << 16), v);
           ptx::tmem_wait_ld();
@@ -425,8 +450,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           __syncwarp();
           uint16_t* sl = slots + slot * (EPI_SLOT_BYTES / 2);
 #pragma unroll
-          for (int t = 0; t < EPI_ROWS; ++t)
-            sl[t * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[t]) + bias_f));
+          for (int t = 0; t < EPI_ROWS; ++t) {
+            const uint16_t r =
+                EPI == QGEMM_EPI_RESIDUAL_GATE ? static_cast<uint16_t>(res2[EPI == QGEMM_EPI_RESIDUAL_GATE ? t / 2 : 0] >> (16 * (t & 1))) : 0;
+            const float f = epi::apply<EPI>(__uint_as_float(v[t]) + bias_f, r, gate_f);
+            sl[t * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(f));
+          }
           ptx::fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -452,13 +481,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-template <int BITS>
+template <int BITS, int EPI>
 int launch_fmt(const Problem& pr, int nsm) {
   using C = Cfg<BITS>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(large_m_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    attr_err =
+        cudaFuncSetAttribute(large_m_kernel<BITS, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   });
   int st = cuda_check(attr_err, "cudaFuncSetAttribute(large_m_kernel)");
   if (st != QGEMM_OK) return st;
@@ -510,9 +540,17 @@ int launch_fmt(const Problem& pr, int nsm) {
     kp.m_fastest = live(kp.num_m_tiles, x_panel, w_panel) <= live(kp.num_n_tiles, w_panel, x_panel);
   }
   kp.bias = pr.bias;
+  kp.residual = pr.residual;
+  kp.gate = pr.gate;
+  CUtensorMap tm_res = tm_out;  // the residual update's L2 prefetch box: one tile
+  if (EPI == QGEMM_EPI_RESIDUAL_GATE &&
+      (st = make_tensor_map_2d(&tm_res, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pr.residual, pr.N, pr.M,
+                               uint64_t(pr.N) * 2, TILE_N, TILE_M, CU_TENSOR_MAP_SWIZZLE_NONE, "residual")) != QGEMM_OK)
+    return st;
   kp.wait_limit_ns = wait_limit_ns();
   kp.status = status;
-  large_m_kernel<BITS><<<grid, NUM_THREADS, C::kSmemBytes, pr.stream>>>(tm_x, tm_w, tm_s, tm_b, tm_out, kp);
+  large_m_kernel<BITS, EPI><<<grid, NUM_THREADS, C::kSmemBytes, pr.stream>>>(tm_x, tm_w, tm_s, tm_b, tm_out, tm_res,
+                                                                               kp);
   return cuda_check(cudaGetLastError(), "large_m_kernel launch");
 }
 
@@ -522,10 +560,18 @@ int launch_large_m(const Problem& p) {
   int nsm;
   int st = sm_count(&nsm);
   if (st != QGEMM_OK) return st;
+  auto go = [&](auto bits_tag) {
+    constexpr int B = decltype(bits_tag)::value;
+    switch (p.epi) {
+      case QGEMM_EPI_GELU_TANH: return lm::launch_fmt<B, QGEMM_EPI_GELU_TANH>(p, nsm);
+      case QGEMM_EPI_RESIDUAL_GATE: return lm::launch_fmt<B, QGEMM_EPI_RESIDUAL_GATE>(p, nsm);
+      default: return lm::launch_fmt<B, QGEMM_EPI_NONE>(p, nsm);
+    }
+  };
   switch (p.bits) {
-    case 4: return lm::launch_fmt<4>(p, nsm);
-    case 8: return lm::launch_fmt<8>(p, nsm);
-    default: return lm::launch_fmt<2>(p, nsm);
+    case 4: return go(std::integral_constant<int, 4>{});
+    case 8: return go(std::integral_constant<int, 8>{});
+    default: return go(std::integral_constant<int, 2>{});
   }
 }
 

@@ -86,8 +86,8 @@ int select_path(int M, int N, int K, int bits) {
 
 using namespace qg;
 
-extern "C" int qgemm_ex(const void* X, int32_t M, const qgemm_weights* W, void* out, const void* bias,
-                        int32_t path, void* stream) {
+extern "C" int qgemm_fused(const void* X, int32_t M, const qgemm_weights* W, void* out, const void* bias,
+                           const qgemm_epilogue* epi, int32_t path, void* stream) {
   int st = validate_weights(W);
   if (st != QGEMM_OK) return st;
   if (M < 0) return fail(QGEMM_ERR_INVALID_ARG, "M=%d is negative", M);
@@ -95,6 +95,13 @@ extern "C" int qgemm_ex(const void* X, int32_t M, const qgemm_weights* W, void* 
   path &= 0xFF;
   if (path < QGEMM_PATH_AUTO || path > QGEMM_PATH_LARGE_M) return fail(QGEMM_ERR_INVALID_ARG, "bad path %d", path);
   if (flags & ~QGEMM_FLAG_OVERLAP_PREVIOUS) return fail(QGEMM_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  const int op = epi ? epi->op : QGEMM_EPI_NONE;
+  if (op < QGEMM_EPI_NONE || op > QGEMM_EPI_RESIDUAL_GATE) return fail(QGEMM_ERR_INVALID_ARG, "bad epilogue %d", op);
+  if (op == QGEMM_EPI_RESIDUAL_GATE) {
+    if (!epi->residual || !epi->gate) return fail(QGEMM_ERR_INVALID_ARG, "the residual update needs residual and gate");
+    if (!aligned16(epi->residual)) return fail(QGEMM_ERR_ALIGNMENT, "residual must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(epi->gate) & 1u) return fail(QGEMM_ERR_ALIGNMENT, "gate must be 2-byte aligned");
+  }
   if (M == 0) return QGEMM_OK;
   if (!X || !out) return fail(QGEMM_ERR_INVALID_ARG, "null X or out");
   if (!aligned16(X) || !aligned16(out)) return fail(QGEMM_ERR_ALIGNMENT, "X and out must be 16-byte aligned");
@@ -107,8 +114,15 @@ extern "C" int qgemm_ex(const void* X, int32_t M, const qgemm_weights* W, void* 
   Problem p{X, M, W->N, W->K, W->bits, W->group, static_cast<const uint8_t*>(W->packed),
             static_cast<const uint16_t*>(W->scales), static_cast<const uint16_t*>(W->biases), out,
             static_cast<const uint16_t*>(bias), static_cast<cudaStream_t>(stream),
-            (flags & QGEMM_FLAG_OVERLAP_PREVIOUS) != 0};
+            (flags & QGEMM_FLAG_OVERLAP_PREVIOUS) != 0, op,
+            op == QGEMM_EPI_RESIDUAL_GATE ? static_cast<const uint16_t*>(epi->residual) : nullptr,
+            op == QGEMM_EPI_RESIDUAL_GATE ? static_cast<const uint16_t*>(epi->gate) : nullptr};
   return path == QGEMM_PATH_SMALL_M ? launch_small_m(p) : launch_large_m(p);
+}
+
+extern "C" int qgemm_ex(const void* X, int32_t M, const qgemm_weights* W, void* out, const void* bias,
+                        int32_t path, void* stream) {
+  return qgemm_fused(X, M, W, out, bias, nullptr, path, stream);
 }
 
 extern "C" int qgemm(const void* X, int32_t M, const qgemm_weights* W, void* out, const void* bias, void* stream) {

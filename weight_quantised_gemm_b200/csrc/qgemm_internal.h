@@ -23,6 +23,9 @@ struct Problem {
   const uint16_t* bias;  // bf16 bits [N] or nullptr
   cudaStream_t stream;
   bool overlap;          // launch with programmatic dependent launch (QGEMM_FLAG_OVERLAP_PREVIOUS)
+  int epi;               // QGEMM_EPI_*
+  const uint16_t* residual;  // bf16 bits [M, N] (QGEMM_EPI_RESIDUAL_GATE), may equal out
+  const uint16_t* gate;      // bf16 bits [N] (QGEMM_EPI_RESIDUAL_GATE)
 };
 
 // Records a detail message for qgemm_last_error and returns `code`.

@@ -54,6 +54,7 @@
 #include <mutex>
 
 #include "dequant.cuh"
+#include "epilogue.cuh"
 #include "qgemm_internal.h"
 
 namespace qg {
@@ -90,6 +91,9 @@ struct Params {
   const uint16_t* X;     // bf16 [M, K]
   const uint16_t* bias;  // bf16 [N] or null
   uint16_t* out;         // bf16 [M, N]
+  int epi;               // QGEMM_EPI_*
+  const uint16_t* residual;  // bf16 [M, N] (residual update only; may equal out)
+  const uint16_t* gate;      // bf16 [N] (residual update only)
   int M, N, K;
   int num_stages;        // ceil(K / KS)
   int ring;              // ring depth
@@ -415,7 +419,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
     for (int l = 0; l < GROUP_LANES; ++l) v += red[(l * MT + m) * NLP + nl];
     if (p.bias) v += __bfloat162float(__ushort_as_bfloat16(p.bias[n]));
-    p.out[static_cast<size_t>(m) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    const size_t o = static_cast<size_t>(m) * p.N + n;
+    if (p.epi != QGEMM_EPI_NONE)
+      v = epi::apply_dyn(p.epi, v, p.epi == QGEMM_EPI_RESIDUAL_GATE ? p.residual[o] : uint16_t(0),
+                         p.epi == QGEMM_EPI_RESIDUAL_GATE ? epi::bf16_to_f32(p.gate[n]) : 0.f);
+    p.out[o] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
   }
 }
 
@@ -439,6 +447,9 @@ int launch_fmt(const Problem& pr, int grid) {
   kp.X = static_cast<const uint16_t*>(pr.X);
   kp.bias = pr.bias;
   kp.out = static_cast<uint16_t*>(pr.out);
+  kp.epi = pr.epi;
+  kp.residual = pr.residual;
+  kp.gate = pr.gate;
   kp.M = pr.M;
   kp.N = pr.N;
   kp.K = pr.K;
