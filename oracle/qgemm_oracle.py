@@ -25,6 +25,8 @@ formula and no rounding rule):
   rest at 4" (stable-diffusion.rs README, introduction) names the two widths.
 * ternary {-1, 0, +1} with one fp16 scale per group of 128
   (pictor README, "Extreme quantization is first-class": TQ2_0_g128).
+* 1-bit {-1, +1} with one fp16 scale per group of 128 (the same README's
+  Q1_0_g128, named without a definition).
 
 Packing is round-to-nearest (RTN) in fp64, ties to even:
 
@@ -34,6 +36,8 @@ Packing is round-to-nearest (RTN) in fp64, ties to even:
   2^b - 1), q = 0 where s16 == 0.
 * ternary: s16 = fp16(max |w|); t = clamp(rint(w / s16), -1, 1), t = 0 where
   s16 == 0.
+* 1-bit: s16 = fp16(mean |w|), the scale that minimises the squared error
+  for fixed signs; c = +1 where w >= 0 (-0 included), else -1.
 
 Bit layout, row-major over N with K contiguous, little-endian 32-bit words:
 
@@ -43,6 +47,8 @@ Bit layout, row-major over N with K contiguous, little-endian 32-bit words:
 * ternary: a word holds 16 consecutive k; offset j = 2i in bits 2i..2i+1 and
   j = 2i + 1 in bits 16+2i..17+2i. The 2-bit code is t in two's complement
   (0 -> 00, +1 -> 01, -1 -> 11); code 10 is invalid.
+* 1-bit: a word holds 32 consecutive k; offset j = 2i in bit i and j = 2i + 1
+  in bit 16 + i; bit 1 is +1, bit 0 is -1.
 * scales and biases: fp16 [K / group, N], group-major (the scales of one
   group of k for all rows are contiguous).
 
@@ -52,6 +58,7 @@ Dequantised weight (the bit-exact contract of the dequant-tile entry point):
   (11 + 8 significant bits), so this equals one fp32 FMA followed by one
   round-to-nearest-even to bf16.
 * ternary: wdeq = t * bf16_rn(fl32(s16)), with +0 for t = 0.
+* 1-bit: wdeq = c * bf16_rn(fl32(s16)).
 
 Numerics of the matmul: fp32 accumulation is what the kernels keep (pictor
 README, numerics: "FP32 accumulate is kept", no TF32 or FP16-MAC shortcuts);
@@ -63,6 +70,7 @@ import numpy as np
 
 AFFINE_BITS = (4, 8)
 TERNARY_BITS = 2
+BINARY_BITS = 1
 
 
 # ----------------------------------------------------------------------------
@@ -119,7 +127,8 @@ def pack_codes(codes, bits: int) -> np.ndarray:
     """Integer codes [N, K] -> packed bytes [N, K * bits / 8].
 
     Affine codes are q in [0, 2^b - 1]; ternary codes are t in {-1, 0, +1}
-    and are stored as 2-bit two's complement.
+    and are stored as 2-bit two's complement; 1-bit codes are c in {-1, +1},
+    stored as 1 for +1 and 0 for -1.
     """
     codes = np.asarray(codes)
     N, K = codes.shape
@@ -127,7 +136,12 @@ def pack_codes(codes, bits: int) -> np.ndarray:
     if K % per:
         raise ValueError("K must fill whole 32-bit words")
     mask = (1 << bits) - 1
-    field = codes.astype(np.int64) & mask           # two's complement for t = -1
+    if bits == BINARY_BITS:
+        if not np.all(np.abs(codes) == 1):
+            raise ValueError("1-bit codes are -1 or +1")
+        field = (codes > 0).astype(np.int64)
+    else:
+        field = codes.astype(np.int64) & mask           # two's complement for t = -1
     field = field.astype(np.uint32).reshape(N, K // per, per)
     words = np.zeros((N, K // per), dtype=np.uint32)
     for j in range(per):
@@ -151,6 +165,8 @@ def unpack_codes(packed, bits: int, K: int) -> np.ndarray:
     for j in range(per):
         out[:, :, j] = (words >> np.uint32(code_bit_position(bits, j))) & mask
     out = out.reshape(N, K)
+    if bits == BINARY_BITS:
+        return np.where(out == 1, 1, -1).astype(np.int32)
     if bits == TERNARY_BITS:
         if np.any(out == 2):
             raise ValueError("invalid ternary code 0b10")
@@ -166,11 +182,11 @@ def check_format(bits: int, group: int, K: int) -> None:
     if bits in AFFINE_BITS:
         if group != 64:
             raise ValueError("affine formats use groups of 64")
-    elif bits == TERNARY_BITS:
+    elif bits in (TERNARY_BITS, BINARY_BITS):
         if group != 128:
-            raise ValueError("ternary uses groups of 128")
+            raise ValueError("ternary and 1-bit use groups of 128")
     else:
-        raise ValueError("bits must be 2 (ternary), 4 or 8")
+        raise ValueError("bits must be 1, 2 (ternary), 4 or 8")
     if K % group:
         raise ValueError("K must be a multiple of the group size")
 
@@ -202,6 +218,12 @@ def pack_ref(W, bits: int, group: int):
         q = np.where(s == 0, 0, q)
         codes = q.reshape(N, K).astype(np.int64)
         return pack_codes(codes, bits), np.ascontiguousarray(s16.T), np.ascontiguousarray(b16.T)
+    if bits == BINARY_BITS:
+        s16 = fp16_rn(np.abs(Wg).mean(axis=2))
+        if not np.all(np.isfinite(s16)):
+            raise OverflowError("scale overflows fp16")
+        c = np.where(Wg >= 0, 1, -1)
+        return pack_codes(c.reshape(N, K).astype(np.int64), bits), np.ascontiguousarray(s16.T), None
     s16 = fp16_rn(np.abs(Wg).max(axis=2))
     if not np.all(np.isfinite(s16)):
         raise OverflowError("scale overflows fp16")
@@ -225,7 +247,7 @@ def wq_exact(packed, scales, biases, bits: int, group: int, K: int) -> np.ndarra
     """The quantised weight before any bf16 rounding, fp64 [N, K]: s16*q + b16 or s16*t."""
     codes = unpack_codes(packed, bits, K).astype(np.float64)
     s = _expand(scales, group)
-    if bits == TERNARY_BITS:
+    if bits in (TERNARY_BITS, BINARY_BITS):
         return s * codes
     return s * codes + _expand(biases, group)
 
@@ -241,7 +263,7 @@ def dequant_ref_bits(packed, scales, biases, bits: int, group: int, K: int) -> n
     """
     codes = unpack_codes(packed, bits, K)
     s = _expand(scales, group)
-    if bits == TERNARY_BITS:
+    if bits in (TERNARY_BITS, BINARY_BITS):
         sb = bf16_rn_bits(s.astype(np.float32))
         out = np.where(codes < 0, sb | np.uint16(0x8000), sb)
         return np.where(codes == 0, np.uint16(0), out).astype(np.uint16)
@@ -369,5 +391,5 @@ def within_tolerance(y, ref) -> bool:
 
 def format_bytes(N: int, K: int, bits: int, group: int) -> int:
     """Bytes of one packed weight at rest: codes + fp16 scales (+ fp16 biases)."""
-    per_group = 2 if bits == TERNARY_BITS else 4
+    per_group = 2 if bits in (TERNARY_BITS, BINARY_BITS) else 4
     return N * K * bits // 8 + N * (K // group) * per_group

@@ -453,3 +453,73 @@ def test_fused_reference_composes_the_plain_gemm():
     assert np.array_equal(O.qgemm_ref_epilogue(X, p, s, b, 4, 64, 128, bias, O.EPI_GELU_TANH), O.gelu_tanh_ref(y))
     with pytest.raises(ValueError):
         O.epilogue_ref(y, 7)
+
+
+# ----------------------------------------------------------------------------
+# the 1-bit format (Q1_0_g128)
+# ----------------------------------------------------------------------------
+
+def test_layout_hand_derived_1bit():
+    # +1 at k = 0 (bit 0), k = 1 (bit 16), k = 30 (bit 15) and k = 31 (bit 31);
+    # -1 elsewhere: word = 0x1 | 0x10000 | 0x8000 | 0x80000000 = 0x80018001
+    c = -np.ones((1, 32), dtype=np.int64)
+    c[0, [0, 1, 30, 31]] = 1
+    assert O.pack_codes(c, 1).tolist() == [[0x01, 0x80, 0x01, 0x80]]
+    with pytest.raises(ValueError):
+        O.pack_codes(np.zeros((1, 32), dtype=np.int64), 1)   # 0 is not a 1-bit code
+
+
+def test_1bit_pack_unpack_bijection_and_every_byte():
+    g = np.random.default_rng(11)
+    c = np.where(g.integers(0, 2, size=(7, 256)) == 1, 1, -1)
+    assert np.array_equal(O.unpack_codes(O.pack_codes(c, 1), 1, 256), c)
+    raw = g.integers(0, 256, size=(5, 64), dtype=np.uint8)      # every byte pattern is valid
+    assert np.array_equal(O.pack_codes(O.unpack_codes(raw, 1, 512), 1), raw)
+
+
+def test_1bit_constructed_weights_round_trip_exactly():
+    """W = s16 * c (signs, one fp16 scale per 128) packs back to c and s16."""
+    W = WL.make_w(5, 1, 64, 3072, "binary", 128)
+    packed, s16, b = O.pack_ref(W, 1, 128)
+    assert b is None and packed.shape == (64, 3072 // 8)
+    c = O.unpack_codes(packed, 1, 3072)
+    recon = np.repeat(s16.T.astype(np.float32), 128, axis=1) * c
+    assert np.array_equal(recon.astype(np.float32), W)
+
+
+def test_1bit_scale_is_the_least_squares_one():
+    """For fixed signs the squared error of s * sign(w) is minimised by the
+    mean |w|; no neighbouring fp16 value of the stored scale does better, and
+    the signs follow w (zero and -0 counted as +1)."""
+    g = np.random.default_rng(12)
+    w = (g.standard_normal((3, 256)) * 0.02).astype(np.float32)
+    w[0, 5], w[1, 9] = 0.0, -0.0
+    packed, s16, _ = O.pack_ref(w, 1, 128)
+    c = O.unpack_codes(packed, 1, 256)
+    assert np.array_equal(c, np.where(w >= 0, 1, -1))
+    assert c[0, 5] == 1 and c[1, 9] == 1
+    for n in range(3):
+        for j in range(2):
+            wg = w[n, 128 * j:128 * (j + 1)].astype(np.float64)
+            cg = c[n, 128 * j:128 * (j + 1)]
+            s = float(s16[j, n])
+            err = lambda v: float(np.sum((wg - v * cg) ** 2))
+            up = float(np.nextafter(np.float16(s), np.float16(np.inf)))
+            down = float(np.nextafter(np.float16(s), np.float16(0)))
+            assert err(s) <= err(up) and err(s) <= err(down)
+
+
+def test_1bit_dequant_is_signed_scale_and_gemm_matches_triple_loop():
+    g = np.random.default_rng(13)
+    c = np.where(g.integers(0, 2, size=(6, 256)) == 1, 1, -1)
+    s16 = g.uniform(0.01, 0.05, size=(6, 2)).astype(np.float16)
+    packed = O.pack_codes(c, 1)
+    bits = O.dequant_ref_bits(packed, np.ascontiguousarray(s16.T), None, 1, 128, 256)
+    sb = torch.from_numpy(np.repeat(s16.astype(np.float32), 128, axis=1)).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(O.bf16_bits_to_f64(bits), c * sb.astype(np.float64))
+    X, W, bias = WL.random_case(2, 4, 5, 128, 1, with_bias=True)
+    p, s, b = O.pack_ref(W, 1, 128)
+    ref = O.qgemm_ref(X, p, s, b, 1, 128, 128, bias)
+    brute = _naive(O.bf16_bits_to_f64(X), O.wq_exact(p, s, b, 1, 128, 128), O.bf16_bits_to_f64(bias))
+    assert np.allclose(ref, brute, rtol=1e-12, atol=1e-14)
+    assert O.format_bytes(12288, 3072, 1, 128) == 12288 * 3072 // 8 + 12288 * 24 * 2

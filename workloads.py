@@ -32,8 +32,8 @@ class Linear:
     M: int
     N: int
     K: int
-    bits: int            # 2 = ternary, 4 or 8 = group-wise affine
-    group: int           # 64 for affine, 128 for ternary
+    bits: int            # 1 = 1-bit, 2 = ternary, 4 or 8 = group-wise affine
+    group: int           # 64 for affine, 128 for ternary and 1-bit
     bias: bool           # bf16 bias [N] ~ N(0, 0.01)
     x_dist: str          # "normal" = N(0,1); "gelu" = tanh-GELU of N(0,1)
     w_dist: str          # "normal" = N(0, 0.02) fp32; "ternary" = s16 * t
@@ -58,6 +58,10 @@ def _tern(name, M, N=12288, K=3072):
     return Linear(name, M, N, K, 2, 128, False, "normal", "ternary")
 
 
+def _bin(name, M, N=12288, K=3072):
+    return Linear(name, M, N, K, 1, 128, False, "normal", "binary")
+
+
 WORKLOADS = (
     Workload(0, "tiny 4-bit [64,512]x[512,512]",
              (_aff("tiny", 64, 512, 512, 4),)),
@@ -76,6 +80,9 @@ WORKLOADS = (
               _aff("out_proj", 4608, 3072, 3072, 8),
               _aff("mlp_up", 4608, 12288, 3072, 4),
               _aff("mlp_down", 4608, 3072, 12288, 8, x="gelu"))),
+    Workload(5, "sub-byte formats at DiT shapes: ternary prefill M=4096 and 1-bit (Q1_0_g128) decode M=1 and "
+                "prefill M=4096, [M,3072]x[12288,3072]",
+             (_tern("tern_prefill", 4096), _bin("bin_m1", 1), _bin("bin_prefill", 4096))),
 )
 
 
@@ -125,7 +132,8 @@ def make_w(cid: int, lin_idx: int, N: int, K: int, dist: str, group: int = 128,
     "normal": N(0, 0.02).  "ternary": W = fp32(s16) * t with t uniform on
     {-1, 0, +1} (P(0) = 1/3) and one fp16 scale s16 ~ U(0.01, 0.05) per group
     of `group` consecutive k, so the weights are exactly representable by the
-    ternary format.
+    ternary format.  "binary": the same with signs uniform on {-1, +1}, exactly
+    representable by the 1-bit format.
     """
     if dist == "normal":
         return (_rng(cid, lin_idx, _T_W, extra).standard_normal((N, K)) * 0.02).astype(np.float32)
@@ -134,6 +142,11 @@ def make_w(cid: int, lin_idx: int, N: int, K: int, dist: str, group: int = 128,
         s = _rng(cid, lin_idx, _T_SCALE, extra).uniform(0.01, 0.05, size=(N, K // group))
         s16 = s.astype(np.float16).astype(np.float32)
         return (t * np.repeat(s16, group, axis=1)).astype(np.float32)
+    if dist == "binary":
+        c = 2.0 * _rng(cid, lin_idx, _T_TERN, extra).integers(0, 2, size=(N, K)).astype(np.float32) - 1.0
+        s = _rng(cid, lin_idx, _T_SCALE, extra).uniform(0.01, 0.05, size=(N, K // group))
+        s16 = s.astype(np.float16).astype(np.float32)
+        return (c * np.repeat(s16, group, axis=1)).astype(np.float32)
     raise ValueError(dist)
 
 
@@ -157,7 +170,11 @@ def random_case(seed: int, M: int, N: int, K: int, bits: int, with_bias: bool,
     """A seeded off-config case (ragged sizes, edge tests)."""
     g = np.random.default_rng(np.random.SeedSequence([1, seed, M, N, K, bits]))
     X = f32_to_bf16_bits((g.standard_normal((M, K)) * x_scale).astype(np.float32))
-    if bits == 2:
+    if bits == 1:
+        c = 2.0 * g.integers(0, 2, size=(N, K)).astype(np.float32) - 1.0
+        s16 = g.uniform(0.01, 0.05, size=(N, K // 128)).astype(np.float16).astype(np.float32)
+        W = (c * np.repeat(s16, 128, axis=1)).astype(np.float32)
+    elif bits == 2:
         t = g.integers(-1, 2, size=(N, K)).astype(np.float32)
         s16 = g.uniform(0.01, 0.05, size=(N, K // 128)).astype(np.float16).astype(np.float32)
         W = (t * np.repeat(s16, 128, axis=1)).astype(np.float32)
