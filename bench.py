@@ -331,7 +331,7 @@ def sweep(peaks):
             entry["frac_of_roofline_overlap_previous"] = round(t_roof / to, 3)
         return entry, sets, host
 
-    for cid in range(5):
+    for cid in range(len(WL.WORKLOADS)):
         wl = WL.workload(cid)
         for li, lin in enumerate(wl.linears):
             entry, sets, host = one(cid, li, lin, lin.M, wq.QGEMM_PATH_AUTO, 100 if lin.M <= 16 else 20)
@@ -377,9 +377,9 @@ def sweep(peaks):
     cross = []
     lin3 = WL.workload(3).linears[0]
     import dataclasses
-    for bits in (2, 4, 8):
+    for bits in (1, 2, 4, 8):
         lin = dataclasses.replace(lin3, bits=bits, group=wq.GROUP_OF_BITS[bits],
-                                  w_dist="ternary" if bits == 2 else "normal")
+                                  w_dist={1: "binary", 2: "ternary"}.get(bits, "normal"))
         for M in (1, 4, 8, 16, 32, 64):
             for path in (wq.QGEMM_PATH_SMALL_M, wq.QGEMM_PATH_LARGE_M):
                 if path == wq.QGEMM_PATH_SMALL_M and M > 16:

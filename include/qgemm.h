@@ -7,7 +7,7 @@
  *
  *     out[M, N] = X[M, K] . dequant(W)[N, K]^T (+ bias[N])
  *
- * with X and out in bf16, W packed in one of three formats, and fp32
+ * with X and out in bf16, W packed in one of four formats, and fp32
  * accumulation throughout (pictor README, numerics: fp32 accumulate is kept,
  * no TF32 or FP16-MAC shortcuts).
  *
@@ -21,7 +21,11 @@
  *                               bits, the rest at 4);
  *   bits = 2, group = 128       ternary t in {-1, 0, +1} with one fp16 scale per
  *                               128 consecutive k (pictor README, "Extreme
- *                               quantization is first-class": TQ2_0_g128).
+ *                               quantization is first-class": TQ2_0_g128);
+ *   bits = 1, group = 128       1-bit c in {-1, +1} with one fp16 scale per 128
+ *                               consecutive k (the same README's Q1_0_g128,
+ *                               named without a definition; this library's
+ *                               reading: w ~ c * s, s = mean |w|).
  *
  * Bit layout (row-major over N, K contiguous, little-endian 32-bit words):
  *   8-bit   byte k holds q[k];
@@ -30,6 +34,8 @@
  *   ternary a word holds 16 consecutive k: j = 2i in bits 2i..2i+1, j = 2i+1
  *           in bits 16+2i..17+2i; the code is t in 2-bit two's complement
  *           (00 = 0, 01 = +1, 11 = -1; 10 is invalid);
+ *   1-bit   a word holds 32 consecutive k: j = 2i in bit i, j = 2i+1 in bit
+ *           16+i; bit 1 is +1, bit 0 is -1;
  *   scales, biases: fp16 [K / group, N], group-major: the values of one
  *           group of k for all N rows are contiguous, so a tile's scales
  *           arrive in one TMA box with its codes.
@@ -39,7 +45,8 @@
  * Dequantised weight (what the kernels multiply; bit-exact contract):
  *   affine   wdeq = bf16_rn( fp32(s) * q + fp32(b) )  — one fp32 FMA, whose
  *            product is exact, then one round-to-nearest-even to bf16;
- *   ternary  wdeq = t * bf16_rn(fp32(s)), +0 for t = 0.
+ *   ternary  wdeq = t * bf16_rn(fp32(s)), +0 for t = 0;
+ *   1-bit    wdeq = c * bf16_rn(fp32(s)).
  *
  * Ownership: the caller allocates every buffer passed in; the library never
  * allocates, frees or keeps user memory. Device-side state is one static
@@ -97,19 +104,19 @@ enum {
 typedef struct qgemm_weights {
   int32_t N;             /* output features (rows of W) */
   int32_t K;             /* input features (columns of W) */
-  int32_t bits;          /* 2 (ternary), 4 or 8 */
-  int32_t group;         /* 128 for ternary, 64 for 4- and 8-bit */
+  int32_t bits;          /* 1 (1-bit), 2 (ternary), 4 or 8 */
+  int32_t group;         /* 128 for 1-bit and ternary, 64 for 4- and 8-bit */
   const void* packed;    /* uint8 [N, K * bits / 8], 16-byte aligned */
   const void* scales;    /* fp16 [K / group, N], 16-byte aligned */
-  const void* biases;    /* fp16 [K / group, N], 16-byte aligned; NULL for ternary */
+  const void* biases;    /* fp16 [K / group, N], 16-byte aligned; NULL for 1-bit and ternary */
 } qgemm_weights;
 
 /*
  * Byte sizes of the three packed arrays for an [N, K] weight.
- * Defined by the layout above. biases_bytes is 0 for ternary.
+ * Defined by the layout above. biases_bytes is 0 for 1-bit and ternary.
  * Returns INVALID_ARG for non-positive sizes or null outputs, UNSUPPORTED
- * for a (bits, group) pair other than (4,64), (8,64), (2,128) or for K not a
- * multiple of 128.
+ * for a (bits, group) pair other than (4,64), (8,64), (2,128), (1,128) or
+ * for K not a multiple of 128.
  */
 int qgemm_pack_sizes(int32_t N, int32_t K, int32_t bits, int32_t group,
                      size_t* packed_bytes, size_t* scales_bytes, size_t* biases_bytes);
@@ -120,11 +127,12 @@ int qgemm_pack_sizes(int32_t N, int32_t K, int32_t bits, int32_t group,
  * Arithmetic is fp64, ties to even:
  *   affine:  s = fp16(fl64((max - min) / (2^bits - 1))), b = fp16(min),
  *            q = clamp(rint((w - b) / s), 0, 2^bits - 1), q = 0 where s == 0;
- *   ternary: s = fp16(max |w|), t = clamp(rint(w / s), -1, 1), t = 0 where s == 0.
+ *   ternary: s = fp16(max |w|), t = clamp(rint(w / s), -1, 1), t = 0 where s == 0;
+ *   1-bit:   s = fp16(mean |w|), c = +1 where w >= 0 (and for -0), else -1.
  * The weights stay packed at rest (stable-diffusion.rs README, introduction).
  * Returns NONFINITE if W holds NaN/Inf, UNSUPPORTED if a scale or bias
  * overflows fp16, plus the errors of qgemm_pack_sizes. biases may be NULL for
- * ternary. Host-only; no device is touched.
+ * 1-bit and ternary. Host-only; no device is touched.
  */
 int qgemm_pack(const float* W, int32_t N, int32_t K, int32_t bits, int32_t group,
                void* packed, void* scales, void* biases);
@@ -136,7 +144,8 @@ int qgemm_pack(const float* W, int32_t N, int32_t K, int32_t bits, int32_t group
  *   W     device-resident packed weights (struct itself is host memory)
  *   out   device bf16 [M, N] row-major, 16-byte aligned
  *   bias  device bf16 [N] or NULL
- * Requires K % 128 == 0 and N % 16 == 0. The path (small-M register path or
+ * Requires K % 128 == 0 and N % 16 == 0 (1-bit weights with K % 256 != 0
+ * always take the large-M path). The path (small-M register path or
  * large-M tensor-core path) is chosen per (bits, M, N, K) from a measured
  * table; the environment variable QGEMM_PATH=small|large overrides it.
  * Returns after enqueueing; a device-side failure (a bounded wait that ran

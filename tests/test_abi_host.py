@@ -40,12 +40,14 @@ def test_pack_sizes():
     assert wq.qgemm_pack_sizes(9216, 3072, 4) == (9216 * 1536, 9216 * 48 * 2, 9216 * 48 * 2)
     assert wq.qgemm_pack_sizes(3072, 12288, 8) == (3072 * 12288, 3072 * 192 * 2, 3072 * 192 * 2)
     assert wq.qgemm_pack_sizes(12288, 3072, 2) == (12288 * 768, 12288 * 24 * 2, 0)
+    assert wq.qgemm_pack_sizes(12288, 3072, 1) == (12288 * 384, 12288 * 24 * 2, 0)
 
 
 @pytest.mark.parametrize("args,status", [
     ((16, 128, 3, 64), wq.QGEMM_ERR_UNSUPPORTED),
     ((16, 128, 4, 128), wq.QGEMM_ERR_UNSUPPORTED),
     ((16, 128, 2, 64), wq.QGEMM_ERR_UNSUPPORTED),
+    ((16, 128, 1, 64), wq.QGEMM_ERR_UNSUPPORTED),
     ((16, 192, 4, 64), wq.QGEMM_ERR_UNSUPPORTED),     # K not a multiple of 128
     ((0, 128, 4, 64), wq.QGEMM_ERR_INVALID_ARG),
     ((16, -128, 4, 64), wq.QGEMM_ERR_INVALID_ARG),
@@ -132,7 +134,11 @@ def test_dequant_tile_rejects_bad_windows_without_device():
 
 
 def test_select_path_table():
-    for bits in (2, 4, 8):
+    # 1-bit rows need K % 256 == 0 on the small path; otherwise the large path
+    assert wq.qgemm_select_path(1, 12288, 1152, 1) == wq.QGEMM_PATH_LARGE_M
+    assert _call(_desc(bits=1, group=128, K=1152, biases=0), M=4, path=wq.QGEMM_PATH_SMALL_M) == \
+        wq.QGEMM_ERR_UNSUPPORTED
+    for bits in (1, 2, 4, 8):
         assert wq.qgemm_select_path(1, 12288, 3072, bits) == wq.QGEMM_PATH_SMALL_M
         assert wq.qgemm_select_path(4096, 9216, 3072, bits) == wq.QGEMM_PATH_LARGE_M
     with pytest.raises(wq.QGemmError):

@@ -42,10 +42,12 @@ def _assert_close(y_bits, ref, what=""):
 # dequantisation: bit-exact
 # ----------------------------------------------------------------------------
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
 def test_dequant_whole_matrix_bit_exact(bits):
     group = wq.GROUP_OF_BITS[bits]
-    if bits == 2:
+    if bits == 1:
+        W = WL.make_w(5, 1, 512, 3072, "binary", 128)
+    elif bits == 2:
         W = WL.make_w(3, 0, 512, 3072, "ternary", 128)
     else:
         W = WL.make_w(0, 0, 512, 1024, "normal")
@@ -57,7 +59,7 @@ def test_dequant_whole_matrix_bit_exact(bits):
     assert np.array_equal(got, ref)
 
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
 def test_dequant_edge_groups_and_windows_bit_exact(bits):
     group = wq.GROUP_OF_BITS[bits]
     g = np.random.default_rng(55 + bits)
@@ -78,13 +80,17 @@ def test_dequant_edge_groups_and_windows_bit_exact(bits):
 # one-hot activations: the GEMM data path bit-exact to the dequantised weights
 # ----------------------------------------------------------------------------
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
 @pytest.mark.parametrize("path,M", [(SMALL, 16), (SMALL, 5), (LARGE, 16), (LARGE, 300)])
 def test_one_hot_rows_reproduce_dequantised_weights(bits, path, M):
     group = wq.GROUP_OF_BITS[bits]
-    N, K = 272, 640
+    N, K = 272, 768
     g = np.random.default_rng(9)
-    if bits == 2:
+    if bits == 1:
+        c = 2.0 * g.integers(0, 2, size=(N, K)).astype(np.float32) - 1.0
+        s = g.uniform(0.01, 0.05, size=(N, K // 128)).astype(np.float16).astype(np.float32)
+        W = (c * np.repeat(s, 128, axis=1)).astype(np.float32)
+    elif bits == 2:
         t = g.integers(-1, 2, size=(N, K)).astype(np.float32)
         s = g.uniform(0.01, 0.05, size=(N, K // 128)).astype(np.float16).astype(np.float32)
         W = (t * np.repeat(s, 128, axis=1)).astype(np.float32)
@@ -110,15 +116,16 @@ def test_tiny_workload_default_path():
     _assert_close(y, _ref(X, W, bias, lin.bits), "tiny")
 
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
 @pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16])
 def test_small_path_ragged(bits, M):
-    X, W, bias = WL.random_case(M * 10 + bits, M, 400, 1152, bits, with_bias=True)
+    K = 1280 if bits == 1 else 1152  # 1-bit rows on the small path: K % 256 == 0
+    X, W, bias = WL.random_case(M * 10 + bits, M, 400, K, bits, with_bias=True)
     y, _ = gpu_qgemm(X, W, bias, bits, path=SMALL)
     _assert_close(y, _ref(X, W, bias, bits), f"small bits={bits} M={M}")
 
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
 @pytest.mark.parametrize("M,N,K", [(1, 128, 128), (17, 144, 256), (255, 272, 384), (256, 256, 512),
                                    (257, 400, 640), (600, 528, 1024)])
 def test_large_path_ragged(bits, M, N, K):
@@ -173,7 +180,7 @@ def test_m_zero_is_a_no_op():
 # every workload at full size, in the launch configuration the bench times
 # ----------------------------------------------------------------------------
 
-FULL = [(cid, li) for cid in (1, 2, 3, 4) for li in range(len(WL.workload(cid).linears))]
+FULL = [(cid, li) for cid in (1, 2, 3, 4, 5) for li in range(len(WL.workload(cid).linears))]
 
 
 @pytest.mark.parametrize("cid,li", FULL)
@@ -290,10 +297,10 @@ def _fused_case(bits, M, N, K, op, seed, path, in_place=False):
 
 
 @pytest.mark.parametrize("op", [wq.QGEMM_EPI_GELU_TANH, wq.QGEMM_EPI_RESIDUAL_GATE])
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
 @pytest.mark.parametrize("path,M", [(SMALL, 1), (SMALL, 13), (LARGE, 300)])
 def test_fused_epilogue_parity(op, bits, path, M):
-    y, ref = _fused_case(bits, M, 400, 640, op, 100 + 10 * op + bits + M, path)
+    y, ref = _fused_case(bits, M, 400, 768, op, 100 + 10 * op + bits + M, path)
     _assert_close(y, ref, f"op={op} bits={bits} path={path} M={M}")
 
 

@@ -15,7 +15,7 @@ def _same(W, bits):
     p, s, b = O.pack_ref(W, bits, group)
     assert np.array_equal(got.packed, p)
     assert np.array_equal(got.scales.view(np.uint16), s.view(np.uint16))
-    if bits == 2:
+    if bits <= 2:
         assert got.biases is None and b is None
     else:
         assert np.array_equal(got.biases.view(np.uint16), b.view(np.uint16))
@@ -33,6 +33,13 @@ def test_ternary_workload_weights():
     lin = WL.workload(3).linears[0]
     W = WL.make_w(3, 0, 512, lin.K, "ternary", 128)
     _same(W, 2)
+
+
+def test_binary_workload_weights():
+    lin = WL.workload(5).linears[1]
+    W = WL.make_w(5, 1, 512, lin.K, "binary", 128)
+    _same(W, 1)
+    _same((np.random.default_rng(4).standard_normal((64, 1024)) * 0.02).astype(np.float32), 1)
 
 
 def _edge_matrix(g, K, group):
@@ -53,14 +60,14 @@ def _edge_matrix(g, K, group):
     return W.astype(np.float32)
 
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
 def test_edge_groups(bits):
     g = np.random.default_rng(100 + bits)
     group = wq.GROUP_OF_BITS[bits]
     _same(_edge_matrix(g, 512, group), bits)
 
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
 def test_random_scales_wide_dynamic_range(bits):
     g = np.random.default_rng(7 * bits)
     K = 256

@@ -39,7 +39,7 @@ QGEMM_EPI_NONE = 0
 QGEMM_EPI_GELU_TANH = 1
 QGEMM_EPI_RESIDUAL_GATE = 2
 
-GROUP_OF_BITS = {2: 128, 4: 64, 8: 64}
+GROUP_OF_BITS = {1: 128, 2: 128, 4: 64, 8: 64}
 
 
 class QGemmError(RuntimeError):

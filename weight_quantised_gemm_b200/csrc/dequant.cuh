@@ -3,6 +3,7 @@
 // include/qgemm.h:
 //   affine   wdeq = bf16_rn(fp32(s) * q + fp32(b))   (product exact, one FMA)
 //   ternary  wdeq = t * bf16_rn(fp32(s))
+//   1-bit    wdeq = c * bf16_rn(fp32(s))
 // The large-M kernel applies these to every weight tile it stages in shared
 // memory; qgemm_dequant_tile exposes the same routines for the bit-exact gate.
 #pragma once
@@ -82,6 +83,42 @@ __device__ __forceinline__ uint4 chunk_ternary(uint32_t w, uint32_t half_scale2)
 
 __device__ __forceinline__ uint4 chunk_ternary_dyn(uint32_t w, int half, uint32_t half_scale2) {
   return half ? chunk_ternary<1>(w, half_scale2) : chunk_ternary<0>(w, half_scale2);
+}
+
+// 1-bit (Q1_0_g128): pair i of a 32-code word (in-word offsets 2i and 2i+1,
+// codes in bits i and 16+i; bit 1 = +1) as bf16x2 of +-sb: the scale's bf16
+// bits in both lanes with the sign bit set where the code bit is 0. The shift
+// brings bits i and 16+i to 15 and 31, the sign positions of the two lanes.
+template <int I>
+__device__ __forceinline__ uint32_t binary_pair(uint32_t w, uint32_t scale2) {
+  return ((~w << (15 - I)) & 0x80008000u) | scale2;
+}
+
+// bf16x2 of bf16_rn(fp32(s)) in both lanes.
+__device__ __forceinline__ uint32_t bf16_scale2(float s) {
+  const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+  return h | (h << 16);
+}
+
+// 1-bit: 8 consecutive k = quarter Q of a 32-code word (Q 0: k 0..7), each
+// weight exactly c * bf16_rn(s).
+template <int Q>
+__device__ __forceinline__ uint4 chunk_binary(uint32_t w, uint32_t scale2) {
+  uint4 o;
+  o.x = binary_pair<4 * Q + 0>(w, scale2);
+  o.y = binary_pair<4 * Q + 1>(w, scale2);
+  o.z = binary_pair<4 * Q + 2>(w, scale2);
+  o.w = binary_pair<4 * Q + 3>(w, scale2);
+  return o;
+}
+
+__device__ __forceinline__ uint4 chunk_binary_dyn(uint32_t w, int quarter, uint32_t scale2) {
+  switch (quarter) {
+    case 0: return chunk_binary<0>(w, scale2);
+    case 1: return chunk_binary<1>(w, scale2);
+    case 2: return chunk_binary<2>(w, scale2);
+    default: return chunk_binary<3>(w, scale2);
+  }
 }
 
 __device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }

@@ -12,7 +12,7 @@ template <int BITS>
 __global__ void dequant_tile_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ scales,
                                     const uint16_t* __restrict__ biases, int N, int K, int n0, int k0, int rows,
                                     int cols, uint4* __restrict__ out) {
-  constexpr int G = BITS == 2 ? 128 : 64;
+  constexpr int G = BITS <= 2 ? 128 : 64;
   const int chunks_per_row = cols / 8;
   const int64_t total = static_cast<int64_t>(rows) * chunks_per_row;
   const size_t row_bytes = static_cast<size_t>(K) * BITS / 8;
@@ -32,9 +32,12 @@ __global__ void dequant_tile_kernel(const uint8_t* __restrict__ packed, const ui
     } else if constexpr (BITS == 8) {
       const uint2 w = *reinterpret_cast<const uint2*>(row + k);
       o = deq::chunk_8bit(w.x, w.y, deq::h2f(scales[sidx]), deq::h2f(biases[sidx]));
-    } else {
+    } else if constexpr (BITS == 2) {
       const uint32_t w = *reinterpret_cast<const uint32_t*>(row + (k / 16) * 4);
       o = deq::chunk_ternary_dyn(w, (k / 8) & 1, deq::ternary_half_scale2(deq::h2f(scales[sidx])));
+    } else {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(row + (k / 32) * 4);
+      o = deq::chunk_binary_dyn(w, (k / 8) & 3, deq::bf16_scale2(deq::h2f(scales[sidx])));
     }
     out[idx] = o;
   }
@@ -58,6 +61,10 @@ int launch_dequant_tile(const Problem& p, int n0, int k0, int rows, int cols) {
       break;
     case 8:
       dequant_tile_kernel<8><<<blocks, threads, 0, p.stream>>>(p.packed, p.scales, p.biases, p.N, p.K, n0, k0, rows,
+                                                               cols, out);
+      break;
+    case 1:
+      dequant_tile_kernel<1><<<blocks, threads, 0, p.stream>>>(p.packed, p.scales, p.biases, p.N, p.K, n0, k0, rows,
                                                                cols, out);
       break;
     default:

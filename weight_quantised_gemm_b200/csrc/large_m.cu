@@ -93,20 +93,22 @@ static_assert(EPI_TOKENS % EPI_ROWS == 0, "epilogue warps cover whole tcgen05.ld
 
 template <int BITS>
 struct Cfg {
-  static constexpr int kGroup = BITS == 2 ? 128 : 64;
+  static constexpr int kGroup = BITS <= 2 ? 128 : 64;
   static constexpr int kGroupsPerStage = BK / kGroup;
   static constexpr int kWRowBytes = BK * BITS / 8;        // packed bytes per row per stage
   static constexpr int kSliceBytes = SLICE_K * BITS / 8;  // packed bytes per row per slice
   static constexpr int kWTileBytes = TILE_N * kWRowBytes;
-  // TMA swizzle of the packed tile: one row is exactly one swizzle span.
+  // TMA swizzle of the packed tile: one row is exactly one swizzle span (a
+  // 1-bit row of 16 bytes is below the smallest span: no swizzle).
   static constexpr CUtensorMapSwizzle kWSwizzle = BITS == 8   ? CU_TENSOR_MAP_SWIZZLE_128B
                                                   : BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                                              : CU_TENSOR_MAP_SWIZZLE_32B;
-  static constexpr uint32_t kSwzMask = BITS == 8 ? 7 : BITS == 4 ? 3 : 1;
+                                                  : BITS == 2 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                              : CU_TENSOR_MAP_SWIZZLE_NONE;
+  static constexpr uint32_t kSwzMask = BITS == 8 ? 7 : BITS == 4 ? 3 : BITS == 2 ? 1 : 0;
   static constexpr int kSBytes = kGroupsPerStage * TILE_N * 2;  // one stage's scales (or biases)
-  static constexpr int kSBStride = BITS == 2 ? kSBytes : 2 * kSBytes;
+  static constexpr int kSBStride = BITS <= 2 ? kSBytes : 2 * kSBytes;
   static constexpr int kS = BITS == 8 ? 2 : 3;                   // stage ring depth
-  static constexpr int kSW = BITS == 8 ? 3 : BITS == 4 ? 2 : 4;  // W ring depth
+  static constexpr int kSW = BITS == 8 ? 3 : BITS == 4 ? 2 : BITS == 2 ? 4 : 8;  // W ring depth
   static constexpr int kSlots = BITS == 8 ? 2 : 1;               // epilogue store slots per warp
   static constexpr int kOffX = 0;
   static constexpr int kOffW = kOffX + kS * X_STAGE_BYTES;
@@ -120,7 +122,7 @@ struct Cfg {
   static_assert(A_COL + kS * A_STAGE_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(kOffW % 1024 == 0 && kWTileBytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static_assert(kOffSB % 128 == 0 && kSBStride % 128 == 0 && kSBytes % 128 == 0, "TMA rows land on 128 B");
-  static_assert(kWRowBytes == 16 * (kSwzMask + 1), "one packed row is one swizzle span");
+  static_assert(kWRowBytes == 16 * (kSwzMask + 1), "one packed row is one swizzle span (or 16 bytes, unswizzled)");
 };
 
 struct Params {
@@ -216,7 +218,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == WARP_WLOAD && lane == 0) {
     ptx::tma_prefetch_desc(&tm_w);
     ptx::tma_prefetch_desc(&tm_s);
-    if (BITS != 2) ptx::tma_prefetch_desc(&tm_b);
+    if (BITS > 2) ptx::tma_prefetch_desc(&tm_b);
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -261,7 +263,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::mbar_arrive_expect_tx(full_w(s), C::kWTileBytes + C::kSBStride);
             ptx::tma_load_2d(wdst, &tm_w, kb * C::kWRowBytes, n_tile * TILE_N, full_w(s));
             ptx::tma_load_2d(sdst, &tm_s, n_tile * TILE_N, grp, full_w(s));
-            if (BITS != 2) ptx::tma_load_2d(sdst + C::kSBytes, &tm_b, n_tile * TILE_N, grp, full_w(s));
+            if (BITS > 2) ptx::tma_load_2d(sdst + C::kSBytes, &tm_b, n_tile * TILE_N, grp, full_w(s));
           }
         }
       }
@@ -343,7 +345,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int g = (j * SLICE_K) / C::kGroup;  // scale group of the slice within the stage
         const uint32_t w_off = static_cast<uint32_t>(r * C::kWRowBytes + j * C::kSliceBytes);
         const float s_cur = deq::h2f(sb[g * TILE_N + r]);
-        const float b_cur = BITS == 2 ? 0.f : deq::h2f(sb[C::kSBytes / 2 + g * TILE_N + r]);
+        const float b_cur = BITS <= 2 ? 0.f : deq::h2f(sb[C::kSBytes / 2 + g * TILE_N + r]);
         uint4 o[4];  // 4 chunks of 8 consecutive k = the slice's 32 k
         if constexpr (BITS == 4) {
           const uint4 v = *reinterpret_cast<const uint4*>(wt + swz<C::kSwzMask>(w_off));
@@ -358,6 +360,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           o[1] = deq::chunk_8bit(v0.z, v0.w, s_cur, b_cur);
           o[2] = deq::chunk_8bit(v1.x, v1.y, s_cur, b_cur);
           o[3] = deq::chunk_8bit(v1.z, v1.w, s_cur, b_cur);
+        } else if constexpr (BITS == 1) {
+          const uint32_t v = *reinterpret_cast<const uint32_t*>(wt + swz<C::kSwzMask>(w_off));
+          const uint32_t s2 = deq::bf16_scale2(s_cur);
+          o[0] = deq::chunk_binary<0>(v, s2);
+          o[1] = deq::chunk_binary<1>(v, s2);
+          o[2] = deq::chunk_binary<2>(v, s2);
+          o[3] = deq::chunk_binary<3>(v, s2);
         } else {
           const uint2 v = *reinterpret_cast<const uint2*>(wt + swz<C::kSwzMask>(w_off));
           const uint32_t hs = deq::ternary_half_scale2(s_cur);
@@ -505,7 +514,7 @@ int launch_fmt(const Problem& pr, int nsm) {
   if ((st = make_tensor_map_2d(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.scales, pr.N, groups, uint64_t(pr.N) * 2,
                                TILE_N, C::kGroupsPerStage, none, "scales")) != QGEMM_OK)
     return st;
-  if (BITS != 2) {
+  if (BITS > 2) {
     if ((st = make_tensor_map_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.biases, pr.N, groups, uint64_t(pr.N) * 2,
                                  TILE_N, C::kGroupsPerStage, none, "biases")) != QGEMM_OK)
       return st;
@@ -571,6 +580,7 @@ int launch_large_m(const Problem& p) {
   switch (p.bits) {
     case 4: return go(std::integral_constant<int, 4>{});
     case 8: return go(std::integral_constant<int, 8>{});
+    case 1: return go(std::integral_constant<int, 1>{});
     default: return go(std::integral_constant<int, 2>{});
   }
 }

@@ -42,11 +42,11 @@ int validate_weights(const qgemm_weights* W) {
   if (!W) return fail(QGEMM_ERR_INVALID_ARG, "null weights descriptor");
   if (W->N <= 0 || W->K <= 0) return fail(QGEMM_ERR_INVALID_ARG, "N=%d K=%d must be positive", W->N, W->K);
   const bool fmt_ok = (W->bits == 4 && W->group == 64) || (W->bits == 8 && W->group == 64) ||
-                      (W->bits == 2 && W->group == 128);
+                      (W->bits == 2 && W->group == 128) || (W->bits == 1 && W->group == 128);
   if (!fmt_ok) return fail(QGEMM_ERR_UNSUPPORTED, "unsupported format bits=%d group=%d", W->bits, W->group);
   if (W->K % 128) return fail(QGEMM_ERR_UNSUPPORTED, "K=%d is not a multiple of 128", W->K);
   if (W->N % 16) return fail(QGEMM_ERR_UNSUPPORTED, "N=%d is not a multiple of 16", W->N);
-  if (!W->packed || !W->scales || (W->bits != 2 && !W->biases))
+  if (!W->packed || !W->scales || (W->bits > 2 && !W->biases))
     return fail(QGEMM_ERR_INVALID_ARG, "null packed/scales/biases pointer");
   if (!aligned16(W->packed) || !aligned16(W->scales) || (W->biases && !aligned16(W->biases)))
     return fail(QGEMM_ERR_ALIGNMENT, "packed weights, scales and biases must be 16-byte aligned");
@@ -78,7 +78,9 @@ uint64_t wait_limit_ns() {
 int select_path(int M, int N, int K, int bits) {
   (void)N;
   (void)K;
-  const int lim = bits == 2 ? kSmallMaxTernary : bits == 4 ? kSmallMax4 : kSmallMax8;
+  // the small-M path streams 1-bit rows in pieces of at least 32 bytes: K % 256 == 0
+  if (bits == 1 && K % 256) return QGEMM_PATH_LARGE_M;
+  const int lim = bits == 1 ? kSmallMaxBinary : bits == 2 ? kSmallMaxTernary : bits == 4 ? kSmallMax4 : kSmallMax8;
   return M <= lim ? QGEMM_PATH_SMALL_M : QGEMM_PATH_LARGE_M;
 }
 
@@ -111,6 +113,8 @@ extern "C" int qgemm_fused(const void* X, int32_t M, const qgemm_weights* W, voi
   if (path == QGEMM_PATH_AUTO) path = select_path(M, W->N, W->K, W->bits);
   if (path == QGEMM_PATH_SMALL_M && M > 16)
     return fail(QGEMM_ERR_UNSUPPORTED, "the small-M path takes M <= 16 (M=%d)", M);
+  if (path == QGEMM_PATH_SMALL_M && W->bits == 1 && W->K % 256)
+    return fail(QGEMM_ERR_UNSUPPORTED, "the small-M path takes 1-bit weights with K %% 256 == 0 (K=%d)", W->K);
   Problem p{X, M, W->N, W->K, W->bits, W->group, static_cast<const uint8_t*>(W->packed),
             static_cast<const uint16_t*>(W->scales), static_cast<const uint16_t*>(W->biases), out,
             static_cast<const uint16_t*>(bias), static_cast<cudaStream_t>(stream),
@@ -131,7 +135,7 @@ extern "C" int qgemm(const void* X, int32_t M, const qgemm_weights* W, void* out
 
 extern "C" int qgemm_select_path(int32_t M, int32_t N, int32_t K, int32_t bits) {
   if (M < 0 || N <= 0 || K <= 0) return -QGEMM_ERR_INVALID_ARG;
-  if (bits != 2 && bits != 4 && bits != 8) return -QGEMM_ERR_UNSUPPORTED;
+  if (bits != 1 && bits != 2 && bits != 4 && bits != 8) return -QGEMM_ERR_UNSUPPORTED;
   std::call_once(g_env_once, read_env);
   if (g_env_path != QGEMM_PATH_AUTO) return g_env_path == QGEMM_PATH_SMALL_M && M > 16 ? QGEMM_PATH_LARGE_M : g_env_path;
   return select_path(M, N, K, bits);

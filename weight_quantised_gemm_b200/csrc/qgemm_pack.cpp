@@ -102,7 +102,16 @@ int pack_rows(const PackJob& jb, int r0, int r1) {
         if (!std::isfinite(wg[i])) return QGEMM_ERR_NONFINITE;
       }
       const size_t sidx = static_cast<size_t>(g) * jb.N + n;  // group-major [K/group, N]
-      if (bits == 2) {
+      if (bits == 1) {
+        // Q1_0_g128: one sign bit per weight (1 = +1, for w >= 0 and -0),
+        // s16 = fp16(mean |w|), the least-squares scale for fixed signs
+        double sum = 0.0;
+        for (int i = 0; i < G; ++i) sum += std::fabs(static_cast<double>(wg[i]));
+        const uint16_t s16 = f64_to_f16_rn(sum / G);
+        if (!is_f16_finite(s16)) return QGEMM_ERR_UNSUPPORTED;
+        jb.scales[sidx] = s16;
+        for (int i = 0; i < G; ++i) codes[i] = wg[i] >= 0.f ? 1 : 0;
+      } else if (bits == 2) {
         double amax = 0.0;
         for (int i = 0; i < G; ++i) amax = std::max(amax, std::fabs(static_cast<double>(wg[i])));
         const uint16_t s16 = f64_to_f16_rn(amax);
@@ -147,7 +156,8 @@ int pack_rows(const PackJob& jb, int r0, int r1) {
 
 int check_format(int32_t N, int32_t K, int32_t bits, int32_t group) {
   if (N <= 0 || K <= 0) return qg::fail(QGEMM_ERR_INVALID_ARG, "N and K must be positive (N=%d K=%d)", N, K);
-  const bool ok = (bits == 4 && group == 64) || (bits == 8 && group == 64) || (bits == 2 && group == 128);
+  const bool ok = (bits == 4 && group == 64) || (bits == 8 && group == 64) || (bits == 2 && group == 128) ||
+                  (bits == 1 && group == 128);
   if (!ok) return qg::fail(QGEMM_ERR_UNSUPPORTED, "unsupported format bits=%d group=%d", bits, group);
   if (K % 128) return qg::fail(QGEMM_ERR_UNSUPPORTED, "K=%d is not a multiple of 128", K);
   return QGEMM_OK;
@@ -163,7 +173,7 @@ extern "C" int qgemm_pack_sizes(int32_t N, int32_t K, int32_t bits, int32_t grou
   if (st != QGEMM_OK) return st;
   *packed_bytes = static_cast<size_t>(N) * K * bits / 8;
   *scales_bytes = static_cast<size_t>(N) * (K / group) * 2;
-  *biases_bytes = bits == 2 ? 0 : *scales_bytes;
+  *biases_bytes = bits <= 2 ? 0 : *scales_bytes;
   return QGEMM_OK;
 }
 
@@ -171,7 +181,7 @@ extern "C" int qgemm_pack(const float* W, int32_t N, int32_t K, int32_t bits, in
                           void* scales, void* biases) {
   const int st = check_format(N, K, bits, group);
   if (st != QGEMM_OK) return st;
-  if (!W || !packed || !scales || (bits != 2 && !biases))
+  if (!W || !packed || !scales || (bits > 2 && !biases))
     return qg::fail(QGEMM_ERR_INVALID_ARG, "null buffer passed to qgemm_pack");
   if (reinterpret_cast<uintptr_t>(packed) % 4)
     return qg::fail(QGEMM_ERR_ALIGNMENT, "packed buffer must be 4-byte aligned");

@@ -71,7 +71,7 @@ constexpr int GS = 8;                   // scale groups per stage
 
 template <int BITS>
 struct Fmt {
-  static constexpr int G = BITS == 2 ? 128 : 64;  // group size
+  static constexpr int G = BITS <= 2 ? 128 : 64;  // group size
   static constexpr int GBYTES = G * BITS / 8;     // packed bytes per row and group
   static constexpr int KS = GS * G;               // k per stage
   static constexpr int ROWB = GS * GBYTES;        // packed bytes per row and stage
@@ -133,7 +133,8 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_
 template <int BITS>
 __device__ __forceinline__ int word_offset(int gs, int k, int c) {
   constexpr int GB = Fmt<BITS>::GBYTES;
-  if constexpr (BITS == 2) return gs * GB + 4 * k;
+  if constexpr (BITS == 1) return gs * GB + 4 * (k >> 1);  // one word per two steps
+  else if constexpr (BITS == 2) return gs * GB + 4 * k;
   else if constexpr (BITS == 4) return gs * GB + 8 * k + 4 * (c >> 1);
   else return gs * GB + 16 * k + 4 * c;
 }
@@ -156,8 +157,14 @@ __device__ __forceinline__ int piece_offset(int off, int ush, int key16) {
 // B operand of one step for quad thread c from its word: codes 4c .. 4c+3 as
 // two bf16x2 registers (k pairs (4c, 4c+1) and (4c+2, 4c+3)).
 template <int BITS>
-__device__ __forceinline__ void decode_word(uint32_t x, int c, uint32_t& b0, uint32_t& b1) {
-  if constexpr (BITS == 2) {
+__device__ __forceinline__ void decode_word(uint32_t x, int c, int k, uint32_t& b0, uint32_t& b1) {
+  if constexpr (BITS == 1) {
+    // pairs 8(k%2) + 2c and +1 of the 32-code word: bf16 {-1, +1}, the sign
+    // set where the code bit is 0 (bits i and 16+i moved to 15 and 31)
+    const int i0 = 8 * (k & 1) + 2 * c;
+    b0 = ((~x << (15 - i0)) & 0x80008000u) | 0x3F803F80u;
+    b1 = ((~x << (14 - i0)) & 0x80008000u) | 0x3F803F80u;
+  } else if constexpr (BITS == 2) {
     // pairs 2c and 2c+1 of the 16-code word: bf16 {-2, 0, +2}
     b0 = (x << (14 - 4 * c)) & 0xC000C000u;
     b1 = (x << (12 - 4 * c)) & 0xC000C000u;
@@ -251,10 +258,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int kt, valid;
       stage_k(t, kt, valid);
       const uint32_t st = sbase + s * p.stage_bytes;
-      ptx::mbar_arrive_expect_tx(full(s), R * F::ROWB + sb_bytes * (BITS == 2 ? 1 : 2) + p.M * valid * 2);
+      ptx::mbar_arrive_expect_tx(full(s), R * F::ROWB + sb_bytes * (BITS <= 2 ? 1 : 2) + p.M * valid * 2);
       ptx::tma_load_3d(st, &tm_w, 0, n0, kt * units, full(s));
       ptx::tma_load_2d(st + p.off_s, &tm_s, n0, kt * GS, full(s));
-      if (BITS != 2) ptx::tma_load_2d(st + p.off_b, &tm_b, n0, kt * GS, full(s));
+      if (BITS > 2) ptx::tma_load_2d(st + p.off_b, &tm_b, n0, kt * GS, full(s));
     };
     auto load_x = [&](int t, int s) {  // all lanes: one bulk copy per token row
       int kt, valid;
@@ -267,7 +274,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       ptx::tma_prefetch_desc(&tm_w);
       ptx::tma_prefetch_desc(&tm_s);
-      if (BITS != 2) ptx::tma_prefetch_desc(&tm_b);
+      if (BITS > 2) ptx::tma_prefetch_desc(&tm_b);
     }
     if (p.overlap) {
       // The weights do not depend on the previous grid: put the first stages
@@ -343,7 +350,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int k = 0; k < STEPS; ++k) {
           const uint2 x0 = ga ? *reinterpret_cast<const uint2*>(xg + 32 * k) : make_uint2(0u, 0u);
           const uint2 x1 = gb ? *reinterpret_cast<const uint2*>(xg + 8 * p.x_stride + 32 * k) : make_uint2(0u, 0u);
-          if constexpr (BITS != 2) {
+          if constexpr (BITS > 2) {
             const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};
             mma_bf16_16816(xs[0], ones, x0.x, x0.y);
             if constexpr (TH > 1) mma_bf16_16816(xs[TH - 1], ones, x1.x, x1.y);
@@ -356,8 +363,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t w0 = *reinterpret_cast<const uint32_t*>(wk + (r0 << ush));
             const uint32_t w1 = *reinterpret_cast<const uint32_t*>(wk + ((r0 + 8) << ush));
             uint32_t a[4];
-            decode_word<BITS>(w0, c, a[0], a[2]);  // row g: k pairs (4c, 4c+1), (4c+2, 4c+3)
-            decode_word<BITS>(w1, c, a[1], a[3]);  // row g + 8
+            decode_word<BITS>(w0, c, k, a[0], a[2]);  // row g: k pairs (4c, 4c+1), (4c+2, 4c+3)
+            decode_word<BITS>(w1, c, k, a[1], a[3]);  // row g + 8
             mma_bf16_16816(tmp[q][0], a, x0.x, x0.y);
             if constexpr (TH > 1) mma_bf16_16816(tmp[q][TH - 1], a, x1.x, x1.y);
           }
@@ -370,7 +377,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int r0 = 16 * (q0 + q) + g;
           const float s2[2] = {deq::h2f(sc[r0]), deq::h2f(sc[r0 + 8])};
           float b2[2] = {0.f, 0.f};
-          if constexpr (BITS != 2) {
+          if constexpr (BITS > 2) {
             b2[0] = deq::h2f(bi[r0]);
             b2[1] = deq::h2f(bi[r0 + 8]);
           }
@@ -379,7 +386,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const float sj = s2[j >> 1];
-              if constexpr (BITS == 2) {
+              if constexpr (BITS == 1) {
+                acc[q][h][j] = fmaf(sj, tmp[q][h][j], acc[q][h][j]);
+              } else if constexpr (BITS == 2) {
                 acc[q][h][j] = fmaf(0.5f * sj, tmp[q][h][j], acc[q][h][j]);
               } else {
                 const float d = BITS == 4 ? fmaf(-128.f, xs[h][j], tmp[q][h][j]) : tmp[q][h][j];
@@ -457,13 +466,14 @@ int launch_fmt(const Problem& pr, int grid) {
   const uint64_t wbytes = static_cast<uint64_t>(pr.K) * BITS / 8;  // packed bytes per weight row
   const int unit = wbytes % 128 == 0 ? 128 : wbytes % 64 == 0 ? 64 : 32;  // K % 128 == 0 makes it at least 32
   kp.unit_shift = unit == 128 ? 7 : unit == 64 ? 6 : 5;
-  if (F::ROWB % unit) return fail(QGEMM_ERR_UNSUPPORTED, "internal: small-M stage is not whole row pieces");
+  if (F::ROWB % unit || wbytes % unit)
+    return fail(QGEMM_ERR_UNSUPPORTED, "internal: small-M rows are not whole %d-byte pieces", unit);
   const int sb = GS * R * 2;
   // TMA tile destinations start on 128-byte boundaries (the packed box on a
   // 1024-byte one, for its swizzle); bulk copies need 16 bytes.
   kp.off_s = R * F::ROWB;
   kp.off_b = (kp.off_s + sb + 127) & ~127;
-  kp.off_x = (kp.off_b + (BITS == 2 ? 0 : sb) + 127) & ~127;
+  kp.off_x = (kp.off_b + (BITS <= 2 ? 0 : sb) + 127) & ~127;
   kp.x_stride = F::KS * 2 + 32;  // +32 B: token rows 8 banks apart, so the 8-byte B fetches do not collide
   kp.stage_bytes = (kp.off_x + pr.M * kp.x_stride + 1023) & ~1023;
   int ring = RING_BUDGET / kp.stage_bytes;
@@ -497,7 +507,7 @@ int launch_fmt(const Problem& pr, int grid) {
   if ((st = make_tensor_map_2d(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.scales, pr.N, groups,
                                uint64_t(pr.N) * 2, R, GS, CU_TENSOR_MAP_SWIZZLE_NONE, "scales")) != QGEMM_OK)
     return st;
-  if (BITS != 2) {
+  if (BITS > 2) {
     if ((st = make_tensor_map_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.biases, pr.N, groups,
                                  uint64_t(pr.N) * 2, R, GS, CU_TENSOR_MAP_SWIZZLE_NONE, "biases")) != QGEMM_OK)
       return st;
@@ -550,6 +560,7 @@ int launch_small_m(const Problem& p) {
   switch (p.bits) {
     case 4: return sm::launch_bits<4>(p, nsm);
     case 8: return sm::launch_bits<8>(p, nsm);
+    case 1: return sm::launch_bits<1>(p, nsm);
     default: return sm::launch_bits<2>(p, nsm);
   }
 }
