@@ -138,6 +138,18 @@ int qgemm_pack(const float* W, int32_t N, int32_t K, int32_t bits, int32_t group
                void* packed, void* scales, void* biases);
 
 /*
+ * qgemm_pack on the GPU: the same packing of a device fp32 matrix W [N, K]
+ * (row-major) into caller-allocated device buffers, bit-identical to
+ * qgemm_pack's output (same fp64 steps in the same order). Enqueued on
+ * `stream`; a non-finite weight or an fp16 overflow is reported later by
+ * qgemm_get_device_status as QGEMM_ERR_NONFINITE or QGEMM_ERR_UNSUPPORTED.
+ * All pointers 16-byte aligned; biases may be NULL for 1-bit and ternary.
+ * Argument errors are those of qgemm_pack_sizes, plus INVALID_ARG / ALIGNMENT.
+ */
+int qgemm_pack_device(const void* W, int32_t N, int32_t K, int32_t bits, int32_t group,
+                      void* packed, void* scales, void* biases, void* stream);
+
+/*
  * out = X . dequant(W)^T (+ bias), enqueued on `stream`.
  *   X     device bf16 [M, K] row-major, 16-byte aligned
  *   M     tokens (rows of X); M = 0 is a no-op returning OK

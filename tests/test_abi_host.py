@@ -179,3 +179,19 @@ def test_fused_rejects_bad_epilogues_without_device():
         assert _fused(d, op, M=0) == wq.QGEMM_OK
     # a NULL epilogue is plain qgemm_ex
     assert wq._lib.qgemm_fused(0x10000, 0, ctypes.byref(d), 0x20000, None, None, 0, None) == wq.QGEMM_OK
+
+
+def test_pack_device_rejects_bad_arguments_without_device():
+    f = wq._lib.qgemm_pack_device
+    ok = dict(W=0x1000, N=16, K=128, bits=4, group=64, p=0x2000, s=0x3000, b=0x4000)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["W"], a["N"], a["K"], a["bits"], a["group"], a["p"], a["s"], a["b"], None)
+    assert call(bits=3) == wq.QGEMM_ERR_UNSUPPORTED
+    assert call(K=192) == wq.QGEMM_ERR_UNSUPPORTED
+    assert call(N=0) == wq.QGEMM_ERR_INVALID_ARG
+    assert call(W=None) == wq.QGEMM_ERR_INVALID_ARG
+    assert call(b=None) == wq.QGEMM_ERR_INVALID_ARG            # affine needs biases
+    assert call(W=0x1004) == wq.QGEMM_ERR_ALIGNMENT
+    assert call(s=0x3002) == wq.QGEMM_ERR_ALIGNMENT

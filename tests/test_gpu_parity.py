@@ -337,3 +337,57 @@ def test_fused_gelu_mlp_up_full_size_sampled_rows():
     rows = np.arange(0, lin.M, 257)
     ref = O.gelu_tanh_ref(O.qgemm_ref_rows(rows, X, p, s, b, lin.bits, lin.group, lin.K, None))
     _assert_close(y[rows], ref, "mlp_up + gelu sampled rows")
+
+
+# ----------------------------------------------------------------------------
+# packing on the device: the host packer's bytes, bit for bit
+# ----------------------------------------------------------------------------
+
+def _edge_rows(g, K):
+    rows = [np.zeros(K), np.full(K, -0.0), np.resize([0.0, -0.0], K), np.full(K, 0.125),
+            g.standard_normal(K) * 1e-7, g.standard_normal(K) * 1e-9, g.standard_normal(K) * 1000.0,
+            np.resize([-1.0, 1.0], K), np.resize(np.arange(64) * 0.5 - 3.75, K),
+            np.resize([0.0, 1e-30, -1e-30, 3.0], K)]
+    return np.concatenate([np.stack(rows), g.standard_normal((22, K)) * 0.02]).astype(np.float32)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
+def test_pack_device_matches_host_packer(bits):
+    g = np.random.default_rng(300 + bits)
+    K = 1024
+    if bits == 1:
+        W = np.concatenate([WL.make_w(5, 1, 96, K, "binary", 128), _edge_rows(g, K)])
+    elif bits == 2:
+        W = np.concatenate([WL.make_w(3, 0, 96, K, "ternary", 128), _edge_rows(g, K)])
+    else:
+        W = np.concatenate([WL.make_w(1, 0, 96, K, "normal"), _edge_rows(g, K)])
+    host = wq.qgemm_pack(W, bits)
+    dev = wq.qgemm_pack_device(torch.from_numpy(W).cuda(), bits)
+    wq.check_device_status()
+    assert np.array_equal(dev.packed.cpu().numpy(), host.packed)
+    assert np.array_equal(dev.scales.cpu().numpy().view(np.uint16).reshape(host.scales.shape),
+                          host.scales.view(np.uint16))
+    if bits > 2:
+        assert np.array_equal(dev.biases.cpu().numpy().view(np.uint16).reshape(host.biases.shape),
+                              host.biases.view(np.uint16))
+    # and the device-packed weights run the GEMM like the host-packed ones
+    X, _, bias = WL.random_case(bits, 5, W.shape[0], K, bits, with_bias=True)
+    Xd, bd = to_dev_bf16(X), to_dev_bf16(bias)
+    y1 = wq.qgemm(Xd, dev, bias=bd)
+    y2 = wq.qgemm(Xd, host.to_device(), bias=bd)
+    wq.check_device_status()
+    assert torch.equal(y1, y2)
+
+
+def test_pack_device_reports_bad_data_through_the_status_word():
+    W = torch.zeros((16, 128), dtype=torch.float32, device="cuda")
+    W[3, 7] = float("nan")
+    wq.qgemm_pack_device(W, 4)
+    assert wq.qgemm_get_device_status() == wq.QGEMM_ERR_NONFINITE
+    W[3, 7] = 0.0
+    W[0, 0], W[0, 1] = -7e5, 7e5          # range / 15 overflows fp16
+    wq.qgemm_pack_device(W, 4)
+    assert wq.qgemm_get_device_status() == wq.QGEMM_ERR_UNSUPPORTED
+    W[0, 0], W[0, 1] = 0.0, 0.0
+    wq.qgemm_pack_device(W, 4)
+    assert wq.qgemm_get_device_status() == wq.QGEMM_OK

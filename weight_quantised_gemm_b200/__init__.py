@@ -68,6 +68,7 @@ def _load():
         "qgemm_pack_sizes": (ctypes.c_int, [i32, i32, i32, i32, ctypes.POINTER(sz), ctypes.POINTER(sz),
                                             ctypes.POINTER(sz)]),
         "qgemm_pack": (ctypes.c_int, [vp, i32, i32, i32, i32, vp, vp, vp]),
+        "qgemm_pack_device": (ctypes.c_int, [vp, i32, i32, i32, i32, vp, vp, vp, vp]),
         "qgemm": (ctypes.c_int, [vp, i32, W, vp, vp, vp]),
         "qgemm_ex": (ctypes.c_int, [vp, i32, W, vp, vp, i32, vp]),
         "qgemm_fused": (ctypes.c_int, [vp, i32, W, vp, vp, ctypes.POINTER(_Epilogue), i32, vp]),
@@ -98,7 +99,8 @@ class _LazyLib:
 
 
 _lib = _LazyLib()
-EXPORTED = ("qgemm_pack_sizes", "qgemm_pack", "qgemm", "qgemm_ex", "qgemm_fused", "qgemm_select_path",
+EXPORTED = ("qgemm_pack_sizes", "qgemm_pack", "qgemm_pack_device", "qgemm", "qgemm_ex", "qgemm_fused",
+            "qgemm_select_path",
             "qgemm_dequant_tile",
             "qgemm_get_device_status", "qgemm_set_wait_limit_ns", "qgemm_debug_wait_timeout",
             "qgemm_status_str", "qgemm_last_error", "qgemm_version")
@@ -193,6 +195,25 @@ def qgemm_pack(W, bits: int, group: Optional[int] = None) -> PackedWeights:
                            None if biases is None else biases.ctypes.data), "qgemm_pack")
     return PackedWeights(N, K, bits, group, packed.reshape(N, -1), scales.reshape(K // group, N),
                          None if biases is None else biases.reshape(K // group, N))
+
+
+def qgemm_pack_device(W, bits: int, group: Optional[int] = None, stream=None) -> "DeviceWeights":
+    """RTN-quantise a device fp32 W [N, K] on the GPU (C ABI qgemm_pack_device):
+    the same bytes as qgemm_pack. Errors in the data surface through
+    check_device_status."""
+    import torch
+    if W.dtype != torch.float32 or not W.is_cuda or W.dim() != 2 or not W.is_contiguous():
+        raise ValueError("W must be a contiguous 2-D fp32 CUDA tensor")
+    N, K = W.shape
+    group = GROUP_OF_BITS.get(bits, 0) if group is None else group
+    pb, sb, bb = qgemm_pack_sizes(N, K, bits, group)
+    packed = torch.empty(pb, dtype=torch.uint8, device=W.device)
+    scales = torch.empty(sb // 2, dtype=torch.int16, device=W.device)
+    biases = torch.empty(bb // 2, dtype=torch.int16, device=W.device) if bb else None
+    _check(_lib.qgemm_pack_device(W.data_ptr(), N, K, bits, group, packed.data_ptr(), scales.data_ptr(),
+                                  None if biases is None else biases.data_ptr(), _stream_handle(stream)),
+           "qgemm_pack_device")
+    return DeviceWeights(N, K, bits, group, packed.view(N, -1), scales, biases)
 
 
 def _stream_handle(stream) -> Optional[int]:

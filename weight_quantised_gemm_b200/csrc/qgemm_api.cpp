@@ -129,6 +129,19 @@ extern "C" int qgemm_ex(const void* X, int32_t M, const qgemm_weights* W, void* 
   return qgemm_fused(X, M, W, out, bias, nullptr, path, stream);
 }
 
+extern "C" int qgemm_pack_device(const void* W, int32_t N, int32_t K, int32_t bits, int32_t group, void* packed,
+                                 void* scales, void* biases, void* stream) {
+  size_t pb, sb, bb;
+  int st = qgemm_pack_sizes(N, K, bits, group, &pb, &sb, &bb);
+  if (st != QGEMM_OK) return st;
+  if (!W || !packed || !scales || (bits > 2 && !biases))
+    return fail(QGEMM_ERR_INVALID_ARG, "null buffer passed to qgemm_pack_device");
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(scales) || (bits > 2 && !aligned16(biases)))
+    return fail(QGEMM_ERR_ALIGNMENT, "W, packed, scales and biases must be 16-byte aligned");
+  return launch_pack_device(static_cast<const float*>(W), N, K, bits, packed, static_cast<uint16_t*>(scales),
+                            static_cast<uint16_t*>(biases), static_cast<cudaStream_t>(stream));
+}
+
 extern "C" int qgemm(const void* X, int32_t M, const qgemm_weights* W, void* out, const void* bias, void* stream) {
   return qgemm_ex(X, M, W, out, bias, QGEMM_PATH_AUTO, stream);
 }

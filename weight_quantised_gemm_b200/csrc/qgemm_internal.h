@@ -57,9 +57,13 @@ int launch_small_m(const Problem& p);
 int launch_large_m(const Problem& p);
 int launch_dequant_tile(const Problem& p, int n0, int k0, int rows, int cols);
 int launch_debug_wait(uint64_t limit_ns, cudaStream_t stream);
+int launch_pack_device(const float* W, int N, int K, int bits, void* packed, uint16_t* scales, uint16_t* biases,
+                       cudaStream_t stream);
 
 // Device status word values (0 = fine).
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusLayout = 2u;  // dynamic shared memory not aligned as the kernel requires
+constexpr unsigned kStatusPackNonfinite = 4u;  // qgemm_pack_device met a NaN or an infinity
+constexpr unsigned kStatusPackOverflow = 8u;   // qgemm_pack_device: a scale or bias overflows fp16
 
 }  // namespace qg

@@ -99,6 +99,11 @@ extern "C" int qgemm_get_device_status(void* stream) {
     const unsigned int zero = 0;
     st = cuda_check(cudaMemcpyToSymbol(g_status_word, &zero, sizeof zero), "clear status word");
     if (st != QGEMM_OK) return st;
+    if (v & kStatusPackNonfinite)
+      return fail(QGEMM_ERR_NONFINITE, "qgemm_pack_device met a non-finite weight (status word 0x%x)", v);
+    if (v & kStatusPackOverflow)
+      return fail(QGEMM_ERR_UNSUPPORTED, "qgemm_pack_device: a group's scale or bias overflows fp16 (status word 0x%x)",
+                  v);
     if (v & kStatusLayout)
       return fail(QGEMM_ERR_CUDA, "a kernel found its shared-memory base off its alignment (status word 0x%x)", v);
     return fail(QGEMM_ERR_DEVICE_TIMEOUT, "a kernel gave up a bounded wait (status word 0x%x)", v);
