@@ -150,6 +150,22 @@ int qgemm_pack_device(const void* W, int32_t N, int32_t K, int32_t bits, int32_t
                       void* packed, void* scales, void* biases, void* stream);
 
 /*
+ * The at-rest file of a packed weight (host buffers): magic "QGEMMW01", then
+ * int32 N, K, bits, group and uint64 packed_bytes, scales_bytes,
+ * biases_bytes (little-endian), then the three arrays in that order.
+ * qgemm_save writes one; qgemm_load_header reads its shape and format (check
+ * them, size buffers with qgemm_pack_sizes); qgemm_load fills caller-
+ * allocated host buffers (biases may be NULL for 1-bit and ternary). A bad
+ * magic, sizes that do not match the format, a short or overlong file, or an
+ * I/O failure return QGEMM_ERR_INVALID_ARG (format errors: those of
+ * qgemm_pack_sizes). No counterpart as an interface in the pages.
+ */
+int qgemm_save(const char* path, int32_t N, int32_t K, int32_t bits, int32_t group,
+               const void* packed, const void* scales, const void* biases);
+int qgemm_load_header(const char* path, int32_t* N, int32_t* K, int32_t* bits, int32_t* group);
+int qgemm_load(const char* path, void* packed, void* scales, void* biases);
+
+/*
  * out = X . dequant(W)^T (+ bias), enqueued on `stream`.
  *   X     device bf16 [M, K] row-major, 16-byte aligned
  *   M     tokens (rows of X); M = 0 is a no-op returning OK

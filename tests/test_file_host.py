@@ -1,0 +1,59 @@
+"""The at-rest file (qgemm_save / qgemm_load_header / qgemm_load) on the host:
+round trips of every format, and the documented rejections."""
+import os
+import struct
+
+import numpy as np
+import pytest
+
+import oracle as O
+import weight_quantised_gemm_b200 as wq
+import workloads as WL
+
+
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
+def test_round_trip_every_format(tmp_path, bits):
+    W = WL.random_case(7, 1, 48, 512, bits, with_bias=False)[1]
+    pw = wq.qgemm_pack(W, bits)
+    path = str(tmp_path / f"w{bits}.qgw")
+    pw.save(path)
+    back = wq.qgemm_load(path)
+    assert (back.N, back.K, back.bits, back.group) == (48, 512, bits, wq.GROUP_OF_BITS[bits])
+    assert np.array_equal(back.packed, pw.packed)
+    assert np.array_equal(back.scales.view(np.uint16), pw.scales.view(np.uint16))
+    if bits > 2:
+        assert np.array_equal(back.biases.view(np.uint16), pw.biases.view(np.uint16))
+    else:
+        assert back.biases is None
+    # the file is exactly header + arrays, and the arrays are the oracle's
+    p, s, b = O.pack_ref(W, bits, wq.GROUP_OF_BITS[bits])
+    size = 48 + p.nbytes + s.nbytes + (0 if b is None else b.nbytes)
+    assert os.path.getsize(path) == size
+    with open(path, "rb") as f:
+        head = f.read(48)
+    assert head[:8] == b"QGEMMW01"
+    assert struct.unpack("<4i3Q", head[8:]) == (48, 512, bits, wq.GROUP_OF_BITS[bits], p.nbytes, s.nbytes,
+                                                 0 if b is None else b.nbytes)
+
+
+def _expect(path, status):
+    with pytest.raises(wq.QGemmError) as e:
+        wq.qgemm_load(path)
+    assert e.value.status == status
+
+
+def test_rejects_corrupt_files(tmp_path):
+    pw = wq.qgemm_pack(WL.random_case(8, 1, 32, 256, 4, with_bias=False)[1], 4)
+    good = str(tmp_path / "good.qgw")
+    pw.save(good)
+    data = open(good, "rb").read()
+    bad = str(tmp_path / "bad.qgw")
+    for blob, status in [(b"XGEMMW01" + data[8:], wq.QGEMM_ERR_INVALID_ARG),        # magic
+                         (data[:40], wq.QGEMM_ERR_INVALID_ARG),                     # short header
+                         (data[:-1], wq.QGEMM_ERR_INVALID_ARG),                     # truncated arrays
+                         (data + b"\0", wq.QGEMM_ERR_INVALID_ARG),                  # trailing bytes
+                         (data[:8] + struct.pack("<4i", 32, 256, 3, 64) + data[24:], wq.QGEMM_ERR_UNSUPPORTED),
+                         (data[:24] + struct.pack("<Q", 1) + data[32:], wq.QGEMM_ERR_INVALID_ARG)]:  # sizes
+        open(bad, "wb").write(blob)
+        _expect(bad, status)
+    _expect(str(tmp_path / "missing.qgw"), wq.QGEMM_ERR_INVALID_ARG)

@@ -69,6 +69,10 @@ def _load():
                                             ctypes.POINTER(sz)]),
         "qgemm_pack": (ctypes.c_int, [vp, i32, i32, i32, i32, vp, vp, vp]),
         "qgemm_pack_device": (ctypes.c_int, [vp, i32, i32, i32, i32, vp, vp, vp, vp]),
+        "qgemm_save": (ctypes.c_int, [ctypes.c_char_p, i32, i32, i32, i32, vp, vp, vp]),
+        "qgemm_load_header": (ctypes.c_int, [ctypes.c_char_p, ctypes.POINTER(i32), ctypes.POINTER(i32),
+                                             ctypes.POINTER(i32), ctypes.POINTER(i32)]),
+        "qgemm_load": (ctypes.c_int, [ctypes.c_char_p, vp, vp, vp]),
         "qgemm": (ctypes.c_int, [vp, i32, W, vp, vp, vp]),
         "qgemm_ex": (ctypes.c_int, [vp, i32, W, vp, vp, i32, vp]),
         "qgemm_fused": (ctypes.c_int, [vp, i32, W, vp, vp, ctypes.POINTER(_Epilogue), i32, vp]),
@@ -99,7 +103,8 @@ class _LazyLib:
 
 
 _lib = _LazyLib()
-EXPORTED = ("qgemm_pack_sizes", "qgemm_pack", "qgemm_pack_device", "qgemm", "qgemm_ex", "qgemm_fused",
+EXPORTED = ("qgemm_pack_sizes", "qgemm_pack", "qgemm_pack_device", "qgemm_save", "qgemm_load_header",
+            "qgemm_load", "qgemm", "qgemm_ex", "qgemm_fused",
             "qgemm_select_path",
             "qgemm_dequant_tile",
             "qgemm_get_device_status", "qgemm_set_wait_limit_ns", "qgemm_debug_wait_timeout",
@@ -149,6 +154,12 @@ class PackedWeights:
     @property
     def nbytes(self) -> int:
         return self.packed.nbytes + self.scales.nbytes + (0 if self.biases is None else self.biases.nbytes)
+
+    def save(self, path: str) -> None:
+        """Writes the at-rest file (C ABI qgemm_save)."""
+        _check(_lib.qgemm_save(os.fsencode(path), self.N, self.K, self.bits, self.group, self.packed.ctypes.data,
+                               self.scales.ctypes.data, None if self.biases is None else self.biases.ctypes.data),
+               "qgemm_save")
 
     def to_device(self, device="cuda") -> "DeviceWeights":
         import torch
@@ -214,6 +225,23 @@ def qgemm_pack_device(W, bits: int, group: Optional[int] = None, stream=None) ->
                                   None if biases is None else biases.data_ptr(), _stream_handle(stream)),
            "qgemm_pack_device")
     return DeviceWeights(N, K, bits, group, packed.view(N, -1), scales, biases)
+
+
+def qgemm_load(path: str) -> PackedWeights:
+    """Reads an at-rest file written by qgemm_save (C ABI qgemm_load_header + qgemm_load)."""
+    N, K, bits, group = (ctypes.c_int32() for _ in range(4))
+    p = os.fsencode(path)
+    _check(_lib.qgemm_load_header(p, ctypes.byref(N), ctypes.byref(K), ctypes.byref(bits), ctypes.byref(group)),
+           "qgemm_load_header")
+    N, K, bits, group = N.value, K.value, bits.value, group.value
+    pb, sb, bb = qgemm_pack_sizes(N, K, bits, group)
+    packed = np.empty(pb, dtype=np.uint8)
+    scales = np.empty(sb // 2, dtype=np.float16)
+    biases = np.empty(bb // 2, dtype=np.float16) if bb else None
+    _check(_lib.qgemm_load(p, packed.ctypes.data, scales.ctypes.data, None if biases is None else biases.ctypes.data),
+           "qgemm_load")
+    return PackedWeights(N, K, bits, group, packed.reshape(N, -1), scales.reshape(K // group, N),
+                         None if biases is None else biases.reshape(K // group, N))
 
 
 def _stream_handle(stream) -> Optional[int]:
