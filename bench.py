@@ -659,6 +659,54 @@ def fused_sweep():
     return rows
 
 
+def policy_sweep():
+    """Every assignment of 4 or 8 bits to the five linears of the mixed FLUX
+    block (workload 4), on its synthetic weights: the block's cosine against
+    dense bf16 (outputs concatenated) and its packed size, with the Pareto
+    front marked. The pages' policy (the layers that multiply the residual
+    stream at 8 bits, the rest at 4) is one of the 32."""
+    import itertools
+
+    import torch
+
+    import weight_quantised_gemm_b200 as wq
+    import workloads as WL
+    wl = WL.workload(4)
+    yq, yd, sizes = {}, [], {}
+    for li, lin in enumerate(wl.linears):
+        X, W, bias = WL.make_inputs(lin, 4, li)
+        Xd = torch.from_numpy(X.view("int16")).cuda().view(torch.bfloat16)
+        bd = None if bias is None else torch.from_numpy(bias.view("int16")).cuda().view(torch.bfloat16)
+        Wb = torch.from_numpy(W).cuda().to(torch.bfloat16)
+        yd.append((Xd @ Wb.T).double().flatten() if bd is None else (Xd @ Wb.T + bd).double().flatten())
+        del Wb
+        for bits in (4, 8):
+            dw = wq.qgemm_pack(W, bits).to_device()
+            yq[(li, bits)] = wq.qgemm(Xd, dw, bias=bd).double().flatten()
+            sizes[(li, bits)] = dw.nbytes
+            del dw
+        wq.check_device_status()
+    dense_bytes = sum(2 * l.N * l.K for l in wl.linears)
+    rows = []
+    d = torch.cat(yd)
+    for combo in itertools.product((4, 8), repeat=len(wl.linears)):
+        q = torch.cat([yq[(li, b)] for li, b in enumerate(combo)])
+        cos = float(torch.nn.functional.cosine_similarity(q, d, dim=0))
+        size = sum(sizes[(li, b)] for li, b in enumerate(combo))
+        rows.append({"bits": dict(zip([l.name for l in wl.linears], combo)), "cosine_vs_dense_bf16": cos,
+                     "packed_over_dense_bf16": round(size / dense_bytes, 4),
+                     "pages_policy": combo == tuple(l.bits for l in wl.linears)})
+    for r in rows:  # Pareto: no other assignment is at least as small and strictly more accurate (or vice versa)
+        r["pareto"] = not any((o["packed_over_dense_bf16"] <= r["packed_over_dense_bf16"] and
+                               o["cosine_vs_dense_bf16"] > r["cosine_vs_dense_bf16"]) or
+                              (o["packed_over_dense_bf16"] < r["packed_over_dense_bf16"] and
+                               o["cosine_vs_dense_bf16"] >= r["cosine_vs_dense_bf16"]) for o in rows)
+    rows.sort(key=lambda r: r["packed_over_dense_bf16"])
+    del yq, yd
+    torch.cuda.empty_cache()
+    return rows
+
+
 def cpu_oracle_single_core():
     """The oracle on one host core for config 0 (tiny) and config 3 at M=1
     (ternary decode): seconds per GEMM, dequantisation included."""
@@ -777,6 +825,7 @@ def main(argv=None):
                 res["workload4_block"] = block
                 res["path_crossover"] = cross
                 res["fused_epilogues"] = fused_sweep()
+                res["policy_sweep"] = policy_sweep()
             if not args.no_cpu and world == 1:
                 v, spent, desc, _ = cpu_oracle_sample(args.cpu_seconds)
                 res["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOP/s", "cores": blas_threads(),
