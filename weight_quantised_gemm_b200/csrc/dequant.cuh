@@ -4,8 +4,9 @@
 //   affine   wdeq = bf16_rn(fp32(s) * q + fp32(b))   (product exact, one FMA)
 //   ternary  wdeq = t * bf16_rn(fp32(s))
 //   1-bit    wdeq = c * bf16_rn(fp32(s))
-// The large-M kernel applies these to every weight tile it stages in shared
-// memory; qgemm_dequant_tile exposes the same routines for the bit-exact gate.
+// The large-M kernel applies these to every packed tile before writing it to
+// tensor memory; qgemm_dequant_tile exposes the same routines for the
+// bit-exact gate.
 #pragma once
 
 #include "ptx.cuh"

@@ -1,5 +1,5 @@
 // qgemm_dequant_tile: the dequantised weight of any [rows, cols] window, from
-// the same device routines the large-M kernel runs on its shared-memory tiles.
+// the same device routines the large-M kernel runs on its packed tiles.
 // Used to hold the dequantisation bit-exact to its definition.
 
 #include "dequant.cuh"

@@ -1,6 +1,6 @@
 // Large-M path: TMA -> dequantisation into tensor memory -> tcgen05 MMA
-// (A from TMEM, B from shared memory) -> direct bf16 stores. One persistent
-// CTA per SM.
+// (A from TMEM, B from shared memory) -> bf16 TMA stores. One persistent CTA
+// per SM.
 //
 // "Dequantised inside the matmul kernel a tile at a time" (stable-diffusion.rs
 // README, introduction) maps onto Blackwell as follows. Each output tile is
