@@ -493,13 +493,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 template <int BITS, int EPI>
 int launch_fmt(const Problem& pr, int nsm) {
   using C = Cfg<BITS>;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err =
-        cudaFuncSetAttribute(large_m_kernel<BITS, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-  });
-  int st = cuda_check(attr_err, "cudaFuncSetAttribute(large_m_kernel)");
+  int st = smem_opt_in(reinterpret_cast<const void*>(large_m_kernel<BITS, EPI>), C::kSmemBytes,
+                       "cudaFuncSetAttribute(large_m_kernel)");
   if (st != QGEMM_OK) return st;
   CUtensorMap tm_x, tm_w, tm_s, tm_b;
   const uint64_t wbytes = static_cast<uint64_t>(pr.K) * BITS / 8;

@@ -37,6 +37,9 @@ uint64_t wait_limit_ns();
 // Device address of the current device's status word (cached per device).
 int status_word(unsigned int** ptr);
 int sm_count(int* n);
+// Raises the kernel's dynamic shared-memory limit to `bytes` on the current
+// device, once per (device, kernel).
+int smem_opt_in(const void* func, int bytes, const char* what);
 
 // 2-D TMA descriptor: `inner` x `outer` elements, rows `row_stride_bytes`
 // apart, box `box_inner` x `box_outer`. Reads outside the tensor return zeros

@@ -443,13 +443,8 @@ template <int BITS, int MT, int NP>
 int launch_fmt(const Problem& pr, int grid) {
   using F = Fmt<BITS>;
   constexpr int R = 16 * NP;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err =
-        cudaFuncSetAttribute(small_m_kernel<BITS, MT, NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_LIMIT);
-  });
-  int st = cuda_check(attr_err, "cudaFuncSetAttribute(small_m_kernel)");
+  int st = smem_opt_in(reinterpret_cast<const void*>(small_m_kernel<BITS, MT, NP>), SMEM_LIMIT,
+                       "cudaFuncSetAttribute(small_m_kernel)");
   if (st != QGEMM_OK) return st;
 
   Params kp;

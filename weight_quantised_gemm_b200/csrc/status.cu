@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "ptx.cuh"
 #include "qgemm_internal.h"
@@ -50,6 +52,18 @@ int status_word(unsigned int** ptr) {
   }
   *ptr = g_status_ptr[dev];
   return QGEMM_OK;
+}
+
+int smem_opt_in(const void* func, int bytes, const char* what) {
+  int dev;
+  int st = current_device(&dev);
+  if (st != QGEMM_OK) return st;
+  static std::set<std::pair<int, const void*>> done;  // (device, kernel) pairs already configured
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (done.count({dev, func})) return QGEMM_OK;
+  st = cuda_check(cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes), what);
+  if (st == QGEMM_OK) done.insert({dev, func});
+  return st;
 }
 
 int sm_count(int* n) {
