@@ -11,10 +11,13 @@
 //   shared-memory ring, one stage per 8 scale groups of K. A stage takes one 3-D TMA box for the packed codes of all the CTA's
 //   rows (viewed as [row][unit][U bytes], U = 128, 64 or 32, the box lands as
 //   [unit][row][U bytes] with the U-byte swizzle, so the per-lane row reads
-//   are free of bank conflicts), one 2-D box each for the stage's fp16 scales
-//   and biases, and one bulk copy per token row of the activations, issued by
-//   the producer warp's lanes in parallel. (Per-lane 16-byte cp.async pieces
-//   for the activations were measured slower at M = 16.)
+//   are free of bank conflicts) and one 2-D box each for the stage's fp16
+//   scales and biases. The activations do not pass through the ring: the
+//   consumer warps load their B fragments straight from global memory (every
+//   CTA reads the same rows, so they come from L2), before waiting for the
+//   stage's weights. A TMA copy costs the SM's copy unit on the order of a
+//   hundred cycles whatever its size; one per token row per stage made M = 16
+//   pay for 48 (ternary) to 384 (8-bit, K = 12288) of them.
 // * Eight consumer warps. Normally warp w takes scale group w of every stage
 //   for all the CTA's rows; where that would not fit in registers (16 tokens
 //   and 12 or more row pairs) the rows split into two halves and warps w and
@@ -26,10 +29,10 @@
 //   bank-conflict free) and a coalesced pass adds them, adds the bias and
 //   writes bf16.
 // * Overlap (programmatic dependent launch, when the caller asks for it): the
-//   producer puts the first stages' weight, scale and bias loads in flight,
-//   lets the next grid in the stream launch, and only then waits for the
-//   previous grid to finish before it copies activations. Every thread waits
-//   for the previous grid before it reads the bias or writes the output. A
+//   producer puts the first stages' weight, scale and bias loads in flight and
+//   lets the next grid in the stream launch; the consumers wait for the
+//   previous grid to finish before they read activations, and every thread
+//   waits for it before it reads the bias or writes the output. A
 //   CTA of the next launch then takes an SM the moment this grid's CTA there
 //   exits, and its weight stream overlaps the other SMs' last stages instead
 //   of waiting for the whole grid and a fresh launch. Without the launch
@@ -81,6 +84,11 @@ struct Fmt {
 // Row halves for a CTA of NP pairs and MT tokens: 2 where one warp's
 // accumulators for all NP pairs would not fit in registers.
 __host__ __device__ constexpr int split_rows(int MT, int NP) { return MT > 8 && NP >= 6 ? 2 : 1; }
+// Split-row CTAs give each warp two groups per stage; holding both groups'
+// activation fragments in registers across the stage wait spills, so their
+// activations come through the ring (one bulk copy per token row) instead of
+// straight from global memory.
+__host__ __device__ constexpr bool x_in_ring(int MT, int NP) { return split_rows(MT, NP) == 2; }
 
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -100,7 +108,8 @@ struct Params {
   int unit_shift;        // log2 of U, the bytes per swizzled row piece (128, 64 or 32)
   int stage_bytes;       // bytes per ring stage (multiple of 1024)
   int data_bytes;        // ring (or the partial sums, if larger); the mbarriers follow
-  int off_s, off_b, off_x, x_stride;  // offsets inside a stage; activation row stride in bytes
+  int off_s, off_b;      // offsets of the scales and biases inside a stage
+  int off_x, x_stride;   // activations in the ring (split-row CTAs): offset, token row stride in bytes
   int overlap;           // launched with programmatic dependent launch
   uint64_t wait_limit_ns;
   unsigned int* status;
@@ -199,6 +208,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr int GPL = GS / GROUP_LANES;      // groups per warp and stage
   constexpr int TH = MT > 8 ? 2 : 1;         // 8-token halves
   constexpr int NLP = R + 4;                 // row pitch of the partial sums: 2 * NLP = 8 (mod 32) banks
+  constexpr bool XR = x_in_ring(MT, NP);     // activations through the ring, else from global memory
   static_assert(NP % PH == 0, "the halves take whole 16-row pairs");
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = ptx::smem_u32(smem);
@@ -258,7 +268,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int kt, valid;
       stage_k(t, kt, valid);
       const uint32_t st = sbase + s * p.stage_bytes;
-      ptx::mbar_arrive_expect_tx(full(s), R * F::ROWB + sb_bytes * (BITS <= 2 ? 1 : 2) + p.M * valid * 2);
+      ptx::mbar_arrive_expect_tx(full(s), R * F::ROWB + sb_bytes * (BITS <= 2 ? 1 : 2) + (XR ? p.M * valid * 2 : 0));
       ptx::tma_load_3d(st, &tm_w, 0, n0, kt * units, full(s));
       ptx::tma_load_2d(st + p.off_s, &tm_s, n0, kt * GS, full(s));
       if (BITS > 2) ptx::tma_load_2d(st + p.off_b, &tm_b, n0, kt * GS, full(s));
@@ -276,19 +286,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::tma_prefetch_desc(&tm_s);
       if (BITS > 2) ptx::tma_prefetch_desc(&tm_b);
     }
-    if (p.overlap) {
-      // The weights do not depend on the previous grid: put the first stages
-      // in flight before waiting for it. (The TMA unit takes copies in issue
-      // order, so the activation copies then queue behind all of them.)
+    if (!XR || p.overlap) {
+      // The weights do not depend on the previous grid: the first stages go
+      // out at once, and the next grid may launch (both no-ops without the
+      // launch attribute). Ring activations follow once that grid is done
+      // (the TMA unit takes copies in issue order, so they queue behind).
       if (lane == 0)
         for (int t = 0; t < pre; ++t) load_weights(t, t);
       griddep_launch_dependents();
-      griddep_wait();  // the activations may be the previous grid's output
-      __syncwarp();  // the transaction counts are raised before any activation copy can land
-      for (int t = 0; t < pre; ++t) load_x(t, t);
+      if constexpr (XR) {
+        griddep_wait();
+        __syncwarp();  // the transaction counts are raised before any activation copy can land
+        for (int t = 0; t < pre; ++t) load_x(t, t);
+      }
     } else {
-      // Nothing to wait for: each stage's activations right behind its weights,
-      // so that the first stage is complete as early as possible.
+      // Nothing to wait for: each stage's activations right behind its
+      // weights, so that the first stage is complete as early as possible.
       for (int t = 0; t < pre; ++t) {
         if (lane == 0) load_weights(t, t);
         __syncwarp();
@@ -303,8 +316,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       if (lane == 0) load_weights(t, s);
-      __syncwarp();
-      load_x(t, s);
+      if constexpr (XR) {
+        __syncwarp();
+        load_x(t, s);
+      }
     }
     // Let every copy issued above land before the block can exit.
     if (lane == 0) {
@@ -314,26 +329,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ---------------- consumers ----------------
     griddep_launch_dependents();
+    if constexpr (!XR) griddep_wait();  // the activations may be the previous grid's output
     const int ush = p.unit_shift;
     const int key16 = swizzle_key16(g, ush);
     const int gl = warp % GROUP_LANES;  // group lane: groups gl, gl + GROUP_LANES, ... of every stage
     const int q0 = (warp / GROUP_LANES) * NPH;  // first 16-row pair of this warp's half
+    const bool ga = g < p.M, gb = MT > 8 && g + 8 < p.M;  // tokens g and g + 8 exist
     for (int t = 0; t < p.num_stages; ++t) {
       const int s = t % p.ring;
+      const int kt = (t + rot) % p.num_stages;
+      // The activations of this warp's groups (the B operand: tokens g and
+      // g + 8, k = gs*G + 16*step + 4c .. +3) straight from global memory,
+      // where every CTA reads the same rows (L2 hits); issued before the
+      // stage's weights are waited for, so the two latencies overlap.
+      uint2 xr[XR ? 1 : GPL][STEPS][TH];
+#pragma unroll
+      for (int gi = 0; gi < (XR ? 0 : GPL); ++gi) {
+        const int k0 = kt * F::KS + (gl + GROUP_LANES * gi) * F::G;
+        const bool in = k0 < p.K;
+        const uint2* x0p = reinterpret_cast<const uint2*>(p.X + static_cast<size_t>(g) * p.K + k0 + 4 * c);
+        const uint2* x1p = reinterpret_cast<const uint2*>(p.X + static_cast<size_t>(g + 8) * p.K + k0 + 4 * c);
+#pragma unroll
+        for (int k = 0; k < STEPS; ++k) {
+          xr[gi][k][0] = (in && ga) ? __ldg(x0p + 4 * k) : make_uint2(0u, 0u);
+          if constexpr (TH > 1) xr[gi][k][TH - 1] = (in && gb) ? __ldg(x1p + 4 * k) : make_uint2(0u, 0u);
+        }
+      }
       if (!warp_wait(full(s), (t / p.ring) & 1, lim, abort_flag)) {
         if (lane == 0) give_up();
         break;
       }
       const uint8_t* st = smem + s * p.stage_bytes;
-      const int kt = (t + rot) % p.num_stages;
 #pragma unroll
       for (int gi = 0; gi < GPL; ++gi) {
         const int gs = gl + GROUP_LANES * gi;
         if (kt * F::KS + gs * F::G >= p.K) break;
-        // activations of this group (the B operand): tokens g and g + 8,
-        // k = gs*G + 16*step + 4c .. +3
-        const uint8_t* xg = st + p.off_x + g * p.x_stride + (gs * F::G + 4 * c) * 2;
-        const bool ga = g < p.M, gb = MT > 8 && g + 8 < p.M;
         float xs[TH][4];  // sum of x over the group per token (affine)
         float tmp[NPH][TH][4];
 #pragma unroll
@@ -348,8 +378,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int j = 0; j < 4; ++j) tmp[q][h][j] = 0.f;
 #pragma unroll
         for (int k = 0; k < STEPS; ++k) {
-          const uint2 x0 = ga ? *reinterpret_cast<const uint2*>(xg + 32 * k) : make_uint2(0u, 0u);
-          const uint2 x1 = gb ? *reinterpret_cast<const uint2*>(xg + 8 * p.x_stride + 32 * k) : make_uint2(0u, 0u);
+          uint2 x0, x1;
+          if constexpr (XR) {
+            const uint8_t* xg = st + p.off_x + g * p.x_stride + (gs * F::G + 16 * k + 4 * c) * 2;
+            x0 = ga ? *reinterpret_cast<const uint2*>(xg) : make_uint2(0u, 0u);
+            x1 = gb ? *reinterpret_cast<const uint2*>(xg + 8 * p.x_stride) : make_uint2(0u, 0u);
+          } else {
+            x0 = xr[gi][k][0];
+            x1 = xr[gi][k][TH - 1];
+          }
           if constexpr (BITS > 2) {
             const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};
             mma_bf16_16816(xs[0], ones, x0.x, x0.y);
@@ -470,7 +507,7 @@ int launch_fmt(const Problem& pr, int grid) {
   kp.off_b = (kp.off_s + sb + 127) & ~127;
   kp.off_x = (kp.off_b + (BITS <= 2 ? 0 : sb) + 127) & ~127;
   kp.x_stride = F::KS * 2 + 32;  // +32 B: token rows 8 banks apart, so the 8-byte B fetches do not collide
-  kp.stage_bytes = (kp.off_x + pr.M * kp.x_stride + 1023) & ~1023;
+  kp.stage_bytes = (kp.off_x + (x_in_ring(MT, NP) ? pr.M * kp.x_stride : 0) + 1023) & ~1023;
   int ring = RING_BUDGET / kp.stage_bytes;
   ring = ring < MAX_STAGES ? ring : MAX_STAGES;
   ring = ring < kp.num_stages ? ring : kp.num_stages;
