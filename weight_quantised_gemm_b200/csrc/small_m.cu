@@ -12,12 +12,16 @@
 //   rows (viewed as [row][unit][U bytes], U = 128, 64 or 32, the box lands as
 //   [unit][row][U bytes] with the U-byte swizzle, so the per-lane row reads
 //   are free of bank conflicts) and one 2-D box each for the stage's fp16
-//   scales and biases. The activations do not pass through the ring: the
-//   consumer warps load their B fragments straight from global memory (every
-//   CTA reads the same rows, so they come from L2), before waiting for the
-//   stage's weights. A TMA copy costs the SM's copy unit on the order of a
-//   hundred cycles whatever its size; one per token row per stage made M = 16
-//   pay for 48 (ternary) to 384 (8-bit, K = 12288) of them.
+//   scales and biases. The activations normally do not pass through the
+//   ring: the consumer warps load their B fragments straight from global
+//   memory (every CTA reads the same rows, so they come from L2), before
+//   waiting for the stage's weights. A TMA copy costs the SM's copy unit on
+//   the order of a hundred cycles whatever its size; one per token row per
+//   stage made M = 16 pay for 48 (ternary) to 384 (8-bit, K = 12288) of them.
+//   Split-row CTAs (below) are the exception: a warp there takes two groups
+//   per stage, and holding both groups' fragments across the wait spills
+//   registers, so the producer bulk-copies their activation rows into the
+//   stage.
 // * Eight consumer warps. Normally warp w takes scale group w of every stage
 //   for all the CTA's rows; where that would not fit in registers (16 tokens
 //   and 12 or more row pairs) the rows split into two halves and warps w and
@@ -30,9 +34,10 @@
 //   writes bf16.
 // * Overlap (programmatic dependent launch, when the caller asks for it): the
 //   producer puts the first stages' weight, scale and bias loads in flight and
-//   lets the next grid in the stream launch; the consumers wait for the
-//   previous grid to finish before they read activations, and every thread
-//   waits for it before it reads the bias or writes the output. A
+//   lets the next grid in the stream launch; whoever reads the activations
+//   (the consumers, or for split-row CTAs the producer's copies) waits for
+//   the previous grid to finish first, and every thread waits for it before
+//   it reads the bias or writes the output. A
 //   CTA of the next launch then takes an SM the moment this grid's CTA there
 //   exits, and its weight stream overlaps the other SMs' last stages instead
 //   of waiting for the whole grid and a fresh launch. Without the launch
