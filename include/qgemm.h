@@ -231,9 +231,15 @@ int qgemm_dequant_tile(const qgemm_weights* W, int32_t n0, int32_t k0, int32_t r
 
 /*
  * Synchronises `stream`, then reads and clears the current device's status
- * word. Returns QGEMM_OK, QGEMM_ERR_DEVICE_TIMEOUT if a kernel gave up a
- * bounded wait since the last read, or QGEMM_ERR_CUDA if the stream reports
- * an error.
+ * word (all conditions recorded since the last read). Returns, first match:
+ *   QGEMM_ERR_CUDA          the stream reports a CUDA error;
+ *   QGEMM_ERR_NONFINITE     qgemm_pack_device met a NaN or infinite weight;
+ *   QGEMM_ERR_UNSUPPORTED   qgemm_pack_device: a scale or bias overflows fp16;
+ *   QGEMM_ERR_CUDA          a kernel found its shared memory misaligned and
+ *                           returned without computing;
+ *   QGEMM_ERR_DEVICE_TIMEOUT a kernel gave up a bounded wait;
+ *   QGEMM_OK                none of these.
+ * qgemm_last_error() then names the condition and the raw status word.
  */
 int qgemm_get_device_status(void* stream);
 
