@@ -195,3 +195,16 @@ def test_pack_device_rejects_bad_arguments_without_device():
     assert call(b=None) == wq.QGEMM_ERR_INVALID_ARG            # affine needs biases
     assert call(W=0x1004) == wq.QGEMM_ERR_ALIGNMENT
     assert call(s=0x3002) == wq.QGEMM_ERR_ALIGNMENT
+
+
+def test_binding_device_check_is_host_logic():
+    """The binding's same-device check (run before every launch) needs no GPU:
+    a weight or output buffer on another device is refused by name."""
+    import torch
+    cpu = torch.zeros(4)
+    W = wq.DeviceWeights(16, 128, 4, 64, cpu, cpu, cpu)
+    with pytest.raises(ValueError, match="W.packed is on cpu"):
+        wq._same_device(torch.device("cuda", 0), W)
+    with pytest.raises(ValueError, match="out is on meta"):
+        wq._same_device(torch.device("cpu"), W, out=torch.zeros(2, device="meta"))
+    wq._same_device(torch.device("cpu"), W, out=cpu, bias=None)   # one device throughout: accepted

@@ -391,3 +391,20 @@ def test_pack_device_reports_bad_data_through_the_status_word():
     W[0, 0], W[0, 1] = 0.0, 0.0
     wq.qgemm_pack_device(W, 4)
     assert wq.qgemm_get_device_status() == wq.QGEMM_OK
+
+
+def test_binding_refuses_buffers_off_the_device():
+    """The library takes raw pointers and launches on X's device, so the
+    binding refuses a host buffer before any launch; the normal call works."""
+    dw = wq.qgemm_pack(np.zeros((256, 256), dtype=np.float32), 4).to_device("cuda")
+    X = torch.zeros((2, 256), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError, match="out is on cpu"):
+        wq.qgemm(X, dw, out=torch.empty((2, 256), dtype=torch.bfloat16))
+    host_packed = wq.DeviceWeights(dw.N, dw.K, dw.bits, dw.group, dw.packed.cpu(), dw.scales, dw.biases)
+    with pytest.raises(ValueError, match="W.packed is on cpu"):
+        wq.qgemm(X, host_packed)
+    with pytest.raises(ValueError, match="out is on cpu"):
+        wq.qgemm_dequant_tile(dw, out=torch.empty((256, 256), dtype=torch.bfloat16))
+    y = wq.qgemm(X, dw)
+    wq.check_device_status()
+    assert y.shape == (2, 256) and bool(torch.all(y == 0))

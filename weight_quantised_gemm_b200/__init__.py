@@ -221,9 +221,10 @@ def qgemm_pack_device(W, bits: int, group: Optional[int] = None, stream=None) ->
     packed = torch.empty(pb, dtype=torch.uint8, device=W.device)
     scales = torch.empty(sb // 2, dtype=torch.int16, device=W.device)
     biases = torch.empty(bb // 2, dtype=torch.int16, device=W.device) if bb else None
-    _check(_lib.qgemm_pack_device(W.data_ptr(), N, K, bits, group, packed.data_ptr(), scales.data_ptr(),
-                                  None if biases is None else biases.data_ptr(), _stream_handle(stream)),
-           "qgemm_pack_device")
+    with torch.cuda.device(W.device):
+        _check(_lib.qgemm_pack_device(W.data_ptr(), N, K, bits, group, packed.data_ptr(), scales.data_ptr(),
+                                      None if biases is None else biases.data_ptr(),
+                                      _stream_handle(stream, W.device)), "qgemm_pack_device")
     return DeviceWeights(N, K, bits, group, packed.view(N, -1), scales, biases)
 
 
@@ -244,11 +245,23 @@ def qgemm_load(path: str) -> PackedWeights:
                          None if biases is None else biases.reshape(K // group, N))
 
 
-def _stream_handle(stream) -> Optional[int]:
+def _stream_handle(stream, device=None) -> Optional[int]:
     import torch
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif device is not None and stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
     return stream.cuda_stream
+
+
+def _same_device(device, W: "DeviceWeights", **tensors) -> None:
+    """Every tensor argument on X's CUDA device: the library launches on the
+    current device and takes raw pointers, so a host or other-device buffer
+    must be refused here, before any launch."""
+    arrays = {"W.packed": W.packed, "W.scales": W.scales, "W.biases": W.biases, **tensors}
+    for name, t in arrays.items():
+        if t is not None and t.device != device:
+            raise ValueError(f"{name} is on {t.device}, X on {device}")
 
 
 def qgemm(X, W: DeviceWeights, bias=None, out=None, path: int = QGEMM_PATH_AUTO, stream=None,
@@ -268,11 +281,13 @@ def qgemm(X, W: DeviceWeights, bias=None, out=None, path: int = QGEMM_PATH_AUTO,
         raise ValueError("out must be a contiguous bf16 [M, N] tensor")
     if bias is not None and (bias.dtype != torch.bfloat16 or bias.numel() != W.N or not bias.is_cuda):
         raise ValueError("bias must be a bf16 CUDA tensor of N elements")
+    _same_device(X.device, W, out=out, bias=bias)
     desc = W.descriptor()
     flags = QGEMM_FLAG_OVERLAP_PREVIOUS if overlap_previous else 0
-    _check(_lib.qgemm_ex(X.data_ptr(), M, ctypes.byref(desc), out.data_ptr(),
-                         None if bias is None else bias.data_ptr(), int(path) | flags, _stream_handle(stream)),
-           "qgemm")
+    with torch.cuda.device(X.device):
+        _check(_lib.qgemm_ex(X.data_ptr(), M, ctypes.byref(desc), out.data_ptr(),
+                             None if bias is None else bias.data_ptr(), int(path) | flags,
+                             _stream_handle(stream, X.device)), "qgemm")
     return out
 
 
@@ -299,13 +314,15 @@ def qgemm_fused(X, W: DeviceWeights, op: int, bias=None, residual=None, gate=Non
             raise ValueError("residual must be a contiguous bf16 [M, N] tensor")
         if gate.dtype != torch.bfloat16 or gate.numel() != W.N or not gate.is_cuda:
             raise ValueError("gate must be a bf16 CUDA tensor of N elements")
+    _same_device(X.device, W, out=out, bias=bias, residual=residual, gate=gate)
     epi = _Epilogue(int(op), None if residual is None else residual.data_ptr(),
                     None if gate is None else gate.data_ptr())
     desc = W.descriptor()
     flags = QGEMM_FLAG_OVERLAP_PREVIOUS if overlap_previous else 0
-    _check(_lib.qgemm_fused(X.data_ptr(), M, ctypes.byref(desc), out.data_ptr(),
-                            None if bias is None else bias.data_ptr(), ctypes.byref(epi), int(path) | flags,
-                            _stream_handle(stream)), "qgemm_fused")
+    with torch.cuda.device(X.device):
+        _check(_lib.qgemm_fused(X.data_ptr(), M, ctypes.byref(desc), out.data_ptr(),
+                                None if bias is None else bias.data_ptr(), ctypes.byref(epi), int(path) | flags,
+                                _stream_handle(stream, X.device)), "qgemm_fused")
     return out
 
 
@@ -322,11 +339,16 @@ def qgemm_dequant_tile(W: DeviceWeights, n0: int = 0, k0: int = 0, rows: Optiona
     import torch
     rows = W.N - n0 if rows is None else rows
     cols = W.K - k0 if cols is None else cols
+    dev = W.packed.device
     if out is None:
-        out = torch.empty((rows, cols), dtype=torch.bfloat16, device=W.packed.device)
+        out = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev)
+    elif out.dtype != torch.bfloat16 or tuple(out.shape) != (rows, cols) or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 [rows, cols] tensor")
+    _same_device(dev, W, out=out)
     desc = W.descriptor()
-    _check(_lib.qgemm_dequant_tile(ctypes.byref(desc), n0, k0, rows, cols, out.data_ptr(),
-                                   _stream_handle(stream)), "qgemm_dequant_tile")
+    with torch.cuda.device(dev):
+        _check(_lib.qgemm_dequant_tile(ctypes.byref(desc), n0, k0, rows, cols, out.data_ptr(),
+                                       _stream_handle(stream, dev)), "qgemm_dequant_tile")
     return out
 
 
