@@ -37,7 +37,11 @@ Packing is round-to-nearest (RTN) in fp64, ties to even:
 * ternary: s16 = fp16(max |w|); t = clamp(rint(w / s16), -1, 1), t = 0 where
   s16 == 0.
 * 1-bit: s16 = fp16(mean |w|), the scale that minimises the squared error
-  for fixed signs; c = +1 where w >= 0 (-0 included), else -1.
+  for fixed signs, with the sum of |w| taken in fp64 in k order (a running
+  sum) and then divided by 128; c = +1 where w >= 0 (-0 included), else -1.
+  The order is part of the reading: this sum decides a stored value, and on
+  groups whose values span many binades another order can round it to the
+  neighbouring fp16 value.
 
 Bit layout, row-major over N with K contiguous, little-endian 32-bit words:
 
@@ -219,7 +223,7 @@ def pack_ref(W, bits: int, group: int):
         codes = q.reshape(N, K).astype(np.int64)
         return pack_codes(codes, bits), np.ascontiguousarray(s16.T), np.ascontiguousarray(b16.T)
     if bits == BINARY_BITS:
-        s16 = fp16_rn(np.abs(Wg).mean(axis=2))
+        s16 = fp16_rn(np.add.accumulate(np.abs(Wg), axis=2)[:, :, -1] / group)
         if not np.all(np.isfinite(s16)):
             raise OverflowError("scale overflows fp16")
         c = np.where(Wg >= 0, 1, -1)

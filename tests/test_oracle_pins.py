@@ -523,3 +523,32 @@ def test_1bit_dequant_is_signed_scale_and_gemm_matches_triple_loop():
     brute = _naive(O.bf16_bits_to_f64(X), O.wq_exact(p, s, b, 1, 128, 128), O.bf16_bits_to_f64(bias))
     assert np.allclose(ref, brute, rtol=1e-12, atol=1e-14)
     assert O.format_bytes(12288, 3072, 1, 128) == 12288 * 3072 // 8 + 12288 * 24 * 2
+
+
+def test_1bit_scale_is_a_running_sum_in_k_order():
+    """The 1-bit scale is fp16(sum_k |w_k| / 128), the sum taken in fp64 in k
+    order. One weight of 1049088 (= 8196 * 128, the tie between the fp16
+    values 8192 and 8200) and 127 of 2^-38 separate the orders: first in k
+    order, the large weight swallows each tiny one, the mean is the tie
+    itself and rounds to even (8192); last, the tiny ones add up to almost
+    2^-31 before meeting it and the mean lands above the tie (8200)."""
+    w = np.full((1, 128), 2.0 ** -38, dtype=np.float32)
+    w[0, 0] = 1049088.0
+    total = 0.0
+    for v in w[0]:                      # Python floats: fp64, one term at a time
+        total += abs(float(v))
+    assert total / 128 == 8196.0
+    _, s16, _ = O.pack_ref(w, 1, 128)
+    assert float(s16[0, 0]) == 8192.0
+    _, s16r, _ = O.pack_ref(np.ascontiguousarray(w[:, ::-1]), 1, 128)
+    assert float(s16r[0, 0]) == 8200.0
+    # on ordinary groups the running sum is the mean
+    g = np.random.default_rng(13)
+    wr = (g.standard_normal((4, 256)) * 0.02).astype(np.float32)
+    _, s16g, _ = O.pack_ref(wr, 1, 128)
+    for n in range(4):
+        for j in range(2):
+            acc = 0.0
+            for v in wr[n, 128 * j:128 * (j + 1)]:
+                acc += abs(float(v))
+            assert s16g[j, n] == np.float16(acc / 128)

@@ -85,3 +85,16 @@ def test_multithreaded_pack_matches_single_rows():
     assert np.array_equal(whole.packed[1000:1016], part.packed)
     assert np.array_equal(whole.scales[:, 1000:1016].view(np.uint16), part.scales.view(np.uint16))
     assert whole.scales.shape == (lin.K // 64, 2048)
+
+
+def test_1bit_scale_order_matches_oracle():
+    """A group whose 1-bit scale depends on the order of the sum of |w|
+    (see the oracle pin): the host packer takes it in k order like the oracle."""
+    w = np.full((16, 128), 2.0 ** -38, dtype=np.float32)
+    w[::2, 0] = 1049088.0                # even rows: the large weight first
+    w[1::2, 127] = 1049088.0             # odd rows: the large weight last
+    pw = wq.qgemm_pack(w, 1)
+    p, s16, _ = O.pack_ref(w, 1, 128)
+    assert np.array_equal(pw.scales.view(np.uint16), s16.view(np.uint16))
+    assert np.array_equal(pw.packed, p)
+    assert float(pw.scales[0, 0]) == 8192.0 and float(pw.scales[0, 1]) == 8200.0
