@@ -31,8 +31,9 @@ formula and no rounding rule):
 Packing is round-to-nearest (RTN) in fp64, ties to even:
 
 * affine: lo = min, hi = max of the group; s16 = fp16(fl64((hi - lo) /
-  (2^b - 1))), b16 = fp16(lo) (a zero minimum as +0, so the sign of a zero
-  weight never decides a stored bit); q = clamp(rint((w - b16) / s16), 0,
+  (2^b - 1))), b16 = fp16(lo) (a zero minimum or maximum taken as +0, so the
+  sign of a zero weight never decides a stored bit: a group of zeros stores
+  +0 for both its scale and its bias); q = clamp(rint((w - b16) / s16), 0,
   2^b - 1), q = 0 where s16 == 0.
 * ternary: s16 = fp16(max |w|); t = clamp(rint(w / s16), -1, 1), t = 0 where
   s16 == 0.
@@ -87,7 +88,8 @@ def fp16_rn(x) -> np.ndarray:
     Pinned in the tests against CPython's own IEEE half packing
     (``struct.pack('e')``) on every fp16 value, every midpoint and random doubles.
     """
-    return np.asarray(x, dtype=np.float64).astype(np.float16)
+    with np.errstate(over="ignore"):    # overflow gives inf, which the callers refuse
+        return np.asarray(x, dtype=np.float64).astype(np.float16)
 
 
 def bf16_rn_bits(x32) -> np.ndarray:
@@ -210,7 +212,7 @@ def pack_ref(W, bits: int, group: int):
     if bits in AFFINE_BITS:
         qmax = (1 << bits) - 1
         lo = Wg.min(axis=2) + 0.0      # a zero minimum is stored as +0, never -0
-        hi = Wg.max(axis=2)
+        hi = Wg.max(axis=2) + 0.0      # so a zero range gives a +0 scale, whichever zeros the group holds
         s16 = fp16_rn((hi - lo) / qmax)
         b16 = fp16_rn(lo)
         if not (np.all(np.isfinite(s16)) and np.all(np.isfinite(b16))):

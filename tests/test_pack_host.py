@@ -98,3 +98,42 @@ def test_1bit_scale_order_matches_oracle():
     assert np.array_equal(pw.scales.view(np.uint16), s16.view(np.uint16))
     assert np.array_equal(pw.packed, p)
     assert float(pw.scales[0, 0]) == 8192.0 and float(pw.scales[0, 1]) == 8200.0
+
+
+@pytest.mark.parametrize("limit", [3e4, 3.3999999521443642e+38], ids=["fp16-range", "fp32-range"])
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
+def test_host_packer_matches_oracle_on_arbitrary_fp32(bits, limit):
+    """Property test: any finite fp32 weights (subnormals, signed zeros,
+    repeated values, rounding ties, values near and past the fp16 range) pack
+    to the oracle's bytes, scales and biases exactly, and a group whose scale
+    or bias overflows fp16 is refused by both."""
+    pytest.importorskip("hypothesis")
+    from hypothesis import HealthCheck, given, settings, strategies as st
+    from hypothesis.extra.numpy import arrays
+
+    group = wq.GROUP_OF_BITS[bits]
+    elems = st.one_of(st.floats(-limit, limit, width=32, allow_nan=False, allow_infinity=False),
+                      st.sampled_from([0.0, -0.0, 0.5, -0.5, 1.5, 2.5, 2.0 ** -149, -(2.0 ** -130),
+                                       65504.0, -65504.0, 65520.0]))
+
+    @settings(max_examples=40, deadline=None, derandomize=True, database=None,
+              suppress_health_check=list(HealthCheck))
+    @given(W=arrays(np.float32, (16, 2 * group), elements=elems))
+    def check(W):
+        try:
+            pw, refused = wq.qgemm_pack(W, bits), None
+        except wq.QGemmError as e:
+            pw, refused = None, e.status
+        try:
+            p, s16, b16 = O.pack_ref(W, bits, group)
+            expect = None
+        except OverflowError:
+            expect = wq.QGEMM_ERR_UNSUPPORTED
+        assert refused == expect
+        if expect is None:
+            assert np.array_equal(pw.packed, p)
+            assert np.array_equal(pw.scales.view(np.uint16), s16.view(np.uint16))
+            if bits > 2:
+                assert np.array_equal(pw.biases.view(np.uint16), b16.view(np.uint16))
+
+    check()

@@ -71,6 +71,7 @@ __global__ void pack_kernel(const float* __restrict__ W, int N, int K, uint32_t*
         hi = hi < v ? v : hi;
       }
       lo = lo + 0.0;  // a zero minimum is stored as +0
+      hi = hi + 0.0;  // and a zero range gives a +0 scale, whichever zeros the group holds
       const uint16_t s16 = f64_to_f16_bits((hi - lo) / qmax);
       const uint16_t b16 = f64_to_f16_bits(lo);
       if (!f16_finite(s16) || !f16_finite(b16)) ptx::set_status(status, kStatusPackOverflow);

@@ -131,6 +131,7 @@ int pack_rows(const PackJob& jb, int r0, int r1) {
           hi = std::max(hi, static_cast<double>(wg[i]));
         }
         lo = lo + 0.0;  // a zero minimum is stored as +0
+        hi = hi + 0.0;  // and a zero range gives a +0 scale, whichever zeros the group holds
         const uint16_t s16 = f64_to_f16_rn((hi - lo) / qmax);
         const uint16_t b16 = f64_to_f16_rn(lo);
         if (!is_f16_finite(s16) || !is_f16_finite(b16)) return QGEMM_ERR_UNSUPPORTED;
