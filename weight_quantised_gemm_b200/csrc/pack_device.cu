@@ -65,7 +65,7 @@ __global__ void pack_kernel(const float* __restrict__ W, int N, int K, uint32_t*
       double lo = static_cast<double>(wg[0]), hi = lo;
       for (int i = 1; i < G; ++i) {
         // the host's std::min / std::max exactly: on equal values (+0 and -0)
-        // the running value stays, which decides the sign of a zero scale
+        // the running value stays
         const double v = static_cast<double>(wg[i]);
         lo = v < lo ? v : lo;
         hi = hi < v ? v : hi;
