@@ -155,10 +155,12 @@ int qgemm_pack_device(const void* W, int32_t N, int32_t K, int32_t bits, int32_t
  * biases_bytes (little-endian), then the three arrays in that order.
  * qgemm_save writes one; qgemm_load_header reads its shape and format (check
  * them, size buffers with qgemm_pack_sizes); qgemm_load fills caller-
- * allocated host buffers (biases may be NULL for 1-bit and ternary). A bad
- * magic, sizes that do not match the format, a short or overlong file, or an
- * I/O failure return QGEMM_ERR_INVALID_ARG (format errors: those of
- * qgemm_pack_sizes). No counterpart as an interface in the pages.
+ * allocated host buffers (biases may be NULL for 1-bit and ternary). Both
+ * readers check the whole file before returning OK or copying anything: a
+ * bad magic, array sizes that do not match the format, a file length other
+ * than the header plus the three arrays, or an I/O failure return
+ * QGEMM_ERR_INVALID_ARG (format errors: those of qgemm_pack_sizes). No
+ * counterpart as an interface in the pages.
  */
 int qgemm_save(const char* path, int32_t N, int32_t K, int32_t bits, int32_t group,
                const void* packed, const void* scales, const void* biases);

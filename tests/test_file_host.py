@@ -1,5 +1,6 @@
 """The at-rest file (qgemm_save / qgemm_load_header / qgemm_load) on the host:
 round trips of every format, and the documented rejections."""
+import ctypes
 import os
 import struct
 
@@ -57,3 +58,33 @@ def test_rejects_corrupt_files(tmp_path):
         open(bad, "wb").write(blob)
         _expect(bad, status)
     _expect(str(tmp_path / "missing.qgw"), wq.QGEMM_ERR_INVALID_ARG)
+
+
+def test_truncation_at_every_offset_and_a_lying_header(tmp_path):
+    """Every proper prefix of a valid file, and the file with one byte more,
+    is refused by both readers; a header whose shape claims far more data
+    than the file holds is refused by qgemm_load_header before any buffer is
+    sized from it."""
+    pw = wq.qgemm_pack(WL.random_case(9, 1, 16, 128, 4, with_bias=False)[1], 4)
+    good = str(tmp_path / "good.qgw")
+    pw.save(good)
+    data = open(good, "rb").read()
+    bad = str(tmp_path / "bad.qgw")
+    N, K, bits, group = (ctypes.c_int32() for _ in range(4))
+    for cut in list(range(len(data))) + [len(data) + 1]:
+        open(bad, "wb").write(data[:cut] if cut < len(data) else data + b"\0")
+        st = wq._lib.qgemm_load_header(bad.encode(), ctypes.byref(N), ctypes.byref(K), ctypes.byref(bits),
+                                       ctypes.byref(group))
+        assert st == wq.QGEMM_ERR_INVALID_ARG, cut
+        _expect(bad, wq.QGEMM_ERR_INVALID_ARG)
+    # a consistent header for [2^20, 2^20] 8-bit weights (1 TiB of codes) over the small file's bytes
+    n = k = 1 << 20
+    lying = data[:8] + struct.pack("<4i3Q", n, k, 8, 64, n * k, n * (k // 64) * 2, n * (k // 64) * 2) + data[48:]
+    open(bad, "wb").write(lying)
+    st = wq._lib.qgemm_load_header(bad.encode(), ctypes.byref(N), ctypes.byref(K), ctypes.byref(bits),
+                                   ctypes.byref(group))
+    assert st == wq.QGEMM_ERR_INVALID_ARG
+    _expect(bad, wq.QGEMM_ERR_INVALID_ARG)
+    # and the untouched file still loads
+    back = wq.qgemm_load(good)
+    assert np.array_equal(back.packed, pw.packed)

@@ -44,6 +44,16 @@ int read_header(FILE* f, const char* path, Header* h) {
   if (pb != h->packed_bytes || sb != h->scales_bytes || bb != h->biases_bytes)
     return qg::fail(QGEMM_ERR_INVALID_ARG, "%s: array sizes do not match N=%d K=%d bits=%d", path, h->N, h->K,
                     h->bits);
+  // The file holds exactly the header and the three arrays: a short or
+  // overlong file is refused here, before a caller sizes buffers from the
+  // header or any array byte is copied out.
+  if (std::fseek(f, 0, SEEK_END) != 0) return qg::fail(QGEMM_ERR_INVALID_ARG, "%s: cannot seek", path);
+  const long end = std::ftell(f);
+  if (end < 0 || std::fseek(f, static_cast<long>(sizeof(Header)), SEEK_SET) != 0)
+    return qg::fail(QGEMM_ERR_INVALID_ARG, "%s: cannot seek", path);
+  const unsigned long long want = sizeof(Header) + static_cast<unsigned long long>(pb) + sb + bb;
+  if (static_cast<unsigned long long>(end) != want)
+    return qg::fail(QGEMM_ERR_INVALID_ARG, "%s: %ld bytes, the header describes %llu", path, end, want);
   return QGEMM_OK;
 }
 
