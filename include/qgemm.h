@@ -115,8 +115,8 @@ typedef struct qgemm_weights {
  * Byte sizes of the three packed arrays for an [N, K] weight.
  * Defined by the layout above. biases_bytes is 0 for 1-bit and ternary.
  * Returns INVALID_ARG for non-positive sizes or null outputs, UNSUPPORTED
- * for a (bits, group) pair other than (4,64), (8,64), (2,128), (1,128) or
- * for K not a multiple of 128.
+ * for a (bits, group) pair other than (4,64), (8,64), (2,128), (1,128), for
+ * K not a multiple of 128, or for N or K above 2^30.
  */
 int qgemm_pack_sizes(int32_t N, int32_t K, int32_t bits, int32_t group,
                      size_t* packed_bytes, size_t* scales_bytes, size_t* biases_bytes);
@@ -174,7 +174,8 @@ int qgemm_load(const char* path, void* packed, void* scales, void* biases);
  *   W     device-resident packed weights (struct itself is host memory)
  *   out   device bf16 [M, N] row-major, 16-byte aligned
  *   bias  device bf16 [N] or NULL
- * Requires K % 128 == 0 and N % 16 == 0 (1-bit weights with K % 256 != 0
+ * Requires K % 128 == 0, N % 16 == 0 and M, N, K <= 2^30, the same limit as
+ * qgemm_pack_sizes (larger: UNSUPPORTED) (1-bit weights with K % 256 != 0
  * always take the large-M path). The path (small-M register path or
  * large-M tensor-core path) is chosen per (bits, M, N, K) from a measured
  * table; the environment variable QGEMM_PATH=small|large overrides it.

@@ -51,6 +51,8 @@ def test_pack_sizes():
     ((16, 192, 4, 64), wq.QGEMM_ERR_UNSUPPORTED),     # K not a multiple of 128
     ((0, 128, 4, 64), wq.QGEMM_ERR_INVALID_ARG),
     ((16, -128, 4, 64), wq.QGEMM_ERR_INVALID_ARG),
+    (((1 << 30) + 16, 128, 4, 64), wq.QGEMM_ERR_UNSUPPORTED),   # N above 2^30
+    ((16, (1 << 30) + 128, 2, 128), wq.QGEMM_ERR_UNSUPPORTED),  # K above 2^30
 ])
 def test_pack_sizes_rejects(args, status):
     with pytest.raises(wq.QGemmError) as e:
@@ -98,6 +100,8 @@ def _call(desc, X=0x10000, M=64, out=0x20000, bias=None, path=0):
     (dict(biases=0), wq.QGEMM_ERR_INVALID_ARG),      # affine needs biases
     (dict(packed=0x1008), wq.QGEMM_ERR_ALIGNMENT),
     (dict(scales=0x2002), wq.QGEMM_ERR_ALIGNMENT),
+    (dict(N=(1 << 30) + 16), wq.QGEMM_ERR_UNSUPPORTED),         # above the 2^30 limit
+    (dict(K=(1 << 30) + 128), wq.QGEMM_ERR_UNSUPPORTED),
 ])
 def test_qgemm_rejects_bad_weights_without_device(kw, status):
     assert _call(_desc(**kw)) == status
@@ -116,6 +120,8 @@ def test_qgemm_rejects_bad_operands_without_device():
     assert _call(d, path=wq.QGEMM_PATH_LARGE_M | 0x200) == wq.QGEMM_ERR_INVALID_ARG   # unknown flag bit
     assert _call(d, M=0, path=wq.QGEMM_PATH_SMALL_M | wq.QGEMM_FLAG_OVERLAP_PREVIOUS) == wq.QGEMM_OK
     assert _call(d, M=17, path=wq.QGEMM_PATH_SMALL_M) == wq.QGEMM_ERR_UNSUPPORTED
+    assert _call(d, M=(1 << 30) + 1) == wq.QGEMM_ERR_UNSUPPORTED                      # above the 2^30 limit
+    assert _call(d, M=(1 << 31) - 1) == wq.QGEMM_ERR_UNSUPPORTED
     # M = 0 is a no-op that never touches the device
     assert _call(d, M=0) == wq.QGEMM_OK
     # ternary needs no biases
@@ -143,6 +149,9 @@ def test_select_path_table():
         assert wq.qgemm_select_path(4096, 9216, 3072, bits) == wq.QGEMM_PATH_LARGE_M
     with pytest.raises(wq.QGemmError):
         wq.qgemm_select_path(1, 16, 128, 3)
+    with pytest.raises(wq.QGemmError) as e:
+        wq.qgemm_select_path((1 << 31) - 1, 16, 128, 4)
+    assert e.value.status == wq.QGEMM_ERR_UNSUPPORTED
 
 
 def test_missing_library_fails_loudly_on_first_call(tmp_path):

@@ -528,6 +528,8 @@ int launch_fmt(const Problem& pr, int nsm) {
   kp.K = pr.K;
   kp.num_m_tiles = (pr.M + TILE_M - 1) / TILE_M;
   kp.num_n_tiles = (pr.N + TILE_N - 1) / TILE_N;
+  if (static_cast<int64_t>(kp.num_m_tiles) * kp.num_n_tiles > INT32_MAX)
+    return fail(QGEMM_ERR_UNSUPPORTED, "M=%d x N=%d: more output tiles than one launch indexes", pr.M, pr.N);
   kp.num_tiles = kp.num_m_tiles * kp.num_n_tiles;
   kp.num_kb = pr.K / BK;
   const int grid = kp.num_tiles < nsm ? kp.num_tiles : nsm;

@@ -41,6 +41,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 int validate_weights(const qgemm_weights* W) {
   if (!W) return fail(QGEMM_ERR_INVALID_ARG, "null weights descriptor");
   if (W->N <= 0 || W->K <= 0) return fail(QGEMM_ERR_INVALID_ARG, "N=%d K=%d must be positive", W->N, W->K);
+  if (W->N > kMaxDim || W->K > kMaxDim)
+    return fail(QGEMM_ERR_UNSUPPORTED, "N=%d K=%d: at most %d each", W->N, W->K, kMaxDim);
   const bool fmt_ok = (W->bits == 4 && W->group == 64) || (W->bits == 8 && W->group == 64) ||
                       (W->bits == 2 && W->group == 128) || (W->bits == 1 && W->group == 128);
   if (!fmt_ok) return fail(QGEMM_ERR_UNSUPPORTED, "unsupported format bits=%d group=%d", W->bits, W->group);
@@ -93,6 +95,7 @@ extern "C" int qgemm_fused(const void* X, int32_t M, const qgemm_weights* W, voi
   int st = validate_weights(W);
   if (st != QGEMM_OK) return st;
   if (M < 0) return fail(QGEMM_ERR_INVALID_ARG, "M=%d is negative", M);
+  if (M > kMaxDim) return fail(QGEMM_ERR_UNSUPPORTED, "M=%d: at most %d", M, kMaxDim);
   const int32_t flags = path & ~0xFF;
   path &= 0xFF;
   if (path < QGEMM_PATH_AUTO || path > QGEMM_PATH_LARGE_M) return fail(QGEMM_ERR_INVALID_ARG, "bad path %d", path);
@@ -148,6 +151,7 @@ extern "C" int qgemm(const void* X, int32_t M, const qgemm_weights* W, void* out
 
 extern "C" int qgemm_select_path(int32_t M, int32_t N, int32_t K, int32_t bits) {
   if (M < 0 || N <= 0 || K <= 0) return -QGEMM_ERR_INVALID_ARG;
+  if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return -QGEMM_ERR_UNSUPPORTED;
   if (bits != 1 && bits != 2 && bits != 4 && bits != 8) return -QGEMM_ERR_UNSUPPORTED;
   std::call_once(g_env_once, read_env);
   if (g_env_path != QGEMM_PATH_AUTO) return g_env_path == QGEMM_PATH_SMALL_M && M > 16 ? QGEMM_PATH_LARGE_M : g_env_path;

@@ -64,6 +64,10 @@ int launch_pack_device(const float* W, int N, int K, int bits, void* packed, uin
                        cudaStream_t stream);
 
 // Device status word values (0 = fine).
+// Largest M, N or K the library accepts (2^30): keeps every launcher's int
+// arithmetic (rounded-up tile and stage counts) inside int32.
+constexpr int32_t kMaxDim = 1 << 30;
+
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusLayout = 2u;  // dynamic shared memory not aligned as the kernel requires
 constexpr unsigned kStatusPackNonfinite = 4u;  // qgemm_pack_device met a NaN or an infinity

@@ -157,6 +157,8 @@ int pack_rows(const PackJob& jb, int r0, int r1) {
 
 int check_format(int32_t N, int32_t K, int32_t bits, int32_t group) {
   if (N <= 0 || K <= 0) return qg::fail(QGEMM_ERR_INVALID_ARG, "N and K must be positive (N=%d K=%d)", N, K);
+  if (N > qg::kMaxDim || K > qg::kMaxDim)
+    return qg::fail(QGEMM_ERR_UNSUPPORTED, "N=%d K=%d: at most %d each", N, K, qg::kMaxDim);
   const bool ok = (bits == 4 && group == 64) || (bits == 8 && group == 64) || (bits == 2 && group == 128) ||
                   (bits == 1 && group == 128);
   if (!ok) return qg::fail(QGEMM_ERR_UNSUPPORTED, "unsupported format bits=%d group=%d", bits, group);
