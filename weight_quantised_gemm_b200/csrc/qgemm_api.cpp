@@ -1,5 +1,6 @@
 // The C ABI: argument validation, path choice and dispatch to the kernels.
 
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -14,7 +15,7 @@ namespace qg {
 
 namespace {
 thread_local std::string t_last_error;
-uint64_t g_wait_limit_ns = 0;  // 0 = not yet resolved
+std::atomic<uint64_t> g_wait_limit_ns{0};  // 0 = not yet resolved; read by every launch, set by any thread
 std::once_flag g_env_once;
 int g_env_path = QGEMM_PATH_AUTO;
 
@@ -27,7 +28,8 @@ void read_env() {
   }
   if (const char* w = std::getenv("QGEMM_WAIT_LIMIT_NS")) {
     const unsigned long long v = std::strtoull(w, nullptr, 10);
-    if (v > 0 && g_wait_limit_ns == 0) g_wait_limit_ns = v;
+    uint64_t unset = 0;
+    if (v > 0) g_wait_limit_ns.compare_exchange_strong(unset, v);
   }
 }
 
@@ -74,7 +76,8 @@ int cuda_check(cudaError_t e, const char* what) {
 
 uint64_t wait_limit_ns() {
   std::call_once(g_env_once, read_env);
-  return g_wait_limit_ns ? g_wait_limit_ns : kDefaultWaitLimitNs;
+  const uint64_t v = g_wait_limit_ns.load();
+  return v ? v : kDefaultWaitLimitNs;
 }
 
 int select_path(int M, int N, int K, int bits) {
@@ -177,7 +180,7 @@ extern "C" int qgemm_dequant_tile(const qgemm_weights* W, int32_t n0, int32_t k0
 
 extern "C" int qgemm_set_wait_limit_ns(uint64_t limit_ns) {
   std::call_once(g_env_once, read_env);
-  g_wait_limit_ns = limit_ns ? limit_ns : kDefaultWaitLimitNs;
+  g_wait_limit_ns.store(limit_ns ? limit_ns : kDefaultWaitLimitNs);
   return QGEMM_OK;
 }
 
