@@ -736,6 +736,9 @@ def cpu_oracle_single_core():
     return out
 
 
+REFERENCE_SECONDS = 150.0   # the reference arm's whole run (warm-up and timed steps)
+
+
 def run_reference(args, rank, world):
     """The base contract's reference arm, here the oracle on the host cores:
     each step is a bounded sample of the headline workload."""
@@ -749,18 +752,22 @@ def run_reference(args, rank, world):
     X, W, bias = WL.make_inputs(lin, HEADLINE_CID, HEADLINE_LIN)
     p, s, b = O.pack_ref(W, lin.bits, lin.group)
     total_steps = args.steps + args.warmup
-    budget = 150.0 / max(total_steps, 1)       # seconds per step so the run ends within minutes
+    budget = REFERENCE_SECONDS / max(total_steps, 1)   # seconds per step so the run ends within minutes
+
+    def w_rows(n):
+        # the first n rows of W: scales and biases are group-major [K / group, N]
+        return O.wq_exact(p[:n], s[:, :n], None if b is None else b[:, :n], lin.bits, lin.group, lin.K)
+
     # a step: dequantise a block of W rows and multiply a block of X rows with it
-    n_rows = lin.N
     t0 = time.perf_counter()
-    Wq = O.wq_exact(p[:256], s[:256], None if b is None else b[:256], lin.bits, lin.group, lin.K)
+    w_rows(256)
     t_deq_256 = time.perf_counter() - t0
     n_rows = int(max(64, min(lin.N, 256 * budget * 0.5 / max(t_deq_256, 1e-6))))
     n_rows -= n_rows % 16
     m_rows = 64
 
     def one_step():
-        Wq = O.wq_exact(p[:n_rows], s[:n_rows], None if b is None else b[:n_rows], lin.bits, lin.group, lin.K)
+        Wq = w_rows(n_rows)
         out = O.bf16_bits_to_f64(X[:m_rows]) @ Wq.T
         if bias is not None:
             out += O.bf16_bits_to_f64(bias[:n_rows])[None, :]

@@ -39,3 +39,20 @@ def test_reason_bits_are_distinct():
     assert len(set(bits)) == len(bits)
     names = {n for n, _ in bench.ClockSampler.REASONS}
     assert {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"} <= names
+
+
+def test_reference_arm_prints_a_complete_line(monkeypatch):
+    """The reference arm (the oracle on the host cores) runs end to end on a
+    small budget and reports the contract's keys; rank 0 alone works."""
+    import argparse
+
+    monkeypatch.setattr(bench, "REFERENCE_SECONDS", 1.0)
+    args = argparse.Namespace(steps=2, warmup=1)
+    assert bench.run_reference(args, 1, 2) is None          # other ranks do no work
+    r = bench.run_reference(args, 0, 1)
+    assert r["impl"] == "reference" and r["steps"] == 2 and r["warmup"] == 1
+    assert r["value"] > 0 and r["unit"] == "TFLOP/s" and r["higher_is_better"] is True
+    cb = r["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == r["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert r["e2e"] == {"value": r["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert r["config"]["M"] == 4096 and r["config"]["N"] == 9216 and r["config"]["K"] == 3072
