@@ -56,3 +56,14 @@ def test_reference_arm_prints_a_complete_line(monkeypatch):
     assert cb["kind"] == "oracle" and cb["value"] == r["value"] and cb["cores"] >= 1 and cb["sample"]
     assert r["e2e"] == {"value": r["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert r["config"]["M"] == 4096 and r["config"]["N"] == 9216 and r["config"]["K"] == 3072
+
+
+def test_cpu_baseline_legs_run_on_the_host():
+    """The main arm's CPU-baseline legs (the oracle on a bounded sample of the
+    headline workload, and the single-core runs) need no GPU: run them on a
+    small budget and check what they report."""
+    tflops, spent, desc, rows = bench.cpu_oracle_sample(0.5)
+    assert tflops > 0 and spent > 0 and 16 <= rows <= 4096 and "extrapolated" in desc
+    single = bench.cpu_oracle_single_core()
+    assert set(single) == {"0:tiny", "3:tern_m1"}
+    assert all(v["seconds"] > 0 and v["gflops"] > 0 for v in single.values())
