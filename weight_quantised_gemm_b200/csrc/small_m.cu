@@ -24,7 +24,7 @@
 //   stage.
 // * Eight consumer warps. Normally warp w takes scale group w of every stage
 //   for all the CTA's rows; where that would not fit in registers (16 tokens
-//   and 12 or more row pairs) the rows split into two halves and warps w and
+//   and 6 or more 16-row pairs) the rows split into two halves and warps w and
 //   w + 4 take groups w % 4 and w % 4 + 4 of every stage, each for its half.
 //   A warp turns codes into bf16 in registers and feeds warp-level mma.sync
 //   (m16n8k16, bf16 in, fp32 accumulate): the weights are the 16-row A
