@@ -126,6 +126,18 @@ def test_small_path_ragged(bits, M):
 
 
 @pytest.mark.parametrize("bits", [1, 2, 4, 8])
+@pytest.mark.parametrize("M,N", [(16, 12288), (11, 16384)])
+def test_small_path_split_rows(bits, M, N):
+    """More than 8 tokens and 96 or more weight rows per CTA (N above 9472 on
+    148 SMs: 6 or 8 16-row pairs): the rows split into two halves, each warp
+    takes two groups per stage, and the activations come through the ring."""
+    K = 1024
+    X, W, bias = WL.random_case(M + N + bits, M, N, K, bits, with_bias=True)
+    y, _ = gpu_qgemm(X, W, bias, bits, path=SMALL)
+    _assert_close(y, _ref(X, W, bias, bits), f"small split rows bits={bits} M={M} N={N}")
+
+
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
 @pytest.mark.parametrize("M,N,K", [(1, 128, 128), (17, 144, 256), (255, 272, 384), (256, 256, 512),
                                    (257, 400, 640), (600, 528, 1024)])
 def test_large_path_ragged(bits, M, N, K):
