@@ -126,15 +126,17 @@ def test_small_path_ragged(bits, M):
 
 
 @pytest.mark.parametrize("bits", [1, 2, 4, 8])
-@pytest.mark.parametrize("M,N", [(16, 12288), (11, 16384)])
-def test_small_path_split_rows(bits, M, N):
-    """More than 8 tokens and 96 or more weight rows per CTA (N above 9472 on
-    148 SMs: 6 or 8 16-row pairs): the rows split into two halves, each warp
-    takes two groups per stage, and the activations come through the ring."""
-    K = 1024
+@pytest.mark.parametrize("M,N", [(5, 8176), (3, 12272), (5, 16368), (16, 8176), (16, 12272), (11, 16368)])
+def test_small_path_every_row_count(bits, M, N):
+    """Every rows-per-CTA choice beyond the smallest at both token widths: on
+    148 SMs N = 8176, 12272 and 16368 take 4, 6 and 8 16-row pairs per CTA,
+    each one pair short of whole CTAs, so the last CTA is ragged. With more
+    than 8 tokens, 6 or 8 pairs split the rows into halves, each warp taking
+    two groups per stage, and the activations come through the ring."""
+    K = 512
     X, W, bias = WL.random_case(M + N + bits, M, N, K, bits, with_bias=True)
     y, _ = gpu_qgemm(X, W, bias, bits, path=SMALL)
-    _assert_close(y, _ref(X, W, bias, bits), f"small split rows bits={bits} M={M} N={N}")
+    _assert_close(y, _ref(X, W, bias, bits), f"small bits={bits} M={M} N={N}")
 
 
 @pytest.mark.parametrize("bits", [1, 2, 4, 8])
