@@ -288,7 +288,7 @@ def dequant_ref(packed, scales, biases, bits: int, group: int, K: int) -> np.nda
 
 def qgemm_ref(X_bits, packed, scales, biases, bits: int, group: int, K: int,
               bias_bits=None) -> np.ndarray:
-    """fp64 out[M, N] = X . Wq_exact^T (+ bias): the reference the kernels are judged by."""
+    """fp64 out[M, N] = X . Wq_exact^T (+ bias): the reference the kernels are checked against."""
     X = bf16_bits_to_f64(X_bits)
     out = X @ wq_exact(packed, scales, biases, bits, group, K).T
     if bias_bits is not None:

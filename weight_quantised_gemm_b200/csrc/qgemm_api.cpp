@@ -33,9 +33,10 @@ void read_env() {
   }
 }
 
-// Largest M served by the small-M path, per format. Measured on B200: see the
-// path sweep in the design notes; below the crossover the weights' bytes set the
-// time and the register path streams them faster than the tile pipeline fills.
+// Largest M served by the small-M path, per format, from timing both paths at
+// M = 1..64 on B200 (the bench's path crossover sweep): below the crossover the
+// weights' bytes set the time and the register path streams them faster than
+// the tile pipeline fills.
 #include "path_table.inc"
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

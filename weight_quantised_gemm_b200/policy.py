@@ -1,7 +1,7 @@
 """Mixed-precision policy: which bit width each linear of a model gets.
 
 The method holds most layers at 4 bits and the layers that multiply the
-residual stream at 8, and judges a policy by the cosine of the model's output
+residual stream at 8, and rates a policy by the cosine of the model's output
 against the dense one and by its size against dense (stable-diffusion.rs
 README, introduction). This module chooses such policies from measurements:
 given, for every linear, its dense output and its output at each candidate
