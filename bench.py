@@ -672,8 +672,8 @@ def policy_sweep():
     """Every assignment of 4 or 8 bits to the five linears of the mixed FLUX
     block (workload 4), on its synthetic weights: the block's cosine against
     dense bf16 (outputs concatenated) and its packed size, with the Pareto
-    front marked. The pages' policy (the layers that multiply the residual
-    stream at 8 bits, the rest at 4) is one of the 32."""
+    front marked. The pages' policy (8 bits for the linears whose output
+    scales the residual stream, 4 for the rest) is one of the 32."""
     import itertools
 
     import torch

@@ -1,24 +1,25 @@
 /*
  * qgemm — weight-only quantised GEMM for NVIDIA B200 (sm_100a).
  *
- * The operation (stable-diffusion.rs README, introduction): weights are held
- * quantised at rest as packed bits and are dequantised inside the matmul one
- * tile at a time, so a layer whose dense weights would not fit still runs.
+ * The operation (stable-diffusion.rs README, introduction): weights stay
+ * packed in their quantised form in memory and are expanded to bf16 within the
+ * GEMM kernel itself, tile by tile, so a layer whose dense weights would not
+ * fit still runs.
  *
  *     out[M, N] = X[M, K] . dequant(W)[N, K]^T (+ bias[N])
  *
  * with X and out in bf16, W packed in one of four formats, and fp32
- * accumulation throughout (pictor README, numerics: fp32 accumulate is kept,
- * no TF32 or FP16-MAC shortcuts).
+ * accumulation throughout (pictor README, numerics: accumulation stays in
+ * fp32, without reduced-precision TF32 or fp16 multiply-accumulate).
  *
  * Formats (the pages give no bit layout, scale formula or rounding rule; this
  * library fixes the following):
  *   bits = 4 or 8, group = 64   group-wise affine, w ~ s * q + b, with an fp16
  *                               scale s and an fp16 bias b per 64 consecutive
  *                               k of a row, q in [0, 2^bits - 1]
- *                               (stable-diffusion.rs README, introduction: the
- *                               layers that multiply the residual stream at 8
- *                               bits, the rest at 4);
+ *                               (stable-diffusion.rs README, introduction: 8
+ *                               bits for the linears whose output scales the
+ *                               residual stream, 4 for the others);
  *   bits = 2, group = 128       ternary t in {-1, 0, +1} with one fp16 scale per
  *                               128 consecutive k (pictor README, "Extreme
  *                               quantization is first-class": TQ2_0_g128);
@@ -193,8 +194,8 @@ int qgemm_ex(const void* X, int32_t M, const qgemm_weights* W, void* out,
 
 /* Fused epilogues for qgemm_fused: the elementwise steps on either side of a
  * FLUX block's linears. The pages (stable-diffusion.rs README, introduction)
- * name "the layers that multiply the residual stream" without formulas; these
- * are FLUX's: the MLP up projection's tanh GELU, and a residual-writing
+ * single out the linears whose output scales the residual stream but give no
+ * formulas; these are FLUX's: the MLP up projection's tanh GELU, and a residual-writing
  * layer's gated update of the residual stream. v = acc + bias in fp32; the
  * result is rounded to bf16 once. */
 enum {

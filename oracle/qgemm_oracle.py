@@ -8,9 +8,9 @@ two meet only through the seeded inputs of ``workloads.py``.
 
 What the method computes
 ------------------------
-stable-diffusion.rs README (andreinknv), introduction: weights are held
-quantised at rest as packed bits and are dequantised inside the matmul, one
-tile at a time. The result it reaches is, up to rounding order, the plain
+stable-diffusion.rs README (andreinknv), introduction: weights stay packed
+in their quantised form and are expanded to full precision within the GEMM
+kernel, tile by tile. The result it reaches is, up to rounding order, the plain
 product of the activations with the dequantised weights, so this oracle is
 that definition written out in fp64:
 
@@ -21,8 +21,9 @@ formula and no rounding rule):
 
 * 4-bit and 8-bit group-wise affine, groups of 64 consecutive k in a row:
   ``w ~ s16 * q + b16`` with fp16 scale s16 and fp16 bias b16 per group,
-  q in [0, 2^b - 1]. The pages' "4-bit everywhere ... held at 8 bits and the
-  rest at 4" (stable-diffusion.rs README, introduction) names the two widths.
+  q in [0, 2^b - 1]. The two widths are the pages' (stable-diffusion.rs
+  README, introduction: 4 bits for most linears, 8 for those whose output
+  scales the residual stream).
 * ternary {-1, 0, +1} with one fp16 scale per group of 128
   (pictor README, "Extreme quantization is first-class": TQ2_0_g128).
 * 1-bit {-1, +1} with one fp16 scale per group of 128 (the same README's
@@ -66,7 +67,8 @@ Dequantised weight (the bit-exact contract of the dequant-tile entry point):
 * 1-bit: wdeq = c * bf16_rn(fl32(s16)).
 
 Numerics of the matmul: fp32 accumulation is what the kernels keep (pictor
-README, numerics: "FP32 accumulate is kept", no TF32 or FP16-MAC shortcuts);
+README, numerics: accumulation stays in fp32, without reduced-precision TF32
+or fp16 multiply-accumulate);
 the oracle accumulates in fp64.
 """
 from __future__ import annotations
@@ -325,11 +327,11 @@ def dense_ref(X_bits, W, bias_bits=None) -> np.ndarray:
 
 # ----------------------------------------------------------------------------
 # fused epilogues: the elementwise steps on either side of a FLUX block's
-# linears (stable-diffusion.rs README, introduction: the layers "that multiply
-# the residual stream"). The pages give no formula; the readings are FLUX's
-# own: the MLP's up projection is followed by the tanh-approximate GELU, and a
-# residual-writing linear's output y updates the stream as r + gate * y with
-# one gate value per output feature.
+# linears (stable-diffusion.rs README, introduction, singles out the linears
+# whose output scales the residual stream). The pages give no formula; the
+# readings are FLUX's own: the MLP's up projection is followed by the
+# tanh-approximate GELU, and a residual-writing linear's output y updates the
+# stream as r + gate * y with one gate value per output feature.
 # ----------------------------------------------------------------------------
 
 EPI_NONE, EPI_GELU_TANH, EPI_RESIDUAL_GATE = 0, 1, 2

@@ -2,8 +2,9 @@
 // (A from TMEM, B from shared memory) -> bf16 TMA stores. One persistent CTA
 // per SM.
 //
-// "Dequantised inside the matmul kernel a tile at a time" (stable-diffusion.rs
-// README, introduction) maps onto Blackwell as follows. Each output tile is
+// The method expands packed weights to bf16 within the GEMM kernel itself,
+// tile by tile (stable-diffusion.rs README, introduction); on Blackwell that
+// maps as follows. Each output tile is
 // 128 weight rows x 256 tokens, computed as D[n, m] = sum_k Wdeq[n, k] X[m, k]
 // by tcgen05.mma with M = 128 (weight rows), N = 256 (tokens), K = 16 per
 // instruction, bf16 inputs and fp32 accumulation in tensor memory. Putting the

@@ -1,7 +1,7 @@
 // qgemm_pack_device: the at-rest packing of qgemm_pack, run on the GPU over a
-// device fp32 weight, bit-identical to the host packer. The weights are "held
-// quantised at rest, packed bits" (stable-diffusion.rs README, introduction);
-// this makes that step a device pass for weights that already live in HBM.
+// device fp32 weight, bit-identical to the host packer. The method stores its
+// weights packed (stable-diffusion.rs README, introduction); this makes the
+// packing a device pass for weights that already live in HBM.
 //
 // One thread packs one (row, group): it takes the same fp64 steps in the same
 // order as the host packer (min / max, or max |w|, or a running sum of |w|;

@@ -1,6 +1,6 @@
-// At-rest file format of a packed weight: the "held quantised at rest,
-// packed bits" form (stable-diffusion.rs README, introduction) written to
-// and read from disk. Host-only; plain stdio.
+// At-rest file format of a packed weight: the stored, still-quantised form of
+// the weights (stable-diffusion.rs README, introduction, keeps weights packed
+// when stored) written to and read from disk. Host-only; plain stdio.
 //
 // Layout, little-endian:
 //   bytes 0-7    magic "QGEMMW01"

@@ -1,8 +1,8 @@
 // Host packer: round-to-nearest group quantisation of fp32 weights into the
 // at-rest format described in include/qgemm.h.
 //
-// The weights are "held quantised at rest — packed bits" (stable-diffusion.rs
-// README, introduction); this is the offline step that produces those bits.
+// The method stores its weights packed (stable-diffusion.rs README,
+// introduction); this is the offline step that produces those bits.
 // All decisions are taken in fp64 with ties to even, and the fp64 -> fp16
 // rounding is written here from the IEEE 754 binary16 definition.
 

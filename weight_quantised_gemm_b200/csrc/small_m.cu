@@ -1,8 +1,9 @@
 // Small-M path (M <= 16): a memory-bound kernel that streams the packed
 // weights once.
 //
-// pictor's README ("Extreme quantization is first-class") names GEMV paths
-// built for sub-byte weights; at decode-sized M the packed bytes set the time,
+// pictor's README ("Extreme quantization is first-class") has GEMV paths
+// designed around weights narrower than a byte; at decode-sized M the packed
+// bytes set the time,
 // so this kernel is built around keeping HBM busy from its first microsecond:
 //
 // * One CTA per SM owns 16 * NP consecutive weight rows (it takes most of the

@@ -1,6 +1,6 @@
 """Mixed-precision policy: which bit width each linear of a model gets.
 
-The method holds most layers at 4 bits and the layers that multiply the
+The method keeps most linears at 4 bits and those whose output scales the
 residual stream at 8, and rates a policy by the cosine of the model's output
 against the dense one and by its size against dense (stable-diffusion.rs
 README, introduction). This module chooses such policies from measurements:
