@@ -797,6 +797,17 @@ def run_reference(args, rank, world):
 
 # ----------------------------------------------------------------------------
 
+def report_section(res: dict, key: str, fn):
+    """Runs an optional part of the report after the headline measurement:
+    a failure is recorded in the line (`errors`) instead of losing the
+    measurement already taken. Returns fn()'s result, or None."""
+    try:
+        return fn()
+    except Exception as e:  # noqa: BLE001 - any failure of an optional section
+        res.setdefault("errors", {})[key] = f"{type(e).__name__}: {e}"[:500]
+        return None
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -836,17 +847,18 @@ def main(argv=None):
         res, peaks = run_ours(args, rank, world, local_rank)
         if rank == 0:
             if not args.no_sweep and world == 1:
-                per, block, cross = sweep(peaks)
-                res["sweep"] = per
-                res["workload4_block"] = block
-                res["path_crossover"] = cross
-                res["fused_epilogues"] = fused_sweep()
-                res["policy_sweep"] = policy_sweep()
+                out = report_section(res, "sweep", lambda: sweep(peaks))
+                if out is not None:
+                    res["sweep"], res["workload4_block"], res["path_crossover"] = out
+                res["fused_epilogues"] = report_section(res, "fused_epilogues", fused_sweep)
+                res["policy_sweep"] = report_section(res, "policy_sweep", policy_sweep)
             if not args.no_cpu and world == 1:
-                v, spent, desc, _ = cpu_oracle_sample(args.cpu_seconds)
-                res["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOP/s", "cores": blas_threads(),
-                                       "kind": "oracle", "sample": desc, "seconds": round(spent, 2)}
-                res["cpu_oracle_single_core"] = cpu_oracle_single_core()
+                def cpu_legs():
+                    v, spent, desc, _ = cpu_oracle_sample(args.cpu_seconds)
+                    res["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOP/s", "cores": blas_threads(),
+                                           "kind": "oracle", "sample": desc, "seconds": round(spent, 2)}
+                    res["cpu_oracle_single_core"] = cpu_oracle_single_core()
+                report_section(res, "cpu_baseline", cpu_legs)
             res["peaks"] = peaks
             print(json.dumps(res), flush=True)
     finally:

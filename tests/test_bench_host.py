@@ -67,3 +67,13 @@ def test_cpu_baseline_legs_run_on_the_host():
     single = bench.cpu_oracle_single_core()
     assert set(single) == {"0:tiny", "3:tern_m1"}
     assert all(v["seconds"] > 0 and v["gflops"] > 0 for v in single.values())
+
+
+def test_an_optional_section_that_fails_is_recorded_not_fatal():
+    res = {"value": 1.0}
+    assert bench.report_section(res, "ok", lambda: 3) == 3 and "errors" not in res
+
+    def boom():
+        raise RuntimeError("out of memory")
+    assert bench.report_section(res, "sweep", boom) is None
+    assert res["errors"] == {"sweep": "RuntimeError: out of memory"} and res["value"] == 1.0
