@@ -120,6 +120,8 @@ def bf16_bits_to_f64(b) -> np.ndarray:
 # ----------------------------------------------------------------------------
 
 def codes_per_word(bits: int) -> int:
+    """Codes per little-endian 32-bit word of the packed layout (32 / bits). The pages give no
+    bit layout; this is the layout the module header fixes."""
     return 32 // bits
 
 
@@ -132,7 +134,8 @@ def code_bit_position(bits: int, j: int) -> int:
 
 
 def pack_codes(codes, bits: int) -> np.ndarray:
-    """Integer codes [N, K] -> packed bytes [N, K * bits / 8].
+    """Integer codes [N, K] -> packed bytes [N, K * bits / 8], in the bit
+    layout the module header fixes (the pages give none).
 
     Affine codes are q in [0, 2^b - 1]; ternary codes are t in {-1, 0, +1}
     and are stored as 2-bit two's complement; 1-bit codes are c in {-1, +1},
@@ -158,7 +161,8 @@ def pack_codes(codes, bits: int) -> np.ndarray:
 
 
 def unpack_codes(packed, bits: int, K: int) -> np.ndarray:
-    """Packed bytes [N, K * bits / 8] -> integer codes [N, K] (int32).
+    """Packed bytes [N, K * bits / 8] -> integer codes [N, K] (int32): the
+    inverse of pack_codes.
 
     Raises ValueError on the invalid ternary code 10.
     """
@@ -187,6 +191,9 @@ def unpack_codes(packed, bits: int, K: int) -> np.ndarray:
 # ----------------------------------------------------------------------------
 
 def check_format(bits: int, group: int, K: int) -> None:
+    """The (bits, group) pairs the formats define: 64 for the affine widths the mixed policy uses
+    (stable-diffusion.rs README, introduction), 128 for TQ2_0_g128 and Q1_0_g128 (pictor README,
+    "Extreme quantization is first-class"); K a whole number of groups."""
     if bits in AFFINE_BITS:
         if group != 64:
             raise ValueError("affine formats use groups of 64")
@@ -200,7 +207,9 @@ def check_format(bits: int, group: int, K: int) -> None:
 
 
 def pack_ref(W, bits: int, group: int):
-    """RTN group quantisation of fp32 W [N, K].
+    """RTN group quantisation of fp32 W [N, K]: the packing that keeps weights
+    quantised in memory (stable-diffusion.rs README, introduction), with the
+    scale, bias and rounding readings of the module header.
 
     Returns (packed uint8 [N, K*b/8], scales fp16 [K/g, N], biases fp16
     [K/g, N] or None for ternary), in the at-rest layout.
@@ -252,7 +261,8 @@ def _expand(groupwise, group: int) -> np.ndarray:
 
 
 def wq_exact(packed, scales, biases, bits: int, group: int, K: int) -> np.ndarray:
-    """The quantised weight before any bf16 rounding, fp64 [N, K]: s16*q + b16 or s16*t."""
+    """The quantised weight before any bf16 rounding, fp64 [N, K]: s16*q + b16 or s16*t (or s16*c):
+    the weights the method multiplies by, exactly (stable-diffusion.rs README, introduction)."""
     codes = unpack_codes(packed, bits, K).astype(np.float64)
     s = _expand(scales, group)
     if bits in (TERNARY_BITS, BINARY_BITS):
@@ -261,7 +271,9 @@ def wq_exact(packed, scales, biases, bits: int, group: int, K: int) -> np.ndarra
 
 
 def dequant_ref_bits(packed, scales, biases, bits: int, group: int, K: int) -> np.ndarray:
-    """The dequantised weight as bf16 bits [N, K] (the bit-exact contract).
+    """The dequantised weight as bf16 bits [N, K] (the bit-exact contract):
+    the tile the method expands to inside the matmul (stable-diffusion.rs
+    README, introduction), in the precision the module header fixes.
 
     affine: s16*q + b16 is exact in fp64 (at most 11+8 significant bits in the
     product and an fp16 addend; the sum spans under 53 bits), so casting it to
@@ -280,7 +292,7 @@ def dequant_ref_bits(packed, scales, biases, bits: int, group: int, K: int) -> n
 
 
 def dequant_ref(packed, scales, biases, bits: int, group: int, K: int) -> np.ndarray:
-    """The dequantised weight as fp64 values [N, K]."""
+    """The dequantised weight as fp64 values [N, K] (dequant_ref_bits, widened exactly)."""
     return bf16_bits_to_f64(dequant_ref_bits(packed, scales, biases, bits, group, K))
 
 
@@ -290,7 +302,9 @@ def dequant_ref(packed, scales, biases, bits: int, group: int, K: int) -> np.nda
 
 def qgemm_ref(X_bits, packed, scales, biases, bits: int, group: int, K: int,
               bias_bits=None) -> np.ndarray:
-    """fp64 out[M, N] = X . Wq_exact^T (+ bias): the reference the kernels are checked against."""
+    """fp64 out[M, N] = X . Wq_exact^T (+ bias): the reference the kernels are checked against.
+    The matmul against the dequantised weights (stable-diffusion.rs README, introduction), taken in
+    fp64 where the kernels keep fp32 accumulation (pictor README, numerics)."""
     X = bf16_bits_to_f64(X_bits)
     out = X @ wq_exact(packed, scales, biases, bits, group, K).T
     if bias_bits is not None:
@@ -316,7 +330,8 @@ def qgemm_ref_rows(rows, X_bits, packed, scales, biases, bits: int, group: int, 
 
 
 def dense_ref(X_bits, W, bias_bits=None) -> np.ndarray:
-    """fp64 X . bf16_rn(W)^T (+ bias): the dense bf16 layer the quantised one replaces."""
+    """fp64 X . bf16_rn(W)^T (+ bias): the dense bf16 layer the quantised one replaces, the
+    reference of the cosine the mixed policy is rated by (stable-diffusion.rs README, introduction)."""
     X = bf16_bits_to_f64(X_bits)
     Wb = bf16_bits_to_f64(bf16_rn_bits(np.asarray(W, dtype=np.float32)))
     out = X @ Wb.T
@@ -373,6 +388,7 @@ MAX_ABS_TOL = 3e-2       # max |Y - ref| / max |ref|
 
 
 def rel_frobenius(y, ref) -> float:
+    """||y - ref||_F / ||ref||_F: half of the parity gate applied to the kernels (<= REL_FROB_TOL)."""
     y = np.asarray(y, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     den = np.linalg.norm(ref)
@@ -380,6 +396,7 @@ def rel_frobenius(y, ref) -> float:
 
 
 def max_abs_rel(y, ref) -> float:
+    """max |y - ref| / max |ref|: the other half of the parity gate (<= MAX_ABS_TOL)."""
     y = np.asarray(y, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     den = np.max(np.abs(ref)) if ref.size else 0.0
@@ -388,12 +405,15 @@ def max_abs_rel(y, ref) -> float:
 
 
 def cosine(a, b) -> float:
+    """Cosine of two outputs, flattened: the accuracy measure the mixed policy is rated by, against
+    the dense output (stable-diffusion.rs README, introduction)."""
     a = np.asarray(a, dtype=np.float64).ravel()
     b = np.asarray(b, dtype=np.float64).ravel()
     return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b)))
 
 
 def within_tolerance(y, ref) -> bool:
+    """Both halves of the parity gate at once."""
     return rel_frobenius(y, ref) <= REL_FROB_TOL and max_abs_rel(y, ref) <= MAX_ABS_TOL
 
 
