@@ -3,6 +3,7 @@ point include/qgemm.h declares, and rejects bad arguments with the documented
 status before touching a device."""
 import ctypes
 import os
+import pathlib
 import re
 
 import numpy as np
@@ -14,7 +15,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _declared_functions():
-    src = open(os.path.join(ROOT, "include", "qgemm.h")).read()
+    src = pathlib.Path(ROOT, "include", "qgemm.h").read_text()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(qgemm[a-z_]*)\s*\(", src)))
 

@@ -2,6 +2,7 @@
 round trips of every format, and the documented rejections."""
 import ctypes
 import os
+import pathlib
 import struct
 
 import numpy as np
@@ -47,7 +48,7 @@ def test_rejects_corrupt_files(tmp_path):
     pw = wq.qgemm_pack(WL.random_case(8, 1, 32, 256, 4, with_bias=False)[1], 4)
     good = str(tmp_path / "good.qgw")
     pw.save(good)
-    data = open(good, "rb").read()
+    data = pathlib.Path(good).read_bytes()
     bad = str(tmp_path / "bad.qgw")
     for blob, status in [(b"XGEMMW01" + data[8:], wq.QGEMM_ERR_INVALID_ARG),        # magic
                          (data[:40], wq.QGEMM_ERR_INVALID_ARG),                     # short header
@@ -55,7 +56,7 @@ def test_rejects_corrupt_files(tmp_path):
                          (data + b"\0", wq.QGEMM_ERR_INVALID_ARG),                  # trailing bytes
                          (data[:8] + struct.pack("<4i", 32, 256, 3, 64) + data[24:], wq.QGEMM_ERR_UNSUPPORTED),
                          (data[:24] + struct.pack("<Q", 1) + data[32:], wq.QGEMM_ERR_INVALID_ARG)]:  # sizes
-        open(bad, "wb").write(blob)
+        pathlib.Path(bad).write_bytes(blob)
         _expect(bad, status)
     _expect(str(tmp_path / "missing.qgw"), wq.QGEMM_ERR_INVALID_ARG)
 
@@ -68,11 +69,11 @@ def test_truncation_at_every_offset_and_a_lying_header(tmp_path):
     pw = wq.qgemm_pack(WL.random_case(9, 1, 16, 128, 4, with_bias=False)[1], 4)
     good = str(tmp_path / "good.qgw")
     pw.save(good)
-    data = open(good, "rb").read()
+    data = pathlib.Path(good).read_bytes()
     bad = str(tmp_path / "bad.qgw")
     N, K, bits, group = (ctypes.c_int32() for _ in range(4))
     for cut in list(range(len(data))) + [len(data) + 1]:
-        open(bad, "wb").write(data[:cut] if cut < len(data) else data + b"\0")
+        pathlib.Path(bad).write_bytes(data[:cut] if cut < len(data) else data + b"\0")
         st = wq._lib.qgemm_load_header(bad.encode(), ctypes.byref(N), ctypes.byref(K), ctypes.byref(bits),
                                        ctypes.byref(group))
         assert st == wq.QGEMM_ERR_INVALID_ARG, cut
@@ -80,7 +81,7 @@ def test_truncation_at_every_offset_and_a_lying_header(tmp_path):
     # a consistent header for [2^20, 2^20] 8-bit weights (1 TiB of codes) over the small file's bytes
     n = k = 1 << 20
     lying = data[:8] + struct.pack("<4i3Q", n, k, 8, 64, n * k, n * (k // 64) * 2, n * (k // 64) * 2) + data[48:]
-    open(bad, "wb").write(lying)
+    pathlib.Path(bad).write_bytes(lying)
     st = wq._lib.qgemm_load_header(bad.encode(), ctypes.byref(N), ctypes.byref(K), ctypes.byref(bits),
                                    ctypes.byref(group))
     assert st == wq.QGEMM_ERR_INVALID_ARG

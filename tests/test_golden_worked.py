@@ -11,6 +11,7 @@ away from even or a -0.0 coded as negative fails here.
 """
 import glob
 import os
+import pathlib
 
 import numpy as np
 import pytest
@@ -25,7 +26,7 @@ FIXTURES = sorted(glob.glob(os.path.join(GOLDEN, "*.txt")))
 
 def _load(path):
     d = {}
-    for line in open(path):
+    for line in pathlib.Path(path).read_text().splitlines():
         if line.startswith("#") or not line.strip():
             continue
         key, *vals = line.split()

@@ -46,7 +46,7 @@ def _worker(rank, world, port, results):
 def test_two_gloo_ranks_take_the_slowest_rank():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:   # no fork of this multi-threaded process
         results = mgr.dict()
         mp.spawn(_worker, args=(world, port, results), nprocs=world, join=True)
         out = dict(results)
