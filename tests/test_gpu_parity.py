@@ -257,6 +257,28 @@ def test_overlap_reads_the_previous_kernels_output(bits):
         _assert_close(from_dev_bf16(y2), _ref(y1_bits, W2, bias2, bits), "second, overlapped")
 
 
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
+def test_overlap_with_split_rows_reads_the_previous_kernels_output(bits):
+    """The same chain with 16 tokens and N2 = 9728 in the overlapped call: 6
+    16-row pairs per CTA, so the rows split into halves and the producer, not
+    the consumers, waits for the previous grid before it copies the
+    activations into the ring."""
+    M, K1, N1, N2 = 16, 1024, 1024, 9728
+    X, W1, _ = WL.random_case(191 + bits, M, N1, K1, bits, with_bias=False)
+    _, W2, bias2 = WL.random_case(192 + bits, M, N2, N1, bits, with_bias=True)
+    d1, d2 = wq.qgemm_pack(W1, bits).to_device(), wq.qgemm_pack(W2, bits).to_device()
+    Xd, b2 = to_dev_bf16(X), to_dev_bf16(bias2)
+    ref1 = _ref(X, W1, None, bits)
+    for _ in range(2):
+        y1 = torch.full((M, N1), float("nan"), dtype=torch.bfloat16, device="cuda")
+        y1 = wq.qgemm(Xd, d1, out=y1, path=SMALL)
+        y2 = wq.qgemm(y1, d2, bias=b2, path=SMALL, overlap_previous=True)
+        wq.check_device_status()
+        y1_bits = from_dev_bf16(y1)
+        _assert_close(y1_bits, ref1, "first")
+        _assert_close(from_dev_bf16(y2), _ref(y1_bits, W2, bias2, bits), "second, overlapped, split rows")
+
+
 def test_overlap_after_a_torch_kernel_and_in_a_graph():
     """The previous kernel is a plain torch one (no trigger of its own), and the
     same overlapped call captured in a CUDA graph gives the same result."""
@@ -316,6 +338,15 @@ def _fused_case(bits, M, N, K, op, seed, path, in_place=False):
 def test_fused_epilogue_parity(op, bits, path, M):
     y, ref = _fused_case(bits, M, 400, 768, op, 100 + 10 * op + bits + M, path)
     _assert_close(y, ref, f"op={op} bits={bits} path={path} M={M}")
+
+
+@pytest.mark.parametrize("op", [wq.QGEMM_EPI_GELU_TANH, wq.QGEMM_EPI_RESIDUAL_GATE])
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
+def test_fused_epilogue_with_split_rows(op, bits):
+    """The fused epilogues on the small-M path with 16 tokens and 6 16-row
+    pairs per CTA (N = 12272): rows split into halves, activations in the ring."""
+    y, ref = _fused_case(bits, 16, 12272, 512, op, 300 + 10 * op + bits, SMALL)
+    _assert_close(y, ref, f"split rows op={op} bits={bits}")
 
 
 @pytest.mark.parametrize("path,M", [(SMALL, 5), (LARGE, 257)])
