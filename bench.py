@@ -696,6 +696,15 @@ def policy_sweep():
             del dw
         wq.check_device_status()
     dense_bytes = sum(2 * l.N * l.K for l in wl.linears)
+    # the per-layer terms the policy module works from, reduced on the device
+    terms = []
+    for li, lin in enumerate(wl.linears):
+        dl = yd[li]
+        opts = {}
+        for bits in (4, 8):
+            e = yq[(li, bits)] - dl
+            opts[bits] = (sizes[(li, bits)], float(e @ dl), float(e @ e))
+        terms.append((lin.name, float(dl @ dl), opts))
     rows = []
     d = torch.cat(yd)
     for combo in itertools.product((4, 8), repeat=len(wl.linears)):
@@ -713,7 +722,23 @@ def policy_sweep():
     rows.sort(key=lambda r: r["packed_over_dense_bf16"])
     del yq, yd
     torch.cuda.empty_cache()
-    return rows
+    return {"assignments": rows, "policy_module": policy_module_report(terms, dense_bytes, rows)}
+
+
+def policy_module_report(terms, dense_bytes, rows, min_cosine=0.999):
+    """The policy module's answers from per-layer terms (name, ||d||^2,
+    {bits: (bytes, <e, d>, ||e||^2)}), with its cosines checked against the
+    directly computed ones of `rows` (every assignment, as policy_sweep
+    reports them)."""
+    import weight_quantised_gemm_b200.policy as P
+    layers = [P.LayerStats(n, D, {b: P.Option(b, nb, a, e) for b, (nb, a, e) in o.items()}) for n, D, o in terms]
+    front = P.frontier(layers)
+    worst = max(abs(P.cosine(layers, r["bits"]) - r["cosine_vs_dense_bf16"]) for r in rows)
+    best = P.cheapest(layers, min_cosine)
+    return {"front": [{"bits": p.bits, "cosine_vs_dense_bf16": p.cosine,
+                       "packed_over_dense_bf16": round(p.nbytes / dense_bytes, 4)} for p in front],
+            "max_abs_cosine_difference_vs_direct": worst,
+            f"cheapest_with_cosine_at_least_{min_cosine}": None if best is None else best.bits}
 
 
 def cpu_oracle_single_core():

@@ -77,3 +77,40 @@ def test_an_optional_section_that_fails_is_recorded_not_fatal():
         raise RuntimeError("out of memory")
     assert bench.report_section(res, "sweep", boom) is None
     assert res["errors"] == {"sweep": "RuntimeError: out of memory"} and res["value"] == 1.0
+
+
+def test_policy_module_report_agrees_with_direct_cosines():
+    """The bench's policy report from per-layer terms, on synthetic outputs:
+    its cosines equal the ones computed directly, and its front and cheapest
+    policy are those of the enumeration."""
+    import itertools
+
+    import numpy as np
+    g = np.random.default_rng(3)
+    names = ["a", "b", "c"]
+    dense, quant, nbytes = {}, {}, {}
+    for n in names:
+        d = g.standard_normal(200)
+        dense[n] = d
+        for bits, amp in ((4, 0.1), (8, 0.006)):
+            quant[(n, bits)] = d + amp * g.standard_normal(200)
+            nbytes[(n, bits)] = 100 * bits + len(n)
+    terms = []
+    for n in names:
+        d = dense[n]
+        opts = {b: (nbytes[(n, b)], float((quant[(n, b)] - d) @ d), float((quant[(n, b)] - d) @ (quant[(n, b)] - d)))
+                for b in (4, 8)}
+        terms.append((n, float(d @ d), opts))
+    rows = []
+    dcat = np.concatenate([dense[n] for n in names])
+    for combo in itertools.product((4, 8), repeat=3):
+        q = np.concatenate([quant[(n, b)] for n, b in zip(names, combo)])
+        rows.append({"bits": dict(zip(names, combo)),
+                     "cosine_vs_dense_bf16": float(q @ dcat / np.sqrt((q @ q) * (dcat @ dcat)))})
+    r = bench.policy_module_report(terms, 10_000, rows, min_cosine=0.9999)
+    assert r["max_abs_cosine_difference_vs_direct"] < 1e-12
+    assert r["front"][0]["bits"] == {"a": 4, "b": 4, "c": 4} and r["front"][-1]["bits"] == {"a": 8, "b": 8, "c": 8}
+    best = r["cheapest_with_cosine_at_least_0.9999"]
+    ok = [row for row in rows if row["cosine_vs_dense_bf16"] >= 0.9999]
+    cheapest = min(ok, key=lambda row: sum(nbytes[(n, b)] for n, b in row["bits"].items()))
+    assert best == cheapest["bits"]
