@@ -89,3 +89,31 @@ def test_truncation_at_every_offset_and_a_lying_header(tmp_path):
     # and the untouched file still loads
     back = wq.qgemm_load(good)
     assert np.array_equal(back.packed, pw.packed)
+
+
+def test_round_trip_property_over_shapes_and_formats(tmp_path):
+    """Any supported shape and format: save then load gives back the same
+    bytes, and the file is exactly the header plus the three arrays."""
+    pytest.importorskip("hypothesis")
+    from hypothesis import HealthCheck, given, settings, strategies as st
+
+    @settings(max_examples=25, deadline=None, derandomize=True, database=None,
+              suppress_health_check=list(HealthCheck))
+    @given(bits=st.sampled_from([1, 2, 4, 8]), n16=st.integers(1, 6), k128=st.integers(1, 8),
+           seed=st.integers(0, 2 ** 16))
+    def check(bits, n16, k128, seed):
+        N, K = 16 * n16, 128 * k128
+        W = (np.random.default_rng(seed).standard_normal((N, K)) * 0.02).astype(np.float32)
+        pw = wq.qgemm_pack(W, bits)
+        path = str(tmp_path / f"p{bits}_{N}_{K}.qgw")
+        pw.save(path)
+        back = wq.qgemm_load(path)
+        assert (back.N, back.K, back.bits, back.group) == (N, K, bits, wq.GROUP_OF_BITS[bits])
+        assert np.array_equal(back.packed, pw.packed)
+        assert np.array_equal(back.scales.view(np.uint16), pw.scales.view(np.uint16))
+        assert (back.biases is None) == (pw.biases is None)
+        if pw.biases is not None:
+            assert np.array_equal(back.biases.view(np.uint16), pw.biases.view(np.uint16))
+        assert os.path.getsize(path) == 48 + pw.nbytes
+
+    check()
