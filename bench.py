@@ -482,7 +482,7 @@ def run_ours(args, rank, world, local_rank):
             "clocks_detail": clk,
             "impl": "ours",
         }
-    return result, peaks
+    return result, peaks, sets[0][3]
 
 
 def run_case(args):
@@ -741,6 +741,29 @@ def policy_module_report(terms, dense_bytes, rows, min_cosine=0.999):
             f"cheapest_with_cosine_at_least_{min_cosine}": None if best is None else best.bits}
 
 
+def headline_parity(out, rows: int = 64) -> dict:
+    """Part of the CPU-baseline leg: the oracle on sampled rows of the
+    headline workload (the first rows and rows spread over all M), against
+    the output of the timed run (`out`, the bf16 [M, N] tensor it wrote),
+    with the parity gate's two measures."""
+    import numpy as np
+    import torch
+
+    import oracle as O
+    import workloads as WL
+    lin = WL.workload(HEADLINE_CID).linears[HEADLINE_LIN]
+    X, W, bias = WL.make_inputs(lin, HEADLINE_CID, HEADLINE_LIN)
+    p, s, b = O.pack_ref(W, lin.bits, lin.group)
+    idx = np.unique(np.concatenate([np.arange(rows // 2), np.linspace(0, lin.M - 1, rows // 2).astype(np.int64)]))
+    ref = O.qgemm_ref_rows(idx, X, p, s, b, lin.bits, lin.group, lin.K, bias)
+    got = out[torch.as_tensor(idx, device=out.device)].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    y = O.bf16_bits_to_f64(got)
+    return {"rows_checked": int(idx.size), "rel_frobenius": O.rel_frobenius(y, ref), "max_abs_rel": O.max_abs_rel(y, ref),
+            "within_tolerance": bool(O.within_tolerance(y, ref)),
+            "tolerance": {"rel_frobenius": O.REL_FROB_TOL, "max_abs_rel": O.MAX_ABS_TOL},
+            "reference": "oracle (fp64, exact quantised weights)"}
+
+
 def cpu_oracle_single_core():
     """The oracle on one host core for config 0 (tiny) and config 3 at M=1
     (ternary decode): seconds per GEMM, dequantisation included."""
@@ -869,7 +892,7 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        res, peaks = run_ours(args, rank, world, local_rank)
+        res, peaks, headline_out = run_ours(args, rank, world, local_rank)
         if rank == 0:
             if not args.no_sweep and world == 1:
                 out = report_section(res, "sweep", lambda: sweep(peaks))
@@ -883,6 +906,7 @@ def main(argv=None):
                     res["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOP/s", "cores": blas_threads(),
                                            "kind": "oracle", "sample": desc, "seconds": round(spent, 2)}
                     res["cpu_oracle_single_core"] = cpu_oracle_single_core()
+                    res["parity"] = headline_parity(headline_out)
                 report_section(res, "cpu_baseline", cpu_legs)
             res["peaks"] = peaks
             print(json.dumps(res), flush=True)

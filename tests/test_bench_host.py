@@ -114,3 +114,26 @@ def test_policy_module_report_agrees_with_direct_cosines():
     ok = [row for row in rows if row["cosine_vs_dense_bf16"] >= 0.9999]
     cheapest = min(ok, key=lambda row: sum(nbytes[(n, b)] for n, b in row["bits"].items()))
     assert best == cheapest["bits"]
+
+
+def test_headline_parity_accepts_the_oracle_and_rejects_a_corrupt_output():
+    """The parity check of the timed run's output, given an output built on
+    the host: the oracle's own result rounded to bf16 passes, the same with a
+    corrupted row does not."""
+    import numpy as np
+    import torch
+
+    import oracle as O
+    import workloads as WL
+    lin = WL.workload(bench.HEADLINE_CID).linears[bench.HEADLINE_LIN]
+    X, W, bias = WL.make_inputs(lin, bench.HEADLINE_CID, bench.HEADLINE_LIN)
+    p, s, b = O.pack_ref(W, lin.bits, lin.group)
+    rows = np.unique(np.concatenate([np.arange(32), np.linspace(0, lin.M - 1, 32).astype(np.int64)]))
+    y = np.zeros((lin.M, lin.N), dtype=np.float32)
+    y[rows] = O.qgemm_ref_rows(rows, X, p, s, b, lin.bits, lin.group, lin.K, bias)
+    out = torch.from_numpy(y).to(torch.bfloat16)
+    r = bench.headline_parity(out)
+    assert r["rows_checked"] == rows.size and r["within_tolerance"] and r["rel_frobenius"] < 3e-3
+    out[rows[5]] = -out[rows[5]]
+    r = bench.headline_parity(out)
+    assert not r["within_tolerance"]
