@@ -3,9 +3,12 @@
 
 One step = one qgemm over the headline workload (FLUX double-stream image
 QKV projection: X bf16 [4096, 3072] times a 4-bit group-64 W [9216, 3072]
-plus a bf16 bias), inputs resident in HBM. Prints ONE JSON line (rank 0).
+plus a bf16 bias), inputs resident in HBM. Prints ONE JSON line on stdout
+(rank 0): the headline, a few KB. The detailed sections (every workload
+linear, the path crossover, the fused epilogues, the policy sweep) go to
+stderr as JSON lines of their own, and to --report FILE when given.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--report FILE]
 
 Multi-GPU (torchrun, one process per GPU): the GEMM runs as independent
 replicas, one per rank, with no collective on the data path ("scaling":
@@ -455,34 +458,43 @@ def run_ours(args, rank, world, local_rank):
 
     result = None
     if rank == 0:
-        value = job["tflops"]
-        achieved = flops / kernel_max / 1e12
-        traffic, traffic_src = profiled_traffic()
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": traffic,
-                "peak_source": peaks["source"] + ", burst bf16 (kernel timed on its own)",
-                "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
-                "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": ab,
-                "traffic_source": traffic_src, "kernel": "large_m_kernel<4>"}
-        result = {
-            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(elapsed_max / args.steps * 1e3, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded; W ~ N(0,0.02) RTN 4-bit g64, X ~ N(0,1), bias ~ N(0,0.01))",
-            "config": {"workload": "FLUX double-stream image QKV projection: X bf16 [4096,3072] x W 4-bit "
-                                   "group-64 [9216,3072] + bias bf16 [9216] -> bf16 [4096,9216]",
-                       "M": lin.M, "N": lin.N, "K": lin.K, "bits": lin.bits, "group": lin.group,
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": f"inputs rotate over {ncopy} copies ({ncopy * ab / 1e6:.0f} MB > 126 MB L2)"},
-            "gbs": round(ab * args.steps * world / elapsed_max / 1e9, 1),
-            "roofline": roof,
-            "e2e": e2e,
-            "gpu_launches": args.steps,
-            "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
-            "clocks_detail": clk,
-            "impl": "ours",
-        }
+        result = assemble_ours(args, world, lin, ncopy, job, kernel_max, e2e, clk, peaks)
     return result, peaks, sets[0][3]
+
+
+def assemble_ours(args, world, lin, ncopy, job, kernel_s, e2e, clk, peaks) -> dict:
+    """The headline result of our arm from its measurements: `job` from
+    replica_throughput, `kernel_s` the mean per-launch event time (max over
+    ranks), `e2e` from run_e2e, `clk` from ClockSampler.stop()."""
+    flops = 2 * lin.M * lin.N * lin.K
+    ab = alg_bytes(lin)
+    achieved = flops / kernel_s / 1e12
+    traffic, traffic_src = profiled_traffic()
+    roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": traffic,
+            "peak_source": peaks["source"] + ", burst bf16 (kernel timed on its own)",
+            "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
+            "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": ab,
+            "traffic_source": traffic_src, "kernel": f"large_m_kernel<{lin.bits}>"}
+    elapsed = job["elapsed_s"]
+    return {
+        "metric": METRIC, "value": round(job["tflops"], 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(elapsed / args.steps * 1e3, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; W ~ N(0,0.02) RTN 4-bit g64, X ~ N(0,1), bias ~ N(0,0.01))",
+        "config": {"workload": "FLUX double-stream image QKV projection: X bf16 [4096,3072] x W 4-bit "
+                               "group-64 [9216,3072] + bias bf16 [9216] -> bf16 [4096,9216]",
+                   "M": lin.M, "N": lin.N, "K": lin.K, "bits": lin.bits, "group": lin.group,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"inputs rotate over {ncopy} copies ({ncopy * ab / 1e6:.0f} MB > 126 MB L2)"},
+        "gbs": round(ab * args.steps * world / elapsed / 1e9, 1),
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": {k: clk.get(k) for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "clocks_detail": clk,
+        "impl": "ours",
+    }
 
 
 def run_case(args):
@@ -593,10 +605,24 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def cpu_oracle_sample(target_s: float, lin=None, cid=HEADLINE_CID, li=HEADLINE_LIN):
-    """Times the oracle (dequant of the whole W + fp64 matmul) on a bounded
-    sample of the workload's rows and extrapolates to the full M: returns
-    (TFLOP/s, seconds spent, description)."""
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's guess."""
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def cpu_oracle_sample(target_s: float, lin=None, cid=HEADLINE_CID, li=HEADLINE_LIN, runs: int = 3):
+    """Times the oracle (dequantisation of the whole W + fp64 matmul) on a
+    bounded sample of the workload's rows, `runs` times, and extrapolates the
+    median run to the full M: returns (TFLOP/s, seconds spent, description,
+    sample rows, per-run TFLOP/s)."""
     import numpy as np
 
     import oracle as O
@@ -604,28 +630,43 @@ def cpu_oracle_sample(target_s: float, lin=None, cid=HEADLINE_CID, li=HEADLINE_L
     lin = WL.workload(cid).linears[li] if lin is None else lin
     X, W, bias = WL.make_inputs(lin, cid, li)
     p, s, b = O.pack_ref(W, lin.bits, lin.group)
-    t0 = time.perf_counter()
-    Wq = O.wq_exact(p, s, b, lin.bits, lin.group, lin.K)
-    t_deq = time.perf_counter() - t0
-    rows = 16
-    spent = t_deq
-    t_mm = 0.0
-    while True:
+
+    def one(rows):
+        t0 = time.perf_counter()
+        Wq = O.wq_exact(p, s, b, lin.bits, lin.group, lin.K)
+        t_deq = time.perf_counter() - t0
         t1 = time.perf_counter()
-        Xs = O.bf16_bits_to_f64(X[:rows])
-        out = Xs @ Wq.T
+        out = O.bf16_bits_to_f64(X[:rows]) @ Wq.T
         if bias is not None:
             out += O.bf16_bits_to_f64(bias)[None, :]
-        t_mm = time.perf_counter() - t1
-        spent += t_mm
-        if spent >= target_s * 0.5 or rows >= lin.M:
+        return t_deq, time.perf_counter() - t1
+
+    # the sample: grow the rows until one run takes its share of the budget or covers M
+    rows, spent = 16, 0.0
+    while True:
+        t_deq, t_mm = one(rows)
+        spent += t_deq + t_mm
+        if t_deq + t_mm >= target_s / (2 * runs) or rows >= lin.M:
             break
         rows = min(lin.M, rows * 4)
-    t_full = t_deq + t_mm * lin.M / rows
     flops = 2 * lin.M * lin.N * lin.K
-    desc = (f"oracle (numpy fp64): dequant of the full W [{lin.N},{lin.K}] ({t_deq:.2f} s) + matmul of "
-            f"X rows 0..{rows - 1} of {lin.M} ({t_mm:.2f} s), extrapolated to all {lin.M} rows")
-    return flops / t_full / 1e12, spent, desc, rows
+    per_run = []
+    for _ in range(runs):
+        t_deq, t_mm = one(rows)
+        spent += t_deq + t_mm
+        per_run.append(flops / (t_deq + t_mm * lin.M / rows) / 1e12)
+    med = statistics.median(per_run)
+    desc = (f"oracle (numpy fp64): dequantisation of the full W [{lin.N},{lin.K}] + matmul of X rows "
+            f"0..{rows - 1} of {lin.M}, extrapolated to all {lin.M} rows; median of {runs} runs")
+    return med, spent, desc, rows, per_run
+
+
+def cpu_baseline(target_s: float) -> dict:
+    """The main arm's cpu_baseline: the oracle on the host cores, median of
+    three runs of a bounded sample of the headline workload."""
+    v, spent, desc, rows, per_run = cpu_oracle_sample(target_s)
+    return {"value": round(v, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle", "sample": desc,
+            "cpu_model": cpu_model(), "runs_tflops": [round(x, 6) for x in per_run], "seconds": round(spent, 2)}
 
 
 def fused_sweep():
@@ -839,7 +880,8 @@ def run_reference(args, rank, world):
                                    "group-64 [9216,3072] + bias bf16 [9216] -> bf16 [4096,9216]",
                        "M": lin.M, "N": lin.N, "K": lin.K, "bits": lin.bits, "group": lin.group},
             "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample,
+                             "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -856,6 +898,57 @@ def report_section(res: dict, key: str, fn):
         return None
 
 
+class Reporter:
+    """The detailed report sections (per-workload sweep, path crossover, fused
+    epilogues, policy sweep): one JSON line each on stderr, and the same lines
+    appended to `path` when one is given. stdout carries only the headline."""
+
+    def __init__(self, path=None):
+        self.path = path
+        if path:
+            os.makedirs(os.path.dirname(os.path.abspath(path)), exist_ok=True)
+            open(path, "w").close()
+
+    def __call__(self, section: str, data) -> None:
+        line = json.dumps({"report": section, "data": data})
+        print(line, file=sys.stderr, flush=True)
+        if self.path:
+            with open(self.path, "a") as fh:
+                fh.write(line + "\n")
+
+
+HEADLINE_KEYS = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                 "scaling", "vs_baseline", "dtype", "data", "config", "gbs", "roofline", "e2e", "gpu_launches",
+                 "clocks", "cpu_baseline", "parity", "peaks", "sweep_summary", "errors", "impl")
+HEADLINE_MAX_BYTES = 6000
+
+
+def sweep_summary(sweep_rows, block, cross) -> dict:
+    """A few numbers per workload linear for the headline line: microseconds
+    per launch (CUDA graph) and the fraction of the shape's roofline; the
+    full rows go to the report sections."""
+    out = {}
+    for e in sweep_rows or ():
+        out[f"{e['workload']}:{e['linear']}"] = [e["us"], e["frac_of_roofline"]]
+    if block:
+        out["4:block"] = [block["us_total"], block.get("cosine_vs_dense_bf16_all_five")]
+    return out
+
+
+def headline_line(res: dict) -> str:
+    """The one JSON line the bench prints on stdout: the contract's keys and
+    the short summaries, never the detailed sections (those go to the
+    Reporter). Long optional values are dropped, in reverse order of
+    importance, until the line is within HEADLINE_MAX_BYTES."""
+    line = {k: res[k] for k in HEADLINE_KEYS if k in res}
+    for drop in ("sweep_summary", "errors", "parity", "peaks", "clocks_detail"):
+        s = json.dumps(line)
+        if len(s) <= HEADLINE_MAX_BYTES:
+            return s
+        line.pop(drop, None)
+    return json.dumps(line)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -865,6 +958,8 @@ def main(argv=None):
     ap.add_argument("--no-sweep", action="store_true", help="skip the per-workload sweep")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--report", default=None,
+                    help="also write the detailed report sections (JSON lines) to this file")
     ap.add_argument("--case", default=None,
                     help="time one workload linear alone, e.g. 3:tern_m1:M=16 (workload:linear[:M=..])")
     args = ap.parse_args(argv)
@@ -894,22 +989,30 @@ def main(argv=None):
     try:
         res, peaks, headline_out = run_ours(args, rank, world, local_rank)
         if rank == 0:
+            report = Reporter(args.report)
             if not args.no_sweep and world == 1:
                 out = report_section(res, "sweep", lambda: sweep(peaks))
                 if out is not None:
-                    res["sweep"], res["workload4_block"], res["path_crossover"] = out
-                res["fused_epilogues"] = report_section(res, "fused_epilogues", fused_sweep)
-                res["policy_sweep"] = report_section(res, "policy_sweep", policy_sweep)
+                    rows, block, cross = out
+                    report("sweep", rows)
+                    report("workload4_block", block)
+                    report("path_crossover", cross)
+                    res["sweep_summary"] = sweep_summary(rows, block, cross)
+                fused = report_section(res, "fused_epilogues", fused_sweep)
+                if fused is not None:
+                    report("fused_epilogues", fused)
+                pol = report_section(res, "policy_sweep", policy_sweep)
+                if pol is not None:
+                    report("policy_sweep", pol)
             if not args.no_cpu and world == 1:
                 def cpu_legs():
-                    v, spent, desc, _ = cpu_oracle_sample(args.cpu_seconds)
-                    res["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOP/s", "cores": blas_threads(),
-                                           "kind": "oracle", "sample": desc, "seconds": round(spent, 2)}
-                    res["cpu_oracle_single_core"] = cpu_oracle_single_core()
+                    res["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+                    report("cpu_oracle_single_core", cpu_oracle_single_core())
                     res["parity"] = headline_parity(headline_out)
                 report_section(res, "cpu_baseline", cpu_legs)
             res["peaks"] = peaks
-            print(json.dumps(res), flush=True)
+            report("clocks_detail", res.get("clocks_detail"))
+            print(headline_line(res), flush=True)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -62,8 +62,10 @@ def test_cpu_baseline_legs_run_on_the_host():
     """The main arm's CPU-baseline legs (the oracle on a bounded sample of the
     headline workload, and the single-core runs) need no GPU: run them on a
     small budget and check what they report."""
-    tflops, spent, desc, rows = bench.cpu_oracle_sample(0.5)
+    tflops, spent, desc, rows, runs = bench.cpu_oracle_sample(0.5)
     assert tflops > 0 and spent > 0 and 16 <= rows <= 4096 and "extrapolated" in desc
+    assert len(runs) == 3 and tflops == sorted(runs)[1]
+    assert bench.cpu_model()
     single = bench.cpu_oracle_single_core()
     assert set(single) == {"0:tiny", "3:tern_m1"}
     assert all(v["seconds"] > 0 and v["gflops"] > 0 for v in single.values())
@@ -137,3 +139,63 @@ def test_headline_parity_accepts_the_oracle_and_rejects_a_corrupt_output():
     out[rows[5]] = -out[rows[5]]
     r = bench.headline_parity(out)
     assert not r["within_tolerance"]
+
+
+def test_main_arm_prints_one_compact_headline_line(monkeypatch, capsys):
+    """The main arm end to end with its GPU measurements stubbed: stdout
+    holds exactly one line, valid JSON within HEADLINE_MAX_BYTES carrying the
+    contract's keys, even when the detailed sections are large; those go to
+    stderr (and the --report file) as lines of their own."""
+    import json
+
+    import torch
+
+    import workloads as WL
+    lin = WL.workload(bench.HEADLINE_CID).linears[bench.HEADLINE_LIN]
+    peaks = {"hbm_gbs": 6553.9, "bf16_tflops": 1638.3, "bf16_tflops_sustained": 1379.1, "source": "test"}
+    clk = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 40}
+    e2e = {"value": 160.0, "unit": "TFLOP/s", "h2d_bytes_per_step": lin.M * lin.K * 2,
+           "d2h_bytes_per_step": lin.M * lin.N * 2}
+
+    def fake_run_ours(args, rank, world, local_rank):
+        job = bench.replica_throughput(2 * lin.M * lin.N * lin.K, args.steps, args.steps * 180e-6, world)
+        res = bench.assemble_ours(args, world, lin, 4, job, 178e-6, e2e, clk, peaks)
+        return res, peaks, None
+
+    big_rows = [{"workload": 4, "linear": f"lin{i}", "us": 100.0 + i, "frac_of_roofline": 0.8, "pad": "x" * 400}
+                for i in range(40)]
+    block = {"us_total": 1184.0, "cosine_vs_dense_bf16_all_five": 0.998}
+    monkeypatch.setattr(torch.cuda, "set_device", lambda *_: None)
+    monkeypatch.setattr(bench, "run_ours", fake_run_ours)
+    monkeypatch.setattr(bench, "sweep", lambda peaks: (big_rows, block, [{"pad": "y" * 300}] * 50))
+    monkeypatch.setattr(bench, "fused_sweep", lambda: [{"pad": "z" * 500}] * 10)
+    monkeypatch.setattr(bench, "policy_sweep", lambda: {"assignments": [{"pad": "w" * 200}] * 32})
+    monkeypatch.setattr(bench, "cpu_baseline", lambda s: {"value": 0.4, "unit": "TFLOP/s", "cores": 16,
+                                                          "kind": "oracle", "sample": "stub", "cpu_model": "cpu"})
+    monkeypatch.setattr(bench, "cpu_oracle_single_core", lambda: {"0:tiny": {"seconds": 0.1}})
+    monkeypatch.setattr(bench, "headline_parity", lambda out: {"within_tolerance": True})
+    assert bench.main(["--steps", "20", "--warmup", "5"]) == 0
+    cap = capsys.readouterr()
+    lines = cap.out.strip().splitlines()
+    assert len(lines) == 1
+    assert len(lines[0]) <= bench.HEADLINE_MAX_BYTES
+    r = json.loads(lines[0])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "config", "dtype",
+              "roofline", "cpu_baseline", "e2e", "clocks", "parity", "peaks", "gpu_launches", "higher_is_better"):
+        assert k in r, k
+    assert r["value"] > 0 and r["steps"] == 20 and r["warmup"] == 5 and r["n_gpus"] == 1
+    assert abs(r["ms_per_step"] - 0.18) < 1e-9
+    assert r["roofline"]["bound"] == "tensor" and 0 < r["roofline"]["frac"] < 1.2
+    assert r["e2e"]["h2d_bytes_per_step"] > 0 and r["e2e"]["d2h_bytes_per_step"] > 0
+    assert r["sweep_summary"]["4:lin0"] == [100.0, 0.8]
+    assert "sweep" not in r and "policy_sweep" not in r and "clocks_detail" not in r
+    sections = [json.loads(x)["report"] for x in cap.err.splitlines() if x.startswith('{"report"')]
+    assert {"sweep", "path_crossover", "fused_epilogues", "policy_sweep", "workload4_block"} <= set(sections)
+
+
+def test_headline_line_drops_summaries_before_exceeding_its_size():
+    import json
+    res = {"metric": "m", "value": 1.0, "sweep_summary": {f"k{i}": [1.0, 0.5] for i in range(2000)}}
+    line = bench.headline_line(res)
+    assert len(line) <= bench.HEADLINE_MAX_BYTES
+    assert json.loads(line) == {"metric": "m", "value": 1.0}
