@@ -39,11 +39,9 @@ Packing is round-to-nearest (RTN) in fp64, ties to even:
 * ternary: s16 = fp16(max |w|); t = clamp(rint(w / s16), -1, 1), t = 0 where
   s16 == 0.
 * 1-bit: s16 = fp16(mean |w|), the scale that minimises the squared error
-  for fixed signs, with the sum of |w| taken in fp64 in k order (a running
-  sum) and then divided by 128; c = +1 where w >= 0 (-0 included), else -1.
-  The order is part of the reading: this sum decides a stored value, and on
-  groups whose values span many binades another order can round it to the
-  neighbouring fp16 value.
+  for fixed signs, rounded once (to nearest, ties to even) from the exact
+  mean of the group's 128 magnitudes; c = +1 where w >= 0 (-0 included),
+  else -1.
 
 Bit layout, row-major over N with K contiguous, little-endian 32-bit words:
 
@@ -73,6 +71,9 @@ the oracle accumulates in fp64.
 """
 from __future__ import annotations
 
+import math
+from fractions import Fraction
+
 import numpy as np
 
 AFFINE_BITS = (4, 8)
@@ -92,6 +93,42 @@ def fp16_rn(x) -> np.ndarray:
     """
     with np.errstate(over="ignore"):    # overflow gives inf, which the callers refuse
         return np.asarray(x, dtype=np.float64).astype(np.float16)
+
+
+def fp16_rn_exact(q: Fraction) -> np.float16:
+    """The fp16 value nearest to the exact rational q >= 0, ties to the even
+    encoding; +inf at and above 65520 (the largest finite fp16, 65504, plus
+    half its spacing).
+
+    Written from the definition: the nearest of the fp16 values that bracket
+    q, found around a first guess and compared exactly.
+    """
+    if q >= 65520:
+        return np.float16(np.inf)
+    guess = np.float16(float(q))
+    cands = {guess, np.nextafter(guess, np.float16(0)), np.nextafter(guess, np.float16(65504))}
+    return min(cands, key=lambda c: (abs(Fraction(float(c)) - q), int(np.array(c).view(np.uint16)) & 1))
+
+
+def mean_abs_fp16(values) -> np.float16:
+    """fp16 of the exact mean of |values| (fp32 weights), rounded once.
+
+    math.fsum gives the exact sum rounded once to fp64; dividing by the
+    group size (a power of two) keeps that exact. Rounding that fp64 value to
+    fp16 gives the same answer as rounding the exact mean, except where the
+    fp64 neighbourhood of the mean straddles an fp16 rounding boundary; only
+    then is the mean formed exactly (fractions.Fraction) and rounded from
+    there.
+    """
+    a = [abs(float(v)) for v in values]
+    n = len(a)
+    v = math.fsum(a) / n
+    lo, hi = np.nextafter(v, -np.inf), np.nextafter(v, np.inf)
+    with np.errstate(over="ignore"):
+        r = np.float16(v)
+        if np.float16(lo) == r == np.float16(hi):
+            return r
+    return fp16_rn_exact(sum(Fraction(x) for x in a) / n)
 
 
 def bf16_rn_bits(x32) -> np.ndarray:
@@ -236,7 +273,14 @@ def pack_ref(W, bits: int, group: int):
         codes = q.reshape(N, K).astype(np.int64)
         return pack_codes(codes, bits), np.ascontiguousarray(s16.T), np.ascontiguousarray(b16.T)
     if bits == BINARY_BITS:
-        s16 = fp16_rn(np.add.accumulate(np.abs(Wg), axis=2)[:, :, -1] / group)
+        # numpy's fp64 sum of 128 non-negative terms is within a relative
+        # 127 * 2^-53 < 2^-46 of the exact sum; where fp16 rounding gives one
+        # value over a relative 2^-40 either side, that is the fp16 of the exact
+        # mean, and the few groups where it does not go through mean_abs_fp16
+        v = np.abs(Wg).sum(axis=2) / group
+        s16 = fp16_rn(v * (1.0 - 2.0 ** -40))
+        for n, j in zip(*np.nonzero(s16 != fp16_rn(v * (1.0 + 2.0 ** -40)))):
+            s16[n, j] = mean_abs_fp16(Wg[n, j])
         if not np.all(np.isfinite(s16)):
             raise OverflowError("scale overflows fp16")
         c = np.where(Wg >= 0, 1, -1)

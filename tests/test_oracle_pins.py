@@ -525,30 +525,92 @@ def test_1bit_dequant_is_signed_scale_and_gemm_matches_triple_loop():
     assert O.format_bytes(12288, 3072, 1, 128) == 12288 * 3072 // 8 + 12288 * 24 * 2
 
 
-def test_1bit_scale_is_a_running_sum_in_k_order():
-    """The 1-bit scale is fp16(sum_k |w_k| / 128), the sum taken in fp64 in k
-    order. One weight of 1049088 (= 8196 * 128, the tie between the fp16
-    values 8192 and 8200) and 127 of 2^-38 separate the orders: first in k
-    order, the large weight swallows each tiny one, the mean is the tie
-    itself and rounds to even (8192); last, the tiny ones add up to almost
-    2^-31 before meeting it and the mean lands above the tie (8200)."""
-    w = np.full((1, 128), 2.0 ** -38, dtype=np.float32)
-    w[0, 0] = 1049088.0
-    total = 0.0
-    for v in w[0]:                      # Python floats: fp64, one term at a time
-        total += abs(float(v))
-    assert total / 128 == 8196.0
-    _, s16, _ = O.pack_ref(w, 1, 128)
-    assert float(s16[0, 0]) == 8192.0
-    _, s16r, _ = O.pack_ref(np.ascontiguousarray(w[:, ::-1]), 1, 128)
-    assert float(s16r[0, 0]) == 8200.0
-    # on ordinary groups the running sum is the mean
+def test_1bit_scale_is_the_exact_mean_rounded_once():
+    """The 1-bit scale is the fp16 value nearest the exact mean of the
+    group's |w| (ties to even), whatever order the weights come in. Groups
+    whose exact means are derived by hand:
+
+    * one weight of 1049088 (= 8196 * 128; 8196 is the tie between the fp16
+      values 8192 and 8200) and 127 of 2^-38: the mean is 8196 + 127 * 2^-45,
+      above the tie, so 8200 in either order (an fp64 running sum in k order
+      swallows each tiny term and would land on the tie itself, giving 8192);
+    * 1049088 and 127 zeros: exactly the tie, rounds to the even 8192;
+    * 1049087.875 (the fp32 value just below) and 127 zeros: below the tie, 8192;
+    * 1049088 + 2^-1 and 127 zeros: above the tie, 8200;
+    * 128 weights of 2^-20: mean 2^-20, an fp16 subnormal (16 * 2^-24), exact;
+    * 127 zeros and one 2^-17 * 3: mean 3 * 2^-24, the third subnormal;
+    * 127 zeros and one 1.5 * 2^-17: mean 1.5 * 2^-24, a tie between the
+      subnormals 1 and 2 (units of 2^-24), rounds to the even 2;
+    * 128 weights of 65520: mean 65520, the fp16 overflow threshold: refused.
+    """
+    def scale(row):
+        w = np.asarray(row, dtype=np.float32)[None, :]
+        return float(O.pack_ref(w, 1, 128)[1][0, 0])
+
+    tiny = [2.0 ** -38] * 127
+    assert scale([1049088.0] + tiny) == 8200.0
+    assert scale(tiny + [1049088.0]) == 8200.0
+    assert scale(tiny[:60] + [1049088.0] + tiny[60:]) == 8200.0
+    assert scale([1049088.0] + [0.0] * 127) == 8192.0
+    assert np.float32(1049087.875) == 1049087.875
+    assert scale([1049087.875] + [0.0] * 127) == 8192.0
+    assert scale([1049088.5] + [0.0] * 127) == 8200.0
+    assert scale([2.0 ** -20] * 128) == 2.0 ** -20
+    assert scale([0.0] * 127 + [3 * 2.0 ** -17]) == 3 * 2.0 ** -24
+    assert scale([0.0] * 127 + [1.5 * 2.0 ** -17]) == 2 * 2.0 ** -24
+    with pytest.raises(OverflowError):
+        O.pack_ref(np.full((1, 128), 65520.0, dtype=np.float32), 1, 128)
+    assert scale([65504.0] * 128) == 65504.0
+    # on ordinary groups the exact mean and an fp64 sum agree after rounding
     g = np.random.default_rng(13)
     wr = (g.standard_normal((4, 256)) * 0.02).astype(np.float32)
     _, s16g, _ = O.pack_ref(wr, 1, 128)
     for n in range(4):
         for j in range(2):
+            assert s16g[j, n] == np.float16(np.abs(wr[n, 128 * j:128 * (j + 1)].astype(np.float64)).mean())
+
+
+def test_fp16_rn_exact_on_rationals():
+    """The exact-rational fp16 rounding on values derived by hand: the
+    midpoint between 1 and 1 + 2^-10 rounds to 1 (even), a hair above it to
+    1 + 2^-10, 1/3 to the fp16 value 0x3555, and the overflow threshold."""
+    from fractions import Fraction as F
+    assert O.fp16_rn_exact(F(2049, 2048)) == 1.0
+    assert O.fp16_rn_exact(F(2049, 2048) + F(1, 10 ** 30)) == 1.0 + 2.0 ** -10
+    assert O.fp16_rn_exact(F(2051, 2048)) == 1.0 + 2 * 2.0 ** -10     # tie of 1 + u and 1 + 2u: the even one
+    assert int(np.array(O.fp16_rn_exact(F(1, 3))).view(np.uint16)) == 0x3555
+    assert O.fp16_rn_exact(F(65519)) == 65504.0
+    assert np.isinf(O.fp16_rn_exact(F(65520)))
+    assert O.fp16_rn_exact(F(0)) == 0.0
+    assert O.fp16_rn_exact(F(1, 2 ** 25)) == 0.0                        # half the smallest subnormal: even 0
+    assert O.fp16_rn_exact(F(3, 2 ** 26)) == 2.0 ** -24                 # above half
+
+
+def test_dense_ref_hand_worked_2x3():
+    """dense_ref on a case worked by hand: W is rounded to bf16 first (1 + 2^-8
+    is the tie between 1 and 1 + 2^-7 and goes to the even 1; 1 + 2^-8 +
+    2^-10 goes up to 1 + 2^-7; fp32 0.1 = 0x3DCCCCCD rounds up to bf16
+    0x3DCD = 0.10009765625), then X . bf16(W)^T + bias in exact arithmetic."""
+    X = WL.f32_to_bf16_bits(np.array([[1.0, 2.0], [-1.0, 0.5]], dtype=np.float32))
+    W = np.array([[1 + 2.0 ** -8, 3.0], [1 + 2.0 ** -8 + 2.0 ** -10, -2.0], [0.1, 0.0]], dtype=np.float32)
+    bias = WL.f32_to_bf16_bits(np.array([0.5, -1.0, 0.25], dtype=np.float32))
+    expect = np.array([[7.5, -3.9921875, 0.35009765625],
+                       [1.0, -3.0078125, 0.14990234375]])
+    assert np.array_equal(O.dense_ref(X, W, bias), expect)
+    assert np.array_equal(O.dense_ref(X, W), expect - np.array([0.5, -1.0, 0.25])[None, :])
+
+
+def test_dense_ref_equals_python_loop_over_torch_bf16_weights():
+    """dense_ref against a pure-Python triple loop over W cast to bf16 by
+    torch (not by the oracle's own rounding helper), with a bias."""
+    X, W, bias = WL.random_case(21, 5, 7, 128, 4, with_bias=True, w_scale=0.3)
+    Wb = torch.from_numpy(W).to(torch.bfloat16).double().numpy()
+    Xf = WL.bf16_bits_to_f32(X).astype(np.float64)
+    bf = WL.bf16_bits_to_f32(bias).astype(np.float64)
+    ref = O.dense_ref(X, W, bias)
+    for m in range(5):
+        for n in range(7):
             acc = 0.0
-            for v in wr[n, 128 * j:128 * (j + 1)]:
-                acc += abs(float(v))
-            assert s16g[j, n] == np.float16(acc / 128)
+            for k in range(128):
+                acc += float(Xf[m, k]) * float(Wb[n, k])
+            assert abs(ref[m, n] - (acc + float(bf[n]))) <= 1e-12 * (1 + abs(acc))

@@ -87,9 +87,10 @@ def test_multithreaded_pack_matches_single_rows():
     assert whole.scales.shape == (lin.K // 64, 2048)
 
 
-def test_1bit_scale_order_matches_oracle():
-    """A group whose 1-bit scale depends on the order of the sum of |w|
-    (see the oracle pin): the host packer takes it in k order like the oracle."""
+def test_1bit_scale_is_exact_in_any_order():
+    """Groups whose 1-bit scale an fp64 running sum would get wrong (see the
+    oracle pin): the host packer rounds the exact mean like the oracle, so
+    the large weight first or last gives the same 8200."""
     w = np.full((16, 128), 2.0 ** -38, dtype=np.float32)
     w[::2, 0] = 1049088.0                # even rows: the large weight first
     w[1::2, 127] = 1049088.0             # odd rows: the large weight last
@@ -97,7 +98,24 @@ def test_1bit_scale_order_matches_oracle():
     p, s16, _ = O.pack_ref(w, 1, 128)
     assert np.array_equal(pw.scales.view(np.uint16), s16.view(np.uint16))
     assert np.array_equal(pw.packed, p)
-    assert float(pw.scales[0, 0]) == 8192.0 and float(pw.scales[0, 1]) == 8200.0
+    assert np.all(pw.scales.astype(np.float64) == 8200.0)
+
+
+def test_1bit_scale_near_fp16_ties_over_many_binades():
+    """Groups built to sit on or next to an fp16 rounding tie, with the
+    remainder spread over many binades and the weights in random order:
+    host packer and oracle agree bit for bit."""
+    g = np.random.default_rng(77)
+    rows = []
+    for i in range(256):
+        big = np.float32(1049088.0 * 2.0 ** int(g.integers(-30, 3)))   # 128 x an fp16 tie value
+        tail = (2.0 ** g.integers(-149, -20, size=127)).astype(np.float32) * g.choice([0, 1, 1], size=127)
+        sign = np.where(g.integers(0, 2, size=128) == 1, 1.0, -1.0)
+        row = np.concatenate([[big], tail]) * sign
+        if i % 3 == 0:
+            row[0] = np.nextafter(np.float32(row[0]), np.float32(0))       # just below the tie
+        rows.append(g.permutation(row))
+    _same(np.stack(rows).astype(np.float32), 1)
 
 
 @pytest.mark.parametrize("limit", [3e4, 3.3999999521443642e+38], ids=["fp16-range", "fp32-range"])

@@ -3,15 +3,16 @@
 // weights packed (stable-diffusion.rs README, introduction); this makes the
 // packing a device pass for weights that already live in HBM.
 //
-// One thread packs one (row, group): it takes the same fp64 steps in the same
-// order as the host packer (min / max, or max |w|, or a running sum of |w|;
-// one division; one round-to-nearest-even to fp16; rint per code), so scales,
+// One thread packs one (row, group): it takes the same steps in the same
+// order as the host packer (min / max or max |w| in fp64, or the exact sum of
+// |w|; one division; one round-to-nearest-even to fp16; rint per code), so scales,
 // biases and codes match it bit for bit. A group's codes fill whole 32-bit
 // words, so no two threads write the same word. Non-finite weights and
 // fp16 overflow are reported through the device status word.
 
 #include <cuda_fp16.h>
 
+#include "exact_abs_sum.h"
 #include "ptx.cuh"
 #include "qgemm_internal.h"
 
@@ -45,9 +46,9 @@ __global__ void pack_kernel(const float* __restrict__ W, int N, int K, uint32_t*
     if (!finite) ptx::set_status(status, kStatusPackNonfinite);
     double s = 0.0, b = 0.0;
     if constexpr (BITS == 1) {
-      double sum = 0.0;
-      for (int i = 0; i < G; ++i) sum += fabs(static_cast<double>(wg[i]));
-      const uint16_t s16 = f64_to_f16_bits(sum / G);
+      ExactAbsSum sum;  // the exact mean |w|, rounded once (G = 128 = 2^7)
+      for (int i = 0; i < G; ++i) sum.add(wg[i]);
+      const uint16_t s16 = sum.to_f16_rn(7);
       if (!f16_finite(s16)) ptx::set_status(status, kStatusPackOverflow);
       scales[sidx] = s16;
     } else if constexpr (BITS == 2) {

@@ -3,8 +3,9 @@
 //
 // The method stores its weights packed (stable-diffusion.rs README,
 // introduction); this is the offline step that produces those bits.
-// All decisions are taken in fp64 with ties to even, and the fp64 -> fp16
-// rounding is written here from the IEEE 754 binary16 definition.
+// All decisions are taken in fp64 with ties to even (the 1-bit scale from an
+// exact sum), and the fp64 -> fp16 rounding is written here from the IEEE 754
+// binary16 definition.
 
 #include <algorithm>
 #include <cmath>
@@ -12,6 +13,7 @@
 #include <thread>
 #include <vector>
 
+#include "exact_abs_sum.h"
 #include "qgemm.h"
 #include "qgemm_internal.h"
 
@@ -104,10 +106,11 @@ int pack_rows(const PackJob& jb, int r0, int r1) {
       const size_t sidx = static_cast<size_t>(g) * jb.N + n;  // group-major [K/group, N]
       if (bits == 1) {
         // Q1_0_g128: one sign bit per weight (1 = +1, for w >= 0 and -0),
-        // s16 = fp16(mean |w|), the least-squares scale for fixed signs
-        double sum = 0.0;
-        for (int i = 0; i < G; ++i) sum += std::fabs(static_cast<double>(wg[i]));
-        const uint16_t s16 = f64_to_f16_rn(sum / G);
+        // s16 = fp16(mean |w|), the least-squares scale for fixed signs,
+        // rounded once from the exact mean (G = 128 = 2^7)
+        qg::ExactAbsSum sum;
+        for (int i = 0; i < G; ++i) sum.add(wg[i]);
+        const uint16_t s16 = sum.to_f16_rn(7);
         if (!is_f16_finite(s16)) return QGEMM_ERR_UNSUPPORTED;
         jb.scales[sidx] = s16;
         for (int i = 0; i < G; ++i) codes[i] = wg[i] >= 0.f ? 1 : 0;
