@@ -806,22 +806,27 @@ def headline_parity(out, rows: int = 64) -> dict:
 
 
 def cpu_oracle_single_core():
-    """The oracle on one host core for config 0 (tiny) and config 3 at M=1
-    (ternary decode): seconds per GEMM, dequantisation included."""
+    """The oracle on one host core for config 0 (tiny; median of 20 runs) and
+    config 3 at M=1 (ternary decode; median of 3 runs): seconds per GEMM,
+    dequantisation included."""
     from threadpoolctl import threadpool_limits
 
     import oracle as O
     import workloads as WL
     out = {}
     with threadpool_limits(limits=1):
-        for cid, li in ((0, 0), (3, 0)):
+        for cid, li, runs in ((0, 0, 20), (3, 0, 3)):
             lin = WL.workload(cid).linears[li]
             X, W, bias = WL.make_inputs(lin, cid, li)
             p, s, b = O.pack_ref(W, lin.bits, lin.group)
-            t0 = time.perf_counter()
-            O.qgemm_ref(X, p, s, b, lin.bits, lin.group, lin.K, bias)
-            t = time.perf_counter() - t0
-            out[f"{cid}:{lin.name}"] = {"seconds": round(t, 4), "gflops": round(2 * lin.M * lin.N * lin.K / t / 1e9, 3)}
+            ts = []
+            for _ in range(runs):
+                t0 = time.perf_counter()
+                O.qgemm_ref(X, p, s, b, lin.bits, lin.group, lin.K, bias)
+                ts.append(time.perf_counter() - t0)
+            t = statistics.median(ts)
+            out[f"{cid}:{lin.name}"] = {"seconds": round(t, 4), "gflops": round(2 * lin.M * lin.N * lin.K / t / 1e9, 3),
+                                        "runs": runs}
     return out
 
 

@@ -129,7 +129,8 @@ int qgemm_pack_sizes(int32_t N, int32_t K, int32_t bits, int32_t group,
  *   affine:  s = fp16(fl64((max - min) / (2^bits - 1))), b = fp16(min),
  *            q = clamp(rint((w - b) / s), 0, 2^bits - 1), q = 0 where s == 0;
  *   ternary: s = fp16(max |w|), t = clamp(rint(w / s), -1, 1), t = 0 where s == 0;
- *   1-bit:   s = fp16(mean |w|), c = +1 where w >= 0 (and for -0), else -1.
+ *   1-bit:   s = fp16(mean |w|), rounded once from the exact mean of the
+ *            group's magnitudes; c = +1 where w >= 0 (and for -0), else -1.
  * The weights stay packed at rest (stable-diffusion.rs README, introduction).
  * Returns NONFINITE if W holds NaN/Inf, UNSUPPORTED if a scale or bias
  * overflows fp16, plus the errors of qgemm_pack_sizes. biases may be NULL for
@@ -141,7 +142,7 @@ int qgemm_pack(const float* W, int32_t N, int32_t K, int32_t bits, int32_t group
 /*
  * qgemm_pack on the GPU: the same packing of a device fp32 matrix W [N, K]
  * (row-major) into caller-allocated device buffers, bit-identical to
- * qgemm_pack's output (same fp64 steps in the same order). Enqueued on
+ * qgemm_pack's output (the same steps in the same order). Enqueued on
  * `stream`; a non-finite weight or an fp16 overflow is reported later by
  * qgemm_get_device_status as QGEMM_ERR_NONFINITE or QGEMM_ERR_UNSUPPORTED.
  * All pointers 16-byte aligned; biases may be NULL for 1-bit and ternary.
@@ -179,7 +180,10 @@ int qgemm_load(const char* path, void* packed, void* scales, void* biases);
  * qgemm_pack_sizes (larger: UNSUPPORTED) (1-bit weights with K % 256 != 0
  * always take the large-M path). The path (small-M register path or
  * large-M tensor-core path) is chosen per (bits, M, N, K) from a measured
- * table; the environment variable QGEMM_PATH=small|large overrides it.
+ * table; the environment variable QGEMM_PATH=small|large overrides it for
+ * every shape the named path can take (QGEMM_PATH=small leaves M > 16, and
+ * 1-bit weights with K % 256 != 0, to the table). qgemm_select_path reports
+ * the same choice.
  * Returns after enqueueing; a device-side failure (a bounded wait that ran
  * out) is reported later by qgemm_get_device_status.
  */
@@ -234,8 +238,11 @@ int qgemm_dequant_tile(const qgemm_weights* W, int32_t n0, int32_t k0, int32_t r
                        int32_t cols, void* out, void* stream);
 
 /*
- * Synchronises `stream`, then reads and clears the current device's status
- * word (all conditions recorded since the last read). Returns, first match:
+ * Reads and clears the current device's status word (all conditions
+ * recorded since the last read) in one atomic step enqueued on `stream`,
+ * after the work already there, then synchronises `stream`. A condition a
+ * kernel on another stream records meanwhile is never lost: this call or the
+ * next one reports it. Returns, first match:
  *   QGEMM_ERR_CUDA          the stream reports a CUDA error;
  *   QGEMM_ERR_NONFINITE     qgemm_pack_device met a NaN or infinite weight;
  *   QGEMM_ERR_UNSUPPORTED   qgemm_pack_device: a scale or bias overflows fp16;

@@ -218,3 +218,34 @@ def test_binding_device_check_is_host_logic():
     with pytest.raises(ValueError, match="out is on meta"):
         wq._same_device(torch.device("cpu"), W, out=torch.zeros(2, device="meta"))
     wq._same_device(torch.device("cpu"), W, out=cpu, bias=None)   # one device throughout: accepted
+
+
+def test_path_variable_defers_to_the_table_where_its_path_cannot_go():
+    """QGEMM_PATH=small (read once per process) forces the small path only
+    where it can take the shape: qgemm_select_path and the dispatch agree,
+    and a call past the small path's limits is not refused. Without a GPU a
+    call that reaches a kernel launcher fails with QGEMM_ERR_CUDA (no device),
+    which tells it apart from a refusal by the dispatch (UNSUPPORTED)."""
+    import subprocess
+    import sys
+    code = r"""
+import ctypes
+import weight_quantised_gemm_b200 as wq
+W = lambda **kw: wq._Weights(kw.get('N', 256), kw.get('K', 512), kw.get('bits', 4), kw.get('group', 64),
+                             0x1000, 0x2000, kw.get('biases', 0x3000))
+call = lambda d, M: wq._lib.qgemm_ex(0x10000, M, ctypes.byref(d), 0x20000, None, 0, None)
+print(wq.qgemm_select_path(16, 256, 512, 4), wq.qgemm_select_path(17, 256, 512, 4),
+      wq.qgemm_select_path(4, 256, 1152, 1), wq.qgemm_select_path(4, 256, 1024, 1))
+print(call(W(), 17), call(W(bits=1, group=128, K=1152, biases=0), 4))
+"""
+    env = dict(os.environ, QGEMM_PATH="small", CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    sel, disp = r.stdout.strip().splitlines()
+    assert sel.split() == [str(wq.QGEMM_PATH_SMALL_M), str(wq.QGEMM_PATH_LARGE_M), str(wq.QGEMM_PATH_LARGE_M),
+                           str(wq.QGEMM_PATH_SMALL_M)]
+    assert disp.split() == [str(wq.QGEMM_ERR_CUDA)] * 2
+    env["QGEMM_PATH"] = "large"
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.split()[:4] == [str(wq.QGEMM_PATH_LARGE_M)] * 4

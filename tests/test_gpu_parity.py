@@ -406,15 +406,27 @@ def test_pack_device_matches_host_packer(bits):
         W = np.concatenate([WL.make_w(3, 0, 96, K, "ternary", 128), _edge_rows(g, K)])
     else:
         W = np.concatenate([WL.make_w(1, 0, 96, K, "normal"), _edge_rows(g, K)])
+    if bits == 1:
+        # groups at and next to fp16 ties of the exact mean, tails over many binades
+        tie = np.full((4, K), 2.0 ** -38)
+        tie[0, 0] = tie[1, 127] = tie[2, 300] = 1049088.0
+        tie[3, :128] = 0.0
+        tie[3, 5] = 1049088.0
+        W = np.concatenate([W, tie.astype(np.float32)])
     host = wq.qgemm_pack(W, bits)
     dev = wq.qgemm_pack_device(torch.from_numpy(W).cuda(), bits)
     wq.check_device_status()
+    p, s, b = O.pack_ref(W, bits, wq.GROUP_OF_BITS[bits])
+    dev_s = dev.scales.cpu().numpy().view(np.uint16).reshape(host.scales.shape)
+    # the device packer against the oracle directly, and against the host packer
+    assert np.array_equal(dev.packed.cpu().numpy(), p)
+    assert np.array_equal(dev_s, s.view(np.uint16))
     assert np.array_equal(dev.packed.cpu().numpy(), host.packed)
-    assert np.array_equal(dev.scales.cpu().numpy().view(np.uint16).reshape(host.scales.shape),
-                          host.scales.view(np.uint16))
+    assert np.array_equal(dev_s, host.scales.view(np.uint16))
     if bits > 2:
-        assert np.array_equal(dev.biases.cpu().numpy().view(np.uint16).reshape(host.biases.shape),
-                              host.biases.view(np.uint16))
+        dev_b = dev.biases.cpu().numpy().view(np.uint16).reshape(host.biases.shape)
+        assert np.array_equal(dev_b, b.view(np.uint16))
+        assert np.array_equal(dev_b, host.biases.view(np.uint16))
     # and the device-packed weights run the GEMM like the host-packed ones
     X, _, bias = WL.random_case(bits, 5, W.shape[0], K, bits, with_bias=True)
     Xd, bd = to_dev_bf16(X), to_dev_bf16(bias)

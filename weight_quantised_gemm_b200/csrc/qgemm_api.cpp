@@ -81,13 +81,24 @@ uint64_t wait_limit_ns() {
   return v ? v : kDefaultWaitLimitNs;
 }
 
+// Whether the small-M path can take this shape at all: M <= 16, and 1-bit
+// rows streamed in pieces of at least 32 bytes (K % 256 == 0).
+bool small_path_takes(int M, int K, int bits) { return M <= 16 && !(bits == 1 && K % 256); }
+
 int select_path(int M, int N, int K, int bits) {
   (void)N;
-  (void)K;
-  // the small-M path streams 1-bit rows in pieces of at least 32 bytes: K % 256 == 0
-  if (bits == 1 && K % 256) return QGEMM_PATH_LARGE_M;
+  if (!small_path_takes(M, K, bits)) return QGEMM_PATH_LARGE_M;
   const int lim = bits == 1 ? kSmallMaxBinary : bits == 2 ? kSmallMaxTernary : bits == 4 ? kSmallMax4 : kSmallMax8;
   return M <= lim ? QGEMM_PATH_SMALL_M : QGEMM_PATH_LARGE_M;
+}
+
+// The path of a QGEMM_PATH_AUTO call: the QGEMM_PATH variable's choice where
+// that path can take the shape, else the measured table.
+int auto_path(int M, int N, int K, int bits) {
+  std::call_once(g_env_once, read_env);
+  if (g_env_path == QGEMM_PATH_LARGE_M) return QGEMM_PATH_LARGE_M;
+  if (g_env_path == QGEMM_PATH_SMALL_M && small_path_takes(M, K, bits)) return QGEMM_PATH_SMALL_M;
+  return select_path(M, N, K, bits);
 }
 
 }  // namespace qg
@@ -115,9 +126,7 @@ extern "C" int qgemm_fused(const void* X, int32_t M, const qgemm_weights* W, voi
   if (!X || !out) return fail(QGEMM_ERR_INVALID_ARG, "null X or out");
   if (!aligned16(X) || !aligned16(out)) return fail(QGEMM_ERR_ALIGNMENT, "X and out must be 16-byte aligned");
   if (bias && (reinterpret_cast<uintptr_t>(bias) & 1u)) return fail(QGEMM_ERR_ALIGNMENT, "bias must be 2-byte aligned");
-  std::call_once(g_env_once, read_env);
-  if (path == QGEMM_PATH_AUTO) path = g_env_path;
-  if (path == QGEMM_PATH_AUTO) path = select_path(M, W->N, W->K, W->bits);
+  if (path == QGEMM_PATH_AUTO) path = auto_path(M, W->N, W->K, W->bits);
   if (path == QGEMM_PATH_SMALL_M && M > 16)
     return fail(QGEMM_ERR_UNSUPPORTED, "the small-M path takes M <= 16 (M=%d)", M);
   if (path == QGEMM_PATH_SMALL_M && W->bits == 1 && W->K % 256)
@@ -157,9 +166,7 @@ extern "C" int qgemm_select_path(int32_t M, int32_t N, int32_t K, int32_t bits) 
   if (M < 0 || N <= 0 || K <= 0) return -QGEMM_ERR_INVALID_ARG;
   if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return -QGEMM_ERR_UNSUPPORTED;
   if (bits != 1 && bits != 2 && bits != 4 && bits != 8) return -QGEMM_ERR_UNSUPPORTED;
-  std::call_once(g_env_once, read_env);
-  if (g_env_path != QGEMM_PATH_AUTO) return g_env_path == QGEMM_PATH_SMALL_M && M > 16 ? QGEMM_PATH_LARGE_M : g_env_path;
-  return select_path(M, N, K, bits);
+  return auto_path(M, N, K, bits);
 }
 
 extern "C" int qgemm_dequant_tile(const qgemm_weights* W, int32_t n0, int32_t k0, int32_t rows, int32_t cols,

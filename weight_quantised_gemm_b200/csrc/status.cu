@@ -15,12 +15,21 @@ namespace qg {
 // it when a bounded wait gives up; qgemm_get_device_status reads and clears
 // it. A file-scope device variable: nothing is allocated.
 __device__ unsigned int g_status_word;
+// The value the status word held when qgemm_get_device_status last took it.
+__device__ unsigned int g_status_taken;
 
 namespace {
 constexpr int kMaxDevices = 64;
 unsigned int* g_status_ptr[kMaxDevices];
 int g_sm_count[kMaxDevices];
 std::mutex g_mu;
+
+std::mutex g_take_mu;  // one qgemm_get_device_status at a time: they share g_status_taken
+
+// Reads and clears the status word in one atomic step, so that a code a
+// kernel on another stream sets in between is never lost: it is either
+// taken now or left for the next read.
+__global__ void take_status_kernel(unsigned int* word, unsigned int* taken) { *taken = atomicExch(word, 0u); }
 
 int current_device(int* dev) {
   int st = cuda_check(cudaGetDevice(dev), "cudaGetDevice");
@@ -104,15 +113,20 @@ extern "C" int qgemm_get_device_status(void* stream) {
   unsigned int* status;
   int st = status_word(&status);
   if (st != QGEMM_OK) return st;
-  st = cuda_check(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)), "cudaStreamSynchronize");
+  std::lock_guard<std::mutex> lk(g_take_mu);
+  void* taken = nullptr;
+  st = cuda_check(cudaGetSymbolAddress(&taken, g_status_taken), "cudaGetSymbolAddress(status copy)");
+  if (st != QGEMM_OK) return st;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  take_status_kernel<<<1, 1, 0, s>>>(status, static_cast<unsigned int*>(taken));
+  st = cuda_check(cudaGetLastError(), "take_status_kernel launch");
   if (st != QGEMM_OK) return st;
   unsigned int v = 0;
-  st = cuda_check(cudaMemcpyFromSymbol(&v, g_status_word, sizeof v), "read status word");
+  st = cuda_check(cudaMemcpyAsync(&v, taken, sizeof v, cudaMemcpyDeviceToHost, s), "read status word");
+  if (st != QGEMM_OK) return st;
+  st = cuda_check(cudaStreamSynchronize(s), "cudaStreamSynchronize");
   if (st != QGEMM_OK) return st;
   if (v) {
-    const unsigned int zero = 0;
-    st = cuda_check(cudaMemcpyToSymbol(g_status_word, &zero, sizeof zero), "clear status word");
-    if (st != QGEMM_OK) return st;
     if (v & kStatusPackNonfinite)
       return fail(QGEMM_ERR_NONFINITE, "qgemm_pack_device met a non-finite weight (status word 0x%x)", v);
     if (v & kStatusPackOverflow)
