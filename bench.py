@@ -305,8 +305,9 @@ def time_graph(fn_list, reps: int = 5):
 
 
 def sweep(peaks):
-    """Every workload linear: time, TFLOP/s, GB/s and roofline fraction, plus
-    the small-M sweep on both paths and config 4's cosine against dense bf16."""
+    """Every workload linear: time, TFLOP/s, GB/s and roofline fraction (small-M
+    rows also with launch overlap and beside the streaming floor of the same
+    launch), and config 4's cosine against dense bf16."""
     import torch
 
     import weight_quantised_gemm_b200 as wq
@@ -333,14 +334,25 @@ def sweep(peaks):
                  "roofline_us": round(t_roof * 1e6, 2), "frac_of_roofline": round(t_roof / t, 3),
                  "copies": ncopy}
         if entry["path"] == "small":
+            def rep(fl):
+                return (fl * (-(-launches // len(fl))))[:max(launches, len(fl))]
             # the same launches with QGEMM_FLAG_OVERLAP_PREVIOUS: each GEMV's weight
             # stream may start while the previous one in the stream finishes
             fo = [(lambda s=s: wq.qgemm(s[0], s[1], bias=s[2], out=s[3], path=path, overlap_previous=True))
                   for s in sets]
-            to = time_graph((fo * (-(-launches // len(fo))))[:max(launches, len(fo))])
+            to = time_graph(rep(fo))
+            # the streaming floor: the same kernel, grid, clusters and ring moving
+            # the same weight bytes with no arithmetic (qgemm_debug_stream)
+            tf = time_graph(rep([(lambda s=s: wq.qgemm_debug_stream(s[0], s[1])) for s in sets]))
+            tfo = time_graph(rep([(lambda s=s: wq.qgemm_debug_stream(s[0], s[1], overlap_previous=True))
+                                  for s in sets]))
             wq.check_device_status()
             entry["us_overlap_previous"] = round(to * 1e6, 2)
             entry["frac_of_roofline_overlap_previous"] = round(t_roof / to, 3)
+            entry["us_stream_floor"] = round(tf * 1e6, 2)
+            entry["us_stream_floor_overlap_previous"] = round(tfo * 1e6, 2)
+            entry["kernel_over_floor"] = round(t / tf, 3)
+            entry["kernel_over_floor_overlap_previous"] = round(to / tfo, 3)
         return entry, sets, host
 
     for cid in range(len(WL.WORKLOADS)):
@@ -385,23 +397,100 @@ def sweep(peaks):
     block["packed_over_dense_bf16"] = round(packed / (2 * dense), 4)
     block["packed_over_dense_fp32"] = round(packed / (4 * dense), 4)
     block["tflops"] = round(sum(2 * l.M * l.N * l.K for l in wl4.linears) / (block["us_total"] * 1e-6) / 1e12, 1)
-    # small-M crossover sweep: both paths on the ternary and 4-bit decode shapes
-    cross = []
-    lin3 = WL.workload(3).linears[0]
-    import dataclasses
-    for bits in (1, 2, 4, 8):
-        lin = dataclasses.replace(lin3, bits=bits, group=wq.GROUP_OF_BITS[bits],
-                                  w_dist={1: "binary", 2: "ternary"}.get(bits, "normal"))
-        for M in (1, 4, 8, 16, 32, 64):
-            for path in (wq.QGEMM_PATH_SMALL_M, wq.QGEMM_PATH_LARGE_M):
-                if path == wq.QGEMM_PATH_SMALL_M and M > 16:
-                    continue
-                e, sets, _ = one(3, 0, lin, M, path, 100)
-                cross.append({k: e[k] for k in ("bits", "M", "path", "us", "gbs", "frac_of_roofline",
-                                                "us_overlap_previous") if k in e})
-                del sets
     torch.cuda.empty_cache()
-    return res, block, cross
+    return res, block
+
+
+def grouped_sweep(peaks):
+    """The mixed FLUX block's five linears at decode M: one grouped launch per
+    format (4-bit QKV and MLP up; 8-bit modulation, out projection and MLP
+    down) against one launch per linear, CUDA-graph timing over rotating
+    weight copies, GB/s against the summed algorithmic bytes."""
+    import numpy as np
+    import torch
+
+    import weight_quantised_gemm_b200 as wq
+    import workloads as WL
+    BW = peaks["hbm_gbs"] * 1e9
+    wl = WL.workload(4)
+    rows = []
+    for M in (1, 16):
+        for bits in (4, 8):
+            lins = [(li, l) for li, l in enumerate(wl.linears) if l.bits == bits]
+            ab = sum(alg_bytes(l, M) for _, l in lins)
+            ncopy = max(4, -(-3 * L2_BYTES // ab))
+            host = []
+            for li, l in lins:
+                X, W, _ = WL.make_inputs(l, 4, li, M=M)
+                host.append((l, X, wq.qgemm_pack(W, bits)))
+            sets = [[(torch.from_numpy(X.view(np.int16)).cuda().view(torch.bfloat16), pw.to_device("cuda"), None,
+                      torch.empty((M, l.N), dtype=torch.bfloat16, device="cuda")) for l, X, pw in host]
+                    for _ in range(ncopy)]
+
+            def grouped(probs, ov):
+                return lambda: wq.qgemm_grouped([(x, d, b) for x, d, b, _ in probs], outs=[o for *_, o in probs],
+                                                overlap_previous=ov)
+
+            def separate(probs, ov):
+                return lambda: [wq.qgemm(x, d, bias=b, out=o, overlap_previous=ov) for x, d, b, o in probs]
+            n = max(ncopy, 24)
+            res = {"M": M, "bits": bits, "linears": [l.name for _, l in lins], "alg_bytes": ab, "copies": ncopy}
+            for name, mk in (("grouped", grouped), ("separate", separate)):
+                for ov in (False, True):
+                    t = time_graph([mk(sets[i % ncopy], ov) for i in range(n)])
+                    key = name + ("_overlap_previous" if ov else "")
+                    res[f"us_{key}"] = round(t * 1e6, 2)
+                    res[f"gbs_{key}"] = round(ab / t / 1e9, 1)
+                    res[f"frac_of_hbm_roofline_{key}"] = round(ab / BW / t, 3)
+            wq.check_device_status()
+            rows.append(res)
+            del sets
+            torch.cuda.empty_cache()
+    return rows
+
+
+CROSSOVER_SHAPES = ((12288, 3072), (9216, 3072), (18432, 3072), (3072, 3072), (3072, 12288))
+CROSSOVER_M = (1, 2, 4, 8, 12, 16, 24, 32, 48, 64)
+
+
+def crossover_sweep():
+    """Both kernel paths at M = 1..64 on every (N, K) of the FLUX workloads in
+    every format (CUDA-graph timing over rotating weight copies): the
+    measurements the path table is read from."""
+    import numpy as np
+    import torch
+
+    import weight_quantised_gemm_b200 as wq
+    import workloads as WL
+    rows = []
+    for N, K in CROSSOVER_SHAPES:
+        for bits in (1, 2, 4, 8):
+            dist = {1: "binary", 2: "ternary"}.get(bits, "normal")
+            W = WL.make_w(9, bits, N, K, dist, wq.GROUP_OF_BITS[bits])
+            pw = wq.qgemm_pack(W, bits)
+            wbytes = pw.nbytes
+            ncopy = max(8, -(-3 * L2_BYTES // wbytes))
+            dws = [pw.to_device("cuda") for _ in range(ncopy)]
+            for M in CROSSOVER_M:
+                X = WL.make_x(9, bits, M, K, "normal")
+                Xd = torch.from_numpy(X.view(np.int16)).cuda().view(torch.bfloat16)
+                out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+                entry = {"N": N, "K": K, "bits": bits, "M": M}
+                for name, path in (("small", wq.QGEMM_PATH_SMALL_M), ("large", wq.QGEMM_PATH_LARGE_M)):
+                    if name == "small" and M > 16:
+                        continue
+                    fns = [(lambda d=d: wq.qgemm(Xd, d, out=out, path=path)) for d in dws]
+                    launches = max(len(fns), 64 if M <= 16 else 16)
+                    t = time_graph((fns * (-(-launches // len(fns))))[:launches])
+                    entry[f"us_{name}"] = round(t * 1e6, 2)
+                wq.check_device_status()
+                entry["faster"] = "small" if entry.get("us_small", float("inf")) < entry["us_large"] else "large"
+                entry["table"] = "small" if wq.qgemm_select_path(M, N, K, bits) == 1 else "large"
+                rows.append(entry)
+                del Xd, out
+            del dws
+            torch.cuda.empty_cache()
+    return rows
 
 
 def run_ours(args, rank, world, local_rank):
@@ -928,7 +1017,7 @@ HEADLINE_KEYS = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per
 HEADLINE_MAX_BYTES = 6000
 
 
-def sweep_summary(sweep_rows, block, cross) -> dict:
+def sweep_summary(sweep_rows, block) -> dict:
     """A few numbers per workload linear for the headline line: microseconds
     per launch (CUDA graph) and the fraction of the shape's roofline; the
     full rows go to the report sections."""
@@ -963,6 +1052,8 @@ def main(argv=None):
     ap.add_argument("--no-sweep", action="store_true", help="skip the per-workload sweep")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--crossover", action="store_true",
+                    help="also time both kernel paths at M = 1..64 on every workload shape and format")
     ap.add_argument("--report", default=None,
                     help="also write the detailed report sections (JSON lines) to this file")
     ap.add_argument("--case", default=None,
@@ -998,11 +1089,20 @@ def main(argv=None):
             if not args.no_sweep and world == 1:
                 out = report_section(res, "sweep", lambda: sweep(peaks))
                 if out is not None:
-                    rows, block, cross = out
+                    rows, block = out
                     report("sweep", rows)
                     report("workload4_block", block)
-                    report("path_crossover", cross)
-                    res["sweep_summary"] = sweep_summary(rows, block, cross)
+                    res["sweep_summary"] = sweep_summary(rows, block)
+                if args.crossover:
+                    cross = report_section(res, "path_crossover", crossover_sweep)
+                    if cross is not None:
+                        report("path_crossover", cross)
+                grp = report_section(res, "grouped", lambda: grouped_sweep(peaks))
+                if grp is not None:
+                    report("grouped", grp)
+                    res.setdefault("sweep_summary", {}).update(
+                        {f"grouped:{r['bits']}bit:M{r['M']}": [r["us_grouped"], r["frac_of_hbm_roofline_grouped"]]
+                         for r in grp})
                 fused = report_section(res, "fused_epilogues", fused_sweep)
                 if fused is not None:
                     report("fused_epilogues", fused)

@@ -222,6 +222,32 @@ typedef struct qgemm_epilogue {
 int qgemm_fused(const void* X, int32_t M, const qgemm_weights* W, void* out,
                 const void* bias, const qgemm_epilogue* epi, int32_t path, void* stream);
 
+/* One GEMV of a grouped call: out = X . dequant(W)^T (+ bias), as qgemm. */
+typedef struct qgemm_problem {
+  const void* X;         /* device bf16 [M, K], 16-byte aligned */
+  int32_t M;             /* tokens, 0 to 16 (0: the problem is skipped) */
+  qgemm_weights W;       /* device-resident packed weights */
+  void* out;             /* device bf16 [M, N], 16-byte aligned */
+  const void* bias;      /* device bf16 [N] or NULL */
+} qgemm_problem;
+
+/*
+ * Several independent small-M GEMVs (M <= 16 each) in one launch, each
+ * computing what qgemm computes for it, on `stream`. At decode-sized M a GEMV
+ * is a read of its packed weights, and a single read of 10-40 MB is bound by
+ * the launch and first-byte latency rather than by bandwidth (pictor README,
+ * "Extreme quantization is first-class": GEMV paths built for sub-byte
+ * weights); one persistent launch streams all the problems' weights back to
+ * back and pays that cost once. Requires 1 to 16 problems whose weights share
+ * one format (bits), each a shape the small-M path takes (1-bit: K % 256 ==
+ * 0), at most 4096 x 32 rows per problem and 4096 blocks of 32 rows in all
+ * (else UNSUPPORTED). No output may overlap another problem's X, out or bias.
+ * flags: 0 or QGEMM_FLAG_OVERLAP_PREVIOUS (as for qgemm_ex). Argument errors
+ * are those of qgemm_ex, checked for every problem before anything is
+ * enqueued. No counterpart as an interface in the pages.
+ */
+int qgemm_grouped(const qgemm_problem* problems, int32_t count, int32_t flags, void* stream);
+
 /* The path qgemm would take for this shape: QGEMM_PATH_SMALL_M or
  * QGEMM_PATH_LARGE_M, or a negative qgemm_status for an invalid shape. */
 int qgemm_select_path(int32_t M, int32_t N, int32_t K, int32_t bits);
@@ -236,6 +262,20 @@ int qgemm_select_path(int32_t M, int32_t N, int32_t K, int32_t bits);
  */
 int qgemm_dequant_tile(const qgemm_weights* W, int32_t n0, int32_t k0, int32_t rows,
                        int32_t cols, void* out, void* stream);
+
+/*
+ * Debug entry point for measurement: the small-M kernel exactly as qgemm would
+ * launch it for (M, W) (same grid, same thread-block clusters, same stage ring
+ * and TMA boxes, QGEMM_FLAG_OVERLAP_PREVIOUS honoured), streaming the packed
+ * weights, scales and biases (and, where the kernel stages them, the
+ * activation rows of X) through its ring while computing and writing nothing.
+ * Its time is the floor of the weight stream itself for this shape: launch,
+ * first-byte latency and bandwidth, without the arithmetic. X: device bf16
+ * [M, K], 16-byte aligned. Requires a shape the small-M path takes (M <= 16;
+ * 1-bit weights with K % 256 == 0), else UNSUPPORTED. No counterpart in the
+ * pages: an instrument of this implementation.
+ */
+int qgemm_debug_stream(const void* X, int32_t M, const qgemm_weights* W, int32_t flags, void* stream);
 
 /*
  * Reads and clears the current device's status word (all conditions

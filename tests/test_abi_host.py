@@ -249,3 +249,52 @@ print(call(W(), 17), call(W(bits=1, group=128, K=1152, biases=0), 4))
     r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr
     assert r.stdout.split()[:4] == [str(wq.QGEMM_PATH_LARGE_M)] * 4
+
+
+def _grouped(problems, flags=0):
+    arr = (wq._Problem * len(problems))(*problems)
+    return wq._lib.qgemm_grouped(arr, len(problems), flags, None)
+
+
+def _problem(M=4, X=0x10000, out=0x20000, bias=None, **kw):
+    return wq._Problem(X, M, _desc(**kw), out, bias)
+
+
+def test_grouped_rejects_bad_lists_without_device():
+    ok = _problem()
+    assert wq._lib.qgemm_grouped(None, 1, 0, None) == wq.QGEMM_ERR_INVALID_ARG
+    assert _grouped([ok], flags=0x200) == wq.QGEMM_ERR_INVALID_ARG
+    arr = (wq._Problem * 17)(*([ok] * 17))
+    assert wq._lib.qgemm_grouped(arr, 17, 0, None) == wq.QGEMM_ERR_INVALID_ARG
+    assert wq._lib.qgemm_grouped(arr, 0, 0, None) == wq.QGEMM_ERR_INVALID_ARG
+    assert _grouped([ok, _problem(bits=8)]) == wq.QGEMM_ERR_UNSUPPORTED            # one format per call
+    assert _grouped([ok, _problem(M=17)]) == wq.QGEMM_ERR_UNSUPPORTED             # small-M only
+    assert _grouped([ok, _problem(M=-1)]) == wq.QGEMM_ERR_UNSUPPORTED
+    assert _grouped([_problem(bits=1, group=128, K=1152, biases=0)]) == wq.QGEMM_ERR_UNSUPPORTED
+    assert _grouped([ok, _problem(X=0)]) == wq.QGEMM_ERR_INVALID_ARG
+    assert _grouped([ok, _problem(out=0x20008)]) == wq.QGEMM_ERR_ALIGNMENT
+    assert _grouped([ok, _problem(bias=0x30001)]) == wq.QGEMM_ERR_ALIGNMENT
+    assert _grouped([ok, _problem(N=264)]) == wq.QGEMM_ERR_UNSUPPORTED           # the weights are checked too
+    # every problem empty: a no-op that never touches the device
+    assert _grouped([_problem(M=0, X=0, out=0), _problem(M=0)]) == wq.QGEMM_OK
+
+
+def test_problem_struct_layout_matches_the_header(tmp_path):
+    """The binding's ctypes mirror of qgemm_problem has the C layout."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc is not installed")
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "qgemm.h"\n'
+                   'int main(void) { printf("%zu %zu %zu %zu %zu\\n", sizeof(qgemm_problem), '
+                   'offsetof(qgemm_problem, M), offsetof(qgemm_problem, W), offsetof(qgemm_problem, out), '
+                   'offsetof(qgemm_problem, bias)); return 0; }\n')
+    exe = tmp_path / "layout"
+    r = subprocess.run([gcc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()]
+    P = wq._Problem
+    assert got == [ctypes.sizeof(P), P.M.offset, P.W.offset, P.out.offset, P.bias.offset]

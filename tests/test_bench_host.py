@@ -167,7 +167,7 @@ def test_main_arm_prints_one_compact_headline_line(monkeypatch, capsys):
     block = {"us_total": 1184.0, "cosine_vs_dense_bf16_all_five": 0.998}
     monkeypatch.setattr(torch.cuda, "set_device", lambda *_: None)
     monkeypatch.setattr(bench, "run_ours", fake_run_ours)
-    monkeypatch.setattr(bench, "sweep", lambda peaks: (big_rows, block, [{"pad": "y" * 300}] * 50))
+    monkeypatch.setattr(bench, "sweep", lambda peaks: (big_rows, block))
     monkeypatch.setattr(bench, "fused_sweep", lambda: [{"pad": "z" * 500}] * 10)
     monkeypatch.setattr(bench, "policy_sweep", lambda: {"assignments": [{"pad": "w" * 200}] * 32})
     monkeypatch.setattr(bench, "cpu_baseline", lambda s: {"value": 0.4, "unit": "TFLOP/s", "cores": 16,
@@ -190,7 +190,7 @@ def test_main_arm_prints_one_compact_headline_line(monkeypatch, capsys):
     assert r["sweep_summary"]["4:lin0"] == [100.0, 0.8]
     assert "sweep" not in r and "policy_sweep" not in r and "clocks_detail" not in r
     sections = [json.loads(x)["report"] for x in cap.err.splitlines() if x.startswith('{"report"')]
-    assert {"sweep", "path_crossover", "fused_epilogues", "policy_sweep", "workload4_block"} <= set(sections)
+    assert {"sweep", "fused_epilogues", "policy_sweep", "workload4_block", "clocks_detail"} <= set(sections)
 
 
 def test_headline_line_drops_summaries_before_exceeding_its_size():

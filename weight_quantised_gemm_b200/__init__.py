@@ -58,6 +58,11 @@ class _Weights(ctypes.Structure):
                 ("biases", ctypes.c_void_p)]
 
 
+class _Problem(ctypes.Structure):
+    _fields_ = [("X", ctypes.c_void_p), ("M", ctypes.c_int32), ("W", _Weights), ("out", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p)]
+
+
 def _load():
     if not os.path.exists(_LIB_PATH):
         raise ImportError(f"{_LIB_PATH} is not built; run `python -m weight_quantised_gemm_b200.build`")
@@ -78,6 +83,8 @@ def _load():
         "qgemm_fused": (ctypes.c_int, [vp, i32, W, vp, vp, ctypes.POINTER(_Epilogue), i32, vp]),
         "qgemm_select_path": (ctypes.c_int, [i32, i32, i32, i32]),
         "qgemm_dequant_tile": (ctypes.c_int, [W, i32, i32, i32, i32, vp, vp]),
+        "qgemm_debug_stream": (ctypes.c_int, [vp, i32, W, i32, vp]),
+        "qgemm_grouped": (ctypes.c_int, [ctypes.POINTER(_Problem), i32, i32, vp]),
         "qgemm_get_device_status": (ctypes.c_int, [vp]),
         "qgemm_set_wait_limit_ns": (ctypes.c_int, [u64]),
         "qgemm_debug_wait_timeout": (ctypes.c_int, [u64, vp]),
@@ -106,7 +113,7 @@ _lib = _LazyLib()
 EXPORTED = ("qgemm_pack_sizes", "qgemm_pack", "qgemm_pack_device", "qgemm_save", "qgemm_load_header",
             "qgemm_load", "qgemm", "qgemm_ex", "qgemm_fused",
             "qgemm_select_path",
-            "qgemm_dequant_tile",
+            "qgemm_dequant_tile", "qgemm_debug_stream", "qgemm_grouped",
             "qgemm_get_device_status", "qgemm_set_wait_limit_ns", "qgemm_debug_wait_timeout",
             "qgemm_status_str", "qgemm_last_error", "qgemm_version")
 
@@ -326,6 +333,40 @@ def qgemm_fused(X, W: DeviceWeights, op: int, bias=None, residual=None, gate=Non
     return out
 
 
+def qgemm_grouped(problems, outs=None, stream=None, overlap_previous: bool = False):
+    """Several independent small-M GEMVs in one launch (C ABI qgemm_grouped):
+    `problems` is a list of (X, W, bias) with X a bf16 [M, K] CUDA tensor
+    (M <= 16), W DeviceWeights (one format for all) and bias a bf16 [N]
+    tensor or None. Returns the outputs (bf16 [M, N] each), written into
+    `outs` when given."""
+    import torch
+    if not problems:
+        raise ValueError("no problems")
+    dev = problems[0][0].device
+    arr = (_Problem * len(problems))()
+    result = []
+    for i, (X, W, bias) in enumerate(problems):
+        if X.dtype != torch.bfloat16 or not X.is_cuda or X.dim() != 2 or not X.is_contiguous():
+            raise ValueError(f"problem {i}: X must be a contiguous 2-D bf16 CUDA tensor")
+        M, K = X.shape
+        if K != W.K:
+            raise ValueError(f"problem {i}: X has K={K}, weights have K={W.K}")
+        out = None if outs is None else outs[i]
+        if out is None:
+            out = torch.empty((M, W.N), dtype=torch.bfloat16, device=dev)
+        elif out.dtype != torch.bfloat16 or tuple(out.shape) != (M, W.N) or not out.is_contiguous():
+            raise ValueError(f"problem {i}: out must be a contiguous bf16 [M, N] tensor")
+        if bias is not None and (bias.dtype != torch.bfloat16 or bias.numel() != W.N or not bias.is_cuda):
+            raise ValueError(f"problem {i}: bias must be a bf16 CUDA tensor of N elements")
+        _same_device(dev, W, X=X, out=out, bias=bias)
+        arr[i] = _Problem(X.data_ptr(), M, W.descriptor(), out.data_ptr(), None if bias is None else bias.data_ptr())
+        result.append(out)
+    flags = QGEMM_FLAG_OVERLAP_PREVIOUS if overlap_previous else 0
+    with torch.cuda.device(dev):
+        _check(_lib.qgemm_grouped(arr, len(problems), flags, _stream_handle(stream, dev)), "qgemm_grouped")
+    return result
+
+
 def qgemm_select_path(M: int, N: int, K: int, bits: int) -> int:
     r = _lib.qgemm_select_path(M, N, K, bits)
     if r < 0:
@@ -350,6 +391,23 @@ def qgemm_dequant_tile(W: DeviceWeights, n0: int = 0, k0: int = 0, rows: Optiona
         _check(_lib.qgemm_dequant_tile(ctypes.byref(desc), n0, k0, rows, cols, out.data_ptr(),
                                        _stream_handle(stream, dev)), "qgemm_dequant_tile")
     return out
+
+
+def qgemm_debug_stream(X, W: DeviceWeights, stream=None, overlap_previous: bool = False) -> None:
+    """The small-M kernel as qgemm would launch it for (X, W), streaming the
+    packed weights through its ring and computing nothing (C ABI
+    qgemm_debug_stream): the streaming floor of the shape."""
+    import torch
+    if X.dtype != torch.bfloat16 or not X.is_cuda or X.dim() != 2 or not X.is_contiguous():
+        raise ValueError("X must be a contiguous 2-D bf16 CUDA tensor")
+    if X.shape[1] != W.K:
+        raise ValueError(f"X has K={X.shape[1]}, weights have K={W.K}")
+    _same_device(X.device, W)
+    desc = W.descriptor()
+    with torch.cuda.device(X.device):
+        _check(_lib.qgemm_debug_stream(X.data_ptr(), X.shape[0], ctypes.byref(desc),
+                                       QGEMM_FLAG_OVERLAP_PREVIOUS if overlap_previous else 0,
+                                       _stream_handle(stream, X.device)), "qgemm_debug_stream")
 
 
 def qgemm_get_device_status(stream=None) -> int:

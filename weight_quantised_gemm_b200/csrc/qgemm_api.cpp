@@ -186,6 +186,58 @@ extern "C" int qgemm_dequant_tile(const qgemm_weights* W, int32_t n0, int32_t k0
   return launch_dequant_tile(p, n0, k0, rows, cols);
 }
 
+extern "C" int qgemm_grouped(const qgemm_problem* problems, int32_t count, int32_t flags, void* stream) {
+  if (!problems) return fail(QGEMM_ERR_INVALID_ARG, "null problem list");
+  if (count < 1 || count > kGroupedMaxProblems)
+    return fail(QGEMM_ERR_INVALID_ARG, "count=%d: 1 to %d problems per grouped call", count, kGroupedMaxProblems);
+  if (flags & ~QGEMM_FLAG_OVERLAP_PREVIOUS) return fail(QGEMM_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  Problem probs[kGroupedMaxProblems];
+  bool any = false;
+  for (int i = 0; i < count; ++i) {
+    const qgemm_problem& q = problems[i];
+    int st = validate_weights(&q.W);
+    if (st != QGEMM_OK) return st;
+    if (q.W.bits != problems[0].W.bits)
+      return fail(QGEMM_ERR_UNSUPPORTED, "grouped: problem %d has %d-bit weights, problem 0 %d-bit", i, q.W.bits,
+                  problems[0].W.bits);
+    if (q.M < 0 || q.M > 16) return fail(QGEMM_ERR_UNSUPPORTED, "grouped: problem %d has M=%d (0 to 16)", i, q.M);
+    if (!small_path_takes(q.M, q.W.K, q.W.bits))
+      return fail(QGEMM_ERR_UNSUPPORTED, "grouped: problem %d (1-bit weights need K %% 256 == 0)", i);
+    if (q.M > 0) {
+      if (!q.X || !q.out) return fail(QGEMM_ERR_INVALID_ARG, "grouped: problem %d has a null X or out", i);
+      if (!aligned16(q.X) || !aligned16(q.out))
+        return fail(QGEMM_ERR_ALIGNMENT, "grouped: problem %d: X and out must be 16-byte aligned", i);
+      if (q.bias && (reinterpret_cast<uintptr_t>(q.bias) & 1u))
+        return fail(QGEMM_ERR_ALIGNMENT, "grouped: problem %d: bias must be 2-byte aligned", i);
+      any = true;
+    }
+    probs[i] = Problem{q.X, q.M, q.W.N, q.W.K, q.W.bits, q.W.group, static_cast<const uint8_t*>(q.W.packed),
+                       static_cast<const uint16_t*>(q.W.scales), static_cast<const uint16_t*>(q.W.biases), q.out,
+                       static_cast<const uint16_t*>(q.bias), static_cast<cudaStream_t>(stream),
+                       (flags & QGEMM_FLAG_OVERLAP_PREVIOUS) != 0, QGEMM_EPI_NONE, nullptr, nullptr};
+  }
+  if (!any) return QGEMM_OK;
+  return launch_small_m_grouped(probs, count, (flags & QGEMM_FLAG_OVERLAP_PREVIOUS) != 0,
+                                static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int qgemm_debug_stream(const void* X, int32_t M, const qgemm_weights* W, int32_t flags, void* stream) {
+  int st = validate_weights(W);
+  if (st != QGEMM_OK) return st;
+  if (M < 0) return fail(QGEMM_ERR_INVALID_ARG, "M=%d is negative", M);
+  if (flags & ~QGEMM_FLAG_OVERLAP_PREVIOUS) return fail(QGEMM_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  if (!small_path_takes(M, W->K, W->bits))
+    return fail(QGEMM_ERR_UNSUPPORTED, "the small-M path does not take M=%d, K=%d, bits=%d", M, W->K, W->bits);
+  if (M == 0) return QGEMM_OK;
+  if (!X) return fail(QGEMM_ERR_INVALID_ARG, "null X");
+  if (!aligned16(X)) return fail(QGEMM_ERR_ALIGNMENT, "X must be 16-byte aligned");
+  Problem p{X, M, W->N, W->K, W->bits, W->group, static_cast<const uint8_t*>(W->packed),
+            static_cast<const uint16_t*>(W->scales), static_cast<const uint16_t*>(W->biases), nullptr, nullptr,
+            static_cast<cudaStream_t>(stream), (flags & QGEMM_FLAG_OVERLAP_PREVIOUS) != 0, QGEMM_EPI_NONE,
+            nullptr, nullptr, true};
+  return launch_small_m(p);
+}
+
 extern "C" int qgemm_set_wait_limit_ns(uint64_t limit_ns) {
   std::call_once(g_env_once, read_env);
   g_wait_limit_ns.store(limit_ns ? limit_ns : kDefaultWaitLimitNs);

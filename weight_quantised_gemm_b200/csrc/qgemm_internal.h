@@ -26,6 +26,7 @@ struct Problem {
   int epi;               // QGEMM_EPI_*
   const uint16_t* residual;  // bf16 bits [M, N] (QGEMM_EPI_RESIDUAL_GATE), may equal out
   const uint16_t* gate;      // bf16 bits [N] (QGEMM_EPI_RESIDUAL_GATE)
+  bool floor_only = false;   // small-M: stream the weights through the ring, compute and write nothing
 };
 
 // Records a detail message for qgemm_last_error and returns `code`.
@@ -57,6 +58,8 @@ int make_tensor_map_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* bas
 
 // Kernel launchers (one per kernel family). Each enqueues on p.stream.
 int launch_small_m(const Problem& p);
+// Several small-M problems of one format in one launch (qgemm_grouped).
+int launch_small_m_grouped(const Problem* probs, int count, bool overlap, cudaStream_t stream);
 int launch_large_m(const Problem& p);
 int launch_dequant_tile(const Problem& p, int n0, int k0, int rows, int cols);
 int launch_debug_wait(uint64_t limit_ns, cudaStream_t stream);
@@ -67,6 +70,11 @@ int launch_pack_device(const float* W, int N, int K, int bits, void* packed, uin
 // Largest M, N or K the library accepts (2^30): keeps every launcher's int
 // arithmetic (rounded-up tile and stage counts) inside int32.
 constexpr int32_t kMaxDim = 1 << 30;
+
+// Grouped small-M launches: problems per launch, CTAs, and 32-row work items.
+constexpr int kGroupedMaxProblems = 16;
+constexpr int kGroupedMaxCtas = 256;
+constexpr int kGroupedMaxItems = 4096;
 
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusLayout = 2u;  // dynamic shared memory not aligned as the kernel requires

@@ -60,11 +60,14 @@
 
 #include <cuda.h>
 
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "dequant.cuh"
 #include "epilogue.cuh"
 #include "qgemm_internal.h"
+#include "small_m_common.cuh"
 #include "small_m_layout.cuh"
 
 namespace qg {
@@ -87,11 +90,6 @@ __host__ __device__ constexpr int split_rows(int MT, int NP) { return MT > 8 && 
 // straight from global memory.
 __host__ __device__ constexpr bool x_in_ring(int MT, int NP) { return split_rows(MT, NP) == 2; }
 
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
 struct Params {
   const uint16_t* X;     // bf16 [M, K]
   const uint16_t* bias;  // bf16 [N] or null
@@ -108,60 +106,32 @@ struct Params {
   int off_s, off_b;      // offsets of the scales and biases inside a stage
   int off_x, x_stride;   // activations in the ring (split-row CTAs): offset, token row stride in bytes
   int overlap;           // launched with programmatic dependent launch
+  int ksplit;            // K slices per row block: the CTAs of one thread-block cluster (1 = no cluster)
+  int floor_only;        // stream the weights through the ring and compute nothing (the streaming floor)
   uint64_t wait_limit_ns;
   unsigned int* status;
 };
 
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+// Thread-block cluster helpers (K-split launches).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-
-__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-               : "memory");
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
 }
-
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_t lim, const volatile int* abort) {
-  const bool ok = ptx::mbar_wait(bar, parity, lim, abort);
-  return __all_sync(0xffffffffu, ok);
+// The shared-memory address `addr` of this CTA, as the same offset in CTA
+// `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
 }
-
-
-// B operand of one step for quad thread c from its word: codes 4c .. 4c+3 as
-// two bf16x2 registers (k pairs (4c, 4c+1) and (4c+2, 4c+3)).
-template <int BITS>
-__device__ __forceinline__ void decode_word(uint32_t x, int c, int k, uint32_t& b0, uint32_t& b1) {
-  if constexpr (BITS == 1) {
-    // pairs 8(k%2) + 2c and +1 of the 32-code word: bf16 {-1, +1}, the sign
-    // set where the code bit is 0 (bits i and 16+i moved to 15 and 31)
-    const int i0 = 8 * (k & 1) + 2 * c;
-    b0 = ((~x << (15 - i0)) & 0x80008000u) | 0x3F803F80u;
-    b1 = ((~x << (14 - i0)) & 0x80008000u) | 0x3F803F80u;
-  } else if constexpr (BITS == 2) {
-    // pairs 2c and 2c+1 of the 16-code word: bf16 {-2, 0, +2}
-    b0 = (x << (14 - 4 * c)) & 0xC000C000u;
-    b1 = (x << (12 - 4 * c)) & 0xC000C000u;
-  } else if constexpr (BITS == 4) {
-    // pairs 2(c%2) and 2(c%2)+1 of the 8-code word: bf16 128 + q
-    const int sh = 8 * (c & 1);
-    b0 = ((x >> sh) & 0x000F000Fu) | 0x43004300u;
-    b1 = ((x >> (sh + 4)) & 0x000F000Fu) | 0x43004300u;
-  } else {
-    // byte j is code 4c + j; exact q through an fp32 magic number
-    const float2 q01 = ptx::add2(make_float2(__uint_as_float(ptx::prmt(x, deq::kMagic, 0x7650u)),
-                                             __uint_as_float(ptx::prmt(x, deq::kMagic, 0x7651u))),
-                                 make_float2(-deq::kMagicF, -deq::kMagicF));
-    const float2 q23 = ptx::add2(make_float2(__uint_as_float(ptx::prmt(x, deq::kMagic, 0x7652u)),
-                                             __uint_as_float(ptx::prmt(x, deq::kMagic, 0x7653u))),
-                                 make_float2(-deq::kMagicF, -deq::kMagicF));
-    b0 = ptx::cvt_bf16x2(q01.x, q01.y);
-    b1 = ptx::cvt_bf16x2(q23.x, q23.y);
-  }
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 template <int BITS, int MT, int NP>
@@ -181,13 +151,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   static_assert(NP % PH == 0, "the halves take whole 16-row pairs");
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = ptx::smem_u32(smem);
-  if (sbase & 1023u) {  // the swizzled boxes need it; uniform across the block
+  if (sbase & 1023u) {  // the swizzled boxes need it; uniform across the block (and the cluster)
     if (threadIdx.x == 0) ptx::set_status(p.status, kStatusLayout);
+    if (p.ksplit > 1) {  // the cluster's peers pass both of its barriers whatever happens here
+      cluster_sync();
+      cluster_sync();
+    }
     return;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
-  const int n0 = blockIdx.x * R;
+  // K-split launches: the CTAs of a cluster share one row block, CTA `kslice`
+  // taking K stages [ks0, ks0 + ns) of it; the partial sums meet at the end.
+  const int kslice = p.ksplit > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int n0 = (blockIdx.x / p.ksplit) * R;
+  const int ks0 = kslice * p.num_stages / p.ksplit;
+  const int ns = (kslice + 1) * p.num_stages / p.ksplit - ks0;
   const int U = 1 << p.unit_shift;
 
   const uint32_t bar0 = sbase + p.data_bytes;
@@ -198,7 +177,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // Each CTA walks the K stages starting at its own offset: every CTA reads
   // the same activations, and rotating the order spreads those reads over
   // the L2 instead of sending all CTAs to the same lines at once.
-  const int rot = blockIdx.x % p.num_stages;
+  const int rot = (blockIdx.x / p.ksplit) % ns;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.ring; ++s) {
@@ -228,9 +207,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ---------------- producer: TMA boxes and bulk copies into the ring ----------------
     constexpr int sb_bytes = GS * R * 2;
     const int units = F::ROWB / U;  // row pieces per stage
-    const int pre = p.ring < p.num_stages ? p.ring : p.num_stages;
+    const int pre = p.ring < ns ? p.ring : ns;
     auto stage_k = [&](int t, int& kt, int& valid) {
-      kt = (t + rot) % p.num_stages;  // which K stage ring round t carries
+      kt = ks0 + (t + rot) % ns;  // which K stage ring round t carries
       valid = min(F::KS, p.K - kt * F::KS);
     };
     auto load_weights = [&](int t, int s) {  // lane 0: the stage's packed codes, scales and biases
@@ -278,7 +257,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
     int t = pre;
-    for (; t < p.num_stages; ++t) {
+    for (; t < ns; ++t) {
       const int s = t % p.ring;
       if (!warp_wait(empty(s), ((t / p.ring) & 1) ^ 1, lim, abort_flag)) {
         if (lane == 0) give_up();
@@ -304,9 +283,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int gl = warp % GROUP_LANES;  // group lane: groups gl, gl + GROUP_LANES, ... of every stage
     const int q0 = (warp / GROUP_LANES) * NPH;  // first 16-row pair of this warp's half
     const bool ga = g < p.M, gb = MT > 8 && g + 8 < p.M;  // tokens g and g + 8 exist
-    for (int t = 0; t < p.num_stages; ++t) {
+    const bool compute = !p.floor_only;
+    for (int t = 0; t < ns; ++t) {
       const int s = t % p.ring;
-      const int kt = (t + rot) % p.num_stages;
+      const int kt = ks0 + (t + rot) % ns;
       // The activations of this warp's groups (the B operand: tokens g and
       // g + 8, k = gs*G + 16*step + 4c .. +3) straight from global memory,
       // where every CTA reads the same rows (L2 hits); issued before the
@@ -315,7 +295,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int gi = 0; gi < (XR ? 0 : GPL); ++gi) {
         const int k0 = kt * F::KS + (gl + GROUP_LANES * gi) * F::G;
-        const bool in = k0 < p.K;
+        const bool in = compute && k0 < p.K;
         const uint2* x0p = reinterpret_cast<const uint2*>(p.X + static_cast<size_t>(g) * p.K + k0 + 4 * c);
         const uint2* x1p = reinterpret_cast<const uint2*>(p.X + static_cast<size_t>(g + 8) * p.K + k0 + 4 * c);
 #pragma unroll
@@ -332,7 +312,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int gi = 0; gi < GPL; ++gi) {
         const int gs = gl + GROUP_LANES * gi;
-        if (kt * F::KS + gs * F::G >= p.K) break;
+        if (!compute || kt * F::KS + gs * F::G >= p.K) break;
         float xs[TH][4];  // sum of x over the group per token (affine)
         float tmp[NPH][TH][4];
 #pragma unroll
@@ -426,34 +406,68 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
   }
   __syncthreads();
+  if (p.ksplit == 1) {
+    if (p.floor_only) return;
+    for (int i = threadIdx.x; i < p.M * R; i += NUM_THREADS) {
+      const int m = i / R, nl = i - m * R;
+      const int n = n0 + nl;
+      if (n >= p.N) continue;
+      float v = 0.f;
+#pragma unroll
+      for (int l = 0; l < GROUP_LANES; ++l) v += red[(l * MT + m) * NLP + nl];
+      if (p.bias) v += __bfloat162float(__ushort_as_bfloat16(p.bias[n]));
+      const size_t o = static_cast<size_t>(m) * p.N + n;
+      if (p.epi != QGEMM_EPI_NONE)
+        v = epi::apply_dyn(p.epi, v, p.epi == QGEMM_EPI_RESIDUAL_GATE ? p.residual[o] : uint16_t(0),
+                           p.epi == QGEMM_EPI_RESIDUAL_GATE ? epi::bf16_to_f32(p.gate[n]) : 0.f);
+      p.out[o] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    }
+    return;
+  }
+  // K-split: each CTA first sums its own group lanes into loc[m][R], then,
+  // once every slice of the cluster has, finishes outputs i = kslice, kslice
+  // + ksplit, ... by adding the slices' sums in slice order over distributed
+  // shared memory. The second cluster barrier keeps every CTA (and so its
+  // shared memory) alive until its peers have read it.
+  float* loc = red + GROUP_LANES * MT * NLP;
   for (int i = threadIdx.x; i < p.M * R; i += NUM_THREADS) {
     const int m = i / R, nl = i - m * R;
-    const int n = n0 + nl;
-    if (n >= p.N) continue;
     float v = 0.f;
 #pragma unroll
     for (int l = 0; l < GROUP_LANES; ++l) v += red[(l * MT + m) * NLP + nl];
-    if (p.bias) v += __bfloat162float(__ushort_as_bfloat16(p.bias[n]));
-    const size_t o = static_cast<size_t>(m) * p.N + n;
-    if (p.epi != QGEMM_EPI_NONE)
-      v = epi::apply_dyn(p.epi, v, p.epi == QGEMM_EPI_RESIDUAL_GATE ? p.residual[o] : uint16_t(0),
-                         p.epi == QGEMM_EPI_RESIDUAL_GATE ? epi::bf16_to_f32(p.gate[n]) : 0.f);
-    p.out[o] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    loc[i] = v;
   }
+  cluster_sync();
+  if (!p.floor_only) {
+    const uint32_t loc_addr = ptx::smem_u32(loc);
+    for (int i = threadIdx.x + kslice * NUM_THREADS; i < p.M * R; i += p.ksplit * NUM_THREADS) {
+      const int m = i / R, nl = i - m * R;
+      const int n = n0 + nl;
+      if (n >= p.N) continue;
+      float v = 0.f;
+      for (int r = 0; r < p.ksplit; ++r) v += ld_shared_cluster_f32(mapa_shared(loc_addr + 4u * i, r));
+      if (p.bias) v += __bfloat162float(__ushort_as_bfloat16(p.bias[n]));
+      const size_t o = static_cast<size_t>(m) * p.N + n;
+      if (p.epi != QGEMM_EPI_NONE)
+        v = epi::apply_dyn(p.epi, v, p.epi == QGEMM_EPI_RESIDUAL_GATE ? p.residual[o] : uint16_t(0),
+                           p.epi == QGEMM_EPI_RESIDUAL_GATE ? epi::bf16_to_f32(p.gate[n]) : 0.f);
+      p.out[o] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    }
+  }
+  cluster_sync();
 }
 
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
+// The stage layout and kernel parameters of one configuration (format BITS,
+// MT tokens, 16 NP rows per CTA, `ksplit` K slices per row block) for a
+// problem, and the dynamic shared memory it takes.
 template <int BITS, int MT, int NP>
-int launch_fmt(const Problem& pr, int grid) {
+int make_params(const Problem& pr, int ksplit, Params& kp, int& smem) {
   using F = Fmt<BITS>;
   constexpr int R = 16 * NP;
-  int st = smem_opt_in(reinterpret_cast<const void*>(small_m_kernel<BITS, MT, NP>), SMEM_LIMIT,
-                       "cudaFuncSetAttribute(small_m_kernel)");
-  if (st != QGEMM_OK) return st;
-
-  Params kp;
+  kp = Params{};
   kp.X = static_cast<const uint16_t*>(pr.X);
   kp.bias = pr.bias;
   kp.out = static_cast<uint16_t*>(pr.out);
@@ -464,6 +478,10 @@ int launch_fmt(const Problem& pr, int grid) {
   kp.N = pr.N;
   kp.K = pr.K;
   kp.num_stages = (pr.K + F::KS - 1) / F::KS;
+  kp.ksplit = ksplit;
+  if (ksplit < 1 || ksplit > kp.num_stages)
+    return fail(QGEMM_ERR_UNSUPPORTED, "internal: %d K slices for %d stages", ksplit, kp.num_stages);
+  const int slice_stages = (kp.num_stages + ksplit - 1) / ksplit;  // the longest slice
   const uint64_t wbytes = static_cast<uint64_t>(pr.K) * BITS / 8;  // packed bytes per weight row
   const int unit = wbytes % 128 == 0 ? 128 : wbytes % 64 == 0 ? 64 : 32;  // K % 128 == 0 makes it at least 32
   kp.unit_shift = unit == 128 ? 7 : unit == 64 ? 6 : 5;
@@ -479,18 +497,35 @@ int launch_fmt(const Problem& pr, int grid) {
   kp.stage_bytes = (kp.off_x + (x_in_ring(MT, NP) ? pr.M * kp.x_stride : 0) + 1023) & ~1023;
   int ring = RING_BUDGET / kp.stage_bytes;
   ring = ring < MAX_STAGES ? ring : MAX_STAGES;
-  ring = ring < kp.num_stages ? ring : kp.num_stages;
+  ring = ring < slice_stages ? ring : slice_stages;
   kp.ring = ring < 1 ? 1 : ring;
-  const int red_bytes = NUM_CONSUMER_WARPS / split_rows(MT, NP) * MT * (R + 4) * 4;
+  // the warps' partial sums (and, K-split, the CTA's own sums over them) reuse the ring at the end
+  const int red_bytes = NUM_CONSUMER_WARPS / split_rows(MT, NP) * MT * (R + 4) * 4 + (ksplit > 1 ? MT * R * 4 : 0);
   kp.data_bytes = kp.ring * kp.stage_bytes > red_bytes ? kp.ring * kp.stage_bytes : red_bytes;
   if (kp.data_bytes < SMEM_FLOOR) kp.data_bytes = SMEM_FLOOR;
-  const int smem = kp.data_bytes + 16 * MAX_STAGES + 16;
+  smem = kp.data_bytes + 16 * MAX_STAGES + 16;
   if (smem > SMEM_LIMIT) return fail(QGEMM_ERR_UNSUPPORTED, "small-M stage of %d bytes does not fit", kp.stage_bytes);
   if (kp.off_s % 1024 || kp.off_b % 128 || kp.off_x % 128 || kp.x_stride % 16 || kp.stage_bytes % 1024 ||
       kp.data_bytes % 8)
     return fail(QGEMM_ERR_UNSUPPORTED, "internal: small-M stage layout misaligned");
+  kp.overlap = pr.overlap ? 1 : 0;
+  kp.floor_only = pr.floor_only ? 1 : 0;
   kp.wait_limit_ns = wait_limit_ns();
-  if ((st = status_word(&kp.status)) != QGEMM_OK) return st;
+  return status_word(&kp.status);
+}
+
+template <int BITS, int MT, int NP>
+int launch_fmt(const Problem& pr, int ksplit, int grid) {
+  using F = Fmt<BITS>;
+  constexpr int R = 16 * NP;
+  const void* fn = reinterpret_cast<const void*>(small_m_kernel<BITS, MT, NP>);
+  int st = smem_opt_in(fn, SMEM_LIMIT, "cudaFuncSetAttribute(small_m_kernel)");
+  if (st != QGEMM_OK) return st;
+  Params kp;
+  int smem = 0;
+  if ((st = make_params<BITS, MT, NP>(pr, ksplit, kp, smem)) != QGEMM_OK) return st;
+  const int unit = 1 << kp.unit_shift;
+  const uint64_t wbytes = static_cast<uint64_t>(pr.K) * BITS / 8;
 
   CUtensorMap tm_w, tm_s, tm_b;
   const uint64_t groups = static_cast<uint64_t>(pr.K) / F::G;
@@ -515,35 +550,142 @@ int launch_fmt(const Problem& pr, int grid) {
   } else {
     tm_b = tm_s;  // unused for ternary
   }
-  kp.overlap = pr.overlap ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(NUM_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = pr.stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (ksplit > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = ksplit;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pr.overlap) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pr.overlap ? 1 : 0;
+  cfg.numAttrs = na;
   return cuda_check(cudaLaunchKernelEx(&cfg, small_m_kernel<BITS, MT, NP>, tm_w, tm_s, tm_b, kp),
                     "small_m_kernel launch");
 }
 
-// Rows per CTA: the fewest 16-row pairs (from the compiled set) that cover N
-// with at most one CTA per SM.
+// Whether `clusters` clusters of `ksplit` CTAs of this configuration are
+// resident on the device at once (queried once per configuration and device).
+template <int BITS, int MT, int NP>
+int clusters_fit(const Problem& pr, int ksplit, int clusters, bool* ok) {
+  const void* fn = reinterpret_cast<const void*>(small_m_kernel<BITS, MT, NP>);
+  int st = smem_opt_in(fn, SMEM_LIMIT, "cudaFuncSetAttribute(small_m_kernel)");
+  if (st != QGEMM_OK) return st;
+  Params kp;
+  int smem = 0;
+  if ((st = make_params<BITS, MT, NP>(pr, ksplit, kp, smem)) != QGEMM_OK) return st;
+  int dev = 0;
+  if ((st = cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) != QGEMM_OK) return st;
+  static std::mutex mu;
+  static std::map<std::tuple<int, const void*, int, int>, int> cache;  // (device, kernel, ksplit, smem) -> clusters
+  const auto key = std::make_tuple(dev, fn, ksplit, smem);
+  int n = -1;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) n = it->second;
+  }
+  if (n < 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(clusters * ksplit);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = ksplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((st = cuda_check(cudaOccupancyMaxActiveClusters(&n, fn, &cfg), "cudaOccupancyMaxActiveClusters")) != QGEMM_OK)
+      return st;
+    std::lock_guard<std::mutex> lk(mu);
+    cache[key] = n;
+  }
+  *ok = n >= clusters;
+  return QGEMM_OK;
+}
+
+// Rows per CTA (16 NP, NP from the compiled set) and K slices per row block
+// (a cluster of `ksplit` CTAs): the choice that puts the fewest row-stages of
+// packed weights on the busiest CTA with the whole grid resident at once, the
+// fewer slices on a tie. Narrow N with long K (MLP down, the out projection)
+// needs the slices: 3072 rows make only 96 CTAs of 32 rows, while 48 row
+// blocks of 64 rows x 3 slices use 144 SMs with a third less per CTA.
+struct Plan {
+  int np, ksplit, grid;
+};
+
+inline void plan_candidates(int pairs, int nst, int nsm, Plan* out, int* count) {
+  static constexpr int kNP[4] = {2, 4, 6, 8};
+  static constexpr int kS[6] = {1, 2, 3, 4, 6, 8};
+  int n = 0;
+  for (int np : kNP)
+    for (int S : kS) {
+      if (S > nst) continue;
+      const int grid = (pairs + np - 1) / np * S;
+      if (grid > nsm) continue;
+      out[n++] = Plan{np, S, grid};
+    }
+  // cheapest first: row-stages on the busiest CTA, then fewer slices
+  auto cost = [&](const Plan& p) { return p.np * ((nst + p.ksplit - 1) / p.ksplit); };
+  for (int i = 1; i < n; ++i)
+    for (int j = i; j > 0; --j) {
+      const Plan a = out[j - 1], b = out[j];
+      if (cost(b) < cost(a) || (cost(b) == cost(a) && b.ksplit < a.ksplit)) {
+        out[j - 1] = b;
+        out[j] = a;
+      }
+    }
+  *count = n;
+}
+
+template <int BITS, int MT, int NP>
+int try_plan(const Problem& pr, const Plan& pl, bool* launched) {
+  *launched = false;
+  if (pl.ksplit > 1) {
+    bool ok = false;
+    int st = clusters_fit<BITS, MT, NP>(pr, pl.ksplit, pl.grid / pl.ksplit, &ok);
+    if (st != QGEMM_OK) return st;
+    if (!ok) return QGEMM_OK;
+  }
+  *launched = true;
+  return launch_fmt<BITS, MT, NP>(pr, pl.ksplit, pl.grid);
+}
+
 template <int BITS, int MT>
 int launch_rows(const Problem& pr, int nsm) {
+  using F = Fmt<BITS>;
   const int pairs = pr.N / 16;
-  const int need = (pairs + nsm - 1) / nsm;
-  const int np = need <= 2 ? 2 : need <= 4 ? 4 : need <= 6 ? 6 : 8;
-  const int grid = (pairs + np - 1) / np;
-  switch (np) {
-    case 2: return launch_fmt<BITS, MT, 2>(pr, grid);
-    case 4: return launch_fmt<BITS, MT, 4>(pr, grid);
-    case 6: return launch_fmt<BITS, MT, 6>(pr, grid);
-    default: return launch_fmt<BITS, MT, 8>(pr, grid);
+  const int nst = (pr.K + F::KS - 1) / F::KS;
+  Plan cands[24];
+  int count = 0;
+  plan_candidates(pairs, nst, nsm, cands, &count);
+  for (int i = 0; i < count; ++i) {
+    const Plan& pl = cands[i];
+    bool launched = false;
+    int st = QGEMM_OK;
+    switch (pl.np) {
+      case 2: st = try_plan<BITS, MT, 2>(pr, pl, &launched); break;
+      case 4: st = try_plan<BITS, MT, 4>(pr, pl, &launched); break;
+      case 6: st = try_plan<BITS, MT, 6>(pr, pl, &launched); break;
+      default: st = try_plan<BITS, MT, 8>(pr, pl, &launched);
+    }
+    if (st != QGEMM_OK || launched) return st;
   }
+  // more rows than one wave of 128-row CTAs covers: several waves, no slices
+  return launch_fmt<BITS, MT, 8>(pr, 1, (pairs + 7) / 8);
 }
 
 template <int BITS>
