@@ -615,10 +615,17 @@ def run_case(args):
     torch.cuda.synchronize()
     wq.check_device_status()
     t = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e-3
+    fns = [(lambda s=s: wq.qgemm(s[0], s[1], bias=s[2], out=s[3])) for s in sets]
+    launches = max(len(fns), 100 if M <= 16 else 20)
+    tg = time_graph((fns * (-(-launches // len(fns))))[:launches])
+    wq.check_device_status()
+    flops = 2 * M * lin.N * lin.K
     return {"case": args.case, "M": M, "N": lin.N, "K": lin.K, "bits": lin.bits,
             "path": "small" if wq.qgemm_select_path(M, lin.N, lin.K, lin.bits) == 1 else "large",
-            "us_per_launch_events": round(t * 1e6, 2), "copies": ncopy,
-            "note": "per-launch events include host launch gaps for short kernels; the sweep's graph timing does not"}
+            "us_per_launch_events": round(t * 1e6, 2), "us_graph": round(tg * 1e6, 2),
+            "tflops_graph": round(flops / tg / 1e12, 1), "gbs_graph": round(ab / tg / 1e9, 1), "copies": ncopy,
+            "env": {k: os.environ[k] for k in ("QGEMM_PATH", "QGEMM_LARGE_PAIR") if k in os.environ},
+            "note": "per-launch events include host launch gaps for short kernels; the graph timing does not"}
 
 
 def run_e2e(sets, X_host_bits, lin, args, world):

@@ -53,8 +53,10 @@
 
 #include <cuda.h>
 
+#include <map>
 #include <mutex>
 #include <type_traits>
+#include <utility>
 
 #include "dequant.cuh"
 #include "epilogue.cuh"
@@ -78,8 +80,6 @@ constexpr int WARP_WLOAD = 2;
 constexpr int WARP_DEQ0 = 3;
 constexpr int WARP_EPI0 = WARP_DEQ0 + NUM_DEQ_WARPS;
 constexpr int NUM_THREADS = 32 * (WARP_EPI0 + NUM_EPI_WARPS);
-constexpr int X_BOX_BYTES = TILE_M * BOX_K * 2;  // 32 KB
-constexpr int X_STAGE_BYTES = 2 * X_BOX_BYTES;    // 64 KB
 constexpr int EPI_ROWS = 32;                      // tokens per tcgen05.ld
 constexpr int EPI_SLOT_BYTES = EPI_ROWS * 32 * 2; // one 32 tokens x 32 features bf16 block
 constexpr int EPI_TOKENS = TILE_M / (NUM_EPI_WARPS / 4);  // tokens per epilogue warp
@@ -88,12 +88,22 @@ constexpr uint32_t ACC_COL = 0;                   // fp32 accumulator: columns 0
 constexpr uint32_t A_COL = TILE_M;                // A stages: columns 256..
 constexpr uint32_t A_STAGE_COLS = BK / 2;         // 128 bf16 per row = 64 columns
 constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TILE_N, TILE_M);
+constexpr uint32_t IDESC_PAIR = ptx::idesc_bf16_f32(2 * TILE_N, TILE_M);  // cta_group::2: M = 256 over the pair
 constexpr int EPI_BAR_ID = 1;
 static_assert(NUM_THREADS <= 1024, "one CTA holds at most 1024 threads");
 static_assert(EPI_TOKENS % EPI_ROWS == 0, "epilogue warps cover whole tcgen05.ld chunks");
 
-template <int BITS>
+// PAIR: the CTA-pair form. Two CTAs of a cluster compute a 256-row x
+// 256-token tile with tcgen05.mma.cta_group::2 (M = 256): each CTA holds
+// its 128 weight rows' A stages and accumulator in its own tensor memory and
+// stages 128 of the 256 tokens (the MMA reads the B operand from both CTAs'
+// shared memory), so an activation stage takes 32 KB instead of 64 and four
+// fit where one CTA alone holds two.
+template <int BITS, bool PAIR = false>
 struct Cfg {
+  static constexpr int kTokens = PAIR ? TILE_M / 2 : TILE_M;  // tokens this CTA stages
+  static constexpr int kXBoxBytes = kTokens * BOX_K * 2;
+  static constexpr int kXStageBytes = 2 * kXBoxBytes;
   static constexpr int kGroup = BITS <= 2 ? 128 : 64;
   static constexpr int kGroupsPerStage = BK / kGroup;
   static constexpr int kWRowBytes = BK * BITS / 8;        // packed bytes per row per stage
@@ -108,15 +118,15 @@ struct Cfg {
   static constexpr uint32_t kSwzMask = BITS == 8 ? 7 : BITS == 4 ? 3 : BITS == 2 ? 1 : 0;
   static constexpr int kSBytes = kGroupsPerStage * TILE_N * 2;  // one stage's scales (or biases)
   static constexpr int kSBStride = BITS <= 2 ? kSBytes : 2 * kSBytes;
-  static constexpr int kS = BITS == 8 ? 2 : 3;                   // stage ring depth
+  static constexpr int kS = PAIR ? 4 : BITS == 8 ? 2 : 3;        // stage ring depth
   static constexpr int kSW = BITS == 8 ? 3 : BITS == 4 ? 2 : BITS == 2 ? 4 : 8;  // W ring depth
   static constexpr int kSlots = BITS == 8 ? 2 : 1;               // epilogue store slots per warp
   static constexpr int kOffX = 0;
-  static constexpr int kOffW = kOffX + kS * X_STAGE_BYTES;
+  static constexpr int kOffW = kOffX + kS * kXStageBytes;
   static constexpr int kOffOut = kOffW + kSW * kWTileBytes;
   static constexpr int kOffSB = kOffOut + NUM_EPI_WARPS * kSlots * EPI_SLOT_BYTES;
   static constexpr int kOffBar = kOffSB + kSW * kSBStride;
-  static constexpr int kNumBars = 2 * kS + 2 * kSW + 3;
+  static constexpr int kNumBars = 3 * kS + 2 * kSW + 3;  // full, empty, X landed (pair), W ring, accumulator
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -162,24 +172,43 @@ __device__ __forceinline__ uint32_t swz(uint32_t off) {
   return off ^ (((off >> 7) & MASK) << 4);
 }
 
-template <int BITS, int EPI>
+// Bounded waits on barriers that the other CTA of a pair may arrive on.
+__device__ __forceinline__ bool warp_wait_cluster(uint32_t bar, uint32_t parity, uint64_t lim,
+                                                  const volatile int* abort) {
+  const bool ok = ptx::mbar_wait_cluster(bar, parity, lim, abort);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int BITS, int EPI, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     large_m_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                    const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_res,
                    const Params p) {
-  using C = Cfg<BITS>;
+  using C = Cfg<BITS, PAIR>;
   constexpr int S = C::kS, SW = C::kSW;
+  constexpr int TILE_ROWS = PAIR ? 2 * TILE_N : TILE_N;  // weight rows of one output tile
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = ptx::smem_u32(smem);
-  if (sbase & 1023u) {  // the swizzled tiles need it; uniform across the block
+  if (sbase & 1023u) {  // the swizzled tiles need it; uniform across the block (and the pair)
     if (threadIdx.x == 0) ptx::set_status(p.status, kStatusLayout);
+    if constexpr (PAIR) {  // the peer passes both of its cluster barriers whatever happens here
+      ptx::cluster_sync();
+      ptx::cluster_sync();
+    }
     return;
   }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // The pair: CTA `rank` holds weight rows rank * 128 .. +127 of each tile and
+  // stages tokens rank * 128 .. +127; the even CTA issues the MMAs.
+  const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;
+  const int unit = PAIR ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
+  const int units = PAIR ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
+  const int row0 = static_cast<int>(rank) * TILE_N;     // this CTA's first row inside a tile
+  const int tok0 = static_cast<int>(rank) * C::kTokens;  // this CTA's first staged token inside a tile
 
-  auto x_stage = [&](int s) { return sbase + C::kOffX + s * X_STAGE_BYTES; };
+  auto x_stage = [&](int s) { return sbase + C::kOffX + s * C::kXStageBytes; };
   const uint32_t bar0 = sbase + C::kOffBar;
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (S + s); };
@@ -188,29 +217,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t acc_full = bar0 + 8u * (2 * S + 2 * SW);
   const uint32_t acc_empty = acc_full + 8u;
   const uint32_t drain_bar = acc_full + 16u;
+  auto xfull = [&](int s) { return bar0 + 8u * (2 * S + 2 * SW + 3 + s); };  // pair: this CTA's X landed
+  // where this CTA's arrivals for a stage and for the accumulator go: the
+  // even CTA's barriers (a shared::cluster address; the CTA's own one alone)
+  auto full_arrive = [&](int s) {
+    if constexpr (PAIR) ptx::mbar_arrive_remote(ptx::mapa_shared(full(s), 0));
+    else ptx::mbar_arrive(full(s));
+  };
+  auto acc_empty_arrive = [&]() {
+    if constexpr (PAIR) ptx::mbar_arrive_remote(ptx::mapa_shared(acc_empty, 0));
+    else ptx::mbar_arrive(acc_empty);
+  };
+  // waits on barriers the other CTA of a pair (or its commits) may complete
+  auto wait_x = [&](uint32_t bar, uint32_t par) {
+    if constexpr (PAIR) return ptx::mbar_wait_cluster(bar, par, p.wait_limit_ns, nullptr);
+    else return ptx::mbar_wait(bar, par, p.wait_limit_ns, nullptr);
+  };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   volatile int* epi_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      ptx::mbar_init(full(s), 1 + NUM_DEQ_WARPS);  // the X producer's arrival + one per dequantiser
+      // the X producer's arrival + one per dequantiser; a pair's even CTA also
+      // counts the odd one's dequantisers and its relayed X arrival
+      ptx::mbar_init(full(s), PAIR ? 2 + 2 * NUM_DEQ_WARPS : 1 + NUM_DEQ_WARPS);
       ptx::mbar_init(empty(s), 1);
+      ptx::mbar_init(xfull(s), 1);
     }
     for (int s = 0; s < SW; ++s) {
       ptx::mbar_init(full_w(s), 1);
       ptx::mbar_init(empty_w(s), NUM_DEQ_WARPS);
     }
     ptx::mbar_init(acc_full, 1);
-    ptx::mbar_init(acc_empty, NUM_EPI_WARPS);
+    ptx::mbar_init(acc_empty, PAIR ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS);
     ptx::mbar_init(drain_bar, 1);
     *abort_flag = 0;
     *epi_abort = 0;
     ptx::fence_mbarrier_init();
   }
   if (warp == WARP_MMA) {
-    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), TMEM_COLS);
-    ptx::tmem_relinquish();
+    if constexpr (PAIR) {
+      ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), TMEM_COLS);
+      ptx::tmem_relinquish_pair();
+    } else {
+      ptx::tmem_alloc(ptx::smem_u32(tmem_slot), TMEM_COLS);
+      ptx::tmem_relinquish();
+    }
   }
   if (warp == WARP_XLOAD && lane == 0) {
     ptx::tma_prefetch_desc(&tm_x);
@@ -223,11 +276,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   ptx::tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) ptx::cluster_sync();  // both CTAs' barriers and TMEM are ready before any cross-CTA use
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint64_t lim = p.wait_limit_ns;
-  const int my_tiles = (p.num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
-                       static_cast<int>(gridDim.x);
+  const int my_tiles = (p.num_tiles - unit + units - 1) / units;
   const uint32_t total = static_cast<uint32_t>(my_tiles) * static_cast<uint32_t>(p.num_kb);
 
   auto give_up = [&]() {
@@ -242,29 +295,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int R = is_x ? S : SW;
       uint32_t it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      for (int tile = unit; ok && tile < p.num_tiles; tile += units) {
         int n_tile, m_tile;
         tile_coords(p, tile, n_tile, m_tile);
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
           const int s = it % R;
           const uint32_t par = ((it / R) & 1) ^ 1;
-          if (!ptx::mbar_wait(is_x ? empty(s) : empty_w(s), par, lim, abort_flag)) {
+          const bool waited = is_x && PAIR ? ptx::mbar_wait_cluster(empty(s), par, lim, abort_flag)
+                                           : ptx::mbar_wait(is_x ? empty(s) : empty_w(s), par, lim, abort_flag);
+          if (!waited) {
             give_up();
             ok = false;
             break;
           }
           if (is_x) {
-            ptx::mbar_arrive_expect_tx(full(s), X_STAGE_BYTES);
-            ptx::tma_load_2d(x_stage(s), &tm_x, kb * BK, m_tile * TILE_M, full(s));
-            ptx::tma_load_2d(x_stage(s) + X_BOX_BYTES, &tm_x, kb * BK + BOX_K, m_tile * TILE_M, full(s));
+            // the odd CTA of a pair counts its bytes on its own barrier; the MMA
+            // warp there relays the stage to the even CTA once they land
+            const uint32_t xb = PAIR && rank ? xfull(s) : full(s);
+            ptx::mbar_arrive_expect_tx(xb, C::kXStageBytes);
+            ptx::tma_load_2d(x_stage(s), &tm_x, kb * BK, m_tile * TILE_M + tok0, xb);
+            ptx::tma_load_2d(x_stage(s) + C::kXBoxBytes, &tm_x, kb * BK + BOX_K, m_tile * TILE_M + tok0, xb);
           } else {
             const uint32_t wdst = sbase + C::kOffW + s * C::kWTileBytes;
             const uint32_t sdst = sbase + C::kOffSB + s * C::kSBStride;
             const int grp = kb * C::kGroupsPerStage;
             ptx::mbar_arrive_expect_tx(full_w(s), C::kWTileBytes + C::kSBStride);
-            ptx::tma_load_2d(wdst, &tm_w, kb * C::kWRowBytes, n_tile * TILE_N, full_w(s));
-            ptx::tma_load_2d(sdst, &tm_s, n_tile * TILE_N, grp, full_w(s));
-            if (BITS > 2) ptx::tma_load_2d(sdst + C::kSBytes, &tm_b, n_tile * TILE_N, grp, full_w(s));
+            const int nr = n_tile * TILE_ROWS + row0;
+            ptx::tma_load_2d(wdst, &tm_w, kb * C::kWRowBytes, nr, full_w(s));
+            ptx::tma_load_2d(sdst, &tm_s, nr, grp, full_w(s));
+            if (BITS > 2) ptx::tma_load_2d(sdst + C::kSBytes, &tm_b, nr, grp, full_w(s));
           }
         }
       }
@@ -274,11 +333,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t first = it > static_cast<uint32_t>(R) ? it - R : 0;
       for (uint32_t i = first; i < it; ++i) {
         if (is_x)
-          ptx::mbar_wait(empty(i % R), (i / R) & 1, lim, nullptr);
+          wait_x(empty(i % R), (i / R) & 1);
         else
           ptx::mbar_wait(full_w(i % R), (i / R) & 1, lim, nullptr);
       }
     }
+  } else if (warp == WARP_MMA && PAIR && rank != 0) {
+    // ---------------- the odd CTA of a pair: relay ----------------
+    // Its X stages land on its own barrier; once one has, tell the even CTA,
+    // whose MMA reads this CTA's half of the B operand.
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = unit; ok && tile < p.num_tiles; tile += units)
+      for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+        const int s = it % S;
+        if (!warp_wait(xfull(s), (it / S) & 1, lim, abort_flag)) {
+          if (lane == 0) give_up();
+          ok = false;
+          break;
+        }
+        if (lane == 0) full_arrive(s);
+        __syncwarp();
+      }
+    // the even CTA's last commit says every MMA of the pair is done: only
+    // then may this CTA's tensor memory be freed
+    if (lane == 0) ptx::mbar_wait_cluster(drain_bar, 0, lim, nullptr);
+    __syncwarp();
   } else if (warp == WARP_MMA) {
     // ---------------- MMA issuer ----------------
     // The whole warp runs the loop and waits; one elected lane issues. Keeping
@@ -287,15 +367,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t it = 0, tcount = 0;
     bool ok = true;
     const bool leader = ptx::elect_one();
-    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tcount) {
-      if (!warp_wait(acc_empty, (tcount & 1) ^ 1, lim, abort_flag)) {
+    auto wait_ok = [&](uint32_t bar, uint32_t par) {
+      return PAIR ? warp_wait_cluster(bar, par, lim, abort_flag) : warp_wait(bar, par, lim, abort_flag);
+    };
+    for (int tile = unit; ok && tile < p.num_tiles; tile += units, ++tcount) {
+      if (!wait_ok(acc_empty, (tcount & 1) ^ 1)) {
         if (leader) give_up();
         break;
       }
       ptx::tc_fence_after();
       for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
         const int s = it % S;
-        if (!warp_wait(full(s), (it / S) & 1, lim, abort_flag)) {
+        if (!wait_ok(full(s), (it / S) & 1)) {
           if (leader) give_up();
           ok = false;
           break;
@@ -306,20 +389,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint64_t d0 = ptx::smem_desc_sw128_kmajor(x_stage(s));
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-            const uint32_t xo = (kk / (BOX_K / UMMA_K)) * X_BOX_BYTES + (kk % (BOX_K / UMMA_K)) * UMMA_K * 2;
-            ptx::tc_mma_f16_ts(tmem_base + ACC_COL, a0 + kk * (UMMA_K / 2), d0 + (xo >> 4), IDESC, (kb | kk) != 0);
+            const uint32_t xo = (kk / (BOX_K / UMMA_K)) * C::kXBoxBytes + (kk % (BOX_K / UMMA_K)) * UMMA_K * 2;
+            if constexpr (PAIR)
+              ptx::tc_mma_f16_ts_pair(tmem_base + ACC_COL, a0 + kk * (UMMA_K / 2), d0 + (xo >> 4), IDESC_PAIR,
+                                      (kb | kk) != 0);
+            else
+              ptx::tc_mma_f16_ts(tmem_base + ACC_COL, a0 + kk * (UMMA_K / 2), d0 + (xo >> 4), IDESC, (kb | kk) != 0);
           }
-          ptx::tc_commit(empty(s));
+          if constexpr (PAIR) ptx::tc_commit_pair(empty(s), 0x3);
+          else ptx::tc_commit(empty(s));
         }
         __syncwarp();
       }
       if (!ok) break;
-      if (leader) ptx::tc_commit(acc_full);
+      if (leader) {
+        if constexpr (PAIR) ptx::tc_commit_pair(acc_full, 0x3);
+        else ptx::tc_commit(acc_full);
+      }
       __syncwarp();
     }
     if (leader) {
-      ptx::tc_commit(drain_bar);
-      ptx::mbar_wait(drain_bar, 0, lim, nullptr);
+      if constexpr (PAIR) {
+        ptx::tc_commit_pair(drain_bar, 0x3);
+        ptx::mbar_wait_cluster(drain_bar, 0, lim, nullptr);
+      } else {
+        ptx::tc_commit(drain_bar);
+        ptx::mbar_wait(drain_bar, 0, lim, nullptr);
+      }
     }
     __syncwarp();
   } else if (warp < WARP_EPI0) {
@@ -332,7 +428,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (uint32_t it = 0; it < total; ++it) {
       const int s = it % S, sw = it % SW;
       if (!warp_wait(full_w(sw), (it / SW) & 1, lim, abort_flag) ||
-          !warp_wait(empty(s), ((it / S) & 1) ^ 1, lim, abort_flag)) {
+          !(PAIR ? warp_wait_cluster(empty(s), ((it / S) & 1) ^ 1, lim, abort_flag)
+                 : warp_wait(empty(s), ((it / S) & 1) ^ 1, lim, abort_flag))) {
         if (lane == 0) give_up();
         break;
       }
@@ -393,7 +490,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(full(s));
+      if (lane == 0) full_arrive(s);
     }
   } else {
     // ---------------- epilogue ----------------
@@ -404,10 +501,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint16_t* slots = reinterpret_cast<uint16_t*>(smem + C::kOffOut + e * C::kSlots * EPI_SLOT_BYTES);
     const uint32_t slots_u32 = sbase + C::kOffOut + e * C::kSlots * EPI_SLOT_BYTES;
     uint32_t tcount = 0, nstore = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+    for (int tile = unit; tile < p.num_tiles; tile += units, ++tcount) {
       int n_tile, m_tile;
       tile_coords(p, tile, n_tile, m_tile);
-      const int n = n_tile * TILE_N + n_local;
+      const int nr = n_tile * TILE_ROWS + row0;  // this CTA's first weight row of the tile
+      const int n = nr + n_local;
       const int m0 = m_tile * TILE_M + t0;
       const bool n_ok = n < p.N;
       const float bias_f = (p.bias && n_ok) ? __bfloat162float(__ushort_as_bfloat16(p.bias[n])) : 0.f;
@@ -415,9 +513,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if constexpr (EPI == QGEMM_EPI_RESIDUAL_GATE) {
         if (n_ok) gate_f = epi::bf16_to_f32(p.gate[n]);
         // while the tile's MMAs run, bring its residual block into L2
-        if (e == 0 && lane == 0) ptx::tma_prefetch_l2_2d(&tm_res, n_tile * TILE_N, m_tile * TILE_M);
+        if (e == 0 && lane == 0) ptx::tma_prefetch_l2_2d(&tm_res, nr, m_tile * TILE_M);
       }
-      const bool got = warp_wait(acc_full, tcount & 1, lim, abort_flag);
+      const bool got = PAIR ? warp_wait_cluster(acc_full, tcount & 1, lim, abort_flag)
+                            : warp_wait(acc_full, tcount & 1, lim, abort_flag);
       if (!got && lane == 0) {
         *epi_abort = 1;
         give_up();
@@ -451,9 +550,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // this warp's last read of the accumulator: hand it back before storing
           ptx::tc_fence_before();
           __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(acc_empty);
+          if (lane == 0) acc_empty_arrive();
         }
-        if (c < chunks && n_tile * TILE_N + 32 * q < p.N) {
+        if (c < chunks && nr + 32 * q < p.N) {
           const uint32_t slot = nstore % C::kSlots;
           // the TMA store that last used this slot has finished reading it
           if (lane == 0) ptx::bulk_wait_group_read<C::kSlots - 1>();
@@ -470,7 +569,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           __syncwarp();
           if (lane == 0) {
             // rows past M and columns past N fall outside the tensor map and are dropped
-            ptx::tma_store_2d(&tm_out, slots_u32 + slot * EPI_SLOT_BYTES, n_tile * TILE_N + 32 * q, m0 + c * EPI_ROWS);
+            ptx::tma_store_2d(&tm_out, slots_u32 + slot * EPI_SLOT_BYTES, nr + 32 * q, m0 + c * EPI_ROWS);
             ptx::bulk_commit_group();
           }
           ++nstore;
@@ -482,27 +581,64 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   ptx::tc_fence_before();
   __syncthreads();
+  // a pair: neither CTA leaves (or frees its tensor memory) while the other
+  // may still arrive on its barriers or the MMAs read its operands
+  if constexpr (PAIR) ptx::cluster_sync();
   if (warp == WARP_MMA) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+    if constexpr (PAIR) ptx::tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else ptx::tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-template <int BITS, int EPI>
+// How many CTA pairs of this kernel can be resident at once (queried once
+// per device and kernel): the grid of a pair launch takes no more, so that
+// every pair starts at once and the static tile order stays balanced.
+inline int max_pairs(const void* fn, int smem, int nsm) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nsm / 2;
+  static std::mutex mu;
+  static std::map<std::pair<int, const void*>, int> cache;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find({dev, fn});
+    if (it != cache.end()) return it->second;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (nsm / 2));
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n < 1) n = nsm / 2;
+  n = n < nsm / 2 ? n : nsm / 2;
+  std::lock_guard<std::mutex> lk(mu);
+  cache[{dev, fn}] = n;
+  return n;
+}
+
+template <int BITS, int EPI, bool PAIR>
 int launch_fmt(const Problem& pr, int nsm) {
-  using C = Cfg<BITS>;
-  int st = smem_opt_in(reinterpret_cast<const void*>(large_m_kernel<BITS, EPI>), C::kSmemBytes,
-                       "cudaFuncSetAttribute(large_m_kernel)");
+  using C = Cfg<BITS, PAIR>;
+  constexpr int TILE_ROWS = PAIR ? 2 * TILE_N : TILE_N;
+  const void* fn = reinterpret_cast<const void*>(large_m_kernel<BITS, EPI, PAIR>);
+  int st = smem_opt_in(fn, C::kSmemBytes, "cudaFuncSetAttribute(large_m_kernel)");
   if (st != QGEMM_OK) return st;
   CUtensorMap tm_x, tm_w, tm_s, tm_b;
   const uint64_t wbytes = static_cast<uint64_t>(pr.K) * BITS / 8;
   const uint64_t groups = static_cast<uint64_t>(pr.K) / C::kGroup;
   const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;
   if ((st = make_tensor_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pr.X, pr.K, pr.M, uint64_t(pr.K) * 2, BOX_K,
-                               TILE_M, CU_TENSOR_MAP_SWIZZLE_128B, "X")) != QGEMM_OK)
+                               C::kTokens, CU_TENSOR_MAP_SWIZZLE_128B, "X")) != QGEMM_OK)
     return st;
   if ((st = make_tensor_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.packed, wbytes, pr.N, wbytes, C::kWRowBytes,
                                TILE_N, C::kWSwizzle, "W")) != QGEMM_OK)
@@ -528,37 +664,52 @@ int launch_fmt(const Problem& pr, int nsm) {
   kp.N = pr.N;
   kp.K = pr.K;
   kp.num_m_tiles = (pr.M + TILE_M - 1) / TILE_M;
-  kp.num_n_tiles = (pr.N + TILE_N - 1) / TILE_N;
+  kp.num_n_tiles = (pr.N + TILE_ROWS - 1) / TILE_ROWS;
   if (static_cast<int64_t>(kp.num_m_tiles) * kp.num_n_tiles > INT32_MAX)
     return fail(QGEMM_ERR_UNSUPPORTED, "M=%d x N=%d: more output tiles than one launch indexes", pr.M, pr.N);
   kp.num_tiles = kp.num_m_tiles * kp.num_n_tiles;
   kp.num_kb = pr.K / BK;
-  const int grid = kp.num_tiles < nsm ? kp.num_tiles : nsm;
-  // The grid works on `grid` consecutive tiles at a time. Walk the dimension
+  // one CTA per SM, or one pair per two SMs; `units` tiles are in flight at once
+  const int cap = PAIR ? max_pairs(fn, C::kSmemBytes, nsm) : nsm;
+  const int units = kp.num_tiles < cap ? kp.num_tiles : cap;
+  const int grid = PAIR ? 2 * units : units;
+  // The grid works on `units` consecutive tiles at a time. Walk the dimension
   // that keeps fewer bytes of activation panels (256 tokens x K) and weight
-  // panels (128 rows x K, packed) live in L2 at once.
+  // panels (TILE_ROWS rows x K, packed) live in L2 at once.
   {
     const double x_panel = double(TILE_M) * pr.K * 2;
-    const double w_panel = double(TILE_N) * pr.K * BITS / 8;
+    const double w_panel = double(TILE_ROWS) * pr.K * BITS / 8;
     auto live = [&](int fast, double fast_panel, double slow_panel) {
-      const int f = fast < grid ? fast : grid;
-      return f * fast_panel + double((grid + fast - 1) / fast) * slow_panel;
+      const int f = fast < units ? fast : units;
+      return f * fast_panel + double((units + fast - 1) / fast) * slow_panel;
     };
     kp.m_fastest = live(kp.num_m_tiles, x_panel, w_panel) <= live(kp.num_n_tiles, w_panel, x_panel);
   }
   kp.bias = pr.bias;
   kp.residual = pr.residual;
   kp.gate = pr.gate;
-  CUtensorMap tm_res = tm_out;  // the residual update's L2 prefetch box: one tile
+  CUtensorMap tm_res = tm_out;  // the residual update's L2 prefetch box: this CTA's part of a tile
   if (EPI == QGEMM_EPI_RESIDUAL_GATE &&
       (st = make_tensor_map_2d(&tm_res, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pr.residual, pr.N, pr.M,
                                uint64_t(pr.N) * 2, TILE_N, TILE_M, CU_TENSOR_MAP_SWIZZLE_NONE, "residual")) != QGEMM_OK)
     return st;
   kp.wait_limit_ns = wait_limit_ns();
   kp.status = status;
-  large_m_kernel<BITS, EPI><<<grid, NUM_THREADS, C::kSmemBytes, pr.stream>>>(tm_x, tm_w, tm_s, tm_b, tm_out, tm_res,
-                                                                               kp);
-  return cuda_check(cudaGetLastError(), "large_m_kernel launch");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = pr.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = PAIR ? 1 : 0;
+  return cuda_check(cudaLaunchKernelEx(&cfg, large_m_kernel<BITS, EPI, PAIR>, tm_x, tm_w, tm_s, tm_b, tm_out, tm_res,
+                                       kp),
+                    "large_m_kernel launch");
 }
 
 }  // namespace lm
@@ -567,19 +718,26 @@ int launch_large_m(const Problem& p) {
   int nsm;
   int st = sm_count(&nsm);
   if (st != QGEMM_OK) return st;
-  auto go = [&](auto bits_tag) {
+  // the CTA-pair form where it pays (see large_pair_mode)
+  const int mode = large_pair_mode();
+  const bool pair = nsm >= 2 && (mode == 1 || (mode < 0 && p.bits == 8));
+  auto go = [&](auto bits_tag, auto pair_tag) {
     constexpr int B = decltype(bits_tag)::value;
+    constexpr bool P = decltype(pair_tag)::value;
     switch (p.epi) {
-      case QGEMM_EPI_GELU_TANH: return lm::launch_fmt<B, QGEMM_EPI_GELU_TANH>(p, nsm);
-      case QGEMM_EPI_RESIDUAL_GATE: return lm::launch_fmt<B, QGEMM_EPI_RESIDUAL_GATE>(p, nsm);
-      default: return lm::launch_fmt<B, QGEMM_EPI_NONE>(p, nsm);
+      case QGEMM_EPI_GELU_TANH: return lm::launch_fmt<B, QGEMM_EPI_GELU_TANH, P>(p, nsm);
+      case QGEMM_EPI_RESIDUAL_GATE: return lm::launch_fmt<B, QGEMM_EPI_RESIDUAL_GATE, P>(p, nsm);
+      default: return lm::launch_fmt<B, QGEMM_EPI_NONE, P>(p, nsm);
     }
   };
+  auto go_bits = [&](auto bits_tag) {
+    return pair ? go(bits_tag, std::true_type{}) : go(bits_tag, std::false_type{});
+  };
   switch (p.bits) {
-    case 4: return go(std::integral_constant<int, 4>{});
-    case 8: return go(std::integral_constant<int, 8>{});
-    case 1: return go(std::integral_constant<int, 1>{});
-    default: return go(std::integral_constant<int, 2>{});
+    case 4: return go_bits(std::integral_constant<int, 4>{});
+    case 8: return go_bits(std::integral_constant<int, 8>{});
+    case 1: return go_bits(std::integral_constant<int, 1>{});
+    default: return go_bits(std::integral_constant<int, 2>{});
   }
 }
 

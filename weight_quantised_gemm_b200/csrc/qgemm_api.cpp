@@ -18,6 +18,7 @@ thread_local std::string t_last_error;
 std::atomic<uint64_t> g_wait_limit_ns{0};  // 0 = not yet resolved; read by every launch, set by any thread
 std::once_flag g_env_once;
 int g_env_path = QGEMM_PATH_AUTO;
+int g_env_pair = -1;
 
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
 
@@ -25,6 +26,10 @@ void read_env() {
   if (const char* p = std::getenv("QGEMM_PATH")) {
     if (!std::strcmp(p, "small")) g_env_path = QGEMM_PATH_SMALL_M;
     else if (!std::strcmp(p, "large")) g_env_path = QGEMM_PATH_LARGE_M;
+  }
+  if (const char* pr = std::getenv("QGEMM_LARGE_PAIR")) {
+    if (!std::strcmp(pr, "0")) g_env_pair = 0;
+    else if (!std::strcmp(pr, "1")) g_env_pair = 1;
   }
   if (const char* w = std::getenv("QGEMM_WAIT_LIMIT_NS")) {
     const unsigned long long v = std::strtoull(w, nullptr, 10);
@@ -84,6 +89,11 @@ uint64_t wait_limit_ns() {
 // Whether the small-M path can take this shape at all: M <= 16, and 1-bit
 // rows streamed in pieces of at least 32 bytes (K % 256 == 0).
 bool small_path_takes(int M, int K, int bits) { return M <= 16 && !(bits == 1 && K % 256); }
+
+int large_pair_mode() {
+  std::call_once(g_env_once, read_env);
+  return g_env_pair;
+}
 
 int select_path(int M, int N, int K, int bits) {
   (void)N;

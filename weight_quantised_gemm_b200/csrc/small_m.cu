@@ -112,22 +112,8 @@ struct Params {
   unsigned int* status;
 };
 
-// Thread-block cluster helpers (K-split launches).
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// The shared-memory address `addr` of this CTA, as the same offset in CTA
-// `rank` of the cluster.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
+// Thread-block cluster helpers (K-split launches): a load from a peer CTA's
+// shared memory.
 __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
@@ -154,8 +140,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (sbase & 1023u) {  // the swizzled boxes need it; uniform across the block (and the cluster)
     if (threadIdx.x == 0) ptx::set_status(p.status, kStatusLayout);
     if (p.ksplit > 1) {  // the cluster's peers pass both of its barriers whatever happens here
-      cluster_sync();
-      cluster_sync();
+      ptx::cluster_sync();
+      ptx::cluster_sync();
     }
     return;
   }
@@ -163,7 +149,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int g = lane >> 2, c = lane & 3;
   // K-split launches: the CTAs of a cluster share one row block, CTA `kslice`
   // taking K stages [ks0, ks0 + ns) of it; the partial sums meet at the end.
-  const int kslice = p.ksplit > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int kslice = p.ksplit > 1 ? static_cast<int>(ptx::cluster_ctarank()) : 0;
   const int n0 = (blockIdx.x / p.ksplit) * R;
   const int ks0 = kslice * p.num_stages / p.ksplit;
   const int ns = (kslice + 1) * p.num_stages / p.ksplit - ks0;
@@ -437,7 +423,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int l = 0; l < GROUP_LANES; ++l) v += red[(l * MT + m) * NLP + nl];
     loc[i] = v;
   }
-  cluster_sync();
+  ptx::cluster_sync();
   if (!p.floor_only) {
     const uint32_t loc_addr = ptx::smem_u32(loc);
     for (int i = threadIdx.x + kslice * NUM_THREADS; i < p.M * R; i += p.ksplit * NUM_THREADS) {
@@ -445,7 +431,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int n = n0 + nl;
       if (n >= p.N) continue;
       float v = 0.f;
-      for (int r = 0; r < p.ksplit; ++r) v += ld_shared_cluster_f32(mapa_shared(loc_addr + 4u * i, r));
+      for (int r = 0; r < p.ksplit; ++r) v += ld_shared_cluster_f32(ptx::mapa_shared(loc_addr + 4u * i, r));
       if (p.bias) v += __bfloat162float(__ushort_as_bfloat16(p.bias[n]));
       const size_t o = static_cast<size_t>(m) * p.N + n;
       if (p.epi != QGEMM_EPI_NONE)
@@ -454,7 +440,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       p.out[o] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
     }
   }
-  cluster_sync();
+  ptx::cluster_sync();
 }
 
 // ---------------------------------------------------------------------------
