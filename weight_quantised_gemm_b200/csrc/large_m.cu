@@ -119,8 +119,8 @@ struct Cfg {
   static constexpr int kSBytes = kGroupsPerStage * TILE_N * 2;  // one stage's scales (or biases)
   static constexpr int kSBStride = BITS <= 2 ? kSBytes : 2 * kSBytes;
   static constexpr int kS = PAIR ? 4 : BITS == 8 ? 2 : 3;        // stage ring depth
-  static constexpr int kSW = BITS == 8 ? 3 : BITS == 4 ? 2 : BITS == 2 ? 4 : 8;  // W ring depth
-  static constexpr int kSlots = BITS == 8 ? 2 : 1;               // epilogue store slots per warp
+  static constexpr int kSW = BITS == 8 ? 3 : BITS == 4 ? (PAIR ? 4 : 2) : BITS == 2 ? 4 : 8;  // W ring depth
+  static constexpr int kSlots = PAIR || BITS == 8 ? 2 : 1;      // epilogue store slots per warp
   static constexpr int kOffX = 0;
   static constexpr int kOffW = kOffX + kS * kXStageBytes;
   static constexpr int kOffOut = kOffW + kSW * kWTileBytes;

@@ -38,10 +38,10 @@ void read_env() {
   }
 }
 
-// Largest M served by the small-M path, per format, from timing both paths at
-// M = 1..64 on B200 (the bench's path crossover sweep): below the crossover the
-// weights' bytes set the time and the register path streams them faster than
-// the tile pipeline fills.
+// Largest M served by the small-M path, per format and shape class, from
+// timing both paths at M = 1..64 on B200 (the bench's path crossover sweep):
+// below the crossover the weights' bytes set the time and the register path
+// streams them faster than the tile pipeline fills.
 #include "path_table.inc"
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -96,10 +96,10 @@ int large_pair_mode() {
 }
 
 int select_path(int M, int N, int K, int bits) {
-  (void)N;
   if (!small_path_takes(M, K, bits)) return QGEMM_PATH_LARGE_M;
-  const int lim = bits == 1 ? kSmallMaxBinary : bits == 2 ? kSmallMaxTernary : bits == 4 ? kSmallMax4 : kSmallMax8;
-  return M <= lim ? QGEMM_PATH_SMALL_M : QGEMM_PATH_LARGE_M;
+  for (const PathEntry& e : kPathTable)
+    if (e.bits == bits && N <= e.n_max && K <= e.k_max) return M <= e.small_max ? QGEMM_PATH_SMALL_M : QGEMM_PATH_LARGE_M;
+  return QGEMM_PATH_LARGE_M;
 }
 
 // The path of a QGEMM_PATH_AUTO call: the QGEMM_PATH variable's choice where
