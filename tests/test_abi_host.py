@@ -148,6 +148,12 @@ def test_select_path_table():
     for bits in (1, 2, 4, 8):
         assert wq.qgemm_select_path(1, 12288, 3072, bits) == wq.QGEMM_PATH_SMALL_M
         assert wq.qgemm_select_path(4096, 9216, 3072, bits) == wq.QGEMM_PATH_LARGE_M
+        # every (N, K) of the FLUX workloads: the measured table's choice at decode and prefill M
+        for N, K in ((12288, 3072), (9216, 3072), (18432, 3072), (3072, 3072), (3072, 12288)):
+            for M in (1, 4, 8, 16):
+                assert wq.qgemm_select_path(M, N, K, bits) == wq.QGEMM_PATH_SMALL_M, (bits, N, K, M)
+            for M in (17, 64, 4608):
+                assert wq.qgemm_select_path(M, N, K, bits) == wq.QGEMM_PATH_LARGE_M, (bits, N, K, M)
     with pytest.raises(wq.QGemmError):
         wq.qgemm_select_path(1, 16, 128, 3)
     with pytest.raises(wq.QGemmError) as e:

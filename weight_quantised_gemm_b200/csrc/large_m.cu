@@ -527,6 +527,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int rows_left = p.M - m0;  // tokens of this warp's half still inside X
       const int chunks = rows_left >= EPI_TOKENS ? EPI_TOKENS / EPI_ROWS
                                                  : (rows_left > 0 ? (rows_left + EPI_ROWS - 1) / EPI_ROWS : 0);
+      if constexpr (EPI == QGEMM_EPI_NONE) {
+        // Read this warp's share of the accumulator 16 tokens at a time, add
+        // the bias and round to bf16 pairs in registers, then hand the
+        // accumulator back to the MMA before any shared-memory or TMA store:
+        // the next tile's MMAs wait only for the tensor-memory reads. (The
+        // fused epilogues keep the per-chunk order below: their arithmetic
+        // and residual loads would not fit beside 64 held pairs.)
+        constexpr int LD = 16;        // tokens per tcgen05.ld
+        uint32_t pk[EPI_TOKENS / 2];  // tokens 2i and 2i + 1 as a bf16 pair
+#pragma unroll
+        for (int c = 0; c < EPI_TOKENS / LD; ++c) {
+          uint32_t v[LD];
+          if (c * LD < rows_left) {
+            ptx::tmem_ld_32x32b_x16(tmem_base + ACC_COL + t0 + c * LD + (static_cast<uint32_t>(32 * q) << 16), v);
+            ptx::tmem_wait_ld();
+          }
+#pragma unroll
+          for (int i = 0; i < LD / 2; ++i)
+            pk[c * (LD / 2) + i] = ptx::cvt_bf16x2(__uint_as_float(v[2 * i]) + bias_f,
+                                                   __uint_as_float(v[2 * i + 1]) + bias_f);
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) acc_empty_arrive();
+#pragma unroll
+        for (int c = 0; c < EPI_TOKENS / EPI_ROWS; ++c) {
+          if (c < chunks && nr + 32 * q < p.N) {
+            const uint32_t slot = nstore % C::kSlots;
+            // the TMA store that last used this slot has finished reading it
+            if (lane == 0) ptx::bulk_wait_group_read<C::kSlots - 1>();
+            __syncwarp();
+            uint16_t* sl = slots + slot * (EPI_SLOT_BYTES / 2);
+#pragma unroll
+            for (int t = 0; t < EPI_ROWS; ++t)
+              sl[t * 32 + lane] = static_cast<uint16_t>(pk[c * (EPI_ROWS / 2) + t / 2] >> (16 * (t & 1)));
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              // rows past M and columns past N fall outside the tensor map and are dropped
+              ptx::tma_store_2d(&tm_out, slots_u32 + slot * EPI_SLOT_BYTES, nr + 32 * q, m0 + c * EPI_ROWS);
+              ptx::bulk_commit_group();
+            }
+            ++nstore;
+          }
+        }
+        continue;
+      }
       for (int c = 0; c < EPI_TOKENS / EPI_ROWS; ++c) {
         uint32_t v[32];
         // the residual update's 32 residual values of this chunk, two tokens per
