@@ -628,6 +628,47 @@ def run_case(args):
             "note": "per-launch events include host launch gaps for short kernels; the graph timing does not"}
 
 
+def run_grouped_case(args):
+    """The mixed FLUX block's linears of one format at decode M as one grouped
+    launch, back to back with a CUDA event pair per launch (the form a
+    profiler captures). --grouped BITS:M, e.g. 8:1"""
+    import numpy as np
+    import torch
+
+    import weight_quantised_gemm_b200 as wq
+    import workloads as WL
+    bits, M = (int(v) for v in args.grouped.split(":"))
+    wl = WL.workload(4)
+    lins = [(li, l) for li, l in enumerate(wl.linears) if l.bits == bits]
+    if not lins:
+        raise SystemExit(f"the mixed block has no {bits}-bit linear")
+    ab = sum(alg_bytes(l, M) for _, l in lins)
+    ncopy = max(4, -(-3 * L2_BYTES // ab))
+    host = []
+    for li, l in lins:
+        X, W, _ = WL.make_inputs(l, 4, li, M=M)
+        host.append((l, X, wq.qgemm_pack(W, bits)))
+    sets = [[(torch.from_numpy(X.view(np.int16)).cuda().view(torch.bfloat16), pw.to_device("cuda"), None)
+             for l, X, pw in host] for _ in range(ncopy)]
+    outs = [torch.empty((M, l.N), dtype=torch.bfloat16, device="cuda") for l, _, _ in host]
+    for i in range(args.warmup):
+        wq.qgemm_grouped(sets[i % ncopy], outs=outs)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        ev[i][0].record()
+        wq.qgemm_grouped(sets[i % ncopy], outs=outs)
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    wq.check_device_status()
+    t = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e-3
+    tg = time_graph([(lambda s=s: wq.qgemm_grouped(s, outs=outs)) for s in sets] * max(1, 24 // ncopy))
+    wq.check_device_status()
+    return {"grouped": args.grouped, "linears": [l.name for l, _, _ in host], "alg_bytes": ab, "copies": ncopy,
+            "us_per_launch_events": round(t * 1e6, 2), "us_graph": round(tg * 1e6, 2),
+            "gbs_graph": round(ab / tg / 1e9, 1)}
+
+
 def run_e2e(sets, X_host_bits, lin, args, world):
     """Pipelined host->device->host: per step, copy X in from pinned memory,
     qgemm, copy out back to pinned memory, on three streams (PCIe in, compute,
@@ -1063,6 +1104,8 @@ def main(argv=None):
                     help="also time both kernel paths at M = 1..64 on every workload shape and format")
     ap.add_argument("--report", default=None,
                     help="also write the detailed report sections (JSON lines) to this file")
+    ap.add_argument("--grouped", default=None,
+                    help="time the mixed block's linears of one format as one grouped launch, BITS:M (e.g. 8:1)")
     ap.add_argument("--case", default=None,
                     help="time one workload linear alone, e.g. 3:tern_m1:M=16 (workload:linear[:M=..])")
     args = ap.parse_args(argv)
@@ -1082,6 +1125,9 @@ def main(argv=None):
     torch.cuda.set_device(local_rank)
     if args.case:
         print(json.dumps(run_case(args)), flush=True)
+        return 0
+    if args.grouped:
+        print(json.dumps(run_grouped_case(args)), flush=True)
         return 0
     if world > 1:
         import datetime

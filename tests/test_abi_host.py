@@ -304,3 +304,15 @@ def test_problem_struct_layout_matches_the_header(tmp_path):
     got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()]
     P = wq._Problem
     assert got == [ctypes.sizeof(P), P.M.offset, P.W.offset, P.out.offset, P.bias.offset]
+
+
+def test_debug_stream_rejects_bad_arguments_without_device():
+    d = _desc()
+    f = wq._lib.qgemm_debug_stream
+    assert f(0x10000, 17, ctypes.byref(d), 0, None) == wq.QGEMM_ERR_UNSUPPORTED       # small-M shapes only
+    assert f(0x10000, -1, ctypes.byref(d), 0, None) == wq.QGEMM_ERR_INVALID_ARG
+    assert f(0x10000, 4, ctypes.byref(d), 0x200, None) == wq.QGEMM_ERR_INVALID_ARG    # unknown flag
+    assert f(None, 4, ctypes.byref(d), 0, None) == wq.QGEMM_ERR_INVALID_ARG
+    assert f(0x10004, 4, ctypes.byref(d), 0, None) == wq.QGEMM_ERR_ALIGNMENT
+    assert f(0x10000, 4, None, 0, None) == wq.QGEMM_ERR_INVALID_ARG
+    assert f(0x10000, 0, ctypes.byref(d), 0, None) == wq.QGEMM_OK                    # M = 0: nothing to stream
