@@ -38,7 +38,7 @@ for bits in (1, 2, 4, 8):
         p, s, b = O.pack_ref(W, bits, group)
         close(y, O.qgemm_ref(X, p, s, b, bits, group, K, bias), f"bits={bits} M={M} N={N} K={K}")
     # one-hot tokens: the output is the dequantised weight, bit for bit
-    N, K, M = 520, 768, 300
+    N, K, M = 528, 768, 300
     g = np.random.default_rng(9 + bits)
     _, W, _ = WL.random_case(7 + bits, 1, N, K, bits, with_bias=False)
     ks = g.choice(K, size=M)

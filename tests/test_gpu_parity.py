@@ -408,10 +408,11 @@ def test_pack_device_matches_host_packer(bits):
         W = np.concatenate([WL.make_w(1, 0, 96, K, "normal"), _edge_rows(g, K)])
     if bits == 1:
         # groups at and next to fp16 ties of the exact mean, tails over many binades
-        tie = np.full((4, K), 2.0 ** -38)
-        tie[0, 0] = tie[1, 127] = tie[2, 300] = 1049088.0
-        tie[3, :128] = 0.0
-        tie[3, 5] = 1049088.0
+        tie = np.full((16, K), 2.0 ** -38)       # 16 rows: N stays a multiple of 16 for the GEMM below
+        for i in range(12):
+            tie[i, (37 * i) % K] = 1049088.0
+        tie[12:, :128] = 0.0
+        tie[12:, 5] = 1049088.0
         W = np.concatenate([W, tie.astype(np.float32)])
     host = wq.qgemm_pack(W, bits)
     dev = wq.qgemm_pack_device(torch.from_numpy(W).cuda(), bits)
