@@ -765,9 +765,12 @@ int launch_large_m(const Problem& p) {
   int nsm;
   int st = sm_count(&nsm);
   if (st != QGEMM_OK) return st;
-  // the CTA-pair form where it pays (see large_pair_mode)
+  // The CTA-pair form only when asked for (QGEMM_LARGE_PAIR=1): measured on
+  // B200 it is slower than one CTA per tile in every format (8-bit FLUX
+  // linears 22-31 % slower, 4-bit QKV 34 %), so the library's choice is the
+  // one-CTA form.
   const int mode = large_pair_mode();
-  const bool pair = nsm >= 2 && (mode == 1 || (mode < 0 && p.bits == 8));
+  const bool pair = nsm >= 2 && mode == 1;
   auto go = [&](auto bits_tag, auto pair_tag) {
     constexpr int B = decltype(bits_tag)::value;
     constexpr bool P = decltype(pair_tag)::value;

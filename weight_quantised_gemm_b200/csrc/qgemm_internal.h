@@ -35,8 +35,8 @@ int fail(int code, const char* fmt, ...);
 int cuda_check(cudaError_t e, const char* what);
 
 uint64_t wait_limit_ns();
-// The large-M kernel's CTA-pair form: -1 = the library's choice per format,
-// 0 = never, 1 = always (QGEMM_LARGE_PAIR=0|1, read once).
+// The large-M kernel's CTA-pair form: -1 = the library's choice (the
+// one-CTA form), 0 = never, 1 = always (QGEMM_LARGE_PAIR=0|1, read once).
 int large_pair_mode();
 // Device address of the current device's status word (cached per device).
 int status_word(unsigned int** ptr);

@@ -80,7 +80,6 @@ constexpr int MAX_STAGES = 8;
 constexpr int SMEM_LIMIT = 232448;      // the most a CTA may have
 constexpr int RING_BUDGET = 196608;     // bytes of shared memory for the ring
 constexpr int SMEM_FLOOR = 118784;      // at least this much, so that one grid's CTAs never share an SM
-constexpr int kXResMax = 49152;         // resident activations: at most this many bytes
 
 // Row halves for a CTA of NP pairs and MT tokens: 2 where one warp's
 // accumulators for all NP pairs would not fit in registers.
@@ -107,8 +106,6 @@ struct Params {
   int off_s, off_b;      // offsets of the scales and biases inside a stage
   int off_x, x_stride;   // activations in the ring (split-row CTAs): offset, token row stride in bytes
   int overlap;           // launched with programmatic dependent launch
-  int x_res;             // the CTA's K slice of X staged once in shared memory (else per stage from L2)
-  int off_xres, xres_pitch;  // where it sits and its token row stride in bytes
   int ksplit;            // K slices per row block: the CTAs of one thread-block cluster (1 = no cluster)
   int floor_only;        // stream the weights through the ring and compute nothing (the streaming floor)
   uint64_t wait_limit_ns;
@@ -162,7 +159,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (MAX_STAGES + s); };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + p.data_bytes + 16 * MAX_STAGES);
-  const uint32_t xbar = bar0 + 16u * MAX_STAGES + 8u;  // the resident activations have landed
   const uint64_t lim = p.wait_limit_ns;
   // Each CTA walks the K stages starting at its own offset: every CTA reads
   // the same activations, and rotating the order spreads those reads over
@@ -174,7 +170,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(full(s), 1);
       ptx::mbar_init(empty(s), NUM_CONSUMER_WARPS);
     }
-    ptx::mbar_init(xbar, 1);
     *abort_flag = 0;
     ptx::fence_mbarrier_init();
   }
@@ -220,36 +215,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         bulk_copy_g2s(st + p.off_x + m * p.x_stride, p.X + static_cast<size_t>(m) * p.K + kt * F::KS, valid * 2,
                       full(s));
     };
-    auto load_xres = [&]() {  // all lanes: the CTA's K slice of every token row, once
-      const int k_begin = ks0 * F::KS;
-      const int kend = (ks0 + ns) * F::KS < p.K ? (ks0 + ns) * F::KS : p.K;
-      const uint32_t bytes = static_cast<uint32_t>(kend - k_begin) * 2u;
-      if (lane == 0) ptx::mbar_arrive_expect_tx(xbar, p.M * bytes);
-      __syncwarp();  // the transaction count is raised before any copy can land
-      for (int m = lane; m < p.M; m += 32)
-        bulk_copy_g2s(sbase + p.off_xres + m * p.xres_pitch, p.X + static_cast<size_t>(m) * p.K + k_begin, bytes,
-                      xbar);
-    };
     if (lane == 0) {
       ptx::tma_prefetch_desc(&tm_w);
       ptx::tma_prefetch_desc(&tm_s);
       if (BITS > 2) ptx::tma_prefetch_desc(&tm_b);
     }
     if (!XR || p.overlap) {
-      // Resident activations, when nothing precedes this grid to wait for, go
-      // out first: they are small, and every stage needs them.
-      if (p.x_res && !p.overlap) load_xres();
       // The weights do not depend on the previous grid: the first stages go
       // out at once, and the next grid may launch (both no-ops without the
-      // launch attribute). Activations follow once that grid is done (the
-      // TMA unit takes copies in issue order, so they queue behind).
+      // launch attribute). Ring activations follow once that grid is done
+      // (the TMA unit takes copies in issue order, so they queue behind).
       if (lane == 0)
         for (int t = 0; t < pre; ++t) load_weights(t, t);
       griddep_launch_dependents();
-      if (p.x_res && p.overlap) {
-        griddep_wait();
-        load_xres();
-      }
       if constexpr (XR) {
         griddep_wait();
         __syncwarp();  // the transaction counts are raised before any activation copy can land
@@ -281,27 +259,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       const int first = t > p.ring ? t - p.ring : 0;
       for (int i = first; i < t; ++i) ptx::mbar_wait(full(i % p.ring), (i / p.ring) & 1, lim, nullptr);
-      if (p.x_res) ptx::mbar_wait(xbar, 0, lim, nullptr);
     }
   } else {
     // ---------------- consumers ----------------
     griddep_launch_dependents();
-    // the activations may be the previous grid's output: wait for it, or for
-    // the resident copy the producer makes once it is done
-    bool xok = true;
-    if constexpr (!XR) {
-      if (!p.x_res) griddep_wait();
-      else xok = warp_wait(xbar, 0, lim, abort_flag);
-      if (!xok && lane == 0) give_up();
-    }
-    const uint8_t* xres = smem + p.off_xres;  // resident activations: [token][k of the slice]
+    if constexpr (!XR) griddep_wait();  // the activations may be the previous grid's output
     const int ush = p.unit_shift;
     const int key16 = swizzle_key16(g, ush);
     const int gl = warp % GROUP_LANES;  // group lane: groups gl, gl + GROUP_LANES, ... of every stage
     const int q0 = (warp / GROUP_LANES) * NPH;  // first 16-row pair of this warp's half
     const bool ga = g < p.M, gb = MT > 8 && g + 8 < p.M;  // tokens g and g + 8 exist
     const bool compute = !p.floor_only;
-    for (int t = 0; xok && t < ns; ++t) {
+    for (int t = 0; t < ns; ++t) {
       const int s = t % p.ring;
       const int kt = ks0 + (t + rot) % ns;
       // The activations of this warp's groups (the B operand: tokens g and
@@ -312,7 +281,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int gi = 0; gi < (XR ? 0 : GPL); ++gi) {
         const int k0 = kt * F::KS + (gl + GROUP_LANES * gi) * F::G;
-        const bool in = compute && !p.x_res && k0 < p.K;
+        const bool in = compute && k0 < p.K;
         const uint2* x0p = reinterpret_cast<const uint2*>(p.X + static_cast<size_t>(g) * p.K + k0 + 4 * c);
         const uint2* x1p = reinterpret_cast<const uint2*>(p.X + static_cast<size_t>(g + 8) * p.K + k0 + 4 * c);
 #pragma unroll
@@ -349,10 +318,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint8_t* xg = st + p.off_x + g * p.x_stride + (gs * F::G + 16 * k + 4 * c) * 2;
             x0 = ga ? *reinterpret_cast<const uint2*>(xg) : make_uint2(0u, 0u);
             x1 = gb ? *reinterpret_cast<const uint2*>(xg + 8 * p.x_stride) : make_uint2(0u, 0u);
-          } else if (p.x_res) {
-            const uint8_t* xg = xres + g * p.xres_pitch + ((kt - ks0) * F::KS + gs * F::G + 16 * k + 4 * c) * 2;
-            x0 = ga ? *reinterpret_cast<const uint2*>(xg) : make_uint2(0u, 0u);
-            x1 = gb ? *reinterpret_cast<const uint2*>(xg + 8 * p.xres_pitch) : make_uint2(0u, 0u);
           } else {
             x0 = xr[gi][k][0];
             x1 = xr[gi][k][TH - 1];
@@ -516,27 +481,18 @@ int make_params(const Problem& pr, int ksplit, Params& kp, int& smem) {
   kp.off_x = (kp.off_b + (BITS <= 2 ? 0 : sb) + 127) & ~127;
   kp.x_stride = F::KS * 2 + 32;  // +32 B: token rows 8 banks apart, so the 8-byte B fetches do not collide
   kp.stage_bytes = (kp.off_x + (x_in_ring(MT, NP) ? pr.M * kp.x_stride : 0) + 1023) & ~1023;
-  // Activations staged once per CTA (its K slice of every token row) where
-  // they take little room, instead of a round trip to L2 in every stage.
-  // Rows 32 bytes longer than the slice: 8 banks apart, so the 8-byte B
-  // fetches of four tokens do not collide.
-  const int slice_k = slice_stages * F::KS < pr.K ? slice_stages * F::KS : pr.K;
-  kp.xres_pitch = slice_k * 2 + 32;
-  kp.x_res = !x_in_ring(MT, NP) && pr.M * kp.xres_pitch <= kXResMax ? 1 : 0;
-  const int xres_bytes = kp.x_res ? (pr.M * kp.xres_pitch + 1023) & ~1023 : 0;
-  int ring = (RING_BUDGET - xres_bytes) / kp.stage_bytes;
+  int ring = RING_BUDGET / kp.stage_bytes;
   ring = ring < MAX_STAGES ? ring : MAX_STAGES;
   ring = ring < slice_stages ? ring : slice_stages;
   kp.ring = ring < 1 ? 1 : ring;
   // the warps' partial sums (and, K-split, the CTA's own sums over them) reuse the ring at the end
   const int red_bytes = NUM_CONSUMER_WARPS / split_rows(MT, NP) * MT * (R + 4) * 4 + (ksplit > 1 ? MT * R * 4 : 0);
-  kp.off_xres = kp.ring * kp.stage_bytes;
-  kp.data_bytes = kp.off_xres + xres_bytes > red_bytes ? kp.off_xres + xres_bytes : red_bytes;
+  kp.data_bytes = kp.ring * kp.stage_bytes > red_bytes ? kp.ring * kp.stage_bytes : red_bytes;
   if (kp.data_bytes < SMEM_FLOOR) kp.data_bytes = SMEM_FLOOR;
   smem = kp.data_bytes + 16 * MAX_STAGES + 16;
   if (smem > SMEM_LIMIT) return fail(QGEMM_ERR_UNSUPPORTED, "small-M stage of %d bytes does not fit", kp.stage_bytes);
   if (kp.off_s % 1024 || kp.off_b % 128 || kp.off_x % 128 || kp.x_stride % 16 || kp.stage_bytes % 1024 ||
-      kp.data_bytes % 8 || kp.off_xres % 16 || kp.xres_pitch % 16)
+      kp.data_bytes % 8)
     return fail(QGEMM_ERR_UNSUPPORTED, "internal: small-M stage layout misaligned");
   kp.overlap = pr.overlap ? 1 : 0;
   kp.floor_only = pr.floor_only ? 1 : 0;

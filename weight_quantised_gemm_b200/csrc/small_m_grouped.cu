@@ -48,10 +48,6 @@ constexpr int R = 16 * NP;         // weight rows per item
 constexpr int MAX_STAGES = 24;     // ring slots: 32-row stages are small (5-18 KB)
 constexpr int SMEM_LIMIT = 232448;
 constexpr int CONSUMER_BAR = 1;    // named barrier of the consumer warps
-constexpr int XRES_MAX = 65536;    // resident activations: at most this many bytes
-// Resident activation rows are padded by 32 bytes: 8 banks apart, so the
-// 8-byte B fetches of four tokens do not collide.
-__host__ __device__ constexpr int xres_pitch(int K) { return K * 2 + 32; }
 
 struct GProblem {
   const uint16_t* X;     // bf16 [M, K]
@@ -60,7 +56,6 @@ struct GProblem {
   int M, N, K;
   int num_stages;        // ceil(K / KS)
   int unit_shift;        // log2 of U, the bytes per swizzled row piece
-  int xres_off;          // resident activations (GParams::x_res): offset of this problem's rows
 };
 
 struct GParams {
@@ -70,8 +65,6 @@ struct GParams {
   int off_s, off_b;      // scales and biases inside a stage
   int red_off;           // the consumers' reduction area
   int bar_off;           // mbarriers and the abort flag
-  int x_res;             // every problem's X staged once in shared memory (else per stage from L2)
-  int count;             // problems
   uint64_t wait_limit_ns;
   unsigned int* status;
   uint16_t cta_begin[kGroupedMaxCtas + 1];  // CTA c works on items[cta_begin[c] .. cta_begin[c + 1])
@@ -118,7 +111,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (MAX_STAGES + s); };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + p.bar_off + 16 * MAX_STAGES);
-  const uint32_t xbar = bar0 + 16u * MAX_STAGES + 8u;  // the resident activations have landed
   const uint64_t lim = p.wait_limit_ns;
   const int ib = p.cta_begin[blockIdx.x], ie = p.cta_begin[blockIdx.x + 1];
 
@@ -127,7 +119,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(full(s), 1);
       ptx::mbar_init(empty(s), NUM_CONSUMER_WARPS);
     }
-    ptx::mbar_init(xbar, 1);
     *abort_flag = 0;
     ptx::fence_mbarrier_init();
   }
@@ -142,20 +133,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // The weights do not depend on the previous grid: stream at once, and let
     // the next grid launch (both no-ops without the launch attribute).
     sm::griddep_launch_dependents();
-    if (p.x_res) {
-      // every problem's activations, once (after the previous grid, which may write them)
-      sm::griddep_wait();
-      uint32_t bytes = 0;
-      for (int i = 0; i < p.count; ++i) bytes += static_cast<uint32_t>(p.prob[i].M) * p.prob[i].K * 2u;
-      if (lane == 0) ptx::mbar_arrive_expect_tx(xbar, bytes);
-      __syncwarp();  // the transaction count is raised before any copy can land
-      for (int i = 0; i < p.count; ++i) {
-        const GProblem& P = p.prob[i];
-        for (int m = lane; m < P.M; m += 32)
-          sm::bulk_copy_g2s(sbase + P.xres_off + m * xres_pitch(P.K), P.X + static_cast<size_t>(m) * P.K,
-                            static_cast<uint32_t>(P.K) * 2u, xbar);
-      }
-    }
     if (lane == 0) {
       constexpr int sb_bytes = GS * R * 2;
       uint32_t gs = 0;  // stages issued so far, over all items
@@ -184,17 +161,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // let every copy issued above land before the block can exit
       const uint32_t first = gs > static_cast<uint32_t>(p.ring) ? gs - p.ring : 0;
       for (uint32_t i = first; i < gs; ++i) ptx::mbar_wait(full(i % p.ring), (i / p.ring) & 1, lim, nullptr);
-      if (p.x_res) ptx::mbar_wait(xbar, 0, lim, nullptr);
     }
   } else {
     // ---------------- consumers ----------------
     sm::griddep_launch_dependents();
-    // X may be the previous grid's output, and out may still be read by it:
-    // wait for that grid, or for the resident copy the producer makes after it
-    bool xok = true;
-    if (!p.x_res) sm::griddep_wait();
-    else xok = sm::warp_wait(xbar, 0, lim, abort_flag);
-    if (!xok && lane == 0) give_up();
+    sm::griddep_wait();  // X may be the previous grid's output, and out may still be read by it
     const int gl = warp;  // scale group gl of every stage
     float* red = reinterpret_cast<float*>(smem + p.red_off);  // [group lane][token][NLP]
     uint32_t gs = 0;
@@ -213,35 +184,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int h = 0; h < TH; ++h)
 #pragma unroll
           for (int j = 0; j < 4; ++j) acc[q][h][j] = 0.f;
-      bool ok = xok;
-      const uint8_t* xres = smem + P.xres_off;  // resident activations of this problem: [token][k]
-      const int pitch = xres_pitch(P.K);
-      for (int t = 0; ok && t < nst; ++t, ++gs) {
+      bool ok = true;
+      for (int t = 0; t < nst; ++t, ++gs) {
         const int s = gs % p.ring;
         const int kt = (t + rot) % nst;
         const int k0 = kt * F::KS + gl * F::G;
         const bool in = k0 < P.K;
-        // the B fragments (tokens g and g + 8): resident in shared memory, or
-        // straight from global memory, issued before the wait so that the two
-        // latencies overlap
+        // the B fragments (tokens g and g + 8) straight from global memory,
+        // issued before the wait so that the two latencies overlap
         uint2 xr[STEPS][TH];
-        if (p.x_res) {
-          const uint8_t* x0s = xres + g * pitch + (k0 + 4 * c) * 2;
+        const uint2* x0p = reinterpret_cast<const uint2*>(P.X + static_cast<size_t>(g) * P.K + k0 + 4 * c);
+        const uint2* x1p = reinterpret_cast<const uint2*>(P.X + static_cast<size_t>(g + 8) * P.K + k0 + 4 * c);
 #pragma unroll
-          for (int k = 0; k < STEPS; ++k) {
-            xr[k][0] = (in && ga) ? *reinterpret_cast<const uint2*>(x0s + 32 * k) : make_uint2(0u, 0u);
-            if constexpr (TH > 1)
-              xr[k][TH - 1] = (in && gb) ? *reinterpret_cast<const uint2*>(x0s + 8 * pitch + 32 * k)
-                                         : make_uint2(0u, 0u);
-          }
-        } else {
-          const uint2* x0p = reinterpret_cast<const uint2*>(P.X + static_cast<size_t>(g) * P.K + k0 + 4 * c);
-          const uint2* x1p = reinterpret_cast<const uint2*>(P.X + static_cast<size_t>(g + 8) * P.K + k0 + 4 * c);
-#pragma unroll
-          for (int k = 0; k < STEPS; ++k) {
-            xr[k][0] = (in && ga) ? __ldg(x0p + 4 * k) : make_uint2(0u, 0u);
-            if constexpr (TH > 1) xr[k][TH - 1] = (in && gb) ? __ldg(x1p + 4 * k) : make_uint2(0u, 0u);
-          }
+        for (int k = 0; k < STEPS; ++k) {
+          xr[k][0] = (in && ga) ? __ldg(x0p + 4 * k) : make_uint2(0u, 0u);
+          if constexpr (TH > 1) xr[k][TH - 1] = (in && gb) ? __ldg(x1p + 4 * k) : make_uint2(0u, 0u);
         }
         if (!sm::warp_wait(full(s), (gs / p.ring) & 1, lim, abort_flag)) {
           if (lane == 0) give_up();
@@ -395,27 +352,15 @@ int launch(const Problem* probs, int count, bool overlap, cudaStream_t stream, i
   kp.off_b = (kp.off_s + sb + 127) & ~127;
   kp.stage_bytes = (kp.off_b + (BITS <= 2 ? 0 : sb) + 1023) & ~1023;
   const int red_bytes = NUM_CONSUMER_WARPS * MT * (R + 4) * 4;
-  // every problem's activations resident in shared memory when they take little room
-  int xres_bytes = 0;
-  for (int i = 0; i < count; ++i) xres_bytes += probs[i].M * xres_pitch(probs[i].K);
-  kp.x_res = xres_bytes <= XRES_MAX ? 1 : 0;
-  if (!kp.x_res) xres_bytes = 0;
-  const int tail = xres_bytes + red_bytes + 16 * MAX_STAGES + 16;
+  const int tail = red_bytes + 16 * MAX_STAGES + 16;
   int ring = (SMEM_LIMIT - tail) / kp.stage_bytes;
   ring = ring < MAX_STAGES ? ring : MAX_STAGES;
   if (ring < 2) return fail(QGEMM_ERR_UNSUPPORTED, "internal: grouped stage of %d bytes", kp.stage_bytes);
   kp.ring = ring;
-  int xoff = ring * kp.stage_bytes;
-  for (int i = 0; i < count; ++i) {
-    kp.prob[i].xres_off = xoff;
-    if (kp.x_res) xoff += probs[i].M * xres_pitch(probs[i].K);
-  }
-  kp.red_off = (xoff + 15) & ~15;
+  kp.red_off = ring * kp.stage_bytes;
   kp.bar_off = (kp.red_off + red_bytes + 7) & ~7;
-  kp.count = count;
   const int smem = kp.bar_off + 16 * MAX_STAGES + 16;
-  if (smem > SMEM_LIMIT || kp.off_s % 1024 || kp.off_b % 128 || kp.stage_bytes % 1024 || kp.red_off % 16 ||
-      kp.prob[0].xres_off % 16)
+  if (smem > SMEM_LIMIT || kp.off_s % 1024 || kp.off_b % 128 || kp.stage_bytes % 1024 || kp.red_off % 16)
     return fail(QGEMM_ERR_UNSUPPORTED, "internal: grouped small-M layout");
   kp.wait_limit_ns = wait_limit_ns();
   if ((st = status_word(&kp.status)) != QGEMM_OK) return st;
