@@ -126,7 +126,7 @@ struct Cfg {
   static constexpr int kOffOut = kOffW + kSW * kWTileBytes;
   static constexpr int kOffSB = kOffOut + NUM_EPI_WARPS * kSlots * EPI_SLOT_BYTES;
   static constexpr int kOffBar = kOffSB + kSW * kSBStride;
-  static constexpr int kNumBars = 3 * kS + 2 * kSW + 3;  // full, empty, X landed (pair), W ring, accumulator
+  static constexpr int kNumBars = 2 * kS + 2 * kSW + 3;  // stage full / empty, W ring full / empty, accumulator
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -217,22 +217,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t acc_full = bar0 + 8u * (2 * S + 2 * SW);
   const uint32_t acc_empty = acc_full + 8u;
   const uint32_t drain_bar = acc_full + 16u;
-  auto xfull = [&](int s) { return bar0 + 8u * (2 * S + 2 * SW + 3 + s); };  // pair: this CTA's X landed
-  // where this CTA's arrivals for a stage and for the accumulator go: the
-  // even CTA's barriers (a shared::cluster address; the CTA's own one alone)
-  auto full_arrive = [&](int s) {
-    if constexpr (PAIR) ptx::mbar_arrive_remote(ptx::mapa_shared(full(s), 0));
-    else ptx::mbar_arrive(full(s));
-  };
+  // where this CTA's epilogue warps report the accumulator drained: the even
+  // CTA's barrier (a shared::cluster address; the CTA's own one alone)
   auto acc_empty_arrive = [&]() {
     if constexpr (PAIR) ptx::mbar_arrive_remote(ptx::mapa_shared(acc_empty, 0));
     else ptx::mbar_arrive(acc_empty);
   };
-  // waits on barriers the other CTA of a pair (or its commits) may complete
-  auto wait_x = [&](uint32_t bar, uint32_t par) {
-    if constexpr (PAIR) return ptx::mbar_wait_cluster(bar, par, p.wait_limit_ns, nullptr);
-    else return ptx::mbar_wait(bar, par, p.wait_limit_ns, nullptr);
-  };
+
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   volatile int* epi_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
@@ -240,10 +231,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       // the X producer's arrival + one per dequantiser; a pair's even CTA also
-      // counts the odd one's dequantisers and its relayed X arrival
-      ptx::mbar_init(full(s), PAIR ? 2 + 2 * NUM_DEQ_WARPS : 1 + NUM_DEQ_WARPS);
+      // counts the odd CTA's one relayed arrival for the same stage
+      ptx::mbar_init(full(s), PAIR && rank == 0 ? 2 + NUM_DEQ_WARPS : 1 + NUM_DEQ_WARPS);
       ptx::mbar_init(empty(s), 1);
-      ptx::mbar_init(xfull(s), 1);
     }
     for (int s = 0; s < SW; ++s) {
       ptx::mbar_init(full_w(s), 1);
@@ -301,20 +291,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
           const int s = it % R;
           const uint32_t par = ((it / R) & 1) ^ 1;
-          const bool waited = is_x && PAIR ? ptx::mbar_wait_cluster(empty(s), par, lim, abort_flag)
-                                           : ptx::mbar_wait(is_x ? empty(s) : empty_w(s), par, lim, abort_flag);
-          if (!waited) {
+          if (!ptx::mbar_wait(is_x ? empty(s) : empty_w(s), par, lim, abort_flag)) {
             give_up();
             ok = false;
             break;
           }
           if (is_x) {
-            // the odd CTA of a pair counts its bytes on its own barrier; the MMA
-            // warp there relays the stage to the even CTA once they land
-            const uint32_t xb = PAIR && rank ? xfull(s) : full(s);
-            ptx::mbar_arrive_expect_tx(xb, C::kXStageBytes);
-            ptx::tma_load_2d(x_stage(s), &tm_x, kb * BK, m_tile * TILE_M + tok0, xb);
-            ptx::tma_load_2d(x_stage(s) + C::kXBoxBytes, &tm_x, kb * BK + BOX_K, m_tile * TILE_M + tok0, xb);
+            ptx::mbar_arrive_expect_tx(full(s), C::kXStageBytes);
+            ptx::tma_load_2d(x_stage(s), &tm_x, kb * BK, m_tile * TILE_M + tok0, full(s));
+            ptx::tma_load_2d(x_stage(s) + C::kXBoxBytes, &tm_x, kb * BK + BOX_K, m_tile * TILE_M + tok0, full(s));
           } else {
             const uint32_t wdst = sbase + C::kOffW + s * C::kWTileBytes;
             const uint32_t sdst = sbase + C::kOffSB + s * C::kSBStride;
@@ -333,31 +318,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t first = it > static_cast<uint32_t>(R) ? it - R : 0;
       for (uint32_t i = first; i < it; ++i) {
         if (is_x)
-          wait_x(empty(i % R), (i / R) & 1);
+          ptx::mbar_wait(empty(i % R), (i / R) & 1, lim, nullptr);
         else
           ptx::mbar_wait(full_w(i % R), (i / R) & 1, lim, nullptr);
       }
     }
   } else if (warp == WARP_MMA && PAIR && rank != 0) {
     // ---------------- the odd CTA of a pair: relay ----------------
-    // Its X stages land on its own barrier; once one has, tell the even CTA,
-    // whose MMA reads this CTA's half of the B operand.
+    // A stage is complete here when this CTA's activation bytes have landed
+    // and its dequantisers have written their A rows; then one arrival (one
+    // cluster-scope release) tells the even CTA, whose MMA reads both.
     uint32_t it = 0;
     bool ok = true;
     for (int tile = unit; ok && tile < p.num_tiles; tile += units)
       for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
         const int s = it % S;
-        if (!warp_wait(xfull(s), (it / S) & 1, lim, abort_flag)) {
+        if (!warp_wait(full(s), (it / S) & 1, lim, abort_flag)) {
           if (lane == 0) give_up();
           ok = false;
           break;
         }
-        if (lane == 0) full_arrive(s);
+        if (lane == 0) ptx::mbar_arrive_remote(ptx::mapa_shared(full(s), 0));
         __syncwarp();
       }
     // the even CTA's last commit says every MMA of the pair is done: only
     // then may this CTA's tensor memory be freed
-    if (lane == 0) ptx::mbar_wait_cluster(drain_bar, 0, lim, nullptr);
+    if (lane == 0) ptx::mbar_wait(drain_bar, 0, lim, nullptr);
     __syncwarp();
   } else if (warp == WARP_MMA) {
     // ---------------- MMA issuer ----------------
@@ -428,8 +414,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (uint32_t it = 0; it < total; ++it) {
       const int s = it % S, sw = it % SW;
       if (!warp_wait(full_w(sw), (it / SW) & 1, lim, abort_flag) ||
-          !(PAIR ? warp_wait_cluster(empty(s), ((it / S) & 1) ^ 1, lim, abort_flag)
-                 : warp_wait(empty(s), ((it / S) & 1) ^ 1, lim, abort_flag))) {
+          !warp_wait(empty(s), ((it / S) & 1) ^ 1, lim, abort_flag)) {
         if (lane == 0) give_up();
         break;
       }
@@ -490,7 +475,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) full_arrive(s);
+      if (lane == 0) ptx::mbar_arrive(full(s));
     }
   } else {
     // ---------------- epilogue ----------------
@@ -515,8 +500,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // while the tile's MMAs run, bring its residual block into L2
         if (e == 0 && lane == 0) ptx::tma_prefetch_l2_2d(&tm_res, nr, m_tile * TILE_M);
       }
-      const bool got = PAIR ? warp_wait_cluster(acc_full, tcount & 1, lim, abort_flag)
-                            : warp_wait(acc_full, tcount & 1, lim, abort_flag);
+      const bool got = warp_wait(acc_full, tcount & 1, lim, abort_flag);
       if (!got && lane == 0) {
         *epi_abort = 1;
         give_up();
