@@ -13,19 +13,20 @@
 //   rows (viewed as [row][unit][U bytes], U = 128, 64 or 32, the box lands as
 //   [unit][row][U bytes] with the U-byte swizzle, so the per-lane row reads
 //   are free of bank conflicts) and one 2-D box each for the stage's fp16
-//   scales and biases. The activations do not pass through the ring: the
-//   consumer warps load their B fragments straight from global memory
-//   (every CTA reads the same rows, so they come from L2), before waiting
-//   for the stage's weights, so the two latencies overlap. (Staging a CTA's
-//   activations in shared memory once, or bulk-copying them into every
-//   stage, was measured slower: the per-stage loads are hidden behind the
-//   weight stream.)
-// * Sixteen consumer warps, two row halves of eight: warp w takes scale
-//   group w % 8 of every stage for the 16-row pairs of half w / 8. At
-//   decode M the consumers' decode and mma.sync issue, not the memory
-//   system, set the time above the streaming floor, and with eight consumer
-//   warps (nine per SM) 61 % of the issue slots were idle with no single
-//   stall reason dominant: twice the warps hide twice the latency.
+//   scales and biases. The activations normally do not pass through the
+//   ring: the consumer warps load their B fragments straight from global
+//   memory (every CTA reads the same rows, so they come from L2), before
+//   waiting for the stage's weights. A TMA copy costs the SM's copy unit on
+//   the order of a hundred cycles whatever its size; one per token row per
+//   stage made M = 16 pay for 48 (ternary) to 384 (8-bit, K = 12288) of them.
+//   Split-row CTAs (below) are the exception: a warp there takes two groups
+//   per stage, and holding both groups' fragments across the wait spills
+//   registers, so the producer bulk-copies their activation rows into the
+//   stage.
+// * Eight consumer warps. Normally warp w takes scale group w of every stage
+//   for all the CTA's rows; where that would not fit in registers (16 tokens
+//   and 6 or more 16-row pairs) the rows split into two halves and warps w and
+//   w + 4 take groups w % 4 and w % 4 + 4 of every stage, each for its half.
 //   A warp turns codes into bf16 in registers and feeds warp-level mma.sync
 //   (m16n8k16, bf16 in, fp32 accumulate): the weights are the 16-row A
 //   operand, the activations the 8-column B (tokens past M are zero). At the
@@ -34,9 +35,10 @@
 //   writes bf16.
 // * Overlap (programmatic dependent launch, when the caller asks for it): the
 //   producer puts the first stages' weight, scale and bias loads in flight and
-//   lets the next grid in the stream launch; the consumers wait for the
-//   previous grid to finish before they read the activations, and every
-//   thread waits for it before it reads the bias or writes the output. A
+//   lets the next grid in the stream launch; whoever reads the activations
+//   (the consumers, or for split-row CTAs the producer's copies) waits for
+//   the previous grid to finish first, and every thread waits for it before
+//   it reads the bias or writes the output. A
 //   CTA of the next launch then takes an SM the moment this grid's CTA there
 //   exits, and its weight stream overlaps the other SMs' last stages instead
 //   of waiting for the whole grid and a fresh launch. Without the launch
@@ -71,15 +73,22 @@
 namespace qg {
 namespace sm {
 
-constexpr int NUM_CONSUMER_WARPS = 16;
-constexpr int GROUP_LANES = 8;           // warps per row half: warp w takes scale group w % 8 of every stage
-constexpr int PH = NUM_CONSUMER_WARPS / GROUP_LANES;  // row halves
+constexpr int NUM_CONSUMER_WARPS = 8;
 constexpr int WARP_PRODUCER = NUM_CONSUMER_WARPS;
 constexpr int NUM_THREADS = 32 * (NUM_CONSUMER_WARPS + 1);  // 288
 constexpr int MAX_STAGES = 8;
 constexpr int SMEM_LIMIT = 232448;      // the most a CTA may have
 constexpr int RING_BUDGET = 196608;     // bytes of shared memory for the ring
 constexpr int SMEM_FLOOR = 118784;      // at least this much, so that one grid's CTAs never share an SM
+
+// Row halves for a CTA of NP pairs and MT tokens: 2 where one warp's
+// accumulators for all NP pairs would not fit in registers.
+__host__ __device__ constexpr int split_rows(int MT, int NP) { return MT > 8 && NP >= 6 ? 2 : 1; }
+// Split-row CTAs give each warp two groups per stage; holding both groups'
+// activation fragments in registers across the stage wait spills, so their
+// activations come through the ring (one bulk copy per token row) instead of
+// straight from global memory.
+__host__ __device__ constexpr bool x_in_ring(int MT, int NP) { return split_rows(MT, NP) == 2; }
 
 struct Params {
   const uint16_t* X;     // bf16 [M, K]
@@ -95,6 +104,7 @@ struct Params {
   int stage_bytes;       // bytes per ring stage (multiple of 1024)
   int data_bytes;        // ring (or the partial sums, if larger); the mbarriers follow
   int off_s, off_b;      // offsets of the scales and biases inside a stage
+  int off_x, x_stride;   // activations in the ring (split-row CTAs): offset, token row stride in bytes
   int overlap;           // launched with programmatic dependent launch
   int ksplit;            // K slices per row block: the CTAs of one thread-block cluster (1 = no cluster)
   int floor_only;        // stream the weights through the ring and compute nothing (the streaming floor)
@@ -117,10 +127,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   using F = Fmt<BITS>;
   constexpr int STEPS = F::STEPS;
   constexpr int R = 16 * NP;                 // weight rows of the CTA
+  constexpr int PH = split_rows(MT, NP);     // row halves (1 or 2)
+  constexpr int GROUP_LANES = NUM_CONSUMER_WARPS / PH;  // warps w and w + GROUP_LANES share a group lane
   constexpr int NPH = NP / PH;               // 16-row pairs per warp
   constexpr int GPL = GS / GROUP_LANES;      // groups per warp and stage
   constexpr int TH = MT > 8 ? 2 : 1;         // 8-token halves
   constexpr int NLP = R + 4;                 // row pitch of the partial sums: 2 * NLP = 8 (mod 32) banks
+  constexpr bool XR = x_in_ring(MT, NP);     // activations through the ring, else from global memory
   static_assert(NP % PH == 0, "the halves take whole 16-row pairs");
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = ptx::smem_u32(smem);
@@ -189,21 +202,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int kt, valid;
       stage_k(t, kt, valid);
       const uint32_t st = sbase + s * p.stage_bytes;
-      ptx::mbar_arrive_expect_tx(full(s), R * F::ROWB + sb_bytes * (BITS <= 2 ? 1 : 2));
+      ptx::mbar_arrive_expect_tx(full(s), R * F::ROWB + sb_bytes * (BITS <= 2 ? 1 : 2) + (XR ? p.M * valid * 2 : 0));
       ptx::tma_load_3d(st, &tm_w, 0, n0, kt * units, full(s));
       ptx::tma_load_2d(st + p.off_s, &tm_s, n0, kt * GS, full(s));
       if (BITS > 2) ptx::tma_load_2d(st + p.off_b, &tm_b, n0, kt * GS, full(s));
+    };
+    auto load_x = [&](int t, int s) {  // all lanes: one bulk copy per token row
+      int kt, valid;
+      stage_k(t, kt, valid);
+      const uint32_t st = sbase + s * p.stage_bytes;
+      for (int m = lane; m < p.M; m += 32)
+        bulk_copy_g2s(st + p.off_x + m * p.x_stride, p.X + static_cast<size_t>(m) * p.K + kt * F::KS, valid * 2,
+                      full(s));
     };
     if (lane == 0) {
       ptx::tma_prefetch_desc(&tm_w);
       ptx::tma_prefetch_desc(&tm_s);
       if (BITS > 2) ptx::tma_prefetch_desc(&tm_b);
     }
-    // The weights do not depend on the previous grid: the first stages go out
-    // at once, and the next grid may launch (no-op without the attribute).
-    if (lane == 0)
-      for (int t = 0; t < pre; ++t) load_weights(t, t);
-    griddep_launch_dependents();
+    if (!XR || p.overlap) {
+      // The weights do not depend on the previous grid: the first stages go
+      // out at once, and the next grid may launch (both no-ops without the
+      // launch attribute). Ring activations follow once that grid is done
+      // (the TMA unit takes copies in issue order, so they queue behind).
+      if (lane == 0)
+        for (int t = 0; t < pre; ++t) load_weights(t, t);
+      griddep_launch_dependents();
+      if constexpr (XR) {
+        griddep_wait();
+        __syncwarp();  // the transaction counts are raised before any activation copy can land
+        for (int t = 0; t < pre; ++t) load_x(t, t);
+      }
+    } else {
+      // Nothing to wait for: each stage's activations right behind its
+      // weights, so that the first stage is complete as early as possible.
+      for (int t = 0; t < pre; ++t) {
+        if (lane == 0) load_weights(t, t);
+        __syncwarp();
+        load_x(t, t);
+      }
+    }
     int t = pre;
     for (; t < ns; ++t) {
       const int s = t % p.ring;
@@ -212,6 +250,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       if (lane == 0) load_weights(t, s);
+      if constexpr (XR) {
+        __syncwarp();
+        load_x(t, s);
+      }
     }
     // Let every copy issued above land before the block can exit.
     if (lane == 0) {
@@ -221,7 +263,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ---------------- consumers ----------------
     griddep_launch_dependents();
-    griddep_wait();  // the activations may be the previous grid's output
+    if constexpr (!XR) griddep_wait();  // the activations may be the previous grid's output
     const int ush = p.unit_shift;
     const int key16 = swizzle_key16(g, ush);
     const int gl = warp % GROUP_LANES;  // group lane: groups gl, gl + GROUP_LANES, ... of every stage
@@ -235,9 +277,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // g + 8, k = gs*G + 16*step + 4c .. +3) straight from global memory,
       // where every CTA reads the same rows (L2 hits); issued before the
       // stage's weights are waited for, so the two latencies overlap.
-      uint2 xr[GPL][STEPS][TH];
+      uint2 xr[XR ? 1 : GPL][STEPS][TH];
 #pragma unroll
-      for (int gi = 0; gi < GPL; ++gi) {
+      for (int gi = 0; gi < (XR ? 0 : GPL); ++gi) {
         const int k0 = kt * F::KS + (gl + GROUP_LANES * gi) * F::G;
         const bool in = compute && k0 < p.K;
         const uint2* x0p = reinterpret_cast<const uint2*>(p.X + static_cast<size_t>(g) * p.K + k0 + 4 * c);
@@ -271,7 +313,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int j = 0; j < 4; ++j) tmp[q][h][j] = 0.f;
 #pragma unroll
         for (int k = 0; k < STEPS; ++k) {
-          const uint2 x0 = xr[gi][k][0], x1 = xr[gi][k][TH - 1];
+          uint2 x0, x1;
+          if constexpr (XR) {
+            const uint8_t* xg = st + p.off_x + g * p.x_stride + (gs * F::G + 16 * k + 4 * c) * 2;
+            x0 = ga ? *reinterpret_cast<const uint2*>(xg) : make_uint2(0u, 0u);
+            x1 = gb ? *reinterpret_cast<const uint2*>(xg + 8 * p.x_stride) : make_uint2(0u, 0u);
+          } else {
+            x0 = xr[gi][k][0];
+            x1 = xr[gi][k][TH - 1];
+          }
           if constexpr (BITS > 2) {
             const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};
             mma_bf16_16816(xs[0], ones, x0.x, x0.y);
@@ -428,18 +478,20 @@ int make_params(const Problem& pr, int ksplit, Params& kp, int& smem) {
   // 1024-byte one, for its swizzle); bulk copies need 16 bytes.
   kp.off_s = R * F::ROWB;
   kp.off_b = (kp.off_s + sb + 127) & ~127;
-  kp.stage_bytes = (kp.off_b + (BITS <= 2 ? 0 : sb) + 1023) & ~1023;
+  kp.off_x = (kp.off_b + (BITS <= 2 ? 0 : sb) + 127) & ~127;
+  kp.x_stride = F::KS * 2 + 32;  // +32 B: token rows 8 banks apart, so the 8-byte B fetches do not collide
+  kp.stage_bytes = (kp.off_x + (x_in_ring(MT, NP) ? pr.M * kp.x_stride : 0) + 1023) & ~1023;
   int ring = RING_BUDGET / kp.stage_bytes;
   ring = ring < MAX_STAGES ? ring : MAX_STAGES;
   ring = ring < slice_stages ? ring : slice_stages;
   kp.ring = ring < 1 ? 1 : ring;
   // the warps' partial sums (and, K-split, the CTA's own sums over them) reuse the ring at the end
-  const int red_bytes = GROUP_LANES * MT * (R + 4) * 4 + (ksplit > 1 ? MT * R * 4 : 0);
+  const int red_bytes = NUM_CONSUMER_WARPS / split_rows(MT, NP) * MT * (R + 4) * 4 + (ksplit > 1 ? MT * R * 4 : 0);
   kp.data_bytes = kp.ring * kp.stage_bytes > red_bytes ? kp.ring * kp.stage_bytes : red_bytes;
   if (kp.data_bytes < SMEM_FLOOR) kp.data_bytes = SMEM_FLOOR;
   smem = kp.data_bytes + 16 * MAX_STAGES + 16;
   if (smem > SMEM_LIMIT) return fail(QGEMM_ERR_UNSUPPORTED, "small-M stage of %d bytes does not fit", kp.stage_bytes);
-  if (kp.off_s % 1024 || kp.off_b % 128 || kp.stage_bytes % 1024 ||
+  if (kp.off_s % 1024 || kp.off_b % 128 || kp.off_x % 128 || kp.x_stride % 16 || kp.stage_bytes % 1024 ||
       kp.data_bytes % 8)
     return fail(QGEMM_ERR_UNSUPPORTED, "internal: small-M stage layout misaligned");
   kp.overlap = pr.overlap ? 1 : 0;

@@ -15,10 +15,9 @@
 // problem. The host assigns items to CTAs longest first, each to the least
 // loaded CTA (load = the item's K stages), and passes each CTA its list. One
 // CTA per SM; a producer warp streams every item's stages through one
-// shared-memory ring without a break between items, and sixteen consumer
-// warps (warp w: scale group w % 8 of every stage for 16-row pair w / 8 of
-// the item) turn codes into bf16 and feed mma.sync as in the one-problem
-// kernel. At the end of an item the
+// shared-memory ring without a break between items, and eight consumer
+// warps (warp w: scale group w of every stage) turn codes into bf16 and feed
+// mma.sync as in the one-problem kernel. At the end of an item the
 // consumers' partial sums meet in a reduction area of their own (the ring
 // keeps filling meanwhile), and they write the item's outputs with the bias.
 
@@ -40,12 +39,11 @@ namespace smg {
 using sm::Fmt;
 using sm::GS;
 
-constexpr int NUM_CONSUMER_WARPS = 16;   // two row halves x eight scale-group lanes
-constexpr int GROUP_LANES = 8;
+constexpr int NUM_CONSUMER_WARPS = 8;
 constexpr int WARP_PRODUCER = NUM_CONSUMER_WARPS;
 constexpr int NUM_THREADS = 32 * (NUM_CONSUMER_WARPS + 1);
 constexpr int CONSUMER_THREADS = 32 * NUM_CONSUMER_WARPS;
-constexpr int NP = 2;              // 16-row pairs per item: one per row half
+constexpr int NP = 2;              // 16-row pairs per item
 constexpr int R = 16 * NP;         // weight rows per item
 constexpr int MAX_STAGES = 24;     // ring slots: 32-row stages are small (5-18 KB)
 constexpr int SMEM_LIMIT = 232448;
@@ -168,8 +166,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ---------------- consumers ----------------
     sm::griddep_launch_dependents();
     sm::griddep_wait();  // X may be the previous grid's output, and out may still be read by it
-    const int gl = warp % GROUP_LANES;  // scale group gl of every stage
-    const int qh = warp / GROUP_LANES;  // the item's 16-row pair this warp takes
+    const int gl = warp;  // scale group gl of every stage
     float* red = reinterpret_cast<float*>(smem + p.red_off);  // [group lane][token][NLP]
     uint32_t gs = 0;
     for (int it = ib; it < ie; ++it) {
@@ -179,12 +176,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int ush = P.unit_shift;
       const int key16 = sm::swizzle_key16(g, ush);
       const bool ga = g < P.M, gb = MT > 8 && g + 8 < P.M;  // tokens g and g + 8 exist
-      // acc[h][j]: weight rows 16 qh + g (j < 2) and 16 qh + g + 8 (j >= 2), tokens 8h + 2c + (j & 1)
-      float acc[TH][4];
+      // acc[q][h][j]: weight rows 16q + g (j < 2) and 16q + g + 8 (j >= 2), tokens 8h + 2c + (j & 1)
+      float acc[NP][TH][4];
 #pragma unroll
-      for (int h = 0; h < TH; ++h)
+      for (int q = 0; q < NP; ++q)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[h][j] = 0.f;
+        for (int h = 0; h < TH; ++h)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[q][h][j] = 0.f;
       bool ok = true;
       for (int t = 0; t < nst; ++t, ++gs) {
         const int s = gs % p.ring;
@@ -209,11 +208,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint8_t* st = smem + s * p.stage_bytes;
         if (in) {
           float xs[TH][4];  // sum of x over the group per token (affine)
-          float tmp[TH][4];
+          float tmp[NP][TH][4];
 #pragma unroll
           for (int h = 0; h < TH; ++h)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) xs[h][j] = tmp[h][j] = 0.f;
+            for (int j = 0; j < 4; ++j) xs[h][j] = 0.f;
+#pragma unroll
+          for (int q = 0; q < NP; ++q)
+#pragma unroll
+            for (int h = 0; h < TH; ++h)
+#pragma unroll
+              for (int j = 0; j < 4; ++j) tmp[q][h][j] = 0.f;
 #pragma unroll
           for (int k = 0; k < STEPS; ++k) {
             const uint2 x0 = xr[k][0], x1 = xr[k][TH - 1];
@@ -223,20 +228,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               if constexpr (TH > 1) sm::mma_bf16_16816(xs[TH - 1], ones, x1.x, x1.y);
             }
             const uint8_t* wk = st + sm::piece_offset<R>(sm::word_offset<BITS>(gl, k, c), ush, key16);
-            const int r0 = 16 * qh + g;  // rows r0 and r0 + 8 share the swizzle key
-            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(wk + (r0 << ush));
-            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(wk + ((r0 + 8) << ush));
-            uint32_t a[4];
-            sm::decode_word<BITS>(w0, c, k, a[0], a[2]);
-            sm::decode_word<BITS>(w1, c, k, a[1], a[3]);
-            sm::mma_bf16_16816(tmp[0], a, x0.x, x0.y);
-            if constexpr (TH > 1) sm::mma_bf16_16816(tmp[TH - 1], a, x1.x, x1.y);
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+              const int r0 = 16 * q + g;  // rows r0 and r0 + 8 share the swizzle key
+              const uint32_t w0 = *reinterpret_cast<const uint32_t*>(wk + (r0 << ush));
+              const uint32_t w1 = *reinterpret_cast<const uint32_t*>(wk + ((r0 + 8) << ush));
+              uint32_t a[4];
+              sm::decode_word<BITS>(w0, c, k, a[0], a[2]);
+              sm::decode_word<BITS>(w1, c, k, a[1], a[3]);
+              sm::mma_bf16_16816(tmp[q][0], a, x0.x, x0.y);
+              if constexpr (TH > 1) sm::mma_bf16_16816(tmp[q][TH - 1], a, x1.x, x1.y);
+            }
           }
           // the group's scale (and bias) of rows 16q + g and 16q + g + 8
           const uint16_t* sc = reinterpret_cast<const uint16_t*>(st + p.off_s) + gl * R;
           const uint16_t* bi = reinterpret_cast<const uint16_t*>(st + p.off_b) + gl * R;
-          {
-            const int r0 = 16 * qh + g;
+#pragma unroll
+          for (int q = 0; q < NP; ++q) {
+            const int r0 = 16 * q + g;
             const float s2[2] = {deq::h2f(sc[r0]), deq::h2f(sc[r0 + 8])};
             float b2[2] = {0.f, 0.f};
             if constexpr (BITS > 2) {
@@ -249,13 +258,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               for (int j = 0; j < 4; ++j) {
                 const float sj = s2[j >> 1];
                 if constexpr (BITS == 1) {
-                  acc[h][j] = fmaf(sj, tmp[h][j], acc[h][j]);
+                  acc[q][h][j] = fmaf(sj, tmp[q][h][j], acc[q][h][j]);
                 } else if constexpr (BITS == 2) {
-                  acc[h][j] = fmaf(0.5f * sj, tmp[h][j], acc[h][j]);
+                  acc[q][h][j] = fmaf(0.5f * sj, tmp[q][h][j], acc[q][h][j]);
                 } else {
-                  const float d = BITS == 4 ? fmaf(-128.f, xs[h][j], tmp[h][j]) : tmp[h][j];
-                  const float e = fmaf(b2[j >> 1], xs[h][j], acc[h][j]);
-                  acc[h][j] = fmaf(sj, d, e);
+                  const float d = BITS == 4 ? fmaf(-128.f, xs[h][j], tmp[q][h][j]) : tmp[q][h][j];
+                  const float e = fmaf(b2[j >> 1], xs[h][j], acc[q][h][j]);
+                  acc[q][h][j] = fmaf(sj, d, e);
                 }
               }
           }
@@ -267,12 +276,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // not its waits succeeded; if any gave up, all leave together.
       if (bar_any(CONSUMER_BAR, CONSUMER_THREADS, !ok)) break;
 #pragma unroll
-      for (int h = 0; h < TH; ++h)
+      for (int q = 0; q < NP; ++q)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int m = 8 * h + 2 * c + (j & 1), nl = 16 * qh + g + 8 * (j >> 1);
-          red[(gl * MT + m) * NLP + nl] = acc[h][j];
-        }
+        for (int h = 0; h < TH; ++h)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int m = 8 * h + 2 * c + (j & 1), nl = 16 * q + g + 8 * (j >> 1);
+            red[(gl * MT + m) * NLP + nl] = acc[q][h][j];
+          }
       ptx::named_bar_sync(CONSUMER_BAR, CONSUMER_THREADS);
       for (int i = threadIdx.x; i < P.M * R; i += CONSUMER_THREADS) {
         const int m = i / R, nl = i - m * R;
@@ -280,7 +291,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (n >= P.N) continue;
         float v = 0.f;
 #pragma unroll
-        for (int l = 0; l < GROUP_LANES; ++l) v += red[(l * MT + m) * NLP + nl];
+        for (int l = 0; l < NUM_CONSUMER_WARPS; ++l) v += red[(l * MT + m) * NLP + nl];
         if (P.bias) v += __bfloat162float(__ushort_as_bfloat16(P.bias[n]));
         P.out[static_cast<size_t>(m) * P.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
       }
@@ -340,7 +351,7 @@ int launch(const Problem* probs, int count, bool overlap, cudaStream_t stream, i
   kp.off_s = R * F::ROWB;
   kp.off_b = (kp.off_s + sb + 127) & ~127;
   kp.stage_bytes = (kp.off_b + (BITS <= 2 ? 0 : sb) + 1023) & ~1023;
-  const int red_bytes = GROUP_LANES * MT * (R + 4) * 4;
+  const int red_bytes = NUM_CONSUMER_WARPS * MT * (R + 4) * 4;
   const int tail = red_bytes + 16 * MAX_STAGES + 16;
   int ring = (SMEM_LIMIT - tail) / kp.stage_bytes;
   ring = ring < MAX_STAGES ? ring : MAX_STAGES;
