@@ -274,20 +274,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int s = t % p.ring;
       const int kt = ks0 + (t + rot) % ns;
       // The activations of this warp's groups (the B operand: tokens g and
-      // g + 8, k = gs*G + 16*step + 4c .. +3) straight from global memory,
-      // where every CTA reads the same rows (L2 hits); issued before the
-      // stage's weights are waited for, so the two latencies overlap.
-      uint2 xr[XR ? 1 : GPL][STEPS][TH];
+      // g + 8, thread c's chunk k = gs*G + c*G/4 .. + G/4 - 1) straight from
+      // global memory, where every CTA reads the same rows (L2 hits); issued
+      // before the stage's weights are waited for, so the two latencies overlap.
+      constexpr int XV = F::G / 32;  // 16-byte pieces of a thread's activation chunk
+      uint4 xr[XR ? 1 : GPL][TH][XV];
 #pragma unroll
       for (int gi = 0; gi < (XR ? 0 : GPL); ++gi) {
-        const int k0 = kt * F::KS + (gl + GROUP_LANES * gi) * F::G;
+        const int k0 = kt * F::KS + (gl + GROUP_LANES * gi) * F::G + c * (F::G / 4);
         const bool in = compute && k0 < p.K;
-        const uint2* x0p = reinterpret_cast<const uint2*>(p.X + static_cast<size_t>(g) * p.K + k0 + 4 * c);
-        const uint2* x1p = reinterpret_cast<const uint2*>(p.X + static_cast<size_t>(g + 8) * p.K + k0 + 4 * c);
+        const uint4* x0p = reinterpret_cast<const uint4*>(p.X + static_cast<size_t>(g) * p.K + k0);
+        const uint4* x1p = reinterpret_cast<const uint4*>(p.X + static_cast<size_t>(g + 8) * p.K + k0);
 #pragma unroll
-        for (int k = 0; k < STEPS; ++k) {
-          xr[gi][k][0] = (in && ga) ? __ldg(x0p + 4 * k) : make_uint2(0u, 0u);
-          if constexpr (TH > 1) xr[gi][k][TH - 1] = (in && gb) ? __ldg(x1p + 4 * k) : make_uint2(0u, 0u);
+        for (int v = 0; v < XV; ++v) {
+          xr[gi][0][v] = (in && ga) ? __ldg(x0p + v) : make_uint4(0u, 0u, 0u, 0u);
+          if constexpr (TH > 1) xr[gi][TH - 1][v] = (in && gb) ? __ldg(x1p + v) : make_uint4(0u, 0u, 0u, 0u);
         }
       }
       if (!warp_wait(full(s), (t / p.ring) & 1, lim, abort_flag)) {
@@ -311,32 +312,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int h = 0; h < TH; ++h)
 #pragma unroll
             for (int j = 0; j < 4; ++j) tmp[q][h][j] = 0.f;
+        // this thread's packed chunks of the group for rows 16q + g and
+        // 16q + g + 8 of every pair (the two rows share the swizzle key): one
+        // shared-memory load per row for all of the group's steps
+        constexpr int CW = Chunk<BITS>::WORDS;
+        uint32_t w0[NPH][CW], w1[NPH][CW];
+        {
+          const uint8_t* wc = st + piece_offset<R>(chunk_offset<BITS>(gs, c), ush, key16);
+#pragma unroll
+          for (int q = 0; q < NPH; ++q) {
+            const int r0 = 16 * (q0 + q) + g;
+            load_chunk<BITS>(wc + (r0 << ush), w0[q]);
+            load_chunk<BITS>(wc + ((r0 + 8) << ush), w1[q]);
+          }
+        }
 #pragma unroll
         for (int k = 0; k < STEPS; ++k) {
           uint2 x0, x1;
           if constexpr (XR) {
-            const uint8_t* xg = st + p.off_x + g * p.x_stride + (gs * F::G + 16 * k + 4 * c) * 2;
+            const uint8_t* xg = st + p.off_x + g * p.x_stride + (gs * F::G + c * (F::G / 4) + 4 * k) * 2;
             x0 = ga ? *reinterpret_cast<const uint2*>(xg) : make_uint2(0u, 0u);
             x1 = gb ? *reinterpret_cast<const uint2*>(xg + 8 * p.x_stride) : make_uint2(0u, 0u);
           } else {
-            x0 = xr[gi][k][0];
-            x1 = xr[gi][k][TH - 1];
+            x0 = x_step(xr[gi][0], k);
+            x1 = x_step(xr[gi][TH - 1], k);
           }
           if constexpr (BITS > 2) {
             const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};
             mma_bf16_16816(xs[0], ones, x0.x, x0.y);
             if constexpr (TH > 1) mma_bf16_16816(xs[TH - 1], ones, x1.x, x1.y);
           }
-          const uint8_t* wk = st + piece_offset<R>(word_offset<BITS>(gs, k, c), ush, key16);
 #pragma unroll
           for (int q = 0; q < NPH; ++q) {
-            // rows 16q + g and 16q + g + 8 share the swizzle key
-            const int r0 = 16 * (q0 + q) + g;
-            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(wk + (r0 << ush));
-            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(wk + ((r0 + 8) << ush));
             uint32_t a[4];
-            decode_word<BITS>(w0, c, k, a[0], a[2]);  // row g: k pairs (4c, 4c+1), (4c+2, 4c+3)
-            decode_word<BITS>(w1, c, k, a[1], a[3]);  // row g + 8
+            decode_quad<BITS>(w0[q][step_word<BITS>(k)], step_quad<BITS>(k), a[0], a[2]);  // row g
+            decode_quad<BITS>(w1[q][step_word<BITS>(k)], step_quad<BITS>(k), a[1], a[3]);  // row g + 8
             mma_bf16_16816(tmp[q][0], a, x0.x, x0.y);
             if constexpr (TH > 1) mma_bf16_16816(tmp[q][TH - 1], a, x1.x, x1.y);
           }

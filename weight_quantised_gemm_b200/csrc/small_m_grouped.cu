@@ -190,15 +190,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int kt = (t + rot) % nst;
         const int k0 = kt * F::KS + gl * F::G;
         const bool in = k0 < P.K;
-        // the B fragments (tokens g and g + 8) straight from global memory,
-        // issued before the wait so that the two latencies overlap
-        uint2 xr[STEPS][TH];
-        const uint2* x0p = reinterpret_cast<const uint2*>(P.X + static_cast<size_t>(g) * P.K + k0 + 4 * c);
-        const uint2* x1p = reinterpret_cast<const uint2*>(P.X + static_cast<size_t>(g + 8) * P.K + k0 + 4 * c);
+        // the B fragments (tokens g and g + 8, thread c's chunk of the group)
+        // straight from global memory, issued before the wait so that the two
+        // latencies overlap
+        constexpr int XV = F::G / 32;
+        uint4 xr[TH][XV];
+        const uint4* x0p = reinterpret_cast<const uint4*>(P.X + static_cast<size_t>(g) * P.K + k0 + c * (F::G / 4));
+        const uint4* x1p =
+            reinterpret_cast<const uint4*>(P.X + static_cast<size_t>(g + 8) * P.K + k0 + c * (F::G / 4));
 #pragma unroll
-        for (int k = 0; k < STEPS; ++k) {
-          xr[k][0] = (in && ga) ? __ldg(x0p + 4 * k) : make_uint2(0u, 0u);
-          if constexpr (TH > 1) xr[k][TH - 1] = (in && gb) ? __ldg(x1p + 4 * k) : make_uint2(0u, 0u);
+        for (int v = 0; v < XV; ++v) {
+          xr[0][v] = (in && ga) ? __ldg(x0p + v) : make_uint4(0u, 0u, 0u, 0u);
+          if constexpr (TH > 1) xr[TH - 1][v] = (in && gb) ? __ldg(x1p + v) : make_uint4(0u, 0u, 0u, 0u);
         }
         if (!sm::warp_wait(full(s), (gs / p.ring) & 1, lim, abort_flag)) {
           if (lane == 0) give_up();
@@ -219,23 +222,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int h = 0; h < TH; ++h)
 #pragma unroll
               for (int j = 0; j < 4; ++j) tmp[q][h][j] = 0.f;
+          // this thread's packed chunks of the group, rows 16q + g and 16q + g + 8
+          // (the two rows share the swizzle key), one load per row
+          constexpr int CW = sm::Chunk<BITS>::WORDS;
+          uint32_t w0[NP][CW], w1[NP][CW];
+          {
+            const uint8_t* wc = st + sm::piece_offset<R>(sm::chunk_offset<BITS>(gl, c), ush, key16);
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+              const int r0 = 16 * q + g;
+              sm::load_chunk<BITS>(wc + (r0 << ush), w0[q]);
+              sm::load_chunk<BITS>(wc + ((r0 + 8) << ush), w1[q]);
+            }
+          }
 #pragma unroll
           for (int k = 0; k < STEPS; ++k) {
-            const uint2 x0 = xr[k][0], x1 = xr[k][TH - 1];
+            const uint2 x0 = sm::x_step(xr[0], k), x1 = sm::x_step(xr[TH - 1], k);
             if constexpr (BITS > 2) {
               const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};
               sm::mma_bf16_16816(xs[0], ones, x0.x, x0.y);
               if constexpr (TH > 1) sm::mma_bf16_16816(xs[TH - 1], ones, x1.x, x1.y);
             }
-            const uint8_t* wk = st + sm::piece_offset<R>(sm::word_offset<BITS>(gl, k, c), ush, key16);
 #pragma unroll
             for (int q = 0; q < NP; ++q) {
-              const int r0 = 16 * q + g;  // rows r0 and r0 + 8 share the swizzle key
-              const uint32_t w0 = *reinterpret_cast<const uint32_t*>(wk + (r0 << ush));
-              const uint32_t w1 = *reinterpret_cast<const uint32_t*>(wk + ((r0 + 8) << ush));
               uint32_t a[4];
-              sm::decode_word<BITS>(w0, c, k, a[0], a[2]);
-              sm::decode_word<BITS>(w1, c, k, a[1], a[3]);
+              sm::decode_quad<BITS>(w0[q][sm::step_word<BITS>(k)], sm::step_quad<BITS>(k), a[0], a[2]);
+              sm::decode_quad<BITS>(w1[q][sm::step_word<BITS>(k)], sm::step_quad<BITS>(k), a[1], a[3]);
               sm::mma_bf16_16816(tmp[q][0], a, x0.x, x0.y);
               if constexpr (TH > 1) sm::mma_bf16_16816(tmp[q][TH - 1], a, x1.x, x1.y);
             }

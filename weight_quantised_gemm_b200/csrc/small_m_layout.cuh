@@ -19,20 +19,34 @@ struct Fmt {
   static constexpr int STEPS = G / 16;            // mma k-steps per group
 };
 
-// Logical byte offset, inside a stage row of packed codes, of the 32-bit word
-// that holds quad thread c's 4 codes (k = 4c .. 4c+3) of step k of group gs:
-//   1-bit:   one word per two 16-k steps (quad threads share it);
-//   ternary: one word per 16-k step (quad threads share it);
-//   4-bit:   two words per step, thread c reads word c / 2;
-//   8-bit:   four words per step, thread c reads word c.
+// Each quad thread c owns a contiguous quarter of every scale group: codes
+// c G/4 .. (c + 1) G/4 - 1 of the group, CHUNK bytes of a packed row (1-bit
+// 4, ternary and 4-bit 8, 8-bit 16), read with one shared-memory load per
+// row and group. MMA step s of the group puts the thread's codes
+// 4s .. 4s + 3 in the four k slots the fragment layout gives thread c: the
+// tensor core sums all 16 slots of a step, so any assignment of the group's
+// k to (step, thread, slot) works as long as the activations follow the same
+// one (thread c's activation chunk is k = c G/4 .. + G/4 - 1 as well).
 template <int BITS>
-__host__ __device__ __forceinline__ int word_offset(int gs, int k, int c) {
-  constexpr int GB = Fmt<BITS>::GBYTES;
-  if constexpr (BITS == 1) return gs * GB + 4 * (k >> 1);  // one word per two steps
-  else if constexpr (BITS == 2) return gs * GB + 4 * k;
-  else if constexpr (BITS == 4) return gs * GB + 8 * k + 4 * (c >> 1);
-  else return gs * GB + 16 * k + 4 * c;
+struct Chunk {
+  static constexpr int BYTES = Fmt<BITS>::GBYTES / 4;  // packed bytes per thread, row and group
+  static constexpr int WORDS = BYTES < 4 ? 1 : BYTES / 4;
+  static constexpr int QUADS_PER_WORD = 8 / BITS;       // groups of four codes in a 32-bit word
+};
+
+// Logical byte offset, inside a stage row of packed codes, of quad thread
+// c's chunk of scale group gs.
+template <int BITS>
+__host__ __device__ __forceinline__ int chunk_offset(int gs, int c) {
+  return gs * Fmt<BITS>::GBYTES + c * Chunk<BITS>::BYTES;
 }
+
+// The word of a thread's chunk that holds its codes of step s, and which four
+// codes of that word they are (codes 4 quad .. 4 quad + 3 of the word).
+template <int BITS>
+__host__ __device__ constexpr int step_word(int s) { return s / Chunk<BITS>::QUADS_PER_WORD; }
+template <int BITS>
+__host__ __device__ constexpr int step_quad(int s) { return s % Chunk<BITS>::QUADS_PER_WORD; }
 
 // The box lands as [off / U][row][U bytes] (U = 2^ush), each U-byte row piece
 // swizzled by the TMA: the 16-byte unit index of byte x of a plane is XORed
