@@ -52,11 +52,13 @@
 // (the factor 2 folded into s / 2), 8-bit q exactly through an fp32 magic
 // number. sum_k x_k per group comes from one extra mma against ones.
 //
-// Inside one mma step (16 consecutive k of one group) thread c of each quad
-// takes k = 4c .. 4c+3: the tensor core sums all 16 slots, so any assignment
-// works, and this one makes each activation fetch one 8-byte vector and puts
-// the thread's code pairs where the packed layout keeps them (even and odd k
-// in the two half-words of a 32-bit word).
+// Thread c of each quad owns a contiguous quarter of every group, codes
+// c G/4 .. (c + 1) G/4 - 1, and MMA step s takes codes 4s .. 4s + 3 of it: the
+// tensor core sums all 16 slots of a step, so any assignment works as long as
+// the activations follow it. This one makes a thread's codes of a group one
+// shared-memory load per row and its activations of a group one to four
+// 16-byte loads, and keeps each step's code pairs where the packed layout has
+// them (even and odd k in the two half-words of a 32-bit word).
 
 #include <cuda.h>
 
