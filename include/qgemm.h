@@ -82,7 +82,7 @@ typedef enum qgemm_status {
 /* Kernel path selection for qgemm_ex (low byte of its `path` argument). */
 enum {
   QGEMM_PATH_AUTO = 0,     /* pick per shape from the measured table */
-  QGEMM_PATH_SMALL_M = 1,  /* memory-bound path: registers + mma.sync, M <= 16 */
+  QGEMM_PATH_SMALL_M = 1,  /* memory-bound path: registers + mma.sync, M <= 32 */
   QGEMM_PATH_LARGE_M = 2   /* tensor-core path: TMA + dequant into TMEM + tcgen05 MMA */
 };
 
@@ -183,7 +183,10 @@ int qgemm_load(const char* path, void* packed, void* scales, void* biases);
  * table; the environment variable QGEMM_PATH=small|large overrides it for
  * every shape the named path can take (QGEMM_PATH=small leaves M > 16, and
  * 1-bit weights with K % 256 != 0, to the table). qgemm_select_path reports
- * the same choice.
+ * the same choice. QGEMM_SMALL_TC=1 runs the small-M path's launches without
+ * QGEMM_FLAG_OVERLAP_PREVIOUS on its tcgen05 kernel (weights decoded into
+ * tensor memory, N = 16 tokens per MMA) instead of the warp-level mma.sync
+ * kernel; it is slower on B200 at every measured shape and off by default.
  * Returns after enqueueing; a device-side failure (a bounded wait that ran
  * out) is reported later by qgemm_get_device_status.
  */
@@ -271,7 +274,7 @@ int qgemm_dequant_tile(const qgemm_weights* W, int32_t n0, int32_t k0, int32_t r
  * activation rows of X) through its ring while computing and writing nothing.
  * Its time is the floor of the weight stream itself for this shape: launch,
  * first-byte latency and bandwidth, without the arithmetic. X: device bf16
- * [M, K], 16-byte aligned. Requires a shape the small-M path takes (M <= 16;
+ * [M, K], 16-byte aligned. Requires a shape the small-M path takes (M <= 32;
  * 1-bit weights with K % 256 == 0), else UNSUPPORTED. No counterpart in the
  * pages: an instrument of this implementation.
  */

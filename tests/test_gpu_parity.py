@@ -117,7 +117,7 @@ def test_tiny_workload_default_path():
 
 
 @pytest.mark.parametrize("bits", [1, 2, 4, 8])
-@pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16])
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16, 17, 24, 31, 32])
 def test_small_path_ragged(bits, M):
     K = 1280 if bits == 1 else 1152  # 1-bit rows on the small path: K % 256 == 0
     X, W, bias = WL.random_case(M * 10 + bits, M, 400, K, bits, with_bias=True)
@@ -126,13 +126,16 @@ def test_small_path_ragged(bits, M):
 
 
 @pytest.mark.parametrize("bits", [1, 2, 4, 8])
-@pytest.mark.parametrize("M,N", [(5, 8176), (3, 12272), (5, 16368), (16, 8176), (16, 12272), (11, 16368)])
+@pytest.mark.parametrize("M,N", [(5, 8176), (3, 12272), (5, 16368), (16, 8176), (16, 12272), (11, 16368),
+                                 (20, 4080), (32, 8176)])
 def test_small_path_every_row_count(bits, M, N):
-    """Every rows-per-CTA choice beyond the smallest at both token widths: on
+    """Every rows-per-CTA choice beyond the smallest at every token width: on
     148 SMs N = 8176, 12272 and 16368 take 4, 6 and 8 16-row pairs per CTA,
     each one pair short of whole CTAs, so the last CTA is ragged. With more
     than 8 tokens, 6 or 8 pairs split the rows into halves, each warp taking
-    two groups per stage, and the activations come through the ring."""
+    two groups per stage, and the activations come through the ring. With
+    more than 16 tokens CTAs take 2 (N = 4080) or 4 pairs (N = 8176, rows
+    split into halves), the activations always through the ring."""
     K = 512
     X, W, bias = WL.random_case(M + N + bits, M, N, K, bits, with_bias=True)
     y, _ = gpu_qgemm(X, W, bias, bits, path=SMALL)

@@ -45,6 +45,17 @@ def test_k_split_narrow_shapes(bits, M, N, K):
 
 
 @pytest.mark.parametrize("bits", [1, 2, 4, 8])
+@pytest.mark.parametrize("M", [17, 32])
+@pytest.mark.parametrize("N,K", [(3072, 12288), (3072, 3072)])
+def test_k_split_narrow_shapes_32_tokens(bits, M, N, K):
+    """32-token CTAs (4 MMA column tiles, activations through the ring) on
+    the K-split shapes."""
+    X, W, bias = WL.random_case(N // 64 + K // 512 + M + bits, M, N, K, bits, with_bias=True)
+    y, _ = gpu_qgemm(X, W, bias, bits, path=SMALL)
+    _assert_close(y, _ref(X, W, bias, bits), f"bits={bits} M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
 def test_k_split_one_hot_rows_are_bit_exact(bits):
     """One non-zero activation per token: every K slice but one contributes
     exact zeros, so the cluster's sum is the dequantised weight itself."""

@@ -19,6 +19,7 @@ std::atomic<uint64_t> g_wait_limit_ns{0};  // 0 = not yet resolved; read by ever
 std::once_flag g_env_once;
 int g_env_path = QGEMM_PATH_AUTO;
 int g_env_pair = -1;
+int g_env_small_tc = -1;
 
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
 
@@ -30,6 +31,10 @@ void read_env() {
   if (const char* pr = std::getenv("QGEMM_LARGE_PAIR")) {
     if (!std::strcmp(pr, "0")) g_env_pair = 0;
     else if (!std::strcmp(pr, "1")) g_env_pair = 1;
+  }
+  if (const char* tc = std::getenv("QGEMM_SMALL_TC")) {
+    if (!std::strcmp(tc, "0")) g_env_small_tc = 0;
+    else if (!std::strcmp(tc, "1")) g_env_small_tc = 1;
   }
   if (const char* w = std::getenv("QGEMM_WAIT_LIMIT_NS")) {
     const unsigned long long v = std::strtoull(w, nullptr, 10);
@@ -86,13 +91,18 @@ uint64_t wait_limit_ns() {
   return v ? v : kDefaultWaitLimitNs;
 }
 
-// Whether the small-M path can take this shape at all: M <= 16, and 1-bit
+// Whether the small-M path can take this shape at all: M <= 32, and 1-bit
 // rows streamed in pieces of at least 32 bytes (K % 256 == 0).
-bool small_path_takes(int M, int K, int bits) { return M <= 16 && !(bits == 1 && K % 256); }
+bool small_path_takes(int M, int K, int bits) { return M <= kSmallMaxM && !(bits == 1 && K % 256); }
 
 int large_pair_mode() {
   std::call_once(g_env_once, read_env);
   return g_env_pair;
+}
+
+int small_tc_mode() {
+  std::call_once(g_env_once, read_env);
+  return g_env_small_tc;
 }
 
 int select_path(int M, int N, int K, int bits) {
@@ -137,8 +147,8 @@ extern "C" int qgemm_fused(const void* X, int32_t M, const qgemm_weights* W, voi
   if (!aligned16(X) || !aligned16(out)) return fail(QGEMM_ERR_ALIGNMENT, "X and out must be 16-byte aligned");
   if (bias && (reinterpret_cast<uintptr_t>(bias) & 1u)) return fail(QGEMM_ERR_ALIGNMENT, "bias must be 2-byte aligned");
   if (path == QGEMM_PATH_AUTO) path = auto_path(M, W->N, W->K, W->bits);
-  if (path == QGEMM_PATH_SMALL_M && M > 16)
-    return fail(QGEMM_ERR_UNSUPPORTED, "the small-M path takes M <= 16 (M=%d)", M);
+  if (path == QGEMM_PATH_SMALL_M && M > kSmallMaxM)
+    return fail(QGEMM_ERR_UNSUPPORTED, "the small-M path takes M <= %d (M=%d)", kSmallMaxM, M);
   if (path == QGEMM_PATH_SMALL_M && W->bits == 1 && W->K % 256)
     return fail(QGEMM_ERR_UNSUPPORTED, "the small-M path takes 1-bit weights with K %% 256 == 0 (K=%d)", W->K);
   Problem p{X, M, W->N, W->K, W->bits, W->group, static_cast<const uint8_t*>(W->packed),
@@ -147,7 +157,9 @@ extern "C" int qgemm_fused(const void* X, int32_t M, const qgemm_weights* W, voi
             (flags & QGEMM_FLAG_OVERLAP_PREVIOUS) != 0, op,
             op == QGEMM_EPI_RESIDUAL_GATE ? static_cast<const uint16_t*>(epi->residual) : nullptr,
             op == QGEMM_EPI_RESIDUAL_GATE ? static_cast<const uint16_t*>(epi->gate) : nullptr};
-  return path == QGEMM_PATH_SMALL_M ? launch_small_m(p) : launch_large_m(p);
+  if (path == QGEMM_PATH_SMALL_M)
+    return small_tc_mode() == 1 && !p.overlap && M <= kSmallGroupedMaxM ? launch_small_m_tc(p) : launch_small_m(p);
+  return launch_large_m(p);
 }
 
 extern "C" int qgemm_ex(const void* X, int32_t M, const qgemm_weights* W, void* out, const void* bias,
@@ -210,7 +222,8 @@ extern "C" int qgemm_grouped(const qgemm_problem* problems, int32_t count, int32
     if (q.W.bits != problems[0].W.bits)
       return fail(QGEMM_ERR_UNSUPPORTED, "grouped: problem %d has %d-bit weights, problem 0 %d-bit", i, q.W.bits,
                   problems[0].W.bits);
-    if (q.M < 0 || q.M > 16) return fail(QGEMM_ERR_UNSUPPORTED, "grouped: problem %d has M=%d (0 to 16)", i, q.M);
+    if (q.M < 0 || q.M > kSmallGroupedMaxM)
+      return fail(QGEMM_ERR_UNSUPPORTED, "grouped: problem %d has M=%d (0 to %d)", i, q.M, kSmallGroupedMaxM);
     if (!small_path_takes(q.M, q.W.K, q.W.bits))
       return fail(QGEMM_ERR_UNSUPPORTED, "grouped: problem %d (1-bit weights need K %% 256 == 0)", i);
     if (q.M > 0) {

@@ -38,6 +38,9 @@ uint64_t wait_limit_ns();
 // The large-M kernel's CTA-pair form: -1 = the library's choice (the
 // one-CTA form), 0 = never, 1 = always (QGEMM_LARGE_PAIR=0|1, read once).
 int large_pair_mode();
+// The small-M kernel family: -1 = the library's choice, 0 = the mma.sync
+// kernel, 1 = the tcgen05 kernel (QGEMM_SMALL_TC=0|1, read once).
+int small_tc_mode();
 // Device address of the current device's status word (cached per device).
 int status_word(unsigned int** ptr);
 int sm_count(int* n);
@@ -61,6 +64,8 @@ int make_tensor_map_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* bas
 
 // Kernel launchers (one per kernel family). Each enqueues on p.stream.
 int launch_small_m(const Problem& p);
+// The tcgen05 small-M kernel (M <= 16, no launch overlap).
+int launch_small_m_tc(const Problem& p);
 // Several small-M problems of one format in one launch (qgemm_grouped).
 int launch_small_m_grouped(const Problem* probs, int count, bool overlap, cudaStream_t stream);
 int launch_large_m(const Problem& p);
@@ -73,6 +78,11 @@ int launch_pack_device(const float* W, int N, int K, int bits, void* packed, uin
 // Largest M, N or K the library accepts (2^30): keeps every launcher's int
 // arithmetic (rounded-up tile and stage counts) inside int32.
 constexpr int32_t kMaxDim = 1 << 30;
+
+// Largest M of the small-M (register) kernel; its grouped form and its
+// tcgen05 variant take at most 16.
+constexpr int kSmallMaxM = 32;
+constexpr int kSmallGroupedMaxM = 16;
 
 // Grouped small-M launches: problems per launch, CTAs, and 32-row work items.
 constexpr int kGroupedMaxProblems = 16;

@@ -84,13 +84,17 @@ constexpr int RING_BUDGET = 196608;     // bytes of shared memory for the ring
 constexpr int SMEM_FLOOR = 118784;      // at least this much, so that one grid's CTAs never share an SM
 
 // Row halves for a CTA of NP pairs and MT tokens: 2 where one warp's
-// accumulators for all NP pairs would not fit in registers.
-__host__ __device__ constexpr int split_rows(int MT, int NP) { return MT > 8 && NP >= 6 ? 2 : 1; }
+// accumulators for all NP pairs would not fit in registers (16 tokens and 6
+// or more pairs, 32 tokens and 4 or more; 32-token CTAs take 2 or 4 pairs).
+__host__ __device__ constexpr int split_rows(int MT, int NP) {
+  return (MT == 16 && NP >= 6) || (MT == 32 && NP >= 4) ? 2 : 1;
+}
 // Split-row CTAs give each warp two groups per stage; holding both groups'
 // activation fragments in registers across the stage wait spills, so their
 // activations come through the ring (one bulk copy per token row) instead of
-// straight from global memory.
-__host__ __device__ constexpr bool x_in_ring(int MT, int NP) { return split_rows(MT, NP) == 2; }
+// straight from global memory. So do 32-token CTAs, whose four 8-token
+// fragments per step would not fit either.
+__host__ __device__ constexpr bool x_in_ring(int MT, int NP) { return MT > 16 || split_rows(MT, NP) == 2; }
 
 struct Params {
   const uint16_t* X;     // bf16 [M, K]
@@ -133,10 +137,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr int GROUP_LANES = NUM_CONSUMER_WARPS / PH;  // warps w and w + GROUP_LANES share a group lane
   constexpr int NPH = NP / PH;               // 16-row pairs per warp
   constexpr int GPL = GS / GROUP_LANES;      // groups per warp and stage
-  constexpr int TH = MT > 8 ? 2 : 1;         // 8-token halves
+  constexpr int TH = MT / 8;                 // 8-token MMA column tiles (1, 2 or 4)
   constexpr int NLP = R + 4;                 // row pitch of the partial sums: 2 * NLP = 8 (mod 32) banks
   constexpr bool XR = x_in_ring(MT, NP);     // activations through the ring, else from global memory
   static_assert(NP % PH == 0, "the halves take whole 16-row pairs");
+  static_assert(MT == 8 || MT == 16 || MT == 32, "8, 16 or 32 tokens");
+  static_assert(TH <= 2 || XR, "four token tiles take their activations from the ring");
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = ptx::smem_u32(smem);
   if (sbase & 1023u) {  // the swizzled boxes need it; uniform across the block (and the cluster)
@@ -270,7 +276,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int key16 = swizzle_key16(g, ush);
     const int gl = warp % GROUP_LANES;  // group lane: groups gl, gl + GROUP_LANES, ... of every stage
     const int q0 = (warp / GROUP_LANES) * NPH;  // first 16-row pair of this warp's half
-    const bool ga = g < p.M, gb = MT > 8 && g + 8 < p.M;  // tokens g and g + 8 exist
+    bool gt[TH];  // token g + 8 h exists
+#pragma unroll
+    for (int h = 0; h < TH; ++h) gt[h] = g + 8 * h < p.M;
     const bool compute = !p.floor_only;
     for (int t = 0; t < ns; ++t) {
       const int s = t % p.ring;
@@ -289,8 +297,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint4* x1p = reinterpret_cast<const uint4*>(p.X + static_cast<size_t>(g + 8) * p.K + k0);
 #pragma unroll
         for (int v = 0; v < XV; ++v) {
-          xr[gi][0][v] = (in && ga) ? __ldg(x0p + v) : make_uint4(0u, 0u, 0u, 0u);
-          if constexpr (TH > 1) xr[gi][TH - 1][v] = (in && gb) ? __ldg(x1p + v) : make_uint4(0u, 0u, 0u, 0u);
+          xr[gi][0][v] = (in && gt[0]) ? __ldg(x0p + v) : make_uint4(0u, 0u, 0u, 0u);
+          if constexpr (TH == 2) xr[gi][1][v] = (in && gt[1]) ? __ldg(x1p + v) : make_uint4(0u, 0u, 0u, 0u);
         }
       }
       if (!warp_wait(full(s), (t / p.ring) & 1, lim, abort_flag)) {
@@ -330,27 +338,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
 #pragma unroll
         for (int k = 0; k < STEPS; ++k) {
-          uint2 x0, x1;
+          uint2 xh[TH];  // B fragments: token g + 8 h of tile h, this thread's k of the step
           if constexpr (XR) {
             const uint8_t* xg = st + p.off_x + g * p.x_stride + (gs * F::G + c * (F::G / 4) + 4 * k) * 2;
-            x0 = ga ? *reinterpret_cast<const uint2*>(xg) : make_uint2(0u, 0u);
-            x1 = gb ? *reinterpret_cast<const uint2*>(xg + 8 * p.x_stride) : make_uint2(0u, 0u);
+#pragma unroll
+            for (int h = 0; h < TH; ++h)
+              xh[h] = gt[h] ? *reinterpret_cast<const uint2*>(xg + 8 * h * p.x_stride) : make_uint2(0u, 0u);
           } else {
-            x0 = x_step(xr[gi][0], k);
-            x1 = x_step(xr[gi][TH - 1], k);
+            xh[0] = x_step(xr[gi][0], k);
+            if constexpr (TH == 2) xh[1] = x_step(xr[gi][1], k);
           }
           if constexpr (BITS > 2) {
             const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};
-            mma_bf16_16816(xs[0], ones, x0.x, x0.y);
-            if constexpr (TH > 1) mma_bf16_16816(xs[TH - 1], ones, x1.x, x1.y);
+#pragma unroll
+            for (int h = 0; h < TH; ++h) mma_bf16_16816(xs[h], ones, xh[h].x, xh[h].y);
           }
 #pragma unroll
           for (int q = 0; q < NPH; ++q) {
             uint32_t a[4];
             decode_quad<BITS>(w0[q][step_word<BITS>(k)], step_quad<BITS>(k), a[0], a[2]);  // row g
             decode_quad<BITS>(w1[q][step_word<BITS>(k)], step_quad<BITS>(k), a[1], a[3]);  // row g + 8
-            mma_bf16_16816(tmp[q][0], a, x0.x, x0.y);
-            if constexpr (TH > 1) mma_bf16_16816(tmp[q][TH - 1], a, x1.x, x1.y);
+#pragma unroll
+            for (int h = 0; h < TH; ++h) mma_bf16_16816(tmp[q][h], a, xh[h].x, xh[h].y);
           }
         }
         // apply the group's scale (and bias) of rows 16q + g and 16q + g + 8
@@ -625,12 +634,13 @@ struct Plan {
   int np, ksplit, grid;
 };
 
-inline void plan_candidates(int pairs, int nst, int nsm, Plan* out, int* count) {
+inline void plan_candidates(int pairs, int nst, int nsm, int np_max, Plan* out, int* count) {
   static constexpr int kNP[4] = {2, 4, 6, 8};
   static constexpr int kS[6] = {1, 2, 3, 4, 6, 8};
   int n = 0;
   for (int np : kNP)
     for (int S : kS) {
+      if (np > np_max) continue;
       if (S > nst) continue;
       const int grid = (pairs + np - 1) / np * S;
       if (grid > nsm) continue;
@@ -662,14 +672,16 @@ int try_plan(const Problem& pr, const Plan& pl, bool* launched) {
   return launch_fmt<BITS, MT, NP>(pr, pl.ksplit, pl.grid);
 }
 
+// 32-token CTAs take at most 4 pairs (their accumulators fill the registers).
 template <int BITS, int MT>
 int launch_rows(const Problem& pr, int nsm) {
   using F = Fmt<BITS>;
+  constexpr int NP_MAX = MT == 32 ? 4 : 8;
   const int pairs = pr.N / 16;
   const int nst = (pr.K + F::KS - 1) / F::KS;
   Plan cands[24];
   int count = 0;
-  plan_candidates(pairs, nst, nsm, cands, &count);
+  plan_candidates(pairs, nst, nsm, NP_MAX, cands, &count);
   for (int i = 0; i < count; ++i) {
     const Plan& pl = cands[i];
     bool launched = false;
@@ -677,18 +689,21 @@ int launch_rows(const Problem& pr, int nsm) {
     switch (pl.np) {
       case 2: st = try_plan<BITS, MT, 2>(pr, pl, &launched); break;
       case 4: st = try_plan<BITS, MT, 4>(pr, pl, &launched); break;
-      case 6: st = try_plan<BITS, MT, 6>(pr, pl, &launched); break;
-      default: st = try_plan<BITS, MT, 8>(pr, pl, &launched);
+      case 6: if constexpr (NP_MAX >= 6) st = try_plan<BITS, MT, 6>(pr, pl, &launched); break;
+      default: if constexpr (NP_MAX >= 8) st = try_plan<BITS, MT, 8>(pr, pl, &launched);
     }
     if (st != QGEMM_OK || launched) return st;
   }
-  // more rows than one wave of 128-row CTAs covers: several waves, no slices
-  return launch_fmt<BITS, MT, 8>(pr, 1, (pairs + 7) / 8);
+  // more rows than one wave of CTAs covers: several waves, no slices
+  constexpr int NPW = NP_MAX;
+  return launch_fmt<BITS, MT, NPW>(pr, 1, (pairs + NPW - 1) / NPW);
 }
 
 template <int BITS>
 int launch_bits(const Problem& pr, int nsm) {
-  return pr.M <= 8 ? launch_rows<BITS, 8>(pr, nsm) : launch_rows<BITS, 16>(pr, nsm);
+  if (pr.M <= 8) return launch_rows<BITS, 8>(pr, nsm);
+  if (pr.M <= 16) return launch_rows<BITS, 16>(pr, nsm);
+  return launch_rows<BITS, 32>(pr, nsm);
 }
 
 }  // namespace sm
@@ -697,7 +712,7 @@ int launch_small_m(const Problem& p) {
   int nsm;
   int st = sm_count(&nsm);
   if (st != QGEMM_OK) return st;
-  if (p.M > 16) return fail(QGEMM_ERR_UNSUPPORTED, "small-M path takes M <= 16");
+  if (p.M > kSmallMaxM) return fail(QGEMM_ERR_UNSUPPORTED, "small-M path takes M <= %d", kSmallMaxM);
   switch (p.bits) {
     case 4: return sm::launch_bits<4>(p, nsm);
     case 8: return sm::launch_bits<8>(p, nsm);
