@@ -127,15 +127,17 @@ def test_small_path_ragged(bits, M):
 
 @pytest.mark.parametrize("bits", [1, 2, 4, 8])
 @pytest.mark.parametrize("M,N", [(5, 8176), (3, 12272), (5, 16368), (16, 8176), (16, 12272), (11, 16368),
-                                 (20, 4080), (32, 8176)])
+                                 (20, 4080), (32, 8176), (32, 12272), (24, 16368)])
 def test_small_path_every_row_count(bits, M, N):
     """Every rows-per-CTA choice beyond the smallest at every token width: on
     148 SMs N = 8176, 12272 and 16368 take 4, 6 and 8 16-row pairs per CTA,
     each one pair short of whole CTAs, so the last CTA is ragged. With more
     than 8 tokens, 6 or 8 pairs split the rows into halves, each warp taking
     two groups per stage, and the activations come through the ring. With
-    more than 16 tokens CTAs take 2 (N = 4080) or 4 pairs (N = 8176, rows
-    split into halves), the activations always through the ring."""
+    more than 16 tokens CTAs take 2 (N = 4080), 4 (N = 8176, rows split into
+    halves) or 8 pairs (N = 12272 and 16368, rows split into quarters, each
+    warp taking four groups per stage), the activations always through the
+    ring."""
     K = 512
     X, W, bias = WL.random_case(M + N + bits, M, N, K, bits, with_bias=True)
     y, _ = gpu_qgemm(X, W, bias, bits, path=SMALL)

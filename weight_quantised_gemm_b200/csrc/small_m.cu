@@ -83,11 +83,13 @@ constexpr int SMEM_LIMIT = 232448;      // the most a CTA may have
 constexpr int RING_BUDGET = 196608;     // bytes of shared memory for the ring
 constexpr int SMEM_FLOOR = 118784;      // at least this much, so that one grid's CTAs never share an SM
 
-// Row halves for a CTA of NP pairs and MT tokens: 2 where one warp's
-// accumulators for all NP pairs would not fit in registers (16 tokens and 6
-// or more pairs, 32 tokens and 4 or more; 32-token CTAs take 2 or 4 pairs).
+// Row parts for a CTA of NP pairs and MT tokens: where one warp's
+// accumulators for all NP pairs would not fit in registers the rows split
+// into halves (16 tokens and 6 or more pairs, 32 tokens and 4 pairs) or
+// quarters (32 tokens and 8 pairs), the warps of a part sharing out the
+// stage's groups. 32-token CTAs take 2, 4 or 8 pairs.
 __host__ __device__ constexpr int split_rows(int MT, int NP) {
-  return (MT == 16 && NP >= 6) || (MT == 32 && NP >= 4) ? 2 : 1;
+  return MT == 32 ? (NP >= 8 ? 4 : NP >= 4 ? 2 : 1) : (MT == 16 && NP >= 6 ? 2 : 1);
 }
 // Split-row CTAs give each warp two groups per stage; holding both groups'
 // activation fragments in registers across the stage wait spills, so their
@@ -500,9 +502,15 @@ int make_params(const Problem& pr, int ksplit, Params& kp, int& smem) {
   kp.off_s = R * F::ROWB;
   kp.off_b = (kp.off_s + sb + 127) & ~127;
   kp.off_x = (kp.off_b + (BITS <= 2 ? 0 : sb) + 127) & ~127;
-  kp.x_stride = F::KS * 2 + 32;  // +32 B: token rows 8 banks apart, so the 8-byte B fetches do not collide
+  // +16 B: consecutive token rows 4 banks apart. A half-warp's 8-byte B fetches
+  // (4 token rows x the 4 quad threads' chunks, G / 2 bytes apart) then meet
+  // at most two to a bank, the least a 16-byte-aligned row stride allows.
+  kp.x_stride = F::KS * 2 + 16;
   kp.stage_bytes = (kp.off_x + (x_in_ring(MT, NP) ? pr.M * kp.x_stride : 0) + 1023) & ~1023;
-  int ring = RING_BUDGET / kp.stage_bytes;
+  // Stages that carry the activations are up to twice as large: those rings
+  // take all of shared memory (two 100 KB stages for 32 tokens x 128 rows).
+  const int budget = x_in_ring(MT, NP) ? SMEM_LIMIT - 16 * MAX_STAGES - 16 : RING_BUDGET;
+  int ring = budget / kp.stage_bytes;
   ring = ring < MAX_STAGES ? ring : MAX_STAGES;
   ring = ring < slice_stages ? ring : slice_stages;
   kp.ring = ring < 1 ? 1 : ring;
@@ -634,13 +642,14 @@ struct Plan {
   int np, ksplit, grid;
 };
 
-inline void plan_candidates(int pairs, int nst, int nsm, int np_max, Plan* out, int* count) {
+// np_mask: bit np set for each rows-per-CTA choice the caller compiled.
+inline void plan_candidates(int pairs, int nst, int nsm, unsigned np_mask, Plan* out, int* count) {
   static constexpr int kNP[4] = {2, 4, 6, 8};
   static constexpr int kS[6] = {1, 2, 3, 4, 6, 8};
   int n = 0;
   for (int np : kNP)
     for (int S : kS) {
-      if (np > np_max) continue;
+      if (!(np_mask >> np & 1u)) continue;
       if (S > nst) continue;
       const int grid = (pairs + np - 1) / np * S;
       if (grid > nsm) continue;
@@ -672,16 +681,17 @@ int try_plan(const Problem& pr, const Plan& pl, bool* launched) {
   return launch_fmt<BITS, MT, NP>(pr, pl.ksplit, pl.grid);
 }
 
-// 32-token CTAs take at most 4 pairs (their accumulators fill the registers).
+// 32-token CTAs take 2, 4 or 8 pairs: 6 would leave three pairs per warp,
+// more accumulators than the registers hold.
 template <int BITS, int MT>
 int launch_rows(const Problem& pr, int nsm) {
   using F = Fmt<BITS>;
-  constexpr int NP_MAX = MT == 32 ? 4 : 8;
+  constexpr unsigned NP_MASK = MT == 32 ? (1u << 2 | 1u << 4 | 1u << 8) : (1u << 2 | 1u << 4 | 1u << 6 | 1u << 8);
   const int pairs = pr.N / 16;
   const int nst = (pr.K + F::KS - 1) / F::KS;
   Plan cands[24];
   int count = 0;
-  plan_candidates(pairs, nst, nsm, NP_MAX, cands, &count);
+  plan_candidates(pairs, nst, nsm, NP_MASK, cands, &count);
   for (int i = 0; i < count; ++i) {
     const Plan& pl = cands[i];
     bool launched = false;
@@ -689,14 +699,13 @@ int launch_rows(const Problem& pr, int nsm) {
     switch (pl.np) {
       case 2: st = try_plan<BITS, MT, 2>(pr, pl, &launched); break;
       case 4: st = try_plan<BITS, MT, 4>(pr, pl, &launched); break;
-      case 6: if constexpr (NP_MAX >= 6) st = try_plan<BITS, MT, 6>(pr, pl, &launched); break;
-      default: if constexpr (NP_MAX >= 8) st = try_plan<BITS, MT, 8>(pr, pl, &launched);
+      case 6: if constexpr (MT != 32) st = try_plan<BITS, MT, 6>(pr, pl, &launched); break;
+      default: st = try_plan<BITS, MT, 8>(pr, pl, &launched);
     }
     if (st != QGEMM_OK || launched) return st;
   }
-  // more rows than one wave of CTAs covers: several waves, no slices
-  constexpr int NPW = NP_MAX;
-  return launch_fmt<BITS, MT, NPW>(pr, 1, (pairs + NPW - 1) / NPW);
+  // more rows than one wave of 128-row CTAs covers: several waves, no slices
+  return launch_fmt<BITS, MT, 8>(pr, 1, (pairs + 7) / 8);
 }
 
 template <int BITS>
