@@ -150,7 +150,7 @@ def test_select_path_table():
         assert wq.qgemm_select_path(4096, 9216, 3072, bits) == wq.QGEMM_PATH_LARGE_M
         # every (N, K) of the FLUX workloads: the measured table's choice at decode and prefill M
         for N, K in ((12288, 3072), (9216, 3072), (18432, 3072), (3072, 3072), (3072, 12288)):
-            small_max = 32 if N <= 9216 else 16
+            small_max = 32 if N <= 9216 or bits <= 2 else 16
             for M in (1, 4, 8, 16, 17, 24, 32):
                 want = wq.QGEMM_PATH_SMALL_M if M <= small_max else wq.QGEMM_PATH_LARGE_M
                 assert wq.qgemm_select_path(M, N, K, bits) == want, (bits, N, K, M)
