@@ -645,7 +645,7 @@ struct Plan {
 // np_mask: bit np set for each rows-per-CTA choice the caller compiled.
 inline void plan_candidates(int pairs, int nst, int nsm, unsigned np_mask, Plan* out, int* count) {
   static constexpr int kNP[4] = {2, 4, 6, 8};
-  static constexpr int kS[6] = {1, 2, 3, 4, 6, 8};
+  static constexpr int kS[7] = {1, 2, 3, 4, 5, 6, 8};
   int n = 0;
   for (int np : kNP)
     for (int S : kS) {
@@ -689,7 +689,7 @@ int launch_rows(const Problem& pr, int nsm) {
   constexpr unsigned NP_MASK = MT == 32 ? (1u << 2 | 1u << 4 | 1u << 8) : (1u << 2 | 1u << 4 | 1u << 6 | 1u << 8);
   const int pairs = pr.N / 16;
   const int nst = (pr.K + F::KS - 1) / F::KS;
-  Plan cands[24];
+  Plan cands[28];
   int count = 0;
   plan_candidates(pairs, nst, nsm, NP_MASK, cands, &count);
   for (int i = 0; i < count; ++i) {
