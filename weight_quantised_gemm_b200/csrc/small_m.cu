@@ -175,13 +175,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // the L2 instead of sending all CTAs to the same lines at once.
   const int rot = (blockIdx.x / p.ksplit) % ns;
 
-  if (threadIdx.x == 0) {
+  constexpr int sb_bytes = GS * R * 2;
+  const int units = F::ROWB / U;  // row pieces per stage
+  const int pre = p.ring < ns ? p.ring : ns;
+  auto stage_k = [&](int t, int& kt, int& valid) {
+    kt = ks0 + (t + rot) % ns;  // which K stage ring round t carries
+    valid = min(F::KS, p.K - kt * F::KS);
+  };
+  auto load_weights = [&](int t, int s) {  // lane 0: the stage's packed codes, scales and biases
+    int kt, valid;
+    stage_k(t, kt, valid);
+    const uint32_t st = sbase + s * p.stage_bytes;
+    ptx::mbar_arrive_expect_tx(full(s), R * F::ROWB + sb_bytes * (BITS <= 2 ? 1 : 2) + (XR ? p.M * valid * 2 : 0));
+    ptx::tma_load_3d(st, &tm_w, 0, n0, kt * units, full(s));
+    ptx::tma_load_2d(st + p.off_s, &tm_s, n0, kt * GS, full(s));
+    if (BITS > 2) ptx::tma_load_2d(st + p.off_b, &tm_b, n0, kt * GS, full(s));
+  };
+  auto load_x = [&](int t, int s) {  // all lanes: one bulk copy per token row
+    int kt, valid;
+    stage_k(t, kt, valid);
+    const uint32_t st = sbase + s * p.stage_bytes;
+    for (int m = lane; m < p.M; m += 32)
+      bulk_copy_g2s(st + p.off_x + m * p.x_stride, p.X + static_cast<size_t>(m) * p.K + kt * F::KS, valid * 2,
+                    full(s));
+  };
+  // The producer's lane 0 sets up the barriers and puts the first stage's
+  // weight loads in flight before the block-wide barrier, so that the weight
+  // stream starts as soon as this warp runs (measured: 0.4-0.7 us less per
+  // decode GEMV). Only the first stage: issuing all of them here held the
+  // other warps at the barrier and cost more than it saved on 4-bit.
+  if (threadIdx.x == 32 * WARP_PRODUCER) {
     for (int s = 0; s < p.ring; ++s) {
       ptx::mbar_init(full(s), 1);
       ptx::mbar_init(empty(s), NUM_CONSUMER_WARPS);
     }
     *abort_flag = 0;
     ptx::fence_mbarrier_init();
+    if (pre > 0) load_weights(0, 0);
+    ptx::tma_prefetch_desc(&tm_w);
+    ptx::tma_prefetch_desc(&tm_s);
+    if (BITS > 2) ptx::tma_prefetch_desc(&tm_b);
   }
   __syncthreads();
   auto give_up = [&]() {
@@ -201,42 +234,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == WARP_PRODUCER) {
     // ---------------- producer: TMA boxes and bulk copies into the ring ----------------
-    constexpr int sb_bytes = GS * R * 2;
-    const int units = F::ROWB / U;  // row pieces per stage
-    const int pre = p.ring < ns ? p.ring : ns;
-    auto stage_k = [&](int t, int& kt, int& valid) {
-      kt = ks0 + (t + rot) % ns;  // which K stage ring round t carries
-      valid = min(F::KS, p.K - kt * F::KS);
-    };
-    auto load_weights = [&](int t, int s) {  // lane 0: the stage's packed codes, scales and biases
-      int kt, valid;
-      stage_k(t, kt, valid);
-      const uint32_t st = sbase + s * p.stage_bytes;
-      ptx::mbar_arrive_expect_tx(full(s), R * F::ROWB + sb_bytes * (BITS <= 2 ? 1 : 2) + (XR ? p.M * valid * 2 : 0));
-      ptx::tma_load_3d(st, &tm_w, 0, n0, kt * units, full(s));
-      ptx::tma_load_2d(st + p.off_s, &tm_s, n0, kt * GS, full(s));
-      if (BITS > 2) ptx::tma_load_2d(st + p.off_b, &tm_b, n0, kt * GS, full(s));
-    };
-    auto load_x = [&](int t, int s) {  // all lanes: one bulk copy per token row
-      int kt, valid;
-      stage_k(t, kt, valid);
-      const uint32_t st = sbase + s * p.stage_bytes;
-      for (int m = lane; m < p.M; m += 32)
-        bulk_copy_g2s(st + p.off_x + m * p.x_stride, p.X + static_cast<size_t>(m) * p.K + kt * F::KS, valid * 2,
-                      full(s));
-    };
-    if (lane == 0) {
-      ptx::tma_prefetch_desc(&tm_w);
-      ptx::tma_prefetch_desc(&tm_s);
-      if (BITS > 2) ptx::tma_prefetch_desc(&tm_b);
-    }
     if (!XR || p.overlap) {
       // The weights do not depend on the previous grid: the first stages go
-      // out at once, and the next grid may launch (both no-ops without the
-      // launch attribute). Ring activations follow once that grid is done
-      // (the TMA unit takes copies in issue order, so they queue behind).
+      // out at once (the first already has), and the next grid may launch
+      // (both no-ops without the launch attribute). Ring activations follow
+      // once that grid is done (the TMA unit takes copies in issue order, so
+      // they queue behind).
       if (lane == 0)
-        for (int t = 0; t < pre; ++t) load_weights(t, t);
+        for (int t = 1; t < pre; ++t) load_weights(t, t);
       griddep_launch_dependents();
       if constexpr (XR) {
         griddep_wait();
@@ -247,7 +252,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // Nothing to wait for: each stage's activations right behind its
       // weights, so that the first stage is complete as early as possible.
       for (int t = 0; t < pre; ++t) {
-        if (lane == 0) load_weights(t, t);
+        if (lane == 0 && t > 0) load_weights(t, t);
         __syncwarp();
         load_x(t, t);
       }
