@@ -114,13 +114,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint64_t lim = p.wait_limit_ns;
   const int ib = p.cta_begin[blockIdx.x], ie = p.cta_begin[blockIdx.x + 1];
 
-  if (threadIdx.x == 0) {
+  // Stage t of item `it` (the CTA's gs-th stage overall) into ring slot gs % ring.
+  auto issue_stage = [&](int it, int t, uint32_t gs) {
+    constexpr int sb_bytes = GS * R * 2;
+    const int pi = p.items[it] >> 12, rb = p.items[it] & 0xFFF;
+    const GProblem& P = p.prob[pi];
+    const int n0 = rb * R, nst = P.num_stages, rot = rb % nst;
+    const int units = F::ROWB >> P.unit_shift;
+    const int s = gs % p.ring, kt = (t + rot) % nst;
+    const uint32_t st = sbase + s * p.stage_bytes;
+    ptx::mbar_arrive_expect_tx(full(s), R * F::ROWB + sb_bytes * (BITS <= 2 ? 1 : 2));
+    ptx::tma_load_3d(st, &maps.w[pi], 0, n0, kt * units, full(s));
+    ptx::tma_load_2d(st + p.off_s, &maps.s[pi], n0, kt * GS, full(s));
+    if (BITS > 2) ptx::tma_load_2d(st + p.off_b, &maps.b[pi], n0, kt * GS, full(s));
+  };
+  // The producer's lane 0 sets up the ring and puts the first stage in flight
+  // before the block-wide barrier (as in the one-problem kernel).
+  if (threadIdx.x == 32 * WARP_PRODUCER) {
     for (int s = 0; s < p.ring; ++s) {
       ptx::mbar_init(full(s), 1);
       ptx::mbar_init(empty(s), NUM_CONSUMER_WARPS);
     }
     *abort_flag = 0;
     ptx::fence_mbarrier_init();
+    if (ib < ie) issue_stage(ib, 0, 0);
   }
   __syncthreads();
   auto give_up = [&]() {
@@ -134,15 +151,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // the next grid launch (both no-ops without the launch attribute).
     sm::griddep_launch_dependents();
     if (lane == 0) {
-      constexpr int sb_bytes = GS * R * 2;
       uint32_t gs = 0;  // stages issued so far, over all items
       bool ok = true;
       for (int it = ib; ok && it < ie; ++it) {
-        const int pi = p.items[it] >> 12, rb = p.items[it] & 0xFFF;
-        const GProblem& P = p.prob[pi];
-        const int n0 = rb * R, nst = P.num_stages, rot = rb % nst;
-        const int units = F::ROWB >> P.unit_shift;
+        const int nst = p.prob[p.items[it] >> 12].num_stages;
         for (int t = 0; t < nst; ++t, ++gs) {
+          if (gs == 0) continue;  // issued before the block-wide barrier
           const int s = gs % p.ring;
           if (gs >= static_cast<uint32_t>(p.ring) &&
               !ptx::mbar_wait(empty(s), ((gs / p.ring) & 1) ^ 1, lim, abort_flag)) {
@@ -150,12 +164,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
-          const int kt = (t + rot) % nst;
-          const uint32_t st = sbase + s * p.stage_bytes;
-          ptx::mbar_arrive_expect_tx(full(s), R * F::ROWB + sb_bytes * (BITS <= 2 ? 1 : 2));
-          ptx::tma_load_3d(st, &maps.w[pi], 0, n0, kt * units, full(s));
-          ptx::tma_load_2d(st + p.off_s, &maps.s[pi], n0, kt * GS, full(s));
-          if (BITS > 2) ptx::tma_load_2d(st + p.off_b, &maps.b[pi], n0, kt * GS, full(s));
+          issue_stage(it, t, gs);
         }
       }
       // let every copy issued above land before the block can exit
