@@ -106,7 +106,7 @@ class ClockSampler:
                   "clocks_event_reasons.hw_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
                   "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.hw_power_brake_slowdown")
 
-    def __init__(self, device_id: str, period_s: float = 0.005):
+    def __init__(self, device_id: str, period_s: float = 0.001):
         self.dev = device_id
         self.period = period_s
         self.samples = []  # (t, sm_mhz, power_w, [reason names])
@@ -116,6 +116,7 @@ class ClockSampler:
         self._stop = threading.Event()
         self.thread = None
         self.proc = None
+        self._read = None  # one NVML sample -> (t, sm_mhz, power_w, reasons), or None
 
     def _nvml_handle(self):
         import pynvml
@@ -132,16 +133,28 @@ class ClockSampler:
                 nv.nvmlDeviceGetCurrentClocksThrottleReasons
             self.source = "nvml"
 
+            def read_one():
+                t = time.monotonic()
+                try:
+                    clk = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                except Exception:  # a failed read only loses that sample
+                    return None
+                try:
+                    pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                except Exception:
+                    pw = None
+                try:
+                    bits = get_reasons(h)
+                except Exception:
+                    bits = 0
+                return (t, clk, pw, [n for n, b in self.REASONS if bits & b])
+            self._read = read_one
+
             def loop():
                 while not self._stop.is_set():
-                    try:
-                        t = time.monotonic()
-                        clk = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
-                        bits = get_reasons(h)
-                        self.samples.append((t, float(clk), pw, [n for n, b in self.REASONS if bits & b]))
-                    except Exception:  # a failed read only loses that sample
-                        pass
+                    r = read_one()
+                    if r is not None:
+                        self.samples.append(r)
                     self._stop.wait(self.period)
             self.thread = threading.Thread(target=loop, daemon=True)
             self.thread.start()
@@ -172,6 +185,15 @@ class ClockSampler:
         self.thread = threading.Thread(target=read, daemon=True)
         self.thread.start()
 
+    def sample_now(self):
+        """One sample from the calling thread (NVML only): called while the
+        timed launches are queued on the GPU, so that even a timed region
+        shorter than the sampling period holds at least one sample."""
+        if self._read is not None:
+            r = self._read()
+            if r is not None:
+                self.samples.append(r)
+
     def mark_begin(self):
         self.t_begin = time.monotonic()
 
@@ -198,7 +220,8 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(r[1] for r in timed) if timed else None, "sm_max_mhz": self.sm_max,
                 "reasons": reasons, "samples": len(rows), "samples_in_timed_region": len(timed),
                 "sm_mhz_min_in_timed_region": min((r[1] for r in timed), default=None),
-                "power_w_max": max(r[2] for r in rows), "period_ms": self.period * 1e3, "source": self.source}
+                "power_w_max": max((r[2] for r in rows if r[2] is not None), default=None),
+                "period_ms": self.period * 1e3, "source": self.source}
 
 
 # ----------------------------------------------------------------------------
@@ -529,6 +552,7 @@ def run_ours(args, rank, world, local_rank):
         step(i)
         ev[i][1].record(stream)
     t1.record(stream)
+    clocks.sample_now()  # the queued launches are running now
     barrier(world)
     clocks.mark_end()
     clk = clocks.stop()

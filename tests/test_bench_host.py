@@ -34,6 +34,23 @@ def test_clock_report_without_samples():
     assert r["sm_mhz"] is None and r["samples"] == 0
 
 
+def test_a_timed_region_shorter_than_the_period_still_holds_a_sample():
+    """sample_now(), called while the timed launches run, puts a sample inside
+    the region even when the sampling thread never woke up there; a sample
+    without a power reading still counts."""
+    import time
+    c = bench.ClockSampler("0")
+    c.sm_max, c.source = 1965.0, "test"
+    c._read = lambda: (time.monotonic(), 1950.0, None, [])
+    c.samples = [(time.monotonic() - 10.0, 1965.0, 120.0, [])]   # before the region
+    c.mark_begin()
+    c.sample_now()
+    c.mark_end()
+    r = c.stop()
+    assert r["samples_in_timed_region"] == 1 and r["sm_mhz"] == 1950.0
+    assert r["power_w_max"] == 120.0
+
+
 def test_reason_bits_are_distinct():
     bits = [b for _, b in bench.ClockSampler.REASONS]
     assert len(set(bits)) == len(bits)
