@@ -56,10 +56,12 @@ def test_k_split_narrow_shapes_32_tokens(bits, M, N, K):
 
 
 @pytest.mark.parametrize("bits", [1, 2, 4, 8])
-def test_k_split_one_hot_rows_are_bit_exact(bits):
+@pytest.mark.parametrize("M", [9, 25])
+def test_k_split_one_hot_rows_are_bit_exact(bits, M):
     """One non-zero activation per token: every K slice but one contributes
-    exact zeros, so the cluster's sum is the dequantised weight itself."""
-    N, K, M = 3072, 3072, 9
+    exact zeros, so the cluster's sum is the dequantised weight itself (16-
+    and 32-token CTAs)."""
+    N, K = 3072, 3072
     g = np.random.default_rng(31 + bits)
     _, W, _ = WL.random_case(41 + bits, 1, N, K, bits, with_bias=False)
     ks = g.choice(K, size=M, replace=False)
