@@ -71,6 +71,7 @@
 #include "qgemm_internal.h"
 #include "small_m_common.cuh"
 #include "small_m_layout.cuh"
+#include "small_m_plan.h"
 
 namespace qg {
 namespace sm {
@@ -637,49 +638,7 @@ int clusters_fit(const Problem& pr, int ksplit, int clusters, bool* ok) {
   return QGEMM_OK;
 }
 
-// Rows per CTA (16 NP, NP from the compiled set) and K slices per row block
-// (a cluster of `ksplit` CTAs): the choice that puts the fewest row-stages of
-// packed weights on the busiest CTA with the whole grid resident at once, the
-// fewer slices on a tie. With 32 tokens a tie goes against CTAs of 32 rows
-// first: a stage's activations are two (8-bit) to eight (ternary) times such
-// a CTA's packed weights, and twice as many rows per CTA halve the
-// activation bytes each SM reads (3072 x 12288 ternary at M = 32: 19.0 us
-// against 25.4; 3072 x 3072 8-bit: 11.9 against 14.0). Narrow N with long K (MLP down, the out projection)
-// needs the slices: 3072 rows make only 96 CTAs of 32 rows, while 48 row
-// blocks of 64 rows x 3 slices use 144 SMs with a third less per CTA.
-struct Plan {
-  int np, ksplit, grid;
-};
-
-// np_mask: bit np set for each rows-per-CTA choice the caller compiled;
-// demote_np2: 32-row plans lose ties on row-stages.
-inline void plan_candidates(int pairs, int nst, int nsm, unsigned np_mask, bool demote_np2, Plan* out, int* count) {
-  static constexpr int kNP[4] = {2, 4, 6, 8};
-  static constexpr int kS[7] = {1, 2, 3, 4, 5, 6, 8};
-  int n = 0;
-  for (int np : kNP)
-    for (int S : kS) {
-      if (!(np_mask >> np & 1u)) continue;
-      if (S > nst) continue;
-      const int grid = (pairs + np - 1) / np * S;
-      if (grid > nsm) continue;
-      out[n++] = Plan{np, S, grid};
-    }
-  // cheapest first: row-stages on the busiest CTA, then (demote_np2) more
-  // than 32 rows, then fewer slices
-  auto cost = [&](const Plan& p) { return p.np * ((nst + p.ksplit - 1) / p.ksplit); };
-  auto np2 = [&](const Plan& p) { return demote_np2 && p.np == 2 ? 1 : 0; };
-  for (int i = 1; i < n; ++i)
-    for (int j = i; j > 0; --j) {
-      const Plan a = out[j - 1], b = out[j];
-      if (cost(b) < cost(a) ||
-          (cost(b) == cost(a) && (np2(b) < np2(a) || (np2(b) == np2(a) && b.ksplit < a.ksplit)))) {
-        out[j - 1] = b;
-        out[j] = a;
-      }
-    }
-  *count = n;
-}
+// Launch shapes: Plan and plan_candidates (small_m_plan.h).
 
 template <int BITS, int MT, int NP>
 int try_plan(const Problem& pr, const Plan& pl, bool* launched) {
@@ -702,7 +661,7 @@ int launch_rows(const Problem& pr, int nsm) {
   constexpr unsigned NP_MASK = MT == 32 ? (1u << 2 | 1u << 4 | 1u << 8) : (1u << 2 | 1u << 4 | 1u << 6 | 1u << 8);
   const int pairs = pr.N / 16;
   const int nst = (pr.K + F::KS - 1) / F::KS;
-  Plan cands[28];
+  Plan cands[kMaxPlans];
   int count = 0;
   plan_candidates(pairs, nst, nsm, NP_MASK, MT == 32, cands, &count);
   for (int i = 0; i < count; ++i) {
