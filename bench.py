@@ -500,7 +500,7 @@ def crossover_sweep():
                 out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
                 entry = {"N": N, "K": K, "bits": bits, "M": M}
                 for name, path in (("small", wq.QGEMM_PATH_SMALL_M), ("large", wq.QGEMM_PATH_LARGE_M)):
-                    if name == "small" and M > 32:
+                    if name == "small" and M > 64:
                         continue
                     fns = [(lambda d=d: wq.qgemm(Xd, d, out=out, path=path)) for d in dws]
                     launches = max(len(fns), 64 if M <= 32 else 16)

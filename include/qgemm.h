@@ -82,7 +82,8 @@ typedef enum qgemm_status {
 /* Kernel path selection for qgemm_ex (low byte of its `path` argument). */
 enum {
   QGEMM_PATH_AUTO = 0,     /* pick per shape from the measured table */
-  QGEMM_PATH_SMALL_M = 1,  /* memory-bound path: registers + mma.sync, M <= 32 */
+  QGEMM_PATH_SMALL_M = 1,  /* memory-bound path: registers + mma.sync, M <= 64 (launches of
+                              up to 32 token rows, back to back on the stream, past 32) */
   QGEMM_PATH_LARGE_M = 2   /* tensor-core path: TMA + dequant into TMEM + tcgen05 MMA */
 };
 
@@ -274,7 +275,7 @@ int qgemm_dequant_tile(const qgemm_weights* W, int32_t n0, int32_t k0, int32_t r
  * activation rows of X) through its ring while computing and writing nothing.
  * Its time is the floor of the weight stream itself for this shape: launch,
  * first-byte latency and bandwidth, without the arithmetic. X: device bf16
- * [M, K], 16-byte aligned. Requires a shape the small-M path takes (M <= 32;
+ * [M, K], 16-byte aligned. Requires a shape the small-M path takes (M <= 64;
  * 1-bit weights with K % 256 == 0), else UNSUPPORTED. No counterpart in the
  * pages: an instrument of this implementation.
  */

@@ -120,7 +120,7 @@ def test_qgemm_rejects_bad_operands_without_device():
     assert _call(d, path=7) == wq.QGEMM_ERR_INVALID_ARG
     assert _call(d, path=wq.QGEMM_PATH_LARGE_M | 0x200) == wq.QGEMM_ERR_INVALID_ARG   # unknown flag bit
     assert _call(d, M=0, path=wq.QGEMM_PATH_SMALL_M | wq.QGEMM_FLAG_OVERLAP_PREVIOUS) == wq.QGEMM_OK
-    assert _call(d, M=33, path=wq.QGEMM_PATH_SMALL_M) == wq.QGEMM_ERR_UNSUPPORTED
+    assert _call(d, M=65, path=wq.QGEMM_PATH_SMALL_M) == wq.QGEMM_ERR_UNSUPPORTED      # small path: M <= 64
     assert _call(d, M=(1 << 30) + 1) == wq.QGEMM_ERR_UNSUPPORTED                      # above the 2^30 limit
     assert _call(d, M=(1 << 31) - 1) == wq.QGEMM_ERR_UNSUPPORTED
     # M = 0 is a no-op that never touches the device
@@ -150,11 +150,16 @@ def test_select_path_table():
         assert wq.qgemm_select_path(4096, 9216, 3072, bits) == wq.QGEMM_PATH_LARGE_M
         # every (N, K) of the FLUX workloads: the measured table's choice at decode and prefill M
         for N, K in ((12288, 3072), (9216, 3072), (18432, 3072), (3072, 3072), (3072, 12288)):
-            small_max = 32 if N <= 9216 or bits <= 2 else 16
-            for M in (1, 4, 8, 16, 17, 24, 32):
+            if N <= 3072:
+                small_max = 64
+            elif bits <= 2:
+                small_max = 48 if N <= 9216 else 32
+            else:
+                small_max = 32 if N <= 9216 else 16
+            for M in (1, 4, 8, 16, 17, 24, 32, 33, 48, 49, 64):
                 want = wq.QGEMM_PATH_SMALL_M if M <= small_max else wq.QGEMM_PATH_LARGE_M
                 assert wq.qgemm_select_path(M, N, K, bits) == want, (bits, N, K, M)
-            for M in (33, 64, 4608):
+            for M in (65, 256, 4608):
                 assert wq.qgemm_select_path(M, N, K, bits) == wq.QGEMM_PATH_LARGE_M, (bits, N, K, M)
     with pytest.raises(wq.QGemmError):
         wq.qgemm_select_path(1, 16, 128, 3)
@@ -242,7 +247,7 @@ import weight_quantised_gemm_b200 as wq
 W = lambda **kw: wq._Weights(kw.get('N', 256), kw.get('K', 512), kw.get('bits', 4), kw.get('group', 64),
                              0x1000, 0x2000, kw.get('biases', 0x3000))
 call = lambda d, M: wq._lib.qgemm_ex(0x10000, M, ctypes.byref(d), 0x20000, None, 0, None)
-print(wq.qgemm_select_path(16, 256, 512, 4), wq.qgemm_select_path(33, 256, 512, 4),
+print(wq.qgemm_select_path(16, 256, 512, 4), wq.qgemm_select_path(65, 256, 512, 4),
       wq.qgemm_select_path(4, 256, 1152, 1), wq.qgemm_select_path(4, 256, 1024, 1))
 print(call(W(), 33), call(W(bits=1, group=128, K=1152, biases=0), 4))
 """
@@ -311,7 +316,7 @@ def test_problem_struct_layout_matches_the_header(tmp_path):
 def test_debug_stream_rejects_bad_arguments_without_device():
     d = _desc()
     f = wq._lib.qgemm_debug_stream
-    assert f(0x10000, 33, ctypes.byref(d), 0, None) == wq.QGEMM_ERR_UNSUPPORTED       # small-M shapes only
+    assert f(0x10000, 65, ctypes.byref(d), 0, None) == wq.QGEMM_ERR_UNSUPPORTED       # small-M shapes only
     assert f(0x10000, -1, ctypes.byref(d), 0, None) == wq.QGEMM_ERR_INVALID_ARG
     assert f(0x10000, 4, ctypes.byref(d), 0x200, None) == wq.QGEMM_ERR_INVALID_ARG    # unknown flag
     assert f(None, 4, ctypes.byref(d), 0, None) == wq.QGEMM_ERR_INVALID_ARG

@@ -339,7 +339,7 @@ def _fused_case(bits, M, N, K, op, seed, path, in_place=False):
 
 @pytest.mark.parametrize("op", [wq.QGEMM_EPI_GELU_TANH, wq.QGEMM_EPI_RESIDUAL_GATE])
 @pytest.mark.parametrize("bits", [1, 2, 4, 8])
-@pytest.mark.parametrize("path,M", [(SMALL, 1), (SMALL, 13), (SMALL, 29), (LARGE, 300)])
+@pytest.mark.parametrize("path,M", [(SMALL, 1), (SMALL, 13), (SMALL, 29), (SMALL, 45), (LARGE, 300)])
 def test_fused_epilogue_parity(op, bits, path, M):
     y, ref = _fused_case(bits, M, 400, 768, op, 100 + 10 * op + bits + M, path)
     _assert_close(y, ref, f"op={op} bits={bits} path={path} M={M}")
@@ -354,7 +354,7 @@ def test_fused_epilogue_with_split_rows(op, bits):
     _assert_close(y, ref, f"split rows op={op} bits={bits}")
 
 
-@pytest.mark.parametrize("path,M", [(SMALL, 5), (SMALL, 27), (LARGE, 257)])
+@pytest.mark.parametrize("path,M", [(SMALL, 5), (SMALL, 27), (SMALL, 50), (LARGE, 257)])
 def test_fused_residual_update_in_place(path, M):
     """out may be the residual itself: the same bits as the out-of-place call."""
     y_out, ref = _fused_case(4, M, 528, 512, wq.QGEMM_EPI_RESIDUAL_GATE, 77, path)

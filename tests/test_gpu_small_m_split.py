@@ -115,7 +115,19 @@ def test_k_split_overlap_reads_the_previous_kernels_output(bits):
 
 
 @pytest.mark.parametrize("bits", [1, 2, 4, 8])
-@pytest.mark.parametrize("M,N,K", [(1, 12288, 3072), (16, 12288, 3072), (1, 3072, 12288), (16, 12272, 512)])
+@pytest.mark.parametrize("M", [33, 47, 64])
+@pytest.mark.parametrize("N,K", [(3072, 12288), (1008, 1024)])
+def test_small_path_past_32_tokens(bits, M, N, K):
+    """M = 33..64 on the small path: launches of 32 token rows back to back
+    (the later ones overlapping the one before), the last one ragged."""
+    X, W, bias = WL.random_case(900 + M + bits + N // 8, M, N, K, bits, with_bias=True)
+    y, _ = gpu_qgemm(X, W, bias, bits, path=SMALL)
+    _assert_close(y, _ref(X, W, bias, bits), f"bits={bits} M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
+@pytest.mark.parametrize("M,N,K", [(1, 12288, 3072), (16, 12288, 3072), (1, 3072, 12288), (16, 12272, 512),
+                                   (48, 3072, 3072)])
 def test_stream_floor_runs_clean_and_leaves_the_output_alone(bits, M, N, K):
     """The streaming-floor launch (same grid, clusters and ring as the GEMV,
     no arithmetic) completes with a clean status, in both launch modes, and a

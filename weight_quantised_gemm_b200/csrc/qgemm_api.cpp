@@ -93,7 +93,31 @@ uint64_t wait_limit_ns() {
 
 // Whether the small-M path can take this shape at all: M <= 32, and 1-bit
 // rows streamed in pieces of at least 32 bytes (K % 256 == 0).
-bool small_path_takes(int M, int K, int bits) { return M <= kSmallMaxM && !(bits == 1 && K % 256); }
+bool small_path_takes(int M, int K, int bits) { return M <= kSmallPathMaxM && !(bits == 1 && K % 256); }
+
+// The small-M path for any M it takes: one launch up to kSmallMaxM tokens,
+// else launches of kSmallMaxM token rows back to back on the caller's stream
+// (each streams all the weights; they write disjoint output rows). Launches
+// after the first overlap their weight stream with the previous one's last
+// stages (programmatic dependent launch): each reads its activations and
+// writes its rows only once the launch before it has finished, which in turn
+// ran after whatever preceded the call.
+int launch_small_rows(const Problem& p) {
+  if (p.M <= kSmallMaxM)
+    return small_tc_mode() == 1 && !p.overlap && !p.floor_only && p.M <= kSmallGroupedMaxM ? launch_small_m_tc(p)
+                                                                                          : launch_small_m(p);
+  for (int m0 = 0; m0 < p.M; m0 += kSmallMaxM) {
+    Problem q = p;
+    q.M = p.M - m0 < kSmallMaxM ? p.M - m0 : kSmallMaxM;
+    q.X = static_cast<const uint16_t*>(p.X) + static_cast<size_t>(m0) * p.K;
+    if (p.out) q.out = static_cast<uint16_t*>(p.out) + static_cast<size_t>(m0) * p.N;
+    if (p.residual) q.residual = p.residual + static_cast<size_t>(m0) * p.N;
+    if (m0 > 0) q.overlap = true;
+    const int st = launch_small_m(q);
+    if (st != QGEMM_OK) return st;
+  }
+  return QGEMM_OK;
+}
 
 int large_pair_mode() {
   std::call_once(g_env_once, read_env);
@@ -147,8 +171,8 @@ extern "C" int qgemm_fused(const void* X, int32_t M, const qgemm_weights* W, voi
   if (!aligned16(X) || !aligned16(out)) return fail(QGEMM_ERR_ALIGNMENT, "X and out must be 16-byte aligned");
   if (bias && (reinterpret_cast<uintptr_t>(bias) & 1u)) return fail(QGEMM_ERR_ALIGNMENT, "bias must be 2-byte aligned");
   if (path == QGEMM_PATH_AUTO) path = auto_path(M, W->N, W->K, W->bits);
-  if (path == QGEMM_PATH_SMALL_M && M > kSmallMaxM)
-    return fail(QGEMM_ERR_UNSUPPORTED, "the small-M path takes M <= %d (M=%d)", kSmallMaxM, M);
+  if (path == QGEMM_PATH_SMALL_M && M > kSmallPathMaxM)
+    return fail(QGEMM_ERR_UNSUPPORTED, "the small-M path takes M <= %d (M=%d)", kSmallPathMaxM, M);
   if (path == QGEMM_PATH_SMALL_M && W->bits == 1 && W->K % 256)
     return fail(QGEMM_ERR_UNSUPPORTED, "the small-M path takes 1-bit weights with K %% 256 == 0 (K=%d)", W->K);
   Problem p{X, M, W->N, W->K, W->bits, W->group, static_cast<const uint8_t*>(W->packed),
@@ -157,8 +181,7 @@ extern "C" int qgemm_fused(const void* X, int32_t M, const qgemm_weights* W, voi
             (flags & QGEMM_FLAG_OVERLAP_PREVIOUS) != 0, op,
             op == QGEMM_EPI_RESIDUAL_GATE ? static_cast<const uint16_t*>(epi->residual) : nullptr,
             op == QGEMM_EPI_RESIDUAL_GATE ? static_cast<const uint16_t*>(epi->gate) : nullptr};
-  if (path == QGEMM_PATH_SMALL_M)
-    return small_tc_mode() == 1 && !p.overlap && M <= kSmallGroupedMaxM ? launch_small_m_tc(p) : launch_small_m(p);
+  if (path == QGEMM_PATH_SMALL_M) return launch_small_rows(p);
   return launch_large_m(p);
 }
 
@@ -258,7 +281,7 @@ extern "C" int qgemm_debug_stream(const void* X, int32_t M, const qgemm_weights*
             static_cast<const uint16_t*>(W->scales), static_cast<const uint16_t*>(W->biases), nullptr, nullptr,
             static_cast<cudaStream_t>(stream), (flags & QGEMM_FLAG_OVERLAP_PREVIOUS) != 0, QGEMM_EPI_NONE,
             nullptr, nullptr, true};
-  return launch_small_m(p);
+  return launch_small_rows(p);
 }
 
 extern "C" int qgemm_set_wait_limit_ns(uint64_t limit_ns) {

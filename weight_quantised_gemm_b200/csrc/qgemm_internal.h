@@ -79,9 +79,11 @@ int launch_pack_device(const float* W, int N, int K, int bits, void* packed, uin
 // arithmetic (rounded-up tile and stage counts) inside int32.
 constexpr int32_t kMaxDim = 1 << 30;
 
-// Largest M of the small-M (register) kernel; its grouped form and its
-// tcgen05 variant take at most 16.
+// Largest M of one small-M (register) kernel launch; its grouped form and its
+// tcgen05 variant take at most 16. The small-M path as a whole takes up to
+// kSmallPathMaxM: larger M runs as launches of kSmallMaxM tokens back to back.
 constexpr int kSmallMaxM = 32;
+constexpr int kSmallPathMaxM = 64;
 constexpr int kSmallGroupedMaxM = 16;
 
 // Grouped small-M launches: problems per launch, CTAs, and 32-row work items.
