@@ -161,6 +161,9 @@ def test_select_path_table():
                 assert wq.qgemm_select_path(M, N, K, bits) == want, (bits, N, K, M)
             for M in (65, 256, 4608):
                 assert wq.qgemm_select_path(M, N, K, bits) == wq.QGEMM_PATH_LARGE_M, (bits, N, K, M)
+        # narrow N below K = 3072 keeps the one-launch limits: the tiny 64 x 512 x 512 case on the tile path
+        assert wq.qgemm_select_path(64, 512, 512, bits) == wq.QGEMM_PATH_LARGE_M
+        assert wq.qgemm_select_path(32, 512, 512, bits) == wq.QGEMM_PATH_SMALL_M
     with pytest.raises(wq.QGemmError):
         wq.qgemm_select_path(1, 16, 128, 3)
     with pytest.raises(wq.QGemmError) as e:

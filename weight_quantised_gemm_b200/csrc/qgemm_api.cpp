@@ -132,7 +132,8 @@ int small_tc_mode() {
 int select_path(int M, int N, int K, int bits) {
   if (!small_path_takes(M, K, bits)) return QGEMM_PATH_LARGE_M;
   for (const PathEntry& e : kPathTable)
-    if (e.bits == bits && N <= e.n_max && K <= e.k_max) return M <= e.small_max ? QGEMM_PATH_SMALL_M : QGEMM_PATH_LARGE_M;
+    if (e.bits == bits && N <= e.n_max && K >= e.k_min && K <= e.k_max)
+      return M <= e.small_max ? QGEMM_PATH_SMALL_M : QGEMM_PATH_LARGE_M;
   return QGEMM_PATH_LARGE_M;
 }
 
