@@ -89,15 +89,16 @@ enum {
 
 /* Flags OR-ed into qgemm_ex's `path` argument.
  *
- * QGEMM_FLAG_OVERLAP_PREVIOUS: launch the small-M kernel with programmatic
- * dependent launch. Its CTAs may start while the previous kernel in the stream
- * is still running and put the packed weights, scales and biases in flight at
- * once; they wait for that kernel to complete (and its writes to be visible)
- * before reading X or bias and before writing out. Ask for it only when the
+ * QGEMM_FLAG_OVERLAP_PREVIOUS: launch the kernel (either path) with
+ * programmatic dependent launch. Its CTAs may start while the previous kernel
+ * in the stream is still running (taking SMs as that kernel's CTAs leave) and
+ * put the packed weights, scales and biases in flight at once (the large-M
+ * path also dequantises them and runs its first stages' setup); they wait
+ * for that kernel to complete (and its writes to be visible) before reading
+ * X, bias, gate or residual and before writing out. Ask for it only when the
  * weight buffers are not written by the work that precedes the call in the
- * stream (static weights, as in inference). It has no effect on the large-M
- * path. No counterpart in the method's description: a launch-overlap option
- * of this implementation. */
+ * stream (static weights, as in inference). No counterpart in the method's
+ * description: a launch-overlap option of this implementation. */
 enum {
   QGEMM_FLAG_OVERLAP_PREVIOUS = 0x100
 };

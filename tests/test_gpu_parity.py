@@ -284,6 +284,45 @@ def test_overlap_with_split_rows_reads_the_previous_kernels_output(bits):
         _assert_close(from_dev_bf16(y2), _ref(y1_bits, W2, bias2, bits), "second, overlapped, split rows")
 
 
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_large_path_overlap_reads_and_writes_after_the_previous_kernel(bits):
+    """The tile path with launch overlap. A chain y1 = X W1^T, y2 = y1 W2^T
+    (the second reads what the first wrote); a gated residual update of y1 in
+    place (it reads y1 as its residual); and a call whose output buffer the
+    previous call also wrote (its stores must land last)."""
+    M, K1, N1, N2 = 300, 1024, 2048, 1536
+    X, W1, _ = WL.random_case(391 + bits, M, N1, K1, bits, with_bias=False)
+    _, W2, bias2 = WL.random_case(392 + bits, M, N2, N1, bits, with_bias=True)
+    _, W3, _ = WL.random_case(393 + bits, M, N1, K1, bits, with_bias=False)
+    d1, d2, d3 = (wq.qgemm_pack(w, bits).to_device() for w in (W1, W2, W3))
+    Xd, b2 = to_dev_bf16(X), to_dev_bf16(bias2)
+    g_bits = _bf16_normal(394 + bits, (N1,))
+    gd = to_dev_bf16(g_bits)
+    group = wq.GROUP_OF_BITS[bits]
+    for _ in range(2):
+        y1 = torch.full((M, N1), float("nan"), dtype=torch.bfloat16, device="cuda")
+        y1 = wq.qgemm(Xd, d1, out=y1, path=LARGE)
+        y2 = wq.qgemm(y1, d2, bias=b2, path=LARGE, overlap_previous=True)
+        wq.check_device_status()
+        y1_bits = from_dev_bf16(y1)
+        _assert_close(y1_bits, _ref(X, W1, None, bits), "first")
+        _assert_close(from_dev_bf16(y2), _ref(y1_bits, W2, bias2, bits), "second, overlapped")
+        # y1 <- y1 + gate * (X W3^T), in place, overlapping the kernel that wrote y1
+        y1 = wq.qgemm(Xd, d1, out=y1, path=LARGE)
+        wq.qgemm_fused(Xd, d3, wq.QGEMM_EPI_RESIDUAL_GATE, residual=y1, gate=gd, out=y1, path=LARGE,
+                       overlap_previous=True)
+        wq.check_device_status()
+        p3, s3, b3 = O.pack_ref(W3, bits, group)
+        ref = O.qgemm_ref_epilogue(X, p3, s3, b3, bits, group, K1, None, wq.QGEMM_EPI_RESIDUAL_GATE, y1_bits, g_bits)
+        _assert_close(from_dev_bf16(y1), ref, "residual update in place, overlapped")
+        # two calls into one buffer: the overlapped second one's output stands
+        buf = torch.empty((M, N1), dtype=torch.bfloat16, device="cuda")
+        wq.qgemm(Xd, d1, out=buf, path=LARGE)
+        wq.qgemm(Xd, d3, out=buf, path=LARGE, overlap_previous=True)
+        wq.check_device_status()
+        _assert_close(from_dev_bf16(buf), _ref(X, W3, None, bits), "same output buffer, overlapped")
+
+
 def test_overlap_after_a_torch_kernel_and_in_a_graph():
     """The previous kernel is a plain torch one (no trigger of its own), and the
     same overlapped call captured in a CUDA graph gives the same result."""

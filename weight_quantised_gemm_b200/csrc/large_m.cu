@@ -268,6 +268,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   if constexpr (PAIR) ptx::cluster_sync();  // both CTAs' barriers and TMEM are ready before any cross-CTA use
   ptx::tc_fence_after();
+  // Launched with programmatic dependent launch (QGEMM_FLAG_OVERLAP_PREVIOUS):
+  // the next grid may launch now (its CTAs take SMs as this grid's leave),
+  // and this grid's weight stream, dequantisation and MMAs on it do not wait
+  // for the previous one; the X producer waits before its first activation
+  // load and the epilogue before it reads bias, gate or residual or stores
+  // out. Without the launch attribute both are no-ops.
+  ptx::griddep_launch_dependents();
   const uint32_t tmem_base = *tmem_slot;
   const uint64_t lim = p.wait_limit_ns;
   const int my_tiles = (p.num_tiles - unit + units - 1) / units;
@@ -282,6 +289,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ---------------- TMA producers ----------------
     if (lane == 0) {
       const bool is_x = warp == WARP_XLOAD;
+      if (is_x) ptx::griddep_wait();  // X may be the previous grid's output
       const int R = is_x ? S : SW;
       uint32_t it = 0;
       bool ok = true;
@@ -479,6 +487,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ---------------- epilogue ----------------
+    ptx::griddep_wait();  // bias, gate and residual may be the previous grid's output, out may still be read by it
     const int e = warp - WARP_EPI0;
     const int q = warp & 3;                // TMEM lane quarter this warp may read
     const int t0 = (e >> 2) * EPI_TOKENS;  // first token (accumulator column) of this warp
@@ -731,13 +740,22 @@ int launch_fmt(const Problem& pr, int nsm) {
   cfg.blockDim = dim3(NUM_THREADS);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = pr.stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (PAIR) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 2;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pr.overlap) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = PAIR ? 1 : 0;
+  cfg.numAttrs = na;
   return cuda_check(cudaLaunchKernelEx(&cfg, large_m_kernel<BITS, EPI, PAIR>, tm_x, tm_w, tm_s, tm_b, tm_out, tm_res,
                                        kp),
                     "large_m_kernel launch");
