@@ -99,7 +99,7 @@ static_assert(EPI_TOKENS % EPI_ROWS == 0, "epilogue warps cover whole tcgen05.ld
 // stages 128 of the 256 tokens (the MMA reads the B operand from both CTAs'
 // shared memory), so an activation stage takes 32 KB instead of 64 and four
 // fit where one CTA alone holds two.
-template <int BITS, bool PAIR = false>
+template <int BITS, bool PAIR = false, bool PLAIN = false>
 struct Cfg {
   static constexpr int kTokens = PAIR ? TILE_M / 2 : TILE_M;  // tokens this CTA stages
   static constexpr int kXBoxBytes = kTokens * BOX_K * 2;
@@ -118,9 +118,18 @@ struct Cfg {
   static constexpr uint32_t kSwzMask = BITS == 8 ? 7 : BITS == 4 ? 3 : BITS == 2 ? 1 : 0;
   static constexpr int kSBytes = kGroupsPerStage * TILE_N * 2;  // one stage's scales (or biases)
   static constexpr int kSBStride = BITS <= 2 ? kSBytes : 2 * kSBytes;
-  static constexpr int kS = PAIR ? 4 : BITS == 8 ? 2 : 3;        // stage ring depth
-  static constexpr int kSW = BITS == 8 ? 3 : BITS == 4 ? (PAIR ? 4 : 2) : BITS == 2 ? 4 : 8;  // W ring depth
-  static constexpr int kSlots = PAIR || BITS == 8 ? 2 : 1;      // epilogue store slots per warp
+  // 8-bit on one CTA with the plain epilogue (PLAIN): the epilogue stores
+  // straight to global memory instead of through shared-memory slots and TMA,
+  // which leaves room for a third activation stage beside the 16 KB packed
+  // tiles. It reads its whole share of the accumulator and hands it back
+  // before the first store, so the stores never hold the MMA. (The fused
+  // epilogues store chunk by chunk before their last accumulator read; there
+  // the slower 2-byte global stores held the MMA and cost 22 % on the fused
+  // out projection, so they keep two stages and the slots.)
+  static constexpr bool kDirect = BITS == 8 && !PAIR && PLAIN;
+  static constexpr int kS = PAIR ? 4 : BITS == 8 && !kDirect ? 2 : 3;  // stage ring depth
+  static constexpr int kSW = BITS == 8 ? (kDirect ? 2 : 3) : BITS == 4 ? (PAIR ? 4 : 2) : BITS == 2 ? 4 : 8;  // W ring depth
+  static constexpr int kSlots = kDirect ? 0 : PAIR || BITS == 8 ? 2 : 1;  // epilogue store slots per warp
   static constexpr int kOffX = 0;
   static constexpr int kOffW = kOffX + kS * kXStageBytes;
   static constexpr int kOffOut = kOffW + kSW * kWTileBytes;
@@ -141,6 +150,7 @@ struct Params {
   int num_m_tiles, num_n_tiles, num_tiles, num_kb;
   int m_fastest;  // tile order: 1 = consecutive tiles walk the token dimension, 0 = the feature dimension
   const uint16_t* bias;
+  uint16_t* out;             // bf16 [M, N] (written directly by the Cfg::kDirect epilogue)
   const uint16_t* residual;  // bf16 [M, N] (residual update only)
   const uint16_t* gate;      // bf16 [N] (residual update only)
   uint64_t wait_limit_ns;
@@ -185,7 +195,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                    const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_res,
                    const Params p) {
-  using C = Cfg<BITS, PAIR>;
+  using C = Cfg<BITS, PAIR, EPI == QGEMM_EPI_NONE>;
   constexpr int S = C::kS, SW = C::kSW;
   constexpr int TILE_ROWS = PAIR ? 2 * TILE_N : TILE_N;  // weight rows of one output tile
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -544,6 +554,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) acc_empty_arrive();
+        if constexpr (C::kDirect) {
+          // token m of this warp's rows: 32 lanes write 32 consecutive features (64 bytes)
+          if (n_ok) {
+#pragma unroll
+            for (int t = 0; t < EPI_TOKENS; ++t)
+              if (t < rows_left)
+                p.out[static_cast<size_t>(m0 + t) * p.N + n] = static_cast<uint16_t>(pk[t / 2] >> (16 * (t & 1)));
+          }
+          continue;
+        } else {
 #pragma unroll
         for (int c = 0; c < EPI_TOKENS / EPI_ROWS; ++c) {
           if (c < chunks && nr + 32 * q < p.N) {
@@ -566,6 +586,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         continue;
+        }
       }
       for (int c = 0; c < EPI_TOKENS / EPI_ROWS; ++c) {
         uint32_t v[32];
@@ -592,7 +613,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           __syncwarp();
           if (lane == 0) acc_empty_arrive();
         }
-        if (c < chunks && nr + 32 * q < p.N) {
+        if constexpr (C::kDirect) {
+          if (c < chunks && n_ok) {
+#pragma unroll
+            for (int t = 0; t < EPI_ROWS; ++t) {
+              const int m = m0 + c * EPI_ROWS + t;
+              const uint16_t r = EPI == QGEMM_EPI_RESIDUAL_GATE ? static_cast<uint16_t>(res2[EPI == QGEMM_EPI_RESIDUAL_GATE ? t / 2 : 0] >> (16 * (t & 1))) : 0;
+              const float f = epi::apply<EPI>(__uint_as_float(v[t]) + bias_f, r, gate_f);
+              if (m < p.M) p.out[static_cast<size_t>(m) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(f));
+            }
+          }
+        } else if (c < chunks && nr + 32 * q < p.N) {
           const uint32_t slot = nstore % C::kSlots;
           // the TMA store that last used this slot has finished reading it
           if (lane == 0) ptx::bulk_wait_group_read<C::kSlots - 1>();
@@ -668,7 +699,7 @@ inline int max_pairs(const void* fn, int smem, int nsm) {
 
 template <int BITS, int EPI, bool PAIR>
 int launch_fmt(const Problem& pr, int nsm) {
-  using C = Cfg<BITS, PAIR>;
+  using C = Cfg<BITS, PAIR, EPI == QGEMM_EPI_NONE>;
   constexpr int TILE_ROWS = PAIR ? 2 * TILE_N : TILE_N;
   const void* fn = reinterpret_cast<const void*>(large_m_kernel<BITS, EPI, PAIR>);
   int st = smem_opt_in(fn, C::kSmemBytes, "cudaFuncSetAttribute(large_m_kernel)");
@@ -726,6 +757,7 @@ int launch_fmt(const Problem& pr, int nsm) {
     kp.m_fastest = live(kp.num_m_tiles, x_panel, w_panel) <= live(kp.num_n_tiles, w_panel, x_panel);
   }
   kp.bias = pr.bias;
+  kp.out = static_cast<uint16_t*>(pr.out);
   kp.residual = pr.residual;
   kp.gate = pr.gate;
   CUtensorMap tm_res = tm_out;  // the residual update's L2 prefetch box: this CTA's part of a tile
