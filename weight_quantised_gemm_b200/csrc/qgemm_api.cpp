@@ -91,7 +91,8 @@ uint64_t wait_limit_ns() {
   return v ? v : kDefaultWaitLimitNs;
 }
 
-// Whether the small-M path can take this shape at all: M <= 32, and 1-bit
+// Whether the small-M path can take this shape at all: M <= 64 (launches of
+// up to 32 token rows), and 1-bit
 // rows streamed in pieces of at least 32 bytes (K % 256 == 0).
 bool small_path_takes(int M, int K, int bits) { return M <= kSmallPathMaxM && !(bits == 1 && K % 256); }
 

@@ -1,4 +1,5 @@
-// Small-M path (M <= 16): a memory-bound kernel that streams the packed
+// Small-M path (up to 32 tokens per launch; the API runs M = 33-64 as
+// launches of 32 token rows): a memory-bound kernel that streams the packed
 // weights once.
 //
 // pictor's README ("Extreme quantization is first-class") has GEMV paths
@@ -25,11 +26,12 @@
 //   stage.
 // * Eight consumer warps. Normally warp w takes scale group w of every stage
 //   for all the CTA's rows; where that would not fit in registers (16 tokens
-//   and 6 or more 16-row pairs) the rows split into two halves and warps w and
-//   w + 4 take groups w % 4 and w % 4 + 4 of every stage, each for its half.
-//   A warp turns codes into bf16 in registers and feeds warp-level mma.sync
-//   (m16n8k16, bf16 in, fp32 accumulate): the weights are the 16-row A
-//   operand, the activations the 8-column B (tokens past M are zero). At the
+//   and 6 or more 16-row pairs, 32 tokens and 4 or 8 pairs) the rows split
+//   into halves or quarters whose warps share out the stage's groups, each
+//   for its part. A warp turns codes into bf16 in registers and feeds
+//   warp-level mma.sync (m16n8k16, bf16 in, fp32 accumulate): the weights are
+//   the 16-row A operand, the activations the 8-column B tiles (one, two or
+//   four of 8 tokens; tokens past M are zero). At the
 //   end the warps' fp32 partial sums meet in shared memory (token-major,
 //   bank-conflict free) and a coalesced pass adds them, adds the bias and
 //   writes bf16.
