@@ -125,6 +125,35 @@ def test_small_path_past_32_tokens(bits, M, N, K):
     _assert_close(y, _ref(X, W, bias, bits), f"bits={bits} M={M} N={N} K={K}")
 
 
+@pytest.mark.parametrize("bits", [2, 8])
+@pytest.mark.parametrize("M", [47, 64])
+def test_small_path_past_32_tokens_equals_calls_on_the_pieces(bits, M):
+    """Past 32 tokens each launch is the one a call on its 32 (or fewer) rows
+    makes: the same bits as separate calls on the pieces, fused residual
+    update in place included."""
+    N, K = 3072, 3072
+    X, W, bias = WL.random_case(950 + M + bits, M, N, K, bits, with_bias=True)
+    dw = wq.qgemm_pack(W, bits).to_device()
+    Xd, bd = to_dev_bf16(X), to_dev_bf16(bias)
+    y = wq.qgemm(Xd, dw, bias=bd, path=SMALL)
+    parts = [wq.qgemm(Xd[m0:m0 + 32].contiguous(), dw, bias=bd, path=SMALL) for m0 in range(0, M, 32)]
+    wq.check_device_status()
+    assert torch.equal(y, torch.cat(parts))
+    g = np.random.default_rng(960 + M + bits)
+    r = to_dev_bf16(WL.f32_to_bf16_bits(g.standard_normal((M, N)).astype(np.float32)))
+    gate = to_dev_bf16(WL.f32_to_bf16_bits(g.standard_normal(N).astype(np.float32)))
+    whole = r.clone()
+    wq.qgemm_fused(Xd, dw, wq.QGEMM_EPI_RESIDUAL_GATE, bias=bd, residual=whole, gate=gate, out=whole, path=SMALL)
+    pieces = []
+    for m0 in range(0, M, 32):
+        rp = r[m0:m0 + 32].clone()
+        wq.qgemm_fused(Xd[m0:m0 + 32].contiguous(), dw, wq.QGEMM_EPI_RESIDUAL_GATE, bias=bd, residual=rp, gate=gate,
+                       out=rp, path=SMALL)
+        pieces.append(rp)
+    wq.check_device_status()
+    assert torch.equal(whole, torch.cat(pieces))
+
+
 @pytest.mark.parametrize("bits", [1, 2, 4, 8])
 @pytest.mark.parametrize("M,N,K", [(1, 12288, 3072), (16, 12288, 3072), (1, 3072, 12288), (16, 12272, 512),
                                    (48, 3072, 3072)])
