@@ -425,10 +425,11 @@ def sweep(peaks):
 
 
 def grouped_sweep(peaks):
-    """The mixed FLUX block's five linears at decode M: one grouped launch per
+    """The mixed FLUX block's five linears at decode M: one grouped call per
     format (4-bit QKV and MLP up; 8-bit modulation, out projection and MLP
-    down) against one launch per linear, CUDA-graph timing over rotating
-    weight copies, GB/s against the summed algorithmic bytes."""
+    down), as consecutive overlapped launches (the default) and as one
+    persistent launch, against one plain call per linear, CUDA-graph timing
+    over rotating weight copies, GB/s against the summed algorithmic bytes."""
     import numpy as np
     import torch
 
@@ -454,11 +455,15 @@ def grouped_sweep(peaks):
                 return lambda: wq.qgemm_grouped([(x, d, b) for x, d, b, _ in probs], outs=[o for *_, o in probs],
                                                 overlap_previous=ov)
 
+            def grouped_one_launch(probs, ov):
+                return lambda: wq.qgemm_grouped([(x, d, b) for x, d, b, _ in probs], outs=[o for *_, o in probs],
+                                                overlap_previous=ov, one_launch=True)
+
             def separate(probs, ov):
                 return lambda: [wq.qgemm(x, d, bias=b, out=o, overlap_previous=ov) for x, d, b, o in probs]
             n = max(ncopy, 24)
             res = {"M": M, "bits": bits, "linears": [l.name for _, l in lins], "alg_bytes": ab, "copies": ncopy}
-            for name, mk in (("grouped", grouped), ("separate", separate)):
+            for name, mk in (("grouped", grouped), ("grouped_one_launch", grouped_one_launch), ("separate", separate)):
                 for ov in (False, True):
                     t = time_graph([mk(sets[i % ncopy], ov) for i in range(n)])
                     key = name + ("_overlap_previous" if ov else "")
@@ -653,9 +658,10 @@ def run_case(args):
 
 
 def run_grouped_case(args):
-    """The mixed FLUX block's linears of one format at decode M as one grouped
-    launch, back to back with a CUDA event pair per launch (the form a
-    profiler captures). --grouped BITS:M, e.g. 8:1"""
+    """The mixed FLUX block's linears of one format at decode M as one
+    persistent grouped launch (QGEMM_FLAG_GROUPED_ONE_LAUNCH), back to back
+    with a CUDA event pair per launch (the form a profiler captures).
+    --grouped BITS:M, e.g. 8:1"""
     import numpy as np
     import torch
 
@@ -676,17 +682,17 @@ def run_grouped_case(args):
              for l, X, pw in host] for _ in range(ncopy)]
     outs = [torch.empty((M, l.N), dtype=torch.bfloat16, device="cuda") for l, _, _ in host]
     for i in range(args.warmup):
-        wq.qgemm_grouped(sets[i % ncopy], outs=outs)
+        wq.qgemm_grouped(sets[i % ncopy], outs=outs, one_launch=True)
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for i in range(args.steps):
         ev[i][0].record()
-        wq.qgemm_grouped(sets[i % ncopy], outs=outs)
+        wq.qgemm_grouped(sets[i % ncopy], outs=outs, one_launch=True)
         ev[i][1].record()
     torch.cuda.synchronize()
     wq.check_device_status()
     t = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e-3
-    tg = time_graph([(lambda s=s: wq.qgemm_grouped(s, outs=outs)) for s in sets] * max(1, 24 // ncopy))
+    tg = time_graph([(lambda s=s: wq.qgemm_grouped(s, outs=outs, one_launch=True)) for s in sets] * max(1, 24 // ncopy))
     wq.check_device_status()
     return {"grouped": args.grouped, "linears": [l.name for l, _, _ in host], "alg_bytes": ab, "copies": ncopy,
             "us_per_launch_events": round(t * 1e6, 2), "us_graph": round(tg * 1e6, 2),
@@ -1129,7 +1135,8 @@ def main(argv=None):
     ap.add_argument("--report", default=None,
                     help="also write the detailed report sections (JSON lines) to this file")
     ap.add_argument("--grouped", default=None,
-                    help="time the mixed block's linears of one format as one grouped launch, BITS:M (e.g. 8:1)")
+                    help="time the mixed block's linears of one format as one persistent grouped launch, BITS:M "
+                         "(e.g. 8:1)")
     ap.add_argument("--case", default=None,
                     help="time one workload linear alone, e.g. 3:tern_m1:M=16 (workload:linear[:M=..])")
     args = ap.parse_args(argv)

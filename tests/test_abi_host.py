@@ -279,7 +279,10 @@ def _problem(M=4, X=0x10000, out=0x20000, bias=None, **kw):
 def test_grouped_rejects_bad_lists_without_device():
     ok = _problem()
     assert wq._lib.qgemm_grouped(None, 1, 0, None) == wq.QGEMM_ERR_INVALID_ARG
-    assert _grouped([ok], flags=0x200) == wq.QGEMM_ERR_INVALID_ARG
+    assert _grouped([ok], flags=0x400) == wq.QGEMM_ERR_INVALID_ARG
+    # the one-launch flag is known: the call gets past the argument checks (and,
+    # without a device, fails at the launch)
+    assert _grouped([ok], flags=wq.QGEMM_FLAG_GROUPED_ONE_LAUNCH) == wq.QGEMM_ERR_CUDA
     arr = (wq._Problem * 17)(*([ok] * 17))
     assert wq._lib.qgemm_grouped(arr, 17, 0, None) == wq.QGEMM_ERR_INVALID_ARG
     assert wq._lib.qgemm_grouped(arr, 0, 0, None) == wq.QGEMM_ERR_INVALID_ARG

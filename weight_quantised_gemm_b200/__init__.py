@@ -34,6 +34,7 @@ QGEMM_PATH_AUTO = 0
 QGEMM_PATH_SMALL_M = 1
 QGEMM_PATH_LARGE_M = 2
 QGEMM_FLAG_OVERLAP_PREVIOUS = 0x100
+QGEMM_FLAG_GROUPED_ONE_LAUNCH = 0x200
 
 QGEMM_EPI_NONE = 0
 QGEMM_EPI_GELU_TANH = 1
@@ -333,12 +334,13 @@ def qgemm_fused(X, W: DeviceWeights, op: int, bias=None, residual=None, gate=Non
     return out
 
 
-def qgemm_grouped(problems, outs=None, stream=None, overlap_previous: bool = False):
-    """Several independent small-M GEMVs in one launch (C ABI qgemm_grouped):
-    `problems` is a list of (X, W, bias) with X a bf16 [M, K] CUDA tensor
-    (M <= 16), W DeviceWeights (one format for all) and bias a bf16 [N]
-    tensor or None. Returns the outputs (bf16 [M, N] each), written into
-    `outs` when given."""
+def qgemm_grouped(problems, outs=None, stream=None, overlap_previous: bool = False, one_launch: bool = False):
+    """Several independent small-M GEMVs (C ABI qgemm_grouped): `problems` is
+    a list of (X, W, bias) with X a bf16 [M, K] CUDA tensor (M <= 16), W
+    DeviceWeights (one format for all) and bias a bf16 [N] tensor or None.
+    Consecutive overlapped launches, or one persistent launch with
+    `one_launch` (QGEMM_FLAG_GROUPED_ONE_LAUNCH). Returns the outputs (bf16
+    [M, N] each), written into `outs` when given."""
     import torch
     if not problems:
         raise ValueError("no problems")
@@ -361,7 +363,7 @@ def qgemm_grouped(problems, outs=None, stream=None, overlap_previous: bool = Fal
         _same_device(dev, W, X=X, out=out, bias=bias)
         arr[i] = _Problem(X.data_ptr(), M, W.descriptor(), out.data_ptr(), None if bias is None else bias.data_ptr())
         result.append(out)
-    flags = QGEMM_FLAG_OVERLAP_PREVIOUS if overlap_previous else 0
+    flags = (QGEMM_FLAG_OVERLAP_PREVIOUS if overlap_previous else 0) | (QGEMM_FLAG_GROUPED_ONE_LAUNCH if one_launch else 0)
     with torch.cuda.device(dev):
         _check(_lib.qgemm_grouped(arr, len(problems), flags, _stream_handle(stream, dev)), "qgemm_grouped")
     return result

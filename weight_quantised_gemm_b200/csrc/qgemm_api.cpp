@@ -237,7 +237,8 @@ extern "C" int qgemm_grouped(const qgemm_problem* problems, int32_t count, int32
   if (!problems) return fail(QGEMM_ERR_INVALID_ARG, "null problem list");
   if (count < 1 || count > kGroupedMaxProblems)
     return fail(QGEMM_ERR_INVALID_ARG, "count=%d: 1 to %d problems per grouped call", count, kGroupedMaxProblems);
-  if (flags & ~QGEMM_FLAG_OVERLAP_PREVIOUS) return fail(QGEMM_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  if (flags & ~(QGEMM_FLAG_OVERLAP_PREVIOUS | QGEMM_FLAG_GROUPED_ONE_LAUNCH))
+    return fail(QGEMM_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
   Problem probs[kGroupedMaxProblems];
   bool any = false;
   for (int i = 0; i < count; ++i) {
@@ -265,8 +266,21 @@ extern "C" int qgemm_grouped(const qgemm_problem* problems, int32_t count, int32
                        (flags & QGEMM_FLAG_OVERLAP_PREVIOUS) != 0, QGEMM_EPI_NONE, nullptr, nullptr};
   }
   if (!any) return QGEMM_OK;
-  return launch_small_m_grouped(probs, count, (flags & QGEMM_FLAG_OVERLAP_PREVIOUS) != 0,
-                                static_cast<cudaStream_t>(stream));
+  if (flags & QGEMM_FLAG_GROUPED_ONE_LAUNCH)
+    return launch_small_m_grouped(probs, count, (flags & QGEMM_FLAG_OVERLAP_PREVIOUS) != 0,
+                                  static_cast<cudaStream_t>(stream));
+  // consecutive launches, the later ones overlapping the one before: the
+  // problems are independent (no output overlaps another problem's operands)
+  bool first = true;
+  for (int i = 0; i < count; ++i) {
+    if (probs[i].M == 0) continue;
+    Problem p = probs[i];
+    if (!first) p.overlap = true;
+    first = false;
+    const int st = launch_small_rows(p);
+    if (st != QGEMM_OK) return st;
+  }
+  return QGEMM_OK;
 }
 
 extern "C" int qgemm_debug_stream(const void* X, int32_t M, const qgemm_weights* W, int32_t flags, void* stream) {
